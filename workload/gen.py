@@ -1,0 +1,344 @@
+"""Seeded synthetic paged-KV decode workloads.
+
+This module only *creates inputs*: sequence lengths, a shuffled physical block
+pool, per-sequence block tables (with a shared, reference-counted prefix where
+asked), query / key / value values drawn from N(0, 1) and rounded to the
+activation dtype, and the per-tensor fp8 scales.  It holds none of the
+method's arithmetic: no slot addressing, no cache write, no quantisation, no
+attention.  Both the CUDA path and the CPU oracle consume what it returns, each
+doing the method's steps on its own.
+
+Values are returned as raw 16-bit patterns (``np.uint16``) in the activation
+dtype ("f16" = IEEE binary16, "bf16" = bfloat16) so that neither consumer
+depends on the other's numeric types.
+
+The five named workloads follow the decode configurations that the pages'
+problem statement is built around:
+
+1. tiny: GQA 4/2, d=64, lengths [10, 45, 20, 33], f16, a 32-block pool;
+2. Qwen3-8B-shaped: 64 sequences, 32/8 heads, d=128, lengths U[512, 4096], bf16;
+3. Llama-3-70B-shaped: 32 sequences, 64/8 heads, lengths U[2048, 2560], bf16;
+4. long context: 8 x 32768 tokens, 64/8 heads, fp8-E4M3 KV with a per-tensor
+   scale, bf16 query;
+5. continuous batching: 256 sequences, MHA 32/32, all sharing one 1024-token
+   prefix (same physical blocks, refcount 256) plus private lognormal tails of
+   mean 300 tokens clipped to [1, 2048], f16.
+
+Block size is 16 tokens throughout ("Transformer 推理优化：KV Cache、PagedAttention
+与 vLLM", §3.2).  The pool holds the blocks in use plus 10 % free blocks; the
+physical ids are a seeded Fisher-Yates permutation of the pool, handed out in
+sequence order, so logically adjacent blocks sit far apart in memory.
+"""
+
+from __future__ import annotations
+
+import dataclasses
+import math
+from typing import List, Optional, Sequence
+
+import numpy as np
+import torch
+
+SEED_BASE = 369000
+BLOCK_SIZE = 16
+_CHUNK = 1 << 24  # values drawn per chunk when filling large K/V arrays
+
+
+@dataclasses.dataclass
+class Workload:
+    """One decode step's inputs plus the cache contents that precede it."""
+
+    name: str
+    seed: int
+    num_seqs: int
+    num_q_heads: int
+    num_kv_heads: int
+    head_dim: int
+    block_size: int
+    num_blocks: int
+    act_dtype: str  # dtype of q, of the new K/V rows and of the output
+    kv_dtype: str  # dtype of the cache pools: "f16" | "bf16" | "e4m3"
+    seq_lens: np.ndarray  # int32 [S]; counts the token written by this step
+    block_tables: np.ndarray  # int32 [S, max_blocks_per_seq]
+    refcount: np.ndarray  # int32 [num_blocks]: tables referencing each block
+    q: np.ndarray  # uint16 [S, Hq, d]
+    # tokens already in the cache before this step (positions < seq_len - 1)
+    prefill_seq: np.ndarray  # int32 [Tp]
+    prefill_pos: np.ndarray  # int32 [Tp]
+    k_prefill: np.ndarray  # uint16 [Tp, Hk, d]
+    v_prefill: np.ndarray  # uint16 [Tp, Hk, d]
+    # this step's new token of every sequence, at position seq_len - 1
+    k_new: np.ndarray  # uint16 [S, Hk, d]
+    v_new: np.ndarray  # uint16 [S, Hk, d]
+    k_scale: float  # fp32 value; 1.0 unless kv_dtype == "e4m3"
+    v_scale: float
+    free_blocks: np.ndarray  # int32: physical ids no table references
+    shared_prefix_blocks: int = 0
+
+    @property
+    def group(self) -> int:
+        return self.num_q_heads // self.num_kv_heads
+
+    @property
+    def max_blocks_per_seq(self) -> int:
+        return int(self.block_tables.shape[1])
+
+    @property
+    def max_seq_len(self) -> int:
+        return int(self.seq_lens.max()) if self.num_seqs else 0
+
+    @property
+    def softmax_scale(self) -> float:
+        return 1.0 / math.sqrt(self.head_dim)
+
+    @property
+    def new_seq(self) -> np.ndarray:
+        """Sequence index of each new token (one per sequence)."""
+        return np.arange(self.num_seqs, dtype=np.int32)
+
+    @property
+    def new_pos(self) -> np.ndarray:
+        """Position of each new token: the last one of its sequence."""
+        return (self.seq_lens - 1).astype(np.int32)
+
+    def kv_elem_bytes(self) -> int:
+        return 1 if self.kv_dtype == "e4m3" else 2
+
+    def act_elem_bytes(self) -> int:
+        return 2
+
+    def kv_bytes_logical(self) -> int:
+        """K+V bytes one decode pass reads: sum_s L_s * Hk * 2 * d * b_kv."""
+        return int(self.seq_lens.astype(np.int64).sum()) * self.num_kv_heads * 2 * self.head_dim * self.kv_elem_bytes()
+
+    def step_bytes(self) -> int:
+        """Algorithmic bytes of one step: K/V read once, q read, out written,
+        block tables and lengths read, and the new K/V rows written once
+        (read as activations, written into the pools)."""
+        S, Hq, Hk, d = self.num_seqs, self.num_q_heads, self.num_kv_heads, self.head_dim
+        qo = 2 * S * Hq * d * self.act_elem_bytes()
+        tables = self.block_tables.size * 4 + S * 4
+        new_rows = S * Hk * d * 2 * (self.act_elem_bytes() + self.kv_elem_bytes())
+        return self.kv_bytes_logical() + qo + tables + new_rows
+
+    def pool_elems(self) -> int:
+        return self.num_blocks * self.num_kv_heads * self.block_size * self.head_dim
+
+
+# ----------------------------------------------------------------------------
+# value drawing
+# ----------------------------------------------------------------------------
+
+def f32_to_bits(x: np.ndarray, dtype: str) -> np.ndarray:
+    """Round fp32 values to f16 / bf16 (round to nearest even) and return the
+    16-bit patterns.  This is input creation, done by torch's converters."""
+    t = torch.from_numpy(np.ascontiguousarray(x, dtype=np.float32))
+    if dtype == "f16":
+        return t.to(torch.float16).view(torch.int16).numpy().view(np.uint16)
+    if dtype == "bf16":
+        return t.to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    raise ValueError(f"unsupported activation dtype {dtype!r}")
+
+
+def bits_to_f32(bits: np.ndarray, dtype: str) -> np.ndarray:
+    """Widen 16-bit patterns back to fp32 (exact)."""
+    t = torch.from_numpy(np.ascontiguousarray(bits).view(np.int16))
+    if dtype == "f16":
+        return t.view(torch.float16).float().numpy()
+    if dtype == "bf16":
+        return t.view(torch.bfloat16).float().numpy()
+    raise ValueError(dtype)
+
+
+def draw_normal_bits(rng: np.random.Generator, shape, dtype: str) -> np.ndarray:
+    """N(0, 1) values drawn in fp32 and rounded to ``dtype``, filled in chunks."""
+    n = int(np.prod(shape))
+    out = np.empty(n, dtype=np.uint16)
+    for lo in range(0, n, _CHUNK):
+        hi = min(n, lo + _CHUNK)
+        out[lo:hi] = f32_to_bits(rng.standard_normal(hi - lo, dtype=np.float32), dtype)
+    return out.reshape(shape)
+
+
+def amax_of_bits(*arrays: np.ndarray, dtype: str) -> float:
+    m = 0.0
+    for a in arrays:
+        flat = a.reshape(-1)
+        for lo in range(0, flat.size, _CHUNK):
+            m = max(m, float(np.abs(bits_to_f32(flat[lo:lo + _CHUNK], dtype)).max(initial=0.0)))
+    return m
+
+
+def per_tensor_e4m3_scale(amax: float) -> float:
+    """Per-tensor fp8 scale amax / 448 as an fp32 value (448 is the E4M3
+    maximum: "大语言模型推理引擎深度剖析", §4.2).  A zero amax gives scale 1."""
+    if amax <= 0.0:
+        return 1.0
+    return float(np.float32(amax) / np.float32(448.0))
+
+
+# ----------------------------------------------------------------------------
+# block pool and tables
+# ----------------------------------------------------------------------------
+
+def blocks_needed(length: int, block_size: int) -> int:
+    return -(-int(length) // block_size)
+
+
+def build(
+    name: str,
+    seed: int,
+    seq_lens: Sequence[int],
+    num_q_heads: int,
+    num_kv_heads: int,
+    head_dim: int,
+    act_dtype: str,
+    kv_dtype: str,
+    block_size: int = BLOCK_SIZE,
+    num_blocks: Optional[int] = None,
+    pool_slack: float = 0.10,
+    shared_prefix_tokens: int = 0,
+    extra_table_cols: int = 0,
+    draw_kv: bool = True,
+) -> Workload:
+    """Draw one workload.
+
+    ``shared_prefix_tokens`` (a multiple of ``block_size``) makes every table
+    start with the same physical blocks.  ``extra_table_cols`` appends unused
+    table columns (filled with a free block id, so an over-read lands on
+    poisoned memory instead of outside the pool).  ``draw_kv=False`` skips the
+    prefill values (shape-only workloads for host-side tests).
+    """
+    rng = np.random.default_rng(seed)
+    seq_lens = np.asarray(seq_lens, dtype=np.int32)
+    S = int(seq_lens.size)
+    if shared_prefix_tokens % block_size:
+        raise ValueError("shared prefix must be block aligned")
+    if shared_prefix_tokens and S and int(seq_lens.min()) <= shared_prefix_tokens:
+        raise ValueError("every sequence must extend past the shared prefix")
+    nprefix = shared_prefix_tokens // block_size
+    nblk = [blocks_needed(L, block_size) for L in seq_lens]
+    private = [b - nprefix for b in nblk] if nprefix else nblk
+    used = nprefix + int(sum(private))
+    if num_blocks is None:
+        num_blocks = max(used + 1, int(math.ceil(used * (1.0 + pool_slack))))
+    if num_blocks < used:
+        raise ValueError("pool too small")
+    perm = rng.permutation(num_blocks).astype(np.int32)  # Fisher-Yates shuffle
+    mbs = max(max(nblk, default=0), 1) + extra_table_cols
+    cursor = 0
+    prefix_ids = perm[cursor:cursor + nprefix]
+    cursor += nprefix
+    tables = np.empty((S, mbs), dtype=np.int32)
+    refcount = np.zeros(num_blocks, dtype=np.int32)
+    for s in range(S):
+        own = perm[cursor:cursor + private[s]]
+        cursor += private[s]
+        row = np.concatenate([prefix_ids, own]) if nprefix else own
+        tables[s, :row.size] = row
+        refcount[row] += 1
+        tables[s, row.size:] = -1
+    free = perm[cursor:].copy()
+    pad = int(free[0]) if free.size else 0
+    tables[tables < 0] = pad
+
+    q = draw_normal_bits(rng, (S, num_q_heads, head_dim), act_dtype)
+    k_new = draw_normal_bits(rng, (S, num_kv_heads, head_dim), act_dtype)
+    v_new = draw_normal_bits(rng, (S, num_kv_heads, head_dim), act_dtype)
+
+    # tokens present before this step: the shared prefix once (through the
+    # first table), then every sequence's own tokens up to position L - 2
+    pseq: List[np.ndarray] = []
+    ppos: List[np.ndarray] = []
+    if nprefix and S:
+        pseq.append(np.zeros(shared_prefix_tokens, dtype=np.int32))
+        ppos.append(np.arange(shared_prefix_tokens, dtype=np.int32))
+    for s in range(S):
+        lo = shared_prefix_tokens if nprefix else 0
+        hi = int(seq_lens[s]) - 1
+        if hi > lo:
+            pseq.append(np.full(hi - lo, s, dtype=np.int32))
+            ppos.append(np.arange(lo, hi, dtype=np.int32))
+    prefill_seq = np.concatenate(pseq) if pseq else np.zeros(0, np.int32)
+    prefill_pos = np.concatenate(ppos) if ppos else np.zeros(0, np.int32)
+    Tp = int(prefill_seq.size)
+    if draw_kv:
+        k_prefill = draw_normal_bits(rng, (Tp, num_kv_heads, head_dim), act_dtype)
+        v_prefill = draw_normal_bits(rng, (Tp, num_kv_heads, head_dim), act_dtype)
+    else:
+        k_prefill = np.zeros((0, num_kv_heads, head_dim), np.uint16)
+        v_prefill = np.zeros((0, num_kv_heads, head_dim), np.uint16)
+        prefill_seq = prefill_seq[:0]
+        prefill_pos = prefill_pos[:0]
+
+    k_scale = v_scale = 1.0
+    if kv_dtype == "e4m3":
+        k_scale = per_tensor_e4m3_scale(amax_of_bits(k_prefill, k_new, dtype=act_dtype))
+        v_scale = per_tensor_e4m3_scale(amax_of_bits(v_prefill, v_new, dtype=act_dtype))
+    elif kv_dtype != act_dtype:
+        raise ValueError("a 16-bit cache must have the activation dtype")
+
+    return Workload(
+        name=name, seed=seed, num_seqs=S, num_q_heads=num_q_heads, num_kv_heads=num_kv_heads,
+        head_dim=head_dim, block_size=block_size, num_blocks=int(num_blocks),
+        act_dtype=act_dtype, kv_dtype=kv_dtype, seq_lens=seq_lens, block_tables=tables,
+        refcount=refcount, q=q, prefill_seq=prefill_seq, prefill_pos=prefill_pos,
+        k_prefill=k_prefill, v_prefill=v_prefill, k_new=k_new, v_new=v_new,
+        k_scale=k_scale, v_scale=v_scale, free_blocks=free, shared_prefix_blocks=nprefix,
+    )
+
+
+# ----------------------------------------------------------------------------
+# the five named decode workloads
+# ----------------------------------------------------------------------------
+
+CONFIG_NAMES = {
+    1: "tiny paged decode: GQA 4/2, d64, lens [10,45,20,33], f16, 32-block pool",
+    2: "Qwen3-8B-shaped decode: 64 seqs, 32/8 heads, d128, lens U[512,4096], bf16",
+    3: "Llama-3-70B-shaped decode: 32 seqs, 64/8 heads, d128, lens U[2048,2560], bf16",
+    4: "long-context fp8 KV: 8 x 32768, 64/8 heads, d128, E4M3 per-tensor scale, bf16 q, split 512",
+    5: "continuous batching: 256 seqs, MHA 32/32, d128, shared 1024-token prefix + lognormal tails, f16",
+}
+
+
+def config_seq_lens(cfg: int, rng: np.random.Generator) -> np.ndarray:
+    if cfg == 1:
+        return np.array([10, 45, 20, 33], dtype=np.int32)
+    if cfg == 2:
+        return rng.integers(512, 4096, size=64, endpoint=True).astype(np.int32)
+    if cfg == 3:
+        return rng.integers(2048, 2560, size=32, endpoint=True).astype(np.int32)
+    if cfg == 4:
+        return np.full(8, 32768, dtype=np.int32)
+    if cfg == 5:
+        sigma = 1.0
+        mu = math.log(300.0) - sigma * sigma / 2.0  # pre-clip mean 300
+        tails = np.rint(rng.lognormal(mu, sigma, size=256))
+        tails = np.clip(tails, 1, 2048).astype(np.int32)
+        return (1024 + tails).astype(np.int32)
+    raise ValueError(f"unknown config {cfg}")
+
+
+def config(cfg: int, draw_kv: bool = True) -> Workload:
+    """The named decode workload ``cfg`` (1..5), seeded with 369000 + cfg."""
+    seed = SEED_BASE + cfg
+    lens = config_seq_lens(cfg, np.random.default_rng([seed, 1]))
+    name = CONFIG_NAMES[cfg]
+    if cfg == 1:
+        return build(name, seed, lens, 4, 2, 64, "f16", "f16", num_blocks=32, draw_kv=draw_kv)
+    if cfg == 2:
+        return build(name, seed, lens, 32, 8, 128, "bf16", "bf16", draw_kv=draw_kv)
+    if cfg == 3:
+        return build(name, seed, lens, 64, 8, 128, "bf16", "bf16", draw_kv=draw_kv)
+    if cfg == 4:
+        return build(name, seed, lens, 64, 8, 128, "bf16", "e4m3", draw_kv=draw_kv)
+    if cfg == 5:
+        return build(name, seed, lens, 32, 32, 128, "f16", "f16", shared_prefix_tokens=1024,
+                     draw_kv=draw_kv)
+    raise ValueError(cfg)
+
+
+def poison_byte() -> int:
+    """Fill byte for pools before any write: 0xFF makes every f16 / bf16 pair
+    and every E4M3 byte a NaN, so any read of an unwritten slot shows up."""
+    return 0xFF
