@@ -1,0 +1,447 @@
+"""Benchmark of one paged decode step on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--config 2] [--mode split|single] [--partition 512]
+
+A step is one pass of the whole hot path over one batch: slot mapping of the
+new tokens, cache write of their K/V rows, and decode attention (split-KV
+partition + reduce by default).  The default workload is the Qwen3-8B-shaped
+decode step: 64 sequences, 32 query / 8 KV heads, head_dim 128, bf16, lengths
+U[512, 4096], 16-token blocks in a shuffled pool.  Its K/V (~585 MB) is larger
+than L2 (126 MB), so no L2 flush is needed between steps.
+
+Output: one JSON line on rank 0.  ``value`` is KV GB/s of the whole job
+(algorithmic step bytes of all ranks / max-over-ranks step time); ``e2e`` is
+the same with the step's inputs copied from pinned host memory and its output
+read back inside the timed region; ``roofline`` is for the attention launch
+(partition + reduce kernels) against the measured HBM copy bandwidth;
+``cpu_baseline`` times the CPU oracle on a bounded sample.
+
+``--impl reference`` times the CPU oracle itself as the reference arm (rank 0
+only; other ranks exit without work).
+
+Multi-GPU: independent replicas (the decode path needs no exchange), one
+process per GPU under torchrun; weak scaling.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "paged decode attention KV GB/s & tokens/s per step; % of B200 HBM roofline"
+FALLBACK_HBM_GBS = 6650.0
+
+
+# ---------------------------------------------------------------------------
+# helpers
+# ---------------------------------------------------------------------------
+
+def measured_hbm_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except Exception:  # noqa: BLE001
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "paged_kv_cache_369_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode())
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(cfg: int, mode: str):
+    """DRAM bytes per attention launch from the committed ncu summary, if it
+    was taken on the current kernel sources (else None)."""
+    path = os.path.join(ROOT, "profiles", "decode_traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f)
+    except Exception:  # noqa: BLE001
+        return None
+    key = f"config{cfg}_{mode}"
+    ent = rec.get(key)
+    if not ent or ent.get("kernel_hash") != kernel_source_hash():
+        return None
+    return ent.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """SM clock and throttle reasons from NVML, sampled in a thread."""
+
+    REASONS = {
+        0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+        0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+        0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+        0x100: "display_clock_setting",
+    }
+
+    def __init__(self, device_index: int, period_s: float = 0.005):
+        self.samples = []
+        self.reasons = set()
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._t = None
+        self.period = period_s
+        self.ok = False
+        try:
+            import pynvml
+
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:  # noqa: BLE001
+            self.ok = False
+
+    def _sample(self):
+        nv = self._nv
+        self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+        try:
+            mask = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+        except Exception:  # noqa: BLE001
+            mask = nv.nvmlDeviceGetCurrentClocksThrottleReasons(self._h)
+        for bit, name in self.REASONS.items():
+            if mask & bit:
+                self.reasons.add(name)
+
+    def _run(self):
+        while not self._stop.is_set():
+            self._sample()
+            time.sleep(self.period)
+
+    def start(self):
+        if self.ok:
+            self._sample()
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+
+    def stop(self):
+        if self.ok:
+            self._stop.set()
+            self._t.join()
+            self._sample()
+
+    def summary(self):
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvml unavailable"]}
+        return {"sm_mhz": float(statistics.median(self.samples)), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons - {"gpu_idle"}), "samples": len(self.samples)}
+
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def max_over_ranks(x: float, device) -> float:
+    """Max of a per-rank float over the process group (identity without one)."""
+    import torch
+    import torch.distributed as dist
+
+    if not (dist.is_available() and dist.is_initialized()):
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def sum_over_ranks(x: float, device) -> float:
+    import torch
+    import torch.distributed as dist
+
+    if not (dist.is_available() and dist.is_initialized()):
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+def workload_config(w, cfg: int, mode: str, P: int) -> dict:
+    return {
+        "workload": w.name, "config_id": cfg, "num_seqs": w.num_seqs,
+        "num_q_heads": w.num_q_heads, "num_kv_heads": w.num_kv_heads, "head_dim": w.head_dim,
+        "block_size": w.block_size, "kv_dtype": w.kv_dtype, "act_dtype": w.act_dtype,
+        "seq_len_mean": float(w.seq_lens.mean()), "seq_len_min": int(w.seq_lens.min()),
+        "seq_len_max": int(w.seq_lens.max()), "num_blocks": w.num_blocks, "seed": w.seed,
+        "mode": mode, "partition_size": P if mode == "split" else None,
+        "l2": "inputs larger than L2: no flush" if w.kv_bytes_logical() > 256e6
+        else "L2 flushed (256 MB write) between steps",
+    }
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle timing (reference arm and cpu_baseline)
+# ---------------------------------------------------------------------------
+
+def oracle_units(w):
+    """(sequence, KV head) units of the workload, each with its query heads."""
+    return [(s, h) for s in range(w.num_seqs) for h in range(w.num_kv_heads)]
+
+
+def time_oracle_units(w, kc, vc, units, budget_s=None):
+    """Run the oracle's decode over the query heads of the given units; return
+    (seconds, KV bytes those units read once, units done)."""
+    import oracle
+
+    g = w.group
+    done = 0
+    kv_bytes = 0
+    t0 = time.perf_counter()
+    for (s, kvh) in units:
+        pairs = np.array([(s, kvh * g + i) for i in range(g)], dtype=np.int32)
+        oracle.decode_for(w, kc, vc, pairs)
+        kv_bytes += int(w.seq_lens[s]) * 2 * w.head_dim * w.kv_elem_bytes()
+        done += 1
+        if budget_s is not None and time.perf_counter() - t0 > budget_s:
+            break
+    return time.perf_counter() - t0, kv_bytes, done
+
+
+def cpu_baseline(w, budget_s: float = 15.0):
+    import oracle
+
+    t0 = time.perf_counter()
+    kc, vc = oracle.caches_for(w)
+    build_s = time.perf_counter() - t0
+    units = oracle_units(w)
+    rng = np.random.default_rng(0)
+    order = rng.permutation(len(units))
+    secs, kv_bytes, done = time_oracle_units(w, kc, vc, [units[i] for i in order], budget_s)
+    return {
+        "value": kv_bytes / secs / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle",
+        "sample": f"{done} of {len(units)} (sequence, KV head) units of the same workload, "
+                  f"fp64 C oracle, one thread ({secs:.1f} s; pools built in {build_s:.1f} s, untimed)",
+    }
+
+
+def run_reference(args):
+    world, rank, _ = dist_env()
+    if rank != 0:
+        return 0
+    import workload
+
+    w = workload.config(args.config)
+    import oracle
+
+    kc, vc = oracle.caches_for(w)
+    units = oracle_units(w)
+    for i in range(args.warmup):
+        time_oracle_units(w, kc, vc, [units[i % len(units)]])
+    tot_s, tot_b = 0.0, 0
+    for i in range(args.steps):
+        secs, b, _ = time_oracle_units(w, kc, vc, [units[(args.warmup + i) % len(units)]])
+        tot_s += secs
+        tot_b += b
+    value = tot_b / tot_s / 1e9
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * tot_s / max(1, args.steps), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": workload_config(w, args.config, args.mode, args.partition),
+        "cpu_baseline": {"value": value, "unit": "GB/s", "cores": 1, "kind": "oracle",
+                         "sample": "each step: the query heads of one (sequence, KV head) unit "
+                                   "of the workload, fp64 C oracle, one thread"},
+        "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------------------
+# the CUDA path
+# ---------------------------------------------------------------------------
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    world, rank, local = dist_env()
+    if args.gpus != world and world > 1:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE {world}")
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120),
+                                device_id=device)
+
+    import workload
+    from paged_kv_cache_369_b200.runner import PagedDecode, algorithmic_decode_bytes
+
+    w = workload.config(args.config)
+    stream = torch.cuda.Stream(device)
+    with torch.cuda.stream(stream):
+        dec = PagedDecode(w, device=str(device), mode=args.mode, partition_size=args.partition,
+                          stream=stream)
+    step_bytes = w.step_bytes()
+    attn_bytes = algorithmic_decode_bytes(w)
+    flush = None
+    if w.kv_bytes_logical() <= 256e6:
+        flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=device)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize(device)
+
+    # ---- device-resident timing ------------------------------------------
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            dec.step()
+            if flush is not None:
+                flush.fill_(1)
+    barrier()
+    dec.dev_err.zero_()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    flush_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)] \
+        if flush is not None else None
+    clocks = ClockSampler(device.index if device.index is not None else 0)
+    clocks.start()
+    barrier()
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        t_start.record(stream)
+        for i in range(args.steps):
+            e0, e1, e2 = ev[i]
+            e0.record(stream)
+            dec.write_new()
+            e1.record(stream)
+            dec.attend()
+            e2.record(stream)
+            if flush is not None:
+                flush_ev[i][0].record(stream)
+                flush.fill_(1)
+                flush_ev[i][1].record(stream)
+        t_end.record(stream)
+    barrier()
+    clocks.stop()
+    total_ms = t_start.elapsed_time(t_end)
+    flush_ms = sum(a.elapsed_time(b) for a, b in flush_ev) if flush_ev else 0.0
+    step_ms_local = (total_ms - flush_ms) / args.steps
+    attn_ms = statistics.mean(e1.elapsed_time(e2) for _, e1, e2 in ev)
+    write_ms = statistics.mean(e0.elapsed_time(e1) for e0, e1, _ in ev)
+    err = dec.error()
+    step_ms = max_over_ranks(step_ms_local, device)
+    total_bytes = sum_over_ranks(float(step_bytes), device)
+    value = total_bytes / (step_ms * 1e-3) / 1e9
+
+    # ---- end to end: pinned host inputs in, output out, every step --------
+    host_q = dec.q.cpu().pin_memory()
+    host_kn = dec.k_new.cpu().pin_memory()
+    host_vn = dec.v_new.cpu().pin_memory()
+    host_bt = dec.block_tables.cpu().pin_memory()
+    host_sl = dec.seq_lens.cpu().pin_memory()
+    host_out = torch.empty_like(dec.out, device="cpu").pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in (host_q, host_kn, host_vn, host_bt, host_sl))
+    d2h = host_out.numel() * host_out.element_size()
+    e2e_steps = max(1, min(args.steps, 200))
+    barrier()
+    e_s = torch.cuda.Event(enable_timing=True)
+    e_e = torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        e_s.record(stream)
+        for _ in range(e2e_steps):
+            dec.q.copy_(host_q, non_blocking=True)
+            dec.k_new.copy_(host_kn, non_blocking=True)
+            dec.v_new.copy_(host_vn, non_blocking=True)
+            dec.block_tables.copy_(host_bt, non_blocking=True)
+            dec.seq_lens.copy_(host_sl, non_blocking=True)
+            dec.step()
+            host_out.copy_(dec.out, non_blocking=True)
+            if flush is not None:
+                flush.fill_(1)
+        e_e.record(stream)
+    barrier()
+    e2e_ms = max_over_ranks(e_s.elapsed_time(e_e) / e2e_steps, device)
+    e2e_value = total_bytes / (e2e_ms * 1e-3) / 1e9
+
+    result = None
+    if rank == 0:
+        peak, peak_kind = measured_hbm_peak()
+        achieved = attn_bytes / (attn_ms * 1e-3) / 1e9
+        traffic = recorded_traffic(args.config, args.mode)
+        result = {
+            "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": w.kv_dtype if w.kv_dtype != "e4m3" else "e4m3 KV / bf16 q, f32 math",
+            "data": "synthetic: seeded N(0,1) q/K/V, shuffled block pool, no dataset",
+            "config": workload_config(w, args.config, args.mode, args.partition),
+            "us_per_step": step_ms * 1e3,
+            "tokens_per_s": world * w.num_seqs / (step_ms * 1e-3),
+            "attention_us": attn_ms * 1e3,
+            "cache_write_us": write_ms * 1e3,
+            "kv_bytes_per_step": w.kv_bytes_logical(),
+            "step_bytes": step_bytes,
+            "roofline": {
+                "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                "frac": achieved / peak, "traffic": traffic,
+                "kernel": "attention launch (decode partition kernel + split reduce kernel)"
+                if args.mode == "split" else "decode kernel (single pass)",
+                "peak_source": f"{peak_kind} HBM copy bandwidth (MEASURED_PEAKS.json hbm_gbs)"
+                if peak_kind == "measured" else "fallback 6.65 TB/s",
+                "algorithmic_bytes_per_launch": attn_bytes,
+            },
+            "e2e": {"value": e2e_value, "unit": "GB/s", "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h, "steps": e2e_steps},
+            "gpu_launches": args.steps * dec.launches_per_step(),
+            "clocks": clocks.summary(),
+            "device_error": err,
+        }
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        if world == 1 and not args.no_cpu_baseline:
+            result["cpu_baseline"] = cpu_baseline(w, budget_s=args.cpu_budget)
+        print(json.dumps(result), flush=True)
+    return 0
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--config", type=int, default=2, choices=(1, 2, 3, 4, 5))
+    ap.add_argument("--mode", choices=("split", "single"), default="split")
+    ap.add_argument("--partition", type=int, default=512)
+    ap.add_argument("--cpu-budget", type=float, default=15.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,192 @@
+/*
+ * pa.h -- C ABI of the B200 paged-KV-cache decode library (libpa369.so).
+ *
+ * The operation, as the pages state it:
+ *   - the KV cache is cut into fixed blocks of 16 tokens that sit anywhere in a
+ *     physical block pool; each sequence owns a block table mapping its logical
+ *     blocks to physical ones ("Transformer 推理优化：KV Cache、PagedAttention 与
+ *     vLLM", §3.2-§3.3; "KV Cache 与 PageAttention深度实战", §3.1-§3.2);
+ *   - a decode step computes, for the single new query row of each sequence,
+ *     Attention(Q_t, [K_prefix, K_t], [V_prefix, V_t]) =
+ *     softmax(Q_t K^T / sqrt(d_k)) V, reading K and V through the block table
+ *     ("KV Cache 与 PageAttention深度实战", §1.2 and §3.2-§3.3);
+ *   - the new token's K/V row is appended into its (block, offset) slot; a new
+ *     block is opened every 16 tokens ("vLLM推理引擎深度解析：PagedAttention与
+ *     连续批处理", §2.2-§2.3);
+ *   - the cache may hold FP8 E4M3 values (range +-448) in place of 16-bit ones
+ *     ("大语言模型推理引擎深度剖析：从 KV Cache 内存管理到 PagedAttention、投机
+ *     解码与量化加速的完全工程指南", §4.2-§4.3).
+ *
+ * Conventions shared by every entry point:
+ *   - Every pointer argument is DEVICE memory owned by the caller, unless the
+ *     comment says otherwise.  The library allocates nothing, keeps no state
+ *     between calls and never synchronises: work is enqueued on `stream`
+ *     (a cudaStream_t; NULL = the legacy default stream) and the call returns.
+ *   - Layouts are dense, row-major, C order:
+ *       q, out            [num_seqs, num_q_heads, head_dim]
+ *       k_new, v_new      [num_tokens, num_kv_heads, head_dim]
+ *       k_cache, v_cache  [num_blocks, num_kv_heads, block_size, head_dim]
+ *       block_tables      int32 [num_seqs, max_blocks_per_seq]
+ *       seq_lens          int32 [num_seqs]   (tokens in the cache, the one
+ *                                             written this step included)
+ *       slot_mapping      int64 [num_tokens] (slot = block * block_size + offset;
+ *                                             a negative slot is padding)
+ *   - GQA: query head h reads KV head h / (num_q_heads / num_kv_heads).
+ *   - q, out, the caches and k_new / v_new must be 16-byte aligned.
+ *   - Host-side argument checks run before any launch and return
+ *     PA_ERR_INVALID_ARG or PA_ERR_UNSUPPORTED without touching the GPU; a
+ *     failed launch returns PA_ERR_CUDA.
+ *   - `dev_err` (nullable, device int32) receives the first device-side error
+ *     of the call (PA_ERR_DEVICE_BOUNDS for a block-table entry, slot, sequence
+ *     index or length outside its range; PA_ERR_DEVICE_TIMEOUT for an
+ *     asynchronous copy that did not complete in time).  The kernels check every
+ *     such index before using it and skip the access, so a corrupt table never
+ *     makes them read or write outside the buffers; the affected outputs are
+ *     still written (finite).  The caller zeroes *dev_err and reads it after
+ *     synchronising.
+ */
+#ifndef PA369_H
+#define PA369_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum pa_status {
+    PA_OK = 0,
+    PA_ERR_INVALID_ARG = 1,    /* null pointer, bad size, misaligned buffer, ... */
+    PA_ERR_UNSUPPORTED = 2,    /* valid but not implemented (head_dim, dtype pair, ...) */
+    PA_ERR_CUDA = 3,           /* a CUDA launch or query failed */
+    PA_ERR_DEVICE_BOUNDS = 4,  /* written to *dev_err by a kernel */
+    PA_ERR_DEVICE_TIMEOUT = 5  /* written to *dev_err by a kernel */
+} pa_status;
+
+typedef enum pa_dtype {
+    PA_F16 = 0,       /* IEEE binary16 */
+    PA_BF16 = 1,      /* bfloat16 */
+    PA_FP8_E4M3 = 2   /* OCP E4M3 (FN): bias 7, max 448, no infinities */
+} pa_dtype;
+
+/* Human-readable name of a status code (host only, static string). */
+const char *pa_status_string(pa_status status);
+
+/* Library version as MAJOR*10000 + MINOR*100 + PATCH (host only). */
+int pa_version(void);
+
+/*
+ * pa_slot_mapping -- slot of each token to be written (block-table lookup).
+ *
+ * Source: "Transformer 推理优化：KV Cache、PagedAttention 与 vLLM", §3.3: logical
+ * block pos / block_size of sequence s lives in physical block
+ * block_tables[s][pos / block_size]; the token sits at offset pos % block_size.
+ *
+ *   slot_mapping[t] = block_tables[s][pos / B] * B + pos % B,
+ *     s   = token_seq ? token_seq[t] : t         (s < 0: padding, slot = -1)
+ *     pos = token_pos ? token_pos[t] : seq_lens[s] - 1   (decode: last token)
+ *
+ * seq_lens may be NULL when token_pos is given.  A sequence index >= num_seqs,
+ * a position outside [0, max_blocks_per_seq * B) or a table entry outside
+ * [0, num_blocks) gives slot -1 and PA_ERR_DEVICE_BOUNDS in *dev_err.
+ */
+pa_status pa_slot_mapping(int64_t *slot_mapping, const int32_t *block_tables,
+                          int max_blocks_per_seq, const int32_t *seq_lens,
+                          const int32_t *token_seq, const int32_t *token_pos, int num_tokens,
+                          int num_seqs, int block_size, int num_blocks, int *dev_err,
+                          void *stream);
+
+/*
+ * pa_cache_write -- append each token's K/V rows into its cache slot.
+ *
+ * Source: "vLLM推理引擎深度解析：PagedAttention与连续批处理", §2.2 (one new block
+ * every 16 generated tokens; the token goes to its slot) and, for FP8, "大语言
+ * 模型推理引擎深度剖析", §4.3 (KV stored as E4M3, dequantised for attention).
+ *
+ *   k_cache[slot / B][h][slot % B][:] = k_new[t][h][:]   (likewise V)
+ *
+ * act_dtype (of k_new / v_new) is PA_F16 or PA_BF16.  kv_dtype is act_dtype
+ * (a bit-exact copy) or PA_FP8_E4M3, in which case each value is stored as
+ * e4m3(x / scale): x widened to fp32, divided by the per-tensor scale in fp32
+ * (IEEE round to nearest), rounded to nearest even onto the E4M3 grid and
+ * saturated to +-448; k_scale / v_scale must then be finite and > 0.
+ * Negative slots are skipped; a slot >= num_blocks * B is skipped with
+ * PA_ERR_DEVICE_BOUNDS.  Tokens must map to distinct slots.
+ */
+pa_status pa_cache_write(const void *k_new, const void *v_new, void *k_cache, void *v_cache,
+                         const int64_t *slot_mapping, int num_tokens, int num_blocks,
+                         int num_kv_heads, int head_dim, int block_size, pa_dtype act_dtype,
+                         pa_dtype kv_dtype, float k_scale, float v_scale, int *dev_err,
+                         void *stream);
+
+/*
+ * pa_decode -- paged decode attention, one pass per (sequence, KV head).
+ *
+ * Source: "KV Cache 与 PageAttention深度实战", §1.2 (softmax(Q K^T / sqrt(d_k)) V
+ * with one new query row per step), §3.2 (reading K/V through the block table
+ * gathers them implicitly) and §3.3 (paged block addressing, coalesced loads,
+ * the block table kept on chip).
+ *
+ * For every sequence s, query head h, with g = num_q_heads / num_kv_heads and
+ * L = seq_lens[s]:
+ *   out[s][h] = sum_t p_t * V_t,  p = softmax_t(softmax_scale * q[s][h] . K_t),
+ *   t < L, K_t / V_t rows of KV head h / g read at block_tables[s][t / 16],
+ *   offset t % 16.  For an E4M3 cache, K_t = code * k_scale, V_t = code * v_scale.
+ * L = 0 gives a zero row.  Slots at t >= L (the tail of the last block) and
+ * unused table entries are never read into the result.
+ *
+ * Supported: block_size 16, head_dim 64 or 128, num_q_heads a multiple of
+ * num_kv_heads, q_dtype (= out dtype) PA_F16 / PA_BF16, kv_dtype = q_dtype or
+ * PA_FP8_E4M3.  Arithmetic is fp32; out is rounded to nearest even once.
+ */
+pa_status pa_decode(void *out, const void *q, const void *k_cache, const void *v_cache,
+                    const int32_t *block_tables, int max_blocks_per_seq, const int32_t *seq_lens,
+                    int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
+                    int block_size, int num_blocks, float softmax_scale, pa_dtype q_dtype,
+                    pa_dtype kv_dtype, float k_scale, float v_scale, int *dev_err,
+                    void *stream);
+
+/*
+ * Workspace bytes pa_decode_split_reduce needs: with
+ * NP = ceil(max_seq_len / partition_size) partitions,
+ *   lse [num_seqs, num_q_heads, NP] fp32, then o [num_seqs, num_q_heads, NP, head_dim] fp32,
+ * each section starting on a 256-byte boundary.  Returns 0 on invalid input.
+ * Host only.
+ */
+size_t pa_split_workspace_bytes(int num_seqs, int num_q_heads, int head_dim, int max_seq_len,
+                                int partition_size);
+
+/*
+ * pa_decode_split_reduce -- split-KV decode: partition kernel + reduce kernel.
+ *
+ * Same result as pa_decode (up to fp32 rounding order), computed in two
+ * launches for long or uneven contexts.  The pages do not describe this split;
+ * it is the standard log-sum-exp decomposition of the same softmax.
+ *   1. Partition: for every (s, KV head, p) the tokens
+ *      [p * P, min((p + 1) * P, L)) of sequence s give, per query head,
+ *        lse[s][h][p] = ln sum_t exp(softmax_scale * q . K_t)   (-inf if empty)
+ *        o[s][h][p][:] = sum_t softmax-weight_t V_t over the partition (0 if empty)
+ *   2. Reduce: M = max_p lse, w_p = exp(lse_p - M),
+ *        out[s][h] = sum_p w_p o_p / sum_p w_p      (0 if every partition is empty)
+ * partition_size P is a positive multiple of block_size; max_seq_len bounds
+ * every seq_lens[s] (a longer one is truncated and flags PA_ERR_DEVICE_BOUNDS).
+ * workspace (device, caller-owned, >= pa_split_workspace_bytes(...) bytes,
+ * 256-byte aligned) holds the partials in the layout above after the call;
+ * it needs no initialisation.
+ */
+pa_status pa_decode_split_reduce(void *out, const void *q, const void *k_cache,
+                                 const void *v_cache, const int32_t *block_tables,
+                                 int max_blocks_per_seq, const int32_t *seq_lens, int num_seqs,
+                                 int num_q_heads, int num_kv_heads, int head_dim,
+                                 int block_size, int num_blocks, float softmax_scale,
+                                 pa_dtype q_dtype, pa_dtype kv_dtype, float k_scale,
+                                 float v_scale, int partition_size, int max_seq_len,
+                                 void *workspace, size_t workspace_bytes, int *dev_err,
+                                 void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PA369_H */

@@ -287,7 +287,8 @@ def caches_for(w, include_new: bool = True) -> Tuple[np.ndarray, np.ndarray]:
         cache_write(w.k_prefill, w.v_prefill, kc, vc, slots, w.num_blocks, w.num_kv_heads,
                     w.head_dim, w.block_size, w.act_dtype, w.kv_dtype, w.k_scale, w.v_scale)
     if include_new and w.num_seqs:
-        slots = slot_mapping(w.block_tables, w.seq_lens, None, None, w.num_seqs, w.block_size)
+        slots = slot_mapping(w.block_tables, w.seq_lens, w.new_seq, None, w.num_seqs,
+                             w.block_size)
         cache_write(w.k_new, w.v_new, kc, vc, slots, w.num_blocks, w.num_kv_heads, w.head_dim,
                     w.block_size, w.act_dtype, w.kv_dtype, w.k_scale, w.v_scale)
     return kc, vc

@@ -1,0 +1,190 @@
+"""B200-native paged KV cache decode: Python binding of libpa369.so.
+
+Argument marshalling only: every function here forwards to the C ABI of the
+same name (include/pa.h), whose kernels do all of the work.  Tensors are torch
+CUDA tensors (device memory and streams come from PyTorch); integer pointers
+are accepted too.  A non-OK status raises ``PaError``.
+
+The shared library is built in-tree by ``python -m paged_kv_cache_369_b200.build``;
+importing this package without it raises ImportError: there is no fallback.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Union
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libpa369.so")
+
+PA_OK = 0
+PA_ERR_INVALID_ARG = 1
+PA_ERR_UNSUPPORTED = 2
+PA_ERR_CUDA = 3
+PA_ERR_DEVICE_BOUNDS = 4
+PA_ERR_DEVICE_TIMEOUT = 5
+
+PA_F16 = 0
+PA_BF16 = 1
+PA_FP8_E4M3 = 2
+
+# every extern "C" symbol declared in include/pa.h
+SYMBOLS = (
+    "pa_status_string", "pa_version", "pa_slot_mapping", "pa_cache_write", "pa_decode",
+    "pa_split_workspace_bytes", "pa_decode_split_reduce",
+)
+
+
+class PaError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {pa_status_string(status)}")
+
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(
+        f"{LIB_PATH} is missing: build it with `python -m paged_kv_cache_369_b200.build` "
+        "(nvcc, sm_100a). There is no CPU fallback.")
+
+_lib = ctypes.CDLL(LIB_PATH)
+_P, _I, _F, _S = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+
+_lib.pa_status_string.restype = ctypes.c_char_p
+_lib.pa_status_string.argtypes = [_I]
+_lib.pa_version.restype = _I
+_lib.pa_version.argtypes = []
+_lib.pa_slot_mapping.restype = _I
+_lib.pa_slot_mapping.argtypes = [_P, _P, _I, _P, _P, _P, _I, _I, _I, _I, _P, _P]
+_lib.pa_cache_write.restype = _I
+_lib.pa_cache_write.argtypes = [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _F, _P, _P]
+_lib.pa_decode.restype = _I
+_lib.pa_decode.argtypes = [_P, _P, _P, _P, _P, _I, _P, _I, _I, _I, _I, _I, _I, _F, _I, _I, _F,
+                           _F, _P, _P]
+_lib.pa_split_workspace_bytes.restype = _S
+_lib.pa_split_workspace_bytes.argtypes = [_I, _I, _I, _I, _I]
+_lib.pa_decode_split_reduce.restype = _I
+_lib.pa_decode_split_reduce.argtypes = [_P, _P, _P, _P, _P, _I, _P, _I, _I, _I, _I, _I, _I, _F,
+                                        _I, _I, _F, _F, _I, _I, _P, _S, _P, _P]
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded libpa369.so with its argument types set."""
+    return _lib
+
+
+Ptr = Union[None, int, "torch.Tensor"]  # noqa: F821
+
+
+def _ptr(x: Ptr) -> Optional[int]:
+    if x is None:
+        return None
+    if isinstance(x, int):
+        return x
+    return x.data_ptr()
+
+
+def _stream(stream) -> Optional[int]:
+    if stream is None:
+        import torch
+
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _check(status: int, where: str) -> None:
+    if status != PA_OK:
+        raise PaError(status, where)
+
+
+def dtype_code(dtype) -> int:
+    """pa_dtype of a torch dtype (uint8 storage means E4M3 codes)."""
+    import torch
+
+    if dtype == torch.float16:
+        return PA_F16
+    if dtype == torch.bfloat16:
+        return PA_BF16
+    if dtype in (torch.uint8, getattr(torch, "float8_e4m3fn", None)):
+        return PA_FP8_E4M3
+    raise ValueError(f"no pa_dtype for {dtype}")
+
+
+def pa_status_string(status: int) -> str:
+    return _lib.pa_status_string(int(status)).decode()
+
+
+def pa_version() -> int:
+    return int(_lib.pa_version())
+
+
+def pa_slot_mapping(slot_mapping, block_tables, seq_lens, token_seq, token_pos, num_tokens: int,
+                    num_seqs: int, num_blocks: int, block_size: int = 16, dev_err=None,
+                    stream=None) -> None:
+    mbs = int(block_tables.shape[1]) if hasattr(block_tables, "shape") else 0
+    _check(_lib.pa_slot_mapping(_ptr(slot_mapping), _ptr(block_tables), mbs, _ptr(seq_lens),
+                                _ptr(token_seq), _ptr(token_pos), int(num_tokens), int(num_seqs),
+                                int(block_size), int(num_blocks), _ptr(dev_err), _stream(stream)),
+           "pa_slot_mapping")
+
+
+def pa_cache_write(k_new, v_new, k_cache, v_cache, slot_mapping, k_scale: float = 1.0,
+                   v_scale: float = 1.0, dev_err=None, stream=None) -> None:
+    T, Hk, d = (int(x) for x in k_new.shape)
+    nb, _, B, _ = (int(x) for x in k_cache.shape)
+    _check(_lib.pa_cache_write(_ptr(k_new), _ptr(v_new), _ptr(k_cache), _ptr(v_cache),
+                               _ptr(slot_mapping), T, nb, Hk, d, B, dtype_code(k_new.dtype),
+                               dtype_code(k_cache.dtype), float(k_scale), float(v_scale),
+                               _ptr(dev_err), _stream(stream)),
+           "pa_cache_write")
+
+
+def pa_decode(out, q, k_cache, v_cache, block_tables, seq_lens, softmax_scale: float,
+              k_scale: float = 1.0, v_scale: float = 1.0, dev_err=None, stream=None) -> None:
+    S, Hq, d = (int(x) for x in q.shape)
+    nb, Hk, B, _ = (int(x) for x in k_cache.shape)
+    _check(_lib.pa_decode(_ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables),
+                          int(block_tables.shape[1]), _ptr(seq_lens), S, Hq, Hk, d, B, nb,
+                          float(softmax_scale), dtype_code(q.dtype), dtype_code(k_cache.dtype),
+                          float(k_scale), float(v_scale), _ptr(dev_err), _stream(stream)),
+           "pa_decode")
+
+
+def pa_split_workspace_bytes(num_seqs: int, num_q_heads: int, head_dim: int, max_seq_len: int,
+                             partition_size: int) -> int:
+    return int(_lib.pa_split_workspace_bytes(num_seqs, num_q_heads, head_dim, max_seq_len,
+                                             partition_size))
+
+
+def pa_decode_split_reduce(out, q, k_cache, v_cache, block_tables, seq_lens,
+                           softmax_scale: float, partition_size: int, max_seq_len: int,
+                           workspace, k_scale: float = 1.0, v_scale: float = 1.0, dev_err=None,
+                           stream=None) -> None:
+    S, Hq, d = (int(x) for x in q.shape)
+    nb, Hk, B, _ = (int(x) for x in k_cache.shape)
+    ws_bytes = workspace.numel() * workspace.element_size()
+    _check(_lib.pa_decode_split_reduce(_ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache),
+                                       _ptr(block_tables), int(block_tables.shape[1]),
+                                       _ptr(seq_lens), S, Hq, Hk, d, B, nb, float(softmax_scale),
+                                       dtype_code(q.dtype), dtype_code(k_cache.dtype),
+                                       float(k_scale), float(v_scale), int(partition_size),
+                                       int(max_seq_len), _ptr(workspace), ws_bytes,
+                                       _ptr(dev_err), _stream(stream)),
+           "pa_decode_split_reduce")
+
+
+def split_workspace_views(workspace, num_seqs: int, num_q_heads: int, head_dim: int,
+                          max_seq_len: int, partition_size: int):
+    """(lse [S, Hq, NP], o [S, Hq, NP, d]) fp32 views of a split workspace, in
+    the layout pa.h documents."""
+    import torch
+
+    np_ = max(1, -(-max_seq_len // partition_size)) if max_seq_len > 0 else 1
+    rows = num_seqs * num_q_heads * np_
+    lse_bytes = (rows * 4 + 255) // 256 * 256
+    flat = workspace.view(torch.uint8)
+    lse = flat[:rows * 4].view(torch.float32).view(num_seqs, num_q_heads, np_)
+    o = flat[lse_bytes:lse_bytes + rows * head_dim * 4].view(torch.float32)
+    return lse, o.view(num_seqs, num_q_heads, np_, head_dim)

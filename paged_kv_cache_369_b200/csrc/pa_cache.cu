@@ -1,0 +1,130 @@
+// Slot mapping and cache write: the append side of the paged KV cache.
+//
+// Slot of a token: its sequence's block table maps logical block pos / 16 to
+// a physical block; the token sits at offset pos % 16 ("Transformer 推理优化：
+// KV Cache、PagedAttention 与 vLLM", §3.3).  The cache write stores each
+// token's per-head K/V rows there, one new block being opened every 16 tokens
+// ("vLLM推理引擎深度解析：PagedAttention与连续批处理", §2.2), optionally as FP8
+// E4M3 values ("大语言模型推理引擎深度剖析", §4.3).
+//
+// Both kernels are HBM-trivial next to attention (a few MB per step); they are
+// written for full 16-byte vector traffic and a grid of whole waves.
+#include "pa_device.cuh"
+
+namespace pa {
+
+// ---------------------------------------------------------------------------
+// slot mapping: one thread per token
+// ---------------------------------------------------------------------------
+
+__global__ void __launch_bounds__(256) slot_mapping_kernel(const SlotParams p) {
+    const int64_t B = p.block_size;
+    for (int t = blockIdx.x * blockDim.x + threadIdx.x; t < p.num_tokens;
+         t += gridDim.x * blockDim.x) {
+        const int s = p.token_seq ? p.token_seq[t] : t;
+        int64_t slot = -1;
+        if (s >= 0) {
+            bool ok = s < p.num_seqs;
+            int64_t pos = -1;
+            if (ok) pos = p.token_pos ? (int64_t)p.token_pos[t] : (int64_t)p.seq_lens[s] - 1;
+            ok = ok && pos >= 0 && pos < (int64_t)p.max_blocks_per_seq * B;
+            if (ok) {
+                const int64_t phys = p.block_tables[(int64_t)s * p.max_blocks_per_seq + pos / B];
+                ok = phys >= 0 && phys < p.num_blocks;
+                if (ok) slot = phys * B + pos % B;
+            }
+            if (!ok) flag_error(p.err, kErrBounds);
+        }
+        p.slot_mapping[t] = slot;
+    }
+}
+
+cudaError_t launch_slot_mapping(const SlotParams &p, cudaStream_t stream) {
+    if (p.num_tokens <= 0) return cudaSuccess;
+    const int threads = 256;
+    int blocks = (p.num_tokens + threads - 1) / threads;
+    if (blocks > 65536) blocks = 65536;
+    slot_mapping_kernel<<<blocks, threads, 0, stream>>>(p);
+    return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// cache write: one thread per 8-element vector of one (token, head) row,
+// handling the K and the V vector at the same position
+// ---------------------------------------------------------------------------
+
+// fp32 pair -> packed E4M3 pair (low byte = first element); round to nearest
+// even, saturating finite overflow to +-448.
+__device__ __forceinline__ uint16_t e4m3x2_rn_sat(float first, float second) {
+    uint16_t r;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(second), "f"(first));
+    return r;
+}
+
+template <typename ACT>
+__device__ __forceinline__ uint2 quantise8(const uint4 &in, float scale) {
+    const uint32_t w[4] = {in.x, in.y, in.z, in.w};
+    float f[8];
+    Unpack<ACT, 8>::run(w, f);
+    uint16_t c[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+        c[i] = e4m3x2_rn_sat(__fdiv_rn(f[2 * i], scale), __fdiv_rn(f[2 * i + 1], scale));
+    return make_uint2((uint32_t)c[0] | ((uint32_t)c[1] << 16), (uint32_t)c[2] | ((uint32_t)c[3] << 16));
+}
+
+template <typename ACT, bool FP8>
+__global__ void __launch_bounds__(256) cache_write_kernel(const CacheWriteParams p) {
+    const int vecs_per_row = p.head_dim / 8;
+    const int64_t per_token = (int64_t)p.num_kv_heads * vecs_per_row;
+    const int64_t total = (int64_t)p.num_tokens * per_token;
+    const int64_t nslots = (int64_t)p.num_blocks * p.block_size;
+    for (int64_t g = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; g < total;
+         g += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t t = g / per_token;
+        const int64_t rem = g - t * per_token;
+        const int64_t h = rem / vecs_per_row;
+        const int64_t c = rem - h * vecs_per_row;
+        const int64_t slot = p.slot_mapping[t];
+        if (slot < 0) continue;
+        if (slot >= nslots) {
+            if (h == 0 && c == 0) flag_error(p.err, kErrBounds);
+            continue;
+        }
+        const int64_t blk = slot / p.block_size, off = slot - blk * p.block_size;
+        const int64_t src = ((t * p.num_kv_heads + h) * p.head_dim + c * 8);
+        const int64_t dst = (((blk * p.num_kv_heads + h) * p.block_size + off) * p.head_dim + c * 8);
+        const uint4 kin = *reinterpret_cast<const uint4 *>(static_cast<const uint16_t *>(p.k_new) + src);
+        const uint4 vin = *reinterpret_cast<const uint4 *>(static_cast<const uint16_t *>(p.v_new) + src);
+        if constexpr (FP8) {
+            *reinterpret_cast<uint2 *>(static_cast<uint8_t *>(p.k_cache) + dst) = quantise8<ACT>(kin, p.k_scale);
+            *reinterpret_cast<uint2 *>(static_cast<uint8_t *>(p.v_cache) + dst) = quantise8<ACT>(vin, p.v_scale);
+        } else {
+            *reinterpret_cast<uint4 *>(static_cast<uint16_t *>(p.k_cache) + dst) = kin;
+            *reinterpret_cast<uint4 *>(static_cast<uint16_t *>(p.v_cache) + dst) = vin;
+        }
+    }
+}
+
+cudaError_t launch_cache_write(const CacheWriteParams &p, DType act, DType kv, cudaStream_t stream) {
+    const int64_t total = (int64_t)p.num_tokens * p.num_kv_heads * (p.head_dim / 8);
+    if (total <= 0) return cudaSuccess;
+    const int threads = 256;
+    int64_t blocks = (total + threads - 1) / threads;
+    if (blocks > (1 << 20)) blocks = 1 << 20;
+    const bool fp8 = kv == DType::E4M3;
+    if (act == DType::F16) {
+        if (fp8)
+            cache_write_kernel<f16_t, true><<<(unsigned)blocks, threads, 0, stream>>>(p);
+        else
+            cache_write_kernel<f16_t, false><<<(unsigned)blocks, threads, 0, stream>>>(p);
+    } else {
+        if (fp8)
+            cache_write_kernel<bf16_t, true><<<(unsigned)blocks, threads, 0, stream>>>(p);
+        else
+            cache_write_kernel<bf16_t, false><<<(unsigned)blocks, threads, 0, stream>>>(p);
+    }
+    return cudaGetLastError();
+}
+
+}  // namespace pa

@@ -1,0 +1,260 @@
+// C ABI of libpa369.so (declared in include/pa.h): host-side argument checks,
+// launch configuration and dispatch to the kernel launchers.  No entry point
+// allocates memory, synchronises, or touches the GPU before its checks pass.
+#include <math.h>
+#include <stdint.h>
+
+#include "../../include/pa.h"
+#include "pa_internal.h"
+
+namespace {
+
+constexpr int kVersion = 10000;  // 1.0.0
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool is_act(pa_dtype t) { return t == PA_F16 || t == PA_BF16; }
+
+pa::DType to_internal(pa_dtype t) { return static_cast<pa::DType>(static_cast<int>(t)); }
+
+size_t align256(size_t n) { return (n + 255) & ~size_t(255); }
+
+// Template group size (1, 2, 4 or 8) used for a GQA group of g query heads;
+// groups larger than 8 run as ceil(g / 8) CTAs per KV head.
+int template_group(int g) {
+    if (g >= 8) return 8;
+    int t = 1;
+    while (t < g) t <<= 1;
+    return t;
+}
+
+pa_status from_cuda(cudaError_t e) { return e == cudaSuccess ? PA_OK : PA_ERR_CUDA; }
+
+struct DecodeArgs {
+    void *out;
+    const void *q;
+    const void *k_cache;
+    const void *v_cache;
+    const int32_t *block_tables;
+    int max_blocks_per_seq;
+    const int32_t *seq_lens;
+    int num_seqs;
+    int num_q_heads;
+    int num_kv_heads;
+    int head_dim;
+    int block_size;
+    int num_blocks;
+    float softmax_scale;
+    pa_dtype q_dtype;
+    pa_dtype kv_dtype;
+    float k_scale;
+    float v_scale;
+};
+
+pa_status check_decode(const DecodeArgs &a) {
+    if (a.num_seqs < 0 || a.num_q_heads <= 0 || a.num_kv_heads <= 0 || a.head_dim <= 0 ||
+        a.block_size <= 0)
+        return PA_ERR_INVALID_ARG;
+    if (a.num_q_heads % a.num_kv_heads != 0) return PA_ERR_INVALID_ARG;
+    if (!is_act(a.q_dtype)) return PA_ERR_UNSUPPORTED;
+    if (a.kv_dtype != a.q_dtype && a.kv_dtype != PA_FP8_E4M3) return PA_ERR_UNSUPPORTED;
+    if (a.head_dim != 64 && a.head_dim != 128) return PA_ERR_UNSUPPORTED;
+    if (a.block_size != pa::kBlockSize) return PA_ERR_UNSUPPORTED;
+    if (!isfinite(a.softmax_scale)) return PA_ERR_INVALID_ARG;
+    if (a.kv_dtype == PA_FP8_E4M3 &&
+        !(isfinite(a.k_scale) && a.k_scale > 0.f && isfinite(a.v_scale) && a.v_scale > 0.f))
+        return PA_ERR_INVALID_ARG;
+    if (a.num_seqs == 0) return PA_OK;
+    if (!a.out || !a.q || !a.k_cache || !a.v_cache || !a.block_tables || !a.seq_lens)
+        return PA_ERR_INVALID_ARG;
+    if (!aligned16(a.out) || !aligned16(a.q) || !aligned16(a.k_cache) || !aligned16(a.v_cache))
+        return PA_ERR_INVALID_ARG;
+    if (a.max_blocks_per_seq <= 0 || a.num_blocks <= 0) return PA_ERR_INVALID_ARG;
+    const int g = a.num_q_heads / a.num_kv_heads;
+    const int tg = template_group(g);
+    const int64_t ycta = (int64_t)a.num_kv_heads * ((g + tg - 1) / tg);
+    if (ycta > 65535) return PA_ERR_UNSUPPORTED;
+    return PA_OK;
+}
+
+pa::DecodeParams make_decode_params(const DecodeArgs &a, int *dev_err) {
+    pa::DecodeParams p = {};
+    const bool fp8 = a.kv_dtype == PA_FP8_E4M3;
+    const int g = a.num_q_heads / a.num_kv_heads;
+    const int tg = template_group(g);
+    p.out = a.out;
+    p.q = a.q;
+    p.k_cache = static_cast<const uint8_t *>(a.k_cache);
+    p.v_cache = static_cast<const uint8_t *>(a.v_cache);
+    p.block_tables = a.block_tables;
+    p.seq_lens = a.seq_lens;
+    p.err = dev_err;
+    p.max_blocks_per_seq = a.max_blocks_per_seq;
+    p.num_seqs = a.num_seqs;
+    p.num_q_heads = a.num_q_heads;
+    p.num_kv_heads = a.num_kv_heads;
+    p.num_blocks = a.num_blocks;
+    p.group = g;
+    p.head_groups = (g + tg - 1) / tg;
+    const double log2e = 1.4426950408889634074;
+    p.qk_scale_log2 = (float)((double)a.softmax_scale * (fp8 ? (double)a.k_scale : 1.0) * log2e);
+    p.v_scale = fp8 ? a.v_scale : 1.0f;
+    return p;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *pa_status_string(pa_status status) {
+    switch (status) {
+        case PA_OK: return "PA_OK";
+        case PA_ERR_INVALID_ARG: return "PA_ERR_INVALID_ARG: invalid argument";
+        case PA_ERR_UNSUPPORTED: return "PA_ERR_UNSUPPORTED: configuration not supported";
+        case PA_ERR_CUDA: return "PA_ERR_CUDA: a CUDA launch or query failed";
+        case PA_ERR_DEVICE_BOUNDS: return "PA_ERR_DEVICE_BOUNDS: index or length out of range on the device";
+        case PA_ERR_DEVICE_TIMEOUT: return "PA_ERR_DEVICE_TIMEOUT: a device wait timed out";
+    }
+    return "unknown pa_status";
+}
+
+int pa_version(void) { return kVersion; }
+
+pa_status pa_slot_mapping(int64_t *slot_mapping, const int32_t *block_tables,
+                          int max_blocks_per_seq, const int32_t *seq_lens,
+                          const int32_t *token_seq, const int32_t *token_pos, int num_tokens,
+                          int num_seqs, int block_size, int num_blocks, int *dev_err,
+                          void *stream) {
+    if (num_tokens < 0 || num_seqs < 0 || block_size <= 0 || num_blocks < 0)
+        return PA_ERR_INVALID_ARG;
+    if (num_tokens == 0) return PA_OK;
+    if (!slot_mapping || !block_tables || max_blocks_per_seq <= 0) return PA_ERR_INVALID_ARG;
+    if (!token_pos && !seq_lens) return PA_ERR_INVALID_ARG;
+    if (!token_seq && num_tokens > num_seqs) return PA_ERR_INVALID_ARG;  // token t is sequence t
+    pa::SlotParams p = {};
+    p.slot_mapping = slot_mapping;
+    p.block_tables = block_tables;
+    p.seq_lens = seq_lens;
+    p.token_seq = token_seq;
+    p.token_pos = token_pos;
+    p.err = dev_err;
+    p.max_blocks_per_seq = max_blocks_per_seq;
+    p.num_tokens = num_tokens;
+    p.num_seqs = num_seqs;
+    p.block_size = block_size;
+    p.num_blocks = num_blocks;
+    return from_cuda(pa::launch_slot_mapping(p, static_cast<cudaStream_t>(stream)));
+}
+
+pa_status pa_cache_write(const void *k_new, const void *v_new, void *k_cache, void *v_cache,
+                         const int64_t *slot_mapping, int num_tokens, int num_blocks,
+                         int num_kv_heads, int head_dim, int block_size, pa_dtype act_dtype,
+                         pa_dtype kv_dtype, float k_scale, float v_scale, int *dev_err,
+                         void *stream) {
+    if (num_tokens < 0 || num_blocks < 0 || num_kv_heads <= 0 || head_dim <= 0 || block_size <= 0)
+        return PA_ERR_INVALID_ARG;
+    if (!is_act(act_dtype)) return PA_ERR_UNSUPPORTED;
+    if (kv_dtype != act_dtype && kv_dtype != PA_FP8_E4M3) return PA_ERR_UNSUPPORTED;
+    if (head_dim % 8 != 0) return PA_ERR_UNSUPPORTED;
+    if (kv_dtype == PA_FP8_E4M3 &&
+        !(isfinite(k_scale) && k_scale > 0.f && isfinite(v_scale) && v_scale > 0.f))
+        return PA_ERR_INVALID_ARG;
+    if (num_tokens == 0) return PA_OK;
+    if (!k_new || !v_new || !k_cache || !v_cache || !slot_mapping) return PA_ERR_INVALID_ARG;
+    if (!aligned16(k_new) || !aligned16(v_new) || !aligned16(k_cache) || !aligned16(v_cache))
+        return PA_ERR_INVALID_ARG;
+    pa::CacheWriteParams p = {};
+    p.k_new = k_new;
+    p.v_new = v_new;
+    p.k_cache = k_cache;
+    p.v_cache = v_cache;
+    p.slot_mapping = slot_mapping;
+    p.err = dev_err;
+    p.num_tokens = num_tokens;
+    p.num_blocks = num_blocks;
+    p.num_kv_heads = num_kv_heads;
+    p.head_dim = head_dim;
+    p.block_size = block_size;
+    p.k_scale = k_scale;
+    p.v_scale = v_scale;
+    return from_cuda(pa::launch_cache_write(p, to_internal(act_dtype), to_internal(kv_dtype),
+                                            static_cast<cudaStream_t>(stream)));
+}
+
+pa_status pa_decode(void *out, const void *q, const void *k_cache, const void *v_cache,
+                    const int32_t *block_tables, int max_blocks_per_seq, const int32_t *seq_lens,
+                    int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
+                    int block_size, int num_blocks, float softmax_scale, pa_dtype q_dtype,
+                    pa_dtype kv_dtype, float k_scale, float v_scale, int *dev_err,
+                    void *stream) {
+    const DecodeArgs a = {out, q, k_cache, v_cache, block_tables, max_blocks_per_seq, seq_lens,
+                          num_seqs, num_q_heads, num_kv_heads, head_dim, block_size, num_blocks,
+                          softmax_scale, q_dtype, kv_dtype, k_scale, v_scale};
+    const pa_status st = check_decode(a);
+    if (st != PA_OK || num_seqs == 0) return st;
+    pa::DecodeParams p = make_decode_params(a, dev_err);
+    p.partition_blocks = max_blocks_per_seq;
+    p.num_partitions = 1;
+    p.split = 0;
+    return from_cuda(pa::launch_decode(p, to_internal(q_dtype), to_internal(kv_dtype), head_dim,
+                                       template_group(p.group), static_cast<cudaStream_t>(stream)));
+}
+
+size_t pa_split_workspace_bytes(int num_seqs, int num_q_heads, int head_dim, int max_seq_len,
+                                int partition_size) {
+    if (num_seqs < 0 || num_q_heads <= 0 || head_dim <= 0 || max_seq_len < 0 ||
+        partition_size <= 0)
+        return 0;
+    const size_t np = max_seq_len > 0 ? (size_t)((max_seq_len + partition_size - 1) / partition_size) : 1;
+    const size_t rows = (size_t)num_seqs * (size_t)num_q_heads * np;
+    return align256(rows * sizeof(float)) + align256(rows * (size_t)head_dim * sizeof(float));
+}
+
+pa_status pa_decode_split_reduce(void *out, const void *q, const void *k_cache,
+                                 const void *v_cache, const int32_t *block_tables,
+                                 int max_blocks_per_seq, const int32_t *seq_lens, int num_seqs,
+                                 int num_q_heads, int num_kv_heads, int head_dim,
+                                 int block_size, int num_blocks, float softmax_scale,
+                                 pa_dtype q_dtype, pa_dtype kv_dtype, float k_scale,
+                                 float v_scale, int partition_size, int max_seq_len,
+                                 void *workspace, size_t workspace_bytes, int *dev_err,
+                                 void *stream) {
+    const DecodeArgs a = {out, q, k_cache, v_cache, block_tables, max_blocks_per_seq, seq_lens,
+                          num_seqs, num_q_heads, num_kv_heads, head_dim, block_size, num_blocks,
+                          softmax_scale, q_dtype, kv_dtype, k_scale, v_scale};
+    pa_status st = check_decode(a);
+    if (st != PA_OK) return st;
+    if (partition_size <= 0 || partition_size % pa::kBlockSize != 0 || max_seq_len < 0)
+        return PA_ERR_INVALID_ARG;
+    if (num_seqs == 0) return PA_OK;
+    const size_t need = pa_split_workspace_bytes(num_seqs, num_q_heads, head_dim, max_seq_len,
+                                                 partition_size);
+    if (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+        return PA_ERR_INVALID_ARG;
+    const int np = max_seq_len > 0 ? (max_seq_len + partition_size - 1) / partition_size : 1;
+    if ((int64_t)num_seqs * np > 0x7FFFFFFF) return PA_ERR_UNSUPPORTED;
+
+    pa::DecodeParams p = make_decode_params(a, dev_err);
+    const size_t rows = (size_t)num_seqs * num_q_heads * np;
+    p.ws_lse = static_cast<float *>(workspace);
+    p.ws_o = reinterpret_cast<float *>(static_cast<uint8_t *>(workspace) + align256(rows * sizeof(float)));
+    p.partition_blocks = partition_size / pa::kBlockSize;
+    p.num_partitions = np;
+    p.split = 1;
+    const cudaStream_t s = static_cast<cudaStream_t>(stream);
+    cudaError_t e = pa::launch_decode(p, to_internal(q_dtype), to_internal(kv_dtype), head_dim,
+                                      template_group(p.group), s);
+    if (e != cudaSuccess) return PA_ERR_CUDA;
+    pa::ReduceParams r = {};
+    r.out = out;
+    r.ws_lse = p.ws_lse;
+    r.ws_o = p.ws_o;
+    r.seq_lens = seq_lens;
+    r.num_seqs = num_seqs;
+    r.num_q_heads = num_q_heads;
+    r.num_partitions = np;
+    r.partition_size = partition_size;
+    return from_cuda(pa::launch_reduce(r, to_internal(q_dtype), head_dim, s));
+}
+
+}  // extern "C"

@@ -1,0 +1,224 @@
+// Device helpers for the sm_100a paged-KV kernels: element conversions,
+// mbarrier + bulk-copy (TMA, non-tensor, no multicast) primitives, bounded
+// waits and device-side error reporting.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <stdint.h>
+
+#include "pa_internal.h"
+
+namespace pa {
+
+// ---------------------------------------------------------------------------
+// element types
+// ---------------------------------------------------------------------------
+
+struct f16_t {
+    uint16_t bits;
+};
+struct bf16_t {
+    uint16_t bits;
+};
+struct e4m3_t {
+    uint8_t bits;
+};
+
+template <typename T> struct Elem;
+template <> struct Elem<f16_t> {
+    static constexpr int kBytes = 2;
+};
+template <> struct Elem<bf16_t> {
+    static constexpr int kBytes = 2;
+};
+template <> struct Elem<e4m3_t> {
+    static constexpr int kBytes = 1;
+};
+
+// Two packed 16-bit values -> two floats (exact).
+__device__ __forceinline__ void unpack2(f16_t, uint32_t w, float &lo, float &hi) {
+    __half2 h = *reinterpret_cast<__half2 *>(&w);
+    float2 f = __half22float2(h);
+    lo = f.x;
+    hi = f.y;
+}
+__device__ __forceinline__ void unpack2(bf16_t, uint32_t w, float &lo, float &hi) {
+    lo = __uint_as_float(w << 16);
+    hi = __uint_as_float(w & 0xFFFF0000u);
+}
+
+// Two packed E4M3 codes (low byte first) -> two floats (exact: every E4M3
+// value is an f16 value).
+__device__ __forceinline__ void unpack2_e4m3(uint16_t w, float &lo, float &hi) {
+    uint32_t h2;
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(w));
+    __half2 h = *reinterpret_cast<__half2 *>(&h2);
+    float2 f = __half22float2(h);
+    lo = f.x;
+    hi = f.y;
+}
+
+// N consecutive elements held in registers (raw words) -> N floats.
+template <typename T, int N> struct Unpack;
+template <int N> struct Unpack<f16_t, N> {
+    static __device__ __forceinline__ void run(const uint32_t *w, float *f) {
+#pragma unroll
+        for (int i = 0; i < N / 2; ++i) unpack2(f16_t{}, w[i], f[2 * i], f[2 * i + 1]);
+    }
+};
+template <int N> struct Unpack<bf16_t, N> {
+    static __device__ __forceinline__ void run(const uint32_t *w, float *f) {
+#pragma unroll
+        for (int i = 0; i < N / 2; ++i) unpack2(bf16_t{}, w[i], f[2 * i], f[2 * i + 1]);
+    }
+};
+template <int N> struct Unpack<e4m3_t, N> {
+    static __device__ __forceinline__ void run(const uint32_t *w, float *f) {
+#pragma unroll
+        for (int i = 0; i < N / 4; ++i) {
+            unpack2_e4m3((uint16_t)(w[i] & 0xFFFFu), f[4 * i], f[4 * i + 1]);
+            unpack2_e4m3((uint16_t)(w[i] >> 16), f[4 * i + 2], f[4 * i + 3]);
+        }
+        if constexpr (N % 4 == 2) unpack2_e4m3((uint16_t)(w[N / 4] & 0xFFFFu), f[N - 2], f[N - 1]);
+    }
+};
+
+__device__ __forceinline__ float to_float(f16_t, uint16_t b) {
+    return __half2float(__ushort_as_half(b));
+}
+__device__ __forceinline__ float to_float(bf16_t, uint16_t b) {
+    return __uint_as_float((uint32_t)b << 16);
+}
+__device__ __forceinline__ uint16_t from_float(f16_t, float x) {
+    return __half_as_ushort(__float2half_rn(x));
+}
+__device__ __forceinline__ uint16_t from_float(bf16_t, float x) {
+    return __bfloat16_as_ushort(__float2bfloat16_rn(x));
+}
+
+// ---------------------------------------------------------------------------
+// shared-memory loads of 2 / 4 / 8 / 16 bytes into 32-bit words
+// ---------------------------------------------------------------------------
+
+template <int BYTES> __device__ __forceinline__ void lds(uint32_t *w, uint32_t addr) {
+    if constexpr (BYTES == 16) {
+        asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                     : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3])
+                     : "r"(addr));
+    } else if constexpr (BYTES == 8) {
+        asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(w[0]), "=r"(w[1]) : "r"(addr));
+    } else if constexpr (BYTES == 4) {
+        asm volatile("ld.shared.u32 %0, [%1];" : "=r"(w[0]) : "r"(addr));
+    } else {
+        static_assert(BYTES == 2, "unsupported load width");
+        uint16_t h;
+        asm volatile("ld.shared.u16 %0, [%1];" : "=h"(h) : "r"(addr));
+        w[0] = h;
+    }
+}
+
+__device__ __forceinline__ uint32_t smem_addr(const void *p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+// ---------------------------------------------------------------------------
+// mbarrier + bulk async copy
+// ---------------------------------------------------------------------------
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void mbar_init_fence() {
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred P1;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 P1, [%1], %2;\n\t"
+        "selp.b32 %0, 1, 0, P1;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+__device__ __forceinline__ uint64_t global_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+// Wait for phase `parity` of an mbarrier, giving up after `limit_ns`
+// nanoseconds of wall time.  Returns false on timeout.
+__device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity,
+                                                  uint64_t limit_ns) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = global_ns();
+    for (;;) {
+#pragma unroll 1
+        for (int i = 0; i < 64; ++i)
+            if (mbar_try_wait(bar, parity)) return true;
+        if (global_ns() - t0 > limit_ns) return false;
+    }
+}
+
+// One bulk (non-tensor) global -> shared copy completing on `bar`.
+// dst / src 16-byte aligned, bytes a multiple of 16.
+__device__ __forceinline__ void bulk_g2s(uint32_t dst, const void *src, uint32_t bytes,
+                                         uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+            dst),
+        "l"(src), "r"(bytes), "r"(bar)
+        : "memory");
+}
+
+// Same, with an L2 eviction-priority policy (createpolicy) attached.
+__device__ __forceinline__ void bulk_g2s_hint(uint32_t dst, const void *src, uint32_t bytes,
+                                              uint32_t bar, uint64_t policy) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], %2, [%3], %4;" ::"r"(
+            dst),
+        "l"(src), "r"(bytes), "r"(bar), "l"(policy)
+        : "memory");
+}
+
+__device__ __forceinline__ uint64_t policy_evict_first() {
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+
+__device__ __forceinline__ uint64_t policy_evict_last() {
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+
+// ---------------------------------------------------------------------------
+// programmatic dependent launch
+// ---------------------------------------------------------------------------
+
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// ---------------------------------------------------------------------------
+// device-side errors: the first one wins
+// ---------------------------------------------------------------------------
+
+__device__ __forceinline__ void flag_error(int *err, int code) {
+    if (err) atomicCAS(err, 0, code);
+}
+
+}  // namespace pa

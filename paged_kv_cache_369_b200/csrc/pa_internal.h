@@ -1,0 +1,91 @@
+// Internal interface between the C-ABI shim (pa_capi.cu) and the kernel
+// translation units.  Not installed; the public ABI is include/pa.h.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace pa {
+
+constexpr int kBlockSize = 16;        // tokens per KV block
+constexpr int kDecodeWarps = 4;       // consumer warps per decode CTA
+constexpr uint64_t kWaitLimitNs = 1000000000ull;  // 1 s bound on any device wait
+constexpr int kErrBounds = 4;         // = PA_ERR_DEVICE_BOUNDS
+constexpr int kErrTimeout = 5;        // = PA_ERR_DEVICE_TIMEOUT
+
+enum class DType : int { F16 = 0, BF16 = 1, E4M3 = 2 };
+
+struct SlotParams {
+    int64_t *slot_mapping;
+    const int32_t *block_tables;
+    const int32_t *seq_lens;
+    const int32_t *token_seq;
+    const int32_t *token_pos;
+    int *err;
+    int max_blocks_per_seq;
+    int num_tokens;
+    int num_seqs;
+    int block_size;
+    int num_blocks;
+};
+
+struct CacheWriteParams {
+    const void *k_new;
+    const void *v_new;
+    void *k_cache;
+    void *v_cache;
+    const int64_t *slot_mapping;
+    int *err;
+    int num_tokens;
+    int num_blocks;
+    int num_kv_heads;
+    int head_dim;
+    int block_size;
+    float k_scale;
+    float v_scale;
+};
+
+struct DecodeParams {
+    void *out;                  // [S, Hq, D] q dtype (single pass)
+    const void *q;              // [S, Hq, D]
+    const uint8_t *k_cache;     // [NB, Hk, 16, D] kv dtype, as bytes
+    const uint8_t *v_cache;
+    const int32_t *block_tables;
+    const int32_t *seq_lens;
+    float *ws_lse;              // split: [S, Hq, NP]
+    float *ws_o;                // split: [S, Hq, NP, D]
+    int *err;
+    int max_blocks_per_seq;
+    int num_seqs;
+    int num_q_heads;
+    int num_kv_heads;
+    int num_blocks;
+    int group;                  // Hq / Hk
+    int head_groups;            // CTAs per KV head (ceil(group / G))
+    int partition_blocks;       // KV blocks per partition
+    int num_partitions;         // NP (1 in single-pass mode)
+    int split;                  // 1: write partials to the workspace
+    float qk_scale_log2;        // softmax_scale * k_scale * log2(e)
+    float v_scale;              // applied to the output (1 for 16-bit caches)
+};
+
+struct ReduceParams {
+    void *out;
+    const float *ws_lse;
+    const float *ws_o;
+    const int32_t *seq_lens;
+    int num_seqs;
+    int num_q_heads;
+    int num_partitions;
+    int partition_size;
+};
+
+// Launchers: return cudaSuccess or the launch error.
+cudaError_t launch_slot_mapping(const SlotParams &p, cudaStream_t stream);
+cudaError_t launch_cache_write(const CacheWriteParams &p, DType act, DType kv, cudaStream_t stream);
+cudaError_t launch_decode(const DecodeParams &p, DType q, DType kv, int head_dim, int tpl_group,
+                          cudaStream_t stream);
+cudaError_t launch_reduce(const ReduceParams &p, DType q, int head_dim, cudaStream_t stream);
+
+}  // namespace pa

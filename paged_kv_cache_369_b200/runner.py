@@ -1,0 +1,135 @@
+"""Device-resident decode state and the step that runs the hot path.
+
+``PagedDecode`` uploads one workload (any object with the attributes of
+``workload.Workload``): q, this step's new K/V rows, block tables and
+lengths, and K/V pools filled with 0xFF (NaN in every cache format) into which
+the earlier tokens are written by the library's own slot-mapping and
+cache-write kernels.  ``step()`` is one pass of the hot path, all through the
+C ABI: slot mapping of the new tokens, cache write, decode (single pass or
+split-KV partition + reduce).
+
+PyTorch only provides device memory and streams here.
+"""
+
+from __future__ import annotations
+
+import math
+from typing import Optional
+
+import numpy as np
+import torch
+
+from . import (pa_cache_write, pa_decode, pa_decode_split_reduce, pa_slot_mapping,
+               pa_split_workspace_bytes)
+
+_TORCH_ACT = {"f16": torch.float16, "bf16": torch.bfloat16}
+_UPLOAD_CHUNK_TOKENS = 1 << 16
+
+
+def _bits_to_device(bits: np.ndarray, act: str, device) -> torch.Tensor:
+    t = torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(_TORCH_ACT[act])
+    return t.to(device, non_blocking=False)
+
+
+class PagedDecode:
+    """One decode workload resident on a GPU."""
+
+    def __init__(self, w, device: str = "cuda", mode: str = "split", partition_size: int = 512,
+                 prefill: bool = True, stream: Optional[torch.cuda.Stream] = None):
+        if mode not in ("split", "single"):
+            raise ValueError(mode)
+        self.w = w
+        self.device = torch.device(device)
+        self.mode = mode
+        self.partition_size = partition_size
+        self.stream = stream
+        S, Hq, Hk, d = w.num_seqs, w.num_q_heads, w.num_kv_heads, w.head_dim
+        dev = self.device
+        act = _TORCH_ACT[w.act_dtype]
+        self.q = _bits_to_device(w.q, w.act_dtype, dev)
+        self.k_new = _bits_to_device(w.k_new, w.act_dtype, dev)
+        self.v_new = _bits_to_device(w.v_new, w.act_dtype, dev)
+        self.block_tables = torch.from_numpy(np.ascontiguousarray(w.block_tables)).to(dev)
+        self.seq_lens = torch.from_numpy(np.ascontiguousarray(w.seq_lens)).to(dev)
+        pool_dtype = torch.uint8 if w.kv_dtype == "e4m3" else act
+        shape = (w.num_blocks, Hk, w.block_size, d)
+        self.k_cache = torch.empty(shape, dtype=pool_dtype, device=dev)
+        self.v_cache = torch.empty(shape, dtype=pool_dtype, device=dev)
+        self.k_cache.view(torch.uint8).fill_(0xFF)
+        self.v_cache.view(torch.uint8).fill_(0xFF)
+        self.slot_mapping = torch.empty(S, dtype=torch.int64, device=dev)
+        # the new token of sequence s (padding -1 for an empty sequence)
+        self.new_seq = torch.from_numpy(np.ascontiguousarray(w.new_seq)).to(dev)
+        self.out = torch.empty((S, Hq, d), dtype=act, device=dev)
+        self.dev_err = torch.zeros(1, dtype=torch.int32, device=dev)
+        self.max_seq_len = int(w.seq_lens.max()) if S else 0
+        nbytes = pa_split_workspace_bytes(S, Hq, d, self.max_seq_len, partition_size)
+        self.workspace = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=dev)
+        if prefill:
+            self.prefill()
+
+    # -- cache contents that precede the step --------------------------------
+    def prefill(self) -> None:
+        """Write every earlier token's K/V rows through pa_slot_mapping +
+        pa_cache_write, in chunks of tokens."""
+        w = self.w
+        Tp = int(w.prefill_seq.size)
+        dev = self.device
+        for lo in range(0, Tp, _UPLOAD_CHUNK_TOKENS):
+            hi = min(Tp, lo + _UPLOAD_CHUNK_TOKENS)
+            tseq = torch.from_numpy(w.prefill_seq[lo:hi]).to(dev)
+            tpos = torch.from_numpy(w.prefill_pos[lo:hi]).to(dev)
+            kn = _bits_to_device(w.k_prefill[lo:hi], w.act_dtype, dev)
+            vn = _bits_to_device(w.v_prefill[lo:hi], w.act_dtype, dev)
+            slots = torch.empty(hi - lo, dtype=torch.int64, device=dev)
+            pa_slot_mapping(slots, self.block_tables, self.seq_lens, tseq, tpos, hi - lo,
+                            w.num_seqs, w.num_blocks, w.block_size, self.dev_err, self.stream)
+            pa_cache_write(kn, vn, self.k_cache, self.v_cache, slots, w.k_scale, w.v_scale,
+                           self.dev_err, self.stream)
+        torch.cuda.synchronize(dev)
+
+    # -- the hot path ----------------------------------------------------------
+    def write_new(self) -> None:
+        w = self.w
+        pa_slot_mapping(self.slot_mapping, self.block_tables, self.seq_lens, self.new_seq, None,
+                        w.num_seqs, w.num_seqs, w.num_blocks, w.block_size, self.dev_err,
+                        self.stream)
+        pa_cache_write(self.k_new, self.v_new, self.k_cache, self.v_cache, self.slot_mapping,
+                       w.k_scale, w.v_scale, self.dev_err, self.stream)
+
+    def attend(self) -> None:
+        w = self.w
+        if self.mode == "single":
+            pa_decode(self.out, self.q, self.k_cache, self.v_cache, self.block_tables,
+                      self.seq_lens, w.softmax_scale, w.k_scale, w.v_scale, self.dev_err,
+                      self.stream)
+        else:
+            pa_decode_split_reduce(self.out, self.q, self.k_cache, self.v_cache,
+                                   self.block_tables, self.seq_lens, w.softmax_scale,
+                                   self.partition_size, self.max_seq_len, self.workspace,
+                                   w.k_scale, w.v_scale, self.dev_err, self.stream)
+
+    def step(self) -> None:
+        """One decode step: slot mapping, cache write, attention."""
+        self.write_new()
+        self.attend()
+
+    def launches_per_step(self) -> int:
+        return 2 + (1 if self.mode == "single" else 2)
+
+    def error(self) -> int:
+        return int(self.dev_err.item())
+
+
+def default_partition_size(w) -> int:
+    """512-token partitions (32 blocks): enough CTAs to fill 148 SMs several
+    times over for the decode workloads, few enough partials to merge."""
+    return 512
+
+
+def algorithmic_decode_bytes(w) -> int:
+    """Bytes the attention launch must move: every K/V row read once, q read,
+    the output written, block tables and lengths read."""
+    S, Hq, d = w.num_seqs, w.num_q_heads, w.head_dim
+    return w.kv_bytes_logical() + 2 * S * Hq * d * 2 + int(sum(
+        math.ceil(int(L) / w.block_size) for L in w.seq_lens)) * 4 + S * 4

@@ -1,0 +1,142 @@
+"""The C ABI without a GPU: the library loads, exports every symbol that
+include/pa.h declares, and its host-side checks reject bad arguments with the
+documented status before any CUDA call."""
+
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+from tests.conftest import ROOT
+
+HEADER = os.path.join(ROOT, "include", "pa.h")
+
+
+@pytest.fixture(scope="module")
+def pa():
+    from paged_kv_cache_369_b200 import build as b
+
+    b.build()
+    import paged_kv_cache_369_b200 as m
+
+    return m
+
+
+def header_symbols():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(pa_[a-z_0-9]+)\s*\(", text)))
+
+
+def test_header_declares_the_boundary():
+    syms = header_symbols()
+    for s in ("pa_slot_mapping", "pa_cache_write", "pa_decode", "pa_decode_split_reduce",
+              "pa_split_workspace_bytes", "pa_status_string"):
+        assert s in syms
+
+
+def test_library_exports_every_header_symbol(pa):
+    out = subprocess.run(["nm", "-D", "--defined-only", pa.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = set(re.findall(r"\bT (pa_[a-z_0-9]+)\b", out))
+    missing = [s for s in header_symbols() if s not in exported]
+    assert not missing, f"declared but not exported: {missing}"
+    lib = ctypes.CDLL(pa.LIB_PATH)
+    for s in header_symbols():
+        assert hasattr(lib, s)
+    assert sorted(pa.SYMBOLS) == sorted(header_symbols())
+
+
+def test_status_strings(pa):
+    for code in range(6):
+        assert pa.pa_status_string(code).startswith("PA_")
+    assert pa.pa_status_string(99) == "unknown pa_status"
+    assert pa.pa_version() == 10000
+
+
+A = 1 << 20  # a 16-byte aligned non-null stand-in pointer; never dereferenced
+
+
+def _decode(pa, **kw):
+    args = dict(out=A, q=A, k=A, v=A, bt=A, mbs=4, sl=A, S=2, Hq=8, Hk=2, d=128, B=16, NB=10,
+                scale=0.1, qd=pa.PA_BF16, kvd=pa.PA_BF16, ks=1.0, vs=1.0)
+    args.update(kw)
+    return pa.lib().pa_decode(args["out"], args["q"], args["k"], args["v"], args["bt"],
+                              args["mbs"], args["sl"], args["S"], args["Hq"], args["Hk"],
+                              args["d"], args["B"], args["NB"], args["scale"], args["qd"],
+                              args["kvd"], args["ks"], args["vs"], None, None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(d=96), 2),                                  # head_dim
+    (dict(d=256), 2),
+    (dict(B=32), 2),                                  # block size
+    (dict(Hq=8, Hk=3), 1),                            # Hq % Hk
+    (dict(Hk=0), 1),
+    (dict(qd=2), 2),                                  # fp8 query
+    (dict(qd=0, kvd=1), 2),                           # f16 q with bf16 cache
+    (dict(q=0), 1),                                   # null pointers
+    (dict(out=0), 1),
+    (dict(bt=0), 1),
+    (dict(sl=0), 1),
+    (dict(k=A + 8), 1),                               # misaligned
+    (dict(out=A + 2), 1),
+    (dict(NB=0), 1),
+    (dict(mbs=0), 1),
+    (dict(scale=float("inf")), 1),
+    (dict(kvd=2, ks=0.0), 1),                         # fp8 needs positive scales
+    (dict(kvd=2, vs=float("nan")), 1),
+    (dict(S=-1), 1),
+])
+def test_decode_rejects(pa, kw, status):
+    assert _decode(pa, **kw) == status
+
+
+def test_decode_empty_batch_is_a_noop(pa):
+    assert _decode(pa, S=0, q=0, out=0) == 0
+
+
+def test_split_checks(pa):
+    L = pa.lib()
+    need = pa.pa_split_workspace_bytes(2, 8, 128, 1000, 512)
+    assert need == 256 + (2 * 8 * 2 * 128 * 4 + 255) // 256 * 256
+    assert pa.pa_split_workspace_bytes(2, 8, 128, 1000, 0) == 0
+
+    def call(P=512, maxlen=1000, ws=A, wsb=need):
+        return L.pa_decode_split_reduce(A, A, A, A, A, 4, A, 2, 8, 2, 128, 16, 10, 0.1,
+                                        pa.PA_BF16, pa.PA_BF16, 1.0, 1.0, P, maxlen, ws, wsb,
+                                        None, None)
+
+    assert call(P=24) == 1            # not a multiple of the block size
+    assert call(P=0) == 1
+    assert call(maxlen=-1) == 1
+    assert call(wsb=need - 1) == 1    # workspace too small
+    assert call(ws=0) == 1
+    assert call(ws=A + 128) == 1      # workspace must be 256-byte aligned
+
+
+def test_cache_write_and_slot_checks(pa):
+    L = pa.lib()
+    cw = lambda **k: L.pa_cache_write(k.get("kn", A), A, k.get("kc", A), A, k.get("sm", A),
+                                      k.get("T", 4), 10, 2, k.get("d", 128), 16,
+                                      k.get("act", pa.PA_BF16), k.get("kv", pa.PA_BF16),
+                                      k.get("ks", 1.0), 1.0, None, None)
+    assert cw(act=pa.PA_FP8_E4M3) == 2
+    assert cw(act=pa.PA_F16, kv=pa.PA_BF16) == 2
+    assert cw(d=12) == 2
+    assert cw(kv=pa.PA_FP8_E4M3, ks=-1.0) == 1
+    assert cw(kn=0) == 1
+    assert cw(kc=A + 4) == 1
+    assert cw(T=-1) == 1
+    assert cw(T=0, kn=0) == 0
+    sm = lambda **k: L.pa_slot_mapping(k.get("out", A), k.get("bt", A), k.get("mbs", 4),
+                                       k.get("sl", A), k.get("ts", None), k.get("tp", None),
+                                       k.get("T", 2), k.get("S", 2), 16, 10, None, None)
+    assert sm(out=0) == 1
+    assert sm(bt=0) == 1
+    assert sm(mbs=0) == 1
+    assert sm(sl=None) == 1           # decode form needs seq_lens
+    assert sm(T=3, S=2) == 1          # token t is sequence t: T <= S
+    assert sm(T=0, out=0) == 0

@@ -93,8 +93,10 @@ class Workload:
 
     @property
     def new_seq(self) -> np.ndarray:
-        """Sequence index of each new token (one per sequence)."""
-        return np.arange(self.num_seqs, dtype=np.int32)
+        """Sequence index of each new token (one per sequence); -1 (padding)
+        for an empty sequence, which has no token to write."""
+        idx = np.arange(self.num_seqs, dtype=np.int32)
+        return np.where(self.seq_lens > 0, idx, -1).astype(np.int32)
 
     @property
     def new_pos(self) -> np.ndarray:
@@ -214,6 +216,8 @@ def build(
     S = int(seq_lens.size)
     if shared_prefix_tokens % block_size:
         raise ValueError("shared prefix must be block aligned")
+    if seq_lens.size and int(seq_lens.min()) < 0:
+        raise ValueError("negative sequence length")
     if shared_prefix_tokens and S and int(seq_lens.min()) <= shared_prefix_tokens:
         raise ValueError("every sequence must extend past the shared prefix")
     nprefix = shared_prefix_tokens // block_size
