@@ -3,6 +3,8 @@
 // allocates memory, synchronises, or touches the GPU before its checks pass.
 #include <math.h>
 #include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
 
 #include "../../include/pa.h"
 #include "pa_internal.h"
@@ -29,6 +31,30 @@ int template_group(int g) {
 }
 
 pa_status from_cuda(cudaError_t e) { return e == cudaSuccess ? PA_OK : PA_ERR_CUDA; }
+
+// Decode kernel choice: the tensor-core kernel wherever it supports the shape;
+// the CUDA-core kernel otherwise, or everywhere when the environment variable
+// PA369_DECODE_KERNEL is "simt" (kept for A/B measurement and tests).
+bool use_mma(pa_dtype kv, int head_dim, int num_blocks, int num_kv_heads) {
+    const char *env = getenv("PA369_DECODE_KERNEL");
+    if (env && strcmp(env, "simt") == 0) return false;
+    return pa::mma_decode_supported(static_cast<pa::DType>(static_cast<int>(kv)), head_dim,
+                                    num_blocks, num_kv_heads);
+}
+
+// Launch whichever decode kernel applies, with its own head grouping.
+cudaError_t launch_any_decode(pa::DecodeParams &p, pa_dtype q, pa_dtype kv, int head_dim,
+                              cudaStream_t stream) {
+    const int g = p.group;
+    if (use_mma(kv, head_dim, p.num_blocks, p.num_kv_heads)) {
+        const int rows = g <= 8 ? 8 : 16;
+        p.head_groups = (g + rows - 1) / rows;
+        return pa::launch_decode_mma(p, to_internal(q), to_internal(kv), head_dim, rows, stream);
+    }
+    const int tg = template_group(g);
+    p.head_groups = (g + tg - 1) / tg;
+    return pa::launch_decode(p, to_internal(q), to_internal(kv), head_dim, tg, stream);
+}
 
 struct DecodeArgs {
     void *out;
@@ -196,8 +222,7 @@ pa_status pa_decode(void *out, const void *q, const void *k_cache, const void *v
     p.partition_blocks = max_blocks_per_seq;
     p.num_partitions = 1;
     p.split = 0;
-    return from_cuda(pa::launch_decode(p, to_internal(q_dtype), to_internal(kv_dtype), head_dim,
-                                       template_group(p.group), static_cast<cudaStream_t>(stream)));
+    return from_cuda(launch_any_decode(p, q_dtype, kv_dtype, head_dim, static_cast<cudaStream_t>(stream)));
 }
 
 size_t pa_split_workspace_bytes(int num_seqs, int num_q_heads, int head_dim, int max_seq_len,
@@ -242,8 +267,7 @@ pa_status pa_decode_split_reduce(void *out, const void *q, const void *k_cache,
     p.num_partitions = np;
     p.split = 1;
     const cudaStream_t s = static_cast<cudaStream_t>(stream);
-    cudaError_t e = pa::launch_decode(p, to_internal(q_dtype), to_internal(kv_dtype), head_dim,
-                                      template_group(p.group), s);
+    cudaError_t e = launch_any_decode(p, q_dtype, kv_dtype, head_dim, s);
     if (e != cudaSuccess) return PA_ERR_CUDA;
     pa::ReduceParams r = {};
     r.out = out;

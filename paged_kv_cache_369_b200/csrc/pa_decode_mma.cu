@@ -1,0 +1,649 @@
+// Paged decode attention on tensor cores (mma.sync m16n8k16, fp32 accumulate)
+// with TMA tensor copies of the K/V tiles into 128-byte-swizzled shared memory.
+//
+// Same operation as pa_decode.cu ("KV Cache 与 PageAttention深度实战", §1.2,
+// §3.2-§3.3): per sequence and query head, softmax(q K^T / sqrt(d)) V over the
+// 16-token blocks the block table lists.  What changes is where the
+// arithmetic runs: the q.K and P.V contractions of a (sequence, KV head)
+// group are dense tiles -- [G query heads x 16 tokens x d] -- so they go to the
+// tensor cores, leaving the CUDA cores only the softmax.  The per-block cost
+// drops from ~1000 warp instructions (CUDA-core dot products, GQA 4) to ~170,
+// which keeps the kernel on the HBM roofline up to GQA 16 and for FP8 caches.
+//
+// Layout of the work:
+//   - one CTA per (sequence, partition, KV head, head group of <= 16); 4 warps,
+//     each owning every 4th block of the partition with a private ring of
+//     shared-memory stages filled by TMA (cp.async.bulk.tensor.2d, no multicast);
+//   - a tile row is 128 bytes per TMA box (d = 64 16-bit, or half of d = 128
+//     16-bit, or d = 128 E4M3) and the box lands 128B-swizzled, so ldmatrix of
+//     8 token rows at one 16-byte column touches 8 distinct bank groups;
+//   - q.K: S[16 x 16] = Q[16 x d] K^T, M = query heads (zero rows beyond the
+//     group), N = the block's tokens, ldmatrix.x4 feeding B;
+//   - online softmax on the accumulator fragments (row = head); masked tokens
+//     are set to -inf by select;
+//   - P.V: O[16 x d] += P[16 x 16] V, P taken straight from the S fragments;
+//     ldmatrix.x4.trans feeds V.  For a bf16 cache P is split into bf16 hi + lo
+//     (two MMAs), keeping P to ~16 bits; for f16 and E4M3 caches P is f16;
+//   - E4M3 tiles are converted to f16 (exact) in registers with
+//     cvt.rn.f16x2.e4m3x2; the contraction index d is permuted consistently in
+//     q and K so that one ldmatrix word yields both B registers of a k-step.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <math_constants.h>
+
+#include <type_traits>
+
+#include "pa_device.cuh"
+
+namespace pa {
+
+namespace mma_detail {
+
+constexpr unsigned kFull = 0xFFFFFFFFu;
+
+template <typename KVT> struct MmaType;  // element type the tensor cores see
+template <> struct MmaType<bf16_t> {
+    using T = bf16_t;
+};
+template <> struct MmaType<f16_t> {
+    using T = f16_t;
+};
+template <> struct MmaType<e4m3_t> {
+    using T = f16_t;
+};
+
+__device__ __forceinline__ void mma16816(float *c, const uint32_t *a, uint32_t b0, uint32_t b1,
+                                         bf16_t) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+        "{%8,%9}, {%0,%1,%2,%3};"
+        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ void mma16816(float *c, const uint32_t *a, uint32_t b0, uint32_t b1,
+                                         f16_t) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+        "{%8,%9}, {%0,%1,%2,%3};"
+        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ void ldsm_x4(uint32_t *r, uint32_t addr) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t *r, uint32_t addr) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(addr));
+}
+
+// two E4M3 codes (low byte first) -> f16x2, exact
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t two_codes) {
+    uint32_t h2;
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"((uint16_t)two_codes));
+    return h2;
+}
+
+__device__ __forceinline__ uint32_t pack2(float lo, float hi, f16_t) {
+    uint32_t r;
+    asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+__device__ __forceinline__ uint32_t pack2(float lo, float hi, bf16_t) {
+    uint32_t r;
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t sel) {
+    uint32_t r;
+    asm("prmt.b32 %0, %1, 0, %2;" : "=r"(r) : "r"(a), "r"(sel));
+    return r;
+}
+
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, int x, int y,
+                                            uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, "
+        "{%2, %3}], [%4];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
+        : "memory");
+}
+
+}  // namespace mma_detail
+
+template <typename QT, typename KVT, int D, int GT> struct MmaCfg {
+    using ET = typename mma_detail::MmaType<KVT>::T;
+    static constexpr bool FP8 = Elem<KVT>::kBytes == 1;
+    static constexpr bool HILO = (Elem<KVT>::kBytes == 2) && sizeof(ET) == 2 &&
+                                 std::is_same<KVT, bf16_t>::value;
+    static constexpr int NW = kDecodeWarps;
+    static constexpr int EB = Elem<KVT>::kBytes;
+    static constexpr int ROW_BYTES = D * EB;
+    static constexpr int NBOX = ROW_BYTES / 128;  // 128-byte TMA boxes per row
+    static constexpr int BOX_ELEMS = 128 / EB;
+    static constexpr int BOX_BYTES = kBlockSize * 128;  // 2 KiB
+    static constexpr int TILE_BYTES = NBOX * BOX_BYTES;
+    static constexpr int STAGE_BYTES = 2 * TILE_BYTES;
+    static constexpr int NST = (16384 / STAGE_BYTES) < 2 ? 2 : (16384 / STAGE_BYTES);
+    static constexpr int KS = D / 16;   // k-steps of q.K
+    static constexpr int NT = D / 8;    // n-tiles of P.V
+    static constexpr int SZ_STAGES = NW * NST * STAGE_BYTES;
+    static constexpr int OFF_BAR = SZ_STAGES;
+    static constexpr int SMEM = 1024 /* alignment slack */ + OFF_BAR + NW * NST * 8;
+    static constexpr int MERGE_BYTES = NW * (GT * D + 2 * GT) * 4;
+    static_assert(NBOX >= 1 && ROW_BYTES % 128 == 0, "rows must be whole 128-byte boxes");
+    static_assert(MERGE_BYTES <= SZ_STAGES, "merge area must fit in the stage buffers");
+    static_assert(GT == 8 || GT == 16, "MMA rows used: 8 or 16");
+};
+
+// Byte offset of logical 16-byte chunk `c` of token row `r` inside a tile made
+// of 128B-swizzled TMA boxes (box = 16 rows x 128 bytes, 1 KiB aligned).
+__device__ __forceinline__ uint32_t swz(int r, int c) {
+    return (uint32_t)((c >> 3) * (kBlockSize * 128) + r * 128 + (((c & 7) ^ (r & 7)) << 4));
+}
+
+template <typename QT, typename KVT, int D, int GT>
+__global__ void __launch_bounds__(kDecodeWarps * 32)
+    decode_mma_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmap_k,
+                      const __grid_constant__ CUtensorMap tmap_v) {
+    using C = MmaCfg<QT, KVT, D, GT>;
+    using ET = typename C::ET;
+    using namespace mma_detail;
+    constexpr int NW = C::NW, NST = C::NST;
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw_addr = smem_addr(smem_raw);
+    const uint32_t base_addr = (raw_addr + 1023u) & ~1023u;
+    uint8_t *smem = smem_raw + (base_addr - raw_addr);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int g = lane >> 2, kq = lane & 3;  // MMA fragment coordinates
+    const int NP = p.num_partitions;
+    const int s = blockIdx.x / NP, part = blockIdx.x - s * NP;
+    const int kvh = blockIdx.y / p.head_groups, hg = blockIdx.y - kvh * p.head_groups;
+
+    const uint32_t bar0 = base_addr + C::OFF_BAR + warp * NST * 8;
+    const uint32_t stage0 = base_addr + warp * NST * C::STAGE_BYTES;
+
+    if (lane == 0) {
+#pragma unroll
+        for (int i = 0; i < NST; ++i) mbar_init(bar0 + 8 * i, 1);
+        mbar_init_fence();
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_k)) : "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_v)) : "memory");
+    }
+    __syncwarp();
+
+    pdl_wait();
+
+    // ---- sequence length and this CTA's block range -----------------------
+    const int max_tokens = p.max_blocks_per_seq * kBlockSize;
+    int L = p.seq_lens[s];
+    if (L < 0 || L > max_tokens) {
+        if (threadIdx.x == 0) flag_error(p.err, kErrBounds);
+        L = L < 0 ? 0 : max_tokens;
+    }
+    if (p.split) {
+        const int cap = NP * p.partition_blocks * kBlockSize;
+        if (L > cap) {
+            if (threadIdx.x == 0 && part == 0) flag_error(p.err, kErrBounds);
+            L = cap;
+        }
+    }
+    const int nblk_seq = (L + kBlockSize - 1) / kBlockSize;
+    const int blk_begin = part * p.partition_blocks;
+    int blk_end = blk_begin + p.partition_blocks;
+    if (blk_end > nblk_seq) blk_end = nblk_seq;
+    if (p.split && blk_begin >= blk_end) return;
+    const int nblk = blk_end > blk_begin ? blk_end - blk_begin : 0;
+    const int nk = nblk > warp ? (nblk - warp + NW - 1) / NW : 0;
+
+    // ---- block table entries of this warp, one per lane --------------------
+    const int32_t *bt_row = p.block_tables + (int64_t)s * p.max_blocks_per_seq;
+    auto load_batch = [&](int batch) -> int {
+        const int k = batch * 32 + lane;
+        return k < nk ? bt_row[blk_begin + warp + NW * k] : 0;
+    };
+    int cur_batch = 0;
+    int bt_cur = load_batch(0);
+    int bt_nxt = nk > 32 ? load_batch(1) : 0;
+    auto bt_of = [&](int k) -> int {
+        const int a = __shfl_sync(kFull, bt_cur, k & 31);
+        const int b = __shfl_sync(kFull, bt_nxt, k & 31);
+        return (k >> 5) == cur_batch ? a : b;
+    };
+    auto issue = [&](int k) {  // whole warp calls; lane 0 issues the copies
+        int phys = bt_of(k);
+        if (lane == 0) {
+            if ((unsigned)phys >= (unsigned)p.num_blocks) {
+                flag_error(p.err, kErrBounds);
+                phys = 0;  // a valid block whose tokens are all masked
+            }
+            const int st = k % NST;
+            const uint32_t bar = bar0 + 8 * st;
+            const uint32_t dst = stage0 + st * C::STAGE_BYTES;
+            const int y = (phys * p.num_kv_heads + kvh) * kBlockSize;
+            mbar_arrive_expect_tx(bar, C::STAGE_BYTES);
+#pragma unroll
+            for (int b = 0; b < C::NBOX; ++b) {
+                tma_load_2d(dst + b * C::BOX_BYTES, &tmap_k, b * C::BOX_ELEMS, y, bar);
+                tma_load_2d(dst + C::TILE_BYTES + b * C::BOX_BYTES, &tmap_v, b * C::BOX_ELEMS, y, bar);
+            }
+        }
+    };
+    const int npre = nk < NST ? nk : NST;
+    for (int k = 0; k < npre; ++k) issue(k);
+
+    // ---- q as MMA A fragments (rows = heads of this group) ----------------
+    // a[ks][0]: row g, a[ks][1]: row g+8, a[ks][2]: row g (k+8), a[ks][3]: row g+8 (k+8)
+    uint32_t qa[C::KS][4];
+    float qscale = p.qk_scale_log2;
+    {
+        const int group_base = hg * GT;
+        const uint16_t *q16 = static_cast<const uint16_t *>(p.q);
+        float qv[2][C::KS][4];  // [row half][ks][4 values]
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+            const int row = g + 8 * hh;
+            const bool hv = (GT == 16 || hh == 0) && row < GT && group_base + row < p.group;
+            const int64_t hq = (int64_t)kvh * p.group + group_base + row;
+            const uint16_t *qrow = q16 + ((int64_t)s * p.num_q_heads + (hv ? hq : 0)) * D;
+#pragma unroll
+            for (int ks = 0; ks < C::KS; ++ks) {
+                // physical d of the four values this lane feeds in k-step ks
+                int d0, d1, d2, d3;
+                if constexpr (C::FP8) {
+                    d0 = 16 * ks + 4 * kq; d1 = d0 + 1; d2 = d0 + 2; d3 = d0 + 3;
+                } else {
+                    d0 = 16 * ks + 2 * kq; d1 = d0 + 1; d2 = d0 + 8; d3 = d0 + 9;
+                }
+                float v0 = 0.f, v1 = 0.f, v2 = 0.f, v3 = 0.f;
+                if (hv) {
+                    const uint32_t w01 = *reinterpret_cast<const uint32_t *>(qrow + d0);
+                    const uint32_t w23 = *reinterpret_cast<const uint32_t *>(qrow + d2);
+                    unpack2(QT{}, w01, v0, v1);
+                    unpack2(QT{}, w23, v2, v3);
+                }
+                qv[hh][ks][0] = v0; qv[hh][ks][1] = v1; qv[hh][ks][2] = v2; qv[hh][ks][3] = v3;
+            }
+        }
+        if constexpr (!std::is_same<QT, ET>::value) {
+            // bf16 q against an f16 tensor-core path (E4M3 cache): scale q by a
+            // power of two so its largest element sits near 2^14, convert to
+            // f16, and fold the inverse power into the logit scale (exact).
+            float amax = 0.f;
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh)
+#pragma unroll
+                for (int ks = 0; ks < C::KS; ++ks)
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) amax = fmaxf(amax, fabsf(qv[hh][ks][i]));
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, o));
+            int e = 0;
+            if (amax > 0.f) {
+                const int ex = (int)((__float_as_uint(amax) >> 23) & 0xFF) - 127;  // floor(log2)
+                e = 14 - ex;
+                if (e > 100) e = 100;
+                if (e < -100) e = -100;
+            }
+            const float up = __uint_as_float((uint32_t)(127 + e) << 23);   // 2^e, exact
+            qscale = p.qk_scale_log2 * __uint_as_float((uint32_t)(127 - e) << 23);
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh)
+#pragma unroll
+                for (int ks = 0; ks < C::KS; ++ks)
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) qv[hh][ks][i] *= up;
+        }
+#pragma unroll
+        for (int ks = 0; ks < C::KS; ++ks) {
+            qa[ks][0] = pack2(qv[0][ks][0], qv[0][ks][1], ET{});
+            qa[ks][1] = pack2(qv[1][ks][0], qv[1][ks][1], ET{});
+            qa[ks][2] = pack2(qv[0][ks][2], qv[0][ks][3], ET{});
+            qa[ks][3] = pack2(qv[1][ks][2], qv[1][ks][3], ET{});
+        }
+    }
+
+    // ---- main loop ------------------------------------------------------------
+    constexpr int NR = GT / 8;  // accumulator rows a lane owns: g (and g+8)
+    float m_run[NR], l_run[NR];
+    float o[C::NT][4];
+#pragma unroll
+    for (int r = 0; r < NR; ++r) {
+        m_run[r] = -CUDART_INF_F;
+        l_run[r] = 0.f;
+    }
+#pragma unroll
+    for (int n = 0; n < C::NT; ++n)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) o[n][i] = 0.f;
+
+    // per-lane ldmatrix row / chunk selectors
+    const int lrow_b = (lane & 7) + 8 * (lane >> 4);   // q.K: tokens 0-7 | 8-15
+    const int lsel_b = (lane >> 3) & 1;                 // q.K: chunk +0 | +1
+    const int lrow_v = (lane & 7) + 8 * ((lane >> 3) & 1);  // P.V: tokens 0-7 | 8-15
+    const int lsel_v = lane >> 4;                       // P.V: chunk +0 | +1
+    bool timed_out = false;
+    int k = 0;
+
+    for (; k < nk; ++k) {
+        if (k > 0 && (k & 31) == 0) {
+            bt_cur = bt_nxt;
+            ++cur_batch;
+            bt_nxt = nk > (cur_batch + 1) * 32 ? load_batch(cur_batch + 1) : 0;
+        }
+        const int st = k % NST;
+        const bool ok = __all_sync(kFull, mbar_wait_bounded(bar0 + 8 * st, (k / NST) & 1, kWaitLimitNs));
+        if (!ok) {
+            if (lane == 0) flag_error(p.err, kErrTimeout);
+            timed_out = true;
+            break;
+        }
+        const int j = blk_begin + warp + NW * k;
+        const bool valid = (unsigned)bt_of(k) < (unsigned)p.num_blocks;
+        int nvalid = L - j * kBlockSize;
+        nvalid = valid ? (nvalid < kBlockSize ? nvalid : kBlockSize) : 0;
+        const uint32_t kt = stage0 + st * C::STAGE_BYTES;
+        const uint32_t vt = kt + C::TILE_BYTES;
+
+        // S = Q K^T for the block's 16 tokens (two n-tiles of 8)
+        float sc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+        if constexpr (!C::FP8) {
+#pragma unroll
+            for (int ks = 0; ks < C::KS; ++ks) {
+                uint32_t b[4];
+                ldsm_x4(b, kt + swz(lrow_b, 2 * ks + lsel_b));
+                mma16816(sc[0], qa[ks], b[0], b[1], ET{});
+                mma16816(sc[1], qa[ks], b[2], b[3], ET{});
+            }
+        } else {
+#pragma unroll
+            for (int jj = 0; jj < C::KS / 2; ++jj) {
+                uint32_t w[4];  // (nt0, ks=2jj), (nt0, 2jj+1), (nt1, 2jj), (nt1, 2jj+1)
+                ldsm_x4(w, kt + swz(lrow_b, 2 * jj + lsel_b));
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    const int ks = 2 * jj + h;
+                    mma16816(sc[0], qa[ks], e4m3x2_to_f16x2(w[h]), e4m3x2_to_f16x2(w[h] >> 16), ET{});
+                    mma16816(sc[1], qa[ks], e4m3x2_to_f16x2(w[2 + h]), e4m3x2_to_f16x2(w[2 + h] >> 16), ET{});
+                }
+            }
+        }
+
+        // online softmax; lane holds S[row g (+8)][tokens 2kq, 2kq+1, 8+2kq, 9+2kq]
+        const int t0 = 2 * kq;
+        float alpha[NR];
+        float pr[NR][4];
+#pragma unroll
+        for (int r = 0; r < NR; ++r) {
+            float sv[4];
+            sv[0] = t0 < nvalid ? sc[0][2 * r] * qscale : -CUDART_INF_F;
+            sv[1] = t0 + 1 < nvalid ? sc[0][2 * r + 1] * qscale : -CUDART_INF_F;
+            sv[2] = t0 + 8 < nvalid ? sc[1][2 * r] * qscale : -CUDART_INF_F;
+            sv[3] = t0 + 9 < nvalid ? sc[1][2 * r + 1] * qscale : -CUDART_INF_F;
+            float bm = fmaxf(fmaxf(sv[0], sv[1]), fmaxf(sv[2], sv[3]));
+            bm = fmaxf(bm, __shfl_xor_sync(kFull, bm, 1));
+            bm = fmaxf(bm, __shfl_xor_sync(kFull, bm, 2));
+            const float m_new = fmaxf(m_run[r], bm);
+            alpha[r] = 1.f;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) pr[r][i] = 0.f;
+            if (m_new != -CUDART_INF_F) {
+                alpha[r] = exp2f(m_run[r] - m_new);
+#pragma unroll
+                for (int i = 0; i < 4; ++i) pr[r][i] = exp2f(sv[i] - m_new);
+            }
+            l_run[r] = l_run[r] * alpha[r] + ((pr[r][0] + pr[r][1]) + (pr[r][2] + pr[r][3]));
+            m_run[r] = m_new;
+        }
+#pragma unroll
+        for (int n = 0; n < C::NT; ++n) {
+            o[n][0] *= alpha[0];
+            o[n][1] *= alpha[0];
+            if constexpr (NR == 2) {
+                o[n][2] *= alpha[1];
+                o[n][3] *= alpha[1];
+            }
+        }
+
+        // P as A fragments (k = tokens), hi and (bf16 cache) lo parts
+        uint32_t pa_hi[4], pa_lo[4];
+        {
+            const float r1_0 = NR == 2 ? pr[NR - 1][0] : 0.f, r1_1 = NR == 2 ? pr[NR - 1][1] : 0.f;
+            const float r1_2 = NR == 2 ? pr[NR - 1][2] : 0.f, r1_3 = NR == 2 ? pr[NR - 1][3] : 0.f;
+            pa_hi[0] = pack2(pr[0][0], pr[0][1], ET{});
+            pa_hi[1] = pack2(r1_0, r1_1, ET{});
+            pa_hi[2] = pack2(pr[0][2], pr[0][3], ET{});
+            pa_hi[3] = pack2(r1_2, r1_3, ET{});
+            if constexpr (C::HILO) {
+                const float vals[4][2] = {{pr[0][0], pr[0][1]}, {r1_0, r1_1}, {pr[0][2], pr[0][3]}, {r1_2, r1_3}};
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const float h0 = __uint_as_float(pa_hi[i] << 16);
+                    const float h1 = __uint_as_float(pa_hi[i] & 0xFFFF0000u);
+                    pa_lo[i] = pack2(vals[i][0] - h0, vals[i][1] - h1, ET{});
+                }
+            }
+        }
+
+        // O += P V; tokens past nvalid have p = 0 but their V rows may hold
+        // NaN poison (0 * NaN = NaN): zero those V fragments first
+        const bool full = nvalid == kBlockSize;
+        const bool tv0 = t0 < nvalid, tv1 = t0 + 1 < nvalid, tv8 = t0 + 8 < nvalid, tv9 = t0 + 9 < nvalid;
+        if constexpr (!C::FP8) {
+#pragma unroll
+            for (int cp = 0; cp < C::NT / 2; ++cp) {
+                uint32_t b[4];  // (nt 2cp: tok 0-7, tok 8-15), (nt 2cp+1: tok 0-7, tok 8-15)
+                ldsm_x4_t(b, vt + swz(lrow_v, 2 * cp + lsel_v));
+                if (!full) {
+                    // b[0], b[2]: tokens 2kq, 2kq+1; b[1], b[3]: tokens 8+2kq, 9+2kq
+                    const uint32_t m0 = (tv0 ? 0x0000FFFFu : 0u) | (tv1 ? 0xFFFF0000u : 0u);
+                    const uint32_t m8 = (tv8 ? 0x0000FFFFu : 0u) | (tv9 ? 0xFFFF0000u : 0u);
+                    b[0] &= m0; b[2] &= m0; b[1] &= m8; b[3] &= m8;
+                }
+                mma16816(o[2 * cp], pa_hi, b[0], b[1], ET{});
+                mma16816(o[2 * cp + 1], pa_hi, b[2], b[3], ET{});
+                if constexpr (C::HILO) {
+                    mma16816(o[2 * cp], pa_lo, b[0], b[1], ET{});
+                    mma16816(o[2 * cp + 1], pa_lo, b[2], b[3], ET{});
+                }
+            }
+        } else {
+#pragma unroll
+            for (int cp = 0; cp < C::NT / 4; ++cp) {
+                uint32_t w[4];  // chunk 2cp: tok 0-7, tok 8-15; chunk 2cp+1: tok 0-7, tok 8-15
+                ldsm_x4_t(w, vt + swz(lrow_v, 2 * cp + lsel_v));
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    // regroup bytes: low half = (tok 2kq, tok 2kq+1) at even d,
+                    // high half = same tokens at odd d
+                    const uint32_t lo_t = prmt(w[2 * h], 0x3120);
+                    const uint32_t hi_t = prmt(w[2 * h + 1], 0x3120);
+                    uint32_t be0 = e4m3x2_to_f16x2(lo_t), bo0 = e4m3x2_to_f16x2(lo_t >> 16);
+                    uint32_t be1 = e4m3x2_to_f16x2(hi_t), bo1 = e4m3x2_to_f16x2(hi_t >> 16);
+                    if (!full) {
+                        const uint32_t m0 = (tv0 ? 0x0000FFFFu : 0u) | (tv1 ? 0xFFFF0000u : 0u);
+                        const uint32_t m8 = (tv8 ? 0x0000FFFFu : 0u) | (tv9 ? 0xFFFF0000u : 0u);
+                        be0 &= m0; bo0 &= m0; be1 &= m8; bo1 &= m8;
+                    }
+                    const int c = 2 * cp + h;  // 16-element chunk of d
+                    mma16816(o[2 * c], pa_hi, be0, be1, ET{});      // even d of chunk c
+                    mma16816(o[2 * c + 1], pa_hi, bo0, bo1, ET{});  // odd d of chunk c
+                }
+            }
+        }
+        __syncwarp();
+        if (k + NST < nk) issue(k + NST);
+    }
+
+    if (timed_out) {
+        if (lane == 0) {
+            for (int kk = k; kk < nk && kk < k + NST; ++kk)
+                (void)mbar_wait_bounded(bar0 + 8 * (kk % NST), (kk / NST) & 1, kWaitLimitNs / 16);
+        }
+        __syncwarp();
+    }
+
+    pdl_launch_dependents();
+
+    // ---- merge the warps' partial states ---------------------------------------
+#pragma unroll
+    for (int r = 0; r < NR; ++r) {
+        l_run[r] += __shfl_xor_sync(kFull, l_run[r], 1);
+        l_run[r] += __shfl_xor_sync(kFull, l_run[r], 2);
+    }
+    __syncthreads();
+    float *ms = reinterpret_cast<float *>(smem);
+    float *ls = ms + NW * GT;
+    float *accs = ls + NW * GT;
+    if (kq == 0) {
+#pragma unroll
+        for (int r = 0; r < NR; ++r) {
+            ms[warp * GT + g + 8 * r] = m_run[r];
+            ls[warp * GT + g + 8 * r] = l_run[r];
+        }
+    }
+#pragma unroll
+    for (int n = 0; n < C::NT; ++n) {
+#pragma unroll
+        for (int r = 0; r < NR; ++r) {
+#pragma unroll
+            for (int ci = 0; ci < 2; ++ci) {
+                int d;
+                if constexpr (C::FP8) {
+                    d = 16 * (n >> 1) + 4 * kq + 2 * ci + (n & 1);
+                } else {
+                    d = 8 * n + 2 * kq + ci;
+                }
+                accs[(warp * GT + g + 8 * r) * D + d] = o[n][2 * r + ci];
+            }
+        }
+    }
+    __syncthreads();
+
+    const int group_base = hg * GT;
+    for (int idx = threadIdx.x; idx < GT * D; idx += NW * 32) {
+        const int i = idx / D, d = idx - i * D;
+        if (group_base + i >= p.group) continue;
+        const int64_t hq = (int64_t)kvh * p.group + group_base + i;
+        float M = -CUDART_INF_F;
+#pragma unroll
+        for (int w = 0; w < NW; ++w) M = fmaxf(M, ms[w * GT + i]);
+        float O = 0.f, Ls = 0.f;
+        if (M != -CUDART_INF_F) {
+#pragma unroll
+            for (int w = 0; w < NW; ++w) {
+                const float f = exp2f(ms[w * GT + i] - M);
+                Ls = fmaf(f, ls[w * GT + i], Ls);
+                O = fmaf(f, accs[(w * GT + i) * D + d], O);
+            }
+        }
+        const float ov = Ls > 0.f ? (O / Ls) * p.v_scale : 0.f;
+        const int64_t row = (int64_t)s * p.num_q_heads + hq;
+        if (!p.split) {
+            reinterpret_cast<uint16_t *>(p.out)[row * D + d] = from_float(QT{}, ov);
+        } else {
+            p.ws_o[(row * NP + part) * D + d] = ov;
+            if (d == 0)
+                p.ws_lse[row * NP + part] =
+                    Ls > 0.f ? (M + log2f(Ls)) * 0.69314718055994530942f : -CUDART_INF_F;
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
+// host side: tensor maps and launch
+// ---------------------------------------------------------------------------
+
+namespace {
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static bool tried = false;
+    if (!tried) {
+        tried = true;
+        void *f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+    }
+    return fn;
+}
+
+// 2-D view of a pool [NB, Hk, 16, d]: rows = NB * Hk * 16 tokens, d columns;
+// boxes of 16 rows x 128 bytes, 128-byte swizzle.
+bool encode_pool_map(CUtensorMap *m, const void *base, int elem_bytes, int d, int64_t rows) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[2] = {(cuuint64_t)d, (cuuint64_t)rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)d * (cuuint64_t)elem_bytes};
+    const cuuint32_t box[2] = {(cuuint32_t)(128 / elem_bytes), (cuuint32_t)kBlockSize};
+    const cuuint32_t estr[2] = {1, 1};
+    const CUresult r = fn(m, elem_bytes == 1 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_UINT16,
+                          2, const_cast<void *>(base), dims, strides, box, estr,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+template <typename QT, typename KVT, int D, int GT>
+cudaError_t launch_mma_t(const DecodeParams &p, cudaStream_t stream) {
+    using C = MmaCfg<QT, KVT, D, GT>;
+    const int64_t rows = (int64_t)p.num_blocks * p.num_kv_heads * kBlockSize;
+    CUtensorMap mk, mv;
+    if (!encode_pool_map(&mk, p.k_cache, C::EB, D, rows) ||
+        !encode_pool_map(&mv, p.v_cache, C::EB, D, rows))
+        return cudaErrorInvalidValue;
+    auto kern = decode_mma_kernel<QT, KVT, D, GT>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(p.num_seqs * p.num_partitions), (unsigned)(p.num_kv_heads * p.head_groups));
+    cfg.blockDim = dim3(C::NW * 32);
+    cfg.dynamicSmemBytes = C::SMEM;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, p, mk, mv);
+}
+
+template <typename QT, typename KVT, int D>
+cudaError_t mma_by_rows(const DecodeParams &p, int gt, cudaStream_t stream) {
+    return gt == 16 ? launch_mma_t<QT, KVT, D, 16>(p, stream) : launch_mma_t<QT, KVT, D, 8>(p, stream);
+}
+
+}  // namespace
+
+bool mma_decode_supported(DType kv, int head_dim, int num_blocks, int num_kv_heads) {
+    if (!encode_fn()) return false;
+    const int64_t rows = (int64_t)num_blocks * num_kv_heads * kBlockSize;
+    if (rows >= (int64_t(1) << 31)) return false;  // TMA row coordinate is a signed 32-bit int
+    if (kv == DType::E4M3) return head_dim == 128;
+    return head_dim == 64 || head_dim == 128;
+}
+
+cudaError_t launch_decode_mma(const DecodeParams &p, DType q, DType kv, int head_dim, int mma_rows,
+                              cudaStream_t stream) {
+    if (p.num_seqs <= 0) return cudaSuccess;
+    if (kv == DType::E4M3) {
+        if (head_dim != 128) return cudaErrorInvalidValue;
+        return q == DType::F16 ? mma_by_rows<f16_t, e4m3_t, 128>(p, mma_rows, stream)
+                               : mma_by_rows<bf16_t, e4m3_t, 128>(p, mma_rows, stream);
+    }
+    if (q == DType::F16)
+        return head_dim == 64 ? mma_by_rows<f16_t, f16_t, 64>(p, mma_rows, stream)
+                              : mma_by_rows<f16_t, f16_t, 128>(p, mma_rows, stream);
+    return head_dim == 64 ? mma_by_rows<bf16_t, bf16_t, 64>(p, mma_rows, stream)
+                          : mma_by_rows<bf16_t, bf16_t, 128>(p, mma_rows, stream);
+}
+
+}  // namespace pa

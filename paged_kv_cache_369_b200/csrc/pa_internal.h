@@ -88,4 +88,11 @@ cudaError_t launch_decode(const DecodeParams &p, DType q, DType kv, int head_dim
                           cudaStream_t stream);
 cudaError_t launch_reduce(const ReduceParams &p, DType q, int head_dim, cudaStream_t stream);
 
+// Tensor-core decode (pa_decode_mma.cu): rows of the MMA used for the GQA
+// group (8 or 16); supported for head_dim 64/128 16-bit caches and head_dim
+// 128 E4M3 caches whose pool has fewer than 2^31 token rows.
+bool mma_decode_supported(DType kv, int head_dim, int num_blocks, int num_kv_heads);
+cudaError_t launch_decode_mma(const DecodeParams &p, DType q, DType kv, int head_dim, int mma_rows,
+                              cudaStream_t stream);
+
 }  // namespace pa

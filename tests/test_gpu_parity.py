@@ -11,6 +11,7 @@ Bars:
 """
 
 import math
+import os
 
 import numpy as np
 import pytest
@@ -85,9 +86,20 @@ SMALL = [
 ]
 
 
+@pytest.fixture(params=["auto", "simt"])
+def kernel_choice(request, monkeypatch):
+    """Run a test with the default decode kernel (tensor cores wherever the
+    shape allows) and with the CUDA-core kernel forced."""
+    if request.param == "simt":
+        monkeypatch.setenv("PA369_DECODE_KERNEL", "simt")
+    else:
+        monkeypatch.delenv("PA369_DECODE_KERNEL", raising=False)
+    return request.param
+
+
 @pytest.mark.parametrize("mode,P", [("single", 512), ("split", 512), ("split", 16), ("split", 64)])
 @pytest.mark.parametrize("case", range(len(SMALL)))
-def test_small_full_parity(case, mode, P):
+def test_small_full_parity(case, mode, P, kernel_choice):
     pa, PagedDecode = _pa()
     Hq, Hk, d, act, kv, lens, prefix = SMALL[case]
     w = workload.build(f"small{case}", 1000 + case, lens, Hq, Hk, d, act, kv,
@@ -100,14 +112,14 @@ def test_small_full_parity(case, mode, P):
     check_pools(dec, kc, vc)
     ref = oracle.decode_for(w, kc, vc)
     got = _to_f64(dec.out)
-    assert_close(got, ref, f"case {case} {mode} P={P}")
+    assert_close(got, ref, f"case {case} {mode} P={P} kernel={kernel_choice}")
     # empty sequences give exact zeros
     for s in range(w.num_seqs):
         if w.seq_lens[s] == 0:
             assert not got[s].any()
 
 
-def test_split_partials_match_oracle():
+def test_split_partials_match_oracle(kernel_choice):
     pa, PagedDecode = _pa()
     w = workload.build("partials", 77, [1, 16, 17, 100, 513, 1100], 16, 4, 128, "bf16", "bf16")
     P = 128
@@ -131,7 +143,7 @@ def test_split_partials_match_oracle():
         assert_close(o[s, h, :np_s], o_ref[i, :np_s], f"partials s={s} h={h}")
 
 
-def test_single_token_is_exact_v():
+def test_single_token_is_exact_v(kernel_choice):
     """L = 1: p = 1 exactly, so the output equals the new token's v bit for bit."""
     pa, PagedDecode = _pa()
     for act in ("f16", "bf16"):
@@ -144,7 +156,7 @@ def test_single_token_is_exact_v():
             assert torch.equal(dec.out.view(torch.int16), v.view(torch.int16))
 
 
-def test_physical_permutation_bitwise():
+def test_physical_permutation_bitwise(kernel_choice):
     """Moving blocks to other physical ids (tables rewritten) changes nothing."""
     pa, PagedDecode = _pa()
     w = workload.build("perm", 8, [10, 45, 20, 33, 300], 8, 2, 64, "bf16", "bf16", pool_slack=0.5)
@@ -211,6 +223,16 @@ def test_named_workload_parity(cfg):
     assert dec.error() == 0
     out_single = _to_f64(dec.out)
     assert_close(out_single[pairs[:, 0], pairs[:, 1]], ref, f"config {cfg} single")
+    # the CUDA-core kernel on the same state
+    os.environ["PA369_DECODE_KERNEL"] = "simt"
+    try:
+        dec.mode = "split"
+        dec.attend()
+        torch.cuda.synchronize()
+    finally:
+        del os.environ["PA369_DECODE_KERNEL"]
+    assert dec.error() == 0
+    assert_close(_to_f64(dec.out)[pairs[:, 0], pairs[:, 1]], ref, f"config {cfg} simt split")
     # property at full size: every output row is a convex combination of its
     # V rows, so it lies inside their per-element range
     _check_convex_hull(w, dec, out_split)
@@ -241,7 +263,7 @@ def _check_convex_hull(w, dec, out):
 # device-side range checks: corrupt inputs are reported, never dereferenced
 # ---------------------------------------------------------------------------
 
-def test_corrupt_block_table_is_reported():
+def test_corrupt_block_table_is_reported(kernel_choice):
     pa, PagedDecode = _pa()
     w = workload.build("bad", 12, [40, 70], 8, 2, 64, "bf16", "bf16")
     for mode in ("single", "split"):
