@@ -185,6 +185,45 @@ pa_status pa_decode_split_reduce(void *out, const void *q, const void *k_cache,
                                  void *workspace, size_t workspace_bytes, int *dev_err,
                                  void *stream);
 
+/* Bytes of scratch built into the library for
+ * pa_decode_split_reduce_static_scratch (32 MiB). */
+#define PA_STATIC_SCRATCH_BYTES (32u * 1024u * 1024u)
+
+/*
+ * pa_decode_split_reduce_static_scratch -- pa_decode_split_reduce for callers
+ * that cannot allocate device memory.
+ *
+ * No counterpart in the paper: this is a deployment convenience, not part of
+ * the method.  Some callers have no allocator to draw a workspace from: a
+ * plugin or custom-op host that passes tensors but no allocator, a serving
+ * engine that has already reserved all free HBM for its KV block pool, or a
+ * latency-critical loop that must not pay cudaMalloc's implicit device
+ * synchronisation.  This entry point takes no workspace: the per-partition
+ * partials go to a __device__ array of PA_STATIC_SCRATCH_BYTES bytes inside
+ * the library, which a GPU that loads this code may hold until the process
+ * exits.  The caller still provides every input and the output; the call
+ * allocates nothing (no cudaMalloc, cudaFree or allocating library routine).
+ *
+ * Arguments and result are those of pa_decode_split_reduce without
+ * `workspace` / `workspace_bytes`.
+ *   - Returns PA_ERR_INVALID_ARG, before touching the GPU, when the partials
+ *     for these sizes, pa_split_workspace_bytes(num_seqs, num_q_heads,
+ *     head_dim, max_seq_len, partition_size), exceed PA_STATIC_SCRATCH_BYTES.
+ *   - The first call on a device looks up the array's device address on that
+ *     (current) device; make that first call before any stream capture.
+ *     PA_ERR_CUDA if the lookup fails.
+ *   - Every call, on every stream, shares the one array per device, and the
+ *     array keeps the last call's partials: nothing in it has to start at zero
+ *     (each partial is written before it is read), but calls that overlap on
+ *     the GPU race with each other.  Serialise them (one stream, or events).
+ */
+pa_status pa_decode_split_reduce_static_scratch(
+    void *out, const void *q, const void *k_cache, const void *v_cache,
+    const int32_t *block_tables, int max_blocks_per_seq, const int32_t *seq_lens, int num_seqs,
+    int num_q_heads, int num_kv_heads, int head_dim, int block_size, int num_blocks,
+    float softmax_scale, pa_dtype q_dtype, pa_dtype kv_dtype, float k_scale, float v_scale,
+    int partition_size, int max_seq_len, int *dev_err, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

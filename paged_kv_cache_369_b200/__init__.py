@@ -5,8 +5,9 @@ same name (include/pa.h), whose kernels do all of the work.  Tensors are torch
 CUDA tensors (device memory and streams come from PyTorch); integer pointers
 are accepted too.  A non-OK status raises ``PaError``.
 
-The shared library is built in-tree by ``python -m paged_kv_cache_369_b200.build``;
-importing this package without it raises ImportError: there is no fallback.
+The shared library is built in-tree by ``python paged_kv_cache_369_b200/build.py``;
+importing this package without it (or with a stale one) raises ImportError:
+there is no fallback.
 """
 
 from __future__ import annotations
@@ -32,8 +33,10 @@ PA_FP8_E4M3 = 2
 # every extern "C" symbol declared in include/pa.h
 SYMBOLS = (
     "pa_status_string", "pa_version", "pa_slot_mapping", "pa_cache_write", "pa_decode",
-    "pa_split_workspace_bytes", "pa_decode_split_reduce",
+    "pa_split_workspace_bytes", "pa_decode_split_reduce", "pa_decode_split_reduce_static_scratch",
 )
+
+PA_STATIC_SCRATCH_BYTES = 32 * 1024 * 1024
 
 
 class PaError(RuntimeError):
@@ -44,10 +47,14 @@ class PaError(RuntimeError):
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(
-        f"{LIB_PATH} is missing: build it with `python -m paged_kv_cache_369_b200.build` "
+        f"{LIB_PATH} is missing: build it with `python paged_kv_cache_369_b200/build.py` "
         "(nvcc, sm_100a). There is no CPU fallback.")
 
 _lib = ctypes.CDLL(LIB_PATH)
+_missing = [name for name in SYMBOLS if not hasattr(_lib, name)]
+if _missing:
+    raise ImportError(f"{LIB_PATH} is stale (missing {', '.join(_missing)}): rebuild it with "
+                      "`python paged_kv_cache_369_b200/build.py`")
 _P, _I, _F, _S = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
 
 _lib.pa_status_string.restype = ctypes.c_char_p
@@ -66,6 +73,9 @@ _lib.pa_split_workspace_bytes.argtypes = [_I, _I, _I, _I, _I]
 _lib.pa_decode_split_reduce.restype = _I
 _lib.pa_decode_split_reduce.argtypes = [_P, _P, _P, _P, _P, _I, _P, _I, _I, _I, _I, _I, _I, _F,
                                         _I, _I, _F, _F, _I, _I, _P, _S, _P, _P]
+_lib.pa_decode_split_reduce_static_scratch.restype = _I
+_lib.pa_decode_split_reduce_static_scratch.argtypes = [_P, _P, _P, _P, _P, _I, _P, _I, _I, _I, _I,
+                                                       _I, _I, _F, _I, _I, _F, _F, _I, _I, _P, _P]
 
 
 def lib() -> ctypes.CDLL:
@@ -188,3 +198,20 @@ def split_workspace_views(workspace, num_seqs: int, num_q_heads: int, head_dim: 
     lse = flat[:rows * 4].view(torch.float32).view(num_seqs, num_q_heads, np_)
     o = flat[lse_bytes:lse_bytes + rows * head_dim * 4].view(torch.float32)
     return lse, o.view(num_seqs, num_q_heads, np_, head_dim)
+
+
+def pa_decode_split_reduce_static_scratch(out, q, k_cache, v_cache, block_tables, seq_lens,
+                                          softmax_scale: float, partition_size: int,
+                                          max_seq_len: int, k_scale: float = 1.0,
+                                          v_scale: float = 1.0, dev_err=None,
+                                          stream=None) -> None:
+    """Split-KV decode whose partials live in the library's own device array
+    (PA_STATIC_SCRATCH_BYTES), for callers that cannot allocate; see pa.h."""
+    S, Hq, d = (int(x) for x in q.shape)
+    nb, Hk, B, _ = (int(x) for x in k_cache.shape)
+    _check(_lib.pa_decode_split_reduce_static_scratch(
+        _ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables),
+        int(block_tables.shape[1]), _ptr(seq_lens), S, Hq, Hk, d, B, nb, float(softmax_scale),
+        dtype_code(q.dtype), dtype_code(k_cache.dtype), float(k_scale), float(v_scale),
+        int(partition_size), int(max_seq_len), _ptr(dev_err), _stream(stream)),
+        "pa_decode_split_reduce_static_scratch")

@@ -1,6 +1,9 @@
 """Build libpa369.so in-tree with nvcc for sm_100a (B200).
 
-    python -m paged_kv_cache_369_b200.build [--force]
+    python paged_kv_cache_369_b200/build.py [--force] [--ptxas-v]
+
+Run it as a script (or load it by path): it must not import the package,
+whose import loads the library it builds.
 
 Each .cu file under csrc/ is compiled to an object in _build/ (in parallel),
 then linked into paged_kv_cache_369_b200/libpa369.so with the CUDA runtime
@@ -88,3 +91,4 @@ def main():
 
 if __name__ == "__main__":
     main()
+

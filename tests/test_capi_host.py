@@ -16,8 +16,12 @@ HEADER = os.path.join(ROOT, "include", "pa.h")
 
 @pytest.fixture(scope="module")
 def pa():
-    from paged_kv_cache_369_b200 import build as b
+    import importlib.util
 
+    spec = importlib.util.spec_from_file_location(
+        "_pa369_build", os.path.join(ROOT, "paged_kv_cache_369_b200", "build.py"))
+    b = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(b)
     b.build()
     import paged_kv_cache_369_b200 as m
 
