@@ -1,11 +1,14 @@
 """Benchmark of one paged decode step on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--config 2] [--mode split|single] [--partition 512]
+                    [--config 2] [--mode fused|fused_single|split|single] [--partition 512]
 
 A step is one pass of the whole hot path over one batch: slot mapping of the
-new tokens, cache write of their K/V rows, and decode attention (split-KV
-partition + reduce by default).  The default workload is the Qwen3-8B-shaped
+new tokens, cache write of their K/V rows, and decode attention.  The default
+mode ("fused") makes it one pa_decode_append call: the split-KV decode kernel
+stores the new tokens itself, then the reduce kernel merges the partitions
+(2 launches).  "split" / "single" run pa_slot_mapping + pa_cache_write and
+then pa_decode_split_reduce / pa_decode (4 / 3 launches).  The default workload is the Qwen3-8B-shaped
 decode step: 64 sequences, 32 query / 8 KV heads, head_dim 128, bf16, lengths
 U[512, 4096], 16-token blocks in a shuffled pool.  Its K/V (~585 MB) is larger
 than L2 (126 MB), so no L2 flush is needed between steps.
@@ -14,7 +17,8 @@ Output: one JSON line on rank 0.  ``value`` is KV GB/s of the whole job
 (algorithmic step bytes of all ranks / max-over-ranks step time); ``e2e`` is
 the same with the step's inputs copied from pinned host memory and its output
 read back inside the timed region; ``roofline`` is for the attention launch
-(partition + reduce kernels) against the measured HBM copy bandwidth;
+(decode kernel + reduce kernel, event-timed together) against the measured HBM
+copy bandwidth;
 ``cpu_baseline`` times the CPU oracle on a bounded sample.
 
 ``--impl reference`` times the CPU oracle itself as the reference arm (rank 0
@@ -186,7 +190,7 @@ def workload_config(w, cfg: int, mode: str, P: int) -> dict:
         "block_size": w.block_size, "kv_dtype": w.kv_dtype, "act_dtype": w.act_dtype,
         "seq_len_mean": float(w.seq_lens.mean()), "seq_len_min": int(w.seq_lens.min()),
         "seq_len_max": int(w.seq_lens.max()), "num_blocks": w.num_blocks, "seed": w.seed,
-        "mode": mode, "partition_size": P if mode == "split" else None,
+        "mode": mode, "partition_size": P if mode in ("split", "fused") else None,
         "l2": "inputs larger than L2: no flush" if w.kv_bytes_logical() > 256e6
         else "L2 flushed (256 MB write) between steps",
     }
@@ -298,8 +302,10 @@ def run_ours(args):
     with torch.cuda.stream(stream):
         dec = PagedDecode(w, device=str(device), mode=args.mode, partition_size=args.partition,
                           stream=stream)
+    fused = args.mode.startswith("fused")
     step_bytes = w.step_bytes()
-    attn_bytes = algorithmic_decode_bytes(w)
+    # the fused attention launch also reads the new rows and stores them
+    attn_bytes = step_bytes if fused else algorithmic_decode_bytes(w)
     flush = None
     if w.kv_bytes_logical() <= 256e6:
         flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=device)
@@ -330,9 +336,13 @@ def run_ours(args):
         for i in range(args.steps):
             e0, e1, e2 = ev[i]
             e0.record(stream)
-            dec.write_new()
-            e1.record(stream)
-            dec.attend()
+            if fused:
+                e1.record(stream)
+                dec.step()  # one call: new tokens stored by the attention launch
+            else:
+                dec.write_new()
+                e1.record(stream)
+                dec.attend()
             e2.record(stream)
             if flush is not None:
                 flush_ev[i][0].record(stream)
@@ -396,14 +406,17 @@ def run_ours(args):
             "us_per_step": step_ms * 1e3,
             "tokens_per_s": world * w.num_seqs / (step_ms * 1e-3),
             "attention_us": attn_ms * 1e3,
-            "cache_write_us": write_ms * 1e3,
+            "cache_write_us": None if fused else write_ms * 1e3,
             "kv_bytes_per_step": w.kv_bytes_logical(),
             "step_bytes": step_bytes,
             "roofline": {
                 "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                 "frac": achieved / peak, "traffic": traffic,
-                "kernel": "attention launch (decode partition kernel + split reduce kernel)"
-                if args.mode == "split" else "decode kernel (single pass)",
+                "kernel": {
+                    "fused": "pa_decode_append: decode kernel storing the new tokens + split reduce kernel",
+                    "fused_single": "pa_decode_append: single-pass decode kernel storing the new tokens",
+                    "split": "pa_decode_split_reduce: decode partition kernel + split reduce kernel",
+                    "single": "pa_decode: single-pass decode kernel"}[args.mode],
                 "peak_source": f"{peak_kind} HBM copy bandwidth (MEASURED_PEAKS.json hbm_gbs)"
                 if peak_kind == "measured" else "fallback 6.65 TB/s",
                 "algorithmic_bytes_per_launch": attn_bytes,
@@ -431,7 +444,7 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--config", type=int, default=2, choices=(1, 2, 3, 4, 5))
-    ap.add_argument("--mode", choices=("split", "single"), default="split")
+    ap.add_argument("--mode", choices=("fused", "fused_single", "split", "single"), default="fused")
     ap.add_argument("--partition", type=int, default=512)
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")

@@ -148,6 +148,37 @@ pa_status pa_decode(void *out, const void *q, const void *k_cache, const void *v
                     void *stream);
 
 /*
+ * pa_decode_append -- one whole decode step: store every sequence's new token,
+ * then attend (slot mapping + cache write + decode [+ split-KV reduce]).
+ *
+ * Source: the decode form of the pages' step, "KV Cache 与 PageAttention深度
+ * 实战", §1.2: Output_t = Attention(Q_t, [K_prefix, K_t], [V_prefix, V_t]) --
+ * the new K_t / V_t join the cache ("vLLM推理引擎深度解析：PagedAttention与
+ * 连续批处理", §2.2) and take part in the same step's attention.
+ *
+ * For every sequence s with L = seq_lens[s] > 0 (L counts the new token), the
+ * rows k_new[s] / v_new[s] ([num_seqs, num_kv_heads, head_dim], q dtype) are
+ * stored at position L - 1, i.e. slot block_tables[s][(L-1)/16]*16 + (L-1)%16,
+ * exactly as pa_slot_mapping + pa_cache_write store them (same E4M3
+ * quantisation, same bits); then out is computed as by pa_decode
+ * (partition_size == 0: single pass, workspace unused and may be NULL) or by
+ * pa_decode_split_reduce (partition_size > 0: a positive multiple of 16,
+ * workspace as documented there).  The tensor-core kernel stores the new
+ * token from inside the attention launch, so the step is one launch (single
+ * pass) or two (split).  The pools are written: k_cache / v_cache are not
+ * const here.  Errors as for pa_decode_split_reduce; a new token whose table
+ * entry is out of range is not stored (PA_ERR_DEVICE_BOUNDS).
+ */
+pa_status pa_decode_append(void *out, const void *q, const void *k_new, const void *v_new,
+                           void *k_cache, void *v_cache, const int32_t *block_tables,
+                           int max_blocks_per_seq, const int32_t *seq_lens, int num_seqs,
+                           int num_q_heads, int num_kv_heads, int head_dim, int block_size,
+                           int num_blocks, float softmax_scale, pa_dtype q_dtype,
+                           pa_dtype kv_dtype, float k_scale, float v_scale, int partition_size,
+                           int max_seq_len, void *workspace, size_t workspace_bytes, int *dev_err,
+                           void *stream);
+
+/*
  * Workspace bytes pa_decode_split_reduce needs: with
  * NP = ceil(max_seq_len / partition_size) partitions,
  *   lse [num_seqs, num_q_heads, NP] fp32, then o [num_seqs, num_q_heads, NP, head_dim] fp32,

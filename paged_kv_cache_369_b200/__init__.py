@@ -34,6 +34,7 @@ PA_FP8_E4M3 = 2
 SYMBOLS = (
     "pa_status_string", "pa_version", "pa_slot_mapping", "pa_cache_write", "pa_decode",
     "pa_split_workspace_bytes", "pa_decode_split_reduce", "pa_decode_split_reduce_static_scratch",
+    "pa_decode_append",
 )
 
 PA_STATIC_SCRATCH_BYTES = 32 * 1024 * 1024
@@ -73,6 +74,9 @@ _lib.pa_split_workspace_bytes.argtypes = [_I, _I, _I, _I, _I]
 _lib.pa_decode_split_reduce.restype = _I
 _lib.pa_decode_split_reduce.argtypes = [_P, _P, _P, _P, _P, _I, _P, _I, _I, _I, _I, _I, _I, _F,
                                         _I, _I, _F, _F, _I, _I, _P, _S, _P, _P]
+_lib.pa_decode_append.restype = _I
+_lib.pa_decode_append.argtypes = [_P, _P, _P, _P, _P, _P, _P, _I, _P, _I, _I, _I, _I, _I, _I, _F,
+                                  _I, _I, _F, _F, _I, _I, _P, _S, _P, _P]
 _lib.pa_decode_split_reduce_static_scratch.restype = _I
 _lib.pa_decode_split_reduce_static_scratch.argtypes = [_P, _P, _P, _P, _P, _I, _P, _I, _I, _I, _I,
                                                        _I, _I, _F, _I, _I, _F, _F, _I, _I, _P, _P]
@@ -183,6 +187,24 @@ def pa_decode_split_reduce(out, q, k_cache, v_cache, block_tables, seq_lens,
                                        int(max_seq_len), _ptr(workspace), ws_bytes,
                                        _ptr(dev_err), _stream(stream)),
            "pa_decode_split_reduce")
+
+
+def pa_decode_append(out, q, k_new, v_new, k_cache, v_cache, block_tables, seq_lens,
+                     softmax_scale: float, partition_size: int, max_seq_len: int, workspace=None,
+                     k_scale: float = 1.0, v_scale: float = 1.0, dev_err=None,
+                     stream=None) -> None:
+    """One decode step: store each sequence's new token, then attend
+    (partition_size 0: single pass; > 0: split-KV with ``workspace``)."""
+    S, Hq, d = (int(x) for x in q.shape)
+    nb, Hk, B, _ = (int(x) for x in k_cache.shape)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(_lib.pa_decode_append(_ptr(out), _ptr(q), _ptr(k_new), _ptr(v_new), _ptr(k_cache),
+                                 _ptr(v_cache), _ptr(block_tables), int(block_tables.shape[1]),
+                                 _ptr(seq_lens), S, Hq, Hk, d, B, nb, float(softmax_scale),
+                                 dtype_code(q.dtype), dtype_code(k_cache.dtype), float(k_scale),
+                                 float(v_scale), int(partition_size), int(max_seq_len),
+                                 _ptr(workspace), ws_bytes, _ptr(dev_err), _stream(stream)),
+           "pa_decode_append")
 
 
 def split_workspace_views(workspace, num_seqs: int, num_q_heads: int, head_dim: int,

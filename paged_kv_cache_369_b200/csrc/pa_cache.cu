@@ -53,26 +53,6 @@ cudaError_t launch_slot_mapping(const SlotParams &p, cudaStream_t stream) {
 // handling the K and the V vector at the same position
 // ---------------------------------------------------------------------------
 
-// fp32 pair -> packed E4M3 pair (low byte = first element); round to nearest
-// even, saturating finite overflow to +-448.
-__device__ __forceinline__ uint16_t e4m3x2_rn_sat(float first, float second) {
-    uint16_t r;
-    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(second), "f"(first));
-    return r;
-}
-
-template <typename ACT>
-__device__ __forceinline__ uint2 quantise8(const uint4 &in, float scale) {
-    const uint32_t w[4] = {in.x, in.y, in.z, in.w};
-    float f[8];
-    Unpack<ACT, 8>::run(w, f);
-    uint16_t c[4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-        c[i] = e4m3x2_rn_sat(__fdiv_rn(f[2 * i], scale), __fdiv_rn(f[2 * i + 1], scale));
-    return make_uint2((uint32_t)c[0] | ((uint32_t)c[1] << 16), (uint32_t)c[2] | ((uint32_t)c[3] << 16));
-}
-
 template <typename ACT, bool FP8>
 __global__ void __launch_bounds__(256) cache_write_kernel(const CacheWriteParams p) {
     const int vecs_per_row = p.head_dim / 8;
@@ -123,6 +103,72 @@ cudaError_t launch_cache_write(const CacheWriteParams &p, DType act, DType kv, c
             cache_write_kernel<bf16_t, true><<<(unsigned)blocks, threads, 0, stream>>>(p);
         else
             cache_write_kernel<bf16_t, false><<<(unsigned)blocks, threads, 0, stream>>>(p);
+    }
+    return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// append: the decode form of slot mapping + cache write in one kernel.  The
+// new token of sequence s sits at position seq_lens[s] - 1; its slot is
+// computed inline (no slot array).  Used where the decode kernel does not
+// patch the new token itself.
+// ---------------------------------------------------------------------------
+
+template <typename ACT, bool FP8>
+__global__ void __launch_bounds__(256) append_kernel(const AppendParams p) {
+    const int vecs_per_row = p.head_dim / 8;
+    const int64_t per_seq = (int64_t)p.num_kv_heads * vecs_per_row;
+    const int64_t total = (int64_t)p.num_seqs * per_seq;
+    for (int64_t g = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; g < total;
+         g += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t s = g / per_seq;
+        const int64_t rem = g - s * per_seq;
+        const int64_t h = rem / vecs_per_row;
+        const int64_t c = rem - h * vecs_per_row;
+        const int L = p.seq_lens[s];
+        if (L <= 0) continue;  // an empty sequence has no new token
+        const bool first = h == 0 && c == 0;
+        const int64_t pos = L - 1;
+        if (pos >= (int64_t)p.max_blocks_per_seq * kBlockSize) {
+            if (first) flag_error(p.err, kErrBounds);
+            continue;
+        }
+        const int64_t phys = p.block_tables[s * p.max_blocks_per_seq + pos / kBlockSize];
+        if (phys < 0 || phys >= p.num_blocks) {
+            if (first) flag_error(p.err, kErrBounds);
+            continue;
+        }
+        const int64_t src = ((s * p.num_kv_heads + h) * p.head_dim + c * 8);
+        const int64_t dst = (((phys * p.num_kv_heads + h) * kBlockSize + pos % kBlockSize) * p.head_dim + c * 8);
+        const uint4 kin = *reinterpret_cast<const uint4 *>(static_cast<const uint16_t *>(p.k_new) + src);
+        const uint4 vin = *reinterpret_cast<const uint4 *>(static_cast<const uint16_t *>(p.v_new) + src);
+        if constexpr (FP8) {
+            *reinterpret_cast<uint2 *>(static_cast<uint8_t *>(p.k_cache) + dst) = quantise8<ACT>(kin, p.k_scale);
+            *reinterpret_cast<uint2 *>(static_cast<uint8_t *>(p.v_cache) + dst) = quantise8<ACT>(vin, p.v_scale);
+        } else {
+            *reinterpret_cast<uint4 *>(static_cast<uint16_t *>(p.k_cache) + dst) = kin;
+            *reinterpret_cast<uint4 *>(static_cast<uint16_t *>(p.v_cache) + dst) = vin;
+        }
+    }
+}
+
+cudaError_t launch_append(const AppendParams &p, DType act, DType kv, cudaStream_t stream) {
+    const int64_t total = (int64_t)p.num_seqs * p.num_kv_heads * (p.head_dim / 8);
+    if (total <= 0) return cudaSuccess;
+    const int threads = 256;
+    int64_t blocks = (total + threads - 1) / threads;
+    if (blocks > (1 << 20)) blocks = 1 << 20;
+    const bool fp8 = kv == DType::E4M3;
+    if (act == DType::F16) {
+        if (fp8)
+            append_kernel<f16_t, true><<<(unsigned)blocks, threads, 0, stream>>>(p);
+        else
+            append_kernel<f16_t, false><<<(unsigned)blocks, threads, 0, stream>>>(p);
+    } else {
+        if (fp8)
+            append_kernel<bf16_t, true><<<(unsigned)blocks, threads, 0, stream>>>(p);
+        else
+            append_kernel<bf16_t, false><<<(unsigned)blocks, threads, 0, stream>>>(p);
     }
     return cudaGetLastError();
 }

@@ -42,11 +42,34 @@ bool use_mma(pa_dtype kv, int head_dim, int num_blocks, int num_kv_heads) {
                                     num_blocks, num_kv_heads);
 }
 
-// Launch whichever decode kernel applies, with its own head grouping.
+// Launch whichever decode kernel applies, with its own head grouping.  With
+// p.append set, the tensor-core kernel stores the new tokens itself; the
+// CUDA-core route runs the fused append kernel first.
 cudaError_t launch_any_decode(pa::DecodeParams &p, pa_dtype q, pa_dtype kv, int head_dim,
                               cudaStream_t stream) {
     const int g = p.group;
-    if (use_mma(kv, head_dim, p.num_blocks, p.num_kv_heads)) {
+    const bool mma = use_mma(kv, head_dim, p.num_blocks, p.num_kv_heads);
+    if (p.append && !mma) {
+        pa::AppendParams a = {};
+        a.k_new = p.k_new;
+        a.v_new = p.v_new;
+        a.k_cache = p.k_pool_w;
+        a.v_cache = p.v_pool_w;
+        a.block_tables = p.block_tables;
+        a.seq_lens = p.seq_lens;
+        a.err = p.err;
+        a.max_blocks_per_seq = p.max_blocks_per_seq;
+        a.num_seqs = p.num_seqs;
+        a.num_kv_heads = p.num_kv_heads;
+        a.head_dim = head_dim;
+        a.num_blocks = p.num_blocks;
+        a.k_scale = p.k_scale_w;
+        a.v_scale = p.v_scale_w;
+        const cudaError_t e = pa::launch_append(a, to_internal(q), to_internal(kv), stream);
+        if (e != cudaSuccess) return e;
+        p.append = 0;
+    }
+    if (mma) {
         const int rows = g <= 8 ? 8 : 16;
         p.head_groups = (g + rows - 1) / rows;
         return pa::launch_decode_mma(p, to_internal(q), to_internal(kv), head_dim, rows, stream);
@@ -223,6 +246,67 @@ pa_status pa_decode(void *out, const void *q, const void *k_cache, const void *v
     p.num_partitions = 1;
     p.split = 0;
     return from_cuda(launch_any_decode(p, q_dtype, kv_dtype, head_dim, static_cast<cudaStream_t>(stream)));
+}
+
+pa_status pa_decode_append(void *out, const void *q, const void *k_new, const void *v_new,
+                           void *k_cache, void *v_cache, const int32_t *block_tables,
+                           int max_blocks_per_seq, const int32_t *seq_lens, int num_seqs,
+                           int num_q_heads, int num_kv_heads, int head_dim, int block_size,
+                           int num_blocks, float softmax_scale, pa_dtype q_dtype,
+                           pa_dtype kv_dtype, float k_scale, float v_scale, int partition_size,
+                           int max_seq_len, void *workspace, size_t workspace_bytes, int *dev_err,
+                           void *stream) {
+    const DecodeArgs a = {out, q, k_cache, v_cache, block_tables, max_blocks_per_seq, seq_lens,
+                          num_seqs, num_q_heads, num_kv_heads, head_dim, block_size, num_blocks,
+                          softmax_scale, q_dtype, kv_dtype, k_scale, v_scale};
+    pa_status st = check_decode(a);
+    if (st != PA_OK) return st;
+    if (partition_size < 0 || partition_size % pa::kBlockSize != 0 || max_seq_len < 0)
+        return PA_ERR_INVALID_ARG;
+    if (num_seqs == 0) return PA_OK;
+    if (!k_new || !v_new || !aligned16(k_new) || !aligned16(v_new)) return PA_ERR_INVALID_ARG;
+    const bool split = partition_size > 0;
+    int np = 1;
+    if (split) {
+        const size_t need = pa_split_workspace_bytes(num_seqs, num_q_heads, head_dim, max_seq_len,
+                                                     partition_size);
+        if (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+            return PA_ERR_INVALID_ARG;
+        np = max_seq_len > 0 ? (max_seq_len + partition_size - 1) / partition_size : 1;
+        if ((int64_t)num_seqs * np > 0x7FFFFFFF) return PA_ERR_UNSUPPORTED;
+    }
+    pa::DecodeParams p = make_decode_params(a, dev_err);
+    p.append = 1;
+    p.k_new = k_new;
+    p.v_new = v_new;
+    p.k_pool_w = static_cast<uint8_t *>(k_cache);
+    p.v_pool_w = static_cast<uint8_t *>(v_cache);
+    p.k_scale_w = kv_dtype == PA_FP8_E4M3 ? k_scale : 1.0f;
+    p.v_scale_w = kv_dtype == PA_FP8_E4M3 ? v_scale : 1.0f;
+    const cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (!split) {
+        p.partition_blocks = max_blocks_per_seq;
+        p.num_partitions = 1;
+        p.split = 0;
+        return from_cuda(launch_any_decode(p, q_dtype, kv_dtype, head_dim, s));
+    }
+    const size_t rows = (size_t)num_seqs * num_q_heads * np;
+    p.ws_lse = static_cast<float *>(workspace);
+    p.ws_o = reinterpret_cast<float *>(static_cast<uint8_t *>(workspace) + align256(rows * sizeof(float)));
+    p.partition_blocks = partition_size / pa::kBlockSize;
+    p.num_partitions = np;
+    p.split = 1;
+    if (launch_any_decode(p, q_dtype, kv_dtype, head_dim, s) != cudaSuccess) return PA_ERR_CUDA;
+    pa::ReduceParams r = {};
+    r.out = out;
+    r.ws_lse = p.ws_lse;
+    r.ws_o = p.ws_o;
+    r.seq_lens = seq_lens;
+    r.num_seqs = num_seqs;
+    r.num_q_heads = num_q_heads;
+    r.num_partitions = np;
+    r.partition_size = partition_size;
+    return from_cuda(pa::launch_reduce(r, to_internal(q_dtype), head_dim, s));
 }
 
 size_t pa_split_workspace_bytes(int num_seqs, int num_q_heads, int head_dim, int max_seq_len,

@@ -398,11 +398,16 @@ __global__ void __launch_bounds__(kDecodeWarps * 32)
 }
 
 // ---------------------------------------------------------------------------
-// split-KV reduce: one CTA per (sequence, query head), one thread per element
+// split-KV reduce: one CTA per (sequence, query head), one thread per element.
+// The partition weights w_p = exp(lse_p - M) are computed once per chunk of
+// up to D partitions into shared memory; the weighted sum then issues
+// independent loads (no dependent-load chain across partitions).
 // ---------------------------------------------------------------------------
 
 template <typename QT, int D>
 __global__ void __launch_bounds__(D) reduce_kernel(const ReduceParams p) {
+    __shared__ float w_s[D];
+    __shared__ float red[D / 32];
     pdl_wait();
     const int64_t row = blockIdx.x;
     const int s = (int)(row / p.num_q_heads);
@@ -413,15 +418,41 @@ __global__ void __launch_bounds__(D) reduce_kernel(const ReduceParams p) {
     const int np = (L + p.partition_size - 1) / p.partition_size;
     const float *lse = p.ws_lse + row * NP;
     const float *o = p.ws_o + row * NP * D;
-    const int d = threadIdx.x;
-    float M = -CUDART_INF_F;
-    for (int i = 0; i < np; ++i) M = fmaxf(M, lse[i]);
+    const int d = threadIdx.x, lane = d & 31, wid = d >> 5;
+
+    // M = max_p lse_p
+    float m = -CUDART_INF_F;
+    for (int i = d; i < np; i += D) m = fmaxf(m, lse[i]);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, off));
+    if (lane == 0) red[wid] = m;
+    __syncthreads();
+    float M = red[0];
+#pragma unroll
+    for (int w = 1; w < D / 32; ++w) M = fmaxf(M, red[w]);
+
     float num = 0.f, den = 0.f;
     if (M != -CUDART_INF_F) {
-        for (int i = 0; i < np; ++i) {
-            const float w = expf(lse[i] - M);
-            den += w;
-            num = fmaf(w, o[(int64_t)i * D + d], num);
+        for (int base = 0; base < np; base += D) {
+            const int n = np - base < D ? np - base : D;
+            __syncthreads();  // previous chunk's weights are consumed
+            if (d < n) w_s[d] = expf(lse[base + d] - M);
+            __syncthreads();
+            const float *ob = o + (int64_t)base * D + d;
+            int i = 0;
+            for (; i + 4 <= n; i += 4) {
+                const float o0 = ob[(int64_t)i * D], o1 = ob[(int64_t)(i + 1) * D];
+                const float o2 = ob[(int64_t)(i + 2) * D], o3 = ob[(int64_t)(i + 3) * D];
+                num = fmaf(w_s[i], o0, num);
+                num = fmaf(w_s[i + 1], o1, num);
+                num = fmaf(w_s[i + 2], o2, num);
+                num = fmaf(w_s[i + 3], o3, num);
+                den += (w_s[i] + w_s[i + 1]) + (w_s[i + 2] + w_s[i + 3]);
+            }
+            for (; i < n; ++i) {
+                num = fmaf(w_s[i], ob[(int64_t)i * D], num);
+                den += w_s[i];
+            }
         }
     }
     const float r = den > 0.f ? num / den : 0.f;

@@ -193,6 +193,7 @@ __global__ void __launch_bounds__(kDecodeWarps * 32)
             L = cap;
         }
     }
+    const bool len_ok = L == p.seq_lens[s];  // not clamped: the new token's slot is known
     const int nblk_seq = (L + kBlockSize - 1) / kBlockSize;
     const int blk_begin = part * p.partition_blocks;
     int blk_end = blk_begin + p.partition_blocks;
@@ -349,6 +350,43 @@ __global__ void __launch_bounds__(kDecodeWarps * 32)
         nvalid = valid ? (nvalid < kBlockSize ? nvalid : kBlockSize) : 0;
         const uint32_t kt = stage0 + st * C::STAGE_BYTES;
         const uint32_t vt = kt + C::TILE_BYTES;
+
+        // append: the warp holding the sequence's last block writes this step's
+        // new token (position L - 1) into its landed tile and, once per KV head,
+        // into the pool -- the slot mapping and cache write of the step fused
+        // here.  E4M3 codes come from the same quantiser as pa_cache_write.
+        if (p.append && len_ok && valid && j == (L - 1) / kBlockSize) {
+            const int r = (L - 1) & (kBlockSize - 1);
+            const int64_t phys = bt_of(k);
+            constexpr int CPR = C::ROW_BYTES / 16;        // 16-byte chunks per tile row
+            constexpr int SRC_ELEMS = C::FP8 ? 16 : 8;    // activations per chunk
+            const int64_t src_row = ((int64_t)s * p.num_kv_heads + kvh) * D;
+            const int64_t dst_row = ((phys * p.num_kv_heads + kvh) * kBlockSize + r) * C::ROW_BYTES;
+            for (int c = lane; c < 2 * CPR; c += 32) {
+                const bool isv = c >= CPR;
+                const int cc = isv ? c - CPR : c;
+                const uint16_t *src =
+                    static_cast<const uint16_t *>(isv ? p.v_new : p.k_new) + src_row + cc * SRC_ELEMS;
+                uint4 val;
+                if constexpr (C::FP8) {
+                    const float sc = isv ? p.v_scale_w : p.k_scale_w;
+                    const uint2 lo = quantise8<QT>(*reinterpret_cast<const uint4 *>(src), sc);
+                    const uint2 hi = quantise8<QT>(*reinterpret_cast<const uint4 *>(src + 8), sc);
+                    val = make_uint4(lo.x, lo.y, hi.x, hi.y);
+                } else {
+                    val = *reinterpret_cast<const uint4 *>(src);
+                }
+                const uint32_t dst = (isv ? vt : kt) + swz(r, cc);
+                asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(val.x),
+                             "r"(val.y), "r"(val.z), "r"(val.w)
+                             : "memory");
+                if (hg == 0)
+                    *reinterpret_cast<uint4 *>((isv ? p.v_pool_w : p.k_pool_w) + dst_row + cc * 16) = val;
+            }
+            // these generic writes precede the next TMA write into this stage
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            __syncwarp();
+        }
 
         // S = Q K^T for the block's 16 tokens (two n-tiles of 8)
         float sc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};

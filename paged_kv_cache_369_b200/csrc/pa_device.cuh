@@ -98,6 +98,31 @@ __device__ __forceinline__ uint16_t from_float(bf16_t, float x) {
 }
 
 // ---------------------------------------------------------------------------
+// E4M3 quantisation of the cache write (shared by every path that stores
+// E4M3 codes, so they agree bit for bit): x / scale in fp32 with IEEE
+// division, then round to nearest even onto E4M3, saturating to +-448.
+// ---------------------------------------------------------------------------
+
+__device__ __forceinline__ uint16_t e4m3x2_rn_sat(float first, float second) {
+    uint16_t r;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(second), "f"(first));
+    return r;
+}
+
+// eight 16-bit activations (one uint4) -> eight E4M3 codes (one uint2)
+template <typename ACT>
+__device__ __forceinline__ uint2 quantise8(const uint4 &in, float scale) {
+    const uint32_t w[4] = {in.x, in.y, in.z, in.w};
+    float f[8];
+    Unpack<ACT, 8>::run(w, f);
+    uint16_t c[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+        c[i] = e4m3x2_rn_sat(__fdiv_rn(f[2 * i], scale), __fdiv_rn(f[2 * i + 1], scale));
+    return make_uint2((uint32_t)c[0] | ((uint32_t)c[1] << 16), (uint32_t)c[2] | ((uint32_t)c[3] << 16));
+}
+
+// ---------------------------------------------------------------------------
 // shared-memory loads of 2 / 4 / 8 / 16 bytes into 32-bit words
 // ---------------------------------------------------------------------------
 

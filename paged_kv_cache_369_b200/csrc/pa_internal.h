@@ -68,6 +68,32 @@ struct DecodeParams {
     int split;                  // 1: write partials to the workspace
     float qk_scale_log2;        // softmax_scale * k_scale * log2(e)
     float v_scale;              // applied to the output (1 for 16-bit caches)
+    // append (pa_decode_append): this step's new token of every sequence,
+    // stored at position seq_len - 1 before it is attended
+    int append;
+    const void *k_new;          // [S, Hk, D] activation dtype
+    const void *v_new;
+    uint8_t *k_pool_w;          // the pools again, writable
+    uint8_t *v_pool_w;
+    float k_scale_w;            // E4M3 quantisation scales (1 for 16-bit caches)
+    float v_scale_w;
+};
+
+struct AppendParams {  // decode-form slot mapping + cache write in one kernel
+    const void *k_new;
+    const void *v_new;
+    void *k_cache;
+    void *v_cache;
+    const int32_t *block_tables;
+    const int32_t *seq_lens;
+    int *err;
+    int max_blocks_per_seq;
+    int num_seqs;
+    int num_kv_heads;
+    int head_dim;
+    int num_blocks;
+    float k_scale;
+    float v_scale;
 };
 
 struct ReduceParams {
@@ -83,6 +109,7 @@ struct ReduceParams {
 
 // Launchers: return cudaSuccess or the launch error.
 cudaError_t launch_slot_mapping(const SlotParams &p, cudaStream_t stream);
+cudaError_t launch_append(const AppendParams &p, DType act, DType kv, cudaStream_t stream);
 cudaError_t launch_cache_write(const CacheWriteParams &p, DType act, DType kv, cudaStream_t stream);
 cudaError_t launch_decode(const DecodeParams &p, DType q, DType kv, int head_dim, int tpl_group,
                           cudaStream_t stream);

@@ -19,8 +19,8 @@ from typing import Optional
 import numpy as np
 import torch
 
-from . import (pa_cache_write, pa_decode, pa_decode_split_reduce, pa_slot_mapping,
-               pa_split_workspace_bytes)
+from . import (pa_cache_write, pa_decode, pa_decode_append, pa_decode_split_reduce,
+               pa_slot_mapping, pa_split_workspace_bytes)
 
 _TORCH_ACT = {"f16": torch.float16, "bf16": torch.bfloat16}
 _UPLOAD_CHUNK_TOKENS = 1 << 16
@@ -36,7 +36,7 @@ class PagedDecode:
 
     def __init__(self, w, device: str = "cuda", mode: str = "split", partition_size: int = 512,
                  prefill: bool = True, stream: Optional[torch.cuda.Stream] = None):
-        if mode not in ("split", "single"):
+        if mode not in ("split", "single", "fused", "fused_single"):
             raise ValueError(mode)
         self.w = w
         self.device = torch.device(device)
@@ -109,13 +109,28 @@ class PagedDecode:
                                    self.partition_size, self.max_seq_len, self.workspace,
                                    w.k_scale, w.v_scale, self.dev_err, self.stream)
 
+    def fused_step(self) -> None:
+        """One decode step through pa_decode_append: the new tokens are stored
+        by the attention launch itself."""
+        w = self.w
+        P = 0 if self.mode == "fused_single" else self.partition_size
+        pa_decode_append(self.out, self.q, self.k_new, self.v_new, self.k_cache, self.v_cache,
+                         self.block_tables, self.seq_lens, w.softmax_scale, P, self.max_seq_len,
+                         self.workspace if P else None, w.k_scale, w.v_scale, self.dev_err,
+                         self.stream)
+
     def step(self) -> None:
         """One decode step: slot mapping, cache write, attention."""
+        if self.mode.startswith("fused"):
+            self.fused_step()
+            return
         self.write_new()
         self.attend()
 
     def launches_per_step(self) -> int:
-        return 2 + (1 if self.mode == "single" else 2)
+        """Kernel launches of one step (the tensor-core route; the CUDA-core
+        route of a fused step adds one append launch)."""
+        return {"single": 3, "split": 4, "fused": 2, "fused_single": 1}[self.mode]
 
     def error(self) -> int:
         return int(self.dev_err.item())

@@ -144,3 +144,19 @@ def test_cache_write_and_slot_checks(pa):
     assert sm(sl=None) == 1           # decode form needs seq_lens
     assert sm(T=3, S=2) == 1          # token t is sequence t: T <= S
     assert sm(T=0, out=0) == 0
+
+
+def test_decode_append_checks(pa):
+    L = pa.lib()
+
+    def call(kn=A, vn=A, P=512, ws=A, wsb=1 << 30, maxlen=1000, S=2):
+        return L.pa_decode_append(A, A, kn, vn, A, A, A, 4, A, S, 8, 2, 128, 16, 10, 0.1,
+                                  pa.PA_BF16, pa.PA_BF16, 1.0, 1.0, P, maxlen, ws, wsb, None, None)
+
+    assert call(kn=0) == 1            # new rows required
+    assert call(vn=A + 8) == 1        # misaligned
+    assert call(P=24) == 1            # partition not a multiple of 16
+    assert call(P=-16) == 1
+    assert call(ws=0) == 1            # split needs a workspace
+    assert call(wsb=16) == 1
+    assert call(S=0, kn=0) == 0       # empty batch

@@ -97,7 +97,8 @@ def kernel_choice(request, monkeypatch):
     return request.param
 
 
-@pytest.mark.parametrize("mode,P", [("single", 512), ("split", 512), ("split", 16), ("split", 64)])
+@pytest.mark.parametrize("mode,P", [("single", 512), ("split", 512), ("split", 16), ("split", 64),
+                                    ("fused", 512), ("fused", 16), ("fused_single", 512)])
 @pytest.mark.parametrize("case", range(len(SMALL)))
 def test_small_full_parity(case, mode, P, kernel_choice):
     pa, PagedDecode = _pa()
@@ -206,8 +207,8 @@ def _full(cfg):
 def test_named_workload_parity(cfg):
     pa, PagedDecode = _pa()
     w, kc, vc = _full(cfg)
-    dec = PagedDecode(w, mode="split", partition_size=512)
-    dec.step()
+    dec = PagedDecode(w, mode="fused", partition_size=512)
+    dec.step()  # pa_decode_append: the attention launch stores the new tokens
     torch.cuda.synchronize()
     assert dec.error() == 0
     check_pools(dec, kc, vc)
@@ -215,7 +216,12 @@ def test_named_workload_parity(cfg):
     assert np.isfinite(out_split).all()
     pairs = sample_pairs(w, 64 if cfg > 1 else w.num_seqs * w.num_q_heads, seed=cfg)
     ref = oracle.decode_for(w, kc, vc, pairs)
-    assert_close(out_split[pairs[:, 0], pairs[:, 1]], ref, f"config {cfg} split")
+    assert_close(out_split[pairs[:, 0], pairs[:, 1]], ref, f"config {cfg} fused split")
+    # unfused split attention on the same state
+    dec.mode = "split"
+    dec.attend()
+    torch.cuda.synchronize()
+    assert_close(_to_f64(dec.out)[pairs[:, 0], pairs[:, 1]], ref, f"config {cfg} split")
     # single-pass launch on the same state
     dec.mode = "single"
     dec.attend()
