@@ -130,7 +130,8 @@ template <typename QT, typename KVT, int D, int GT> struct MmaCfg {
     static constexpr int STAGE_BYTES = 2 * TILE_BYTES;
     static constexpr int NST = (16384 / STAGE_BYTES) < 2 ? 2 : (16384 / STAGE_BYTES);
     static constexpr int KS = D / 16;   // k-steps of q.K
-    static constexpr int NT = D / 8;    // n-tiles of P.V
+    static constexpr int MT = D / 16;   // m-tiles (16 rows of d) of O^T = V^T P^T
+    static constexpr int NH = GT / 8;   // n-tiles (8 heads) of O^T
     static constexpr int SZ_STAGES = NW * NST * STAGE_BYTES;
     static constexpr int OFF_BAR = SZ_STAGES;
     static constexpr int SMEM = 1024 /* alignment slack */ + OFF_BAR + NW * NST * 8;
@@ -147,7 +148,7 @@ __device__ __forceinline__ uint32_t swz(int r, int c) {
 }
 
 template <typename QT, typename KVT, int D, int GT>
-__global__ void __launch_bounds__(kDecodeWarps * 32)
+__global__ void __launch_bounds__(kDecodeWarps * 32, 3)
     decode_mma_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmap_k,
                       const __grid_constant__ CUtensorMap tmap_v) {
     using C = MmaCfg<QT, KVT, D, GT>;
@@ -312,16 +313,20 @@ __global__ void __launch_bounds__(kDecodeWarps * 32)
     // ---- main loop ------------------------------------------------------------
     constexpr int NR = GT / 8;  // accumulator rows a lane owns: g (and g+8)
     float m_run[NR], l_run[NR];
-    float o[C::NT][4];
+    // O^T accumulators: o[mt][nh] = rows (d) of m-tile mt x heads 8nh..8nh+7;
+    // c0, c1: d-row g, heads 2kq, 2kq+1; c2, c3: d-row g+8, same heads
+    float o[C::MT][C::NH][4];
 #pragma unroll
     for (int r = 0; r < NR; ++r) {
         m_run[r] = -CUDART_INF_F;
         l_run[r] = 0.f;
     }
 #pragma unroll
-    for (int n = 0; n < C::NT; ++n)
+    for (int mt = 0; mt < C::MT; ++mt)
 #pragma unroll
-        for (int i = 0; i < 4; ++i) o[n][i] = 0.f;
+        for (int nh = 0; nh < C::NH; ++nh)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) o[mt][nh][i] = 0.f;
 
     // per-lane ldmatrix row / chunk selectors
     const int lrow_b = (lane & 7) + 8 * (lane >> 4);   // q.K: tokens 0-7 | 8-15
@@ -438,79 +443,84 @@ __global__ void __launch_bounds__(kDecodeWarps * 32)
             l_run[r] = l_run[r] * alpha[r] + ((pr[r][0] + pr[r][1]) + (pr[r][2] + pr[r][3]));
             m_run[r] = m_new;
         }
+        // the O^T columns this lane holds are heads 8nh + 2kq (+1); their
+        // rescale factors live in the lanes whose softmax row is that head
 #pragma unroll
-        for (int n = 0; n < C::NT; ++n) {
-            o[n][0] *= alpha[0];
-            o[n][1] *= alpha[0];
-            if constexpr (NR == 2) {
-                o[n][2] *= alpha[1];
-                o[n][3] *= alpha[1];
+        for (int nh = 0; nh < C::NH; ++nh) {
+            const float a0 = __shfl_sync(kFull, alpha[nh], (2 * kq) * 4);
+            const float a1 = __shfl_sync(kFull, alpha[nh], (2 * kq + 1) * 4);
+#pragma unroll
+            for (int mt = 0; mt < C::MT; ++mt) {
+                o[mt][nh][0] *= a0;
+                o[mt][nh][1] *= a1;
+                o[mt][nh][2] *= a0;
+                o[mt][nh][3] *= a1;
             }
         }
 
-        // P as A fragments (k = tokens), hi and (bf16 cache) lo parts
-        uint32_t pa_hi[4], pa_lo[4];
-        {
-            const float r1_0 = NR == 2 ? pr[NR - 1][0] : 0.f, r1_1 = NR == 2 ? pr[NR - 1][1] : 0.f;
-            const float r1_2 = NR == 2 ? pr[NR - 1][2] : 0.f, r1_3 = NR == 2 ? pr[NR - 1][3] : 0.f;
-            pa_hi[0] = pack2(pr[0][0], pr[0][1], ET{});
-            pa_hi[1] = pack2(r1_0, r1_1, ET{});
-            pa_hi[2] = pack2(pr[0][2], pr[0][3], ET{});
-            pa_hi[3] = pack2(r1_2, r1_3, ET{});
-            if constexpr (C::HILO) {
-                const float vals[4][2] = {{pr[0][0], pr[0][1]}, {r1_0, r1_1}, {pr[0][2], pr[0][3]}, {r1_2, r1_3}};
+        // P as B fragments of O^T = V^T P^T (k = tokens, n = heads): the S
+        // accumulators already sit in that layout -- b0 = tokens 2kq, 2kq+1,
+        // b1 = tokens 8+2kq, 9+2kq of head (8nh + g).  bf16 caches get a hi
+        // and a lo part.
+        uint32_t pb_hi[C::NH][2], pb_lo[C::NH][2];
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const float h0 = __uint_as_float(pa_hi[i] << 16);
-                    const float h1 = __uint_as_float(pa_hi[i] & 0xFFFF0000u);
-                    pa_lo[i] = pack2(vals[i][0] - h0, vals[i][1] - h1, ET{});
+        for (int nh = 0; nh < C::NH; ++nh) {
+            pb_hi[nh][0] = pack2(pr[nh][0], pr[nh][1], ET{});
+            pb_hi[nh][1] = pack2(pr[nh][2], pr[nh][3], ET{});
+            if constexpr (C::HILO) {
+#pragma unroll
+                for (int i = 0; i < 2; ++i) {
+                    const float h0 = __uint_as_float(pb_hi[nh][i] << 16);
+                    const float h1 = __uint_as_float(pb_hi[nh][i] & 0xFFFF0000u);
+                    pb_lo[nh][i] = pack2(pr[nh][2 * i] - h0, pr[nh][2 * i + 1] - h1, ET{});
                 }
             }
         }
 
-        // O += P V; tokens past nvalid have p = 0 but their V rows may hold
-        // NaN poison (0 * NaN = NaN): zero those V fragments first
+        // O^T += V^T P^T; tokens past nvalid have p = 0 but their V rows may
+        // hold NaN poison (0 * NaN = NaN): zero those V fragments first.
+        // A fragment of V^T: a0 = (d-row g, tokens 2kq, 2kq+1), a1 = (d-row g+8,
+        // same tokens), a2 / a3 = the same d-rows, tokens 8+2kq, 9+2kq.
         const bool full = nvalid == kBlockSize;
         const bool tv0 = t0 < nvalid, tv1 = t0 + 1 < nvalid, tv8 = t0 + 8 < nvalid, tv9 = t0 + 9 < nvalid;
+        const uint32_t m0 = (tv0 ? 0x0000FFFFu : 0u) | (tv1 ? 0xFFFF0000u : 0u);
+        const uint32_t m8 = (tv8 ? 0x0000FFFFu : 0u) | (tv9 ? 0xFFFF0000u : 0u);
         if constexpr (!C::FP8) {
+            // m-tile mt = d rows 16mt..16mt+15: ldmatrix.x4.trans of tokens
+            // 0-7 / 8-15 at chunks 2mt (d-rows 0-7) and 2mt+1 (d-rows 8-15)
 #pragma unroll
-            for (int cp = 0; cp < C::NT / 2; ++cp) {
-                uint32_t b[4];  // (nt 2cp: tok 0-7, tok 8-15), (nt 2cp+1: tok 0-7, tok 8-15)
-                ldsm_x4_t(b, vt + swz(lrow_v, 2 * cp + lsel_v));
+            for (int mt = 0; mt < C::MT; ++mt) {
+                uint32_t a[4];  // r0: tok 0-7 chunk 2mt, r1: tok 0-7 chunk 2mt+1, r2/r3: tok 8-15
+                ldsm_x4_t(a, vt + swz(lrow_b, 2 * mt + lsel_b));
+                uint32_t av[4] = {a[0], a[1], a[2], a[3]};
                 if (!full) {
-                    // b[0], b[2]: tokens 2kq, 2kq+1; b[1], b[3]: tokens 8+2kq, 9+2kq
-                    const uint32_t m0 = (tv0 ? 0x0000FFFFu : 0u) | (tv1 ? 0xFFFF0000u : 0u);
-                    const uint32_t m8 = (tv8 ? 0x0000FFFFu : 0u) | (tv9 ? 0xFFFF0000u : 0u);
-                    b[0] &= m0; b[2] &= m0; b[1] &= m8; b[3] &= m8;
+                    av[0] &= m0; av[1] &= m0; av[2] &= m8; av[3] &= m8;
                 }
-                mma16816(o[2 * cp], pa_hi, b[0], b[1], ET{});
-                mma16816(o[2 * cp + 1], pa_hi, b[2], b[3], ET{});
-                if constexpr (C::HILO) {
-                    mma16816(o[2 * cp], pa_lo, b[0], b[1], ET{});
-                    mma16816(o[2 * cp + 1], pa_lo, b[2], b[3], ET{});
+#pragma unroll
+                for (int nh = 0; nh < C::NH; ++nh) {
+                    mma16816(o[mt][nh], av, pb_hi[nh][0], pb_hi[nh][1], ET{});
+                    if constexpr (C::HILO) mma16816(o[mt][nh], av, pb_lo[nh][0], pb_lo[nh][1], ET{});
                 }
             }
         } else {
+            // m-tile mt = the 16 d of chunk mt: rows g / g+8 hold d = 16mt+2g
+            // and 16mt+2g+1 (byte regroup after the transposing load)
 #pragma unroll
-            for (int cp = 0; cp < C::NT / 4; ++cp) {
+            for (int cp = 0; cp < C::MT / 2; ++cp) {
                 uint32_t w[4];  // chunk 2cp: tok 0-7, tok 8-15; chunk 2cp+1: tok 0-7, tok 8-15
                 ldsm_x4_t(w, vt + swz(lrow_v, 2 * cp + lsel_v));
 #pragma unroll
                 for (int h = 0; h < 2; ++h) {
-                    // regroup bytes: low half = (tok 2kq, tok 2kq+1) at even d,
-                    // high half = same tokens at odd d
-                    const uint32_t lo_t = prmt(w[2 * h], 0x3120);
-                    const uint32_t hi_t = prmt(w[2 * h + 1], 0x3120);
-                    uint32_t be0 = e4m3x2_to_f16x2(lo_t), bo0 = e4m3x2_to_f16x2(lo_t >> 16);
-                    uint32_t be1 = e4m3x2_to_f16x2(hi_t), bo1 = e4m3x2_to_f16x2(hi_t >> 16);
+                    const uint32_t lo_t = prmt(w[2 * h], 0x3120);      // tokens 0-7
+                    const uint32_t hi_t = prmt(w[2 * h + 1], 0x3120);  // tokens 8-15
+                    uint32_t av[4] = {e4m3x2_to_f16x2(lo_t), e4m3x2_to_f16x2(lo_t >> 16),
+                                      e4m3x2_to_f16x2(hi_t), e4m3x2_to_f16x2(hi_t >> 16)};
                     if (!full) {
-                        const uint32_t m0 = (tv0 ? 0x0000FFFFu : 0u) | (tv1 ? 0xFFFF0000u : 0u);
-                        const uint32_t m8 = (tv8 ? 0x0000FFFFu : 0u) | (tv9 ? 0xFFFF0000u : 0u);
-                        be0 &= m0; bo0 &= m0; be1 &= m8; bo1 &= m8;
+                        av[0] &= m0; av[1] &= m0; av[2] &= m8; av[3] &= m8;
                     }
-                    const int c = 2 * cp + h;  // 16-element chunk of d
-                    mma16816(o[2 * c], pa_hi, be0, be1, ET{});      // even d of chunk c
-                    mma16816(o[2 * c + 1], pa_hi, bo0, bo1, ET{});  // odd d of chunk c
+                    const int mt = 2 * cp + h;
+#pragma unroll
+                    for (int nh = 0; nh < C::NH; ++nh) mma16816(o[mt][nh], av, pb_hi[nh][0], pb_hi[nh][1], ET{});
                 }
             }
         }
@@ -546,18 +556,20 @@ __global__ void __launch_bounds__(kDecodeWarps * 32)
         }
     }
 #pragma unroll
-    for (int n = 0; n < C::NT; ++n) {
+    for (int mt = 0; mt < C::MT; ++mt) {
 #pragma unroll
-        for (int r = 0; r < NR; ++r) {
+        for (int nh = 0; nh < C::NH; ++nh) {
 #pragma unroll
-            for (int ci = 0; ci < 2; ++ci) {
+            for (int i = 0; i < 4; ++i) {
+                const int head = 8 * nh + 2 * kq + (i & 1);
+                const int hi_row = i >> 1;  // 0: d-row g, 1: d-row g+8
                 int d;
                 if constexpr (C::FP8) {
-                    d = 16 * (n >> 1) + 4 * kq + 2 * ci + (n & 1);
+                    d = 16 * mt + 2 * g + hi_row;
                 } else {
-                    d = 8 * n + 2 * kq + ci;
+                    d = 16 * mt + 8 * hi_row + g;
                 }
-                accs[(warp * GT + g + 8 * r) * D + d] = o[n][2 * r + ci];
+                accs[(warp * GT + head) * D + d] = o[mt][nh][i];
             }
         }
     }
