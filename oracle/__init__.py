@@ -92,6 +92,8 @@ def lib() -> ctypes.CDLL:
                                          i32, i32, f64, i32, i32, P, i32]
         L.orc_split_merge.restype = None
         L.orc_split_merge.argtypes = [P, P, P, i32, i32]
+        L.orc_copy_blocks.restype = i32
+        L.orc_copy_blocks.argtypes = [P, P, P, i32, i32, i32, i32, i32, i32]
         _lib = L
     return _lib
 
@@ -178,6 +180,19 @@ def cache_write(k_new: np.ndarray, v_new: np.ndarray, k_cache: np.ndarray, v_cac
     if r < 0:
         raise ValueError("unsupported dtype pair")
     return int(r)
+
+
+def copy_blocks(k_cache: np.ndarray, v_cache: np.ndarray, pairs: np.ndarray) -> int:
+    """In-place copy-on-write block copy inside the numpy pools
+    [num_blocks, Hk, B, d]: block dst := block src for every (src, dst) row of
+    ``pairs``, in order.  Returns the number of pairs skipped for an
+    out-of-range id."""
+    assert k_cache.flags.c_contiguous and v_cache.flags.c_contiguous
+    assert k_cache.shape == v_cache.shape and k_cache.dtype == v_cache.dtype
+    nb, hk, bs, d = k_cache.shape
+    pr = _c(pairs, np.int32).reshape(-1, 2)
+    return int(lib().orc_copy_blocks(_p(k_cache), _p(v_cache), _p(pr), pr.shape[0], nb, hk, d,
+                                     bs, k_cache.dtype.itemsize))
 
 
 def empty_pool(num_blocks: int, num_kv_heads: int, block_size: int, head_dim: int, kv_dtype: str,

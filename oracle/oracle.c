@@ -16,7 +16,11 @@
  *     Attention(Q_t, [K_prefix, K_t], [V_prefix, V_t]):
  *     "KV Cache 与 PageAttention深度实战", §1.2;
  *   - fp8 E4M3 KV values (max 448): "大语言模型推理引擎深度剖析：从 KV Cache
- *     内存管理到 PagedAttention、投机解码与量化加速的完全工程指南", §4.2-§4.3.
+ *     内存管理到 PagedAttention、投机解码与量化加速的完全工程指南", §4.2-§4.3;
+ *   - copy-on-write of a shared block: first page §3.5 (a beam-search
+ *     candidate that diverges gets a new block for the diverging part only)
+ *     and the fifth page §2.3 (a request about to write into a shared block
+ *     copies it first, refcounts track the sharing).
  *
  * Paging changes only where K and V rows live, so the oracle gathers every
  * sequence's rows into contiguous fp64 arrays and then runs textbook two-pass
@@ -356,4 +360,35 @@ void orc_split_merge(double *out, const double *lse, const double *o, int num_pa
         for (int i = 0; i < head_dim; ++i) out[i] += w * o[(int64_t)p * head_dim + i];
     }
     for (int i = 0; i < head_dim; ++i) out[i] /= den;
+}
+
+/* ------------------------------------------------------------------------- */
+/* copy-on-write block copy                                                   */
+/* ------------------------------------------------------------------------- */
+
+/* Copy whole physical blocks inside both pools [num_blocks, Hk, B, d]: for
+ * each pair i, in order, block pairs[2i+1] of k_cache and of v_cache becomes
+ * a byte copy of block pairs[2i].  This is the copy step of copy-on-write
+ * (first page §3.5; fifth page §2.3): before a sequence writes into a block
+ * it shares with others, the block is duplicated into a free one and the
+ * sequence's table is pointed at the duplicate.  A pair with an id outside
+ * [0, num_blocks) is skipped and counted; the count is returned. */
+int orc_copy_blocks(void *k_cache, void *v_cache, const int32_t *pairs, int num_pairs,
+                    int num_blocks, int num_kv_heads, int head_dim, int block_size,
+                    int elem_bytes) {
+    int64_t block_bytes = (int64_t)num_kv_heads * block_size * head_dim * elem_bytes;
+    int bad = 0;
+    for (int i = 0; i < num_pairs; ++i) {
+        int32_t src = pairs[2 * i], dst = pairs[2 * i + 1];
+        if (src < 0 || src >= num_blocks || dst < 0 || dst >= num_blocks) {
+            ++bad;
+            continue;
+        }
+        for (int pool = 0; pool < 2; ++pool) {
+            uint8_t *base = (uint8_t *)(pool == 0 ? k_cache : v_cache);
+            for (int64_t b = 0; b < block_bytes; ++b)
+                base[(int64_t)dst * block_bytes + b] = base[(int64_t)src * block_bytes + b];
+        }
+    }
+    return bad;
 }

@@ -9,6 +9,7 @@ import numpy as np
 import pytest
 
 import oracle
+from tests import test_oracle_cow as cow
 from tests import test_oracle_pins as pins
 
 SRC = os.path.join(os.path.dirname(oracle.__file__), "oracle.c")
@@ -34,6 +35,12 @@ MUTANTS = {
     "f16_subnormal_exponent": ("v = ldexp((double)m, -24);", "v = ldexp((double)m, -25);"),
     "bf16_bias": ("v = ldexp((double)(128 + m), e - 134);", "v = ldexp((double)(128 + m), e - 133);"),
     "cache_write_skips_v": ("((uint16_t *)v_cache)[dst + i] = ((const uint16_t *)v_new)[src + i];", ""),
+    "copy_blocks_k_pool_only": ("for (int pool = 0; pool < 2; ++pool) {", "for (int pool = 0; pool < 1; ++pool) {"),
+    "copy_blocks_direction_swapped": (
+        "base[(int64_t)dst * block_bytes + b] = base[(int64_t)src * block_bytes + b];",
+        "base[(int64_t)src * block_bytes + b] = base[(int64_t)dst * block_bytes + b];"),
+    "copy_blocks_one_head": ("int64_t block_bytes = (int64_t)num_kv_heads * block_size * head_dim * elem_bytes;",
+                             "int64_t block_bytes = (int64_t)block_size * head_dim * elem_bytes;"),
 }
 
 
@@ -52,6 +59,9 @@ def _run_pins(golden_dir):
         ("closed", lambda: pins.test_closed_forms(oracle)),
         ("split", lambda: pins.test_split_equals_unsplit(oracle, 48)),
         ("roundtrip", lambda: pins.test_cache_write_then_gather_roundtrip(oracle)),
+        ("cow_example", lambda: cow.test_cow_beam_search_example(oracle, golden_dir)),
+        ("cow_brute", lambda: cow.test_copy_blocks_brute_force(oracle, "f16")),
+        ("cow_bounds", lambda: cow.test_copy_blocks_out_of_range_skipped(oracle)),
     ]
     for name, fn in checks:
         try:
