@@ -2,6 +2,7 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                     [--config 2] [--mode fused|fused_single|split|single] [--partition 512]
+    python bench.py --op copy_blocks [--config 2] [--pairs 4096]
 
 A step is one pass of the whole hot path over one batch: slot mapping of the
 new tokens, cache write of their K/V rows, and decode attention.  The default
@@ -276,6 +277,78 @@ def run_reference(args):
 
 
 # ---------------------------------------------------------------------------
+# copy-on-write block copy (pa_copy_blocks), one launch per step
+# ---------------------------------------------------------------------------
+
+def run_copy_blocks(args):
+    """Time pa_copy_blocks on the pool shape of a named workload: ``--pairs``
+    disjoint (src, dst) block pairs drawn from a seeded permutation, K and V
+    pools alike.  Algorithmic bytes: every copied byte read once and written
+    once."""
+    import torch
+
+    import workload
+    import paged_kv_cache_369_b200 as pa
+
+    world, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    w = workload.config(args.config, draw_kv=False)
+    dt = torch.uint8 if w.kv_dtype == "e4m3" else {"f16": torch.float16, "bf16": torch.bfloat16}[w.act_dtype]
+    shape = (w.num_blocks, w.num_kv_heads, w.block_size, w.head_dim)
+    kc = torch.empty(shape, dtype=dt, device=device)
+    vc = torch.empty(shape, dtype=dt, device=device)
+    kc.view(torch.uint8).fill_(0x3C)
+    vc.view(torch.uint8).fill_(0x3C)
+    n = min(args.pairs, w.num_blocks // 2)
+    perm = np.random.default_rng(w.seed).permutation(w.num_blocks)
+    pairs = torch.from_numpy(np.stack([perm[:n], perm[n:2 * n]], 1).astype(np.int32)).to(device)
+    err = torch.zeros(1, dtype=torch.int32, device=device)
+    block_bytes = w.num_kv_heads * w.block_size * w.head_dim * w.kv_elem_bytes()
+    moved = 2 * 2 * n * block_bytes  # K and V, read + write
+    stream = torch.cuda.Stream(device)
+    flush = None if moved > 256e6 else torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=device)
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            pa.pa_copy_blocks(kc, vc, pairs, err, stream)
+    torch.cuda.synchronize(device)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    clocks = ClockSampler(device.index or 0)
+    clocks.start()
+    with torch.cuda.stream(stream):
+        for a, b in ev:
+            a.record(stream)
+            pa.pa_copy_blocks(kc, vc, pairs, err, stream)
+            b.record(stream)
+            if flush is not None:
+                flush.fill_(1)
+    torch.cuda.synchronize(device)
+    clocks.stop()
+    ms = statistics.mean(a.elapsed_time(b) for a, b in ev)
+    value = moved / (ms * 1e-3) / 1e9
+    peak, peak_kind = measured_hbm_peak()
+    line = {
+        "metric": "pa_copy_blocks GB/s (copy-on-write block copy, read + write)",
+        "value": value, "unit": "GB/s", "n_gpus": 1, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": w.kv_dtype, "data": "synthetic pools, seeded block pairs",
+        "config": {"workload": f"copy {n} blocks of {block_bytes} B per pool ({w.name} pool shape)",
+                   "pairs": n, "block_bytes_per_pool": block_bytes, "num_blocks": w.num_blocks,
+                   "l2": "copied bytes larger than L2: no flush" if flush is None
+                   else "L2 flushed (256 MB write) between steps"},
+        "roofline": {"bound": "hbm", "achieved": value, "peak": peak, "unit": "GB/s",
+                     "frac": value / peak, "traffic": None,
+                     "kernel": "copy_blocks_kernel", "algorithmic_bytes_per_launch": moved,
+                     "peak_source": f"{peak_kind} HBM copy bandwidth"},
+        "gpu_launches": args.steps, "clocks": clocks.summary(),
+        "device_error": int(err.item()),
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------------------
 # the CUDA path
 # ---------------------------------------------------------------------------
 
@@ -448,11 +521,16 @@ def main(argv=None):
     ap.add_argument("--partition", type=int, default=512)
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--op", choices=("decode", "copy_blocks"), default="decode",
+                    help="decode: the decode step (default); copy_blocks: pa_copy_blocks alone")
+    ap.add_argument("--pairs", type=int, default=4096, help="block pairs for --op copy_blocks")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
     if args.impl == "reference":
         return run_reference(args)
+    if args.op == "copy_blocks":
+        return run_copy_blocks(args)
     return run_ours(args)
 
 

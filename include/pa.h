@@ -216,6 +216,31 @@ pa_status pa_decode_split_reduce(void *out, const void *q, const void *k_cache,
                                  void *workspace, size_t workspace_bytes, int *dev_err,
                                  void *stream);
 
+/*
+ * pa_copy_blocks -- copy whole KV blocks inside the pools (copy-on-write).
+ *
+ * Source: "Transformer 推理优化：KV Cache、PagedAttention 与 vLLM", §3.5 (beam
+ * search: candidates share their common blocks; only the block where they
+ * diverge is new) and "大语言模型推理引擎深度剖析", §2.3 (before a request
+ * writes into a block it shares, the engine copies the block; refcounts
+ * track the sharing).  The engine decides which blocks to copy and repoints
+ * its block tables; this call moves the bytes.
+ *
+ *   for every i < num_pairs, with (src, dst) = (block_pairs[2i], block_pairs[2i+1]):
+ *     k_cache[dst][:][:][:] = k_cache[src][:][:][:]   and likewise v_cache
+ *   (a block is num_kv_heads x block_size x head_dim elements of kv_dtype).
+ *
+ * block_pairs: device int32 [num_pairs][2].  The pairs are copied
+ * concurrently: no dst may appear twice or also be a src in the same call
+ * (then the result equals copying the pairs in order); src == dst is a
+ * no-op.  A pair with an id outside [0, num_blocks) is skipped and flags
+ * PA_ERR_DEVICE_BOUNDS in *dev_err.  k_cache / v_cache 16-byte aligned;
+ * kv_dtype PA_F16, PA_BF16 or PA_FP8_E4M3 (only its size matters).
+ */
+pa_status pa_copy_blocks(void *k_cache, void *v_cache, const int32_t *block_pairs, int num_pairs,
+                         int num_blocks, int num_kv_heads, int head_dim, int block_size,
+                         pa_dtype kv_dtype, int *dev_err, void *stream);
+
 /* Bytes of scratch built into the library for
  * pa_decode_split_reduce_static_scratch (32 MiB). */
 #define PA_STATIC_SCRATCH_BYTES (32u * 1024u * 1024u)

@@ -34,7 +34,7 @@ PA_FP8_E4M3 = 2
 SYMBOLS = (
     "pa_status_string", "pa_version", "pa_slot_mapping", "pa_cache_write", "pa_decode",
     "pa_split_workspace_bytes", "pa_decode_split_reduce", "pa_decode_split_reduce_static_scratch",
-    "pa_decode_append",
+    "pa_decode_append", "pa_copy_blocks",
 )
 
 PA_STATIC_SCRATCH_BYTES = 32 * 1024 * 1024
@@ -80,6 +80,8 @@ _lib.pa_decode_append.argtypes = [_P, _P, _P, _P, _P, _P, _P, _I, _P, _I, _I, _I
 _lib.pa_decode_split_reduce_static_scratch.restype = _I
 _lib.pa_decode_split_reduce_static_scratch.argtypes = [_P, _P, _P, _P, _P, _I, _P, _I, _I, _I, _I,
                                                        _I, _I, _F, _I, _I, _F, _F, _I, _I, _P, _P]
+_lib.pa_copy_blocks.restype = _I
+_lib.pa_copy_blocks.argtypes = [_P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P]
 
 
 def lib() -> ctypes.CDLL:
@@ -237,3 +239,13 @@ def pa_decode_split_reduce_static_scratch(out, q, k_cache, v_cache, block_tables
         dtype_code(q.dtype), dtype_code(k_cache.dtype), float(k_scale), float(v_scale),
         int(partition_size), int(max_seq_len), _ptr(dev_err), _stream(stream)),
         "pa_decode_split_reduce_static_scratch")
+
+
+def pa_copy_blocks(k_cache, v_cache, block_pairs, dev_err=None, stream=None) -> None:
+    """Copy-on-write block copy: block dst := block src in both pools for
+    every (src, dst) row of ``block_pairs`` (device int32 [n, 2])."""
+    nb, Hk, B, d = (int(x) for x in k_cache.shape)
+    n = int(block_pairs.shape[0]) if block_pairs is not None else 0
+    _check(_lib.pa_copy_blocks(_ptr(k_cache), _ptr(v_cache), _ptr(block_pairs), n, nb, Hk, d, B,
+                               dtype_code(k_cache.dtype), _ptr(dev_err), _stream(stream)),
+           "pa_copy_blocks")

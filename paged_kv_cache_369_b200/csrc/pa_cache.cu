@@ -9,6 +9,13 @@
 //
 // Both kernels are HBM-trivial next to attention (a few MB per step); they are
 // written for full 16-byte vector traffic and a grid of whole waves.
+//
+// Copy-on-write: before a sequence writes into a block it shares with other
+// sequences (a beam-search fork, a shared prompt prefix), the engine copies
+// that block into a free one and repoints the sequence's table entry
+// ("Transformer 推理优化：KV Cache、PagedAttention 与 vLLM", §3.5; "大语言模型推理
+// 引擎深度剖析", §2.3).  copy_blocks_kernel does the copy for a batch of
+// (src, dst) pairs, K and V pools alike.
 #include "pa_device.cuh"
 
 namespace pa {
@@ -170,6 +177,53 @@ cudaError_t launch_append(const AppendParams &p, DType act, DType kv, cudaStream
         else
             append_kernel<bf16_t, false><<<(unsigned)blocks, threads, 0, stream>>>(p);
     }
+    return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// copy-on-write block copy: grid (pair, stripe, pool); a block is one
+// contiguous span of block_bytes in each pool, copied with 16-byte vectors,
+// kCopyUnroll loads in flight per thread before the stores
+// ---------------------------------------------------------------------------
+
+constexpr int kCopyThreads = 256;
+constexpr int kCopyUnroll = 4;
+
+__global__ void __launch_bounds__(kCopyThreads) copy_blocks_kernel(const CopyBlocksParams p) {
+    const int64_t pair = blockIdx.x;
+    const int src = p.pairs[2 * pair], dst = p.pairs[2 * pair + 1];
+    if ((unsigned)src >= (unsigned)p.num_blocks || (unsigned)dst >= (unsigned)p.num_blocks) {
+        if (threadIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0) flag_error(p.err, kErrBounds);
+        return;
+    }
+    if (src == dst) return;
+    uint8_t *pool = blockIdx.z ? p.v_cache : p.k_cache;
+    const uint4 *from = reinterpret_cast<const uint4 *>(pool + (int64_t)src * p.block_bytes);
+    uint4 *to = reinterpret_cast<uint4 *>(pool + (int64_t)dst * p.block_bytes);
+    const int64_t nv = p.block_bytes / 16;
+    const int64_t step = (int64_t)gridDim.y * kCopyThreads * kCopyUnroll;
+    for (int64_t base = (int64_t)blockIdx.y * kCopyThreads * kCopyUnroll + threadIdx.x; base < nv;
+         base += step) {
+        uint4 r[kCopyUnroll];
+#pragma unroll
+        for (int u = 0; u < kCopyUnroll; ++u) {
+            const int64_t i = base + (int64_t)u * kCopyThreads;
+            if (i < nv) r[u] = from[i];
+        }
+#pragma unroll
+        for (int u = 0; u < kCopyUnroll; ++u) {
+            const int64_t i = base + (int64_t)u * kCopyThreads;
+            if (i < nv) to[i] = r[u];
+        }
+    }
+}
+
+cudaError_t launch_copy_blocks(const CopyBlocksParams &p, cudaStream_t stream) {
+    if (p.num_pairs <= 0 || p.block_bytes <= 0) return cudaSuccess;
+    const int64_t per_cta = (int64_t)kCopyThreads * kCopyUnroll * 16;
+    int64_t stripes = (p.block_bytes + per_cta - 1) / per_cta;
+    if (stripes > 65535) stripes = 65535;
+    copy_blocks_kernel<<<dim3((unsigned)p.num_pairs, (unsigned)stripes, 2), kCopyThreads, 0, stream>>>(p);
     return cudaGetLastError();
 }
 

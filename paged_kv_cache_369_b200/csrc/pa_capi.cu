@@ -309,6 +309,30 @@ pa_status pa_decode_append(void *out, const void *q, const void *k_new, const vo
     return from_cuda(pa::launch_reduce(r, to_internal(q_dtype), head_dim, s));
 }
 
+pa_status pa_copy_blocks(void *k_cache, void *v_cache, const int32_t *block_pairs, int num_pairs,
+                         int num_blocks, int num_kv_heads, int head_dim, int block_size,
+                         pa_dtype kv_dtype, int *dev_err, void *stream) {
+    if (num_pairs < 0 || num_blocks <= 0 || num_kv_heads <= 0 || head_dim <= 0 || block_size <= 0)
+        return PA_ERR_INVALID_ARG;
+    if (kv_dtype != PA_F16 && kv_dtype != PA_BF16 && kv_dtype != PA_FP8_E4M3)
+        return PA_ERR_UNSUPPORTED;
+    const int64_t elem = kv_dtype == PA_FP8_E4M3 ? 1 : 2;
+    const int64_t block_bytes = (int64_t)num_kv_heads * block_size * head_dim * elem;
+    if (block_bytes % 16 != 0) return PA_ERR_UNSUPPORTED;
+    if (num_pairs == 0) return PA_OK;
+    if (!k_cache || !v_cache || !block_pairs) return PA_ERR_INVALID_ARG;
+    if (!aligned16(k_cache) || !aligned16(v_cache)) return PA_ERR_INVALID_ARG;
+    pa::CopyBlocksParams p = {};
+    p.k_cache = static_cast<uint8_t *>(k_cache);
+    p.v_cache = static_cast<uint8_t *>(v_cache);
+    p.pairs = block_pairs;
+    p.err = dev_err;
+    p.num_pairs = num_pairs;
+    p.num_blocks = num_blocks;
+    p.block_bytes = block_bytes;
+    return from_cuda(pa::launch_copy_blocks(p, static_cast<cudaStream_t>(stream)));
+}
+
 size_t pa_split_workspace_bytes(int num_seqs, int num_q_heads, int head_dim, int max_seq_len,
                                 int partition_size) {
     if (num_seqs < 0 || num_q_heads <= 0 || head_dim <= 0 || max_seq_len < 0 ||

@@ -96,6 +96,16 @@ struct AppendParams {  // decode-form slot mapping + cache write in one kernel
     float v_scale;
 };
 
+struct CopyBlocksParams {  // copy-on-write: whole blocks inside both pools
+    uint8_t *k_cache;
+    uint8_t *v_cache;
+    const int32_t *pairs;  // [num_pairs][2] = (src, dst)
+    int *err;
+    int num_pairs;
+    int num_blocks;
+    int64_t block_bytes;   // num_kv_heads * block_size * head_dim * elem bytes
+};
+
 struct ReduceParams {
     void *out;
     const float *ws_lse;
@@ -114,6 +124,7 @@ cudaError_t launch_cache_write(const CacheWriteParams &p, DType act, DType kv, c
 cudaError_t launch_decode(const DecodeParams &p, DType q, DType kv, int head_dim, int tpl_group,
                           cudaStream_t stream);
 cudaError_t launch_reduce(const ReduceParams &p, DType q, int head_dim, cudaStream_t stream);
+cudaError_t launch_copy_blocks(const CopyBlocksParams &p, cudaStream_t stream);
 
 // Tensor-core decode (pa_decode_mma.cu): rows of the MMA used for the GQA
 // group (8 or 16); supported for head_dim 64/128 16-bit caches and head_dim

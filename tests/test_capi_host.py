@@ -160,3 +160,19 @@ def test_decode_append_checks(pa):
     assert call(ws=0) == 1            # split needs a workspace
     assert call(wsb=16) == 1
     assert call(S=0, kn=0) == 0       # empty batch
+
+
+def test_copy_blocks_checks(pa):
+    L = pa.lib()
+
+    def call(k=A, v=A, pairs=A, n=3, nb=10, hk=2, d=128, kv=pa.PA_BF16):
+        return L.pa_copy_blocks(k, v, pairs, n, nb, hk, d, 16, kv, None, None)
+
+    assert call(n=-1) == 1
+    assert call(nb=0) == 1
+    assert call(hk=0) == 1
+    assert call(kv=7) == 2            # unknown element type
+    assert call(pairs=0) == 1
+    assert call(k=0) == 1
+    assert call(v=A + 8) == 1         # misaligned pool
+    assert call(n=0, pairs=0, k=0, v=0) == 0   # nothing to copy
