@@ -92,6 +92,9 @@ def lib() -> ctypes.CDLL:
                                          i32, i32, f64, i32, i32, P, i32]
         L.orc_split_merge.restype = None
         L.orc_split_merge.argtypes = [P, P, P, i32, i32]
+        L.orc_prefill.restype = i32
+        L.orc_prefill.argtypes = [P, P, i32, P, P, i32, f64, f64, P, i32, P, P, i32, i32, i32, i32,
+                                  i32, f64]
         L.orc_copy_blocks.restype = i32
         L.orc_copy_blocks.argtypes = [P, P, P, i32, i32, i32, i32, i32, i32]
         _lib = L
@@ -277,6 +280,29 @@ def split_partials(q: np.ndarray, q_dtype: str, k_cache: np.ndarray, v_cache: np
     return lse, o
 
 
+def prefill(q: np.ndarray, q_dtype: str, k_cache: np.ndarray, v_cache: np.ndarray,
+            kv_dtype: str, block_tables: np.ndarray, seq_lens: np.ndarray,
+            query_start: np.ndarray, num_kv_heads: int, softmax_scale: float,
+            k_scale: float = 1.0, v_scale: float = 1.0, block_size: int = 16) -> np.ndarray:
+    """Chunked-prefill attention in fp64: ``q`` holds [T, Hq, d] 16-bit codes,
+    sequence s's chunk is rows query_start[s] .. query_start[s+1] - 1, the
+    last tokens of its seq_lens[s]; causal.  Returns [T, Hq, d] (rows no
+    sequence covers are 0)."""
+    q = _c(q, np.uint16)
+    T, Hq, d = q.shape
+    bt = _c(block_tables, np.int32)
+    sl = _c(seq_lens, np.int32)
+    qs = _c(query_start, np.int32)
+    out = np.zeros((T, Hq, d), dtype=np.float64)
+    r = lib().orc_prefill(_p(out), _p(q), DTYPES[q_dtype], _p(k_cache), _p(v_cache),
+                          DTYPES[kv_dtype], float(k_scale), float(v_scale), _p(bt), bt.shape[1],
+                          _p(sl), _p(qs), int(sl.size), Hq, num_kv_heads, d, block_size,
+                          float(softmax_scale))
+    if r:
+        raise ValueError("invalid prefill configuration")
+    return out
+
+
 def split_merge(lse: np.ndarray, o: np.ndarray) -> np.ndarray:
     lse, o = _c(lse, np.float64), _c(o, np.float64)
     NP, d = o.shape
@@ -307,6 +333,28 @@ def caches_for(w, include_new: bool = True) -> Tuple[np.ndarray, np.ndarray]:
         cache_write(w.k_new, w.v_new, kc, vc, slots, w.num_blocks, w.num_kv_heads, w.head_dim,
                     w.block_size, w.act_dtype, w.kv_dtype, w.k_scale, w.v_scale)
     return kc, vc
+
+
+def chunked_caches_for(w) -> Tuple[np.ndarray, np.ndarray]:
+    """The oracle's pools for a chunked-prefill workload (``workload.build_chunked``):
+    poisoned pools, then every context token and every chunk token written
+    at its slot."""
+    kc = empty_pool(w.num_blocks, w.num_kv_heads, w.block_size, w.head_dim, w.kv_dtype)
+    vc = empty_pool(w.num_blocks, w.num_kv_heads, w.block_size, w.head_dim, w.kv_dtype)
+    for seq, pos, kr, vr in ((w.ctx_seq, w.ctx_pos, w.k_ctx, w.v_ctx),
+                             (w.chunk_seq, w.chunk_pos, w.k_chunk, w.v_chunk)):
+        T = int(seq.size)
+        if T:
+            slots = slot_mapping(w.block_tables, None, seq, pos, T, w.block_size)
+            cache_write(kr, vr, kc, vc, slots, w.num_blocks, w.num_kv_heads, w.head_dim,
+                        w.block_size, w.act_dtype, w.kv_dtype, w.k_scale, w.v_scale)
+    return kc, vc
+
+
+def prefill_for(w, kc: np.ndarray, vc: np.ndarray) -> np.ndarray:
+    return prefill(w.q, w.act_dtype, kc, vc, w.kv_dtype, w.block_tables, w.seq_lens,
+                   w.query_start, w.num_kv_heads, w.softmax_scale, w.k_scale, w.v_scale,
+                   w.block_size)
 
 
 def decode_for(w, kc: np.ndarray, vc: np.ndarray, pairs: Optional[np.ndarray] = None) -> np.ndarray:

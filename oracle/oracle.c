@@ -17,6 +17,9 @@
  *     "KV Cache 与 PageAttention深度实战", §1.2;
  *   - fp8 E4M3 KV values (max 448): "大语言模型推理引擎深度剖析：从 KV Cache
  *     内存管理到 PagedAttention、投机解码与量化加速的完全工程指南", §4.2-§4.3;
+ *   - chunked prefill: a long prompt is cut into chunks (e.g. 512 tokens)
+ *     processed one after another, each chunk's queries attending causally
+ *     over the cache: openeuler page §4.5 and the second page §3.3;
  *   - copy-on-write of a shared block: first page §3.5 (a beam-search
  *     candidate that diverges gets a new block for the diverging part only)
  *     and the fifth page §2.3 (a request about to write into a shared block
@@ -391,4 +394,58 @@ int orc_copy_blocks(void *k_cache, void *v_cache, const int32_t *pairs, int num_
         }
     }
     return bad;
+}
+
+/* ------------------------------------------------------------------------- */
+/* chunked prefill: several query tokens per sequence, causal mask            */
+/* ------------------------------------------------------------------------- */
+
+/* Attention of one chunk of query tokens per sequence over the paged cache,
+ * causally masked (openeuler page §4.5; second page §3.3).  Sequence s holds
+ * L = seq_lens[s] tokens in the cache; the last n = query_start[s+1] -
+ * query_start[s] of them are this chunk.  Its query token j, row
+ * query_start[s] + j of q and out ([T][Hq][d]), sits at position
+ * L - n + j and attends to the keys at positions 0 .. L - n + j.  A decode
+ * step is the case n = 1.  Rows of out that no sequence covers are left as
+ * they are.  Returns -1 on a bad head configuration or a chunk longer than
+ * its sequence. */
+int orc_prefill(double *out, const void *q, int q_dtype, const void *k_cache, const void *v_cache,
+                int kv_dtype, double k_scale, double v_scale, const int32_t *block_tables,
+                int max_blocks_per_seq, const int32_t *seq_lens, const int32_t *query_start,
+                int num_seqs, int num_q_heads, int num_kv_heads, int head_dim, int block_size,
+                double softmax_scale) {
+    if (num_kv_heads <= 0 || num_q_heads % num_kv_heads) return -1;
+    int g = num_q_heads / num_kv_heads;
+    double *qrow = (double *)malloc(sizeof(double) * (size_t)head_dim);
+    for (int s = 0; s < num_seqs; ++s) {
+        int len = seq_lens[s];
+        int n = query_start[s + 1] - query_start[s];
+        if (n < 0 || n > len) {
+            free(qrow);
+            return -1;
+        }
+        if (n == 0) continue;
+        const int32_t *bt = block_tables + (int64_t)s * max_blocks_per_seq;
+        double *K = (double *)malloc(sizeof(double) * ((size_t)len * head_dim + 1));
+        double *V = (double *)malloc(sizeof(double) * ((size_t)len * head_dim + 1));
+        for (int kvh = 0; kvh < num_kv_heads; ++kvh) {
+            orc_gather(K, k_cache, kv_dtype, k_scale, bt, len, num_kv_heads, kvh, head_dim, block_size);
+            orc_gather(V, v_cache, kv_dtype, v_scale, bt, len, num_kv_heads, kvh, head_dim, block_size);
+            for (int j = 0; j < n; ++j) {
+                int pos = len - n + j;
+                int64_t row_tok = (int64_t)query_start[s] + j;
+                for (int hh = 0; hh < g; ++hh) {
+                    int h = kvh * g + hh;
+                    int64_t row = row_tok * num_q_heads + h;
+                    for (int i = 0; i < head_dim; ++i) qrow[i] = orc_elem(q_dtype, q, row * head_dim + i);
+                    orc_attention(out + row * head_dim, NULL, qrow, K, V, pos + 1, head_dim,
+                                  softmax_scale);
+                }
+            }
+        }
+        free(K);
+        free(V);
+    }
+    free(qrow);
+    return 0;
 }

@@ -11,6 +11,7 @@ import pytest
 import oracle
 from tests import test_oracle_cow as cow
 from tests import test_oracle_pins as pins
+from tests import test_oracle_prefill as pre
 
 SRC = os.path.join(os.path.dirname(oracle.__file__), "oracle.c")
 
@@ -39,6 +40,11 @@ MUTANTS = {
     "copy_blocks_direction_swapped": (
         "base[(int64_t)dst * block_bytes + b] = base[(int64_t)src * block_bytes + b];",
         "base[(int64_t)src * block_bytes + b] = base[(int64_t)dst * block_bytes + b];"),
+    "prefill_causal_off_by_one": ("qrow, K, V, pos + 1, head_dim,", "qrow, K, V, pos, head_dim,"),
+    "prefill_position_from_chunk_start": ("int pos = len - n + j;", "int pos = j;"),
+    "prefill_q_row_of_sequence": ("int64_t row_tok = (int64_t)query_start[s] + j;",
+                                  "int64_t row_tok = (int64_t)s + j;"),
+    "prefill_gqa_interleaved": ("int h = kvh * g + hh;", "int h = hh * num_kv_heads + kvh;"),
     "copy_blocks_one_head": ("int64_t block_bytes = (int64_t)num_kv_heads * block_size * head_dim * elem_bytes;",
                              "int64_t block_bytes = (int64_t)block_size * head_dim * elem_bytes;"),
 }
@@ -59,6 +65,9 @@ def _run_pins(golden_dir):
         ("closed", lambda: pins.test_closed_forms(oracle)),
         ("split", lambda: pins.test_split_equals_unsplit(oracle, 48)),
         ("roundtrip", lambda: pins.test_cache_write_then_gather_roundtrip(oracle)),
+        ("prefill_sdpa", lambda: pre.test_prefill_vs_torch_sdpa_causal(
+            oracle, [0, 5, 37, 16], [7, 1, 40, 16], 8, 2, 32, "bf16")),
+        ("prefill_chunks", lambda: pre.test_prefill_rows_do_not_depend_on_chunking(oracle)),
         ("cow_example", lambda: cow.test_cow_beam_search_example(oracle, golden_dir)),
         ("cow_brute", lambda: cow.test_copy_blocks_brute_force(oracle, "f16")),
         ("cow_bounds", lambda: cow.test_copy_blocks_out_of_range_skipped(oracle)),

@@ -346,3 +346,169 @@ def poison_byte() -> int:
     """Fill byte for pools before any write: 0xFF makes every f16 / bf16 pair
     and every E4M3 byte a NaN, so any read of an unwritten slot shows up."""
     return 0xFF
+
+
+# ----------------------------------------------------------------------------
+# chunked prefill: several new query tokens per sequence
+# ----------------------------------------------------------------------------
+
+@dataclasses.dataclass
+class ChunkedWorkload:
+    """One chunked-prefill step: every sequence has ``context_lens[s]`` tokens
+    in the cache and appends a chunk of ``chunk_lens[s]`` tokens, whose
+    queries then attend causally over the context and the chunk."""
+
+    name: str
+    seed: int
+    num_seqs: int
+    num_q_heads: int
+    num_kv_heads: int
+    head_dim: int
+    block_size: int
+    num_blocks: int
+    act_dtype: str
+    kv_dtype: str
+    seq_lens: np.ndarray  # int32 [S]: context + chunk
+    query_start: np.ndarray  # int32 [S + 1]: chunk rows of sequence s in q / out
+    block_tables: np.ndarray  # int32 [S, max_blocks_per_seq]
+    q: np.ndarray  # uint16 [T, Hq, d], T = total chunk tokens
+    ctx_seq: np.ndarray  # int32 [Tc]: context tokens (already cached)
+    ctx_pos: np.ndarray
+    k_ctx: np.ndarray  # uint16 [Tc, Hk, d]
+    v_ctx: np.ndarray
+    chunk_seq: np.ndarray  # int32 [T]: this chunk's tokens, in q row order
+    chunk_pos: np.ndarray
+    k_chunk: np.ndarray  # uint16 [T, Hk, d]
+    v_chunk: np.ndarray
+    k_scale: float
+    v_scale: float
+    free_blocks: np.ndarray
+
+    @property
+    def group(self) -> int:
+        return self.num_q_heads // self.num_kv_heads
+
+    @property
+    def max_blocks_per_seq(self) -> int:
+        return int(self.block_tables.shape[1])
+
+    @property
+    def num_tokens(self) -> int:
+        return int(self.query_start[-1])
+
+    @property
+    def chunk_lens(self) -> np.ndarray:
+        return np.diff(self.query_start).astype(np.int32)
+
+    @property
+    def max_query_len(self) -> int:
+        return int(self.chunk_lens.max()) if self.num_seqs else 0
+
+    @property
+    def softmax_scale(self) -> float:
+        return 1.0 / math.sqrt(self.head_dim)
+
+    def attended_pairs(self) -> int:
+        """(query token, key) pairs under the causal mask, per query head."""
+        n = self.chunk_lens.astype(np.int64)
+        ctx = self.seq_lens.astype(np.int64) - n
+        return int((n * ctx + n * (n + 1) // 2).sum())
+
+    def flops(self) -> int:
+        """Useful multiply-adds x 2 of q.K and P.V under the causal mask."""
+        return 4 * self.head_dim * self.num_q_heads * self.attended_pairs()
+
+
+def build_chunked(
+    name: str,
+    seed: int,
+    context_lens: Sequence[int],
+    chunk_lens: Sequence[int],
+    num_q_heads: int,
+    num_kv_heads: int,
+    head_dim: int,
+    act_dtype: str,
+    kv_dtype: str,
+    block_size: int = BLOCK_SIZE,
+    num_blocks: Optional[int] = None,
+    pool_slack: float = 0.10,
+    extra_table_cols: int = 0,
+) -> ChunkedWorkload:
+    """Draw a chunked-prefill step: tables over a shuffled pool (as ``build``),
+    context K/V rows, the chunk's q and K/V rows, all N(0, 1) rounded to the
+    activation dtype."""
+    rng = np.random.default_rng(seed)
+    ctx = np.asarray(context_lens, dtype=np.int32)
+    chk = np.asarray(chunk_lens, dtype=np.int32)
+    if ctx.shape != chk.shape or (ctx.size and (int(ctx.min()) < 0 or int(chk.min()) < 0)):
+        raise ValueError("context and chunk lengths must be non-negative and paired")
+    S = int(ctx.size)
+    lens = (ctx + chk).astype(np.int32)
+    nblk = [blocks_needed(L, block_size) for L in lens]
+    used = int(sum(nblk))
+    if num_blocks is None:
+        num_blocks = max(used + 1, int(math.ceil(used * (1.0 + pool_slack))))
+    if num_blocks < used:
+        raise ValueError("pool too small")
+    perm = rng.permutation(num_blocks).astype(np.int32)
+    mbs = max(max(nblk, default=0), 1) + extra_table_cols
+    tables = np.empty((S, mbs), dtype=np.int32)
+    cursor = 0
+    for s in range(S):
+        tables[s, :nblk[s]] = perm[cursor:cursor + nblk[s]]
+        cursor += nblk[s]
+    free = perm[cursor:].copy()
+    pad = int(free[0]) if free.size else 0
+    for s in range(S):
+        tables[s, nblk[s]:] = pad
+    query_start = np.zeros(S + 1, dtype=np.int32)
+    query_start[1:] = np.cumsum(chk)
+    T = int(query_start[-1])
+    q = draw_normal_bits(rng, (T, num_q_heads, head_dim), act_dtype)
+    chunk_seq = np.repeat(np.arange(S, dtype=np.int32), chk)
+    chunk_pos = np.concatenate([np.arange(c, c + n, dtype=np.int32) for c, n in zip(ctx, chk)]) \
+        if S else np.zeros(0, np.int32)
+    k_chunk = draw_normal_bits(rng, (T, num_kv_heads, head_dim), act_dtype)
+    v_chunk = draw_normal_bits(rng, (T, num_kv_heads, head_dim), act_dtype)
+    ctx_seq = np.repeat(np.arange(S, dtype=np.int32), ctx)
+    ctx_pos = np.concatenate([np.arange(0, c, dtype=np.int32) for c in ctx]) \
+        if S else np.zeros(0, np.int32)
+    Tc = int(ctx_seq.size)
+    k_ctx = draw_normal_bits(rng, (Tc, num_kv_heads, head_dim), act_dtype)
+    v_ctx = draw_normal_bits(rng, (Tc, num_kv_heads, head_dim), act_dtype)
+    k_scale = v_scale = 1.0
+    if kv_dtype == "e4m3":
+        k_scale = per_tensor_e4m3_scale(amax_of_bits(k_ctx, k_chunk, dtype=act_dtype))
+        v_scale = per_tensor_e4m3_scale(amax_of_bits(v_ctx, v_chunk, dtype=act_dtype))
+    elif kv_dtype != act_dtype:
+        raise ValueError("a 16-bit cache must have the activation dtype")
+    return ChunkedWorkload(
+        name=name, seed=seed, num_seqs=S, num_q_heads=num_q_heads, num_kv_heads=num_kv_heads,
+        head_dim=head_dim, block_size=block_size, num_blocks=int(num_blocks),
+        act_dtype=act_dtype, kv_dtype=kv_dtype, seq_lens=lens, query_start=query_start,
+        block_tables=tables, q=q, ctx_seq=ctx_seq, ctx_pos=ctx_pos, k_ctx=k_ctx, v_ctx=v_ctx,
+        chunk_seq=chunk_seq, chunk_pos=chunk_pos, k_chunk=k_chunk, v_chunk=v_chunk,
+        k_scale=k_scale, v_scale=v_scale, free_blocks=free,
+    )
+
+
+PREFILL_NAMES = {
+    1: "chunked prefill, Qwen3-8B-shaped: 16 seqs x 512-token chunk after contexts U[0,3584], "
+       "32/8 heads, d128, bf16",
+    2: "chunked prefill, Llama-3-70B-shaped: 8 seqs x 512-token chunk after contexts U[1536,2048], "
+       "64/8 heads, d128, bf16",
+}
+
+
+def prefill_config(cfg: int) -> ChunkedWorkload:
+    """Named chunked-prefill workloads: 512-token chunks (the chunk size the
+    pages give) on the decode configurations' model shapes."""
+    seed = SEED_BASE + 100 + cfg
+    rng = np.random.default_rng([seed, 1])
+    if cfg == 1:
+        ctx = rng.integers(0, 3584, size=16, endpoint=True)
+        return build_chunked(PREFILL_NAMES[1], seed, ctx, [512] * 16, 32, 8, 128, "bf16", "bf16")
+    if cfg == 2:
+        ctx = rng.integers(1536, 2048, size=8, endpoint=True)
+        return build_chunked(PREFILL_NAMES[2], seed, ctx, [512] * 8, 64, 8, 128, "bf16", "bf16")
+    raise ValueError(f"unknown prefill config {cfg}")
