@@ -3,6 +3,7 @@
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                     [--config 2] [--mode fused|fused_single|split|single] [--partition 512]
     python bench.py --op copy_blocks [--config 2] [--pairs 4096]
+    python bench.py --op prefill [--pconfig 1]
 
 A step is one pass of the whole hot path over one batch: slot mapping of the
 new tokens, cache write of their K/V rows, and decode attention.  The default
@@ -54,6 +55,15 @@ FALLBACK_HBM_GBS = 6650.0
 # ---------------------------------------------------------------------------
 # helpers
 # ---------------------------------------------------------------------------
+
+def measured_tensor_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return float(json.load(f)["bf16_tflops"]), "measured"
+    except Exception:  # noqa: BLE001
+        return 1590.0, "fallback"
+
 
 def measured_hbm_peak():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
@@ -349,6 +359,70 @@ def run_copy_blocks(args):
 
 
 # ---------------------------------------------------------------------------
+# chunked prefill (pa_prefill), one attention launch per step
+# ---------------------------------------------------------------------------
+
+def run_prefill(args):
+    """Time pa_prefill on a named 512-token-chunk workload.  A step is the
+    chunk's cache append (slot mapping + cache write) and the attention
+    launch; ``value`` counts the useful flops of q.K and P.V under the causal
+    mask (4 * d * Hq per attended (query, key) pair)."""
+    import torch
+
+    import workload
+    from paged_kv_cache_369_b200.runner import PagedPrefill
+
+    world, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    w = workload.prefill_config(args.pconfig)
+    stream = torch.cuda.Stream(device)
+    with torch.cuda.stream(stream):
+        pre = PagedPrefill(w, device=str(device), stream=stream)
+        for _ in range(args.warmup):
+            pre.step()
+    torch.cuda.synchronize(device)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    clocks = ClockSampler(device.index or 0)
+    clocks.start()
+    with torch.cuda.stream(stream):
+        for e0, e1, e2 in ev:
+            e0.record(stream)
+            pre.write_chunk()
+            e1.record(stream)
+            pre.attend()
+            e2.record(stream)
+    torch.cuda.synchronize(device)
+    clocks.stop()
+    step_ms = statistics.mean(a.elapsed_time(c) for a, _, c in ev)
+    attn_ms = statistics.mean(b.elapsed_time(c) for _, b, c in ev)
+    flops = w.flops()
+    value = flops / (step_ms * 1e-3) / 1e12
+    achieved = flops / (attn_ms * 1e-3) / 1e12
+    peak, kind = measured_tensor_peak()
+    line = {
+        "metric": "chunked-prefill attention TFLOP/s (useful causal flops)",
+        "value": value, "unit": "TFLOP/s", "n_gpus": 1, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": w.act_dtype,
+        "data": "synthetic: seeded N(0,1) q/K/V, shuffled block pool",
+        "config": {"workload": w.name, "num_seqs": w.num_seqs, "chunk": int(w.max_query_len),
+                   "num_q_heads": w.num_q_heads, "num_kv_heads": w.num_kv_heads,
+                   "head_dim": w.head_dim, "context_mean": float((w.seq_lens - w.chunk_lens).mean()),
+                   "seed": w.seed, "l2": "K/V re-read across query tiles is meant to hit L2; no flush"},
+        "attention_us": attn_ms * 1e3, "cache_write_us": (step_ms - attn_ms) * 1e3,
+        "tokens_per_s": w.num_tokens / (step_ms * 1e-3),
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                     "frac": achieved / peak, "traffic": None, "kernel": "prefill_kernel (tcgen05)",
+                     "algorithmic_flops_per_launch": flops,
+                     "peak_source": f"{kind} dense bf16 (cuBLAS burst, MEASURED_PEAKS.json bf16_tflops)"},
+        "gpu_launches": 3 * args.steps, "clocks": clocks.summary(), "device_error": pre.error(),
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------------------
 # the CUDA path
 # ---------------------------------------------------------------------------
 
@@ -521,8 +595,11 @@ def main(argv=None):
     ap.add_argument("--partition", type=int, default=512)
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--op", choices=("decode", "copy_blocks"), default="decode",
-                    help="decode: the decode step (default); copy_blocks: pa_copy_blocks alone")
+    ap.add_argument("--op", choices=("decode", "copy_blocks", "prefill"), default="decode",
+                    help="decode: the decode step (default); copy_blocks: pa_copy_blocks alone; "
+                         "prefill: a chunked-prefill step")
+    ap.add_argument("--pconfig", type=int, default=1, choices=(1, 2),
+                    help="named chunked-prefill workload for --op prefill")
     ap.add_argument("--pairs", type=int, default=4096, help="block pairs for --op copy_blocks")
     args = ap.parse_args(argv)
     if args.warmup < 3:
@@ -531,6 +608,8 @@ def main(argv=None):
         return run_reference(args)
     if args.op == "copy_blocks":
         return run_copy_blocks(args)
+    if args.op == "prefill":
+        return run_prefill(args)
     return run_ours(args)
 
 

@@ -217,6 +217,44 @@ pa_status pa_decode_split_reduce(void *out, const void *q, const void *k_cache,
                                  void *stream);
 
 /*
+ * pa_prefill -- chunked-prefill attention: several new query tokens per
+ * sequence, causal, over the paged cache.
+ *
+ * Source: "openeuler.csdn.net 推理优化篇", §4.5 (Chunked Prefill: a long prompt
+ * is cut into chunks, e.g. 512 tokens, processed one after another and mixed
+ * with decode steps) and "vLLM推理引擎深度解析：PagedAttention与连续批处理",
+ * §3.3; the attention itself is the pages' softmax(Q K^T / sqrt(d_k)) V with
+ * K / V read through the block table ("KV Cache 与 PageAttention深度实战",
+ * §1.2, §3.2).
+ *
+ * Sequence s has L = seq_lens[s] tokens in the cache, the chunk included; its
+ * chunk is the last n = query_start[s+1] - query_start[s] of them (its K/V
+ * rows are already stored, e.g. by pa_slot_mapping with token positions +
+ * pa_cache_write).  Its query token j is row query_start[s] + j of q and out
+ * ([num_tokens, num_q_heads, head_dim]) and sits at position L - n + j:
+ *   out[row][h] = sum_t p_t V_t,  p = softmax_t(softmax_scale * q[row][h] . K_t),
+ *   t = 0 .. L - n + j   (causal), KV head h / (num_q_heads / num_kv_heads).
+ * A chunk of one token is a decode step.  query_start ([num_seqs + 1], device
+ * int32) is non-decreasing with query_start[num_seqs] <= num_tokens; rows no
+ * sequence covers are not written.  max_query_len bounds every n.
+ *
+ * Supported: block_size 16, head_dim 64 or 128, q_dtype (= out dtype =
+ * kv_dtype) PA_F16 or PA_BF16 (E4M3 caches return PA_ERR_UNSUPPORTED), GQA
+ * groups up to 128, num_seqs and num_kv_heads up to 65535.  Arithmetic is
+ * fp32 with the probabilities kept to ~16 bits (bf16 hi + lo) or f16; out is
+ * rounded to nearest even once.  Errors as for pa_decode: a chunk longer
+ * than its sequence or than max_query_len, a length past the table, or a
+ * table entry outside the pool flags PA_ERR_DEVICE_BOUNDS (that sequence's
+ * rows are then not written, or the bad block reads as zeros).
+ */
+pa_status pa_prefill(void *out, const void *q, const void *k_cache, const void *v_cache,
+                     const int32_t *block_tables, int max_blocks_per_seq, const int32_t *seq_lens,
+                     const int32_t *query_start, int num_seqs, int num_tokens, int max_query_len,
+                     int num_q_heads, int num_kv_heads, int head_dim, int block_size,
+                     int num_blocks, float softmax_scale, pa_dtype q_dtype, pa_dtype kv_dtype,
+                     int *dev_err, void *stream);
+
+/*
  * pa_copy_blocks -- copy whole KV blocks inside the pools (copy-on-write).
  *
  * Source: "Transformer 推理优化：KV Cache、PagedAttention 与 vLLM", §3.5 (beam

@@ -34,7 +34,7 @@ PA_FP8_E4M3 = 2
 SYMBOLS = (
     "pa_status_string", "pa_version", "pa_slot_mapping", "pa_cache_write", "pa_decode",
     "pa_split_workspace_bytes", "pa_decode_split_reduce", "pa_decode_split_reduce_static_scratch",
-    "pa_decode_append", "pa_copy_blocks",
+    "pa_decode_append", "pa_copy_blocks", "pa_prefill",
 )
 
 PA_STATIC_SCRATCH_BYTES = 32 * 1024 * 1024
@@ -80,6 +80,9 @@ _lib.pa_decode_append.argtypes = [_P, _P, _P, _P, _P, _P, _P, _I, _P, _I, _I, _I
 _lib.pa_decode_split_reduce_static_scratch.restype = _I
 _lib.pa_decode_split_reduce_static_scratch.argtypes = [_P, _P, _P, _P, _P, _I, _P, _I, _I, _I, _I,
                                                        _I, _I, _F, _I, _I, _F, _F, _I, _I, _P, _P]
+_lib.pa_prefill.restype = _I
+_lib.pa_prefill.argtypes = [_P, _P, _P, _P, _P, _I, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _F,
+                            _I, _I, _P, _P]
 _lib.pa_copy_blocks.restype = _I
 _lib.pa_copy_blocks.argtypes = [_P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P]
 
@@ -249,3 +252,19 @@ def pa_copy_blocks(k_cache, v_cache, block_pairs, dev_err=None, stream=None) -> 
     _check(_lib.pa_copy_blocks(_ptr(k_cache), _ptr(v_cache), _ptr(block_pairs), n, nb, Hk, d, B,
                                dtype_code(k_cache.dtype), _ptr(dev_err), _stream(stream)),
            "pa_copy_blocks")
+
+
+def pa_prefill(out, q, k_cache, v_cache, block_tables, seq_lens, query_start, max_query_len: int,
+               softmax_scale: float, dev_err=None, stream=None) -> None:
+    """Chunked-prefill attention: the rows query_start[s] .. query_start[s+1]-1
+    of ``q`` ([T, Hq, d]) are the last tokens of sequence s's seq_lens[s] and
+    attend causally over its cache."""
+    T, Hq, d = (int(x) for x in q.shape)
+    nb, Hk, B, _ = (int(x) for x in k_cache.shape)
+    S = int(seq_lens.shape[0])
+    _check(_lib.pa_prefill(_ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables),
+                           int(block_tables.shape[1]), _ptr(seq_lens), _ptr(query_start), S, T,
+                           int(max_query_len), Hq, Hk, d, B, nb, float(softmax_scale),
+                           dtype_code(q.dtype), dtype_code(k_cache.dtype), _ptr(dev_err),
+                           _stream(stream)),
+           "pa_prefill")

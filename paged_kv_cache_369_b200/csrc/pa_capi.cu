@@ -309,6 +309,57 @@ pa_status pa_decode_append(void *out, const void *q, const void *k_new, const vo
     return from_cuda(pa::launch_reduce(r, to_internal(q_dtype), head_dim, s));
 }
 
+pa_status pa_prefill(void *out, const void *q, const void *k_cache, const void *v_cache,
+                     const int32_t *block_tables, int max_blocks_per_seq, const int32_t *seq_lens,
+                     const int32_t *query_start, int num_seqs, int num_tokens, int max_query_len,
+                     int num_q_heads, int num_kv_heads, int head_dim, int block_size,
+                     int num_blocks, float softmax_scale, pa_dtype q_dtype, pa_dtype kv_dtype,
+                     int *dev_err, void *stream) {
+    if (num_seqs < 0 || num_tokens < 0 || max_query_len < 0 || num_q_heads <= 0 ||
+        num_kv_heads <= 0 || head_dim <= 0 || block_size <= 0)
+        return PA_ERR_INVALID_ARG;
+    if (num_q_heads % num_kv_heads != 0) return PA_ERR_INVALID_ARG;
+    if (!is_act(q_dtype)) return PA_ERR_UNSUPPORTED;
+    if (kv_dtype != q_dtype) return PA_ERR_UNSUPPORTED;  // E4M3 caches: not on this path
+    if (head_dim != 64 && head_dim != 128) return PA_ERR_UNSUPPORTED;
+    if (block_size != pa::kBlockSize) return PA_ERR_UNSUPPORTED;
+    const int g = num_q_heads / num_kv_heads;
+    if (g > 128) return PA_ERR_UNSUPPORTED;
+    if (!isfinite(softmax_scale)) return PA_ERR_INVALID_ARG;
+    if (num_seqs == 0 || num_tokens == 0) return PA_OK;
+    if (!out || !q || !k_cache || !v_cache || !block_tables || !seq_lens || !query_start)
+        return PA_ERR_INVALID_ARG;
+    if (!aligned16(out) || !aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache))
+        return PA_ERR_INVALID_ARG;
+    if (max_blocks_per_seq <= 0 || num_blocks <= 0 || max_query_len <= 0) return PA_ERR_INVALID_ARG;
+    if (num_seqs > 65535 || num_kv_heads > 65535) return PA_ERR_UNSUPPORTED;
+    const int64_t rows = (int64_t)num_blocks * num_kv_heads * pa::kBlockSize;
+    if (rows + pa::kBlockSize >= (int64_t(1) << 31)) return PA_ERR_UNSUPPORTED;
+    if (!pa::prefill_supported()) return PA_ERR_CUDA;
+    pa::PrefillParams p = {};
+    p.out = out;
+    p.q = q;
+    p.k_cache = k_cache;
+    p.v_cache = v_cache;
+    p.block_tables = block_tables;
+    p.seq_lens = seq_lens;
+    p.query_start = query_start;
+    p.err = dev_err;
+    p.max_blocks_per_seq = max_blocks_per_seq;
+    p.num_seqs = num_seqs;
+    p.num_tokens = num_tokens;
+    p.max_query_len = max_query_len;
+    p.num_q_heads = num_q_heads;
+    p.num_kv_heads = num_kv_heads;
+    p.num_blocks = num_blocks;
+    p.group = g;
+    p.tok_per_tile = 128 / g;
+    p.oob_row = (int)rows;
+    p.qk_scale_log2 = (float)((double)softmax_scale * 1.4426950408889634074);
+    return from_cuda(pa::launch_prefill(p, to_internal(q_dtype), head_dim,
+                                        static_cast<cudaStream_t>(stream)));
+}
+
 pa_status pa_copy_blocks(void *k_cache, void *v_cache, const int32_t *block_pairs, int num_pairs,
                          int num_blocks, int num_kv_heads, int head_dim, int block_size,
                          pa_dtype kv_dtype, int *dev_err, void *stream) {

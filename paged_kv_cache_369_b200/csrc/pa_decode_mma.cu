@@ -34,6 +34,7 @@
 #include <type_traits>
 
 #include "pa_device.cuh"
+#include "pa_tmap.h"
 
 namespace pa {
 
@@ -609,8 +610,6 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, 3)
 // host side: tensor maps and launch
 // ---------------------------------------------------------------------------
 
-namespace {
-
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
     static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
     static bool tried = false;
@@ -641,6 +640,8 @@ bool encode_pool_map(CUtensorMap *m, const void *base, int elem_bytes, int d, in
                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
 }
+
+namespace {
 
 template <typename QT, typename KVT, int D, int GT>
 cudaError_t launch_mma_t(const DecodeParams &p, cudaStream_t stream) {

@@ -106,6 +106,28 @@ struct CopyBlocksParams {  // copy-on-write: whole blocks inside both pools
     int64_t block_bytes;   // num_kv_heads * block_size * head_dim * elem bytes
 };
 
+struct PrefillParams {  // chunked prefill (pa_prefill)
+    void *out;                  // [T, Hq, D] q dtype
+    const void *q;              // [T, Hq, D]
+    const void *k_cache;        // [NB, Hk, 16, D]
+    const void *v_cache;
+    const int32_t *block_tables;
+    const int32_t *seq_lens;    // [S] cached tokens, the chunk included
+    const int32_t *query_start; // [S + 1] chunk rows of each sequence
+    int *err;
+    int max_blocks_per_seq;
+    int num_seqs;
+    int num_tokens;             // T
+    int max_query_len;          // bounds every chunk length
+    int num_q_heads;
+    int num_kv_heads;
+    int num_blocks;
+    int group;                  // Hq / Hk
+    int tok_per_tile;           // floor(128 / group) chunk tokens per query tile
+    int oob_row;                // a pool row index past the end (zero-filled loads)
+    float qk_scale_log2;        // softmax_scale * log2(e)
+};
+
 struct ReduceParams {
     void *out;
     const float *ws_lse;
@@ -125,6 +147,11 @@ cudaError_t launch_decode(const DecodeParams &p, DType q, DType kv, int head_dim
                           cudaStream_t stream);
 cudaError_t launch_reduce(const ReduceParams &p, DType q, int head_dim, cudaStream_t stream);
 cudaError_t launch_copy_blocks(const CopyBlocksParams &p, cudaStream_t stream);
+
+// Chunked prefill on tcgen05 tensor cores (pa_prefill.cu): 16-bit caches,
+// head_dim 64 / 128, GQA groups up to 128.
+bool prefill_supported();
+cudaError_t launch_prefill(const PrefillParams &p, DType q, int head_dim, cudaStream_t stream);
 
 // Tensor-core decode (pa_decode_mma.cu): rows of the MMA used for the GQA
 // group (8 or 16); supported for head_dim 64/128 16-bit caches and head_dim

@@ -1,0 +1,570 @@
+// Chunked-prefill attention over the paged KV cache on the fifth-generation
+// tensor cores: tcgen05.mma with accumulators in tensor memory (TMEM),
+// operands staged in shared memory by TMA.
+//
+// What it computes ("openeuler.csdn.net 推理优化篇", §4.5 Chunked Prefill;
+// "vLLM推理引擎深度解析：PagedAttention与连续批处理", §3.3): a long prompt is cut
+// into chunks (the pages' example: 512 tokens); each chunk's K/V rows are
+// appended to the cache (pa_slot_mapping + pa_cache_write) and its query
+// tokens then attend causally over everything cached so far,
+//   out[j][h] = softmax_t(scale * q[j][h] . K_t) V_t,   t <= L - n + j,
+// K_t / V_t read through the sequence's block table ("Transformer 推理优化：
+// KV Cache、PagedAttention 与 vLLM", §3.3).  A decode step is the one-token
+// chunk.
+//
+// Work decomposition: one CTA per (sequence, KV head, query tile).  A query
+// tile is 128 rows = floor(128 / g) chunk tokens x the g query heads of the
+// KV head (row r: token r / g, head r % g), so the whole GQA group shares each
+// K/V tile it reads.  Keys come in tiles of 128 = 8 blocks of 16 tokens.
+//   - warp 4 (one lane), TMA producer: the Q tile once through a 3-D tensor
+//     map over q [T, Hq, d]; per key tile, the 8 K and 8 V blocks named by the
+//     block table through the pool's 2-D map (16-row x 128-byte boxes, 128B
+//     swizzle) into a 2-stage ring.  Blocks past the sequence's end are
+//     fetched from past the end of the map, which the copy fills with zeros.
+//   - warp 5 (one lane), MMA issuer: S_j = Q K_j^T (M 128, N 128, K d) into
+//     one of two TMEM buffers; O += P_j V_j with A = P read from TMEM and
+//     B = V from shared memory (MN-major).  Issue order QK_0, QK_1, PV_0,
+//     QK_2, PV_1, ...: the tensor cores compute the next scores while the
+//     softmax works on the current ones; tcgen05 operations of one thread
+//     run in issue order, which makes the buffer reuse safe.
+//   - warps 0-3, one thread per row: S_j from TMEM, causal mask by select,
+//     online softmax with a lazy rescale (O and l are rescaled only when the
+//     row max grows by more than 8 in log2 units; otherwise p is taken
+//     against the old max, at most 2^8), P written back over S_j (bf16 as
+//     hi + lo halves so P keeps ~16 bits; f16 as one half), O / l at the end.
+// V rows past the sequence's last token (the tail of its last block) are
+// cleared in shared memory before P.V: p = 0 there, but 0 x NaN poison = NaN.
+// Every wait is bounded; a timeout reports PA_ERR_DEVICE_TIMEOUT, makes the
+// other roles give up, drains the copies and MMAs in flight and frees TMEM.
+#include <cuda.h>
+#include <math_constants.h>
+
+#include <type_traits>
+
+#include "pa_device.cuh"
+#include "pa_tmap.h"
+
+namespace pa {
+
+namespace tc {
+
+constexpr unsigned kFull = 0xFFFFFFFFu;
+
+// Shared-memory matrix descriptor (sm_100 form): start, leading / stride
+// byte offsets (16-byte units), version 1, 128-byte swizzle.
+__device__ __forceinline__ uint64_t sdesc(uint32_t addr, uint32_t lbo, uint32_t sbo) {
+    return (uint64_t)((addr >> 4) & 0x3FFFu) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
+           ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
+}
+
+// D[tmem] (+)= A[smem] B[smem]
+__device__ __forceinline__ void mma_ss(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc,
+                                       uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d),
+        "l"(a), "l"(b), "r"(idesc), "r"(accumulate));
+}
+
+// D[tmem] (+)= A[tmem] B[smem]
+__device__ __forceinline__ void mma_ts(uint32_t d, uint32_t a, uint64_t b, uint32_t idesc,
+                                       uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}\n" ::"r"(d),
+        "r"(a), "l"(b), "r"(idesc), "r"(accumulate));
+}
+
+// arrive on `bar` once every tcgen05 operation this thread issued is done
+__device__ __forceinline__ void commit(uint32_t bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                     bar)
+                 : "memory");
+}
+
+__device__ __forceinline__ void fence_before() {
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void fence_after() {
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+__device__ __forceinline__ void alloc(uint32_t slot_addr, uint32_t ncols) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(slot_addr),
+                 "r"(ncols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void dealloc(uint32_t taddr, uint32_t ncols) {
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+                 : "memory");
+}
+
+// 32 consecutive 32-bit columns of this thread's TMEM lane
+__device__ __forceinline__ void ld32(uint32_t taddr, uint32_t *r) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,"
+        "%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+          "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+          "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
+          "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr));
+}
+// Wait for this thread's TMEM loads; the empty asm per register makes every
+// later use of the loaded values come after the wait.
+template <int N> __device__ __forceinline__ void wait_ld(uint32_t *r) {
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+    for (int i = 0; i < N; ++i) asm volatile("" : "+r"(r[i]));
+}
+
+__device__ __forceinline__ void st16(uint32_t taddr, const uint32_t *r) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
+        "%14,%15,%16};" ::"r"(taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+        "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
+        "r"(r[15])
+        : "memory");
+}
+__device__ __forceinline__ void st32(uint32_t taddr, const uint32_t *r) {
+    st16(taddr, r);
+    st16(taddr + 16, r + 16);
+}
+__device__ __forceinline__ void wait_st() {
+    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, int x, int y,
+                                            uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, "
+        "{%2, %3}], [%4];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
+        : "memory");
+}
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap *map, int x, int y,
+                                            int z, uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, "
+        "{%2, %3, %4}], [%5];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(bar)
+        : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
+// Bounded wait on an mbarrier phase that also gives up when another role of
+// the CTA has already given up (abort flag); the thread that runs out of
+// time raises the flag and reports the timeout.
+__device__ __forceinline__ bool wait_phase(uint32_t bar, uint32_t parity, volatile int *abort_flag,
+                                           int *err) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = global_ns();
+    for (;;) {
+#pragma unroll 1
+        for (int i = 0; i < 64; ++i)
+            if (mbar_try_wait(bar, parity)) return true;
+        if (*abort_flag) return false;
+        if (global_ns() - t0 > kWaitLimitNs) {
+            *abort_flag = 1;
+            flag_error(err, kErrTimeout);
+            return false;
+        }
+    }
+}
+
+__device__ __forceinline__ uint32_t pack2(float lo, float hi, bf16_t) {
+    uint32_t r;
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+__device__ __forceinline__ uint32_t pack2(float lo, float hi, f16_t) {
+    uint32_t r;
+    asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+__device__ __forceinline__ void unpack2(uint32_t w, float &lo, float &hi, bf16_t) {
+    lo = __uint_as_float(w << 16);
+    hi = __uint_as_float(w & 0xFFFF0000u);
+}
+
+}  // namespace tc
+
+template <typename T, int D> struct PfCfg {
+    static constexpr int BM = 128;  // query rows per tile (TMEM lanes)
+    static constexpr int BN = 128;  // keys per tile = 8 blocks
+    static constexpr int ST = 2;    // K/V ring stages
+    static constexpr int ATOMS = D / 64;  // 128-byte swizzle atoms across d
+    static constexpr int Q_BYTES = ATOMS * BM * 128;
+    static constexpr int KV_BYTES = ATOMS * BN * 128;
+    static constexpr int OFF_Q = 0;
+    static constexpr int OFF_KV = Q_BYTES;  // stage st: K, then V
+    static constexpr int OFF_BAR = OFF_KV + ST * 2 * KV_BYTES;
+    // q_full, kv_full[ST], kv_empty[ST], s_full[2], p_full[2], pv_done, drain
+    static constexpr int NBAR = 1 + 2 * ST + 2 + 2 + 1 + 1;
+    static constexpr int OFF_SLOT = OFF_BAR + NBAR * 8;
+    static constexpr int OFF_ABORT = OFF_SLOT + 4;
+    static constexpr int USED = OFF_ABORT + 4;
+    // at least 120 KiB so that one CTA holds an SM (and its 512 TMEM columns)
+    static constexpr int SMEM = 1024 + (USED < 120 * 1024 ? 120 * 1024 : USED);
+    static constexpr bool HILO = std::is_same<T, bf16_t>::value;
+    static constexpr uint32_t TMEM_COLS = 512;
+    static constexpr uint32_t COL_S0 = 0, COL_S1 = 128, COL_O = 256;
+    static constexpr uint32_t FMT = HILO ? 1u : 0u;  // kind::f16 operand format: f16 0, bf16 1
+    // instruction descriptors: fp32 accumulate, A/B format, majors, N >> 3, M >> 4
+    static constexpr uint32_t IDESC_QK = (1u << 4) | (FMT << 7) | (FMT << 10) |
+                                         ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
+    static constexpr uint32_t IDESC_PV = (1u << 4) | (FMT << 7) | (FMT << 10) | (1u << 16) |
+                                         ((uint32_t)(D >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
+    static_assert(D == 64 || D == 128, "head_dim 64 or 128");
+    static_assert(SMEM <= 227 * 1024, "shared memory budget");
+};
+
+template <typename T, int D>
+__global__ void __launch_bounds__(192, 1)
+    prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tmap_q,
+                   const __grid_constant__ CUtensorMap tmap_k,
+                   const __grid_constant__ CUtensorMap tmap_v) {
+    using C = PfCfg<T, D>;
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw = smem_addr(smem_raw);
+    const uint32_t base = (raw + 1023u) & ~1023u;
+    uint8_t *smem = smem_raw + (base - raw);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int tile = blockIdx.x, kvh = blockIdx.y, s = blockIdx.z;
+    const int g = p.group, tpt = p.tok_per_tile;
+
+    // ---- this CTA's rows and keys (uniform over the CTA) ---------------------
+    const int L = p.seq_lens[s];
+    const int q0 = p.query_start[s];
+    const int n = p.query_start[s + 1] - q0;
+    if (L < 0 || L > p.max_blocks_per_seq * kBlockSize || n < 0 || n > L || q0 < 0 ||
+        q0 + n > p.num_tokens || n > p.max_query_len) {
+        if (threadIdx.x == 0 && tile == 0 && kvh == 0) flag_error(p.err, kErrBounds);
+        return;
+    }
+    const int tok0 = tile * tpt;
+    if (tok0 >= n) return;
+    const int ntok = min(tpt, n - tok0);
+    const int ctx = L - n;
+    const int nt = (ctx + tok0 + ntok - 1) / C::BN + 1;  // key tiles up to the last row's position
+    const int nblk_seq = (L + kBlockSize - 1) / kBlockSize;
+
+    const uint32_t bars = base + C::OFF_BAR;
+    const uint32_t bar_q = bars;
+    auto bar_kv_full = [&](int st) { return bars + 8u * (1 + st); };
+    auto bar_kv_empty = [&](int st) { return bars + 8u * (1 + C::ST + st); };
+    auto bar_s_full = [&](int b) { return bars + 8u * (1 + 2 * C::ST + b); };
+    auto bar_p_full = [&](int b) { return bars + 8u * (3 + 2 * C::ST + b); };
+    const uint32_t bar_pv = bars + 8u * (5 + 2 * C::ST);
+    const uint32_t bar_drain = bar_pv + 8u;
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + C::OFF_ABORT);
+    uint32_t *slot = reinterpret_cast<uint32_t *>(smem + C::OFF_SLOT);
+
+    if (threadIdx.x == 0) {
+        mbar_init(bar_q, 1);
+#pragma unroll
+        for (int st = 0; st < C::ST; ++st) {
+            mbar_init(bar_kv_full(st), 1);
+            mbar_init(bar_kv_empty(st), 1);
+        }
+#pragma unroll
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(bar_s_full(b), 1);
+            mbar_init(bar_p_full(b), 128);
+        }
+        mbar_init(bar_pv, 1);
+        mbar_init(bar_drain, 1);
+        *abort_flag = 0;
+        mbar_init_fence();
+    }
+    if (warp == 0) tc::alloc(smem_addr(slot), C::TMEM_COLS);
+    tc::fence_before();
+    __syncthreads();
+    tc::fence_after();
+    const uint32_t tmem = *slot;
+
+    const uint32_t q_smem = base + C::OFF_Q;
+    auto k_smem = [&](int st) { return base + C::OFF_KV + (uint32_t)(st * 2 * C::KV_BYTES); };
+    auto v_smem = [&](int st) { return k_smem(st) + (uint32_t)C::KV_BYTES; };
+
+    if (warp == 4) {
+        // ================= TMA producer ===========================================
+        if (lane == 0) {
+            asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_q)) : "memory");
+            asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_k)) : "memory");
+            asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_v)) : "memory");
+            mbar_arrive_expect_tx(bar_q, (uint32_t)(C::ATOMS * tpt * g * 128));
+#pragma unroll
+            for (int a = 0; a < C::ATOMS; ++a)
+                tc::tma_load_3d(q_smem + a * C::BM * 128, &tmap_q, a * 64, kvh * g, q0 + tok0, bar_q);
+            const int32_t *bt = p.block_tables + (int64_t)s * p.max_blocks_per_seq;
+            int j = 0;
+            for (; j < nt; ++j) {
+                const int st = j % C::ST;
+                if (j >= C::ST &&
+                    !tc::wait_phase(bar_kv_empty(st), ((j / C::ST) - 1) & 1, abort_flag, p.err))
+                    break;
+                mbar_arrive_expect_tx(bar_kv_full(st), 2u * C::KV_BYTES);
+#pragma unroll 1
+                for (int b = 0; b < C::BN / kBlockSize; ++b) {
+                    const int lb = j * (C::BN / kBlockSize) + b;
+                    int y = p.oob_row;  // past the pool: a zero-filled box
+                    if (lb < nblk_seq) {
+                        const int phys = bt[lb];
+                        if ((unsigned)phys < (unsigned)p.num_blocks)
+                            y = (phys * p.num_kv_heads + kvh) * kBlockSize;
+                        else
+                            flag_error(p.err, kErrBounds);
+                    }
+#pragma unroll
+                    for (int a = 0; a < C::ATOMS; ++a) {
+                        const uint32_t off = a * C::BN * 128 + b * kBlockSize * 128;
+                        tc::tma_load_2d(k_smem(st) + off, &tmap_k, a * 64, y, bar_kv_full(st));
+                        tc::tma_load_2d(v_smem(st) + off, &tmap_v, a * 64, y, bar_kv_full(st));
+                    }
+                }
+            }
+            // nothing may still be landing in shared memory when the CTA exits
+            (void)mbar_wait_bounded(bar_q, 0, kWaitLimitNs);
+            for (int jj = j - C::ST < 0 ? 0 : j - C::ST; jj < j; ++jj)
+                (void)mbar_wait_bounded(bar_kv_full(jj % C::ST), (jj / C::ST) & 1, kWaitLimitNs);
+        }
+        __syncwarp();
+    } else if (warp == 5) {
+        // ================= MMA issuer ==============================================
+        bool ok = __all_sync(tc::kFull, tc::wait_phase(bar_q, 0, abort_flag, p.err));
+        auto issue_qk = [&](int j) {
+            const uint32_t kaddr = k_smem(j % C::ST);
+            const uint32_t d = tmem + ((j & 1) ? C::COL_S1 : C::COL_S0);
+            if (lane == 0) {
+                tc::fence_after();
+#pragma unroll
+                for (int ks = 0; ks < D / 16; ++ks) {
+                    const uint32_t off = (ks >> 2) * (C::BM * 128) + (ks & 3) * 32;
+                    tc::mma_ss(d, tc::sdesc(q_smem + off, 16, 1024), tc::sdesc(kaddr + off, 16, 1024),
+                               C::IDESC_QK, ks > 0);
+                }
+                tc::commit(bar_s_full(j & 1));
+            }
+            __syncwarp();
+        };
+        auto issue_pv = [&](int j) {
+            const int st = j % C::ST;
+            const uint32_t vaddr = v_smem(st);
+            const uint32_t pcol = tmem + ((j & 1) ? C::COL_S1 : C::COL_S0);
+            if (lane == 0) {
+                tc::fence_after();
+#pragma unroll
+                for (int ks = 0; ks < C::BN / 16; ++ks) {
+                    const uint64_t bdesc = tc::sdesc(vaddr + ks * 2048, C::BN * 128, 1024);
+                    tc::mma_ts(tmem + C::COL_O, pcol + ks * 8, bdesc, C::IDESC_PV, (j > 0 || ks > 0));
+                    if constexpr (C::HILO)
+                        tc::mma_ts(tmem + C::COL_O, pcol + 64 + ks * 8, bdesc, C::IDESC_PV, 1);
+                }
+                tc::commit(bar_pv);
+                tc::commit(bar_kv_empty(st));
+            }
+            __syncwarp();
+        };
+        const int j_tail = (L & (kBlockSize - 1)) ? (nblk_seq - 1) / (C::BN / kBlockSize) : -1;
+        for (int j = 0; ok && j < nt; ++j) {
+            const int st = j % C::ST;
+            ok = __all_sync(tc::kFull, tc::wait_phase(bar_kv_full(st), (j / C::ST) & 1, abort_flag, p.err));
+            if (!ok) break;
+            if (j == j_tail) {
+                // clear the V rows of the last block's unused slots (positions >= L)
+                const int r0 = L - j * C::BN, r1 = nblk_seq * kBlockSize - j * C::BN;
+                const int chunks = (r1 - r0) * C::ATOMS * 8;
+                for (int c = lane; c < chunks; c += 32) {
+                    const int row = r0 + c / (C::ATOMS * 8), rem = c % (C::ATOMS * 8);
+                    const uint32_t addr = v_smem(st) + (rem >> 3) * C::BN * 128 + row * 128 + (rem & 7) * 16;
+                    asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(addr), "r"(0u) : "memory");
+                }
+                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                __syncwarp();
+            }
+            issue_qk(j);
+            if (j >= 1) {
+                ok = __all_sync(tc::kFull,
+                                tc::wait_phase(bar_p_full((j - 1) & 1), ((j - 1) >> 1) & 1, abort_flag, p.err));
+                if (!ok) break;
+                issue_pv(j - 1);
+            }
+        }
+        if (ok) {
+            ok = __all_sync(tc::kFull,
+                            tc::wait_phase(bar_p_full((nt - 1) & 1), ((nt - 1) >> 1) & 1, abort_flag, p.err));
+            if (ok) issue_pv(nt - 1);
+        }
+        // every MMA of this thread must be complete before TMEM is freed
+        if (lane == 0) {
+            tc::commit(bar_drain);
+            (void)mbar_wait_bounded(bar_drain, 0, kWaitLimitNs);
+        }
+        __syncwarp();
+    } else {
+        // ================= softmax: one thread per query row =======================
+        const int r = threadIdx.x;  // 0..127 = TMEM lane
+        const int rtok = r / g;
+        const bool row_ok = r < tpt * g && rtok < ntok;
+        const int pos = ctx + tok0 + rtok;
+        const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
+        const float sl2 = p.qk_scale_log2;
+        float m_ref = -CUDART_INF_F, l = 0.f;
+        bool ok = true;
+        for (int j = 0; j < nt; ++j) {
+            ok = __all_sync(tc::kFull, tc::wait_phase(bar_s_full(j & 1), (j >> 1) & 1, abort_flag, p.err));
+            if (!ok) break;
+            tc::fence_after();
+            const uint32_t scol = lane_base + ((j & 1) ? C::COL_S1 : C::COL_S0);
+            uint32_t raw_s[C::BN];
+#pragma unroll
+            for (int c = 0; c < C::BN; c += 32) tc::ld32(scol + c, raw_s + c);
+            tc::wait_ld<C::BN>(raw_s);
+            const int lim = row_ok ? pos - j * C::BN + 1 : 0;  // keys of this tile the row sees
+            float x[C::BN];
+            float mx = -CUDART_INF_F;
+#pragma unroll
+            for (int c = 0; c < C::BN; ++c) {
+                x[c] = c < lim ? __uint_as_float(raw_s[c]) * sl2 : -CUDART_INF_F;
+                mx = fmaxf(mx, x[c]);
+            }
+            // lazy rescale: move the reference max only when it grows by > 8
+            float alpha = 1.f;
+            const bool grow = mx > m_ref + 8.f;
+            if (grow) {
+                alpha = m_ref == -CUDART_INF_F ? 0.f : exp2f(m_ref - mx);
+                m_ref = mx;
+            }
+            const float mb = m_ref == -CUDART_INF_F ? 0.f : m_ref;
+            l *= alpha;
+            float psum = 0.f;
+#pragma unroll
+            for (int c0 = 0; c0 < C::BN; c0 += 32) {
+                uint32_t hi[16], lo[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    const float p0 = exp2f(x[c0 + 2 * i] - mb), p1 = exp2f(x[c0 + 2 * i + 1] - mb);
+                    psum += p0 + p1;
+                    hi[i] = tc::pack2(p0, p1, T{});
+                    if constexpr (C::HILO) {
+                        float h0, h1;
+                        tc::unpack2(hi[i], h0, h1, bf16_t{});
+                        lo[i] = tc::pack2(p0 - h0, p1 - h1, T{});
+                    }
+                }
+                tc::st16(scol + c0 / 2, hi);
+                if constexpr (C::HILO) tc::st16(scol + C::BN / 2 + c0 / 2, lo);
+            }
+            l += psum;
+            if (j > 0) {
+                // O may be touched only once the previous P.V is complete
+                ok = __all_sync(tc::kFull, tc::wait_phase(bar_pv, (j - 1) & 1, abort_flag, p.err));
+                if (!ok) break;
+                if (__any_sync(tc::kFull, grow)) {
+                    tc::fence_after();
+#pragma unroll
+                    for (int c = 0; c < D; c += 32) {
+                        uint32_t o[32];
+                        tc::ld32(lane_base + C::COL_O + c, o);
+                        tc::wait_ld<32>(o);
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+                        tc::st32(lane_base + C::COL_O + c, o);
+                    }
+                }
+            }
+            tc::wait_st();
+            tc::fence_before();
+            tc::mbar_arrive(bar_p_full(j & 1));
+        }
+        if (ok) ok = __all_sync(tc::kFull, tc::wait_phase(bar_pv, (nt - 1) & 1, abort_flag, p.err));
+        if (ok) {
+            // ---- epilogue: out = O / l, rounded once to the q dtype ----------------
+            tc::fence_after();
+            const float inv = l > 0.f ? 1.f / l : 0.f;
+            const int64_t row = ((int64_t)(q0 + tok0 + rtok) * p.num_q_heads + (int64_t)kvh * g + r % g);
+            uint4 *dst = reinterpret_cast<uint4 *>(static_cast<uint16_t *>(p.out) + row * D);
+#pragma unroll
+            for (int c = 0; c < D; c += 32) {
+                uint32_t o[32];
+                tc::ld32(lane_base + C::COL_O + c, o);
+                tc::wait_ld<32>(o);
+                uint32_t w[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i)
+                    w[i] = tc::pack2(__uint_as_float(o[2 * i]) * inv, __uint_as_float(o[2 * i + 1]) * inv, T{});
+                if (row_ok) {
+#pragma unroll
+                    for (int v = 0; v < 4; ++v)
+                        dst[c / 8 + v] = make_uint4(w[4 * v], w[4 * v + 1], w[4 * v + 2], w[4 * v + 3]);
+                }
+            }
+        }
+    }
+
+    // ---- teardown: every role is done with TMEM --------------------------------
+    tc::fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc::fence_after();
+        tc::dealloc(tmem, C::TMEM_COLS);
+    }
+}
+
+// ---------------------------------------------------------------------------
+// host side
+// ---------------------------------------------------------------------------
+
+namespace {
+
+// q [T, Hq, d] as a 3-D map (d, Hq, T); a box is 64 elements (128 bytes) x g
+// heads x tpt tokens, 128-byte swizzle, so a box lands as tpt * g rows of
+// 128 bytes in row order (token, head).
+bool encode_q_map(CUtensorMap *m, const void *q, int d, int hq, int64_t tokens, int g, int tpt) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)hq, (cuuint64_t)tokens};
+    const cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)hq * d * 2};
+    const cuuint32_t box[3] = {64, (cuuint32_t)g, (cuuint32_t)tpt};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT16, 3, const_cast<void *>(q), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <typename T, int D>
+cudaError_t launch_prefill_t(const PrefillParams &p, cudaStream_t stream) {
+    using C = PfCfg<T, D>;
+    const int64_t rows = (int64_t)p.num_blocks * p.num_kv_heads * kBlockSize;
+    CUtensorMap mq, mk, mv;
+    if (!encode_q_map(&mq, p.q, D, p.num_q_heads, p.num_tokens, p.group, p.tok_per_tile) ||
+        !encode_pool_map(&mk, p.k_cache, 2, D, rows) || !encode_pool_map(&mv, p.v_cache, 2, D, rows))
+        return cudaErrorInvalidValue;
+    auto kern = prefill_kernel<T, D>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+    if (e != cudaSuccess) return e;
+    const dim3 grid((unsigned)((p.max_query_len + p.tok_per_tile - 1) / p.tok_per_tile),
+                    (unsigned)p.num_kv_heads, (unsigned)p.num_seqs);
+    kern<<<grid, 192, C::SMEM, stream>>>(p, mq, mk, mv);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+bool prefill_supported() { return encode_fn() != nullptr; }
+
+cudaError_t launch_prefill(const PrefillParams &p, DType q, int head_dim, cudaStream_t stream) {
+    if (p.num_seqs <= 0 || p.num_tokens <= 0 || p.max_query_len <= 0) return cudaSuccess;
+    if (q == DType::F16)
+        return head_dim == 64 ? launch_prefill_t<f16_t, 64>(p, stream) : launch_prefill_t<f16_t, 128>(p, stream);
+    return head_dim == 64 ? launch_prefill_t<bf16_t, 64>(p, stream) : launch_prefill_t<bf16_t, 128>(p, stream);
+}
+
+}  // namespace pa

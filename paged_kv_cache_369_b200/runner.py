@@ -19,7 +19,7 @@ from typing import Optional
 import numpy as np
 import torch
 
-from . import (pa_cache_write, pa_decode, pa_decode_append, pa_decode_split_reduce,
+from . import (pa_cache_write, pa_decode, pa_decode_append, pa_decode_split_reduce, pa_prefill,
                pa_slot_mapping, pa_split_workspace_bytes)
 
 _TORCH_ACT = {"f16": torch.float16, "bf16": torch.bfloat16}
@@ -148,3 +148,74 @@ def algorithmic_decode_bytes(w) -> int:
     S, Hq, d = w.num_seqs, w.num_q_heads, w.head_dim
     return w.kv_bytes_logical() + 2 * S * Hq * d * 2 + int(sum(
         math.ceil(int(L) / w.block_size) for L in w.seq_lens)) * 4 + S * 4
+
+
+class PagedPrefill:
+    """One chunked-prefill step resident on a GPU (any object with the
+    attributes of ``workload.ChunkedWorkload``).  The context tokens are
+    written into 0xFF-poisoned pools at construction; ``step()`` appends the
+    chunk's K/V rows (pa_slot_mapping with token positions + pa_cache_write)
+    and runs pa_prefill."""
+
+    def __init__(self, w, device: str = "cuda", stream: Optional[torch.cuda.Stream] = None):
+        self.w = w
+        self.device = torch.device(device)
+        self.stream = stream
+        dev = self.device
+        act = _TORCH_ACT[w.act_dtype]
+        T = w.num_tokens
+        self.q = _bits_to_device(w.q, w.act_dtype, dev)
+        self.k_chunk = _bits_to_device(w.k_chunk, w.act_dtype, dev)
+        self.v_chunk = _bits_to_device(w.v_chunk, w.act_dtype, dev)
+        self.chunk_seq = torch.from_numpy(np.ascontiguousarray(w.chunk_seq)).to(dev)
+        self.chunk_pos = torch.from_numpy(np.ascontiguousarray(w.chunk_pos)).to(dev)
+        self.block_tables = torch.from_numpy(np.ascontiguousarray(w.block_tables)).to(dev)
+        self.seq_lens = torch.from_numpy(np.ascontiguousarray(w.seq_lens)).to(dev)
+        self.query_start = torch.from_numpy(np.ascontiguousarray(w.query_start)).to(dev)
+        shape = (w.num_blocks, w.num_kv_heads, w.block_size, w.head_dim)
+        self.k_cache = torch.empty(shape, dtype=act, device=dev)
+        self.v_cache = torch.empty(shape, dtype=act, device=dev)
+        self.k_cache.view(torch.uint8).fill_(0xFF)
+        self.v_cache.view(torch.uint8).fill_(0xFF)
+        self.slots = torch.empty(max(T, 1), dtype=torch.int64, device=dev)
+        self.out = torch.empty((T, w.num_q_heads, w.head_dim), dtype=act, device=dev)
+        self.dev_err = torch.zeros(1, dtype=torch.int32, device=dev)
+        self._write(w.ctx_seq, w.ctx_pos, w.k_ctx, w.v_ctx)
+        torch.cuda.synchronize(dev)
+
+    def _write(self, seq, pos, kr, vr) -> None:
+        w, dev = self.w, self.device
+        for lo in range(0, int(seq.size), _UPLOAD_CHUNK_TOKENS):
+            hi = min(int(seq.size), lo + _UPLOAD_CHUNK_TOKENS)
+            tseq = torch.from_numpy(seq[lo:hi]).to(dev)
+            tpos = torch.from_numpy(pos[lo:hi]).to(dev)
+            kn = _bits_to_device(kr[lo:hi], w.act_dtype, dev)
+            vn = _bits_to_device(vr[lo:hi], w.act_dtype, dev)
+            slots = torch.empty(hi - lo, dtype=torch.int64, device=dev)
+            pa_slot_mapping(slots, self.block_tables, self.seq_lens, tseq, tpos, hi - lo,
+                            w.num_seqs, w.num_blocks, w.block_size, self.dev_err, self.stream)
+            pa_cache_write(kn, vn, self.k_cache, self.v_cache, slots, w.k_scale, w.v_scale,
+                           self.dev_err, self.stream)
+
+    def write_chunk(self) -> None:
+        w = self.w
+        T = w.num_tokens
+        if T == 0:
+            return
+        pa_slot_mapping(self.slots, self.block_tables, self.seq_lens, self.chunk_seq,
+                        self.chunk_pos, T, w.num_seqs, w.num_blocks, w.block_size, self.dev_err,
+                        self.stream)
+        pa_cache_write(self.k_chunk, self.v_chunk, self.k_cache, self.v_cache, self.slots,
+                       w.k_scale, w.v_scale, self.dev_err, self.stream)
+
+    def attend(self) -> None:
+        w = self.w
+        pa_prefill(self.out, self.q, self.k_cache, self.v_cache, self.block_tables, self.seq_lens,
+                   self.query_start, w.max_query_len, w.softmax_scale, self.dev_err, self.stream)
+
+    def step(self) -> None:
+        self.write_chunk()
+        self.attend()
+
+    def error(self) -> int:
+        return int(self.dev_err.item())

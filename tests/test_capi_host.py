@@ -176,3 +176,26 @@ def test_copy_blocks_checks(pa):
     assert call(k=0) == 1
     assert call(v=A + 8) == 1         # misaligned pool
     assert call(n=0, pairs=0, k=0, v=0) == 0   # nothing to copy
+
+
+def test_prefill_checks(pa):
+    L = pa.lib()
+
+    def call(out=A, q=A, qs=A, S=2, T=8, mq=4, Hq=8, Hk=2, d=128, B=16, NB=10, qd=pa.PA_BF16,
+             kvd=pa.PA_BF16, scale=0.1):
+        return L.pa_prefill(out, q, A, A, A, 4, A, qs, S, T, mq, Hq, Hk, d, B, NB, scale, qd, kvd,
+                            None, None)
+
+    assert call(kvd=pa.PA_FP8_E4M3) == 2     # E4M3 caches: not on the prefill path
+    assert call(qd=pa.PA_F16) == 2           # cache dtype must be the q dtype
+    assert call(d=96) == 2
+    assert call(B=32) == 2
+    assert call(Hq=8, Hk=3) == 1
+    assert call(Hq=256, Hk=1) == 2           # group above 128
+    assert call(qs=0) == 1
+    assert call(out=A + 4) == 1
+    assert call(mq=0) == 1
+    assert call(S=-1) == 1
+    assert call(scale=float("nan")) == 1
+    assert call(S=0, q=0) == 0               # nothing to do
+    assert call(T=0, q=0) == 0
