@@ -12,26 +12,30 @@
 // KV Cache、PagedAttention 与 vLLM", §3.3).  A decode step is the one-token
 // chunk.
 //
-// Work decomposition: one CTA per (sequence, KV head, query tile).  A query
-// tile is 128 rows = floor(128 / g) chunk tokens x the g query heads of the
-// KV head (row r: token r / g, head r % g), so the whole GQA group shares each
-// K/V tile it reads.  Keys come in tiles of 128 = 8 blocks of 16 tokens.
-//   - warp 4 (one lane), TMA producer: the Q tile once through a 3-D tensor
-//     map over q [T, Hq, d]; per key tile, the 8 K and 8 V blocks named by the
-//     block table through the pool's 2-D map (16-row x 128-byte boxes, 128B
-//     swizzle) into a 2-stage ring.  Blocks past the sequence's end are
+// Work decomposition: one CTA per (sequence, KV head, pair of query tiles).
+// A query tile is 128 rows = floor(128 / g) chunk tokens x the g query heads
+// of the KV head (row r: token r / g, head r % g), so the whole GQA group
+// shares each K/V tile it reads; the CTA's two tiles (A, B: consecutive token
+// ranges) share them too.  Keys come in tiles of 128 = 8 blocks of 16 tokens.
+//   - warp 8 (one lane), TMA producer: both Q tiles once through a 3-D
+//     tensor map over q [T, Hq, d]; per key tile, the 8 K and 8 V blocks named
+//     by the block table through the pool's 2-D map (16-row x 128-byte boxes,
+//     128B swizzle) into a 2-stage ring.  Blocks past the sequence's end are
 //     fetched from past the end of the map, which the copy fills with zeros.
-//   - warp 5 (one lane), MMA issuer: S_j = Q K_j^T (M 128, N 128, K d) into
-//     one of two TMEM buffers; O += P_j V_j with A = P read from TMEM and
-//     B = V from shared memory (MN-major).  Issue order QK_0, QK_1, PV_0,
-//     QK_2, PV_1, ...: the tensor cores compute the next scores while the
-//     softmax works on the current ones; tcgen05 operations of one thread
-//     run in issue order, which makes the buffer reuse safe.
-//   - warps 0-3, one thread per row: S_j from TMEM, causal mask by select,
-//     online softmax with a lazy rescale (O and l are rescaled only when the
-//     row max grows by more than 8 in log2 units; otherwise p is taken
-//     against the old max, at most 2^8), P written back over S_j (bf16 as
-//     hi + lo halves so P keeps ~16 bits; f16 as one half), O / l at the end.
+//   - warp 9 (one lane), MMA issuer: S_t = Q_t K_j^T (M 128, N 128, K d) into
+//     tile t's TMEM columns; O_t += P_t V_j with A = P read from TMEM and
+//     B = V from shared memory (MN-major).  Issue order per key tile j:
+//     PV_A(j), QK_A(j+1), PV_B(j), QK_B(j+1) -- while one tile's softmax
+//     runs, the tensor cores work on the other tile (ping-pong); tcgen05
+//     operations of one thread run in issue order, which makes reusing S_t's
+//     columns for P_t and then for the next S_t safe.
+//   - warps 0-3 (tile A) and 4-7 (tile B), one thread per row: S from TMEM,
+//     causal mask by select on the diagonal tile only, the scale folded into
+//     one FFMA before ex2, online softmax with a lazy rescale (O and l are
+//     rescaled only when the row max grows by more than 8 in log2 units;
+//     otherwise p is taken against the old max, at most 2^8), P written back
+//     over S (bf16 as hi + lo halves so P keeps ~16 bits; f16 as one half),
+//     O / l at the end.
 // V rows past the sequence's last token (the tail of its last block) are
 // cleared in shared memory before P.V: p = 0 there, but 0 x NaN poison = NaN.
 // Every wait is bounded; a timeout reports PA_ERR_DEVICE_TIMEOUT, makes the
@@ -196,17 +200,17 @@ __device__ __forceinline__ void unpack2(uint32_t w, float &lo, float &hi, bf16_t
 }  // namespace tc
 
 template <typename T, int D> struct PfCfg {
-    static constexpr int BM = 128;  // query rows per tile (TMEM lanes)
+    static constexpr int BM = 128;  // query rows per tile (TMEM lanes); two tiles per CTA
     static constexpr int BN = 128;  // keys per tile = 8 blocks
     static constexpr int ST = 2;    // K/V ring stages
     static constexpr int ATOMS = D / 64;  // 128-byte swizzle atoms across d
-    static constexpr int Q_BYTES = ATOMS * BM * 128;
+    static constexpr int Q_BYTES = ATOMS * BM * 128;  // one query tile
     static constexpr int KV_BYTES = ATOMS * BN * 128;
-    static constexpr int OFF_Q = 0;
-    static constexpr int OFF_KV = Q_BYTES;  // stage st: K, then V
+    static constexpr int OFF_Q = 0;                   // tile A, then tile B
+    static constexpr int OFF_KV = 2 * Q_BYTES;        // stage st: K, then V
     static constexpr int OFF_BAR = OFF_KV + ST * 2 * KV_BYTES;
-    // q_full, kv_full[ST], kv_empty[ST], s_full[2], p_full[2], pv_done, drain
-    static constexpr int NBAR = 1 + 2 * ST + 2 + 2 + 1 + 1;
+    // q_full, kv_full[ST], kv_empty[ST], s_full[2], p_full[2], pv_done[2], drain
+    static constexpr int NBAR = 1 + 2 * ST + 2 + 2 + 2 + 1;
     static constexpr int OFF_SLOT = OFF_BAR + NBAR * 8;
     static constexpr int OFF_ABORT = OFF_SLOT + 4;
     static constexpr int USED = OFF_ABORT + 4;
@@ -214,19 +218,27 @@ template <typename T, int D> struct PfCfg {
     static constexpr int SMEM = 1024 + (USED < 120 * 1024 ? 120 * 1024 : USED);
     static constexpr bool HILO = std::is_same<T, bf16_t>::value;
     static constexpr uint32_t TMEM_COLS = 512;
-    static constexpr uint32_t COL_S0 = 0, COL_S1 = 128, COL_O = 256;
+    // S of tile t at column 128 t (P written over it), O of tile t at 256 + 128 t
+    static constexpr uint32_t COL_S = 0, COL_O = 256;
     static constexpr uint32_t FMT = HILO ? 1u : 0u;  // kind::f16 operand format: f16 0, bf16 1
     // instruction descriptors: fp32 accumulate, A/B format, majors, N >> 3, M >> 4
     static constexpr uint32_t IDESC_QK = (1u << 4) | (FMT << 7) | (FMT << 10) |
                                          ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
     static constexpr uint32_t IDESC_PV = (1u << 4) | (FMT << 7) | (FMT << 10) | (1u << 16) |
                                          ((uint32_t)(D >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
+    static constexpr int THREADS = 320;  // 8 softmax warps, a TMA warp, an MMA warp
     static_assert(D == 64 || D == 128, "head_dim 64 or 128");
     static_assert(SMEM <= 227 * 1024, "shared memory budget");
 };
 
+__device__ __forceinline__ float ex2(float x) {  // 2^x; -inf -> +0
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
 template <typename T, int D>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(320, 1)
     prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tmap_q,
                    const __grid_constant__ CUtensorMap tmap_k,
                    const __grid_constant__ CUtensorMap tmap_v) {
@@ -236,7 +248,7 @@ __global__ void __launch_bounds__(192, 1)
     const uint32_t base = (raw + 1023u) & ~1023u;
     uint8_t *smem = smem_raw + (base - raw);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int tile = blockIdx.x, kvh = blockIdx.y, s = blockIdx.z;
+    const int cta_tile = blockIdx.x, kvh = blockIdx.y, s = blockIdx.z;
     const int g = p.group, tpt = p.tok_per_tile;
 
     // ---- this CTA's rows and keys (uniform over the CTA) ---------------------
@@ -245,12 +257,12 @@ __global__ void __launch_bounds__(192, 1)
     const int n = p.query_start[s + 1] - q0;
     if (L < 0 || L > p.max_blocks_per_seq * kBlockSize || n < 0 || n > L || q0 < 0 ||
         q0 + n > p.num_tokens || n > p.max_query_len) {
-        if (threadIdx.x == 0 && tile == 0 && kvh == 0) flag_error(p.err, kErrBounds);
+        if (threadIdx.x == 0 && cta_tile == 0 && kvh == 0) flag_error(p.err, kErrBounds);
         return;
     }
-    const int tok0 = tile * tpt;
+    const int tok0 = cta_tile * 2 * tpt;  // query tile A: tok0 .., tile B: tok0 + tpt ..
     if (tok0 >= n) return;
-    const int ntok = min(tpt, n - tok0);
+    const int ntok = min(2 * tpt, n - tok0);
     const int ctx = L - n;
     const int nt = (ctx + tok0 + ntok - 1) / C::BN + 1;  // key tiles up to the last row's position
     const int nblk_seq = (L + kBlockSize - 1) / kBlockSize;
@@ -259,10 +271,10 @@ __global__ void __launch_bounds__(192, 1)
     const uint32_t bar_q = bars;
     auto bar_kv_full = [&](int st) { return bars + 8u * (1 + st); };
     auto bar_kv_empty = [&](int st) { return bars + 8u * (1 + C::ST + st); };
-    auto bar_s_full = [&](int b) { return bars + 8u * (1 + 2 * C::ST + b); };
-    auto bar_p_full = [&](int b) { return bars + 8u * (3 + 2 * C::ST + b); };
-    const uint32_t bar_pv = bars + 8u * (5 + 2 * C::ST);
-    const uint32_t bar_drain = bar_pv + 8u;
+    auto bar_s_full = [&](int t) { return bars + 8u * (1 + 2 * C::ST + t); };
+    auto bar_p_full = [&](int t) { return bars + 8u * (3 + 2 * C::ST + t); };
+    auto bar_pv = [&](int t) { return bars + 8u * (5 + 2 * C::ST + t); };
+    const uint32_t bar_drain = bars + 8u * (7 + 2 * C::ST);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + C::OFF_ABORT);
     uint32_t *slot = reinterpret_cast<uint32_t *>(smem + C::OFF_SLOT);
 
@@ -274,11 +286,11 @@ __global__ void __launch_bounds__(192, 1)
             mbar_init(bar_kv_empty(st), 1);
         }
 #pragma unroll
-        for (int b = 0; b < 2; ++b) {
-            mbar_init(bar_s_full(b), 1);
-            mbar_init(bar_p_full(b), 128);
+        for (int t = 0; t < 2; ++t) {
+            mbar_init(bar_s_full(t), 1);
+            mbar_init(bar_p_full(t), 128);
+            mbar_init(bar_pv(t), 1);
         }
-        mbar_init(bar_pv, 1);
         mbar_init(bar_drain, 1);
         *abort_flag = 0;
         mbar_init_fence();
@@ -289,20 +301,23 @@ __global__ void __launch_bounds__(192, 1)
     tc::fence_after();
     const uint32_t tmem = *slot;
 
-    const uint32_t q_smem = base + C::OFF_Q;
+    auto q_smem = [&](int t) { return base + C::OFF_Q + (uint32_t)(t * C::Q_BYTES); };
     auto k_smem = [&](int st) { return base + C::OFF_KV + (uint32_t)(st * 2 * C::KV_BYTES); };
     auto v_smem = [&](int st) { return k_smem(st) + (uint32_t)C::KV_BYTES; };
 
-    if (warp == 4) {
+    if (warp == 8) {
         // ================= TMA producer ===========================================
         if (lane == 0) {
             asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_q)) : "memory");
             asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_k)) : "memory");
             asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_v)) : "memory");
-            mbar_arrive_expect_tx(bar_q, (uint32_t)(C::ATOMS * tpt * g * 128));
+            mbar_arrive_expect_tx(bar_q, (uint32_t)(2 * C::ATOMS * tpt * g * 128));
 #pragma unroll
-            for (int a = 0; a < C::ATOMS; ++a)
-                tc::tma_load_3d(q_smem + a * C::BM * 128, &tmap_q, a * 64, kvh * g, q0 + tok0, bar_q);
+            for (int t = 0; t < 2; ++t)
+#pragma unroll
+                for (int a = 0; a < C::ATOMS; ++a)
+                    tc::tma_load_3d(q_smem(t) + a * C::BM * 128, &tmap_q, a * 64, kvh * g,
+                                    q0 + tok0 + t * tpt, bar_q);
             const int32_t *bt = p.block_tables + (int64_t)s * p.max_blocks_per_seq;
             int j = 0;
             for (; j < nt; ++j) {
@@ -336,47 +351,49 @@ __global__ void __launch_bounds__(192, 1)
                 (void)mbar_wait_bounded(bar_kv_full(jj % C::ST), (jj / C::ST) & 1, kWaitLimitNs);
         }
         __syncwarp();
-    } else if (warp == 5) {
+    } else if (warp == 9) {
         // ================= MMA issuer ==============================================
-        bool ok = __all_sync(tc::kFull, tc::wait_phase(bar_q, 0, abort_flag, p.err));
-        auto issue_qk = [&](int j) {
-            const uint32_t kaddr = k_smem(j % C::ST);
-            const uint32_t d = tmem + ((j & 1) ? C::COL_S1 : C::COL_S0);
+        // order per key tile j: PV_A(j), QK_A(j+1), PV_B(j), QK_B(j+1); the two
+        // query tiles ping-pong, so one tile's softmax overlaps the other's MMAs
+        auto issue_qk = [&](int t, int j) {
+            const uint32_t kaddr = k_smem(j % C::ST), qaddr = q_smem(t);
+            const uint32_t d = tmem + C::COL_S + 128u * t;
             if (lane == 0) {
                 tc::fence_after();
 #pragma unroll
                 for (int ks = 0; ks < D / 16; ++ks) {
                     const uint32_t off = (ks >> 2) * (C::BM * 128) + (ks & 3) * 32;
-                    tc::mma_ss(d, tc::sdesc(q_smem + off, 16, 1024), tc::sdesc(kaddr + off, 16, 1024),
+                    tc::mma_ss(d, tc::sdesc(qaddr + off, 16, 1024), tc::sdesc(kaddr + off, 16, 1024),
                                C::IDESC_QK, ks > 0);
                 }
-                tc::commit(bar_s_full(j & 1));
+                tc::commit(bar_s_full(t));
             }
             __syncwarp();
         };
-        auto issue_pv = [&](int j) {
-            const int st = j % C::ST;
-            const uint32_t vaddr = v_smem(st);
-            const uint32_t pcol = tmem + ((j & 1) ? C::COL_S1 : C::COL_S0);
+        auto issue_pv = [&](int t, int j) {
+            const uint32_t vaddr = v_smem(j % C::ST);
+            const uint32_t pcol = tmem + C::COL_S + 128u * t;
+            const uint32_t ocol = tmem + C::COL_O + 128u * t;
             if (lane == 0) {
                 tc::fence_after();
 #pragma unroll
                 for (int ks = 0; ks < C::BN / 16; ++ks) {
                     const uint64_t bdesc = tc::sdesc(vaddr + ks * 2048, C::BN * 128, 1024);
-                    tc::mma_ts(tmem + C::COL_O, pcol + ks * 8, bdesc, C::IDESC_PV, (j > 0 || ks > 0));
-                    if constexpr (C::HILO)
-                        tc::mma_ts(tmem + C::COL_O, pcol + 64 + ks * 8, bdesc, C::IDESC_PV, 1);
+                    tc::mma_ts(ocol, pcol + ks * 8, bdesc, C::IDESC_PV, (j > 0 || ks > 0));
+                    if constexpr (C::HILO) tc::mma_ts(ocol, pcol + 64 + ks * 8, bdesc, C::IDESC_PV, 1);
                 }
-                tc::commit(bar_pv);
-                tc::commit(bar_kv_empty(st));
+                tc::commit(bar_pv(t));
+                if (t == 1) tc::commit(bar_kv_empty(j % C::ST));  // last reader of the stage
             }
             __syncwarp();
         };
+        auto wait_all = [&](uint32_t bar, uint32_t parity) {
+            return __all_sync(tc::kFull, tc::wait_phase(bar, parity, abort_flag, p.err));
+        };
         const int j_tail = (L & (kBlockSize - 1)) ? (nblk_seq - 1) / (C::BN / kBlockSize) : -1;
-        for (int j = 0; ok && j < nt; ++j) {
+        auto kv_ready = [&](int j) {
             const int st = j % C::ST;
-            ok = __all_sync(tc::kFull, tc::wait_phase(bar_kv_full(st), (j / C::ST) & 1, abort_flag, p.err));
-            if (!ok) break;
+            if (!wait_all(bar_kv_full(st), (j / C::ST) & 1)) return false;
             if (j == j_tail) {
                 // clear the V rows of the last block's unused slots (positions >= L)
                 const int r0 = L - j * C::BN, r1 = nblk_seq * kBlockSize - j * C::BN;
@@ -389,18 +406,27 @@ __global__ void __launch_bounds__(192, 1)
                 asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
                 __syncwarp();
             }
-            issue_qk(j);
-            if (j >= 1) {
-                ok = __all_sync(tc::kFull,
-                                tc::wait_phase(bar_p_full((j - 1) & 1), ((j - 1) >> 1) & 1, abort_flag, p.err));
-                if (!ok) break;
-                issue_pv(j - 1);
-            }
-        }
+            return true;
+        };
+        bool ok = wait_all(bar_q, 0) && kv_ready(0);
         if (ok) {
-            ok = __all_sync(tc::kFull,
-                            tc::wait_phase(bar_p_full((nt - 1) & 1), ((nt - 1) >> 1) & 1, abort_flag, p.err));
-            if (ok) issue_pv(nt - 1);
+            issue_qk(0, 0);
+            issue_qk(1, 0);
+        }
+        for (int j = 0; ok && j < nt; ++j) {
+            ok = wait_all(bar_p_full(0), j & 1);
+            if (!ok) break;
+            issue_pv(0, j);
+            const bool more = j + 1 < nt;
+            if (more) {
+                ok = kv_ready(j + 1);
+                if (!ok) break;
+                issue_qk(0, j + 1);
+            }
+            ok = wait_all(bar_p_full(1), j & 1);
+            if (!ok) break;
+            issue_pv(1, j);
+            if (more) issue_qk(1, j + 1);
         }
         // every MMA of this thread must be complete before TMEM is freed
         if (lane == 0) {
@@ -410,48 +436,54 @@ __global__ void __launch_bounds__(192, 1)
         __syncwarp();
     } else {
         // ================= softmax: one thread per query row =======================
-        const int r = threadIdx.x;  // 0..127 = TMEM lane
-        const int rtok = r / g;
+        const int t = warp >> 2;                  // query tile (0: A, 1: B)
+        const int r = (warp & 3) * 32 + lane;     // row = TMEM lane
+        const int rtok = t * tpt + r / g;         // token within the CTA's range
         const bool row_ok = r < tpt * g && rtok < ntok;
         const int pos = ctx + tok0 + rtok;
-        const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
-        const float sl2 = p.qk_scale_log2;
+        const uint32_t lane_bits = (uint32_t)((warp & 3) * 32) << 16;
+        const uint32_t scol = tmem + lane_bits + C::COL_S + 128u * t;
+        const uint32_t ocol = tmem + lane_bits + C::COL_O + 128u * t;
+        const float sl2 = p.qk_scale_log2;  // > 0
         float m_ref = -CUDART_INF_F, l = 0.f;
         bool ok = true;
         for (int j = 0; j < nt; ++j) {
-            ok = __all_sync(tc::kFull, tc::wait_phase(bar_s_full(j & 1), (j >> 1) & 1, abort_flag, p.err));
+            ok = __all_sync(tc::kFull, tc::wait_phase(bar_s_full(t), j & 1, abort_flag, p.err));
             if (!ok) break;
             tc::fence_after();
-            const uint32_t scol = lane_base + ((j & 1) ? C::COL_S1 : C::COL_S0);
-            uint32_t raw_s[C::BN];
+            uint32_t sv[C::BN];
 #pragma unroll
-            for (int c = 0; c < C::BN; c += 32) tc::ld32(scol + c, raw_s + c);
-            tc::wait_ld<C::BN>(raw_s);
-            const int lim = row_ok ? pos - j * C::BN + 1 : 0;  // keys of this tile the row sees
-            float x[C::BN];
-            float mx = -CUDART_INF_F;
+            for (int c = 0; c < C::BN; c += 32) tc::ld32(scol + c, sv + c);
+            tc::wait_ld<C::BN>(sv);
+            // keys of this tile the row may see: all, a prefix (diagonal tile), none
+            const int lim = row_ok ? pos - j * C::BN + 1 : 0;
+            if (lim < C::BN) {
 #pragma unroll
-            for (int c = 0; c < C::BN; ++c) {
-                x[c] = c < lim ? __uint_as_float(raw_s[c]) * sl2 : -CUDART_INF_F;
-                mx = fmaxf(mx, x[c]);
+                for (int c = 0; c < C::BN; ++c)
+                    if (c >= lim) sv[c] = __float_as_uint(-CUDART_INF_F);
             }
+            float m4[4] = {-CUDART_INF_F, -CUDART_INF_F, -CUDART_INF_F, -CUDART_INF_F};
+#pragma unroll
+            for (int c = 0; c < C::BN; ++c) m4[c & 3] = fmaxf(m4[c & 3], __uint_as_float(sv[c]));
+            const float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * sl2;
             // lazy rescale: move the reference max only when it grows by > 8
             float alpha = 1.f;
             const bool grow = mx > m_ref + 8.f;
             if (grow) {
-                alpha = m_ref == -CUDART_INF_F ? 0.f : exp2f(m_ref - mx);
+                alpha = m_ref == -CUDART_INF_F ? 0.f : ex2(m_ref - mx);
                 m_ref = mx;
             }
-            const float mb = m_ref == -CUDART_INF_F ? 0.f : m_ref;
+            const float nmb = m_ref == -CUDART_INF_F ? 0.f : -m_ref;
             l *= alpha;
-            float psum = 0.f;
+            float ps[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
             for (int c0 = 0; c0 < C::BN; c0 += 32) {
                 uint32_t hi[16], lo[16];
 #pragma unroll
                 for (int i = 0; i < 16; ++i) {
-                    const float p0 = exp2f(x[c0 + 2 * i] - mb), p1 = exp2f(x[c0 + 2 * i + 1] - mb);
-                    psum += p0 + p1;
+                    const float p0 = ex2(fmaf(__uint_as_float(sv[c0 + 2 * i]), sl2, nmb));
+                    const float p1 = ex2(fmaf(__uint_as_float(sv[c0 + 2 * i + 1]), sl2, nmb));
+                    ps[i & 3] += p0 + p1;
                     hi[i] = tc::pack2(p0, p1, T{});
                     if constexpr (C::HILO) {
                         float h0, h1;
@@ -462,29 +494,29 @@ __global__ void __launch_bounds__(192, 1)
                 tc::st16(scol + c0 / 2, hi);
                 if constexpr (C::HILO) tc::st16(scol + C::BN / 2 + c0 / 2, lo);
             }
-            l += psum;
+            l += (ps[0] + ps[1]) + (ps[2] + ps[3]);
             if (j > 0) {
-                // O may be touched only once the previous P.V is complete
-                ok = __all_sync(tc::kFull, tc::wait_phase(bar_pv, (j - 1) & 1, abort_flag, p.err));
+                // O may be touched only once the previous P.V of this tile is complete
+                ok = __all_sync(tc::kFull, tc::wait_phase(bar_pv(t), (j - 1) & 1, abort_flag, p.err));
                 if (!ok) break;
                 if (__any_sync(tc::kFull, grow)) {
                     tc::fence_after();
 #pragma unroll
                     for (int c = 0; c < D; c += 32) {
                         uint32_t o[32];
-                        tc::ld32(lane_base + C::COL_O + c, o);
+                        tc::ld32(ocol + c, o);
                         tc::wait_ld<32>(o);
 #pragma unroll
                         for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-                        tc::st32(lane_base + C::COL_O + c, o);
+                        tc::st32(ocol + c, o);
                     }
                 }
             }
             tc::wait_st();
             tc::fence_before();
-            tc::mbar_arrive(bar_p_full(j & 1));
+            tc::mbar_arrive(bar_p_full(t));
         }
-        if (ok) ok = __all_sync(tc::kFull, tc::wait_phase(bar_pv, (nt - 1) & 1, abort_flag, p.err));
+        if (ok) ok = __all_sync(tc::kFull, tc::wait_phase(bar_pv(t), (nt - 1) & 1, abort_flag, p.err));
         if (ok) {
             // ---- epilogue: out = O / l, rounded once to the q dtype ----------------
             tc::fence_after();
@@ -494,7 +526,7 @@ __global__ void __launch_bounds__(192, 1)
 #pragma unroll
             for (int c = 0; c < D; c += 32) {
                 uint32_t o[32];
-                tc::ld32(lane_base + C::COL_O + c, o);
+                tc::ld32(ocol + c, o);
                 tc::wait_ld<32>(o);
                 uint32_t w[16];
 #pragma unroll
@@ -550,9 +582,10 @@ cudaError_t launch_prefill_t(const PrefillParams &p, cudaStream_t stream) {
     auto kern = prefill_kernel<T, D>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
     if (e != cudaSuccess) return e;
-    const dim3 grid((unsigned)((p.max_query_len + p.tok_per_tile - 1) / p.tok_per_tile),
-                    (unsigned)p.num_kv_heads, (unsigned)p.num_seqs);
-    kern<<<grid, 192, C::SMEM, stream>>>(p, mq, mk, mv);
+    const int per_cta = 2 * p.tok_per_tile;  // two query tiles
+    const dim3 grid((unsigned)((p.max_query_len + per_cta - 1) / per_cta), (unsigned)p.num_kv_heads,
+                    (unsigned)p.num_seqs);
+    kern<<<grid, C::THREADS, C::SMEM, stream>>>(p, mq, mk, mv);
     return cudaGetLastError();
 }
 
