@@ -16,19 +16,20 @@
 // A query tile is 128 rows = floor(128 / g) chunk tokens x the g query heads
 // of the KV head (row r: token r / g, head r % g), so the whole GQA group
 // shares each K/V tile it reads; the CTA's two tiles (A, B: consecutive token
-// ranges) share them too.  Keys come in tiles of 128 = 8 blocks of 16 tokens.
+// ranges) share them too.  Keys come in tiles of 64 = 4 blocks of 16 tokens.
 //   - warp 8 (one lane), TMA producer: both Q tiles once through a 3-D
 //     tensor map over q [T, Hq, d]; per key tile, the 8 K and 8 V blocks named
 //     by the block table through the pool's 2-D map (16-row x 128-byte boxes,
-//     128B swizzle) into a 2-stage ring.  Blocks past the sequence's end are
+//     128B swizzle) into a 4-stage ring.  Blocks past the sequence's end are
 //     fetched from past the end of the map, which the copy fills with zeros.
-//   - warp 9 (one lane), MMA issuer: S_t = Q_t K_j^T (M 128, N 128, K d) into
-//     tile t's TMEM columns; O_t += P_t V_j with A = P read from TMEM and
-//     B = V from shared memory (MN-major).  Issue order per key tile j:
-//     PV_A(j), QK_A(j+1), PV_B(j), QK_B(j+1) -- while one tile's softmax
-//     runs, the tensor cores work on the other tile (ping-pong); tcgen05
-//     operations of one thread run in issue order, which makes reusing S_t's
-//     columns for P_t and then for the next S_t safe.
+//   - warp 9 (one lane), MMA issuer: S_t = Q_t K_j^T (M 128, N 64, K d) into
+//     one of tile t's two TMEM score buffers; O_t += P_t V_j with A = P read
+//     from TMEM and B = V from shared memory (MN-major).  Issue order per key
+//     tile j: PV_A(j), QK_A(j+2), PV_B(j), QK_B(j+2) -- every tile's next
+//     scores are ready before its softmax finishes, and the two tiles
+//     ping-pong on the tensor cores; tcgen05 operations of one thread run in
+//     issue order, which makes reusing a score buffer's columns for P and
+//     then for the scores two tiles later safe.
 //   - warps 0-3 (tile A) and 4-7 (tile B), one thread per row: S from TMEM,
 //     causal mask by select on the diagonal tile only, the scale folded into
 //     one FFMA before ex2, online softmax with a lazy rescale (O and l are
@@ -201,16 +202,16 @@ __device__ __forceinline__ void unpack2(uint32_t w, float &lo, float &hi, bf16_t
 
 template <typename T, int D> struct PfCfg {
     static constexpr int BM = 128;  // query rows per tile (TMEM lanes); two tiles per CTA
-    static constexpr int BN = 128;  // keys per tile = 8 blocks
-    static constexpr int ST = 2;    // K/V ring stages
+    static constexpr int BN = 64;   // keys per tile = 4 blocks
+    static constexpr int ST = 4;    // K/V ring stages
     static constexpr int ATOMS = D / 64;  // 128-byte swizzle atoms across d
     static constexpr int Q_BYTES = ATOMS * BM * 128;  // one query tile
     static constexpr int KV_BYTES = ATOMS * BN * 128;
     static constexpr int OFF_Q = 0;                   // tile A, then tile B
     static constexpr int OFF_KV = 2 * Q_BYTES;        // stage st: K, then V
     static constexpr int OFF_BAR = OFF_KV + ST * 2 * KV_BYTES;
-    // q_full, kv_full[ST], kv_empty[ST], s_full[2], p_full[2], pv_done[2], drain
-    static constexpr int NBAR = 1 + 2 * ST + 2 + 2 + 2 + 1;
+    // q_full, kv_full[ST], kv_empty[ST], s_full[2 tiles][2 buffers], p_full[2], pv_done[2], drain
+    static constexpr int NBAR = 1 + 2 * ST + 4 + 2 + 2 + 1;
     static constexpr int OFF_SLOT = OFF_BAR + NBAR * 8;
     static constexpr int OFF_ABORT = OFF_SLOT + 4;
     static constexpr int USED = OFF_ABORT + 4;
@@ -218,7 +219,8 @@ template <typename T, int D> struct PfCfg {
     static constexpr int SMEM = 1024 + (USED < 120 * 1024 ? 120 * 1024 : USED);
     static constexpr bool HILO = std::is_same<T, bf16_t>::value;
     static constexpr uint32_t TMEM_COLS = 512;
-    // S of tile t at column 128 t (P written over it), O of tile t at 256 + 128 t
+    // score buffer b of tile t at column 64 (2 t + b) (P written over it), O
+    // of tile t at 256 + 128 t
     static constexpr uint32_t COL_S = 0, COL_O = 256;
     static constexpr uint32_t FMT = HILO ? 1u : 0u;  // kind::f16 operand format: f16 0, bf16 1
     // instruction descriptors: fp32 accumulate, A/B format, majors, N >> 3, M >> 4
@@ -271,10 +273,11 @@ __global__ void __launch_bounds__(320, 1)
     const uint32_t bar_q = bars;
     auto bar_kv_full = [&](int st) { return bars + 8u * (1 + st); };
     auto bar_kv_empty = [&](int st) { return bars + 8u * (1 + C::ST + st); };
-    auto bar_s_full = [&](int t) { return bars + 8u * (1 + 2 * C::ST + t); };
-    auto bar_p_full = [&](int t) { return bars + 8u * (3 + 2 * C::ST + t); };
-    auto bar_pv = [&](int t) { return bars + 8u * (5 + 2 * C::ST + t); };
-    const uint32_t bar_drain = bars + 8u * (7 + 2 * C::ST);
+    auto bar_s_full = [&](int t, int b) { return bars + 8u * (1 + 2 * C::ST + 2 * t + b); };
+    auto bar_p_full = [&](int t) { return bars + 8u * (5 + 2 * C::ST + t); };
+    auto bar_pv = [&](int t) { return bars + 8u * (7 + 2 * C::ST + t); };
+    const uint32_t bar_drain = bars + 8u * (9 + 2 * C::ST);
+    auto s_col = [&](int t, int b) { return C::COL_S + 64u * (2 * t + b); };
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + C::OFF_ABORT);
     uint32_t *slot = reinterpret_cast<uint32_t *>(smem + C::OFF_SLOT);
 
@@ -287,7 +290,8 @@ __global__ void __launch_bounds__(320, 1)
         }
 #pragma unroll
         for (int t = 0; t < 2; ++t) {
-            mbar_init(bar_s_full(t), 1);
+            mbar_init(bar_s_full(t, 0), 1);
+            mbar_init(bar_s_full(t, 1), 1);
             mbar_init(bar_p_full(t), 128);
             mbar_init(bar_pv(t), 1);
         }
@@ -353,26 +357,28 @@ __global__ void __launch_bounds__(320, 1)
         __syncwarp();
     } else if (warp == 9) {
         // ================= MMA issuer ==============================================
-        // order per key tile j: PV_A(j), QK_A(j+1), PV_B(j), QK_B(j+1); the two
-        // query tiles ping-pong, so one tile's softmax overlaps the other's MMAs
+        // order per key tile j: PV_A(j), QK_A(j+2), PV_B(j), QK_B(j+2) -- each
+        // tile's scores are computed two key tiles ahead into its other S
+        // buffer, and the two query tiles ping-pong on the tensor cores
         auto issue_qk = [&](int t, int j) {
             const uint32_t kaddr = k_smem(j % C::ST), qaddr = q_smem(t);
-            const uint32_t d = tmem + C::COL_S + 128u * t;
+            const uint32_t d = tmem + s_col(t, j & 1);
             if (lane == 0) {
                 tc::fence_after();
 #pragma unroll
                 for (int ks = 0; ks < D / 16; ++ks) {
-                    const uint32_t off = (ks >> 2) * (C::BM * 128) + (ks & 3) * 32;
-                    tc::mma_ss(d, tc::sdesc(qaddr + off, 16, 1024), tc::sdesc(kaddr + off, 16, 1024),
+                    const uint32_t in_atom = (ks & 3) * 32;
+                    tc::mma_ss(d, tc::sdesc(qaddr + (ks >> 2) * (C::BM * 128) + in_atom, 16, 1024),
+                               tc::sdesc(kaddr + (ks >> 2) * (C::BN * 128) + in_atom, 16, 1024),
                                C::IDESC_QK, ks > 0);
                 }
-                tc::commit(bar_s_full(t));
+                tc::commit(bar_s_full(t, j & 1));
             }
             __syncwarp();
         };
         auto issue_pv = [&](int t, int j) {
             const uint32_t vaddr = v_smem(j % C::ST);
-            const uint32_t pcol = tmem + C::COL_S + 128u * t;
+            const uint32_t pcol = tmem + s_col(t, j & 1);
             const uint32_t ocol = tmem + C::COL_O + 128u * t;
             if (lane == 0) {
                 tc::fence_after();
@@ -380,7 +386,8 @@ __global__ void __launch_bounds__(320, 1)
                 for (int ks = 0; ks < C::BN / 16; ++ks) {
                     const uint64_t bdesc = tc::sdesc(vaddr + ks * 2048, C::BN * 128, 1024);
                     tc::mma_ts(ocol, pcol + ks * 8, bdesc, C::IDESC_PV, (j > 0 || ks > 0));
-                    if constexpr (C::HILO) tc::mma_ts(ocol, pcol + 64 + ks * 8, bdesc, C::IDESC_PV, 1);
+                    if constexpr (C::HILO)
+                        tc::mma_ts(ocol, pcol + C::BN / 2 + ks * 8, bdesc, C::IDESC_PV, 1);
                 }
                 tc::commit(bar_pv(t));
                 if (t == 1) tc::commit(bar_kv_empty(j % C::ST));  // last reader of the stage
@@ -408,25 +415,27 @@ __global__ void __launch_bounds__(320, 1)
             }
             return true;
         };
-        bool ok = wait_all(bar_q, 0) && kv_ready(0);
-        if (ok) {
-            issue_qk(0, 0);
-            issue_qk(1, 0);
+        bool ok = wait_all(bar_q, 0);
+        for (int j = 0; ok && j < 2 && j < nt; ++j) {
+            ok = kv_ready(j);
+            if (!ok) break;
+            issue_qk(0, j);
+            issue_qk(1, j);
         }
         for (int j = 0; ok && j < nt; ++j) {
             ok = wait_all(bar_p_full(0), j & 1);
             if (!ok) break;
             issue_pv(0, j);
-            const bool more = j + 1 < nt;
+            const bool more = j + 2 < nt;
             if (more) {
-                ok = kv_ready(j + 1);
+                ok = kv_ready(j + 2);
                 if (!ok) break;
-                issue_qk(0, j + 1);
+                issue_qk(0, j + 2);
             }
             ok = wait_all(bar_p_full(1), j & 1);
             if (!ok) break;
             issue_pv(1, j);
-            if (more) issue_qk(1, j + 1);
+            if (more) issue_qk(1, j + 2);
         }
         // every MMA of this thread must be complete before TMEM is freed
         if (lane == 0) {
@@ -442,15 +451,15 @@ __global__ void __launch_bounds__(320, 1)
         const bool row_ok = r < tpt * g && rtok < ntok;
         const int pos = ctx + tok0 + rtok;
         const uint32_t lane_bits = (uint32_t)((warp & 3) * 32) << 16;
-        const uint32_t scol = tmem + lane_bits + C::COL_S + 128u * t;
         const uint32_t ocol = tmem + lane_bits + C::COL_O + 128u * t;
         const float sl2 = p.qk_scale_log2;  // > 0
         float m_ref = -CUDART_INF_F, l = 0.f;
         bool ok = true;
         for (int j = 0; j < nt; ++j) {
-            ok = __all_sync(tc::kFull, tc::wait_phase(bar_s_full(t), j & 1, abort_flag, p.err));
+            ok = __all_sync(tc::kFull, tc::wait_phase(bar_s_full(t, j & 1), (j >> 1) & 1, abort_flag, p.err));
             if (!ok) break;
             tc::fence_after();
+            const uint32_t scol = tmem + lane_bits + s_col(t, j & 1);
             uint32_t sv[C::BN];
 #pragma unroll
             for (int c = 0; c < C::BN; c += 32) tc::ld32(scol + c, sv + c);
