@@ -24,7 +24,8 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "oracle.c")
 _LIB = os.path.join(_HERE, "liboracle.so")
 
-DTYPES = {"f16": 0, "bf16": 1, "e4m3": 2}
+DTYPES = {"f16": 0, "bf16": 1, "e4m3": 2, "e5m2": 3, "int8": 4}
+EIGHT_BIT = ("e4m3", "e5m2", "int8")
 
 _lib: Optional[ctypes.CDLL] = None
 
@@ -70,6 +71,14 @@ def lib() -> ctypes.CDLL:
         L.orc_e4m3_decode.argtypes = [ctypes.c_uint8]
         L.orc_e4m3_encode.restype = ctypes.c_uint8
         L.orc_e4m3_encode.argtypes = [f32]
+        L.orc_e5m2_decode.restype = f64
+        L.orc_e5m2_decode.argtypes = [ctypes.c_uint8]
+        L.orc_e5m2_encode.restype = ctypes.c_uint8
+        L.orc_e5m2_encode.argtypes = [f32]
+        L.orc_int8_decode.restype = f64
+        L.orc_int8_decode.argtypes = [ctypes.c_uint8]
+        L.orc_int8_encode.restype = ctypes.c_uint8
+        L.orc_int8_encode.argtypes = [f32]
         L.orc_blocks_for_len.restype = i64
         L.orc_blocks_for_len.argtypes = [i64, i32]
         L.orc_kv_bytes_per_token.restype = i64
@@ -129,9 +138,26 @@ def e4m3_encode(y: float) -> int:
     return int(lib().orc_e4m3_encode(float(np.float32(y))))
 
 
+def e5m2_decode(code: int) -> float:
+    return lib().orc_e5m2_decode(int(code))
+
+
+def e5m2_encode(y: float) -> int:
+    return int(lib().orc_e5m2_encode(float(np.float32(y))))
+
+
+def int8_decode(code: int) -> float:
+    return lib().orc_int8_decode(int(code))
+
+
+def int8_encode(y: float) -> int:
+    return int(lib().orc_int8_encode(float(np.float32(y))))
+
+
 def decode_bits(bits: np.ndarray, dtype: str) -> np.ndarray:
-    """Element values of an array of f16 / bf16 / E4M3 codes as fp64."""
-    fn = {"f16": f16_decode, "bf16": bf16_decode, "e4m3": e4m3_decode}[dtype]
+    """Element values of an array of f16 / bf16 / E4M3 / E5M2 / INT8 codes as fp64."""
+    fn = {"f16": f16_decode, "bf16": bf16_decode, "e4m3": e4m3_decode, "e5m2": e5m2_decode,
+          "int8": int8_decode}[dtype]
     flat = np.asarray(bits).reshape(-1)
     # small arrays only (tests): one C call per element
     return np.array([fn(int(x)) for x in flat], dtype=np.float64).reshape(np.shape(bits))
@@ -200,7 +226,7 @@ def copy_blocks(k_cache: np.ndarray, v_cache: np.ndarray, pairs: np.ndarray) -> 
 
 def empty_pool(num_blocks: int, num_kv_heads: int, block_size: int, head_dim: int, kv_dtype: str,
                fill: int = 0xFF) -> np.ndarray:
-    dt = np.uint8 if kv_dtype == "e4m3" else np.uint16
+    dt = np.uint8 if kv_dtype in EIGHT_BIT else np.uint16
     a = np.empty((num_blocks, num_kv_heads, block_size, head_dim), dtype=dt)
     a.view(np.uint8)[...] = fill
     return a

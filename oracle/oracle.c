@@ -33,7 +33,10 @@
  *   - slot = physical_block * block_size + offset; a negative slot is padding;
  *   - seq_len counts the token written in this step; seq_len 0 gives zeros;
  *   - fp8: y = x / scale in fp32 (IEEE), then round to nearest even onto the
- *     E4M3 grid, saturating to +-448; NaN encodes to 0x7F;
+ *     E4M3 grid, saturating to +-448; NaN encodes to 0x7F.  E5M2 alike,
+ *     saturating to +-57344 (the fifth page's §4.2 range), NaN to 0x7F;
+ *   - INT8 (openeuler page §2.3 lists it beside FP8): symmetric, code =
+ *     round-half-even(x / scale) clamped to [-127, 127], value = code * scale;
  *   - split-KV: partition p covers tokens [p*P, min((p+1)*P, L)), summarised by
  *     its log-sum-exp and normalised output, merged by log-sum-exp weighting.
  */
@@ -45,6 +48,11 @@
 #define ORC_F16 0
 #define ORC_BF16 1
 #define ORC_E4M3 2
+#define ORC_E5M2 3
+#define ORC_INT8 4
+
+/* the 8-bit cache formats: each stores code(x / scale) and reads code * scale */
+static int orc_is_8bit(int dtype) { return dtype == ORC_E4M3 || dtype == ORC_E5M2 || dtype == ORC_INT8; }
 
 /* ------------------------------------------------------------------------- */
 /* element formats                                                            */
@@ -130,10 +138,72 @@ uint8_t orc_e4m3_encode(float y) {
     return sign | (uint8_t)(((e + 7) << 3) | ((int)n - 8));
 }
 
+/* OCP 8-bit floating point, E5M2: 1 sign, 5 exponent (bias 15), 2 fraction
+ * bits; exponent 31 holds infinities (fraction 0) and NaNs; largest finite
+ * value 57344. */
+double orc_e5m2_decode(uint8_t c) {
+    int sign = (c >> 7) & 1;
+    int e = (c >> 2) & 0x1F;
+    int m = c & 3;
+    double v;
+    if (e == 31)
+        v = m ? NAN : INFINITY;
+    else if (e == 0)
+        v = ldexp((double)m, -16);
+    else
+        v = ldexp((double)(4 + m), e - 17);
+    return sign ? -v : v;
+}
+
+/* fp32 -> E5M2, round to nearest even, saturating finite overflow and
+ * infinity to +-57344, NaN -> 0x7F. */
+uint8_t orc_e5m2_encode(float y) {
+    if (isnan(y)) return 0x7F;
+    uint8_t sign = signbit(y) ? 0x80 : 0x00;
+    double a = fabs((double)y);
+    if (a >= 57344.0) return sign | 0x7B;
+    if (a < ldexp(1.0, -14)) {
+        /* subnormal range: multiples of 2^-16; 4 * 2^-16 is the smallest
+         * normal, whose code (exponent 1, fraction 0) is also 4 */
+        double n = orc_rne(a * 65536.0);
+        return sign | (uint8_t)n;
+    }
+    int e;
+    frexp(a, &e);
+    e -= 1; /* a in [2^e, 2^(e+1)) */
+    double n = orc_rne(ldexp(a, 2 - e)); /* in [4, 8] */
+    if (n == 8.0) {
+        n = 4.0;
+        e += 1;
+    }
+    /* a < 57344 rounds to at most 57344 (exponent 30, fraction 3) */
+    return sign | (uint8_t)(((e + 15) << 2) | ((int)n - 4));
+}
+
+/* symmetric INT8: the code is the integer itself */
+double orc_int8_decode(uint8_t c) { return (double)(int8_t)c; }
+
+/* fp32 -> INT8: round half to even, clamp to [-127, 127]; NaN -> 0. */
+uint8_t orc_int8_encode(float y) {
+    if (isnan(y)) return 0;
+    double n = orc_rne(fabs((double)y));
+    if (n > 127.0) n = 127.0;
+    int v = signbit(y) ? -(int)n : (int)n;
+    return (uint8_t)(int8_t)v;
+}
+
 double orc_elem(int dtype, const void *base, int64_t i) {
     if (dtype == ORC_F16) return orc_f16_decode(((const uint16_t *)base)[i]);
     if (dtype == ORC_BF16) return orc_bf16_decode(((const uint16_t *)base)[i]);
+    if (dtype == ORC_E5M2) return orc_e5m2_decode(((const uint8_t *)base)[i]);
+    if (dtype == ORC_INT8) return orc_int8_decode(((const uint8_t *)base)[i]);
     return orc_e4m3_decode(((const uint8_t *)base)[i]);
+}
+
+static uint8_t orc_encode8(int dtype, float y) {
+    if (dtype == ORC_E5M2) return orc_e5m2_encode(y);
+    if (dtype == ORC_INT8) return orc_int8_encode(y);
+    return orc_e4m3_encode(y);
 }
 
 /* ------------------------------------------------------------------------- */
@@ -189,8 +259,8 @@ int orc_cache_write(const void *k_new, const void *v_new, void *k_cache, void *v
                     const int64_t *slots, int num_tokens, int num_blocks, int num_kv_heads,
                     int head_dim, int block_size, int act_dtype, int kv_dtype, float k_scale,
                     float v_scale) {
-    if (act_dtype == ORC_E4M3) return -1;
-    if (kv_dtype != ORC_E4M3 && kv_dtype != act_dtype) return -1;
+    if (orc_is_8bit(act_dtype)) return -1;
+    if (!orc_is_8bit(kv_dtype) && kv_dtype != act_dtype) return -1;
     int bad = 0;
     for (int t = 0; t < num_tokens; ++t) {
         int64_t slot = slots[t];
@@ -204,13 +274,13 @@ int orc_cache_write(const void *k_new, const void *v_new, void *k_cache, void *v
             int64_t src = ((int64_t)t * num_kv_heads + h) * head_dim;
             int64_t dst = ((blk * num_kv_heads + h) * block_size + off) * head_dim;
             for (int i = 0; i < head_dim; ++i) {
-                if (kv_dtype == ORC_E4M3) {
+                if (orc_is_8bit(kv_dtype)) {
                     float xk = (float)orc_elem(act_dtype, k_new, src + i);
                     float xv = (float)orc_elem(act_dtype, v_new, src + i);
                     float yk = xk / k_scale;
                     float yv = xv / v_scale;
-                    ((uint8_t *)k_cache)[dst + i] = orc_e4m3_encode(yk);
-                    ((uint8_t *)v_cache)[dst + i] = orc_e4m3_encode(yv);
+                    ((uint8_t *)k_cache)[dst + i] = orc_encode8(kv_dtype, yk);
+                    ((uint8_t *)v_cache)[dst + i] = orc_encode8(kv_dtype, yv);
                 } else {
                     ((uint16_t *)k_cache)[dst + i] = ((const uint16_t *)k_new)[src + i];
                     ((uint16_t *)v_cache)[dst + i] = ((const uint16_t *)v_new)[src + i];
@@ -236,7 +306,7 @@ void orc_gather(double *rows, const void *cache, int kv_dtype, double scale,
         int64_t base = ((phys * num_kv_heads + kvh) * block_size + off) * head_dim;
         for (int i = 0; i < head_dim; ++i) {
             double v = orc_elem(kv_dtype, cache, base + i);
-            rows[(int64_t)t * head_dim + i] = kv_dtype == ORC_E4M3 ? v * scale : v;
+            rows[(int64_t)t * head_dim + i] = orc_is_8bit(kv_dtype) ? v * scale : v;
         }
     }
 }

@@ -10,6 +10,7 @@ import pytest
 
 import oracle
 from tests import test_oracle_cow as cow
+from tests import test_oracle_kv_formats as kvf
 from tests import test_oracle_pins as pins
 from tests import test_oracle_prefill as pre
 
@@ -24,7 +25,7 @@ MUTANTS = {
     "e4m3_bias_off_by_one": ("v = ldexp((double)(8 + m), e - 10);",
                              "v = ldexp((double)(8 + m), e - 11);"),
     "e4m3_round_half_up": ("return fmod(f, 2.0) == 0.0 ? f : f + 1.0;", "return f + 1.0;"),
-    "fp8_scale_dropped_in_gather": ("rows[(int64_t)t * head_dim + i] = kv_dtype == ORC_E4M3 ? v * scale : v;",
+    "fp8_scale_dropped_in_gather": ("rows[(int64_t)t * head_dim + i] = orc_is_8bit(kv_dtype) ? v * scale : v;",
                                     "rows[(int64_t)t * head_dim + i] = v;"),
     "softmax_scale_dropped": ("s[t] = softmax_scale * dot;", "s[t] = dot;"),
     "softmax_not_normalised": ("double p = s[t] / z;", "double p = s[t];"),
@@ -45,6 +46,12 @@ MUTANTS = {
     "prefill_q_row_of_sequence": ("int64_t row_tok = (int64_t)query_start[s] + j;",
                                   "int64_t row_tok = (int64_t)s + j;"),
     "prefill_gqa_interleaved": ("int h = kvh * g + hh;", "int h = hh * num_kv_heads + kvh;"),
+    "e5m2_bias_off_by_one": ("v = ldexp((double)(4 + m), e - 17);", "v = ldexp((double)(4 + m), e - 16);"),
+    "e5m2_saturates_early": ("if (a >= 57344.0) return sign | 0x7B;", "if (a >= 49152.0) return sign | 0x7B;"),
+    "int8_clamps_at_128": ("if (n > 127.0) n = 127.0;", "if (n > 128.0) n = 128.0;"),
+    "int8_round_half_up": ("double n = orc_rne(fabs((double)y));", "double n = floor(fabs((double)y) + 0.5);"),
+    "int8_scale_dropped_in_gather": ("rows[(int64_t)t * head_dim + i] = orc_is_8bit(kv_dtype) ? v * scale : v;",
+                                     "rows[(int64_t)t * head_dim + i] = kv_dtype == ORC_E4M3 || kv_dtype == ORC_E5M2 ? v * scale : v;"),
     "copy_blocks_one_head": ("int64_t block_bytes = (int64_t)num_kv_heads * block_size * head_dim * elem_bytes;",
                              "int64_t block_bytes = (int64_t)block_size * head_dim * elem_bytes;"),
 }
@@ -68,6 +75,12 @@ def _run_pins(golden_dir):
         ("prefill_sdpa", lambda: pre.test_prefill_vs_torch_sdpa_causal(
             oracle, [0, 5, 37, 16], [7, 1, 40, 16], 8, 2, 32, "bf16")),
         ("prefill_chunks", lambda: pre.test_prefill_rows_do_not_depend_on_chunking(oracle)),
+        ("e5m2_decode", lambda: kvf.test_e5m2_decode_all_codes_vs_torch(oracle)),
+        ("e5m2_mid", lambda: kvf.test_e5m2_encode_identity_and_midpoints_vs_torch(oracle)),
+        ("e5m2_range", lambda: kvf.test_e5m2_range_printed(oracle, golden_dir)),
+        ("int8", lambda: kvf.test_int8_codec_vs_numpy(oracle)),
+        ("sdpa_e5m2", lambda: kvf.test_decode_8bit_vs_torch_sdpa_on_dequantised(oracle, "e5m2")),
+        ("sdpa_int8", lambda: kvf.test_decode_8bit_vs_torch_sdpa_on_dequantised(oracle, "int8")),
         ("cow_example", lambda: cow.test_cow_beam_search_example(oracle, golden_dir)),
         ("cow_brute", lambda: cow.test_copy_blocks_brute_force(oracle, "f16")),
         ("cow_bounds", lambda: cow.test_copy_blocks_out_of_range_skipped(oracle)),

@@ -57,7 +57,7 @@ class Workload:
     block_size: int
     num_blocks: int
     act_dtype: str  # dtype of q, of the new K/V rows and of the output
-    kv_dtype: str  # dtype of the cache pools: "f16" | "bf16" | "e4m3"
+    kv_dtype: str  # dtype of the cache pools: "f16" | "bf16" | "e4m3" | "e5m2" | "int8"
     seq_lens: np.ndarray  # int32 [S]; counts the token written by this step
     block_tables: np.ndarray  # int32 [S, max_blocks_per_seq]
     refcount: np.ndarray  # int32 [num_blocks]: tables referencing each block
@@ -70,7 +70,7 @@ class Workload:
     # this step's new token of every sequence, at position seq_len - 1
     k_new: np.ndarray  # uint16 [S, Hk, d]
     v_new: np.ndarray  # uint16 [S, Hk, d]
-    k_scale: float  # fp32 value; 1.0 unless kv_dtype == "e4m3"
+    k_scale: float  # fp32 value; 1.0 unless the cache is 8-bit
     v_scale: float
     free_blocks: np.ndarray  # int32: physical ids no table references
     shared_prefix_blocks: int = 0
@@ -104,7 +104,7 @@ class Workload:
         return (self.seq_lens - 1).astype(np.int32)
 
     def kv_elem_bytes(self) -> int:
-        return 1 if self.kv_dtype == "e4m3" else 2
+        return 1 if self.kv_dtype in EIGHT_BIT else 2
 
     def act_elem_bytes(self) -> int:
         return 2
@@ -171,12 +171,25 @@ def amax_of_bits(*arrays: np.ndarray, dtype: str) -> float:
     return m
 
 
+EIGHT_BIT = ("e4m3", "e5m2", "int8")
+
+# largest code magnitude of each 8-bit cache format: E4M3 448 and E5M2 57344
+# ("大语言模型推理引擎深度剖析", §4.2), symmetric INT8 127
+CODE_MAX = {"e4m3": 448.0, "e5m2": 57344.0, "int8": 127.0}
+
+
 def per_tensor_e4m3_scale(amax: float) -> float:
     """Per-tensor fp8 scale amax / 448 as an fp32 value (448 is the E4M3
     maximum: "大语言模型推理引擎深度剖析", §4.2).  A zero amax gives scale 1."""
+    return per_tensor_scale(amax, "e4m3")
+
+
+def per_tensor_scale(amax: float, kv_dtype: str) -> float:
+    """Per-tensor scale amax / (largest code) of an 8-bit cache format, as an
+    fp32 value; a zero amax gives scale 1."""
     if amax <= 0.0:
         return 1.0
-    return float(np.float32(amax) / np.float32(448.0))
+    return float(np.float32(amax) / np.float32(CODE_MAX[kv_dtype]))
 
 
 # ----------------------------------------------------------------------------
@@ -276,9 +289,9 @@ def build(
         prefill_pos = prefill_pos[:0]
 
     k_scale = v_scale = 1.0
-    if kv_dtype == "e4m3":
-        k_scale = per_tensor_e4m3_scale(amax_of_bits(k_prefill, k_new, dtype=act_dtype))
-        v_scale = per_tensor_e4m3_scale(amax_of_bits(v_prefill, v_new, dtype=act_dtype))
+    if kv_dtype in EIGHT_BIT:
+        k_scale = per_tensor_scale(amax_of_bits(k_prefill, k_new, dtype=act_dtype), kv_dtype)
+        v_scale = per_tensor_scale(amax_of_bits(v_prefill, v_new, dtype=act_dtype), kv_dtype)
     elif kv_dtype != act_dtype:
         raise ValueError("a 16-bit cache must have the activation dtype")
 
@@ -477,9 +490,9 @@ def build_chunked(
     k_ctx = draw_normal_bits(rng, (Tc, num_kv_heads, head_dim), act_dtype)
     v_ctx = draw_normal_bits(rng, (Tc, num_kv_heads, head_dim), act_dtype)
     k_scale = v_scale = 1.0
-    if kv_dtype == "e4m3":
-        k_scale = per_tensor_e4m3_scale(amax_of_bits(k_ctx, k_chunk, dtype=act_dtype))
-        v_scale = per_tensor_e4m3_scale(amax_of_bits(v_ctx, v_chunk, dtype=act_dtype))
+    if kv_dtype in EIGHT_BIT:
+        k_scale = per_tensor_scale(amax_of_bits(k_ctx, k_chunk, dtype=act_dtype), kv_dtype)
+        v_scale = per_tensor_scale(amax_of_bits(v_ctx, v_chunk, dtype=act_dtype), kv_dtype)
     elif kv_dtype != act_dtype:
         raise ValueError("a 16-bit cache must have the activation dtype")
     return ChunkedWorkload(
