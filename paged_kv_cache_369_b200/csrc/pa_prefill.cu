@@ -210,8 +210,9 @@ template <typename T, int D> struct PfCfg {
     static constexpr int OFF_Q = 0;                   // tile A, then tile B
     static constexpr int OFF_KV = 2 * Q_BYTES;        // stage st: K, then V
     static constexpr int OFF_BAR = OFF_KV + ST * 2 * KV_BYTES;
-    // q_full, kv_full[ST], kv_empty[ST], s_full[2 tiles][2 buffers], p_full[2], pv_done[2], drain
-    static constexpr int NBAR = 1 + 2 * ST + 4 + 2 + 2 + 1;
+    // q_full, kv_full[ST], kv_empty[ST], then per (tile, score buffer):
+    // s_full, p_full, pv_done; drain
+    static constexpr int NBAR = 1 + 2 * ST + 4 + 4 + 4 + 1;
     static constexpr int OFF_SLOT = OFF_BAR + NBAR * 8;
     static constexpr int OFF_ABORT = OFF_SLOT + 4;
     static constexpr int USED = OFF_ABORT + 4;
@@ -273,10 +274,12 @@ __global__ void __launch_bounds__(320, 1)
     const uint32_t bar_q = bars;
     auto bar_kv_full = [&](int st) { return bars + 8u * (1 + st); };
     auto bar_kv_empty = [&](int st) { return bars + 8u * (1 + C::ST + st); };
+    // one barrier per (tile, score buffer): a buffer's next phase needs the
+    // other roles to have used the last one, so no wait can see a phase twice
     auto bar_s_full = [&](int t, int b) { return bars + 8u * (1 + 2 * C::ST + 2 * t + b); };
-    auto bar_p_full = [&](int t) { return bars + 8u * (5 + 2 * C::ST + t); };
-    auto bar_pv = [&](int t) { return bars + 8u * (7 + 2 * C::ST + t); };
-    const uint32_t bar_drain = bars + 8u * (9 + 2 * C::ST);
+    auto bar_p_full = [&](int t, int b) { return bars + 8u * (5 + 2 * C::ST + 2 * t + b); };
+    auto bar_pv = [&](int t, int b) { return bars + 8u * (9 + 2 * C::ST + 2 * t + b); };
+    const uint32_t bar_drain = bars + 8u * (13 + 2 * C::ST);
     auto s_col = [&](int t, int b) { return C::COL_S + 64u * (2 * t + b); };
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + C::OFF_ABORT);
     uint32_t *slot = reinterpret_cast<uint32_t *>(smem + C::OFF_SLOT);
@@ -289,12 +292,13 @@ __global__ void __launch_bounds__(320, 1)
             mbar_init(bar_kv_empty(st), 1);
         }
 #pragma unroll
-        for (int t = 0; t < 2; ++t) {
-            mbar_init(bar_s_full(t, 0), 1);
-            mbar_init(bar_s_full(t, 1), 1);
-            mbar_init(bar_p_full(t), 128);
-            mbar_init(bar_pv(t), 1);
-        }
+        for (int t = 0; t < 2; ++t)
+#pragma unroll
+            for (int b = 0; b < 2; ++b) {
+                mbar_init(bar_s_full(t, b), 1);
+                mbar_init(bar_p_full(t, b), 128);
+                mbar_init(bar_pv(t, b), 1);
+            }
         mbar_init(bar_drain, 1);
         *abort_flag = 0;
         mbar_init_fence();
@@ -389,7 +393,7 @@ __global__ void __launch_bounds__(320, 1)
                     if constexpr (C::HILO)
                         tc::mma_ts(ocol, pcol + C::BN / 2 + ks * 8, bdesc, C::IDESC_PV, 1);
                 }
-                tc::commit(bar_pv(t));
+                tc::commit(bar_pv(t, j & 1));
                 if (t == 1) tc::commit(bar_kv_empty(j % C::ST));  // last reader of the stage
             }
             __syncwarp();
@@ -423,7 +427,7 @@ __global__ void __launch_bounds__(320, 1)
             issue_qk(1, j);
         }
         for (int j = 0; ok && j < nt; ++j) {
-            ok = wait_all(bar_p_full(0), j & 1);
+            ok = wait_all(bar_p_full(0, j & 1), (j >> 1) & 1);
             if (!ok) break;
             issue_pv(0, j);
             const bool more = j + 2 < nt;
@@ -432,7 +436,7 @@ __global__ void __launch_bounds__(320, 1)
                 if (!ok) break;
                 issue_qk(0, j + 2);
             }
-            ok = wait_all(bar_p_full(1), j & 1);
+            ok = wait_all(bar_p_full(1, j & 1), (j >> 1) & 1);
             if (!ok) break;
             issue_pv(1, j);
             if (more) issue_qk(1, j + 2);
@@ -504,11 +508,13 @@ __global__ void __launch_bounds__(320, 1)
                 if constexpr (C::HILO) tc::st16(scol + C::BN / 2 + c0 / 2, lo);
             }
             l += (ps[0] + ps[1]) + (ps[2] + ps[3]);
-            if (j > 0) {
-                // O may be touched only once the previous P.V of this tile is complete
-                ok = __all_sync(tc::kFull, tc::wait_phase(bar_pv(t), (j - 1) & 1, abort_flag, p.err));
+            if (j > 0 && __any_sync(tc::kFull, grow)) {
+                // O may be rescaled only once the previous P.V of this tile is
+                // complete (the earlier ones completed before it)
+                ok = __all_sync(tc::kFull, tc::wait_phase(bar_pv(t, (j - 1) & 1), ((j - 1) >> 1) & 1,
+                                                         abort_flag, p.err));
                 if (!ok) break;
-                if (__any_sync(tc::kFull, grow)) {
+                {
                     tc::fence_after();
 #pragma unroll
                     for (int c = 0; c < D; c += 32) {
@@ -523,9 +529,11 @@ __global__ void __launch_bounds__(320, 1)
             }
             tc::wait_st();
             tc::fence_before();
-            tc::mbar_arrive(bar_p_full(t));
+            tc::mbar_arrive(bar_p_full(t, j & 1));
         }
-        if (ok) ok = __all_sync(tc::kFull, tc::wait_phase(bar_pv(t), (nt - 1) & 1, abort_flag, p.err));
+        if (ok)
+            ok = __all_sync(tc::kFull, tc::wait_phase(bar_pv(t, (nt - 1) & 1), ((nt - 1) >> 1) & 1,
+                                                     abort_flag, p.err));
         if (ok) {
             // ---- epilogue: out = O / l, rounded once to the q dtype ----------------
             tc::fence_after();
