@@ -3,6 +3,7 @@
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                     [--config 2] [--mode fused|fused_single|split|single] [--partition 512]
     python bench.py --op copy_blocks [--config 2] [--pairs 4096]
+    python bench.py --config 4 --kv int8     (another 8-bit cache format)
     python bench.py --op prefill [--pconfig 1]
 
 A step is one pass of the whole hot path over one batch: slot mapping of the
@@ -258,7 +259,7 @@ def run_reference(args):
         return 0
     import workload
 
-    w = workload.config(args.config)
+    w = workload.config(args.config, kv_dtype=args.kv)
     import oracle
 
     kc, vc = oracle.caches_for(w)
@@ -304,7 +305,9 @@ def run_copy_blocks(args):
     torch.cuda.set_device(local)
     device = torch.device("cuda", local)
     w = workload.config(args.config, draw_kv=False)
-    dt = torch.uint8 if w.kv_dtype == "e4m3" else {"f16": torch.float16, "bf16": torch.bfloat16}[w.act_dtype]
+    from paged_kv_cache_369_b200 import pool_torch_dtype
+
+    dt = pool_torch_dtype(w.kv_dtype)
     shape = (w.num_blocks, w.num_kv_heads, w.block_size, w.head_dim)
     kc = torch.empty(shape, dtype=dt, device=device)
     vc = torch.empty(shape, dtype=dt, device=device)
@@ -444,7 +447,7 @@ def run_ours(args):
     import workload
     from paged_kv_cache_369_b200.runner import PagedDecode, algorithmic_decode_bytes
 
-    w = workload.config(args.config)
+    w = workload.config(args.config, kv_dtype=args.kv)
     stream = torch.cuda.Stream(device)
     with torch.cuda.stream(stream):
         dec = PagedDecode(w, device=str(device), mode=args.mode, partition_size=args.partition,
@@ -547,7 +550,8 @@ def run_ours(args):
             "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_ms,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": w.kv_dtype if w.kv_dtype != "e4m3" else "e4m3 KV / bf16 q, f32 math",
+            "dtype": w.kv_dtype if w.kv_dtype not in ("e4m3", "e5m2", "int8")
+            else f"{w.kv_dtype} KV / {w.act_dtype} q, f32 math",
             "data": "synthetic: seeded N(0,1) q/K/V, shuffled block pool, no dataset",
             "config": workload_config(w, args.config, args.mode, args.partition),
             "us_per_step": step_ms * 1e3,
@@ -601,6 +605,8 @@ def main(argv=None):
     ap.add_argument("--pconfig", type=int, default=1, choices=(1, 2),
                     help="named chunked-prefill workload for --op prefill")
     ap.add_argument("--pairs", type=int, default=4096, help="block pairs for --op copy_blocks")
+    ap.add_argument("--kv", choices=("e4m3", "e5m2", "int8"), default=None,
+                    help="replace the workload's cache format by this 8-bit one (per-tensor scale)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")

@@ -13,7 +13,8 @@
  *   - the new token's K/V row is appended into its (block, offset) slot; a new
  *     block is opened every 16 tokens ("vLLM推理引擎深度解析：PagedAttention与
  *     连续批处理", §2.2-§2.3);
- *   - the cache may hold FP8 E4M3 values (range +-448) in place of 16-bit ones
+ *   - the cache may hold 8-bit codes in place of 16-bit values: FP8 E4M3
+ *     (range +-448), FP8 E5M2 or INT8
  *     ("大语言模型推理引擎深度剖析：从 KV Cache 内存管理到 PagedAttention、投机
  *     解码与量化加速的完全工程指南", §4.2-§4.3).
  *
@@ -67,8 +68,23 @@ typedef enum pa_status {
 typedef enum pa_dtype {
     PA_F16 = 0,       /* IEEE binary16 */
     PA_BF16 = 1,      /* bfloat16 */
-    PA_FP8_E4M3 = 2   /* OCP E4M3 (FN): bias 7, max 448, no infinities */
+    PA_FP8_E4M3 = 2,  /* OCP E4M3 (FN): bias 7, max 448, no infinities */
+    PA_FP8_E5M2 = 3,  /* OCP E5M2: bias 15, max 57344 (infinities and NaNs exist) */
+    PA_INT8 = 4       /* symmetric signed 8-bit integer code, -127 .. 127 */
 } pa_dtype;
+
+/*
+ * 8-bit caches (PA_FP8_E4M3, PA_FP8_E5M2, PA_INT8; the openeuler page's §2.3
+ * lists FP8 E5M2 / E4M3 and INT8 KV caches, "大语言模型推理引擎深度剖析"
+ * §4.2-§4.3 the FP8 formats and their ranges) store code(x / scale) with one
+ * fp32 scale per tensor (K and V separately) and read value = code * scale:
+ *   E4M3 / E5M2: x / scale in fp32 (IEEE division), round to nearest even
+ *                onto the format, finite overflow and infinity saturating to
+ *                +-448 / +-57344, NaN -> NaN;
+ *   INT8:        round half to even to an integer, clamped to [-127, 127],
+ *                NaN -> 0.
+ * The scale is the caller's (e.g. amax / 448, amax / 57344, amax / 127).
+ */
 
 /* Human-readable name of a status code (host only, static string). */
 const char *pa_status_string(pa_status status);
@@ -107,10 +123,10 @@ pa_status pa_slot_mapping(int64_t *slot_mapping, const int32_t *block_tables,
  *   k_cache[slot / B][h][slot % B][:] = k_new[t][h][:]   (likewise V)
  *
  * act_dtype (of k_new / v_new) is PA_F16 or PA_BF16.  kv_dtype is act_dtype
- * (a bit-exact copy) or PA_FP8_E4M3, in which case each value is stored as
- * e4m3(x / scale): x widened to fp32, divided by the per-tensor scale in fp32
- * (IEEE round to nearest), rounded to nearest even onto the E4M3 grid and
- * saturated to +-448; k_scale / v_scale must then be finite and > 0.
+ * (a bit-exact copy) or an 8-bit format, in which case each value is stored
+ * as code(x / scale) as described under pa_dtype (E4M3: rounded to
+ * nearest even onto the E4M3 grid and saturated to +-448); k_scale / v_scale
+ * must then be finite and > 0.
  * Negative slots are skipped; a slot >= num_blocks * B is skipped with
  * PA_ERR_DEVICE_BOUNDS.  Tokens must map to distinct slots.
  */
@@ -132,13 +148,14 @@ pa_status pa_cache_write(const void *k_new, const void *v_new, void *k_cache, vo
  * L = seq_lens[s]:
  *   out[s][h] = sum_t p_t * V_t,  p = softmax_t(softmax_scale * q[s][h] . K_t),
  *   t < L, K_t / V_t rows of KV head h / g read at block_tables[s][t / 16],
- *   offset t % 16.  For an E4M3 cache, K_t = code * k_scale, V_t = code * v_scale.
+ *   offset t % 16.  For an 8-bit cache, K_t = code * k_scale, V_t = code * v_scale.
  * L = 0 gives a zero row.  Slots at t >= L (the tail of the last block) and
  * unused table entries are never read into the result.
  *
  * Supported: block_size 16, head_dim 64 or 128, num_q_heads a multiple of
  * num_kv_heads, q_dtype (= out dtype) PA_F16 / PA_BF16, kv_dtype = q_dtype or
- * PA_FP8_E4M3.  Arithmetic is fp32; out is rounded to nearest even once.
+ * an 8-bit format (PA_FP8_E4M3, PA_FP8_E5M2, PA_INT8).  Arithmetic is fp32
+ * (8-bit codes are widened exactly); out is rounded to nearest even once.
  */
 pa_status pa_decode(void *out, const void *q, const void *k_cache, const void *v_cache,
                     const int32_t *block_tables, int max_blocks_per_seq, const int32_t *seq_lens,
@@ -159,7 +176,7 @@ pa_status pa_decode(void *out, const void *q, const void *k_cache, const void *v
  * For every sequence s with L = seq_lens[s] > 0 (L counts the new token), the
  * rows k_new[s] / v_new[s] ([num_seqs, num_kv_heads, head_dim], q dtype) are
  * stored at position L - 1, i.e. slot block_tables[s][(L-1)/16]*16 + (L-1)%16,
- * exactly as pa_slot_mapping + pa_cache_write store them (same E4M3
+ * exactly as pa_slot_mapping + pa_cache_write store them (same 8-bit
  * quantisation, same bits); then out is computed as by pa_decode
  * (partition_size == 0: single pass, workspace unused and may be NULL) or by
  * pa_decode_split_reduce (partition_size > 0: a positive multiple of 16,
@@ -239,7 +256,7 @@ pa_status pa_decode_split_reduce(void *out, const void *q, const void *k_cache,
  * sequence covers are not written.  max_query_len bounds every n.
  *
  * Supported: block_size 16, head_dim 64 or 128, q_dtype (= out dtype =
- * kv_dtype) PA_F16 or PA_BF16 (E4M3 caches return PA_ERR_UNSUPPORTED), GQA
+ * kv_dtype) PA_F16 or PA_BF16 (8-bit caches return PA_ERR_UNSUPPORTED), GQA
  * groups up to 128, num_seqs and num_kv_heads up to 65535.  Arithmetic is
  * fp32 with the probabilities kept to ~16 bits (bf16 hi + lo) or f16; out is
  * rounded to nearest even once.  Errors as for pa_decode: a chunk longer
@@ -273,7 +290,7 @@ pa_status pa_prefill(void *out, const void *q, const void *k_cache, const void *
  * (then the result equals copying the pairs in order); src == dst is a
  * no-op.  A pair with an id outside [0, num_blocks) is skipped and flags
  * PA_ERR_DEVICE_BOUNDS in *dev_err.  k_cache / v_cache 16-byte aligned;
- * kv_dtype PA_F16, PA_BF16 or PA_FP8_E4M3 (only its size matters).
+ * kv_dtype any pa_dtype (only its size matters).
  */
 pa_status pa_copy_blocks(void *k_cache, void *v_cache, const int32_t *block_pairs, int num_pairs,
                          int num_blocks, int num_kv_heads, int head_dim, int block_size,

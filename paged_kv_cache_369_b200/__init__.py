@@ -29,6 +29,8 @@ PA_ERR_DEVICE_TIMEOUT = 5
 PA_F16 = 0
 PA_BF16 = 1
 PA_FP8_E4M3 = 2
+PA_FP8_E5M2 = 3
+PA_INT8 = 4
 
 # every extern "C" symbol declared in include/pa.h
 SYMBOLS = (
@@ -119,7 +121,8 @@ def _check(status: int, where: str) -> None:
 
 
 def dtype_code(dtype) -> int:
-    """pa_dtype of a torch dtype (uint8 storage means E4M3 codes)."""
+    """pa_dtype of a torch dtype: float16, bfloat16, float8_e4m3fn (or uint8
+    storage: E4M3 codes), float8_e5m2, int8."""
     import torch
 
     if dtype == torch.float16:
@@ -128,7 +131,19 @@ def dtype_code(dtype) -> int:
         return PA_BF16
     if dtype in (torch.uint8, getattr(torch, "float8_e4m3fn", None)):
         return PA_FP8_E4M3
+    if dtype == getattr(torch, "float8_e5m2", None):
+        return PA_FP8_E5M2
+    if dtype == torch.int8:
+        return PA_INT8
     raise ValueError(f"no pa_dtype for {dtype}")
+
+
+def pool_torch_dtype(kv: str):
+    """torch storage dtype of each cache format, for pools allocated in Python."""
+    import torch
+
+    return {"f16": torch.float16, "bf16": torch.bfloat16, "e4m3": torch.uint8,
+            "e5m2": torch.float8_e5m2, "int8": torch.int8}[kv]
 
 
 def pa_status_string(status: int) -> str:

@@ -4,8 +4,9 @@
 // a physical block; the token sits at offset pos % 16 ("Transformer 推理优化：
 // KV Cache、PagedAttention 与 vLLM", §3.3).  The cache write stores each
 // token's per-head K/V rows there, one new block being opened every 16 tokens
-// ("vLLM推理引擎深度解析：PagedAttention与连续批处理", §2.2), optionally as FP8
-// E4M3 values ("大语言模型推理引擎深度剖析", §4.3).
+// ("vLLM推理引擎深度解析：PagedAttention与连续批处理", §2.2), optionally as
+// 8-bit codes: FP8 E4M3 ("大语言模型推理引擎深度剖析", §4.3), FP8 E5M2 or INT8
+// (the openeuler page's §2.3 table of KV cache formats).
 //
 // Both kernels are HBM-trivial next to attention (a few MB per step); they are
 // written for full 16-byte vector traffic and a grid of whole waves.
@@ -60,8 +61,9 @@ cudaError_t launch_slot_mapping(const SlotParams &p, cudaStream_t stream) {
 // handling the K and the V vector at the same position
 // ---------------------------------------------------------------------------
 
-template <typename ACT, bool FP8>
+template <typename ACT, typename KVT>
 __global__ void __launch_bounds__(256) cache_write_kernel(const CacheWriteParams p) {
+    constexpr bool FP8 = Elem<KVT>::kBytes == 1;  // any 8-bit code
     const int vecs_per_row = p.head_dim / 8;
     const int64_t per_token = (int64_t)p.num_kv_heads * vecs_per_row;
     const int64_t total = (int64_t)p.num_tokens * per_token;
@@ -84,8 +86,8 @@ __global__ void __launch_bounds__(256) cache_write_kernel(const CacheWriteParams
         const uint4 kin = *reinterpret_cast<const uint4 *>(static_cast<const uint16_t *>(p.k_new) + src);
         const uint4 vin = *reinterpret_cast<const uint4 *>(static_cast<const uint16_t *>(p.v_new) + src);
         if constexpr (FP8) {
-            *reinterpret_cast<uint2 *>(static_cast<uint8_t *>(p.k_cache) + dst) = quantise8<ACT>(kin, p.k_scale);
-            *reinterpret_cast<uint2 *>(static_cast<uint8_t *>(p.v_cache) + dst) = quantise8<ACT>(vin, p.v_scale);
+            *reinterpret_cast<uint2 *>(static_cast<uint8_t *>(p.k_cache) + dst) = quantise8<ACT, KVT>(kin, p.k_scale);
+            *reinterpret_cast<uint2 *>(static_cast<uint8_t *>(p.v_cache) + dst) = quantise8<ACT, KVT>(vin, p.v_scale);
         } else {
             *reinterpret_cast<uint4 *>(static_cast<uint16_t *>(p.k_cache) + dst) = kin;
             *reinterpret_cast<uint4 *>(static_cast<uint16_t *>(p.v_cache) + dst) = vin;
@@ -93,25 +95,37 @@ __global__ void __launch_bounds__(256) cache_write_kernel(const CacheWriteParams
     }
 }
 
+// Launch kernel template K<ACT, KVT> for an (activation, cache) dtype pair.
+template <template <typename, typename> class K, typename P>
+static cudaError_t launch_by_dtypes(const P &p, DType act, DType kv, unsigned blocks, cudaStream_t stream) {
+    auto go = [&](auto act_tag, auto kv_tag) {
+        using A = decltype(act_tag);
+        using KV = decltype(kv_tag);
+        K<A, KV>::launch(p, blocks, stream);
+        return cudaGetLastError();
+    };
+    const bool f16 = act == DType::F16;
+    switch (kv) {
+        case DType::E4M3: return f16 ? go(f16_t{}, e4m3_t{}) : go(bf16_t{}, e4m3_t{});
+        case DType::E5M2: return f16 ? go(f16_t{}, e5m2_t{}) : go(bf16_t{}, e5m2_t{});
+        case DType::I8: return f16 ? go(f16_t{}, i8_t{}) : go(bf16_t{}, i8_t{});
+        default: return f16 ? go(f16_t{}, f16_t{}) : go(bf16_t{}, bf16_t{});
+    }
+}
+
+template <typename ACT, typename KVT> struct CacheWriteLaunch {
+    static void launch(const CacheWriteParams &p, unsigned blocks, cudaStream_t stream) {
+        cache_write_kernel<ACT, KVT><<<blocks, 256, 0, stream>>>(p);
+    }
+};
+
 cudaError_t launch_cache_write(const CacheWriteParams &p, DType act, DType kv, cudaStream_t stream) {
     const int64_t total = (int64_t)p.num_tokens * p.num_kv_heads * (p.head_dim / 8);
     if (total <= 0) return cudaSuccess;
     const int threads = 256;
     int64_t blocks = (total + threads - 1) / threads;
     if (blocks > (1 << 20)) blocks = 1 << 20;
-    const bool fp8 = kv == DType::E4M3;
-    if (act == DType::F16) {
-        if (fp8)
-            cache_write_kernel<f16_t, true><<<(unsigned)blocks, threads, 0, stream>>>(p);
-        else
-            cache_write_kernel<f16_t, false><<<(unsigned)blocks, threads, 0, stream>>>(p);
-    } else {
-        if (fp8)
-            cache_write_kernel<bf16_t, true><<<(unsigned)blocks, threads, 0, stream>>>(p);
-        else
-            cache_write_kernel<bf16_t, false><<<(unsigned)blocks, threads, 0, stream>>>(p);
-    }
-    return cudaGetLastError();
+    return launch_by_dtypes<CacheWriteLaunch>(p, act, kv, (unsigned)blocks, stream);
 }
 
 // ---------------------------------------------------------------------------
@@ -121,8 +135,9 @@ cudaError_t launch_cache_write(const CacheWriteParams &p, DType act, DType kv, c
 // patch the new token itself.
 // ---------------------------------------------------------------------------
 
-template <typename ACT, bool FP8>
+template <typename ACT, typename KVT>
 __global__ void __launch_bounds__(256) append_kernel(const AppendParams p) {
+    constexpr bool FP8 = Elem<KVT>::kBytes == 1;  // any 8-bit code
     const int vecs_per_row = p.head_dim / 8;
     const int64_t per_seq = (int64_t)p.num_kv_heads * vecs_per_row;
     const int64_t total = (int64_t)p.num_seqs * per_seq;
@@ -150,8 +165,8 @@ __global__ void __launch_bounds__(256) append_kernel(const AppendParams p) {
         const uint4 kin = *reinterpret_cast<const uint4 *>(static_cast<const uint16_t *>(p.k_new) + src);
         const uint4 vin = *reinterpret_cast<const uint4 *>(static_cast<const uint16_t *>(p.v_new) + src);
         if constexpr (FP8) {
-            *reinterpret_cast<uint2 *>(static_cast<uint8_t *>(p.k_cache) + dst) = quantise8<ACT>(kin, p.k_scale);
-            *reinterpret_cast<uint2 *>(static_cast<uint8_t *>(p.v_cache) + dst) = quantise8<ACT>(vin, p.v_scale);
+            *reinterpret_cast<uint2 *>(static_cast<uint8_t *>(p.k_cache) + dst) = quantise8<ACT, KVT>(kin, p.k_scale);
+            *reinterpret_cast<uint2 *>(static_cast<uint8_t *>(p.v_cache) + dst) = quantise8<ACT, KVT>(vin, p.v_scale);
         } else {
             *reinterpret_cast<uint4 *>(static_cast<uint16_t *>(p.k_cache) + dst) = kin;
             *reinterpret_cast<uint4 *>(static_cast<uint16_t *>(p.v_cache) + dst) = vin;
@@ -159,25 +174,19 @@ __global__ void __launch_bounds__(256) append_kernel(const AppendParams p) {
     }
 }
 
+template <typename ACT, typename KVT> struct AppendLaunch {
+    static void launch(const AppendParams &p, unsigned blocks, cudaStream_t stream) {
+        append_kernel<ACT, KVT><<<blocks, 256, 0, stream>>>(p);
+    }
+};
+
 cudaError_t launch_append(const AppendParams &p, DType act, DType kv, cudaStream_t stream) {
     const int64_t total = (int64_t)p.num_seqs * p.num_kv_heads * (p.head_dim / 8);
     if (total <= 0) return cudaSuccess;
     const int threads = 256;
     int64_t blocks = (total + threads - 1) / threads;
     if (blocks > (1 << 20)) blocks = 1 << 20;
-    const bool fp8 = kv == DType::E4M3;
-    if (act == DType::F16) {
-        if (fp8)
-            append_kernel<f16_t, true><<<(unsigned)blocks, threads, 0, stream>>>(p);
-        else
-            append_kernel<f16_t, false><<<(unsigned)blocks, threads, 0, stream>>>(p);
-    } else {
-        if (fp8)
-            append_kernel<bf16_t, true><<<(unsigned)blocks, threads, 0, stream>>>(p);
-        else
-            append_kernel<bf16_t, false><<<(unsigned)blocks, threads, 0, stream>>>(p);
-    }
-    return cudaGetLastError();
+    return launch_by_dtypes<AppendLaunch>(p, act, kv, (unsigned)blocks, stream);
 }
 
 // ---------------------------------------------------------------------------

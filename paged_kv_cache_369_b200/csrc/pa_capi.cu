@@ -17,6 +17,9 @@ bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 
 bool is_act(pa_dtype t) { return t == PA_F16 || t == PA_BF16; }
 
+// the 8-bit cache formats: codes of x / scale, values code * scale
+bool is_8bit(pa_dtype t) { return t == PA_FP8_E4M3 || t == PA_FP8_E5M2 || t == PA_INT8; }
+
 pa::DType to_internal(pa_dtype t) { return static_cast<pa::DType>(static_cast<int>(t)); }
 
 size_t align256(size_t n) { return (n + 255) & ~size_t(255); }
@@ -106,11 +109,11 @@ pa_status check_decode(const DecodeArgs &a) {
         return PA_ERR_INVALID_ARG;
     if (a.num_q_heads % a.num_kv_heads != 0) return PA_ERR_INVALID_ARG;
     if (!is_act(a.q_dtype)) return PA_ERR_UNSUPPORTED;
-    if (a.kv_dtype != a.q_dtype && a.kv_dtype != PA_FP8_E4M3) return PA_ERR_UNSUPPORTED;
+    if (a.kv_dtype != a.q_dtype && !is_8bit(a.kv_dtype)) return PA_ERR_UNSUPPORTED;
     if (a.head_dim != 64 && a.head_dim != 128) return PA_ERR_UNSUPPORTED;
     if (a.block_size != pa::kBlockSize) return PA_ERR_UNSUPPORTED;
     if (!isfinite(a.softmax_scale)) return PA_ERR_INVALID_ARG;
-    if (a.kv_dtype == PA_FP8_E4M3 &&
+    if (is_8bit(a.kv_dtype) &&
         !(isfinite(a.k_scale) && a.k_scale > 0.f && isfinite(a.v_scale) && a.v_scale > 0.f))
         return PA_ERR_INVALID_ARG;
     if (a.num_seqs == 0) return PA_OK;
@@ -128,7 +131,7 @@ pa_status check_decode(const DecodeArgs &a) {
 
 pa::DecodeParams make_decode_params(const DecodeArgs &a, int *dev_err) {
     pa::DecodeParams p = {};
-    const bool fp8 = a.kv_dtype == PA_FP8_E4M3;
+    const bool fp8 = is_8bit(a.kv_dtype);
     const int g = a.num_q_heads / a.num_kv_heads;
     const int tg = template_group(g);
     p.out = a.out;
@@ -203,9 +206,9 @@ pa_status pa_cache_write(const void *k_new, const void *v_new, void *k_cache, vo
     if (num_tokens < 0 || num_blocks < 0 || num_kv_heads <= 0 || head_dim <= 0 || block_size <= 0)
         return PA_ERR_INVALID_ARG;
     if (!is_act(act_dtype)) return PA_ERR_UNSUPPORTED;
-    if (kv_dtype != act_dtype && kv_dtype != PA_FP8_E4M3) return PA_ERR_UNSUPPORTED;
+    if (kv_dtype != act_dtype && !is_8bit(kv_dtype)) return PA_ERR_UNSUPPORTED;
     if (head_dim % 8 != 0) return PA_ERR_UNSUPPORTED;
-    if (kv_dtype == PA_FP8_E4M3 &&
+    if (is_8bit(kv_dtype) &&
         !(isfinite(k_scale) && k_scale > 0.f && isfinite(v_scale) && v_scale > 0.f))
         return PA_ERR_INVALID_ARG;
     if (num_tokens == 0) return PA_OK;
@@ -281,8 +284,8 @@ pa_status pa_decode_append(void *out, const void *q, const void *k_new, const vo
     p.v_new = v_new;
     p.k_pool_w = static_cast<uint8_t *>(k_cache);
     p.v_pool_w = static_cast<uint8_t *>(v_cache);
-    p.k_scale_w = kv_dtype == PA_FP8_E4M3 ? k_scale : 1.0f;
-    p.v_scale_w = kv_dtype == PA_FP8_E4M3 ? v_scale : 1.0f;
+    p.k_scale_w = is_8bit(kv_dtype) ? k_scale : 1.0f;
+    p.v_scale_w = is_8bit(kv_dtype) ? v_scale : 1.0f;
     const cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (!split) {
         p.partition_blocks = max_blocks_per_seq;
@@ -320,7 +323,7 @@ pa_status pa_prefill(void *out, const void *q, const void *k_cache, const void *
         return PA_ERR_INVALID_ARG;
     if (num_q_heads % num_kv_heads != 0) return PA_ERR_INVALID_ARG;
     if (!is_act(q_dtype)) return PA_ERR_UNSUPPORTED;
-    if (kv_dtype != q_dtype) return PA_ERR_UNSUPPORTED;  // E4M3 caches: not on this path
+    if (kv_dtype != q_dtype) return PA_ERR_UNSUPPORTED;  // 8-bit caches: not on this path
     if (head_dim != 64 && head_dim != 128) return PA_ERR_UNSUPPORTED;
     if (block_size != pa::kBlockSize) return PA_ERR_UNSUPPORTED;
     const int g = num_q_heads / num_kv_heads;
@@ -365,9 +368,8 @@ pa_status pa_copy_blocks(void *k_cache, void *v_cache, const int32_t *block_pair
                          pa_dtype kv_dtype, int *dev_err, void *stream) {
     if (num_pairs < 0 || num_blocks <= 0 || num_kv_heads <= 0 || head_dim <= 0 || block_size <= 0)
         return PA_ERR_INVALID_ARG;
-    if (kv_dtype != PA_F16 && kv_dtype != PA_BF16 && kv_dtype != PA_FP8_E4M3)
-        return PA_ERR_UNSUPPORTED;
-    const int64_t elem = kv_dtype == PA_FP8_E4M3 ? 1 : 2;
+    if (!is_act(kv_dtype) && !is_8bit(kv_dtype)) return PA_ERR_UNSUPPORTED;
+    const int64_t elem = is_8bit(kv_dtype) ? 1 : 2;
     const int64_t block_bytes = (int64_t)num_kv_heads * block_size * head_dim * elem;
     if (block_bytes % 16 != 0) return PA_ERR_UNSUPPORTED;
     if (num_pairs == 0) return PA_OK;

@@ -510,11 +510,21 @@ static cudaError_t decode_by_dim(const DecodeParams &p, int d, int g, cudaStream
 cudaError_t launch_decode(const DecodeParams &p, DType q, DType kv, int head_dim, int tpl_group,
                           cudaStream_t stream) {
     if (p.num_seqs <= 0) return cudaSuccess;
-    if (q == DType::F16)
-        return kv == DType::E4M3 ? decode_by_dim<f16_t, e4m3_t>(p, head_dim, tpl_group, stream)
-                                 : decode_by_dim<f16_t, f16_t>(p, head_dim, tpl_group, stream);
-    return kv == DType::E4M3 ? decode_by_dim<bf16_t, e4m3_t>(p, head_dim, tpl_group, stream)
-                             : decode_by_dim<bf16_t, bf16_t>(p, head_dim, tpl_group, stream);
+    const bool f16 = q == DType::F16;
+    switch (kv) {
+        case DType::E4M3:
+            return f16 ? decode_by_dim<f16_t, e4m3_t>(p, head_dim, tpl_group, stream)
+                       : decode_by_dim<bf16_t, e4m3_t>(p, head_dim, tpl_group, stream);
+        case DType::E5M2:
+            return f16 ? decode_by_dim<f16_t, e5m2_t>(p, head_dim, tpl_group, stream)
+                       : decode_by_dim<bf16_t, e5m2_t>(p, head_dim, tpl_group, stream);
+        case DType::I8:
+            return f16 ? decode_by_dim<f16_t, i8_t>(p, head_dim, tpl_group, stream)
+                       : decode_by_dim<bf16_t, i8_t>(p, head_dim, tpl_group, stream);
+        default:
+            return f16 ? decode_by_dim<f16_t, f16_t>(p, head_dim, tpl_group, stream)
+                       : decode_by_dim<bf16_t, bf16_t>(p, head_dim, tpl_group, stream);
+    }
 }
 
 cudaError_t launch_reduce(const ReduceParams &p, DType q, int head_dim, cudaStream_t stream) {

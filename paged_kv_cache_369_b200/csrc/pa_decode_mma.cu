@@ -24,9 +24,10 @@
 //   - P.V: O[16 x d] += P[16 x 16] V, P taken straight from the S fragments;
 //     ldmatrix.x4.trans feeds V.  For a bf16 cache P is split into bf16 hi + lo
 //     (two MMAs), keeping P to ~16 bits; for f16 and E4M3 caches P is f16;
-//   - E4M3 tiles are converted to f16 (exact) in registers with
-//     cvt.rn.f16x2.e4m3x2; the contraction index d is permuted consistently in
-//     q and K so that one ldmatrix word yields both B registers of a k-step.
+//   - 8-bit tiles (E4M3, E5M2, INT8) are converted to f16 (exact) in
+//     registers, two codes per instruction pair; the contraction index d is
+//     permuted consistently in q and K so that one ldmatrix word yields both B
+//     registers of a k-step.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <math_constants.h>
@@ -50,6 +51,12 @@ template <> struct MmaType<f16_t> {
     using T = f16_t;
 };
 template <> struct MmaType<e4m3_t> {
+    using T = f16_t;
+};
+template <> struct MmaType<e5m2_t> {
+    using T = f16_t;
+};
+template <> struct MmaType<i8_t> {
     using T = f16_t;
 };
 
@@ -81,11 +88,9 @@ __device__ __forceinline__ void ldsm_x4_t(uint32_t *r, uint32_t addr) {
                  : "r"(addr));
 }
 
-// two E4M3 codes (low byte first) -> f16x2, exact
-__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t two_codes) {
-    uint32_t h2;
-    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"((uint16_t)two_codes));
-    return h2;
+
+template <typename KVT> __device__ __forceinline__ uint32_t cvt8x2_f16x2(uint32_t two) {
+    return ::pa::cvt8x2_f16x2(two, KVT{});
 }
 
 __device__ __forceinline__ uint32_t pack2(float lo, float hi, f16_t) {
@@ -360,7 +365,7 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, 3)
         // append: the warp holding the sequence's last block writes this step's
         // new token (position L - 1) into its landed tile and, once per KV head,
         // into the pool -- the slot mapping and cache write of the step fused
-        // here.  E4M3 codes come from the same quantiser as pa_cache_write.
+        // here.  8-bit codes come from the same quantiser as pa_cache_write.
         if (p.append && len_ok && valid && j == (L - 1) / kBlockSize) {
             const int r = (L - 1) & (kBlockSize - 1);
             const int64_t phys = bt_of(k);
@@ -376,8 +381,8 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, 3)
                 uint4 val;
                 if constexpr (C::FP8) {
                     const float sc = isv ? p.v_scale_w : p.k_scale_w;
-                    const uint2 lo = quantise8<QT>(*reinterpret_cast<const uint4 *>(src), sc);
-                    const uint2 hi = quantise8<QT>(*reinterpret_cast<const uint4 *>(src + 8), sc);
+                    const uint2 lo = quantise8<QT, KVT>(*reinterpret_cast<const uint4 *>(src), sc);
+                    const uint2 hi = quantise8<QT, KVT>(*reinterpret_cast<const uint4 *>(src + 8), sc);
                     val = make_uint4(lo.x, lo.y, hi.x, hi.y);
                 } else {
                     val = *reinterpret_cast<const uint4 *>(src);
@@ -412,8 +417,8 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, 3)
 #pragma unroll
                 for (int h = 0; h < 2; ++h) {
                     const int ks = 2 * jj + h;
-                    mma16816(sc[0], qa[ks], e4m3x2_to_f16x2(w[h]), e4m3x2_to_f16x2(w[h] >> 16), ET{});
-                    mma16816(sc[1], qa[ks], e4m3x2_to_f16x2(w[2 + h]), e4m3x2_to_f16x2(w[2 + h] >> 16), ET{});
+                    mma16816(sc[0], qa[ks], cvt8x2_f16x2<KVT>(w[h]), cvt8x2_f16x2<KVT>(w[h] >> 16), ET{});
+                    mma16816(sc[1], qa[ks], cvt8x2_f16x2<KVT>(w[2 + h]), cvt8x2_f16x2<KVT>(w[2 + h] >> 16), ET{});
                 }
             }
         }
@@ -514,8 +519,8 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, 3)
                 for (int h = 0; h < 2; ++h) {
                     const uint32_t lo_t = prmt(w[2 * h], 0x3120);      // tokens 0-7
                     const uint32_t hi_t = prmt(w[2 * h + 1], 0x3120);  // tokens 8-15
-                    uint32_t av[4] = {e4m3x2_to_f16x2(lo_t), e4m3x2_to_f16x2(lo_t >> 16),
-                                      e4m3x2_to_f16x2(hi_t), e4m3x2_to_f16x2(hi_t >> 16)};
+                    uint32_t av[4] = {cvt8x2_f16x2<KVT>(lo_t), cvt8x2_f16x2<KVT>(lo_t >> 16),
+                                      cvt8x2_f16x2<KVT>(hi_t), cvt8x2_f16x2<KVT>(hi_t >> 16)};
                     if (!full) {
                         av[0] &= m0; av[1] &= m0; av[2] &= m8; av[3] &= m8;
                     }
@@ -678,17 +683,24 @@ bool mma_decode_supported(DType kv, int head_dim, int num_blocks, int num_kv_hea
     if (!encode_fn()) return false;
     const int64_t rows = (int64_t)num_blocks * num_kv_heads * kBlockSize;
     if (rows >= (int64_t(1) << 31)) return false;  // TMA row coordinate is a signed 32-bit int
-    if (kv == DType::E4M3) return head_dim == 128;
+    if (is_8bit(kv)) return head_dim == 128;
     return head_dim == 64 || head_dim == 128;
 }
 
 cudaError_t launch_decode_mma(const DecodeParams &p, DType q, DType kv, int head_dim, int mma_rows,
                               cudaStream_t stream) {
     if (p.num_seqs <= 0) return cudaSuccess;
-    if (kv == DType::E4M3) {
+    if (is_8bit(kv)) {
         if (head_dim != 128) return cudaErrorInvalidValue;
-        return q == DType::F16 ? mma_by_rows<f16_t, e4m3_t, 128>(p, mma_rows, stream)
-                               : mma_by_rows<bf16_t, e4m3_t, 128>(p, mma_rows, stream);
+        const bool f16 = q == DType::F16;
+        if (kv == DType::E4M3)
+            return f16 ? mma_by_rows<f16_t, e4m3_t, 128>(p, mma_rows, stream)
+                       : mma_by_rows<bf16_t, e4m3_t, 128>(p, mma_rows, stream);
+        if (kv == DType::E5M2)
+            return f16 ? mma_by_rows<f16_t, e5m2_t, 128>(p, mma_rows, stream)
+                       : mma_by_rows<bf16_t, e5m2_t, 128>(p, mma_rows, stream);
+        return f16 ? mma_by_rows<f16_t, i8_t, 128>(p, mma_rows, stream)
+                   : mma_by_rows<bf16_t, i8_t, 128>(p, mma_rows, stream);
     }
     if (q == DType::F16)
         return head_dim == 64 ? mma_by_rows<f16_t, f16_t, 64>(p, mma_rows, stream)

@@ -24,6 +24,12 @@ struct bf16_t {
 struct e4m3_t {
     uint8_t bits;
 };
+struct e5m2_t {
+    uint8_t bits;
+};
+struct i8_t {  // symmetric INT8 code
+    uint8_t bits;
+};
 
 template <typename T> struct Elem;
 template <> struct Elem<f16_t> {
@@ -35,6 +41,38 @@ template <> struct Elem<bf16_t> {
 template <> struct Elem<e4m3_t> {
     static constexpr int kBytes = 1;
 };
+template <> struct Elem<e5m2_t> {
+    static constexpr int kBytes = 1;
+};
+template <> struct Elem<i8_t> {
+    static constexpr int kBytes = 1;
+};
+
+// ---------------------------------------------------------------------------
+// two 8-bit cache codes (low byte first) -> f16x2, exact for every format:
+// E4M3 and E5M2 values are f16 values, and so are the integers -127..127
+// ---------------------------------------------------------------------------
+
+__device__ __forceinline__ uint32_t cvt8x2_f16x2(uint32_t two, e4m3_t) {
+    uint32_t h2;
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"((uint16_t)two));
+    return h2;
+}
+__device__ __forceinline__ uint32_t cvt8x2_f16x2(uint32_t two, e5m2_t) {
+    uint32_t h2;
+    asm("cvt.rn.f16x2.e5m2x2 %0, %1;" : "=r"(h2) : "h"((uint16_t)two));
+    return h2;
+}
+// INT8: the biased byte b ^ 0x80 = b + 128 becomes the low mantissa byte of an
+// f16 with exponent byte 0x64 (the value 1024 + b + 128, exact); subtracting
+// 1152 leaves b.
+__device__ __forceinline__ uint32_t cvt8x2_f16x2(uint32_t two, i8_t) {
+    uint32_t h2;
+    asm("prmt.b32 %0, %1, %2, 0x5140;" : "=r"(h2) : "r"((two ^ 0x8080u) & 0xFFFFu), "r"(0x6464u));
+    uint32_t r;
+    asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(h2), "r"(0x64806480u));
+    return r;
+}
 
 // Two packed 16-bit values -> two floats (exact).
 __device__ __forceinline__ void unpack2(f16_t, uint32_t w, float &lo, float &hi) {
@@ -54,6 +92,15 @@ __device__ __forceinline__ void unpack2_e4m3(uint16_t w, float &lo, float &hi) {
     uint32_t h2;
     asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(w));
     __half2 h = *reinterpret_cast<__half2 *>(&h2);
+    float2 f = __half22float2(h);
+    lo = f.x;
+    hi = f.y;
+}
+
+// Two packed 8-bit codes (low byte first) -> two floats (exact).
+template <typename T> __device__ __forceinline__ void unpack2_8(uint32_t two, float &lo, float &hi) {
+    const uint32_t h2 = cvt8x2_f16x2(two, T{});
+    __half2 h = *reinterpret_cast<const __half2 *>(&h2);
     float2 f = __half22float2(h);
     lo = f.x;
     hi = f.y;
@@ -83,6 +130,18 @@ template <int N> struct Unpack<e4m3_t, N> {
         if constexpr (N % 4 == 2) unpack2_e4m3((uint16_t)(w[N / 4] & 0xFFFFu), f[N - 2], f[N - 1]);
     }
 };
+template <typename T8, int N> struct Unpack8 {
+    static __device__ __forceinline__ void run(const uint32_t *w, float *f) {
+#pragma unroll
+        for (int i = 0; i < N / 4; ++i) {
+            unpack2_8<T8>(w[i] & 0xFFFFu, f[4 * i], f[4 * i + 1]);
+            unpack2_8<T8>(w[i] >> 16, f[4 * i + 2], f[4 * i + 3]);
+        }
+        if constexpr (N % 4 == 2) unpack2_8<T8>(w[N / 4] & 0xFFFFu, f[N - 2], f[N - 1]);
+    }
+};
+template <int N> struct Unpack<e5m2_t, N> : Unpack8<e5m2_t, N> {};
+template <int N> struct Unpack<i8_t, N> : Unpack8<i8_t, N> {};
 
 __device__ __forceinline__ float to_float(f16_t, uint16_t b) {
     return __half2float(__ushort_as_half(b));
@@ -98,19 +157,39 @@ __device__ __forceinline__ uint16_t from_float(bf16_t, float x) {
 }
 
 // ---------------------------------------------------------------------------
-// E4M3 quantisation of the cache write (shared by every path that stores
-// E4M3 codes, so they agree bit for bit): x / scale in fp32 with IEEE
-// division, then round to nearest even onto E4M3, saturating to +-448.
+// quantisation of the cache write (shared by every path that stores 8-bit
+// codes, so they agree bit for bit): y = x / scale in fp32 with IEEE
+// division, then
+//   E4M3 / E5M2: round to nearest even onto the format, saturating to the
+//                largest finite value (+-448 / +-57344), NaN -> NaN;
+//   INT8:        round half to even to an integer, clamped to [-127, 127].
 // ---------------------------------------------------------------------------
 
-__device__ __forceinline__ uint16_t e4m3x2_rn_sat(float first, float second) {
+__device__ __forceinline__ uint16_t code8x2(float first, float second, e4m3_t) {
     uint16_t r;
     asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(second), "f"(first));
     return r;
 }
+__device__ __forceinline__ uint16_t code8x2(float first, float second, e5m2_t) {
+    uint16_t r;
+    asm("cvt.rn.satfinite.e5m2x2.f32 %0, %1, %2;" : "=h"(r) : "f"(second), "f"(first));
+    return r;
+}
+__device__ __forceinline__ uint32_t int8_code(float y) {
+    int v = __float2int_rn(y);  // NaN -> 0
+    v = v > 127 ? 127 : (v < -127 ? -127 : v);
+    return (uint32_t)v & 0xFFu;
+}
+__device__ __forceinline__ uint16_t code8x2(float first, float second, i8_t) {
+    return (uint16_t)(int8_code(first) | (int8_code(second) << 8));
+}
 
-// eight 16-bit activations (one uint4) -> eight E4M3 codes (one uint2)
-template <typename ACT>
+__device__ __forceinline__ uint16_t e4m3x2_rn_sat(float first, float second) {
+    return code8x2(first, second, e4m3_t{});
+}
+
+// eight 16-bit activations (one uint4) -> eight 8-bit codes (one uint2)
+template <typename ACT, typename KV = e4m3_t>
 __device__ __forceinline__ uint2 quantise8(const uint4 &in, float scale) {
     const uint32_t w[4] = {in.x, in.y, in.z, in.w};
     float f[8];
@@ -118,7 +197,7 @@ __device__ __forceinline__ uint2 quantise8(const uint4 &in, float scale) {
     uint16_t c[4];
 #pragma unroll
     for (int i = 0; i < 4; ++i)
-        c[i] = e4m3x2_rn_sat(__fdiv_rn(f[2 * i], scale), __fdiv_rn(f[2 * i + 1], scale));
+        c[i] = code8x2(__fdiv_rn(f[2 * i], scale), __fdiv_rn(f[2 * i + 1], scale), KV{});
     return make_uint2((uint32_t)c[0] | ((uint32_t)c[1] << 16), (uint32_t)c[2] | ((uint32_t)c[3] << 16));
 }
 

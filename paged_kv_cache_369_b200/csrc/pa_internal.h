@@ -14,7 +14,9 @@ constexpr uint64_t kWaitLimitNs = 1000000000ull;  // 1 s bound on any device wai
 constexpr int kErrBounds = 4;         // = PA_ERR_DEVICE_BOUNDS
 constexpr int kErrTimeout = 5;        // = PA_ERR_DEVICE_TIMEOUT
 
-enum class DType : int { F16 = 0, BF16 = 1, E4M3 = 2 };
+enum class DType : int { F16 = 0, BF16 = 1, E4M3 = 2, E5M2 = 3, I8 = 4 };
+
+inline bool is_8bit(DType t) { return t == DType::E4M3 || t == DType::E5M2 || t == DType::I8; }
 
 struct SlotParams {
     int64_t *slot_mapping;
@@ -155,7 +157,7 @@ cudaError_t launch_prefill(const PrefillParams &p, DType q, int head_dim, cudaSt
 
 // Tensor-core decode (pa_decode_mma.cu): rows of the MMA used for the GQA
 // group (8 or 16); supported for head_dim 64/128 16-bit caches and head_dim
-// 128 E4M3 caches whose pool has fewer than 2^31 token rows.
+// 128 8-bit caches whose pool has fewer than 2^31 token rows.
 bool mma_decode_supported(DType kv, int head_dim, int num_blocks, int num_kv_heads);
 cudaError_t launch_decode_mma(const DecodeParams &p, DType q, DType kv, int head_dim, int mma_rows,
                               cudaStream_t stream);

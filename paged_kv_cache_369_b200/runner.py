@@ -20,7 +20,7 @@ import numpy as np
 import torch
 
 from . import (pa_cache_write, pa_decode, pa_decode_append, pa_decode_split_reduce, pa_prefill,
-               pa_slot_mapping, pa_split_workspace_bytes)
+               pa_slot_mapping, pa_split_workspace_bytes, pool_torch_dtype)
 
 _TORCH_ACT = {"f16": torch.float16, "bf16": torch.bfloat16}
 _UPLOAD_CHUNK_TOKENS = 1 << 16
@@ -51,7 +51,7 @@ class PagedDecode:
         self.v_new = _bits_to_device(w.v_new, w.act_dtype, dev)
         self.block_tables = torch.from_numpy(np.ascontiguousarray(w.block_tables)).to(dev)
         self.seq_lens = torch.from_numpy(np.ascontiguousarray(w.seq_lens)).to(dev)
-        pool_dtype = torch.uint8 if w.kv_dtype == "e4m3" else act
+        pool_dtype = pool_torch_dtype(w.kv_dtype)
         shape = (w.num_blocks, Hk, w.block_size, d)
         self.k_cache = torch.empty(shape, dtype=pool_dtype, device=dev)
         self.v_cache = torch.empty(shape, dtype=pool_dtype, device=dev)

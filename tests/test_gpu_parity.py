@@ -83,6 +83,12 @@ SMALL = [
     (32, 2, 128, "bf16", "bf16", [300, 77], 0),     # g = 16 (two head groups)
     (12, 2, 64, "bf16", "e4m3", [129, 64], 0),      # g = 6
     (2, 2, 64, "f16", "f16", [0, 1, 0, 5], 0),      # empty sequences
+    (64, 8, 128, "bf16", "e5m2", [600, 1, 17, 1024], 0),
+    (8, 8, 128, "f16", "e5m2", [100, 1100, 33], 0),  # MHA, E5M2
+    (32, 8, 128, "f16", "int8", [300, 16, 33, 1], 0),
+    (64, 4, 128, "bf16", "int8", [700, 129], 0),    # g = 16, INT8
+    (16, 2, 64, "bf16", "int8", [3, 90, 16], 0),    # d = 64: CUDA-core kernel
+    (4, 2, 64, "f16", "e5m2", [45, 20], 0),
 ]
 
 
@@ -194,19 +200,21 @@ def test_identical_v_rows_give_that_row():
 _FULL = {}
 
 
-def _full(cfg):
-    if cfg not in _FULL:
+def _full(cfg, kv=None):
+    key = (cfg, kv)
+    if key not in _FULL:
         _FULL.clear()
-        w = workload.config(cfg)
+        w = workload.config(cfg, kv_dtype=kv)
         kc, vc = oracle.caches_for(w)
-        _FULL[cfg] = (w, kc, vc)
-    return _FULL[cfg]
+        _FULL[key] = (w, kc, vc)
+    return _FULL[key]
 
 
-@pytest.mark.parametrize("cfg", [1, 2, 3, 4, 5])
-def test_named_workload_parity(cfg):
+@pytest.mark.parametrize("cfg,kv", [(1, None), (2, None), (3, None), (4, None), (5, None),
+                                    (4, "e5m2"), (4, "int8")])
+def test_named_workload_parity(cfg, kv):
     pa, PagedDecode = _pa()
-    w, kc, vc = _full(cfg)
+    w, kc, vc = _full(cfg, kv)
     dec = PagedDecode(w, mode="fused", partition_size=512)
     dec.step()  # pa_decode_append: the attention launch stores the new tokens
     torch.cuda.synchronize()
@@ -256,6 +264,8 @@ def _check_convex_hull(w, dec, out):
         rows = vpool[ids]  # [nb, Hk, 16, d]
         if w.kv_dtype == "e4m3":
             rows = rows.view(torch.float8_e4m3fn).float() * w.v_scale
+        elif w.kv_dtype in ("e5m2", "int8"):
+            rows = rows.float() * w.v_scale
         else:
             rows = rows.float()
         rows = rows.permute(1, 0, 2, 3).reshape(w.num_kv_heads, nb * 16, w.head_dim)[:, :L]

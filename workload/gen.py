@@ -336,21 +336,31 @@ def config_seq_lens(cfg: int, rng: np.random.Generator) -> np.ndarray:
     raise ValueError(f"unknown config {cfg}")
 
 
-def config(cfg: int, draw_kv: bool = True) -> Workload:
-    """The named decode workload ``cfg`` (1..5), seeded with 369000 + cfg."""
+def config(cfg: int, draw_kv: bool = True, kv_dtype: Optional[str] = None) -> Workload:
+    """The named decode workload ``cfg`` (1..5), seeded with 369000 + cfg.
+    ``kv_dtype`` replaces the configuration's cache format by an 8-bit one
+    ("e4m3", "e5m2", "int8"; same shapes, lengths and seed)."""
     seed = SEED_BASE + cfg
     lens = config_seq_lens(cfg, np.random.default_rng([seed, 1]))
     name = CONFIG_NAMES[cfg]
+    if kv_dtype is not None and kv_dtype not in EIGHT_BIT:
+        raise ValueError("the cache format can be replaced by an 8-bit one only")
+
+    def kv(default):
+        return kv_dtype or default
+
+    if kv_dtype is not None:
+        name = f"{name} [{kv_dtype} KV, per-tensor scale]"
     if cfg == 1:
-        return build(name, seed, lens, 4, 2, 64, "f16", "f16", num_blocks=32, draw_kv=draw_kv)
+        return build(name, seed, lens, 4, 2, 64, "f16", kv("f16"), num_blocks=32, draw_kv=draw_kv)
     if cfg == 2:
-        return build(name, seed, lens, 32, 8, 128, "bf16", "bf16", draw_kv=draw_kv)
+        return build(name, seed, lens, 32, 8, 128, "bf16", kv("bf16"), draw_kv=draw_kv)
     if cfg == 3:
-        return build(name, seed, lens, 64, 8, 128, "bf16", "bf16", draw_kv=draw_kv)
+        return build(name, seed, lens, 64, 8, 128, "bf16", kv("bf16"), draw_kv=draw_kv)
     if cfg == 4:
-        return build(name, seed, lens, 64, 8, 128, "bf16", "e4m3", draw_kv=draw_kv)
+        return build(name, seed, lens, 64, 8, 128, "bf16", kv("e4m3"), draw_kv=draw_kv)
     if cfg == 5:
-        return build(name, seed, lens, 32, 32, 128, "f16", "f16", shared_prefix_tokens=1024,
+        return build(name, seed, lens, 32, 32, 128, "f16", kv("f16"), shared_prefix_tokens=1024,
                      draw_kv=draw_kv)
     raise ValueError(cfg)
 
