@@ -257,7 +257,8 @@ pa_status pa_decode_split_reduce(void *out, const void *q, const void *k_cache,
  *
  * Supported: block_size 16, head_dim 64 or 128, q_dtype (= out dtype =
  * kv_dtype) PA_F16 or PA_BF16 (8-bit caches return PA_ERR_UNSUPPORTED), GQA
- * groups up to 128, num_seqs and num_kv_heads up to 65535.  Arithmetic is
+ * groups up to 128, num_seqs and num_kv_heads up to 65535, softmax_scale
+ * finite and > 0 (else PA_ERR_INVALID_ARG).  Arithmetic is
  * fp32 with the probabilities kept to ~16 bits (bf16 hi + lo) or f16; out is
  * rounded to nearest even once.  Errors as for pa_decode: a chunk longer
  * than its sequence or than max_query_len, a length past the table, or a

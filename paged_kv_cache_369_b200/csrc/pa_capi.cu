@@ -328,7 +328,7 @@ pa_status pa_prefill(void *out, const void *q, const void *k_cache, const void *
     if (block_size != pa::kBlockSize) return PA_ERR_UNSUPPORTED;
     const int g = num_q_heads / num_kv_heads;
     if (g > 128) return PA_ERR_UNSUPPORTED;
-    if (!isfinite(softmax_scale)) return PA_ERR_INVALID_ARG;
+    if (!isfinite(softmax_scale) || !(softmax_scale > 0.f)) return PA_ERR_INVALID_ARG;
     if (num_seqs == 0 || num_tokens == 0) return PA_OK;
     if (!out || !q || !k_cache || !v_cache || !block_tables || !seq_lens || !query_start)
         return PA_ERR_INVALID_ARG;

@@ -197,5 +197,6 @@ def test_prefill_checks(pa):
     assert call(mq=0) == 1
     assert call(S=-1) == 1
     assert call(scale=float("nan")) == 1
+    assert call(scale=-0.5) == 1             # the softmax scale must be positive
     assert call(S=0, q=0) == 0               # nothing to do
     assert call(T=0, q=0) == 0
