@@ -104,6 +104,11 @@ def lib() -> ctypes.CDLL:
         L.orc_prefill.restype = i32
         L.orc_prefill.argtypes = [P, P, i32, P, P, i32, f64, f64, P, i32, P, P, i32, i32, i32, i32,
                                   i32, f64]
+        L.orc_cache_write_channel.restype = i32
+        L.orc_cache_write_channel.argtypes = [P, P, P, P, P, i32, i32, i32, i32, i32, i32, i32, P, P]
+        L.orc_decode_channel.restype = i32
+        L.orc_decode_channel.argtypes = [P, P, i32, P, P, i32, P, P, P, i32, P, i32, i32, i32, i32,
+                                         i32, f64, P, i32]
         L.orc_copy_blocks.restype = i32
         L.orc_copy_blocks.argtypes = [P, P, P, i32, i32, i32, i32, i32, i32]
         _lib = L
@@ -224,6 +229,24 @@ def copy_blocks(k_cache: np.ndarray, v_cache: np.ndarray, pairs: np.ndarray) -> 
                                      bs, k_cache.dtype.itemsize))
 
 
+def cache_write_channel(k_new: np.ndarray, v_new: np.ndarray, k_cache: np.ndarray,
+                        v_cache: np.ndarray, slots: np.ndarray, num_blocks: int, num_kv_heads: int,
+                        head_dim: int, block_size: int, act_dtype: str, kv_dtype: str,
+                        k_scales: np.ndarray, v_scales: np.ndarray) -> int:
+    """Cache write into an 8-bit pool with per-channel scales [Hk, d] (fp32)."""
+    kn, vn = _c(k_new, np.uint16), _c(v_new, np.uint16)
+    sl = _c(slots, np.int64)
+    ks, vs = _c(k_scales, np.float32), _c(v_scales, np.float32)
+    assert k_cache.flags.c_contiguous and v_cache.flags.c_contiguous
+    r = lib().orc_cache_write_channel(_p(kn), _p(vn), _p(k_cache), _p(v_cache), _p(sl),
+                                      int(sl.size), num_blocks, num_kv_heads, head_dim,
+                                      block_size, DTYPES[act_dtype], DTYPES[kv_dtype], _p(ks),
+                                      _p(vs))
+    if r < 0:
+        raise ValueError("unsupported dtype pair")
+    return int(r)
+
+
 def empty_pool(num_blocks: int, num_kv_heads: int, block_size: int, head_dim: int, kv_dtype: str,
                fill: int = 0xFF) -> np.ndarray:
     dt = np.uint8 if kv_dtype in EIGHT_BIT else np.uint16
@@ -280,6 +303,29 @@ def decode(q: np.ndarray, q_dtype: str, k_cache: np.ndarray, v_cache: np.ndarray
                          _p(pr), 0 if pr is None else pr.shape[0])
     if r:
         raise ValueError("invalid head configuration")
+    return out.reshape(S, Hq, d) if pr is None else out
+
+
+def decode_channel(q: np.ndarray, q_dtype: str, k_cache: np.ndarray, v_cache: np.ndarray,
+                   kv_dtype: str, k_scales: np.ndarray, v_scales: np.ndarray,
+                   block_tables: np.ndarray, seq_lens: np.ndarray, num_kv_heads: int,
+                   softmax_scale: float, block_size: int = 16,
+                   pairs: Optional[np.ndarray] = None) -> np.ndarray:
+    """Paged decode attention over an 8-bit cache with per-channel scales."""
+    q = _c(q, np.uint16)
+    S, Hq, d = q.shape
+    bt = _c(block_tables, np.int32)
+    sl = _c(seq_lens, np.int32)
+    ks, vs = _c(k_scales, np.float32), _c(v_scales, np.float32)
+    pr = None if pairs is None else _c(pairs, np.int32).reshape(-1, 2)
+    n = S * Hq if pr is None else pr.shape[0]
+    out = np.empty((n, d), dtype=np.float64)
+    r = lib().orc_decode_channel(_p(out), _p(q), DTYPES[q_dtype], _p(k_cache), _p(v_cache),
+                                 DTYPES[kv_dtype], _p(ks), _p(vs), _p(bt), bt.shape[1], _p(sl), S,
+                                 Hq, num_kv_heads, d, block_size, float(softmax_scale), _p(pr),
+                                 0 if pr is None else pr.shape[0])
+    if r:
+        raise ValueError("invalid configuration")
     return out.reshape(S, Hq, d) if pr is None else out
 
 
@@ -341,23 +387,31 @@ def split_merge(lse: np.ndarray, o: np.ndarray) -> np.ndarray:
 # whole-workload helpers
 # ---------------------------------------------------------------------------
 
+def _write_rows(w, kr, vr, kc, vc, slots):
+    if getattr(w, "k_chan", None) is not None:
+        cache_write_channel(kr, vr, kc, vc, slots, w.num_blocks, w.num_kv_heads, w.head_dim,
+                            w.block_size, w.act_dtype, w.kv_dtype, w.k_chan, w.v_chan)
+    else:
+        cache_write(kr, vr, kc, vc, slots, w.num_blocks, w.num_kv_heads, w.head_dim,
+                    w.block_size, w.act_dtype, w.kv_dtype, w.k_scale, w.v_scale)
+
+
 def caches_for(w, include_new: bool = True) -> Tuple[np.ndarray, np.ndarray]:
     """The oracle's K/V pools for workload ``w``: poisoned (0xFF) pools, the
     prefill tokens written at their slots, then (``include_new``) this step's
-    new token of every sequence at position seq_len - 1."""
+    new token of every sequence at position seq_len - 1.  A workload with
+    per-channel scales (``k_chan`` / ``v_chan``) is quantised with them."""
     kc = empty_pool(w.num_blocks, w.num_kv_heads, w.block_size, w.head_dim, w.kv_dtype)
     vc = empty_pool(w.num_blocks, w.num_kv_heads, w.block_size, w.head_dim, w.kv_dtype)
     Tp = int(w.prefill_seq.size)
     if Tp:
         slots = slot_mapping(w.block_tables, w.seq_lens, w.prefill_seq, w.prefill_pos, Tp,
                              w.block_size)
-        cache_write(w.k_prefill, w.v_prefill, kc, vc, slots, w.num_blocks, w.num_kv_heads,
-                    w.head_dim, w.block_size, w.act_dtype, w.kv_dtype, w.k_scale, w.v_scale)
+        _write_rows(w, w.k_prefill, w.v_prefill, kc, vc, slots)
     if include_new and w.num_seqs:
         slots = slot_mapping(w.block_tables, w.seq_lens, w.new_seq, None, w.num_seqs,
                              w.block_size)
-        cache_write(w.k_new, w.v_new, kc, vc, slots, w.num_blocks, w.num_kv_heads, w.head_dim,
-                    w.block_size, w.act_dtype, w.kv_dtype, w.k_scale, w.v_scale)
+        _write_rows(w, w.k_new, w.v_new, kc, vc, slots)
     return kc, vc
 
 
@@ -384,5 +438,9 @@ def prefill_for(w, kc: np.ndarray, vc: np.ndarray) -> np.ndarray:
 
 
 def decode_for(w, kc: np.ndarray, vc: np.ndarray, pairs: Optional[np.ndarray] = None) -> np.ndarray:
+    if getattr(w, "k_chan", None) is not None:
+        return decode_channel(w.q, w.act_dtype, kc, vc, w.kv_dtype, w.k_chan, w.v_chan,
+                              w.block_tables, w.seq_lens, w.num_kv_heads, w.softmax_scale,
+                              w.block_size, pairs)
     return decode(w.q, w.act_dtype, kc, vc, w.kv_dtype, w.block_tables, w.seq_lens,
                   w.num_kv_heads, w.softmax_scale, w.k_scale, w.v_scale, w.block_size, pairs)

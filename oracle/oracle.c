@@ -20,6 +20,9 @@
  *   - chunked prefill: a long prompt is cut into chunks (e.g. 512 tokens)
  *     processed one after another, each chunk's queries attending causally
  *     over the cache: openeuler page §4.5 and the second page §3.3;
+ *   - per-channel scales for 8-bit caches: the fifth page's §4.3 quantises
+ *     each channel of K / V separately (one scale per (KV head, element of
+ *     head_dim));
  *   - copy-on-write of a shared block: first page §3.5 (a beam-search
  *     candidate that diverges gets a new block for the diverging part only)
  *     and the fifth page §2.3 (a request about to write into a shared block
@@ -296,19 +299,29 @@ int orc_cache_write(const void *k_new, const void *v_new, void *k_cache, void *v
 /* ------------------------------------------------------------------------- */
 
 /* Contiguous fp64 rows [len][d] of KV head `kvh` of one sequence, read through
- * its block table; fp8 values are decode(code) * scale. */
-void orc_gather(double *rows, const void *cache, int kv_dtype, double scale,
-                const int32_t *block_table_row, int len, int num_kv_heads, int kvh, int head_dim,
-                int block_size) {
+ * its block table; 8-bit values are decode(code) * scale, with the scale of
+ * channel i taken from chan_scales[i] when that row of per-channel scales
+ * is given (else the per-tensor `scale`). */
+static void orc_gather_scaled(double *rows, const void *cache, int kv_dtype, double scale,
+                              const float *chan_scales, const int32_t *block_table_row, int len,
+                              int num_kv_heads, int kvh, int head_dim, int block_size) {
     for (int t = 0; t < len; ++t) {
         int64_t phys = block_table_row[t / block_size];
         int64_t off = t % block_size;
         int64_t base = ((phys * num_kv_heads + kvh) * block_size + off) * head_dim;
         for (int i = 0; i < head_dim; ++i) {
             double v = orc_elem(kv_dtype, cache, base + i);
-            rows[(int64_t)t * head_dim + i] = orc_is_8bit(kv_dtype) ? v * scale : v;
+            double sc = chan_scales ? (double)chan_scales[i] : scale;
+            rows[(int64_t)t * head_dim + i] = orc_is_8bit(kv_dtype) ? v * sc : v;
         }
     }
+}
+
+void orc_gather(double *rows, const void *cache, int kv_dtype, double scale,
+                const int32_t *block_table_row, int len, int num_kv_heads, int kvh, int head_dim,
+                int block_size) {
+    orc_gather_scaled(rows, cache, kv_dtype, scale, NULL, block_table_row, len, num_kv_heads, kvh,
+                      head_dim, block_size);
 }
 
 /* Textbook attention of one query row over contiguous K, V [len][d]:
@@ -513,6 +526,80 @@ int orc_prefill(double *out, const void *q, int q_dtype, const void *k_cache, co
                 }
             }
         }
+        free(K);
+        free(V);
+    }
+    free(qrow);
+    return 0;
+}
+
+/* ------------------------------------------------------------------------- */
+/* per-channel scales for 8-bit caches                                        */
+/* ------------------------------------------------------------------------- */
+
+/* Cache write with one scale per (KV head, channel) (the fifth page's §4.3:
+ * each channel of K / V quantised separately): channel i of head h stores
+ * code(x / k_scales[h * head_dim + i]), x / s in fp32 with IEEE division.
+ * kv_dtype must be an 8-bit format.  Returns -1 on an unsupported dtype
+ * pair, else the number of out-of-range slots (skipped). */
+int orc_cache_write_channel(const void *k_new, const void *v_new, void *k_cache, void *v_cache,
+                            const int64_t *slots, int num_tokens, int num_blocks, int num_kv_heads,
+                            int head_dim, int block_size, int act_dtype, int kv_dtype,
+                            const float *k_scales, const float *v_scales) {
+    if (orc_is_8bit(act_dtype) || !orc_is_8bit(kv_dtype)) return -1;
+    int bad = 0;
+    for (int t = 0; t < num_tokens; ++t) {
+        int64_t slot = slots[t];
+        if (slot < 0) continue;
+        if (slot >= (int64_t)num_blocks * block_size) {
+            ++bad;
+            continue;
+        }
+        int64_t blk = slot / block_size, off = slot % block_size;
+        for (int h = 0; h < num_kv_heads; ++h) {
+            int64_t src = ((int64_t)t * num_kv_heads + h) * head_dim;
+            int64_t dst = ((blk * num_kv_heads + h) * block_size + off) * head_dim;
+            for (int i = 0; i < head_dim; ++i) {
+                float xk = (float)orc_elem(act_dtype, k_new, src + i);
+                float xv = (float)orc_elem(act_dtype, v_new, src + i);
+                float yk = xk / k_scales[(int64_t)h * head_dim + i];
+                float yv = xv / v_scales[(int64_t)h * head_dim + i];
+                ((uint8_t *)k_cache)[dst + i] = orc_encode8(kv_dtype, yk);
+                ((uint8_t *)v_cache)[dst + i] = orc_encode8(kv_dtype, yv);
+            }
+        }
+    }
+    return bad;
+}
+
+/* Decode attention (as orc_decode) over an 8-bit cache with per-channel
+ * scales k_scales / v_scales [num_kv_heads][head_dim]: K_t[i] =
+ * code * k_scales[kvh][i], V_t[i] = code * v_scales[kvh][i]. */
+int orc_decode_channel(double *out, const void *q, int q_dtype, const void *k_cache,
+                       const void *v_cache, int kv_dtype, const float *k_scales,
+                       const float *v_scales, const int32_t *block_tables, int max_blocks_per_seq,
+                       const int32_t *seq_lens, int num_seqs, int num_q_heads, int num_kv_heads,
+                       int head_dim, int block_size, double softmax_scale, const int32_t *pairs,
+                       int npairs) {
+    if (num_kv_heads <= 0 || num_q_heads % num_kv_heads || !orc_is_8bit(kv_dtype)) return -1;
+    int g = num_q_heads / num_kv_heads;
+    int n = pairs ? npairs : num_seqs * num_q_heads;
+    double *qrow = (double *)malloc(sizeof(double) * (size_t)head_dim);
+    for (int w = 0; w < n; ++w) {
+        int s = pairs ? pairs[2 * w] : w / num_q_heads;
+        int h = pairs ? pairs[2 * w + 1] : w % num_q_heads;
+        int len = seq_lens[s];
+        int kvh = h / g;
+        const int32_t *bt = block_tables + (int64_t)s * max_blocks_per_seq;
+        double *K = (double *)malloc(sizeof(double) * ((size_t)len * head_dim + 1));
+        double *V = (double *)malloc(sizeof(double) * ((size_t)len * head_dim + 1));
+        orc_gather_scaled(K, k_cache, kv_dtype, 1.0, k_scales + (int64_t)kvh * head_dim, bt, len,
+                          num_kv_heads, kvh, head_dim, block_size);
+        orc_gather_scaled(V, v_cache, kv_dtype, 1.0, v_scales + (int64_t)kvh * head_dim, bt, len,
+                          num_kv_heads, kvh, head_dim, block_size);
+        int64_t qb = ((int64_t)s * num_q_heads + h) * head_dim;
+        for (int i = 0; i < head_dim; ++i) qrow[i] = orc_elem(q_dtype, q, qb + i);
+        orc_attention(out + (int64_t)w * head_dim, NULL, qrow, K, V, len, head_dim, softmax_scale);
         free(K);
         free(V);
     }

@@ -108,3 +108,62 @@ def test_decode_8bit_vs_torch_sdpa_on_dequantised(orc, kv):
             V[s][t] = dec(vc[phys, :, off, :]) * w.v_scale
     ref = _sdpa_ref(w, K, V)
     np.testing.assert_allclose(got, ref, rtol=1e-12, atol=1e-12)
+
+
+# ---------------------------------------------------------------------------
+# per-channel scales (the fifth page's §4.3: each channel of K / V quantised
+# separately)
+# ---------------------------------------------------------------------------
+
+def test_cache_write_per_channel_vs_torch_quantiser(orc):
+    """Codes = torch's e4m3fn cast of (x / s[h][i]) computed in fp32."""
+    rng = np.random.default_rng(15)
+    T, Hk, d, nb = 40, 3, 32, 8
+    x = (rng.standard_normal((T, Hk, d)) * rng.uniform(0.1, 8.0, size=(1, Hk, d))).astype(np.float32)
+    bits = workload.f32_to_bits(x, "bf16")
+    xf = workload.bits_to_f32(bits, "bf16")
+    sc = workload.gen.per_channel_scales("e4m3", bits, dtype="bf16")
+    assert sc.shape == (Hk, d) and sc.dtype == np.float32
+    ref = torch.from_numpy(xf / sc[None]).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    slots = rng.choice(nb * 16, size=T, replace=False).astype(np.int64)
+    kc = orc.empty_pool(nb, Hk, 16, d, "e4m3")
+    vc = orc.empty_pool(nb, Hk, 16, d, "e4m3")
+    orc.cache_write_channel(bits, bits, kc, vc, slots, nb, Hk, d, 16, "bf16", "e4m3", sc, sc)
+    for t in range(T):
+        b, o = divmod(int(slots[t]), 16)
+        np.testing.assert_array_equal(kc[b, :, o, :], ref[t])
+    # each channel's largest |x| maps onto the largest code
+    assert (np.abs(ref.view(np.uint8) & 0x7F).max(axis=0) == 0x7E).all()
+
+
+@pytest.mark.parametrize("kv", ["e4m3", "int8"])
+def test_decode_per_channel_vs_torch_sdpa(orc, kv):
+    w = workload.build("pinch", 16, [9, 40, 23], 8, 2, 32, "bf16", kv, channel_scales=True)
+    kc, vc = orc.caches_for(w)
+    got = orc.decode_for(w, kc, vc)
+    K, V = _contiguous_kv(w)
+    dec = (lambda a: torch.from_numpy(np.asarray(a, np.uint8)).view(torch.float8_e4m3fn).double().numpy()) \
+        if kv == "e4m3" else (lambda a: np.asarray(a, np.uint8).view(np.int8).astype(np.float64))
+    for s in range(w.num_seqs):
+        for t in range(int(w.seq_lens[s])):
+            phys, off = w.block_tables[s, t // 16], t % 16
+            K[s][t] = dec(kc[phys, :, off, :]) * w.k_chan.astype(np.float64)
+            V[s][t] = dec(vc[phys, :, off, :]) * w.v_chan.astype(np.float64)
+    ref = _sdpa_ref(w, K, V)
+    np.testing.assert_allclose(got, ref, rtol=1e-12, atol=1e-12)
+
+
+def test_per_channel_with_equal_scales_is_per_tensor(orc):
+    """Per-channel scales that all equal the per-tensor scale give the same
+    pools and outputs bit for bit."""
+    w = workload.build("eq", 17, [30, 5, 64], 8, 4, 32, "f16", "e4m3", channel_scales=True)
+    w.k_chan[:] = np.float32(w.k_scale)
+    w.v_chan[:] = np.float32(w.v_scale)
+    kc, vc = orc.caches_for(w)
+    out = orc.decode_for(w, kc, vc)
+    k_chan, v_chan = w.k_chan, w.v_chan
+    w.k_chan = w.v_chan = None
+    kc2, vc2 = orc.caches_for(w)
+    out2 = orc.decode_for(w, kc2, vc2)
+    assert np.array_equal(kc, kc2) and np.array_equal(vc, vc2) and np.array_equal(out, out2)
+    w.k_chan, w.v_chan = k_chan, v_chan

@@ -25,7 +25,7 @@ MUTANTS = {
     "e4m3_bias_off_by_one": ("v = ldexp((double)(8 + m), e - 10);",
                              "v = ldexp((double)(8 + m), e - 11);"),
     "e4m3_round_half_up": ("return fmod(f, 2.0) == 0.0 ? f : f + 1.0;", "return f + 1.0;"),
-    "fp8_scale_dropped_in_gather": ("rows[(int64_t)t * head_dim + i] = orc_is_8bit(kv_dtype) ? v * scale : v;",
+    "fp8_scale_dropped_in_gather": ("rows[(int64_t)t * head_dim + i] = orc_is_8bit(kv_dtype) ? v * sc : v;",
                                     "rows[(int64_t)t * head_dim + i] = v;"),
     "softmax_scale_dropped": ("s[t] = softmax_scale * dot;", "s[t] = dot;"),
     "softmax_not_normalised": ("double p = s[t] / z;", "double p = s[t];"),
@@ -50,8 +50,12 @@ MUTANTS = {
     "e5m2_saturates_early": ("if (a >= 57344.0) return sign | 0x7B;", "if (a >= 49152.0) return sign | 0x7B;"),
     "int8_clamps_at_128": ("if (n > 127.0) n = 127.0;", "if (n > 128.0) n = 128.0;"),
     "int8_round_half_up": ("double n = orc_rne(fabs((double)y));", "double n = floor(fabs((double)y) + 0.5);"),
-    "int8_scale_dropped_in_gather": ("rows[(int64_t)t * head_dim + i] = orc_is_8bit(kv_dtype) ? v * scale : v;",
-                                     "rows[(int64_t)t * head_dim + i] = kv_dtype == ORC_E4M3 || kv_dtype == ORC_E5M2 ? v * scale : v;"),
+    "int8_scale_dropped_in_gather": ("rows[(int64_t)t * head_dim + i] = orc_is_8bit(kv_dtype) ? v * sc : v;",
+                                     "rows[(int64_t)t * head_dim + i] = kv_dtype == ORC_E4M3 || kv_dtype == ORC_E5M2 ? v * sc : v;"),
+    "channel_scale_without_head_offset": ("float yk = xk / k_scales[(int64_t)h * head_dim + i];",
+                                          "float yk = xk / k_scales[i];"),
+    "channel_gather_head0_scales": ("orc_gather_scaled(V, v_cache, kv_dtype, 1.0, v_scales + (int64_t)kvh * head_dim, bt, len,",
+                                    "orc_gather_scaled(V, v_cache, kv_dtype, 1.0, v_scales, bt, len,"),
     "copy_blocks_one_head": ("int64_t block_bytes = (int64_t)num_kv_heads * block_size * head_dim * elem_bytes;",
                              "int64_t block_bytes = (int64_t)block_size * head_dim * elem_bytes;"),
 }
@@ -81,6 +85,8 @@ def _run_pins(golden_dir):
         ("int8", lambda: kvf.test_int8_codec_vs_numpy(oracle)),
         ("sdpa_e5m2", lambda: kvf.test_decode_8bit_vs_torch_sdpa_on_dequantised(oracle, "e5m2")),
         ("sdpa_int8", lambda: kvf.test_decode_8bit_vs_torch_sdpa_on_dequantised(oracle, "int8")),
+        ("chan_write", lambda: kvf.test_cache_write_per_channel_vs_torch_quantiser(oracle)),
+        ("chan_sdpa", lambda: kvf.test_decode_per_channel_vs_torch_sdpa(oracle, "e4m3")),
         ("cow_example", lambda: cow.test_cow_beam_search_example(oracle, golden_dir)),
         ("cow_brute", lambda: cow.test_copy_blocks_brute_force(oracle, "f16")),
         ("cow_bounds", lambda: cow.test_copy_blocks_out_of_range_skipped(oracle)),

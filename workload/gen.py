@@ -74,6 +74,9 @@ class Workload:
     v_scale: float
     free_blocks: np.ndarray  # int32: physical ids no table references
     shared_prefix_blocks: int = 0
+    # per-channel scales of an 8-bit cache, fp32 [Hk, d] (None: per tensor)
+    k_chan: Optional[np.ndarray] = None
+    v_chan: Optional[np.ndarray] = None
 
     @property
     def group(self) -> int:
@@ -184,6 +187,21 @@ def per_tensor_e4m3_scale(amax: float) -> float:
     return per_tensor_scale(amax, "e4m3")
 
 
+def per_channel_scales(kv_dtype: str, *arrays: np.ndarray, dtype: str) -> np.ndarray:
+    """Scale of every (KV head, channel): the channel's amax over all tokens of
+    the given [T, Hk, d] rows / (largest code), fp32 [Hk, d]; zero amax gives 1
+    (the fifth page's §4.3 quantises each channel of K / V separately)."""
+    amax = None
+    for a in arrays:
+        for lo in range(0, a.shape[0], max(1, _CHUNK // max(1, a.shape[1] * a.shape[2]))):
+            hi = min(a.shape[0], lo + max(1, _CHUNK // max(1, a.shape[1] * a.shape[2])))
+            m = np.abs(bits_to_f32(a[lo:hi], dtype)).max(axis=0, initial=0.0)
+            amax = m if amax is None else np.maximum(amax, m)
+    amax = amax.astype(np.float32)
+    sc = amax / np.float32(CODE_MAX[kv_dtype])
+    return np.where(amax > 0, sc, np.float32(1.0)).astype(np.float32)
+
+
 def per_tensor_scale(amax: float, kv_dtype: str) -> float:
     """Per-tensor scale amax / (largest code) of an 8-bit cache format, as an
     fp32 value; a zero amax gives scale 1."""
@@ -215,6 +233,7 @@ def build(
     shared_prefix_tokens: int = 0,
     extra_table_cols: int = 0,
     draw_kv: bool = True,
+    channel_scales: bool = False,
 ) -> Workload:
     """Draw one workload.
 
@@ -223,6 +242,7 @@ def build(
     table columns (filled with a free block id, so an over-read lands on
     poisoned memory instead of outside the pool).  ``draw_kv=False`` skips the
     prefill values (shape-only workloads for host-side tests).
+    ``channel_scales`` gives an 8-bit cache one scale per (KV head, channel).
     """
     rng = np.random.default_rng(seed)
     seq_lens = np.asarray(seq_lens, dtype=np.int32)
@@ -289,11 +309,17 @@ def build(
         prefill_pos = prefill_pos[:0]
 
     k_scale = v_scale = 1.0
+    k_chan = v_chan = None
     if kv_dtype in EIGHT_BIT:
         k_scale = per_tensor_scale(amax_of_bits(k_prefill, k_new, dtype=act_dtype), kv_dtype)
         v_scale = per_tensor_scale(amax_of_bits(v_prefill, v_new, dtype=act_dtype), kv_dtype)
+        if channel_scales:
+            k_chan = per_channel_scales(kv_dtype, k_prefill, k_new, dtype=act_dtype)
+            v_chan = per_channel_scales(kv_dtype, v_prefill, v_new, dtype=act_dtype)
     elif kv_dtype != act_dtype:
         raise ValueError("a 16-bit cache must have the activation dtype")
+    elif channel_scales:
+        raise ValueError("per-channel scales need an 8-bit cache")
 
     return Workload(
         name=name, seed=seed, num_seqs=S, num_q_heads=num_q_heads, num_kv_heads=num_kv_heads,
@@ -302,6 +328,7 @@ def build(
         refcount=refcount, q=q, prefill_seq=prefill_seq, prefill_pos=prefill_pos,
         k_prefill=k_prefill, v_prefill=v_prefill, k_new=k_new, v_new=v_new,
         k_scale=k_scale, v_scale=v_scale, free_blocks=free, shared_prefix_blocks=nprefix,
+        k_chan=k_chan, v_chan=v_chan,
     )
 
 
