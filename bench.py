@@ -259,7 +259,7 @@ def run_reference(args):
         return 0
     import workload
 
-    w = workload.config(args.config, kv_dtype=args.kv)
+    w = workload.config(args.config, kv_dtype=args.kv, channel_scales=args.channel_scales)
     import oracle
 
     kc, vc = oracle.caches_for(w)
@@ -447,7 +447,7 @@ def run_ours(args):
     import workload
     from paged_kv_cache_369_b200.runner import PagedDecode, algorithmic_decode_bytes
 
-    w = workload.config(args.config, kv_dtype=args.kv)
+    w = workload.config(args.config, kv_dtype=args.kv, channel_scales=args.channel_scales)
     stream = torch.cuda.Stream(device)
     with torch.cuda.stream(stream):
         dec = PagedDecode(w, device=str(device), mode=args.mode, partition_size=args.partition,
@@ -607,9 +607,17 @@ def main(argv=None):
     ap.add_argument("--pairs", type=int, default=4096, help="block pairs for --op copy_blocks")
     ap.add_argument("--kv", choices=("e4m3", "e5m2", "int8"), default=None,
                     help="replace the workload's cache format by this 8-bit one (per-tensor scale)")
+    ap.add_argument("--channel-scales", action="store_true",
+                    help="per-channel scales for the 8-bit cache (the cache write is then its own "
+                         "call: --mode fused becomes split)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
+    if args.channel_scales:
+        if args.kv is None and args.config != 4:
+            ap.error("--channel-scales needs an 8-bit cache (--kv or config 4)")
+        if args.mode.startswith("fused"):
+            args.mode = "split" if args.mode == "fused" else "single"
     if args.impl == "reference":
         return run_reference(args)
     if args.op == "copy_blocks":

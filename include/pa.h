@@ -297,6 +297,45 @@ pa_status pa_copy_blocks(void *k_cache, void *v_cache, const int32_t *block_pair
                          int num_blocks, int num_kv_heads, int head_dim, int block_size,
                          pa_dtype kv_dtype, int *dev_err, void *stream);
 
+/*
+ * Per-channel scales for 8-bit caches.
+ *
+ * Source: "大语言模型推理引擎深度剖析：从 KV Cache 内存管理到 PagedAttention、投机
+ * 解码与量化加速的完全工程指南", §4.3 (per-channel FP8/E4M3: each channel of K /
+ * V quantised on its own, stored as FP8, widened for attention).
+ *
+ * k_scales / v_scales: device fp32 [num_kv_heads, head_dim], finite and > 0,
+ * 16-byte aligned for the cache write.  Channel i of KV head h stores
+ * code(x / scales[h][i]) (rounding as under pa_dtype) and reads
+ * code * scales[h][i].  kv_dtype must be an 8-bit format.
+ *
+ * pa_cache_write_per_channel: pa_cache_write with those scales in place of
+ * the per-tensor ones (same slots, same errors).
+ *
+ * pa_decode_per_channel: decode over such a cache; partition_size 0 runs the
+ * single-pass kernel (workspace unused, may be NULL), a positive multiple of
+ * 16 runs split-KV with the workspace of pa_decode_split_reduce.  The K
+ * scales are folded into q (q . (code * s) = (q * s) . code) and the V scales
+ * applied to each output channel, so the inner loop is the per-tensor one.
+ * Results, supported shapes and errors as for pa_decode /
+ * pa_decode_split_reduce.
+ */
+pa_status pa_cache_write_per_channel(const void *k_new, const void *v_new, void *k_cache,
+                                     void *v_cache, const int64_t *slot_mapping, int num_tokens,
+                                     int num_blocks, int num_kv_heads, int head_dim,
+                                     int block_size, pa_dtype act_dtype, pa_dtype kv_dtype,
+                                     const float *k_scales, const float *v_scales, int *dev_err,
+                                     void *stream);
+
+pa_status pa_decode_per_channel(void *out, const void *q, const void *k_cache, const void *v_cache,
+                                const int32_t *block_tables, int max_blocks_per_seq,
+                                const int32_t *seq_lens, int num_seqs, int num_q_heads,
+                                int num_kv_heads, int head_dim, int block_size, int num_blocks,
+                                float softmax_scale, pa_dtype q_dtype, pa_dtype kv_dtype,
+                                const float *k_scales, const float *v_scales, int partition_size,
+                                int max_seq_len, void *workspace, size_t workspace_bytes,
+                                int *dev_err, void *stream);
+
 /* Bytes of scratch built into the library for
  * pa_decode_split_reduce_static_scratch (32 MiB). */
 #define PA_STATIC_SCRATCH_BYTES (32u * 1024u * 1024u)

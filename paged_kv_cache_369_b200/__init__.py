@@ -36,7 +36,8 @@ PA_INT8 = 4
 SYMBOLS = (
     "pa_status_string", "pa_version", "pa_slot_mapping", "pa_cache_write", "pa_decode",
     "pa_split_workspace_bytes", "pa_decode_split_reduce", "pa_decode_split_reduce_static_scratch",
-    "pa_decode_append", "pa_copy_blocks", "pa_prefill",
+    "pa_decode_append", "pa_copy_blocks", "pa_prefill", "pa_cache_write_per_channel",
+    "pa_decode_per_channel",
 )
 
 PA_STATIC_SCRATCH_BYTES = 32 * 1024 * 1024
@@ -85,6 +86,12 @@ _lib.pa_decode_split_reduce_static_scratch.argtypes = [_P, _P, _P, _P, _P, _I, _
 _lib.pa_prefill.restype = _I
 _lib.pa_prefill.argtypes = [_P, _P, _P, _P, _P, _I, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _F,
                             _I, _I, _P, _P]
+_lib.pa_cache_write_per_channel.restype = _I
+_lib.pa_cache_write_per_channel.argtypes = [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _P, _P,
+                                            _P, _P]
+_lib.pa_decode_per_channel.restype = _I
+_lib.pa_decode_per_channel.argtypes = [_P, _P, _P, _P, _P, _I, _P, _I, _I, _I, _I, _I, _I, _F, _I,
+                                       _I, _P, _P, _I, _I, _P, _S, _P, _P]
 _lib.pa_copy_blocks.restype = _I
 _lib.pa_copy_blocks.argtypes = [_P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P]
 
@@ -283,3 +290,34 @@ def pa_prefill(out, q, k_cache, v_cache, block_tables, seq_lens, query_start, ma
                            dtype_code(q.dtype), dtype_code(k_cache.dtype), _ptr(dev_err),
                            _stream(stream)),
            "pa_prefill")
+
+
+def pa_cache_write_per_channel(k_new, v_new, k_cache, v_cache, slot_mapping, k_scales, v_scales,
+                               dev_err=None, stream=None) -> None:
+    """Cache write into an 8-bit pool with per-channel scales (fp32 [Hk, d])."""
+    T, Hk, d = (int(x) for x in k_new.shape)
+    nb, _, B, _ = (int(x) for x in k_cache.shape)
+    _check(_lib.pa_cache_write_per_channel(_ptr(k_new), _ptr(v_new), _ptr(k_cache), _ptr(v_cache),
+                                           _ptr(slot_mapping), T, nb, Hk, d, B,
+                                           dtype_code(k_new.dtype), dtype_code(k_cache.dtype),
+                                           _ptr(k_scales), _ptr(v_scales), _ptr(dev_err),
+                                           _stream(stream)),
+           "pa_cache_write_per_channel")
+
+
+def pa_decode_per_channel(out, q, k_cache, v_cache, block_tables, seq_lens, softmax_scale: float,
+                          k_scales, v_scales, partition_size: int = 0, max_seq_len: int = 0,
+                          workspace=None, dev_err=None, stream=None) -> None:
+    """Decode over an 8-bit cache with per-channel scales (partition_size 0:
+    single pass; > 0: split-KV with ``workspace``)."""
+    S, Hq, d = (int(x) for x in q.shape)
+    nb, Hk, B, _ = (int(x) for x in k_cache.shape)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(_lib.pa_decode_per_channel(_ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache),
+                                      _ptr(block_tables), int(block_tables.shape[1]),
+                                      _ptr(seq_lens), S, Hq, Hk, d, B, nb, float(softmax_scale),
+                                      dtype_code(q.dtype), dtype_code(k_cache.dtype),
+                                      _ptr(k_scales), _ptr(v_scales), int(partition_size),
+                                      int(max_seq_len), _ptr(workspace), ws_bytes, _ptr(dev_err),
+                                      _stream(stream)),
+           "pa_decode_per_channel")

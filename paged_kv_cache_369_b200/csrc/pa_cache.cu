@@ -86,8 +86,21 @@ __global__ void __launch_bounds__(256) cache_write_kernel(const CacheWriteParams
         const uint4 kin = *reinterpret_cast<const uint4 *>(static_cast<const uint16_t *>(p.k_new) + src);
         const uint4 vin = *reinterpret_cast<const uint4 *>(static_cast<const uint16_t *>(p.v_new) + src);
         if constexpr (FP8) {
-            *reinterpret_cast<uint2 *>(static_cast<uint8_t *>(p.k_cache) + dst) = quantise8<ACT, KVT>(kin, p.k_scale);
-            *reinterpret_cast<uint2 *>(static_cast<uint8_t *>(p.v_cache) + dst) = quantise8<ACT, KVT>(vin, p.v_scale);
+            uint2 kq, vq;
+            if (p.k_chan) {  // per-channel scales of this head's 8 elements
+                const float4 *ks = reinterpret_cast<const float4 *>(p.k_chan + h * p.head_dim + c * 8);
+                const float4 *vs = reinterpret_cast<const float4 *>(p.v_chan + h * p.head_dim + c * 8);
+                const float4 k0 = ks[0], k1 = ks[1], v0 = vs[0], v1 = vs[1];
+                const float kk[8] = {k0.x, k0.y, k0.z, k0.w, k1.x, k1.y, k1.z, k1.w};
+                const float vv[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+                kq = quantise8_chan<ACT, KVT>(kin, kk);
+                vq = quantise8_chan<ACT, KVT>(vin, vv);
+            } else {
+                kq = quantise8<ACT, KVT>(kin, p.k_scale);
+                vq = quantise8<ACT, KVT>(vin, p.v_scale);
+            }
+            *reinterpret_cast<uint2 *>(static_cast<uint8_t *>(p.k_cache) + dst) = kq;
+            *reinterpret_cast<uint2 *>(static_cast<uint8_t *>(p.v_cache) + dst) = vq;
         } else {
             *reinterpret_cast<uint4 *>(static_cast<uint16_t *>(p.k_cache) + dst) = kin;
             *reinterpret_cast<uint4 *>(static_cast<uint16_t *>(p.v_cache) + dst) = vin;

@@ -386,6 +386,97 @@ pa_status pa_copy_blocks(void *k_cache, void *v_cache, const int32_t *block_pair
     return from_cuda(pa::launch_copy_blocks(p, static_cast<cudaStream_t>(stream)));
 }
 
+pa_status pa_cache_write_per_channel(const void *k_new, const void *v_new, void *k_cache,
+                                     void *v_cache, const int64_t *slot_mapping, int num_tokens,
+                                     int num_blocks, int num_kv_heads, int head_dim,
+                                     int block_size, pa_dtype act_dtype, pa_dtype kv_dtype,
+                                     const float *k_scales, const float *v_scales, int *dev_err,
+                                     void *stream) {
+    if (num_tokens < 0 || num_blocks < 0 || num_kv_heads <= 0 || head_dim <= 0 || block_size <= 0)
+        return PA_ERR_INVALID_ARG;
+    if (!is_act(act_dtype) || !is_8bit(kv_dtype)) return PA_ERR_UNSUPPORTED;
+    if (head_dim % 8 != 0) return PA_ERR_UNSUPPORTED;
+    if (num_tokens == 0) return PA_OK;
+    if (!k_new || !v_new || !k_cache || !v_cache || !slot_mapping || !k_scales || !v_scales)
+        return PA_ERR_INVALID_ARG;
+    if (!aligned16(k_new) || !aligned16(v_new) || !aligned16(k_cache) || !aligned16(v_cache) ||
+        !aligned16(k_scales) || !aligned16(v_scales))
+        return PA_ERR_INVALID_ARG;
+    pa::CacheWriteParams p = {};
+    p.k_new = k_new;
+    p.v_new = v_new;
+    p.k_cache = k_cache;
+    p.v_cache = v_cache;
+    p.slot_mapping = slot_mapping;
+    p.err = dev_err;
+    p.num_tokens = num_tokens;
+    p.num_blocks = num_blocks;
+    p.num_kv_heads = num_kv_heads;
+    p.head_dim = head_dim;
+    p.block_size = block_size;
+    p.k_scale = 1.0f;
+    p.v_scale = 1.0f;
+    p.k_chan = k_scales;
+    p.v_chan = v_scales;
+    return from_cuda(pa::launch_cache_write(p, to_internal(act_dtype), to_internal(kv_dtype),
+                                            static_cast<cudaStream_t>(stream)));
+}
+
+pa_status pa_decode_per_channel(void *out, const void *q, const void *k_cache, const void *v_cache,
+                                const int32_t *block_tables, int max_blocks_per_seq,
+                                const int32_t *seq_lens, int num_seqs, int num_q_heads,
+                                int num_kv_heads, int head_dim, int block_size, int num_blocks,
+                                float softmax_scale, pa_dtype q_dtype, pa_dtype kv_dtype,
+                                const float *k_scales, const float *v_scales, int partition_size,
+                                int max_seq_len, void *workspace, size_t workspace_bytes,
+                                int *dev_err, void *stream) {
+    const DecodeArgs a = {out, q, k_cache, v_cache, block_tables, max_blocks_per_seq, seq_lens,
+                          num_seqs, num_q_heads, num_kv_heads, head_dim, block_size, num_blocks,
+                          softmax_scale, q_dtype, kv_dtype, 1.0f, 1.0f};
+    if (!is_8bit(kv_dtype)) return PA_ERR_UNSUPPORTED;
+    const pa_status st = check_decode(a);
+    if (st != PA_OK) return st;
+    if (partition_size < 0 || partition_size % pa::kBlockSize != 0 || max_seq_len < 0)
+        return PA_ERR_INVALID_ARG;
+    if (num_seqs == 0) return PA_OK;
+    if (!k_scales || !v_scales || (reinterpret_cast<uintptr_t>(k_scales) & 3u) ||
+        (reinterpret_cast<uintptr_t>(v_scales) & 3u))
+        return PA_ERR_INVALID_ARG;
+    pa::DecodeParams p = make_decode_params(a, dev_err);
+    p.k_chan = k_scales;
+    p.v_chan = v_scales;
+    const cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (partition_size == 0) {
+        p.partition_blocks = max_blocks_per_seq;
+        p.num_partitions = 1;
+        p.split = 0;
+        return from_cuda(launch_any_decode(p, q_dtype, kv_dtype, head_dim, s));
+    }
+    const size_t need = pa_split_workspace_bytes(num_seqs, num_q_heads, head_dim, max_seq_len,
+                                                 partition_size);
+    if (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+        return PA_ERR_INVALID_ARG;
+    const int np = max_seq_len > 0 ? (max_seq_len + partition_size - 1) / partition_size : 1;
+    if ((int64_t)num_seqs * np > 0x7FFFFFFF) return PA_ERR_UNSUPPORTED;
+    const size_t rows = (size_t)num_seqs * num_q_heads * np;
+    p.ws_lse = static_cast<float *>(workspace);
+    p.ws_o = reinterpret_cast<float *>(static_cast<uint8_t *>(workspace) + align256(rows * sizeof(float)));
+    p.partition_blocks = partition_size / pa::kBlockSize;
+    p.num_partitions = np;
+    p.split = 1;
+    if (launch_any_decode(p, q_dtype, kv_dtype, head_dim, s) != cudaSuccess) return PA_ERR_CUDA;
+    pa::ReduceParams r = {};
+    r.out = out;
+    r.ws_lse = p.ws_lse;
+    r.ws_o = p.ws_o;
+    r.seq_lens = seq_lens;
+    r.num_seqs = num_seqs;
+    r.num_q_heads = num_q_heads;
+    r.num_partitions = np;
+    r.partition_size = partition_size;
+    return from_cuda(pa::launch_reduce(r, to_internal(q_dtype), head_dim, s));
+}
+
 size_t pa_split_workspace_bytes(int num_seqs, int num_q_heads, int head_dim, int max_seq_len,
                                 int partition_size) {
     if (num_seqs < 0 || num_q_heads <= 0 || head_dim <= 0 || max_seq_len < 0 ||

@@ -169,7 +169,11 @@ __global__ void __launch_bounds__(kDecodeWarps * 32)
                     float f[8];
                     Unpack<QT, 8>::run(ww, f);
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) qf[i][c * C::EPC + v8 + e] = f[e] * p.qk_scale_log2;
+                    for (int e = 0; e < 8; ++e) {
+                        // per-channel K scales: q.(code * s) = (q * s).code
+                        const float ks = p.k_chan ? p.k_chan[(int64_t)kvh * D + e0 + v8 + e] : 1.f;
+                        qf[i][c * C::EPC + v8 + e] = f[e] * ks * p.qk_scale_log2;
+                    }
                 }
             }
         }
@@ -384,7 +388,8 @@ __global__ void __launch_bounds__(kDecodeWarps * 32)
                 O = fmaf(f, accs[(w * G + i) * D + d], O);
             }
         }
-        const float o = Ls > 0.f ? (O / Ls) * p.v_scale : 0.f;
+        const float vs = p.v_chan ? p.v_chan[(int64_t)kvh * D + d] : p.v_scale;
+        const float o = Ls > 0.f ? (O / Ls) * vs : 0.f;
         const int64_t row = (int64_t)s * p.num_q_heads + hq;
         if (!p.split) {
             reinterpret_cast<uint16_t *>(p.out)[row * D + d] = from_float(QT{}, o);

@@ -274,14 +274,19 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, 3)
                     const uint32_t w23 = *reinterpret_cast<const uint32_t *>(qrow + d2);
                     unpack2(QT{}, w01, v0, v1);
                     unpack2(QT{}, w23, v2, v3);
+                    if (p.k_chan) {  // per-channel K scales: q.(code * s) = (q * s).code
+                        const float *kc = p.k_chan + (int64_t)kvh * D;
+                        v0 *= kc[d0]; v1 *= kc[d1]; v2 *= kc[d2]; v3 *= kc[d3];
+                    }
                 }
                 qv[hh][ks][0] = v0; qv[hh][ks][1] = v1; qv[hh][ks][2] = v2; qv[hh][ks][3] = v3;
             }
         }
-        if constexpr (!std::is_same<QT, ET>::value) {
-            // bf16 q against an f16 tensor-core path (E4M3 cache): scale q by a
-            // power of two so its largest element sits near 2^14, convert to
-            // f16, and fold the inverse power into the logit scale (exact).
+        if (!std::is_same<QT, ET>::value || p.k_chan) {
+            // bf16 q against an f16 tensor-core path (8-bit cache), or q times
+            // per-channel scales: scale q by a power of two so its largest
+            // element sits near 2^14, convert to f16, and fold the inverse
+            // power into the logit scale (exact).
             float amax = 0.f;
 #pragma unroll
             for (int hh = 0; hh < 2; ++hh)
@@ -598,7 +603,8 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, 3)
                 O = fmaf(f, accs[(w * GT + i) * D + d], O);
             }
         }
-        const float ov = Ls > 0.f ? (O / Ls) * p.v_scale : 0.f;
+        const float vs = p.v_chan ? p.v_chan[(int64_t)kvh * D + d] : p.v_scale;
+        const float ov = Ls > 0.f ? (O / Ls) * vs : 0.f;
         const int64_t row = (int64_t)s * p.num_q_heads + hq;
         if (!p.split) {
             reinterpret_cast<uint16_t *>(p.out)[row * D + d] = from_float(QT{}, ov);

@@ -188,6 +188,21 @@ __device__ __forceinline__ uint16_t e4m3x2_rn_sat(float first, float second) {
     return code8x2(first, second, e4m3_t{});
 }
 
+// eight 16-bit activations -> eight 8-bit codes, one scale per element
+// (per-channel scales)
+template <typename ACT, typename KV>
+__device__ __forceinline__ uint2 quantise8_chan(const uint4 &in, const float *scales) {
+    const uint32_t w[4] = {in.x, in.y, in.z, in.w};
+    float f[8];
+    Unpack<ACT, 8>::run(w, f);
+    uint16_t c[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+        c[i] = code8x2(__fdiv_rn(f[2 * i], scales[2 * i]), __fdiv_rn(f[2 * i + 1], scales[2 * i + 1]),
+                       KV{});
+    return make_uint2((uint32_t)c[0] | ((uint32_t)c[1] << 16), (uint32_t)c[2] | ((uint32_t)c[3] << 16));
+}
+
 // eight 16-bit activations (one uint4) -> eight 8-bit codes (one uint2)
 template <typename ACT, typename KV = e4m3_t>
 __device__ __forceinline__ uint2 quantise8(const uint4 &in, float scale) {

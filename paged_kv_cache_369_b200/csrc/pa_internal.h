@@ -46,6 +46,8 @@ struct CacheWriteParams {
     int block_size;
     float k_scale;
     float v_scale;
+    const float *k_chan;        // per-channel scales [Hk, D] (8-bit caches) or null
+    const float *v_chan;
 };
 
 struct DecodeParams {
@@ -70,6 +72,10 @@ struct DecodeParams {
     int split;                  // 1: write partials to the workspace
     float qk_scale_log2;        // softmax_scale * k_scale * log2(e)
     float v_scale;              // applied to the output (1 for 16-bit caches)
+    // per-channel scales of an 8-bit cache, [Hk, D] fp32, or null: K's are
+    // folded into q (k_scale then 1), V's applied to the output per channel
+    const float *k_chan;
+    const float *v_chan;
     // append (pa_decode_append): this step's new token of every sequence,
     // stored at position seq_len - 1 before it is attended
     int append;

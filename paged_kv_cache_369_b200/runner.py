@@ -19,8 +19,9 @@ from typing import Optional
 import numpy as np
 import torch
 
-from . import (pa_cache_write, pa_decode, pa_decode_append, pa_decode_split_reduce, pa_prefill,
-               pa_slot_mapping, pa_split_workspace_bytes, pool_torch_dtype)
+from . import (pa_cache_write, pa_cache_write_per_channel, pa_decode, pa_decode_append,
+               pa_decode_per_channel, pa_decode_split_reduce, pa_prefill, pa_slot_mapping,
+               pa_split_workspace_bytes, pool_torch_dtype)
 
 _TORCH_ACT = {"f16": torch.float16, "bf16": torch.bfloat16}
 _UPLOAD_CHUNK_TOKENS = 1 << 16
@@ -38,6 +39,9 @@ class PagedDecode:
                  prefill: bool = True, stream: Optional[torch.cuda.Stream] = None):
         if mode not in ("split", "single", "fused", "fused_single"):
             raise ValueError(mode)
+        self.per_channel = getattr(w, "k_chan", None) is not None
+        if self.per_channel and mode.startswith("fused"):
+            raise ValueError("per-channel scales: the cache write is its own call (split / single)")
         self.w = w
         self.device = torch.device(device)
         self.mode = mode
@@ -62,6 +66,9 @@ class PagedDecode:
         self.new_seq = torch.from_numpy(np.ascontiguousarray(w.new_seq)).to(dev)
         self.out = torch.empty((S, Hq, d), dtype=act, device=dev)
         self.dev_err = torch.zeros(1, dtype=torch.int32, device=dev)
+        if self.per_channel:
+            self.k_chan = torch.from_numpy(np.ascontiguousarray(w.k_chan, np.float32)).to(dev)
+            self.v_chan = torch.from_numpy(np.ascontiguousarray(w.v_chan, np.float32)).to(dev)
         self.max_seq_len = int(w.seq_lens.max()) if S else 0
         nbytes = pa_split_workspace_bytes(S, Hq, d, self.max_seq_len, partition_size)
         self.workspace = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=dev)
@@ -84,9 +91,17 @@ class PagedDecode:
             slots = torch.empty(hi - lo, dtype=torch.int64, device=dev)
             pa_slot_mapping(slots, self.block_tables, self.seq_lens, tseq, tpos, hi - lo,
                             w.num_seqs, w.num_blocks, w.block_size, self.dev_err, self.stream)
+            self._cache_write(kn, vn, slots)
+        torch.cuda.synchronize(dev)
+
+    def _cache_write(self, kn, vn, slots) -> None:
+        w = self.w
+        if self.per_channel:
+            pa_cache_write_per_channel(kn, vn, self.k_cache, self.v_cache, slots, self.k_chan,
+                                       self.v_chan, self.dev_err, self.stream)
+        else:
             pa_cache_write(kn, vn, self.k_cache, self.v_cache, slots, w.k_scale, w.v_scale,
                            self.dev_err, self.stream)
-        torch.cuda.synchronize(dev)
 
     # -- the hot path ----------------------------------------------------------
     def write_new(self) -> None:
@@ -94,11 +109,17 @@ class PagedDecode:
         pa_slot_mapping(self.slot_mapping, self.block_tables, self.seq_lens, self.new_seq, None,
                         w.num_seqs, w.num_seqs, w.num_blocks, w.block_size, self.dev_err,
                         self.stream)
-        pa_cache_write(self.k_new, self.v_new, self.k_cache, self.v_cache, self.slot_mapping,
-                       w.k_scale, w.v_scale, self.dev_err, self.stream)
+        self._cache_write(self.k_new, self.v_new, self.slot_mapping)
 
     def attend(self) -> None:
         w = self.w
+        if self.per_channel:
+            P = 0 if self.mode == "single" else self.partition_size
+            pa_decode_per_channel(self.out, self.q, self.k_cache, self.v_cache, self.block_tables,
+                                  self.seq_lens, w.softmax_scale, self.k_chan, self.v_chan, P,
+                                  self.max_seq_len, self.workspace if P else None, self.dev_err,
+                                  self.stream)
+            return
         if self.mode == "single":
             pa_decode(self.out, self.q, self.k_cache, self.v_cache, self.block_tables,
                       self.seq_lens, w.softmax_scale, w.k_scale, w.v_scale, self.dev_err,

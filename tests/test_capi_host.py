@@ -200,3 +200,27 @@ def test_prefill_checks(pa):
     assert call(scale=-0.5) == 1             # the softmax scale must be positive
     assert call(S=0, q=0) == 0               # nothing to do
     assert call(T=0, q=0) == 0
+
+
+def test_per_channel_checks(pa):
+    L = pa.lib()
+
+    def cw(kv=pa.PA_FP8_E4M3, ks=A, vs=A, T=4):
+        return L.pa_cache_write_per_channel(A, A, A, A, A, T, 10, 2, 128, 16, pa.PA_BF16, kv, ks,
+                                            vs, None, None)
+
+    assert cw(kv=pa.PA_BF16) == 2           # per-channel scales need an 8-bit cache
+    assert cw(ks=0) == 1
+    assert cw(vs=A + 4) == 1                 # scales read as 16-byte vectors
+    assert cw(T=0, ks=0) == 0
+
+    def dec(kv=pa.PA_FP8_E4M3, ks=A, vs=A, P=0, ws=None, wsb=0, S=2):
+        return L.pa_decode_per_channel(A, A, A, A, A, 4, A, S, 8, 2, 128, 16, 10, 0.1, pa.PA_BF16,
+                                       kv, ks, vs, P, 1000, ws, wsb, None, None)
+
+    assert dec(kv=pa.PA_BF16) == 2
+    assert dec(ks=0) == 1
+    assert dec(vs=A + 2) == 1
+    assert dec(P=24) == 1
+    assert dec(P=512) == 1                   # split needs a workspace
+    assert dec(S=0) == 0                     # empty batch

@@ -126,6 +126,35 @@ def test_small_full_parity(case, mode, P, kernel_choice):
             assert not got[s].any()
 
 
+PER_CHANNEL = [
+    # (Hq, Hk, d, act, kv, lens)
+    (64, 8, 128, "bf16", "e4m3", [600, 1, 17, 1024]),
+    (32, 8, 128, "f16", "e4m3", [300, 16, 33]),
+    (32, 8, 128, "bf16", "int8", [129, 700]),
+    (8, 8, 128, "bf16", "e5m2", [100, 1100]),
+    (16, 2, 64, "f16", "e4m3", [3, 90, 16]),       # d = 64: CUDA-core kernel
+]
+
+
+@pytest.mark.parametrize("mode,P", [("single", 512), ("split", 512), ("split", 64)])
+@pytest.mark.parametrize("case", range(len(PER_CHANNEL)))
+def test_per_channel_scales_parity(case, mode, P, kernel_choice):
+    """8-bit caches with one scale per (KV head, channel): pools bit-exact
+    (pa_cache_write_per_channel) and decode within tolerance."""
+    pa, PagedDecode = _pa()
+    Hq, Hk, d, act, kv, lens = PER_CHANNEL[case]
+    w = workload.build(f"chan{case}", 3000 + case, lens, Hq, Hk, d, act, kv, channel_scales=True,
+                       extra_table_cols=1)
+    dec = PagedDecode(w, mode=mode, partition_size=P)
+    dec.step()
+    torch.cuda.synchronize()
+    assert dec.error() == 0
+    kc, vc = oracle.caches_for(w)
+    check_pools(dec, kc, vc)
+    assert_close(_to_f64(dec.out), oracle.decode_for(w, kc, vc),
+                 f"per-channel case {case} {mode} P={P} kernel={kernel_choice}")
+
+
 def test_split_partials_match_oracle(kernel_choice):
     pa, PagedDecode = _pa()
     w = workload.build("partials", 77, [1, 16, 17, 100, 513, 1100], 16, 4, 128, "bf16", "bf16")
@@ -204,18 +233,20 @@ def _full(cfg, kv=None):
     key = (cfg, kv)
     if key not in _FULL:
         _FULL.clear()
-        w = workload.config(cfg, kv_dtype=kv)
+        chan = kv is not None and kv.endswith("-channel")
+        w = workload.config(cfg, kv_dtype=kv.split("-")[0] if kv else None, channel_scales=chan)
         kc, vc = oracle.caches_for(w)
         _FULL[key] = (w, kc, vc)
     return _FULL[key]
 
 
 @pytest.mark.parametrize("cfg,kv", [(1, None), (2, None), (3, None), (4, None), (5, None),
-                                    (4, "e5m2"), (4, "int8")])
+                                    (4, "e5m2"), (4, "int8"), (4, "e4m3-channel")])
 def test_named_workload_parity(cfg, kv):
     pa, PagedDecode = _pa()
     w, kc, vc = _full(cfg, kv)
-    dec = PagedDecode(w, mode="fused", partition_size=512)
+    chan = w.k_chan is not None
+    dec = PagedDecode(w, mode="split" if chan else "fused", partition_size=512)
     dec.step()  # pa_decode_append: the attention launch stores the new tokens
     torch.cuda.synchronize()
     assert dec.error() == 0
@@ -266,6 +297,10 @@ def _check_convex_hull(w, dec, out):
             rows = rows.view(torch.float8_e4m3fn).float() * w.v_scale
         elif w.kv_dtype in ("e5m2", "int8"):
             rows = rows.float() * w.v_scale
+        if w.v_chan is not None:  # per-channel scales replace the per-tensor one
+            codes = vpool[ids]
+            codes = codes.view(torch.float8_e4m3fn) if w.kv_dtype == "e4m3" else codes
+            rows = codes.float() * torch.from_numpy(w.v_chan).to(codes.device)[None, :, None, :]
         else:
             rows = rows.float()
         rows = rows.permute(1, 0, 2, 3).reshape(w.num_kv_heads, nb * 16, w.head_dim)[:, :L]

@@ -363,10 +363,12 @@ def config_seq_lens(cfg: int, rng: np.random.Generator) -> np.ndarray:
     raise ValueError(f"unknown config {cfg}")
 
 
-def config(cfg: int, draw_kv: bool = True, kv_dtype: Optional[str] = None) -> Workload:
+def config(cfg: int, draw_kv: bool = True, kv_dtype: Optional[str] = None,
+           channel_scales: bool = False) -> Workload:
     """The named decode workload ``cfg`` (1..5), seeded with 369000 + cfg.
     ``kv_dtype`` replaces the configuration's cache format by an 8-bit one
-    ("e4m3", "e5m2", "int8"; same shapes, lengths and seed)."""
+    ("e4m3", "e5m2", "int8"; same shapes, lengths and seed);
+    ``channel_scales`` gives an 8-bit cache per-channel scales."""
     seed = SEED_BASE + cfg
     lens = config_seq_lens(cfg, np.random.default_rng([seed, 1]))
     name = CONFIG_NAMES[cfg]
@@ -376,19 +378,21 @@ def config(cfg: int, draw_kv: bool = True, kv_dtype: Optional[str] = None) -> Wo
     def kv(default):
         return kv_dtype or default
 
-    if kv_dtype is not None:
-        name = f"{name} [{kv_dtype} KV, per-tensor scale]"
+    if kv_dtype is not None or channel_scales:
+        name = f"{name} [{kv_dtype or 'e4m3'} KV, per-{'channel' if channel_scales else 'tensor'} scale]"
+    cs = dict(channel_scales=True) if channel_scales else {}
     if cfg == 1:
-        return build(name, seed, lens, 4, 2, 64, "f16", kv("f16"), num_blocks=32, draw_kv=draw_kv)
+        return build(name, seed, lens, 4, 2, 64, "f16", kv("f16"), num_blocks=32, draw_kv=draw_kv,
+                     **cs)
     if cfg == 2:
-        return build(name, seed, lens, 32, 8, 128, "bf16", kv("bf16"), draw_kv=draw_kv)
+        return build(name, seed, lens, 32, 8, 128, "bf16", kv("bf16"), draw_kv=draw_kv, **cs)
     if cfg == 3:
-        return build(name, seed, lens, 64, 8, 128, "bf16", kv("bf16"), draw_kv=draw_kv)
+        return build(name, seed, lens, 64, 8, 128, "bf16", kv("bf16"), draw_kv=draw_kv, **cs)
     if cfg == 4:
-        return build(name, seed, lens, 64, 8, 128, "bf16", kv("e4m3"), draw_kv=draw_kv)
+        return build(name, seed, lens, 64, 8, 128, "bf16", kv("e4m3"), draw_kv=draw_kv, **cs)
     if cfg == 5:
         return build(name, seed, lens, 32, 32, 128, "f16", kv("f16"), shared_prefix_tokens=1024,
-                     draw_kv=draw_kv)
+                     draw_kv=draw_kv, **cs)
     raise ValueError(cfg)
 
 
