@@ -147,12 +147,13 @@ pa_status pa_cache_write(const void *k_new, const void *v_new, void *k_cache, vo
  * For every sequence s, query head h, with g = num_q_heads / num_kv_heads and
  * L = seq_lens[s]:
  *   out[s][h] = sum_t p_t * V_t,  p = softmax_t(softmax_scale * q[s][h] . K_t),
- *   t < L, K_t / V_t rows of KV head h / g read at block_tables[s][t / 16],
- *   offset t % 16.  For an 8-bit cache, K_t = code * k_scale, V_t = code * v_scale.
+ *   t < L, K_t / V_t rows of KV head h / g read at block_tables[s][t / B],
+ *   offset t % B (B = block_size).  For an 8-bit cache, K_t = code * k_scale, V_t = code * v_scale.
  * L = 0 gives a zero row.  Slots at t >= L (the tail of the last block) and
  * unused table entries are never read into the result.
  *
- * Supported: block_size 16, head_dim 64 or 128, num_q_heads a multiple of
+ * Supported: block_size 16 or 32 (the fifth page's §2.2: blocks of 16-32
+ * tokens), head_dim 64 or 128, num_q_heads a multiple of
  * num_kv_heads, q_dtype (= out dtype) PA_F16 / PA_BF16, kv_dtype = q_dtype or
  * an 8-bit format (PA_FP8_E4M3, PA_FP8_E5M2, PA_INT8).  Arithmetic is fp32
  * (8-bit codes are widened exactly); out is rounded to nearest even once.
@@ -217,7 +218,8 @@ size_t pa_split_workspace_bytes(int num_seqs, int num_q_heads, int head_dim, int
  *        o[s][h][p][:] = sum_t softmax-weight_t V_t over the partition (0 if empty)
  *   2. Reduce: M = max_p lse, w_p = exp(lse_p - M),
  *        out[s][h] = sum_p w_p o_p / sum_p w_p      (0 if every partition is empty)
- * partition_size P is a positive multiple of block_size; max_seq_len bounds
+ * partition_size P is a positive multiple of 16 (a partition may end inside a
+ * 32-token block); max_seq_len bounds
  * every seq_lens[s] (a longer one is truncated and flags PA_ERR_DEVICE_BOUNDS).
  * workspace (device, caller-owned, >= pa_split_workspace_bytes(...) bytes,
  * 256-byte aligned) holds the partials in the layout above after the call;
@@ -255,7 +257,7 @@ pa_status pa_decode_split_reduce(void *out, const void *q, const void *k_cache,
  * int32) is non-decreasing with query_start[num_seqs] <= num_tokens; rows no
  * sequence covers are not written.  max_query_len bounds every n.
  *
- * Supported: block_size 16, head_dim 64 or 128, q_dtype (= out dtype =
+ * Supported: block_size 16 or 32, head_dim 64 or 128, q_dtype (= out dtype =
  * kv_dtype) PA_F16 or PA_BF16 (8-bit caches return PA_ERR_UNSUPPORTED), GQA
  * groups up to 128, num_seqs and num_kv_heads up to 65535, softmax_scale
  * finite and > 0 (else PA_ERR_INVALID_ARG).  Arithmetic is

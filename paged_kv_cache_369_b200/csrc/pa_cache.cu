@@ -164,17 +164,17 @@ __global__ void __launch_bounds__(256) append_kernel(const AppendParams p) {
         if (L <= 0) continue;  // an empty sequence has no new token
         const bool first = h == 0 && c == 0;
         const int64_t pos = L - 1;
-        if (pos >= (int64_t)p.max_blocks_per_seq * kBlockSize) {
+        if (pos >= (int64_t)p.max_blocks_per_seq * p.block_size) {
             if (first) flag_error(p.err, kErrBounds);
             continue;
         }
-        const int64_t phys = p.block_tables[s * p.max_blocks_per_seq + pos / kBlockSize];
+        const int64_t phys = p.block_tables[s * p.max_blocks_per_seq + pos / p.block_size];
         if (phys < 0 || phys >= p.num_blocks) {
             if (first) flag_error(p.err, kErrBounds);
             continue;
         }
         const int64_t src = ((s * p.num_kv_heads + h) * p.head_dim + c * 8);
-        const int64_t dst = (((phys * p.num_kv_heads + h) * kBlockSize + pos % kBlockSize) * p.head_dim + c * 8);
+        const int64_t dst = (((phys * p.num_kv_heads + h) * p.block_size + pos % p.block_size) * p.head_dim + c * 8);
         const uint4 kin = *reinterpret_cast<const uint4 *>(static_cast<const uint16_t *>(p.k_new) + src);
         const uint4 vin = *reinterpret_cast<const uint4 *>(static_cast<const uint16_t *>(p.v_new) + src);
         if constexpr (FP8) {

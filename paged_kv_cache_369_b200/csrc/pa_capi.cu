@@ -38,11 +38,11 @@ pa_status from_cuda(cudaError_t e) { return e == cudaSuccess ? PA_OK : PA_ERR_CU
 // Decode kernel choice: the tensor-core kernel wherever it supports the shape;
 // the CUDA-core kernel otherwise, or everywhere when the environment variable
 // PA369_DECODE_KERNEL is "simt" (kept for A/B measurement and tests).
-bool use_mma(pa_dtype kv, int head_dim, int num_blocks, int num_kv_heads) {
+bool use_mma(pa_dtype kv, int head_dim, int num_blocks, int num_kv_heads, int block_size) {
     const char *env = getenv("PA369_DECODE_KERNEL");
     if (env && strcmp(env, "simt") == 0) return false;
     return pa::mma_decode_supported(static_cast<pa::DType>(static_cast<int>(kv)), head_dim,
-                                    num_blocks, num_kv_heads);
+                                    num_blocks, num_kv_heads, block_size);
 }
 
 // Launch whichever decode kernel applies, with its own head grouping.  With
@@ -51,7 +51,7 @@ bool use_mma(pa_dtype kv, int head_dim, int num_blocks, int num_kv_heads) {
 cudaError_t launch_any_decode(pa::DecodeParams &p, pa_dtype q, pa_dtype kv, int head_dim,
                               cudaStream_t stream) {
     const int g = p.group;
-    const bool mma = use_mma(kv, head_dim, p.num_blocks, p.num_kv_heads);
+    const bool mma = use_mma(kv, head_dim, p.num_blocks, p.num_kv_heads, p.block_size);
     if (p.append && !mma) {
         pa::AppendParams a = {};
         a.k_new = p.k_new;
@@ -66,6 +66,7 @@ cudaError_t launch_any_decode(pa::DecodeParams &p, pa_dtype q, pa_dtype kv, int 
         a.num_kv_heads = p.num_kv_heads;
         a.head_dim = head_dim;
         a.num_blocks = p.num_blocks;
+        a.block_size = p.block_size;
         a.k_scale = p.k_scale_w;
         a.v_scale = p.v_scale_w;
         const cudaError_t e = pa::launch_append(a, to_internal(q), to_internal(kv), stream);
@@ -111,7 +112,7 @@ pa_status check_decode(const DecodeArgs &a) {
     if (!is_act(a.q_dtype)) return PA_ERR_UNSUPPORTED;
     if (a.kv_dtype != a.q_dtype && !is_8bit(a.kv_dtype)) return PA_ERR_UNSUPPORTED;
     if (a.head_dim != 64 && a.head_dim != 128) return PA_ERR_UNSUPPORTED;
-    if (a.block_size != pa::kBlockSize) return PA_ERR_UNSUPPORTED;
+    if (a.block_size != 16 && a.block_size != 32) return PA_ERR_UNSUPPORTED;
     if (!isfinite(a.softmax_scale)) return PA_ERR_INVALID_ARG;
     if (is_8bit(a.kv_dtype) &&
         !(isfinite(a.k_scale) && a.k_scale > 0.f && isfinite(a.v_scale) && a.v_scale > 0.f))
@@ -122,6 +123,7 @@ pa_status check_decode(const DecodeArgs &a) {
     if (!aligned16(a.out) || !aligned16(a.q) || !aligned16(a.k_cache) || !aligned16(a.v_cache))
         return PA_ERR_INVALID_ARG;
     if (a.max_blocks_per_seq <= 0 || a.num_blocks <= 0) return PA_ERR_INVALID_ARG;
+    if ((int64_t)a.max_blocks_per_seq * a.block_size >= (int64_t(1) << 30)) return PA_ERR_UNSUPPORTED;
     const int g = a.num_q_heads / a.num_kv_heads;
     const int tg = template_group(g);
     const int64_t ycta = (int64_t)a.num_kv_heads * ((g + tg - 1) / tg);
@@ -146,6 +148,8 @@ pa::DecodeParams make_decode_params(const DecodeArgs &a, int *dev_err) {
     p.num_q_heads = a.num_q_heads;
     p.num_kv_heads = a.num_kv_heads;
     p.num_blocks = a.num_blocks;
+    p.block_size = a.block_size;
+    p.tile_shift = a.block_size == 32 ? 1 : 0;
     p.group = g;
     p.head_groups = (g + tg - 1) / tg;
     const double log2e = 1.4426950408889634074;
@@ -245,7 +249,7 @@ pa_status pa_decode(void *out, const void *q, const void *k_cache, const void *v
     const pa_status st = check_decode(a);
     if (st != PA_OK || num_seqs == 0) return st;
     pa::DecodeParams p = make_decode_params(a, dev_err);
-    p.partition_blocks = max_blocks_per_seq;
+    p.partition_blocks = max_blocks_per_seq << p.tile_shift;  // every 16-token tile
     p.num_partitions = 1;
     p.split = 0;
     return from_cuda(launch_any_decode(p, q_dtype, kv_dtype, head_dim, static_cast<cudaStream_t>(stream)));
@@ -288,7 +292,7 @@ pa_status pa_decode_append(void *out, const void *q, const void *k_new, const vo
     p.v_scale_w = is_8bit(kv_dtype) ? v_scale : 1.0f;
     const cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (!split) {
-        p.partition_blocks = max_blocks_per_seq;
+        p.partition_blocks = max_blocks_per_seq << p.tile_shift;  // every 16-token tile
         p.num_partitions = 1;
         p.split = 0;
         return from_cuda(launch_any_decode(p, q_dtype, kv_dtype, head_dim, s));
@@ -325,7 +329,7 @@ pa_status pa_prefill(void *out, const void *q, const void *k_cache, const void *
     if (!is_act(q_dtype)) return PA_ERR_UNSUPPORTED;
     if (kv_dtype != q_dtype) return PA_ERR_UNSUPPORTED;  // 8-bit caches: not on this path
     if (head_dim != 64 && head_dim != 128) return PA_ERR_UNSUPPORTED;
-    if (block_size != pa::kBlockSize) return PA_ERR_UNSUPPORTED;
+    if (block_size != 16 && block_size != 32) return PA_ERR_UNSUPPORTED;
     const int g = num_q_heads / num_kv_heads;
     if (g > 128) return PA_ERR_UNSUPPORTED;
     if (!isfinite(softmax_scale) || !(softmax_scale > 0.f)) return PA_ERR_INVALID_ARG;
@@ -336,8 +340,8 @@ pa_status pa_prefill(void *out, const void *q, const void *k_cache, const void *
         return PA_ERR_INVALID_ARG;
     if (max_blocks_per_seq <= 0 || num_blocks <= 0 || max_query_len <= 0) return PA_ERR_INVALID_ARG;
     if (num_seqs > 65535 || num_kv_heads > 65535) return PA_ERR_UNSUPPORTED;
-    const int64_t rows = (int64_t)num_blocks * num_kv_heads * pa::kBlockSize;
-    if (rows + pa::kBlockSize >= (int64_t(1) << 31)) return PA_ERR_UNSUPPORTED;
+    const int64_t rows = (int64_t)num_blocks * num_kv_heads * block_size;
+    if (rows + block_size >= (int64_t(1) << 31)) return PA_ERR_UNSUPPORTED;
     if (!pa::prefill_supported()) return PA_ERR_CUDA;
     pa::PrefillParams p = {};
     p.out = out;
@@ -355,6 +359,8 @@ pa_status pa_prefill(void *out, const void *q, const void *k_cache, const void *
     p.num_q_heads = num_q_heads;
     p.num_kv_heads = num_kv_heads;
     p.num_blocks = num_blocks;
+    p.block_size = block_size;
+    p.tile_shift = block_size == 32 ? 1 : 0;
     p.group = g;
     p.tok_per_tile = 128 / g;
     p.oob_row = (int)rows;
@@ -447,7 +453,7 @@ pa_status pa_decode_per_channel(void *out, const void *q, const void *k_cache, c
     p.v_chan = v_scales;
     const cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (partition_size == 0) {
-        p.partition_blocks = max_blocks_per_seq;
+        p.partition_blocks = max_blocks_per_seq << p.tile_shift;  // every 16-token tile
         p.num_partitions = 1;
         p.split = 0;
         return from_cuda(launch_any_decode(p, q_dtype, kv_dtype, head_dim, s));

@@ -126,7 +126,7 @@ __global__ void __launch_bounds__(kDecodeWarps * 32)
     pdl_wait();
 
     // ---- sequence length and this CTA's block range ----------------------
-    const int max_tokens = p.max_blocks_per_seq * kBlockSize;
+    const int max_tokens = p.max_blocks_per_seq * p.block_size;
     int L = p.seq_lens[s];
     if (L < 0 || L > max_tokens) {
         if (threadIdx.x == 0) flag_error(p.err, kErrBounds);
@@ -182,9 +182,9 @@ __global__ void __launch_bounds__(kDecodeWarps * 32)
     // ---- this warp's block-table entries: lane i holds the entry of the
     //      warp's block 32 * batch + i ----------------------------------------
     const int32_t *bt_row = p.block_tables + (int64_t)s * p.max_blocks_per_seq;
-    auto load_batch = [&](int batch) -> int {
+    auto load_batch = [&](int batch) -> int {  // the block holding each of the warp's tiles
         const int k = batch * 32 + lane;
-        return k < nk ? bt_row[blk_begin + warp + NW * k] : 0;
+        return k < nk ? bt_row[(blk_begin + warp + NW * k) >> p.tile_shift] : 0;
     };
     int cur_batch = 0;
     int bt_cur = load_batch(0);
@@ -196,8 +196,9 @@ __global__ void __launch_bounds__(kDecodeWarps * 32)
     };
 
     const uint8_t *kc = p.k_cache, *vc = p.v_cache;
-    const int64_t head_off = (int64_t)kvh * C::TILE_BYTES;
-    const int64_t blk_stride = (int64_t)p.num_kv_heads * C::TILE_BYTES;
+    const int tiles_per_block = 1 << p.tile_shift;
+    const int64_t head_off = (int64_t)kvh * tiles_per_block * C::TILE_BYTES;
+    const int64_t blk_stride = (int64_t)p.num_kv_heads * tiles_per_block * C::TILE_BYTES;
     auto issue = [&](int k) {  // called by the whole warp
         int phys = bt_of(k);
         if (lane == 0) {
@@ -208,7 +209,8 @@ __global__ void __launch_bounds__(kDecodeWarps * 32)
             const int st = k % NST;
             const uint32_t bar = bar0 + 8 * st;
             const uint32_t dst = stage0 + st * C::STAGE_BYTES;
-            const int64_t off = (int64_t)phys * blk_stride + head_off;
+            const int sub = (blk_begin + warp + NW * k) & (tiles_per_block - 1);  // tile in block
+            const int64_t off = (int64_t)phys * blk_stride + head_off + (int64_t)sub * C::TILE_BYTES;
             mbar_arrive_expect_tx(bar, C::STAGE_BYTES);
             bulk_g2s(dst, kc + off, C::TILE_BYTES, bar);
             bulk_g2s(dst + C::TILE_BYTES, vc + off, C::TILE_BYTES, bar);

@@ -187,7 +187,7 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, 3)
     pdl_wait();
 
     // ---- sequence length and this CTA's block range -----------------------
-    const int max_tokens = p.max_blocks_per_seq * kBlockSize;
+    const int max_tokens = p.max_blocks_per_seq * p.block_size;
     int L = p.seq_lens[s];
     if (L < 0 || L > max_tokens) {
         if (threadIdx.x == 0) flag_error(p.err, kErrBounds);
@@ -211,10 +211,11 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, 3)
 
     // ---- block table entries of this warp, one per lane --------------------
     const int32_t *bt_row = p.block_tables + (int64_t)s * p.max_blocks_per_seq;
-    auto load_batch = [&](int batch) -> int {
+    auto load_batch = [&](int batch) -> int {  // the block holding each of the warp's tiles
         const int k = batch * 32 + lane;
-        return k < nk ? bt_row[blk_begin + warp + NW * k] : 0;
+        return k < nk ? bt_row[(blk_begin + warp + NW * k) >> p.tile_shift] : 0;
     };
+    const int tile_mask = (1 << p.tile_shift) - 1;
     int cur_batch = 0;
     int bt_cur = load_batch(0);
     int bt_nxt = nk > 32 ? load_batch(1) : 0;
@@ -233,7 +234,8 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, 3)
             const int st = k % NST;
             const uint32_t bar = bar0 + 8 * st;
             const uint32_t dst = stage0 + st * C::STAGE_BYTES;
-            const int y = (phys * p.num_kv_heads + kvh) * kBlockSize;
+            const int sub = (blk_begin + warp + NW * k) & tile_mask;  // tile within the block
+            const int y = (phys * p.num_kv_heads + kvh) * p.block_size + sub * kBlockSize;
             mbar_arrive_expect_tx(bar, C::STAGE_BYTES);
 #pragma unroll
             for (int b = 0; b < C::NBOX; ++b) {
@@ -377,7 +379,8 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, 3)
             constexpr int CPR = C::ROW_BYTES / 16;        // 16-byte chunks per tile row
             constexpr int SRC_ELEMS = C::FP8 ? 16 : 8;    // activations per chunk
             const int64_t src_row = ((int64_t)s * p.num_kv_heads + kvh) * D;
-            const int64_t dst_row = ((phys * p.num_kv_heads + kvh) * kBlockSize + r) * C::ROW_BYTES;
+            const int64_t dst_row =
+                ((phys * p.num_kv_heads + kvh) * p.block_size + (L - 1) % p.block_size) * C::ROW_BYTES;
             for (int c = lane; c < 2 * CPR; c += 32) {
                 const bool isv = c >= CPR;
                 const int cc = isv ? c - CPR : c;
@@ -657,7 +660,7 @@ namespace {
 template <typename QT, typename KVT, int D, int GT>
 cudaError_t launch_mma_t(const DecodeParams &p, cudaStream_t stream) {
     using C = MmaCfg<QT, KVT, D, GT>;
-    const int64_t rows = (int64_t)p.num_blocks * p.num_kv_heads * kBlockSize;
+    const int64_t rows = (int64_t)p.num_blocks * p.num_kv_heads * p.block_size;
     CUtensorMap mk, mv;
     if (!encode_pool_map(&mk, p.k_cache, C::EB, D, rows) ||
         !encode_pool_map(&mv, p.v_cache, C::EB, D, rows))
@@ -685,9 +688,9 @@ cudaError_t mma_by_rows(const DecodeParams &p, int gt, cudaStream_t stream) {
 
 }  // namespace
 
-bool mma_decode_supported(DType kv, int head_dim, int num_blocks, int num_kv_heads) {
+bool mma_decode_supported(DType kv, int head_dim, int num_blocks, int num_kv_heads, int block_size) {
     if (!encode_fn()) return false;
-    const int64_t rows = (int64_t)num_blocks * num_kv_heads * kBlockSize;
+    const int64_t rows = (int64_t)num_blocks * num_kv_heads * block_size;
     if (rows >= (int64_t(1) << 31)) return false;  // TMA row coordinate is a signed 32-bit int
     if (is_8bit(kv)) return head_dim == 128;
     return head_dim == 64 || head_dim == 128;

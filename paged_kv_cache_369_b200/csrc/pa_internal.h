@@ -8,7 +8,12 @@
 
 namespace pa {
 
-constexpr int kBlockSize = 16;        // tokens per KV block
+// Kernels work in tiles of 16 tokens (one TMA box, one MMA n-tile).  A pool
+// block holds block_size = 16 or 32 tokens, i.e. 1 or 2 tiles: tile u of a
+// sequence lives in its block u >> tile_shift, at row (u & (tiles per block
+// - 1)) * 16 of that block.
+constexpr int kBlockSize = 16;        // tokens per tile
+constexpr int kMaxBlockSize = 32;     // largest supported pool block
 constexpr int kDecodeWarps = 4;       // consumer warps per decode CTA
 constexpr uint64_t kWaitLimitNs = 1000000000ull;  // 1 s bound on any device wait
 constexpr int kErrBounds = 4;         // = PA_ERR_DEVICE_BOUNDS
@@ -65,9 +70,11 @@ struct DecodeParams {
     int num_q_heads;
     int num_kv_heads;
     int num_blocks;
+    int block_size;             // tokens per pool block: 16 or 32
+    int tile_shift;             // log2(block_size / 16)
     int group;                  // Hq / Hk
     int head_groups;            // CTAs per KV head (ceil(group / G))
-    int partition_blocks;       // KV blocks per partition
+    int partition_blocks;       // 16-token tiles per partition
     int num_partitions;         // NP (1 in single-pass mode)
     int split;                  // 1: write partials to the workspace
     float qk_scale_log2;        // softmax_scale * k_scale * log2(e)
@@ -100,6 +107,7 @@ struct AppendParams {  // decode-form slot mapping + cache write in one kernel
     int num_kv_heads;
     int head_dim;
     int num_blocks;
+    int block_size;
     float k_scale;
     float v_scale;
 };
@@ -130,6 +138,8 @@ struct PrefillParams {  // chunked prefill (pa_prefill)
     int num_q_heads;
     int num_kv_heads;
     int num_blocks;
+    int block_size;             // tokens per pool block: 16 or 32
+    int tile_shift;             // log2(block_size / 16)
     int group;                  // Hq / Hk
     int tok_per_tile;           // floor(128 / group) chunk tokens per query tile
     int oob_row;                // a pool row index past the end (zero-filled loads)
@@ -164,7 +174,7 @@ cudaError_t launch_prefill(const PrefillParams &p, DType q, int head_dim, cudaSt
 // Tensor-core decode (pa_decode_mma.cu): rows of the MMA used for the GQA
 // group (8 or 16); supported for head_dim 64/128 16-bit caches and head_dim
 // 128 8-bit caches whose pool has fewer than 2^31 token rows.
-bool mma_decode_supported(DType kv, int head_dim, int num_blocks, int num_kv_heads);
+bool mma_decode_supported(DType kv, int head_dim, int num_blocks, int num_kv_heads, int block_size);
 cudaError_t launch_decode_mma(const DecodeParams &p, DType q, DType kv, int head_dim, int mma_rows,
                               cudaStream_t stream);
 

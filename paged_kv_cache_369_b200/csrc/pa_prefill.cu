@@ -258,7 +258,7 @@ __global__ void __launch_bounds__(320, 1)
     const int L = p.seq_lens[s];
     const int q0 = p.query_start[s];
     const int n = p.query_start[s + 1] - q0;
-    if (L < 0 || L > p.max_blocks_per_seq * kBlockSize || n < 0 || n > L || q0 < 0 ||
+    if (L < 0 || L > p.max_blocks_per_seq * p.block_size || n < 0 || n > L || q0 < 0 ||
         q0 + n > p.num_tokens || n > p.max_query_len) {
         if (threadIdx.x == 0 && cta_tile == 0 && kvh == 0) flag_error(p.err, kErrBounds);
         return;
@@ -268,7 +268,8 @@ __global__ void __launch_bounds__(320, 1)
     const int ntok = min(2 * tpt, n - tok0);
     const int ctx = L - n;
     const int nt = (ctx + tok0 + ntok - 1) / C::BN + 1;  // key tiles up to the last row's position
-    const int nblk_seq = (L + kBlockSize - 1) / kBlockSize;
+    const int nblk_seq = (L + kBlockSize - 1) / kBlockSize;  // 16-token tiles
+    const int tile_mask = (1 << p.tile_shift) - 1;
 
     const uint32_t bars = base + C::OFF_BAR;
     const uint32_t bar_q = bars;
@@ -339,9 +340,9 @@ __global__ void __launch_bounds__(320, 1)
                     const int lb = j * (C::BN / kBlockSize) + b;
                     int y = p.oob_row;  // past the pool: a zero-filled box
                     if (lb < nblk_seq) {
-                        const int phys = bt[lb];
+                        const int phys = bt[lb >> p.tile_shift];
                         if ((unsigned)phys < (unsigned)p.num_blocks)
-                            y = (phys * p.num_kv_heads + kvh) * kBlockSize;
+                            y = (phys * p.num_kv_heads + kvh) * p.block_size + (lb & tile_mask) * kBlockSize;
                         else
                             flag_error(p.err, kErrBounds);
                     }
@@ -591,7 +592,7 @@ bool encode_q_map(CUtensorMap *m, const void *q, int d, int hq, int64_t tokens, 
 template <typename T, int D>
 cudaError_t launch_prefill_t(const PrefillParams &p, cudaStream_t stream) {
     using C = PfCfg<T, D>;
-    const int64_t rows = (int64_t)p.num_blocks * p.num_kv_heads * kBlockSize;
+    const int64_t rows = (int64_t)p.num_blocks * p.num_kv_heads * p.block_size;
     CUtensorMap mq, mk, mv;
     if (!encode_q_map(&mq, p.q, D, p.num_q_heads, p.num_tokens, p.group, p.tok_per_tile) ||
         !encode_pool_map(&mk, p.k_cache, 2, D, rows) || !encode_pool_map(&mv, p.v_cache, 2, D, rows))

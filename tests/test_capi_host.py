@@ -76,7 +76,8 @@ def _decode(pa, **kw):
 @pytest.mark.parametrize("kw,status", [
     (dict(d=96), 2),                                  # head_dim
     (dict(d=256), 2),
-    (dict(B=32), 2),                                  # block size
+    (dict(B=64), 2),                                  # block size (16 or 32)
+    (dict(B=8), 2),
     (dict(Hq=8, Hk=3), 1),                            # Hq % Hk
     (dict(Hk=0), 1),
     (dict(qd=2), 2),                                  # fp8 query
@@ -189,7 +190,7 @@ def test_prefill_checks(pa):
     assert call(kvd=pa.PA_FP8_E4M3) == 2     # E4M3 caches: not on the prefill path
     assert call(qd=pa.PA_F16) == 2           # cache dtype must be the q dtype
     assert call(d=96) == 2
-    assert call(B=32) == 2
+    assert call(B=64) == 2
     assert call(Hq=8, Hk=3) == 1
     assert call(Hq=256, Hk=1) == 2           # group above 128
     assert call(qs=0) == 1

@@ -31,15 +31,16 @@ def _to_dev(a: np.ndarray, dtype: str) -> torch.Tensor:
     return t.cuda()
 
 
-@pytest.mark.parametrize("kv,Hk,d", [("f16", 2, 64), ("bf16", 8, 128), ("e4m3", 8, 128),
-                                     ("bf16", 1, 64), ("e4m3", 32, 128)])
-def test_copy_blocks_bitwise(kv, Hk, d):
+@pytest.mark.parametrize("kv,Hk,d,B", [("f16", 2, 64, 16), ("bf16", 8, 128, 16), ("e4m3", 8, 128, 16),
+                                       ("bf16", 1, 64, 16), ("e4m3", 32, 128, 16),
+                                       ("bf16", 8, 128, 32)])
+def test_copy_blocks_bitwise(kv, Hk, d, B):
     pa, _ = _pa()
-    rng = np.random.default_rng({"f16": 1, "bf16": 2, "e4m3": 3}[kv] * 1000 + Hk * 10 + d)
+    rng = np.random.default_rng({"f16": 1, "bf16": 2, "e4m3": 3}[kv] * 1000 + Hk * 10 + d + B)
     nb = 96
     dt = np.uint8 if kv == "e4m3" else np.uint16
-    kc = rng.integers(0, np.iinfo(dt).max, size=(nb, Hk, 16, d), dtype=dt)
-    vc = rng.integers(0, np.iinfo(dt).max, size=(nb, Hk, 16, d), dtype=dt)
+    kc = rng.integers(0, np.iinfo(dt).max, size=(nb, Hk, B, d), dtype=dt)
+    vc = rng.integers(0, np.iinfo(dt).max, size=(nb, Hk, B, d), dtype=dt)
     ids = rng.permutation(nb)
     pairs = np.stack([ids[:40], ids[40:80]], 1).astype(np.int32)
     pairs = np.concatenate([pairs, [[int(ids[90]), int(ids[90])]]]).astype(np.int32)  # src == dst

@@ -155,6 +155,36 @@ def test_per_channel_scales_parity(case, mode, P, kernel_choice):
                  f"per-channel case {case} {mode} P={P} kernel={kernel_choice}")
 
 
+BLOCK32 = [
+    # (Hq, Hk, d, act, kv, lens): 32-token pool blocks
+    (32, 8, 128, "bf16", "bf16", [1, 31, 32, 33, 100, 513, 700]),
+    (4, 2, 64, "f16", "f16", [10, 45, 20, 33]),
+    (64, 8, 128, "bf16", "e4m3", [600, 17, 1024]),
+    (8, 8, 128, "f16", "int8", [95, 1]),
+]
+
+
+@pytest.mark.parametrize("mode,P", [("single", 512), ("split", 512), ("split", 16), ("fused", 64),
+                                    ("fused_single", 512)])
+@pytest.mark.parametrize("case", range(len(BLOCK32)))
+def test_block_size_32_parity(case, mode, P, kernel_choice):
+    """Pools of 32-token blocks (the fifth page's §2.2: blocks of 16-32
+    tokens): slot mapping, cache write and append bit-exact, decode within
+    tolerance, including 16-token partitions that end inside a block."""
+    pa, PagedDecode = _pa()
+    Hq, Hk, d, act, kv, lens = BLOCK32[case]
+    w = workload.build(f"b32_{case}", 4000 + case, lens, Hq, Hk, d, act, kv, block_size=32,
+                       extra_table_cols=1)
+    dec = PagedDecode(w, mode=mode, partition_size=P)
+    dec.step()
+    torch.cuda.synchronize()
+    assert dec.error() == 0
+    kc, vc = oracle.caches_for(w)
+    check_pools(dec, kc, vc)
+    assert_close(_to_f64(dec.out), oracle.decode_for(w, kc, vc),
+                 f"block 32 case {case} {mode} P={P} kernel={kernel_choice}")
+
+
 def test_split_partials_match_oracle(kernel_choice):
     pa, PagedDecode = _pa()
     w = workload.build("partials", 77, [1, 16, 17, 100, 513, 1100], 16, 4, 128, "bf16", "bf16")

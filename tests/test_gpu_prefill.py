@@ -139,3 +139,17 @@ def test_prefill_bad_chunk_is_reported():
     assert pre.error() == PA_ERR_DEVICE_BOUNDS
     assert not out[:5].any()              # the bad sequence's rows are not written
     assert torch.isfinite(out.float()).all()
+
+
+@pytest.mark.parametrize("case", [0, 2, 4])
+def test_prefill_block_size_32(case):
+    """32-token pool blocks: the same small shapes as above."""
+    ctx, chunk, Hq, Hk, d, dt = SMALL[case]
+    w = workload.build_chunked(f"pf32_{case}", 2100 + case, ctx, chunk, Hq, Hk, d, dt, dt,
+                               block_size=32, extra_table_cols=1)
+    pre = _run(w)
+    assert pre.error() == 0
+    kc, vc = oracle.chunked_caches_for(w)
+    assert np.array_equal(pool_bytes(pre.k_cache), kc.view(np.uint8).reshape(pool_bytes(pre.k_cache).shape))
+    ref = oracle.prefill_for(w, kc, vc)
+    assert_close(_f64(pre.out), ref, f"prefill block 32 case {case}")
