@@ -153,7 +153,9 @@ __device__ __forceinline__ uint32_t swz(int r, int c) {
     return (uint32_t)((c >> 3) * (kBlockSize * 128) + r * 128 + (((c & 7) ^ (r & 7)) << 4));
 }
 
-template <typename QT, typename KVT, int D, int GT>
+// CHAN: per-channel scales (8-bit caches only), a separate instantiation so
+// that the per-tensor kernels compile exactly as without them
+template <typename QT, typename KVT, int D, int GT, bool CHAN>
 __global__ void __launch_bounds__(kDecodeWarps * 32, 3)
     decode_mma_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmap_k,
                       const __grid_constant__ CUtensorMap tmap_v) {
@@ -276,7 +278,7 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, 3)
                     const uint32_t w23 = *reinterpret_cast<const uint32_t *>(qrow + d2);
                     unpack2(QT{}, w01, v0, v1);
                     unpack2(QT{}, w23, v2, v3);
-                    if (p.k_chan) {  // per-channel K scales: q.(code * s) = (q * s).code
+                    if constexpr (CHAN) {  // per-channel K scales: q.(code * s) = (q * s).code
                         const float *kc = p.k_chan + (int64_t)kvh * D;
                         v0 *= kc[d0]; v1 *= kc[d1]; v2 *= kc[d2]; v3 *= kc[d3];
                     }
@@ -284,7 +286,7 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, 3)
                 qv[hh][ks][0] = v0; qv[hh][ks][1] = v1; qv[hh][ks][2] = v2; qv[hh][ks][3] = v3;
             }
         }
-        if (!std::is_same<QT, ET>::value || p.k_chan) {
+        if constexpr (!std::is_same<QT, ET>::value || CHAN) {
             // bf16 q against an f16 tensor-core path (8-bit cache), or q times
             // per-channel scales: scale q by a power of two so its largest
             // element sits near 2^14, convert to f16, and fold the inverse
@@ -606,7 +608,8 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, 3)
                 O = fmaf(f, accs[(w * GT + i) * D + d], O);
             }
         }
-        const float vs = p.v_chan ? p.v_chan[(int64_t)kvh * D + d] : p.v_scale;
+        float vs = p.v_scale;
+        if constexpr (CHAN) vs = p.v_chan[(int64_t)kvh * D + d];
         const float ov = Ls > 0.f ? (O / Ls) * vs : 0.f;
         const int64_t row = (int64_t)s * p.num_q_heads + hq;
         if (!p.split) {
@@ -657,7 +660,7 @@ bool encode_pool_map(CUtensorMap *m, const void *base, int elem_bytes, int d, in
 
 namespace {
 
-template <typename QT, typename KVT, int D, int GT>
+template <typename QT, typename KVT, int D, int GT, bool CHAN>
 cudaError_t launch_mma_t(const DecodeParams &p, cudaStream_t stream) {
     using C = MmaCfg<QT, KVT, D, GT>;
     const int64_t rows = (int64_t)p.num_blocks * p.num_kv_heads * p.block_size;
@@ -665,7 +668,7 @@ cudaError_t launch_mma_t(const DecodeParams &p, cudaStream_t stream) {
     if (!encode_pool_map(&mk, p.k_cache, C::EB, D, rows) ||
         !encode_pool_map(&mv, p.v_cache, C::EB, D, rows))
         return cudaErrorInvalidValue;
-    auto kern = decode_mma_kernel<QT, KVT, D, GT>;
+    auto kern = decode_mma_kernel<QT, KVT, D, GT, CHAN>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
@@ -683,7 +686,13 @@ cudaError_t launch_mma_t(const DecodeParams &p, cudaStream_t stream) {
 
 template <typename QT, typename KVT, int D>
 cudaError_t mma_by_rows(const DecodeParams &p, int gt, cudaStream_t stream) {
-    return gt == 16 ? launch_mma_t<QT, KVT, D, 16>(p, stream) : launch_mma_t<QT, KVT, D, 8>(p, stream);
+    if constexpr (Elem<KVT>::kBytes == 1) {
+        if (p.k_chan)
+            return gt == 16 ? launch_mma_t<QT, KVT, D, 16, true>(p, stream)
+                            : launch_mma_t<QT, KVT, D, 8, true>(p, stream);
+    }
+    return gt == 16 ? launch_mma_t<QT, KVT, D, 16, false>(p, stream)
+                    : launch_mma_t<QT, KVT, D, 8, false>(p, stream);
 }
 
 }  // namespace
