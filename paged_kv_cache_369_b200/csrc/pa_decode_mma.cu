@@ -11,9 +11,10 @@
 // which keeps the kernel on the HBM roofline up to GQA 16 and for FP8 caches.
 //
 // Layout of the work:
-//   - one CTA per (sequence, partition, KV head, head group of <= 16); 4 warps,
-//     each owning every 4th block of the partition with a private ring of
-//     shared-memory stages filled by TMA (cp.async.bulk.tensor.2d, no multicast);
+//   - one CTA per (sequence, partition, KV head, head group of <= 16); 4 warps
+//     (2 for long split contexts), each owning every 4th (2nd) 16-token tile of
+//     the partition with a private ring of shared-memory stages filled by TMA
+//     (cp.async.bulk.tensor.2d, no multicast);
 //   - a tile row is 128 bytes per TMA box (d = 64 16-bit, or half of d = 128
 //     16-bit, or d = 128 E4M3) and the box lands 128B-swizzled, so ldmatrix of
 //     8 token rows at one 16-byte column touches 8 distinct bank groups;
@@ -121,12 +122,12 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map
 
 }  // namespace mma_detail
 
-template <typename QT, typename KVT, int D, int GT> struct MmaCfg {
+template <typename QT, typename KVT, int D, int GT, int NW_ = kDecodeWarps> struct MmaCfg {
     using ET = typename mma_detail::MmaType<KVT>::T;
     static constexpr bool FP8 = Elem<KVT>::kBytes == 1;
     static constexpr bool HILO = (Elem<KVT>::kBytes == 2) && sizeof(ET) == 2 &&
                                  std::is_same<KVT, bf16_t>::value;
-    static constexpr int NW = kDecodeWarps;
+    static constexpr int NW = NW_;  // warps per CTA
     static constexpr int EB = Elem<KVT>::kBytes;
     static constexpr int ROW_BYTES = D * EB;
     static constexpr int NBOX = ROW_BYTES / 128;  // 128-byte TMA boxes per row
@@ -155,11 +156,11 @@ __device__ __forceinline__ uint32_t swz(int r, int c) {
 
 // CHAN: per-channel scales (8-bit caches only), a separate instantiation so
 // that the per-tensor kernels compile exactly as without them
-template <typename QT, typename KVT, int D, int GT, bool CHAN>
-__global__ void __launch_bounds__(kDecodeWarps * 32, 3)
+template <typename QT, typename KVT, int D, int GT, bool CHAN, int NWARPS>
+__global__ void __launch_bounds__(NWARPS * 32, 12 / NWARPS)
     decode_mma_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmap_k,
                       const __grid_constant__ CUtensorMap tmap_v) {
-    using C = MmaCfg<QT, KVT, D, GT>;
+    using C = MmaCfg<QT, KVT, D, GT, NWARPS>;
     using ET = typename C::ET;
     using namespace mma_detail;
     constexpr int NW = C::NW, NST = C::NST;
@@ -660,15 +661,15 @@ bool encode_pool_map(CUtensorMap *m, const void *base, int elem_bytes, int d, in
 
 namespace {
 
-template <typename QT, typename KVT, int D, int GT, bool CHAN>
+template <typename QT, typename KVT, int D, int GT, bool CHAN, int NWARPS>
 cudaError_t launch_mma_t(const DecodeParams &p, cudaStream_t stream) {
-    using C = MmaCfg<QT, KVT, D, GT>;
+    using C = MmaCfg<QT, KVT, D, GT, NWARPS>;
     const int64_t rows = (int64_t)p.num_blocks * p.num_kv_heads * p.block_size;
     CUtensorMap mk, mv;
     if (!encode_pool_map(&mk, p.k_cache, C::EB, D, rows) ||
         !encode_pool_map(&mv, p.v_cache, C::EB, D, rows))
         return cudaErrorInvalidValue;
-    auto kern = decode_mma_kernel<QT, KVT, D, GT, CHAN>;
+    auto kern = decode_mma_kernel<QT, KVT, D, GT, CHAN, NWARPS>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
@@ -684,15 +685,29 @@ cudaError_t launch_mma_t(const DecodeParams &p, cudaStream_t stream) {
     return cudaLaunchKernelEx(&cfg, kern, p, mk, mv);
 }
 
+// Warps per CTA.  Four warps share a partition's tiles and merge their
+// softmax states; with many partitions per sequence (long contexts) two warps
+// per CTA do better: half the per-CTA q preparation and merge work for the
+// same 12 warps per SM (long-context E4M3 shape, 512-token partitions: 146.6
+// -> 130.1 us), while for shorter, uneven sequences the smaller work units of
+// four warps balance better over the SMs (Qwen3-8B shape: 105.2 vs 111.9 us).
+constexpr int kLongSplitPartitions = 16;
+
+template <typename QT, typename KVT, int D, bool CHAN>
+cudaError_t mma_by_warps(const DecodeParams &p, int gt, cudaStream_t stream) {
+    if (p.split && p.num_partitions >= kLongSplitPartitions)
+        return gt == 16 ? launch_mma_t<QT, KVT, D, 16, CHAN, 2>(p, stream)
+                        : launch_mma_t<QT, KVT, D, 8, CHAN, 2>(p, stream);
+    return gt == 16 ? launch_mma_t<QT, KVT, D, 16, CHAN, kDecodeWarps>(p, stream)
+                    : launch_mma_t<QT, KVT, D, 8, CHAN, kDecodeWarps>(p, stream);
+}
+
 template <typename QT, typename KVT, int D>
 cudaError_t mma_by_rows(const DecodeParams &p, int gt, cudaStream_t stream) {
     if constexpr (Elem<KVT>::kBytes == 1) {
-        if (p.k_chan)
-            return gt == 16 ? launch_mma_t<QT, KVT, D, 16, true>(p, stream)
-                            : launch_mma_t<QT, KVT, D, 8, true>(p, stream);
+        if (p.k_chan) return mma_by_warps<QT, KVT, D, true>(p, gt, stream);
     }
-    return gt == 16 ? launch_mma_t<QT, KVT, D, 16, false>(p, stream)
-                    : launch_mma_t<QT, KVT, D, 8, false>(p, stream);
+    return mma_by_warps<QT, KVT, D, false>(p, gt, stream);
 }
 
 }  // namespace

@@ -18,7 +18,7 @@
 // shares each K/V tile it reads; the CTA's two tiles (A, B: consecutive token
 // ranges) share them too.  Keys come in tiles of 64 = 4 blocks of 16 tokens.
 //   - warp 8 (one lane), TMA producer: both Q tiles once through a 3-D
-//     tensor map over q [T, Hq, d]; per key tile, the 8 K and 8 V blocks named
+//     tensor map over q [T, Hq, d]; per key tile, the 4 K and 4 V blocks named
 //     by the block table through the pool's 2-D map (16-row x 128-byte boxes,
 //     128B swizzle) into a 4-stage ring.  Blocks past the sequence's end are
 //     fetched from past the end of the map, which the copy fills with zeros.
