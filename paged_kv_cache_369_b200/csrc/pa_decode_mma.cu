@@ -94,6 +94,37 @@ template <typename KVT> __device__ __forceinline__ uint32_t cvt8x2_f16x2(uint32_
     return ::pa::cvt8x2_f16x2(two, KVT{});
 }
 
+__device__ __forceinline__ uint32_t prmt2(uint32_t a, uint32_t b, uint32_t sel) {
+    uint32_t r;
+    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(sel));
+    return r;
+}
+__device__ __forceinline__ uint32_t hsub2(uint32_t a, uint32_t b) {
+    uint32_t r;
+    asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+    return r;
+}
+
+// Four 8-bit codes of one word -> two f16x2 (exact).  SEL_LO / SEL_HI name
+// the byte pairs: 0x10 / 0x32 for bytes (0,1) / (2,3), 0x20 / 0x31 for the
+// interleaved pairs (0,2) / (1,3).
+template <typename KVT, uint32_t SEL_LO, uint32_t SEL_HI>
+__device__ __forceinline__ void cvt8x4_f16x2(uint32_t w, uint32_t &lo, uint32_t &hi) {
+    if constexpr (std::is_same<KVT, i8_t>::value) {
+        // the biased byte b ^ 0x80 goes under the f16 exponent byte 0x64
+        // (value 1024 + 128 + b); subtracting 1152 leaves b
+        const uint32_t x = w ^ 0x80808080u;
+        constexpr uint32_t kLo = 0x5040u | ((SEL_LO & 0xFu) | ((SEL_LO >> 4) << 8));
+        constexpr uint32_t kHi = 0x5040u | ((SEL_HI & 0xFu) | ((SEL_HI >> 4) << 8));
+        lo = hsub2(prmt2(x, 0x6464u, kLo), 0x64806480u);
+        hi = hsub2(prmt2(x, 0x6464u, kHi), 0x64806480u);
+    } else {
+        const uint32_t a = (SEL_LO == 0x10u) ? w : prmt2(w, 0u, 0x3120u);
+        lo = cvt8x2_f16x2<KVT>(a);
+        hi = cvt8x2_f16x2<KVT>(a >> 16);
+    }
+}
+
 __device__ __forceinline__ uint32_t pack2(float lo, float hi, f16_t) {
     uint32_t r;
     asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
@@ -428,8 +459,11 @@ __global__ void __launch_bounds__(NWARPS * 32, 12 / NWARPS)
 #pragma unroll
                 for (int h = 0; h < 2; ++h) {
                     const int ks = 2 * jj + h;
-                    mma16816(sc[0], qa[ks], cvt8x2_f16x2<KVT>(w[h]), cvt8x2_f16x2<KVT>(w[h] >> 16), ET{});
-                    mma16816(sc[1], qa[ks], cvt8x2_f16x2<KVT>(w[2 + h]), cvt8x2_f16x2<KVT>(w[2 + h] >> 16), ET{});
+                    uint32_t b0, b1, b2, b3;
+                    cvt8x4_f16x2<KVT, 0x10u, 0x32u>(w[h], b0, b1);
+                    cvt8x4_f16x2<KVT, 0x10u, 0x32u>(w[2 + h], b2, b3);
+                    mma16816(sc[0], qa[ks], b0, b1, ET{});
+                    mma16816(sc[1], qa[ks], b2, b3, ET{});
                 }
             }
         }
@@ -528,10 +562,10 @@ __global__ void __launch_bounds__(NWARPS * 32, 12 / NWARPS)
                 ldsm_x4_t(w, vt + swz(lrow_v, 2 * cp + lsel_v));
 #pragma unroll
                 for (int h = 0; h < 2; ++h) {
-                    const uint32_t lo_t = prmt(w[2 * h], 0x3120);      // tokens 0-7
-                    const uint32_t hi_t = prmt(w[2 * h + 1], 0x3120);  // tokens 8-15
-                    uint32_t av[4] = {cvt8x2_f16x2<KVT>(lo_t), cvt8x2_f16x2<KVT>(lo_t >> 16),
-                                      cvt8x2_f16x2<KVT>(hi_t), cvt8x2_f16x2<KVT>(hi_t >> 16)};
+                    // regroup bytes: (tok 2kq, 2kq+1) at even d, then at odd d
+                    uint32_t av[4];
+                    cvt8x4_f16x2<KVT, 0x20u, 0x31u>(w[2 * h], av[0], av[1]);      // tokens 0-7
+                    cvt8x4_f16x2<KVT, 0x20u, 0x31u>(w[2 * h + 1], av[2], av[3]);  // tokens 8-15
                     if (!full) {
                         av[0] &= m0; av[1] &= m0; av[2] &= m8; av[3] &= m8;
                     }
