@@ -202,7 +202,7 @@ def workload_config(w, cfg: int, mode: str, P: int) -> dict:
         "block_size": w.block_size, "kv_dtype": w.kv_dtype, "act_dtype": w.act_dtype,
         "seq_len_mean": float(w.seq_lens.mean()), "seq_len_min": int(w.seq_lens.min()),
         "seq_len_max": int(w.seq_lens.max()), "num_blocks": w.num_blocks, "seed": w.seed,
-        "mode": mode, "partition_size": P if mode in ("split", "fused") else None,
+        "mode": mode, "partition_size": P if mode in ("split", "fused", "cascade") else None,
         "l2": "inputs larger than L2: no flush" if w.kv_bytes_logical() > 256e6
         else "L2 flushed (256 MB write) between steps",
     }
@@ -445,7 +445,8 @@ def run_ours(args):
                                 device_id=device)
 
     import workload
-    from paged_kv_cache_369_b200.runner import PagedDecode, algorithmic_decode_bytes
+    from paged_kv_cache_369_b200.runner import (PagedDecode, algorithmic_cascade_bytes,
+                                                algorithmic_decode_bytes)
 
     w = workload.config(args.config, kv_dtype=args.kv, channel_scales=args.channel_scales)
     stream = torch.cuda.Stream(device)
@@ -456,6 +457,8 @@ def run_ours(args):
     step_bytes = w.step_bytes()
     # the fused attention launch also reads the new rows and stores them
     attn_bytes = step_bytes if fused else algorithmic_decode_bytes(w)
+    if args.mode == "cascade":  # the shared prefix is read once, not once per sequence
+        attn_bytes = algorithmic_cascade_bytes(w)
     flush = None
     if w.kv_bytes_logical() <= 256e6:
         flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=device)
@@ -567,7 +570,8 @@ def run_ours(args):
                     "fused": "pa_decode_append: decode kernel storing the new tokens + split reduce kernel",
                     "fused_single": "pa_decode_append: single-pass decode kernel storing the new tokens",
                     "split": "pa_decode_split_reduce: decode partition kernel + split reduce kernel",
-                    "single": "pa_decode: single-pass decode kernel"}[args.mode],
+                    "single": "pa_decode: single-pass decode kernel",
+                    "cascade": "pa_decode_shared_prefix: prefix pass (tcgen05) + tail decode + merge"}[args.mode],
                 "peak_source": f"{peak_kind} HBM copy bandwidth (MEASURED_PEAKS.json hbm_gbs)"
                 if peak_kind == "measured" else "fallback 6.65 TB/s",
                 "algorithmic_bytes_per_launch": attn_bytes,
@@ -595,7 +599,9 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--config", type=int, default=2, choices=(1, 2, 3, 4, 5))
-    ap.add_argument("--mode", choices=("fused", "fused_single", "split", "single"), default="fused")
+    ap.add_argument("--mode", choices=("fused", "fused_single", "split", "single", "cascade"),
+                    default="fused",
+                    help="cascade: the shared-prefix decode (config 5's common prefix attended once)")
     ap.add_argument("--partition", type=int, default=512)
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")

@@ -338,6 +338,47 @@ pa_status pa_decode_per_channel(void *out, const void *q, const void *k_cache, c
                                 int max_seq_len, void *workspace, size_t workspace_bytes,
                                 int *dev_err, void *stream);
 
+/*
+ * pa_decode_shared_prefix -- decode for a batch whose sequences all begin with
+ * the same cached prefix (the same physical blocks), computing the prefix once.
+ *
+ * Source: "大语言模型推理引擎深度剖析", §2.3 (requests sharing a system prompt /
+ * prompt prefix share the same KV cache blocks) and "Transformer 推理优化：KV
+ * Cache、PagedAttention 与 vLLM", §3.5; the result is pa_decode's, split by
+ * the log-sum-exp decomposition described at pa_decode_split_reduce.
+ *
+ * Requirements: the first prefix_len / block_size entries of every row of
+ * block_tables are the same blocks (row 0 is read for them; the caller's
+ * allocator guarantees the sharing), prefix_len is a positive multiple of
+ * block_size, every seq_lens[s] >= prefix_len (a shorter one flags
+ * PA_ERR_DEVICE_BOUNDS), kv_dtype = q_dtype (16-bit caches), softmax_scale > 0,
+ * GQA groups up to 128.  Three launches on `stream`:
+ *   1. the prefix: for each KV head, the queries of all sequences against the
+ *      prefix keys as one dense tensor-core pass (the prefix K/V is read once,
+ *      not once per sequence), giving each (sequence, head) a partial
+ *      (lse, o) in workspace slot 0;
+ *   2. the tails (positions prefix_len .. L - 1) in partitions of
+ *      partition_size tokens (a positive multiple of 16): slots 1 ..;
+ *   3. the merge of slot 0 with the tail partitions into out.
+ * workspace: >= pa_shared_prefix_workspace_bytes(num_seqs, num_q_heads,
+ * head_dim, max_seq_len, prefix_len, partition_size) bytes, 256-byte aligned:
+ * lse [S, Hq, NP] fp32, then o [S, Hq, NP, d] fp32, NP = 1 +
+ * ceil((max_seq_len - prefix_len) / partition_size), each section on a
+ * 256-byte boundary.  Other arguments and errors as for
+ * pa_decode_split_reduce.
+ */
+size_t pa_shared_prefix_workspace_bytes(int num_seqs, int num_q_heads, int head_dim,
+                                        int max_seq_len, int prefix_len, int partition_size);
+
+pa_status pa_decode_shared_prefix(void *out, const void *q, const void *k_cache,
+                                  const void *v_cache, const int32_t *block_tables,
+                                  int max_blocks_per_seq, const int32_t *seq_lens, int num_seqs,
+                                  int num_q_heads, int num_kv_heads, int head_dim, int block_size,
+                                  int num_blocks, float softmax_scale, pa_dtype q_dtype,
+                                  pa_dtype kv_dtype, int prefix_len, int partition_size,
+                                  int max_seq_len, void *workspace, size_t workspace_bytes,
+                                  int *dev_err, void *stream);
+
 /* Bytes of scratch built into the library for
  * pa_decode_split_reduce_static_scratch (32 MiB). */
 #define PA_STATIC_SCRATCH_BYTES (32u * 1024u * 1024u)

@@ -37,7 +37,7 @@ SYMBOLS = (
     "pa_status_string", "pa_version", "pa_slot_mapping", "pa_cache_write", "pa_decode",
     "pa_split_workspace_bytes", "pa_decode_split_reduce", "pa_decode_split_reduce_static_scratch",
     "pa_decode_append", "pa_copy_blocks", "pa_prefill", "pa_cache_write_per_channel",
-    "pa_decode_per_channel",
+    "pa_decode_per_channel", "pa_shared_prefix_workspace_bytes", "pa_decode_shared_prefix",
 )
 
 PA_STATIC_SCRATCH_BYTES = 32 * 1024 * 1024
@@ -92,6 +92,11 @@ _lib.pa_cache_write_per_channel.argtypes = [_P, _P, _P, _P, _P, _I, _I, _I, _I, 
 _lib.pa_decode_per_channel.restype = _I
 _lib.pa_decode_per_channel.argtypes = [_P, _P, _P, _P, _P, _I, _P, _I, _I, _I, _I, _I, _I, _F, _I,
                                        _I, _P, _P, _I, _I, _P, _S, _P, _P]
+_lib.pa_shared_prefix_workspace_bytes.restype = _S
+_lib.pa_shared_prefix_workspace_bytes.argtypes = [_I, _I, _I, _I, _I, _I]
+_lib.pa_decode_shared_prefix.restype = _I
+_lib.pa_decode_shared_prefix.argtypes = [_P, _P, _P, _P, _P, _I, _P, _I, _I, _I, _I, _I, _I, _F,
+                                         _I, _I, _I, _I, _I, _P, _S, _P, _P]
 _lib.pa_copy_blocks.restype = _I
 _lib.pa_copy_blocks.argtypes = [_P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P]
 
@@ -321,3 +326,27 @@ def pa_decode_per_channel(out, q, k_cache, v_cache, block_tables, seq_lens, soft
                                       int(max_seq_len), _ptr(workspace), ws_bytes, _ptr(dev_err),
                                       _stream(stream)),
            "pa_decode_per_channel")
+
+
+def pa_shared_prefix_workspace_bytes(num_seqs: int, num_q_heads: int, head_dim: int,
+                                     max_seq_len: int, prefix_len: int,
+                                     partition_size: int) -> int:
+    return int(_lib.pa_shared_prefix_workspace_bytes(num_seqs, num_q_heads, head_dim,
+                                                     max_seq_len, prefix_len, partition_size))
+
+
+def pa_decode_shared_prefix(out, q, k_cache, v_cache, block_tables, seq_lens,
+                            softmax_scale: float, prefix_len: int, partition_size: int,
+                            max_seq_len: int, workspace, dev_err=None, stream=None) -> None:
+    """Decode of sequences sharing their first ``prefix_len`` cached tokens
+    (the same blocks): the prefix is attended once for all of them."""
+    S, Hq, d = (int(x) for x in q.shape)
+    nb, Hk, B, _ = (int(x) for x in k_cache.shape)
+    ws_bytes = workspace.numel() * workspace.element_size()
+    _check(_lib.pa_decode_shared_prefix(_ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache),
+                                        _ptr(block_tables), int(block_tables.shape[1]),
+                                        _ptr(seq_lens), S, Hq, Hk, d, B, nb, float(softmax_scale),
+                                        dtype_code(q.dtype), dtype_code(k_cache.dtype),
+                                        int(prefix_len), int(partition_size), int(max_seq_len),
+                                        _ptr(workspace), ws_bytes, _ptr(dev_err), _stream(stream)),
+           "pa_decode_shared_prefix")

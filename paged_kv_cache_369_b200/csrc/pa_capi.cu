@@ -483,6 +483,111 @@ pa_status pa_decode_per_channel(void *out, const void *q, const void *k_cache, c
     return from_cuda(pa::launch_reduce(r, to_internal(q_dtype), head_dim, s));
 }
 
+size_t pa_shared_prefix_workspace_bytes(int num_seqs, int num_q_heads, int head_dim,
+                                        int max_seq_len, int prefix_len, int partition_size) {
+    if (num_seqs < 0 || num_q_heads <= 0 || head_dim <= 0 || max_seq_len < 0 || prefix_len < 0 ||
+        partition_size <= 0)
+        return 0;
+    const int tail = max_seq_len > prefix_len ? max_seq_len - prefix_len : 0;
+    const size_t np = 1 + (size_t)((tail + partition_size - 1) / partition_size);
+    const size_t rows = (size_t)num_seqs * (size_t)num_q_heads * np;
+    return align256(rows * sizeof(float)) + align256(rows * (size_t)head_dim * sizeof(float));
+}
+
+pa_status pa_decode_shared_prefix(void *out, const void *q, const void *k_cache,
+                                  const void *v_cache, const int32_t *block_tables,
+                                  int max_blocks_per_seq, const int32_t *seq_lens, int num_seqs,
+                                  int num_q_heads, int num_kv_heads, int head_dim, int block_size,
+                                  int num_blocks, float softmax_scale, pa_dtype q_dtype,
+                                  pa_dtype kv_dtype, int prefix_len, int partition_size,
+                                  int max_seq_len, void *workspace, size_t workspace_bytes,
+                                  int *dev_err, void *stream) {
+    const DecodeArgs a = {out, q, k_cache, v_cache, block_tables, max_blocks_per_seq, seq_lens,
+                          num_seqs, num_q_heads, num_kv_heads, head_dim, block_size, num_blocks,
+                          softmax_scale, q_dtype, kv_dtype, 1.0f, 1.0f};
+    pa_status st = check_decode(a);
+    if (st != PA_OK) return st;
+    if (kv_dtype != q_dtype) return PA_ERR_UNSUPPORTED;  // the prefix pass reads 16-bit caches
+    const int g = num_q_heads / num_kv_heads;
+    if (g > 128) return PA_ERR_UNSUPPORTED;
+    if (!(softmax_scale > 0.f)) return PA_ERR_INVALID_ARG;
+    if (partition_size <= 0 || partition_size % pa::kBlockSize != 0 || max_seq_len < 0)
+        return PA_ERR_INVALID_ARG;
+    if (prefix_len <= 0 || prefix_len % block_size != 0 || prefix_len > max_seq_len ||
+        prefix_len > max_blocks_per_seq * block_size)
+        return PA_ERR_INVALID_ARG;
+    if (num_seqs == 0) return PA_OK;
+    if (num_kv_heads > 65535) return PA_ERR_UNSUPPORTED;
+    const int64_t pool_rows = (int64_t)num_blocks * num_kv_heads * block_size;
+    if (pool_rows + block_size >= (int64_t(1) << 31)) return PA_ERR_UNSUPPORTED;
+    const size_t need = pa_shared_prefix_workspace_bytes(num_seqs, num_q_heads, head_dim,
+                                                         max_seq_len, prefix_len, partition_size);
+    if (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+        return PA_ERR_INVALID_ARG;
+    if (!pa::prefill_supported()) return PA_ERR_CUDA;  // no tensor-map encoder in the driver
+    const int np_tail = (max_seq_len - prefix_len + partition_size - 1) / partition_size;
+    const int np = 1 + np_tail;
+    if ((int64_t)num_seqs * (np_tail > 0 ? np_tail : 1) > 0x7FFFFFFF) return PA_ERR_UNSUPPORTED;
+    const size_t rows = (size_t)num_seqs * num_q_heads * np;
+    float *ws_lse = static_cast<float *>(workspace);
+    float *ws_o = reinterpret_cast<float *>(static_cast<uint8_t *>(workspace) + align256(rows * sizeof(float)));
+    const cudaStream_t s = static_cast<cudaStream_t>(stream);
+
+    // 1. the prefix, once for every sequence: workspace slot 0
+    pa::PrefillParams f = {};
+    f.q = q;
+    f.k_cache = k_cache;
+    f.v_cache = v_cache;
+    f.block_tables = block_tables;  // row 0 names the shared blocks
+    f.err = dev_err;
+    f.max_blocks_per_seq = max_blocks_per_seq;
+    f.num_seqs = 1;
+    f.num_tokens = num_seqs;        // one query row per decoding sequence
+    f.max_query_len = num_seqs;
+    f.num_q_heads = num_q_heads;
+    f.num_kv_heads = num_kv_heads;
+    f.num_blocks = num_blocks;
+    f.block_size = block_size;
+    f.tile_shift = block_size == 32 ? 1 : 0;
+    f.group = g;
+    f.tok_per_tile = 128 / g;
+    f.oob_row = (int)pool_rows;
+    f.qk_scale_log2 = (float)((double)softmax_scale * 1.4426950408889634074);
+    f.shared_len = prefix_len;
+    f.ws_o = ws_o;
+    f.ws_lse = ws_lse;
+    f.ws_np = np;
+    if (pa::launch_prefill(f, to_internal(q_dtype), head_dim, s) != cudaSuccess) return PA_ERR_CUDA;
+
+    // 2. every sequence's tail, split into partitions: slots 1 .. np - 1
+    if (np_tail > 0) {
+        pa::DecodeParams p = make_decode_params(a, dev_err);
+        p.ws_lse = ws_lse;
+        p.ws_o = ws_o;
+        p.partition_blocks = partition_size / pa::kBlockSize;
+        p.num_partitions = np_tail;
+        p.split = 1;
+        p.tile_begin = prefix_len / pa::kBlockSize;
+        p.ws_offset = 1;
+        p.ws_np = np;
+        if (launch_any_decode(p, q_dtype, kv_dtype, head_dim, s) != cudaSuccess) return PA_ERR_CUDA;
+    }
+
+    // 3. merge the prefix partial with the tail partitions
+    pa::ReduceParams r = {};
+    r.out = out;
+    r.ws_lse = ws_lse;
+    r.ws_o = ws_o;
+    r.seq_lens = seq_lens;
+    r.num_seqs = num_seqs;
+    r.num_q_heads = num_q_heads;
+    r.num_partitions = np;
+    r.partition_size = partition_size;
+    r.extra = 1;
+    r.token_begin = prefix_len;
+    return from_cuda(pa::launch_reduce(r, to_internal(q_dtype), head_dim, s));
+}
+
 size_t pa_split_workspace_bytes(int num_seqs, int num_q_heads, int head_dim, int max_seq_len,
                                 int partition_size) {
     if (num_seqs < 0 || num_q_heads <= 0 || head_dim <= 0 || max_seq_len < 0 ||

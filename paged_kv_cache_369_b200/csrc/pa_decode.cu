@@ -133,14 +133,18 @@ __global__ void __launch_bounds__(kDecodeWarps * 32)
         L = L < 0 ? 0 : max_tokens;
     }
     if (p.split) {
-        const int cap = NP * p.partition_blocks * kBlockSize;
+        const int cap = (p.tile_begin + NP * p.partition_blocks) * kBlockSize;
         if (L > cap) {
             if (threadIdx.x == 0 && part == 0) flag_error(p.err, kErrBounds);
             L = cap;
         }
     }
     const int nblk_seq = (L + kBlockSize - 1) / kBlockSize;
-    const int blk_begin = part * p.partition_blocks;
+    if (L < p.tile_begin * kBlockSize) {  // shared-prefix decode: shorter than the prefix
+        if (threadIdx.x == 0 && part == 0) flag_error(p.err, kErrBounds);
+        L = p.tile_begin * kBlockSize;
+    }
+    const int blk_begin = p.tile_begin + part * p.partition_blocks;
     int blk_end = blk_begin + p.partition_blocks;
     if (blk_end > nblk_seq) blk_end = nblk_seq;
     if (p.split && blk_begin >= blk_end) return;  // empty partition: nothing to write
@@ -396,9 +400,10 @@ __global__ void __launch_bounds__(kDecodeWarps * 32)
         if (!p.split) {
             reinterpret_cast<uint16_t *>(p.out)[row * D + d] = from_float(QT{}, o);
         } else {
-            p.ws_o[(row * NP + part) * D + d] = o;
+            const int ws_np = p.ws_np > 0 ? p.ws_np : NP, slot = p.ws_offset + part;
+            p.ws_o[(row * ws_np + slot) * D + d] = o;
             if (d == 0)
-                p.ws_lse[row * NP + part] =
+                p.ws_lse[row * ws_np + slot] =
                     Ls > 0.f ? (M + log2f(Ls)) * 0.69314718055994530942f : -CUDART_INF_F;
         }
     }
@@ -419,10 +424,11 @@ __global__ void __launch_bounds__(D) reduce_kernel(const ReduceParams p) {
     const int64_t row = blockIdx.x;
     const int s = (int)(row / p.num_q_heads);
     const int NP = p.num_partitions;
-    int L = p.seq_lens[s];
-    const int cap = NP * p.partition_size;
+    // tokens past token_begin, split into partitions after `extra` leading slots
+    int L = p.seq_lens[s] - p.token_begin;
+    const int cap = (NP - p.extra) * p.partition_size;
     L = L < 0 ? 0 : (L > cap ? cap : L);
-    const int np = (L + p.partition_size - 1) / p.partition_size;
+    const int np = p.extra + (L + p.partition_size - 1) / p.partition_size;
     const float *lse = p.ws_lse + row * NP;
     const float *o = p.ws_o + row * NP * D;
     const int d = threadIdx.x, lane = d & 31, wid = d >> 5;

@@ -228,7 +228,7 @@ __global__ void __launch_bounds__(NWARPS * 32, 12 / NWARPS)
         L = L < 0 ? 0 : max_tokens;
     }
     if (p.split) {
-        const int cap = NP * p.partition_blocks * kBlockSize;
+        const int cap = (p.tile_begin + NP * p.partition_blocks) * kBlockSize;
         if (L > cap) {
             if (threadIdx.x == 0 && part == 0) flag_error(p.err, kErrBounds);
             L = cap;
@@ -236,7 +236,11 @@ __global__ void __launch_bounds__(NWARPS * 32, 12 / NWARPS)
     }
     const bool len_ok = L == p.seq_lens[s];  // not clamped: the new token's slot is known
     const int nblk_seq = (L + kBlockSize - 1) / kBlockSize;
-    const int blk_begin = part * p.partition_blocks;
+    if (L < p.tile_begin * kBlockSize) {  // shared-prefix decode: shorter than the prefix
+        if (threadIdx.x == 0 && part == 0) flag_error(p.err, kErrBounds);
+        L = p.tile_begin * kBlockSize;
+    }
+    const int blk_begin = p.tile_begin + part * p.partition_blocks;
     int blk_end = blk_begin + p.partition_blocks;
     if (blk_end > nblk_seq) blk_end = nblk_seq;
     if (p.split && blk_begin >= blk_end) return;
@@ -650,9 +654,10 @@ __global__ void __launch_bounds__(NWARPS * 32, 12 / NWARPS)
         if (!p.split) {
             reinterpret_cast<uint16_t *>(p.out)[row * D + d] = from_float(QT{}, ov);
         } else {
-            p.ws_o[(row * NP + part) * D + d] = ov;
+            const int ws_np = p.ws_np > 0 ? p.ws_np : NP, slot = p.ws_offset + part;
+            p.ws_o[(row * ws_np + slot) * D + d] = ov;
             if (d == 0)
-                p.ws_lse[row * NP + part] =
+                p.ws_lse[row * ws_np + slot] =
                     Ls > 0.f ? (M + log2f(Ls)) * 0.69314718055994530942f : -CUDART_INF_F;
         }
     }

@@ -77,6 +77,12 @@ struct DecodeParams {
     int partition_blocks;       // 16-token tiles per partition
     int num_partitions;         // NP (1 in single-pass mode)
     int split;                  // 1: write partials to the workspace
+    // shared-prefix decode: the tail of every sequence starts at tile
+    // tile_begin (0 otherwise); partition p is written to workspace slot
+    // ws_offset + p of ws_np slots per row (ws_np 0: num_partitions)
+    int tile_begin;
+    int ws_offset;
+    int ws_np;
     float qk_scale_log2;        // softmax_scale * k_scale * log2(e)
     float v_scale;              // applied to the output (1 for 16-bit caches)
     // per-channel scales of an 8-bit cache, [Hk, D] fp32, or null: K's are
@@ -144,6 +150,14 @@ struct PrefillParams {  // chunked prefill (pa_prefill)
     int tok_per_tile;           // floor(128 / group) chunk tokens per query tile
     int oob_row;                // a pool row index past the end (zero-filled loads)
     float qk_scale_log2;        // softmax_scale * log2(e)
+    // shared-prefix mode (shared_len > 0): one "sequence" = the first
+    // shared_len tokens of block table row 0; the T query rows (one per
+    // decoding sequence) all see every one of them (no causal mask), and each
+    // row's partial (lse, o / l) goes to workspace slot 0 of ws_np per row
+    int shared_len;
+    float *ws_o;
+    float *ws_lse;
+    int ws_np;
 };
 
 struct ReduceParams {
@@ -153,8 +167,12 @@ struct ReduceParams {
     const int32_t *seq_lens;
     int num_seqs;
     int num_q_heads;
-    int num_partitions;
+    int num_partitions;         // workspace slots per row
     int partition_size;
+    // shared-prefix decode: `extra` leading slots hold the prefix partials and
+    // the partitions cover tokens from token_begin (0 / 0 otherwise)
+    int extra;
+    int token_begin;
 };
 
 // Launchers: return cudaSuccess or the launch error.

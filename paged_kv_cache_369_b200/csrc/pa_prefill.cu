@@ -255,10 +255,11 @@ __global__ void __launch_bounds__(320, 1)
     const int g = p.group, tpt = p.tok_per_tile;
 
     // ---- this CTA's rows and keys (uniform over the CTA) ---------------------
-    const int L = p.seq_lens[s];
-    const int q0 = p.query_start[s];
-    const int n = p.query_start[s + 1] - q0;
-    if (L < 0 || L > p.max_blocks_per_seq * p.block_size || n < 0 || n > L || q0 < 0 ||
+    const bool causal = p.shared_len == 0;
+    const int L = causal ? p.seq_lens[s] : p.shared_len;
+    const int q0 = causal ? p.query_start[s] : 0;
+    const int n = causal ? p.query_start[s + 1] - q0 : p.num_tokens;
+    if (L < 0 || L > p.max_blocks_per_seq * p.block_size || n < 0 || (causal && n > L) || q0 < 0 ||
         q0 + n > p.num_tokens || n > p.max_query_len) {
         if (threadIdx.x == 0 && cta_tile == 0 && kvh == 0) flag_error(p.err, kErrBounds);
         return;
@@ -267,7 +268,9 @@ __global__ void __launch_bounds__(320, 1)
     if (tok0 >= n) return;
     const int ntok = min(2 * tpt, n - tok0);
     const int ctx = L - n;
-    const int nt = (ctx + tok0 + ntok - 1) / C::BN + 1;  // key tiles up to the last row's position
+    // key tiles up to the last row's position (all of the prefix without the mask)
+    const int nt = causal ? (ctx + tok0 + ntok - 1) / C::BN + 1 : (L + C::BN - 1) / C::BN;
+    if (nt <= 0) return;  // an empty prefix
     const int nblk_seq = (L + kBlockSize - 1) / kBlockSize;  // 16-token tiles
     const int tile_mask = (1 << p.tile_shift) - 1;
 
@@ -454,7 +457,7 @@ __global__ void __launch_bounds__(320, 1)
         const int r = (warp & 3) * 32 + lane;     // row = TMEM lane
         const int rtok = t * tpt + r / g;         // token within the CTA's range
         const bool row_ok = r < tpt * g && rtok < ntok;
-        const int pos = ctx + tok0 + rtok;
+        const int pos = causal ? ctx + tok0 + rtok : L - 1;
         const uint32_t lane_bits = (uint32_t)((warp & 3) * 32) << 16;
         const uint32_t ocol = tmem + lane_bits + C::COL_O + 128u * t;
         const float sl2 = p.qk_scale_log2;  // > 0
@@ -537,23 +540,43 @@ __global__ void __launch_bounds__(320, 1)
                                                      abort_flag, p.err));
         if (ok) {
             // ---- epilogue: out = O / l, rounded once to the q dtype ----------------
+            // (shared-prefix mode: the partial o / l and its log-sum-exp, fp32)
             tc::fence_after();
             const float inv = l > 0.f ? 1.f / l : 0.f;
             const int64_t row = ((int64_t)(q0 + tok0 + rtok) * p.num_q_heads + (int64_t)kvh * g + r % g);
             uint4 *dst = reinterpret_cast<uint4 *>(static_cast<uint16_t *>(p.out) + row * D);
+            if (!causal) {
+                float4 *wo = reinterpret_cast<float4 *>(p.ws_o + row * p.ws_np * D);
+                if (row_ok)
+                    p.ws_lse[row * p.ws_np] =
+                        l > 0.f ? (m_ref + log2f(l)) * 0.69314718055994530942f : -CUDART_INF_F;
 #pragma unroll
-            for (int c = 0; c < D; c += 32) {
-                uint32_t o[32];
-                tc::ld32(ocol + c, o);
-                tc::wait_ld<32>(o);
-                uint32_t w[16];
+                for (int c = 0; c < D; c += 32) {
+                    uint32_t o[32];
+                    tc::ld32(ocol + c, o);
+                    tc::wait_ld<32>(o);
+                    if (row_ok) {
 #pragma unroll
-                for (int i = 0; i < 16; ++i)
-                    w[i] = tc::pack2(__uint_as_float(o[2 * i]) * inv, __uint_as_float(o[2 * i + 1]) * inv, T{});
-                if (row_ok) {
+                        for (int v = 0; v < 8; ++v)
+                            wo[c / 4 + v] = make_float4(__uint_as_float(o[4 * v]) * inv, __uint_as_float(o[4 * v + 1]) * inv,
+                                                        __uint_as_float(o[4 * v + 2]) * inv, __uint_as_float(o[4 * v + 3]) * inv);
+                    }
+                }
+            } else {
 #pragma unroll
-                    for (int v = 0; v < 4; ++v)
-                        dst[c / 8 + v] = make_uint4(w[4 * v], w[4 * v + 1], w[4 * v + 2], w[4 * v + 3]);
+                for (int c = 0; c < D; c += 32) {
+                    uint32_t o[32];
+                    tc::ld32(ocol + c, o);
+                    tc::wait_ld<32>(o);
+                    uint32_t w[16];
+#pragma unroll
+                    for (int i = 0; i < 16; ++i)
+                        w[i] = tc::pack2(__uint_as_float(o[2 * i]) * inv, __uint_as_float(o[2 * i + 1]) * inv, T{});
+                    if (row_ok) {
+#pragma unroll
+                        for (int v = 0; v < 4; ++v)
+                            dst[c / 8 + v] = make_uint4(w[4 * v], w[4 * v + 1], w[4 * v + 2], w[4 * v + 3]);
+                    }
                 }
             }
         }

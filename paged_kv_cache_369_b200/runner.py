@@ -20,8 +20,9 @@ import numpy as np
 import torch
 
 from . import (pa_cache_write, pa_cache_write_per_channel, pa_decode, pa_decode_append,
-               pa_decode_per_channel, pa_decode_split_reduce, pa_prefill, pa_slot_mapping,
-               pa_split_workspace_bytes, pool_torch_dtype)
+               pa_decode_per_channel, pa_decode_shared_prefix, pa_decode_split_reduce, pa_prefill,
+               pa_shared_prefix_workspace_bytes, pa_slot_mapping, pa_split_workspace_bytes,
+               pool_torch_dtype)
 
 _TORCH_ACT = {"f16": torch.float16, "bf16": torch.bfloat16}
 _UPLOAD_CHUNK_TOKENS = 1 << 16
@@ -37,8 +38,13 @@ class PagedDecode:
 
     def __init__(self, w, device: str = "cuda", mode: str = "split", partition_size: int = 512,
                  prefill: bool = True, stream: Optional[torch.cuda.Stream] = None):
-        if mode not in ("split", "single", "fused", "fused_single"):
+        if mode not in ("split", "single", "fused", "fused_single", "cascade"):
             raise ValueError(mode)
+        # cascade: sequences sharing a prefix of whole blocks (the workload's
+        # shared_prefix_blocks) attend to it once through pa_decode_shared_prefix
+        self.prefix_len = getattr(w, "shared_prefix_blocks", 0) * w.block_size
+        if mode == "cascade" and self.prefix_len <= 0:
+            raise ValueError("cascade mode needs a shared prefix")
         self.per_channel = getattr(w, "k_chan", None) is not None
         if self.per_channel and mode.startswith("fused"):
             raise ValueError("per-channel scales: the cache write is its own call (split / single)")
@@ -71,6 +77,9 @@ class PagedDecode:
             self.v_chan = torch.from_numpy(np.ascontiguousarray(w.v_chan, np.float32)).to(dev)
         self.max_seq_len = int(w.seq_lens.max()) if S else 0
         nbytes = pa_split_workspace_bytes(S, Hq, d, self.max_seq_len, partition_size)
+        if mode == "cascade":
+            nbytes = pa_shared_prefix_workspace_bytes(S, Hq, d, self.max_seq_len, self.prefix_len,
+                                                      partition_size)
         self.workspace = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=dev)
         if prefill:
             self.prefill()
@@ -120,6 +129,12 @@ class PagedDecode:
                                   self.max_seq_len, self.workspace if P else None, self.dev_err,
                                   self.stream)
             return
+        if self.mode == "cascade":
+            pa_decode_shared_prefix(self.out, self.q, self.k_cache, self.v_cache,
+                                    self.block_tables, self.seq_lens, w.softmax_scale,
+                                    self.prefix_len, self.partition_size, self.max_seq_len,
+                                    self.workspace, self.dev_err, self.stream)
+            return
         if self.mode == "single":
             pa_decode(self.out, self.q, self.k_cache, self.v_cache, self.block_tables,
                       self.seq_lens, w.softmax_scale, w.k_scale, w.v_scale, self.dev_err,
@@ -151,7 +166,7 @@ class PagedDecode:
     def launches_per_step(self) -> int:
         """Kernel launches of one step (the tensor-core route; the CUDA-core
         route of a fused step adds one append launch)."""
-        return {"single": 3, "split": 4, "fused": 2, "fused_single": 1}[self.mode]
+        return {"single": 3, "split": 4, "fused": 2, "fused_single": 1, "cascade": 5}[self.mode]
 
     def error(self) -> int:
         return int(self.dev_err.item())
@@ -240,3 +255,15 @@ class PagedPrefill:
 
     def error(self) -> int:
         return int(self.dev_err.item())
+
+
+def algorithmic_cascade_bytes(w) -> int:
+    """Bytes the shared-prefix decode must move: the shared prefix's K/V once,
+    every sequence's tail K/V once, q read, the output written, tables and
+    lengths read."""
+    S, Hq, Hk, d = w.num_seqs, w.num_q_heads, w.num_kv_heads, w.head_dim
+    prefix = w.shared_prefix_blocks * w.block_size
+    per_tok = Hk * 2 * d * w.kv_elem_bytes()
+    tails = int((w.seq_lens.astype(np.int64) - prefix).clip(min=0).sum())
+    return (prefix + tails) * per_tok + 2 * S * Hq * d * 2 + int(sum(
+        math.ceil(int(L) / w.block_size) for L in w.seq_lens)) * 4 + S * 4

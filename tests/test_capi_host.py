@@ -225,3 +225,24 @@ def test_per_channel_checks(pa):
     assert dec(P=24) == 1
     assert dec(P=512) == 1                   # split needs a workspace
     assert dec(S=0) == 0                     # empty batch
+
+
+def test_shared_prefix_checks(pa):
+    L = pa.lib()
+    need = pa.pa_shared_prefix_workspace_bytes(2, 8, 128, 1000, 512, 256)
+    # 1 prefix slot + ceil(488 / 256) = 2 tail partitions
+    assert need == 256 + (2 * 8 * 3 * 128 * 4 + 255) // 256 * 256
+    assert pa.pa_shared_prefix_workspace_bytes(2, 8, 128, 1000, 512, 0) == 0
+
+    def call(prefix=512, P=256, kv=pa.PA_BF16, ws=A, wsb=need, maxlen=1000, B=16, scale=0.1):
+        return L.pa_decode_shared_prefix(A, A, A, A, A, 80, A, 2, 8, 2, 128, B, 10, scale,
+                                         pa.PA_BF16, kv, prefix, P, maxlen, ws, wsb, None, None)
+
+    assert call(kv=pa.PA_FP8_E4M3) == 2     # 16-bit caches only
+    assert call(prefix=0) == 1
+    assert call(prefix=24) == 1              # not a multiple of the block size
+    assert call(prefix=1200) == 1            # longer than max_seq_len
+    assert call(P=24) == 1
+    assert call(wsb=need - 1) == 1
+    assert call(ws=A + 64) == 1
+    assert call(scale=-1.0) == 1

@@ -185,6 +185,68 @@ def test_block_size_32_parity(case, mode, P, kernel_choice):
                  f"block 32 case {case} {mode} P={P} kernel={kernel_choice}")
 
 
+CASCADE = [
+    # (Hq, Hk, d, act, lens, shared prefix tokens, block size)
+    (8, 8, 128, "f16", [1040, 1030, 1100], 1024, 16),
+    (32, 8, 128, "bf16", [100, 65, 66, 700], 64, 16),
+    (16, 2, 64, "f16", [33, 40, 300], 32, 16),
+    (4, 4, 128, "bf16", [17, 18, 200], 16, 16),
+    (32, 8, 128, "f16", [97, 300, 65], 64, 32),
+    (24, 8, 64, "bf16", [130, 129], 128, 16),       # GQA 3
+]
+
+
+@pytest.mark.parametrize("P", [16, 512])
+@pytest.mark.parametrize("case", range(len(CASCADE)))
+def test_shared_prefix_decode_parity(case, P, kernel_choice):
+    """pa_decode_shared_prefix: the prefix attended once for all sequences
+    (tensor-core pass), tails split, merged -- against the oracle's decode."""
+    pa, PagedDecode = _pa()
+    Hq, Hk, d, act, lens, prefix, B = CASCADE[case]
+    w = workload.build(f"casc{case}", 5000 + case, lens, Hq, Hk, d, act, act,
+                       shared_prefix_tokens=prefix, block_size=B, extra_table_cols=1)
+    dec = PagedDecode(w, mode="cascade", partition_size=P)
+    dec.step()
+    torch.cuda.synchronize()
+    assert dec.error() == 0
+    kc, vc = oracle.caches_for(w)
+    check_pools(dec, kc, vc)
+    assert_close(_to_f64(dec.out), oracle.decode_for(w, kc, vc),
+                 f"shared prefix case {case} P={P} kernel={kernel_choice}")
+
+
+def test_shared_prefix_decode_full_size():
+    """The continuous-batching workload (256 sequences sharing a 1024-token
+    prefix): 64 sampled rows against the oracle, every output inside the
+    range of its V rows."""
+    pa, PagedDecode = _pa()
+    w, kc, vc = _full(5)
+    dec = PagedDecode(w, mode="cascade", partition_size=512)
+    dec.step()
+    torch.cuda.synchronize()
+    assert dec.error() == 0
+    check_pools(dec, kc, vc)
+    out = _to_f64(dec.out)
+    pairs = sample_pairs(w, 64, seed=55)
+    ref = oracle.decode_for(w, kc, vc, pairs)
+    assert_close(out[pairs[:, 0], pairs[:, 1]], ref, "config 5 shared prefix")
+    _check_convex_hull(w, dec, out)
+
+
+def test_shared_prefix_shorter_sequence_is_reported():
+    pa, PagedDecode = _pa()
+    w = workload.build("cshort", 5100, [80, 90], 8, 2, 64, "f16", "f16", shared_prefix_tokens=64)
+    dec = PagedDecode(w, mode="cascade", partition_size=64)
+    dec.step()
+    torch.cuda.synchronize()
+    assert dec.error() == 0
+    dec.seq_lens[1] = 40  # shorter than the prefix
+    dec.attend()
+    torch.cuda.synchronize()
+    assert dec.error() == pa.PA_ERR_DEVICE_BOUNDS
+    assert torch.isfinite(dec.out.float()).all()
+
+
 def test_split_partials_match_oracle(kernel_choice):
     pa, PagedDecode = _pa()
     w = workload.build("partials", 77, [1, 16, 17, 100, 513, 1100], 16, 4, 128, "bf16", "bf16")
