@@ -602,7 +602,9 @@ def main(argv=None):
     ap.add_argument("--mode", choices=("fused", "fused_single", "split", "single", "cascade"),
                     default="fused",
                     help="cascade: the shared-prefix decode (config 5's common prefix attended once)")
-    ap.add_argument("--partition", type=int, default=512)
+    ap.add_argument("--partition", type=int, default=None,
+                    help="split-KV partition in tokens (default: 512 for config 4, as it "
+                         "prescribes, else 1024)")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--op", choices=("decode", "copy_blocks", "prefill"), default="decode",
@@ -619,6 +621,8 @@ def main(argv=None):
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
+    if args.partition is None:  # as runner.default_partition_size: 512 where prescribed
+        args.partition = 512 if args.config == 4 else 1024
     if args.channel_scales:
         if args.kv is None and args.config != 4:
             ap.error("--channel-scales needs an 8-bit cache (--kv or config 4)")
