@@ -378,7 +378,7 @@ def run_prefill(args):
     world, rank, local = dist_env()
     torch.cuda.set_device(local)
     device = torch.device("cuda", local)
-    w = workload.prefill_config(args.pconfig)
+    w = workload.prefill_config(args.pconfig, kv_dtype=args.kv)
     stream = torch.cuda.Stream(device)
     with torch.cuda.stream(stream):
         pre = PagedPrefill(w, device=str(device), stream=stream)
@@ -411,7 +411,8 @@ def run_prefill(args):
         "data": "synthetic: seeded N(0,1) q/K/V, shuffled block pool",
         "config": {"workload": w.name, "num_seqs": w.num_seqs, "chunk": int(w.max_query_len),
                    "num_q_heads": w.num_q_heads, "num_kv_heads": w.num_kv_heads,
-                   "head_dim": w.head_dim, "context_mean": float((w.seq_lens - w.chunk_lens).mean()),
+                   "head_dim": w.head_dim, "kv_dtype": w.kv_dtype,
+                   "context_mean": float((w.seq_lens - w.chunk_lens).mean()),
                    "seed": w.seed, "l2": "K/V re-read across query tiles is meant to hit L2; no flush"},
         "attention_us": attn_ms * 1e3, "cache_write_us": (step_ms - attn_ms) * 1e3,
         "tokens_per_s": w.num_tokens / (step_ms * 1e-3),

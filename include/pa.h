@@ -257,8 +257,12 @@ pa_status pa_decode_split_reduce(void *out, const void *q, const void *k_cache,
  * int32) is non-decreasing with query_start[num_seqs] <= num_tokens; rows no
  * sequence covers are not written.  max_query_len bounds every n.
  *
- * Supported: block_size 16 or 32, head_dim 64 or 128, q_dtype (= out dtype =
- * kv_dtype) PA_F16 or PA_BF16 (8-bit caches return PA_ERR_UNSUPPORTED), GQA
+ * Supported: block_size 16 or 32, head_dim 64 or 128, q_dtype (= out dtype)
+ * PA_F16 or PA_BF16, kv_dtype = q_dtype or, with head_dim 128, an 8-bit
+ * format read as code * k_scale / code * v_scale (per-tensor scales, finite
+ * and > 0; ignored for 16-bit caches; the codes are widened to f16 exactly
+ * in shared memory and the MMAs then run in f16, q scaled by a power of two
+ * into f16 range), GQA
  * groups up to 128, num_seqs and num_kv_heads up to 65535, softmax_scale
  * finite and > 0 (else PA_ERR_INVALID_ARG).  Arithmetic is
  * fp32 with the probabilities kept to ~16 bits (bf16 hi + lo) or f16; out is
@@ -272,7 +276,7 @@ pa_status pa_prefill(void *out, const void *q, const void *k_cache, const void *
                      const int32_t *query_start, int num_seqs, int num_tokens, int max_query_len,
                      int num_q_heads, int num_kv_heads, int head_dim, int block_size,
                      int num_blocks, float softmax_scale, pa_dtype q_dtype, pa_dtype kv_dtype,
-                     int *dev_err, void *stream);
+                     float k_scale, float v_scale, int *dev_err, void *stream);
 
 /*
  * pa_copy_blocks -- copy whole KV blocks inside the pools (copy-on-write).
@@ -351,8 +355,9 @@ pa_status pa_decode_per_channel(void *out, const void *q, const void *k_cache, c
  * block_tables are the same blocks (row 0 is read for them; the caller's
  * allocator guarantees the sharing), prefix_len is a positive multiple of
  * block_size, every seq_lens[s] >= prefix_len (a shorter one flags
- * PA_ERR_DEVICE_BOUNDS), kv_dtype = q_dtype (16-bit caches), softmax_scale > 0,
- * GQA groups up to 128.  Three launches on `stream`:
+ * PA_ERR_DEVICE_BOUNDS), kv_dtype = q_dtype or an 8-bit format with
+ * head_dim 128 (per-tensor k_scale / v_scale as for pa_decode),
+ * softmax_scale > 0, GQA groups up to 128.  Three launches on `stream`:
  *   1. the prefix: for each KV head, the queries of all sequences against the
  *      prefix keys as one dense tensor-core pass (the prefix K/V is read once,
  *      not once per sequence), giving each (sequence, head) a partial
@@ -375,9 +380,9 @@ pa_status pa_decode_shared_prefix(void *out, const void *q, const void *k_cache,
                                   int max_blocks_per_seq, const int32_t *seq_lens, int num_seqs,
                                   int num_q_heads, int num_kv_heads, int head_dim, int block_size,
                                   int num_blocks, float softmax_scale, pa_dtype q_dtype,
-                                  pa_dtype kv_dtype, int prefix_len, int partition_size,
-                                  int max_seq_len, void *workspace, size_t workspace_bytes,
-                                  int *dev_err, void *stream);
+                                  pa_dtype kv_dtype, float k_scale, float v_scale, int prefix_len,
+                                  int partition_size, int max_seq_len, void *workspace,
+                                  size_t workspace_bytes, int *dev_err, void *stream);
 
 /* Bytes of scratch built into the library for
  * pa_decode_split_reduce_static_scratch (32 MiB). */

@@ -85,7 +85,7 @@ _lib.pa_decode_split_reduce_static_scratch.argtypes = [_P, _P, _P, _P, _P, _I, _
                                                        _I, _I, _F, _I, _I, _F, _F, _I, _I, _P, _P]
 _lib.pa_prefill.restype = _I
 _lib.pa_prefill.argtypes = [_P, _P, _P, _P, _P, _I, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _F,
-                            _I, _I, _P, _P]
+                            _I, _I, _F, _F, _P, _P]
 _lib.pa_cache_write_per_channel.restype = _I
 _lib.pa_cache_write_per_channel.argtypes = [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _P, _P,
                                             _P, _P]
@@ -96,7 +96,7 @@ _lib.pa_shared_prefix_workspace_bytes.restype = _S
 _lib.pa_shared_prefix_workspace_bytes.argtypes = [_I, _I, _I, _I, _I, _I]
 _lib.pa_decode_shared_prefix.restype = _I
 _lib.pa_decode_shared_prefix.argtypes = [_P, _P, _P, _P, _P, _I, _P, _I, _I, _I, _I, _I, _I, _F,
-                                         _I, _I, _I, _I, _I, _P, _S, _P, _P]
+                                         _I, _I, _F, _F, _I, _I, _I, _P, _S, _P, _P]
 _lib.pa_copy_blocks.restype = _I
 _lib.pa_copy_blocks.argtypes = [_P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P]
 
@@ -282,7 +282,8 @@ def pa_copy_blocks(k_cache, v_cache, block_pairs, dev_err=None, stream=None) -> 
 
 
 def pa_prefill(out, q, k_cache, v_cache, block_tables, seq_lens, query_start, max_query_len: int,
-               softmax_scale: float, dev_err=None, stream=None) -> None:
+               softmax_scale: float, dev_err=None, stream=None, k_scale: float = 1.0,
+               v_scale: float = 1.0) -> None:
     """Chunked-prefill attention: the rows query_start[s] .. query_start[s+1]-1
     of ``q`` ([T, Hq, d]) are the last tokens of sequence s's seq_lens[s] and
     attend causally over its cache."""
@@ -292,8 +293,8 @@ def pa_prefill(out, q, k_cache, v_cache, block_tables, seq_lens, query_start, ma
     _check(_lib.pa_prefill(_ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables),
                            int(block_tables.shape[1]), _ptr(seq_lens), _ptr(query_start), S, T,
                            int(max_query_len), Hq, Hk, d, B, nb, float(softmax_scale),
-                           dtype_code(q.dtype), dtype_code(k_cache.dtype), _ptr(dev_err),
-                           _stream(stream)),
+                           dtype_code(q.dtype), dtype_code(k_cache.dtype), float(k_scale),
+                           float(v_scale), _ptr(dev_err), _stream(stream)),
            "pa_prefill")
 
 
@@ -337,7 +338,8 @@ def pa_shared_prefix_workspace_bytes(num_seqs: int, num_q_heads: int, head_dim: 
 
 def pa_decode_shared_prefix(out, q, k_cache, v_cache, block_tables, seq_lens,
                             softmax_scale: float, prefix_len: int, partition_size: int,
-                            max_seq_len: int, workspace, dev_err=None, stream=None) -> None:
+                            max_seq_len: int, workspace, dev_err=None, stream=None,
+                            k_scale: float = 1.0, v_scale: float = 1.0) -> None:
     """Decode of sequences sharing their first ``prefix_len`` cached tokens
     (the same blocks): the prefix is attended once for all of them."""
     S, Hq, d = (int(x) for x in q.shape)
@@ -347,6 +349,7 @@ def pa_decode_shared_prefix(out, q, k_cache, v_cache, block_tables, seq_lens,
                                         _ptr(block_tables), int(block_tables.shape[1]),
                                         _ptr(seq_lens), S, Hq, Hk, d, B, nb, float(softmax_scale),
                                         dtype_code(q.dtype), dtype_code(k_cache.dtype),
-                                        int(prefix_len), int(partition_size), int(max_seq_len),
+                                        float(k_scale), float(v_scale), int(prefix_len),
+                                        int(partition_size), int(max_seq_len),
                                         _ptr(workspace), ws_bytes, _ptr(dev_err), _stream(stream)),
            "pa_decode_shared_prefix")

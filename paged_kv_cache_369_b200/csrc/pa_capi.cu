@@ -321,14 +321,18 @@ pa_status pa_prefill(void *out, const void *q, const void *k_cache, const void *
                      const int32_t *query_start, int num_seqs, int num_tokens, int max_query_len,
                      int num_q_heads, int num_kv_heads, int head_dim, int block_size,
                      int num_blocks, float softmax_scale, pa_dtype q_dtype, pa_dtype kv_dtype,
-                     int *dev_err, void *stream) {
+                     float k_scale, float v_scale, int *dev_err, void *stream) {
     if (num_seqs < 0 || num_tokens < 0 || max_query_len < 0 || num_q_heads <= 0 ||
         num_kv_heads <= 0 || head_dim <= 0 || block_size <= 0)
         return PA_ERR_INVALID_ARG;
     if (num_q_heads % num_kv_heads != 0) return PA_ERR_INVALID_ARG;
     if (!is_act(q_dtype)) return PA_ERR_UNSUPPORTED;
-    if (kv_dtype != q_dtype) return PA_ERR_UNSUPPORTED;  // 8-bit caches: not on this path
+    if (kv_dtype != q_dtype && !is_8bit(kv_dtype)) return PA_ERR_UNSUPPORTED;
     if (head_dim != 64 && head_dim != 128) return PA_ERR_UNSUPPORTED;
+    if (is_8bit(kv_dtype) && head_dim != 128) return PA_ERR_UNSUPPORTED;
+    if (is_8bit(kv_dtype) &&
+        !(isfinite(k_scale) && k_scale > 0.f && isfinite(v_scale) && v_scale > 0.f))
+        return PA_ERR_INVALID_ARG;
     if (block_size != 16 && block_size != 32) return PA_ERR_UNSUPPORTED;
     const int g = num_q_heads / num_kv_heads;
     if (g > 128) return PA_ERR_UNSUPPORTED;
@@ -364,8 +368,11 @@ pa_status pa_prefill(void *out, const void *q, const void *k_cache, const void *
     p.group = g;
     p.tok_per_tile = 128 / g;
     p.oob_row = (int)rows;
-    p.qk_scale_log2 = (float)((double)softmax_scale * 1.4426950408889634074);
-    return from_cuda(pa::launch_prefill(p, to_internal(q_dtype), head_dim,
+    const bool kv8 = is_8bit(kv_dtype);
+    p.qk_scale_log2 =
+        (float)((double)softmax_scale * (kv8 ? (double)k_scale : 1.0) * 1.4426950408889634074);
+    p.v_scale = kv8 ? v_scale : 1.0f;
+    return from_cuda(pa::launch_prefill(p, to_internal(q_dtype), to_internal(kv_dtype), head_dim,
                                         static_cast<cudaStream_t>(stream)));
 }
 
@@ -499,15 +506,16 @@ pa_status pa_decode_shared_prefix(void *out, const void *q, const void *k_cache,
                                   int max_blocks_per_seq, const int32_t *seq_lens, int num_seqs,
                                   int num_q_heads, int num_kv_heads, int head_dim, int block_size,
                                   int num_blocks, float softmax_scale, pa_dtype q_dtype,
-                                  pa_dtype kv_dtype, int prefix_len, int partition_size,
-                                  int max_seq_len, void *workspace, size_t workspace_bytes,
-                                  int *dev_err, void *stream) {
+                                  pa_dtype kv_dtype, float k_scale, float v_scale, int prefix_len,
+                                  int partition_size, int max_seq_len, void *workspace,
+                                  size_t workspace_bytes, int *dev_err, void *stream) {
     const DecodeArgs a = {out, q, k_cache, v_cache, block_tables, max_blocks_per_seq, seq_lens,
                           num_seqs, num_q_heads, num_kv_heads, head_dim, block_size, num_blocks,
-                          softmax_scale, q_dtype, kv_dtype, 1.0f, 1.0f};
+                          softmax_scale, q_dtype, kv_dtype, k_scale, v_scale};
     pa_status st = check_decode(a);
     if (st != PA_OK) return st;
-    if (kv_dtype != q_dtype) return PA_ERR_UNSUPPORTED;  // the prefix pass reads 16-bit caches
+    const bool kv8 = is_8bit(kv_dtype);
+    if (kv8 && head_dim != 128) return PA_ERR_UNSUPPORTED;  // the prefix pass: 8-bit needs d 128
     const int g = num_q_heads / num_kv_heads;
     if (g > 128) return PA_ERR_UNSUPPORTED;
     if (!(softmax_scale > 0.f)) return PA_ERR_INVALID_ARG;
@@ -552,12 +560,15 @@ pa_status pa_decode_shared_prefix(void *out, const void *q, const void *k_cache,
     f.group = g;
     f.tok_per_tile = 128 / g;
     f.oob_row = (int)pool_rows;
-    f.qk_scale_log2 = (float)((double)softmax_scale * 1.4426950408889634074);
+    f.qk_scale_log2 =
+        (float)((double)softmax_scale * (kv8 ? (double)k_scale : 1.0) * 1.4426950408889634074);
+    f.v_scale = kv8 ? v_scale : 1.0f;
     f.shared_len = prefix_len;
     f.ws_o = ws_o;
     f.ws_lse = ws_lse;
     f.ws_np = np;
-    if (pa::launch_prefill(f, to_internal(q_dtype), head_dim, s) != cudaSuccess) return PA_ERR_CUDA;
+    if (pa::launch_prefill(f, to_internal(q_dtype), to_internal(kv_dtype), head_dim, s) != cudaSuccess)
+        return PA_ERR_CUDA;
 
     // 2. every sequence's tail, split into partitions: slots 1 .. np - 1
     if (np_tail > 0) {

@@ -149,7 +149,8 @@ struct PrefillParams {  // chunked prefill (pa_prefill)
     int group;                  // Hq / Hk
     int tok_per_tile;           // floor(128 / group) chunk tokens per query tile
     int oob_row;                // a pool row index past the end (zero-filled loads)
-    float qk_scale_log2;        // softmax_scale * log2(e)
+    float qk_scale_log2;        // softmax_scale * k_scale * log2(e)
+    float v_scale;              // applied to the output (1 for 16-bit caches)
     // shared-prefix mode (shared_len > 0): one "sequence" = the first
     // shared_len tokens of block table row 0; the T query rows (one per
     // decoding sequence) all see every one of them (no causal mask), and each
@@ -184,10 +185,10 @@ cudaError_t launch_decode(const DecodeParams &p, DType q, DType kv, int head_dim
 cudaError_t launch_reduce(const ReduceParams &p, DType q, int head_dim, cudaStream_t stream);
 cudaError_t launch_copy_blocks(const CopyBlocksParams &p, cudaStream_t stream);
 
-// Chunked prefill on tcgen05 tensor cores (pa_prefill.cu): 16-bit caches,
-// head_dim 64 / 128, GQA groups up to 128.
+// Chunked prefill on tcgen05 tensor cores (pa_prefill.cu): 16-bit caches
+// (head_dim 64 / 128) or 8-bit ones (head_dim 128), GQA groups up to 128.
 bool prefill_supported();
-cudaError_t launch_prefill(const PrefillParams &p, DType q, int head_dim, cudaStream_t stream);
+cudaError_t launch_prefill(const PrefillParams &p, DType q, DType kv, int head_dim, cudaStream_t stream);
 
 // Tensor-core decode (pa_decode_mma.cu): rows of the MMA used for the GQA
 // group (8 or 16); supported for head_dim 64/128 16-bit caches and head_dim

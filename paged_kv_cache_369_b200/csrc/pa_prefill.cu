@@ -200,37 +200,51 @@ __device__ __forceinline__ void unpack2(uint32_t w, float &lo, float &hi, bf16_t
 
 }  // namespace tc
 
-template <typename T, int D> struct PfCfg {
+// T: q / out dtype; KVT: cache dtype (T, or an 8-bit code for which a
+// converter warp widens each landed K/V tile to f16 in shared memory).
+template <typename T, int D, typename KVT = T> struct PfCfg {
+    static constexpr bool KV8 = Elem<KVT>::kBytes == 1;
     static constexpr int BM = 128;  // query rows per tile (TMEM lanes); two tiles per CTA
     static constexpr int BN = 64;   // keys per tile = 4 blocks
-    static constexpr int ST = 4;    // K/V ring stages
-    static constexpr int ATOMS = D / 64;  // 128-byte swizzle atoms across d
+    // K/V operand ring stages (16-bit): the MMA issuer reads tile j + 2's
+    // stage while PV(j) still holds tile j's, so at least 3
+    static constexpr int ST = KV8 ? 3 : 4;
+    static constexpr int SST = KV8 ? 4 : 0;  // 8-bit staging ring stages
+    static constexpr int ATOMS = D / 64;  // 128-byte swizzle atoms across d (16-bit)
     static constexpr int Q_BYTES = ATOMS * BM * 128;  // one query tile
     static constexpr int KV_BYTES = ATOMS * BN * 128;
+    static constexpr int KV8_BYTES = BN * D;          // one 8-bit tile (d = 128: 128-byte rows)
     static constexpr int OFF_Q = 0;                   // tile A, then tile B
     static constexpr int OFF_KV = 2 * Q_BYTES;        // stage st: K, then V
-    static constexpr int OFF_BAR = OFF_KV + ST * 2 * KV_BYTES;
+    static constexpr int OFF_STG = OFF_KV + ST * 2 * KV_BYTES;  // 8-bit stage: K, then V
+    static constexpr int OFF_BAR = OFF_STG + SST * 2 * KV8_BYTES;
     // q_full, kv_full[ST], kv_empty[ST], then per (tile, score buffer):
-    // s_full, p_full, pv_done; drain
-    static constexpr int NBAR = 1 + 2 * ST + 4 + 4 + 4 + 1;
+    // s_full, p_full, pv_done; drain; q_ready, stg_full[SST], stg_empty[SST]
+    static constexpr int NBAR = 1 + 2 * ST + 4 + 4 + 4 + 1 + 1 + 2 * SST;
     static constexpr int OFF_SLOT = OFF_BAR + NBAR * 8;
     static constexpr int OFF_ABORT = OFF_SLOT + 4;
-    static constexpr int USED = OFF_ABORT + 4;
+    static constexpr int OFF_QEXP = OFF_ABORT + 4;    // log2 of the q scaling (8-bit caches)
+    static constexpr int USED = OFF_QEXP + 4;
     // at least 120 KiB so that one CTA holds an SM (and its 512 TMEM columns)
     static constexpr int SMEM = 1024 + (USED < 120 * 1024 ? 120 * 1024 : USED);
-    static constexpr bool HILO = std::is_same<T, bf16_t>::value;
+    // MMA operand type: T, or f16 for 8-bit caches (codes widen to f16 exactly)
+    static constexpr bool OP_BF16 = std::is_same<T, bf16_t>::value && !KV8;
+    static constexpr bool HILO = OP_BF16;
     static constexpr uint32_t TMEM_COLS = 512;
     // score buffer b of tile t at column 64 (2 t + b) (P written over it), O
     // of tile t at 256 + 128 t
     static constexpr uint32_t COL_S = 0, COL_O = 256;
-    static constexpr uint32_t FMT = HILO ? 1u : 0u;  // kind::f16 operand format: f16 0, bf16 1
+    static constexpr uint32_t FMT = OP_BF16 ? 1u : 0u;  // kind::f16 operand format: f16 0, bf16 1
     // instruction descriptors: fp32 accumulate, A/B format, majors, N >> 3, M >> 4
     static constexpr uint32_t IDESC_QK = (1u << 4) | (FMT << 7) | (FMT << 10) |
                                          ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
     static constexpr uint32_t IDESC_PV = (1u << 4) | (FMT << 7) | (FMT << 10) | (1u << 16) |
                                          ((uint32_t)(D >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
-    static constexpr int THREADS = 320;  // 8 softmax warps, a TMA warp, an MMA warp
+    // 8 softmax warps, a TMA warp, an MMA warp (+ a converter warp for 8-bit caches)
+    static constexpr int THREADS = KV8 ? 352 : 320;
     static_assert(D == 64 || D == 128, "head_dim 64 or 128");
+    static_assert(!KV8 || D == 128, "8-bit caches: head_dim 128");
+    static_assert(ST >= 3, "two key tiles of look-ahead plus the one in PV");
     static_assert(SMEM <= 227 * 1024, "shared memory budget");
 };
 
@@ -240,12 +254,13 @@ __device__ __forceinline__ float ex2(float x) {  // 2^x; -inf -> +0
     return y;
 }
 
-template <typename T, int D>
-__global__ void __launch_bounds__(320, 1)
+template <typename T, int D, typename KVT>
+__global__ void __launch_bounds__(PfCfg<T, D, KVT>::THREADS, 1)
     prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tmap_q,
                    const __grid_constant__ CUtensorMap tmap_k,
                    const __grid_constant__ CUtensorMap tmap_v) {
-    using C = PfCfg<T, D>;
+    using C = PfCfg<T, D, KVT>;
+    using OpT = typename std::conditional<C::OP_BF16, bf16_t, f16_t>::type;  // MMA operand type
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_addr(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;
@@ -284,6 +299,10 @@ __global__ void __launch_bounds__(320, 1)
     auto bar_p_full = [&](int t, int b) { return bars + 8u * (5 + 2 * C::ST + 2 * t + b); };
     auto bar_pv = [&](int t, int b) { return bars + 8u * (9 + 2 * C::ST + 2 * t + b); };
     const uint32_t bar_drain = bars + 8u * (13 + 2 * C::ST);
+    // 8-bit caches: Q converted to f16 (q_ready); staging ring of 8-bit tiles
+    const uint32_t bar_q_ready = bars + 8u * (14 + 2 * C::ST);
+    auto bar_stg_full = [&](int st) { return bars + 8u * (15 + 2 * C::ST + st); };
+    auto bar_stg_empty = [&](int st) { return bars + 8u * (15 + 2 * C::ST + C::SST + st); };
     auto s_col = [&](int t, int b) { return C::COL_S + 64u * (2 * t + b); };
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + C::OFF_ABORT);
     uint32_t *slot = reinterpret_cast<uint32_t *>(smem + C::OFF_SLOT);
@@ -304,6 +323,12 @@ __global__ void __launch_bounds__(320, 1)
                 mbar_init(bar_pv(t, b), 1);
             }
         mbar_init(bar_drain, 1);
+        mbar_init(bar_q_ready, 1);
+#pragma unroll
+        for (int st = 0; st < C::SST; ++st) {
+            mbar_init(bar_stg_full(st), 1);
+            mbar_init(bar_stg_empty(st), 1);
+        }
         *abort_flag = 0;
         mbar_init_fence();
     }
@@ -316,6 +341,8 @@ __global__ void __launch_bounds__(320, 1)
     auto q_smem = [&](int t) { return base + C::OFF_Q + (uint32_t)(t * C::Q_BYTES); };
     auto k_smem = [&](int st) { return base + C::OFF_KV + (uint32_t)(st * 2 * C::KV_BYTES); };
     auto v_smem = [&](int st) { return k_smem(st) + (uint32_t)C::KV_BYTES; };
+    auto stg_k = [&](int st) { return base + C::OFF_STG + (uint32_t)(st * 2 * C::KV8_BYTES); };
+    auto stg_v = [&](int st) { return stg_k(st) + (uint32_t)C::KV8_BYTES; };
 
     if (warp == 8) {
         // ================= TMA producer ===========================================
@@ -331,36 +358,47 @@ __global__ void __launch_bounds__(320, 1)
                     tc::tma_load_3d(q_smem(t) + a * C::BM * 128, &tmap_q, a * 64, kvh * g,
                                     q0 + tok0 + t * tpt, bar_q);
             const int32_t *bt = p.block_tables + (int64_t)s * p.max_blocks_per_seq;
+            auto row_of = [&](int lb) -> int {  // pool row of 16-token tile lb (past the pool: zeros)
+                int y = p.oob_row;
+                if (lb < nblk_seq) {
+                    const int phys = bt[lb >> p.tile_shift];
+                    if ((unsigned)phys < (unsigned)p.num_blocks)
+                        y = (phys * p.num_kv_heads + kvh) * p.block_size + (lb & tile_mask) * kBlockSize;
+                    else
+                        flag_error(p.err, kErrBounds);
+                }
+                return y;
+            };
+            constexpr int RING = C::KV8 ? C::SST : C::ST;  // the ring the copies land in
+            auto full_bar = [&](int st) { return C::KV8 ? bar_stg_full(st) : bar_kv_full(st); };
+            auto empty_bar = [&](int st) { return C::KV8 ? bar_stg_empty(st) : bar_kv_empty(st); };
             int j = 0;
             for (; j < nt; ++j) {
-                const int st = j % C::ST;
-                if (j >= C::ST &&
-                    !tc::wait_phase(bar_kv_empty(st), ((j / C::ST) - 1) & 1, abort_flag, p.err))
+                const int st = j % RING;
+                if (j >= RING && !tc::wait_phase(empty_bar(st), ((j / RING) - 1) & 1, abort_flag, p.err))
                     break;
-                mbar_arrive_expect_tx(bar_kv_full(st), 2u * C::KV_BYTES);
+                mbar_arrive_expect_tx(full_bar(st), C::KV8 ? 2u * C::KV8_BYTES : 2u * C::KV_BYTES);
 #pragma unroll 1
                 for (int b = 0; b < C::BN / kBlockSize; ++b) {
-                    const int lb = j * (C::BN / kBlockSize) + b;
-                    int y = p.oob_row;  // past the pool: a zero-filled box
-                    if (lb < nblk_seq) {
-                        const int phys = bt[lb >> p.tile_shift];
-                        if ((unsigned)phys < (unsigned)p.num_blocks)
-                            y = (phys * p.num_kv_heads + kvh) * p.block_size + (lb & tile_mask) * kBlockSize;
-                        else
-                            flag_error(p.err, kErrBounds);
-                    }
+                    const int y = row_of(j * (C::BN / kBlockSize) + b);
+                    if constexpr (C::KV8) {  // 16 rows x 128 codes, 128B swizzle
+                        const uint32_t off = b * kBlockSize * 128;
+                        tc::tma_load_2d(stg_k(st) + off, &tmap_k, 0, y, full_bar(st));
+                        tc::tma_load_2d(stg_v(st) + off, &tmap_v, 0, y, full_bar(st));
+                    } else {
 #pragma unroll
-                    for (int a = 0; a < C::ATOMS; ++a) {
-                        const uint32_t off = a * C::BN * 128 + b * kBlockSize * 128;
-                        tc::tma_load_2d(k_smem(st) + off, &tmap_k, a * 64, y, bar_kv_full(st));
-                        tc::tma_load_2d(v_smem(st) + off, &tmap_v, a * 64, y, bar_kv_full(st));
+                        for (int a = 0; a < C::ATOMS; ++a) {
+                            const uint32_t off = a * C::BN * 128 + b * kBlockSize * 128;
+                            tc::tma_load_2d(k_smem(st) + off, &tmap_k, a * 64, y, full_bar(st));
+                            tc::tma_load_2d(v_smem(st) + off, &tmap_v, a * 64, y, full_bar(st));
+                        }
                     }
                 }
             }
             // nothing may still be landing in shared memory when the CTA exits
             (void)mbar_wait_bounded(bar_q, 0, kWaitLimitNs);
-            for (int jj = j - C::ST < 0 ? 0 : j - C::ST; jj < j; ++jj)
-                (void)mbar_wait_bounded(bar_kv_full(jj % C::ST), (jj / C::ST) & 1, kWaitLimitNs);
+            for (int jj = j - RING < 0 ? 0 : j - RING; jj < j; ++jj)
+                (void)mbar_wait_bounded(full_bar(jj % RING), (jj / RING) & 1, kWaitLimitNs);
         }
         __syncwarp();
     } else if (warp == 9) {
@@ -423,7 +461,7 @@ __global__ void __launch_bounds__(320, 1)
             }
             return true;
         };
-        bool ok = wait_all(bar_q, 0);
+        bool ok = wait_all(C::KV8 ? bar_q_ready : bar_q, 0);  // 8-bit caches: q converted
         for (int j = 0; ok && j < 2 && j < nt; ++j) {
             ok = kv_ready(j);
             if (!ok) break;
@@ -451,6 +489,97 @@ __global__ void __launch_bounds__(320, 1)
             (void)mbar_wait_bounded(bar_drain, 0, kWaitLimitNs);
         }
         __syncwarp();
+    } else if (warp == 10) {
+        // ================= converter (8-bit caches only) ============================
+        // widens q (bf16 -> f16, scaled by a power of two so its largest
+        // magnitude sits near 2^14; the inverse folds into the logit scale)
+        // and every landed 8-bit K / V tile to f16 in the swizzled operand
+        // layout the MMAs read; each code's value is exact in f16
+        if constexpr (C::KV8) {
+            bool ok = __all_sync(tc::kFull, tc::wait_phase(bar_q, 0, abort_flag, p.err));
+            int e = 0;
+            if (ok && std::is_same<T, bf16_t>::value) {
+                const int rows = tpt * g;  // rows the copy wrote in each tile
+                float amax = 0.f;
+                for (int t = 0; t < 2; ++t)
+                    for (int a = 0; a < C::ATOMS; ++a)
+                        for (int idx = lane; idx < rows * 8; idx += 32) {
+                            uint32_t w[4];
+                            lds<16>(w, q_smem(t) + a * C::BM * 128 + (idx >> 3) * 128 + (idx & 7) * 16);
+                            float f[8];
+                            Unpack<bf16_t, 8>::run(w, f);
+#pragma unroll
+                            for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(f[i]));
+                        }
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(tc::kFull, amax, o));
+                if (amax > 0.f && amax <= 3.0e38f) {
+                    e = 14 - ((int)((__float_as_uint(amax) >> 23) & 0xFF) - 127);
+                    e = e > 100 ? 100 : (e < -100 ? -100 : e);
+                }
+                const float up = __uint_as_float((uint32_t)(127 + e) << 23);  // 2^e, exact
+                for (int t = 0; t < 2; ++t)
+                    for (int a = 0; a < C::ATOMS; ++a)
+                        for (int idx = lane; idx < rows * 8; idx += 32) {
+                            const uint32_t addr = q_smem(t) + a * C::BM * 128 + (idx >> 3) * 128 + (idx & 7) * 16;
+                            uint32_t w[4];
+                            lds<16>(w, addr);
+                            float f[8];
+                            Unpack<bf16_t, 8>::run(w, f);
+                            uint32_t h[4];
+#pragma unroll
+                            for (int i = 0; i < 4; ++i) h[i] = tc::pack2(f[2 * i] * up, f[2 * i + 1] * up, f16_t{});
+                            asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(h[0]),
+                                         "r"(h[1]), "r"(h[2]), "r"(h[3])
+                                         : "memory");
+                        }
+                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            }
+            if (lane == 0) *reinterpret_cast<volatile int *>(smem + C::OFF_QEXP) = e;
+            __syncwarp();
+            if (lane == 0) tc::mbar_arrive(bar_q_ready);
+            for (int j = 0; ok && j < nt; ++j) {
+                const int sst = j % C::SST, st = j % C::ST;
+                ok = __all_sync(tc::kFull, tc::wait_phase(bar_stg_full(sst), (j / C::SST) & 1, abort_flag, p.err));
+                if (!ok) break;
+                if (j >= C::ST) {  // the MMAs are done with this operand stage
+                    ok = __all_sync(tc::kFull,
+                                    tc::wait_phase(bar_kv_empty(st), ((j / C::ST) - 1) & 1, abort_flag, p.err));
+                    if (!ok) break;
+                }
+#pragma unroll
+                for (int kv = 0; kv < 2; ++kv) {
+                    const uint32_t src = kv ? stg_v(sst) : stg_k(sst);
+                    const uint32_t dst = kv ? v_smem(st) : k_smem(st);
+                    for (int idx = lane; idx < C::BN * 8; idx += 32) {
+                        const int r = idx >> 3, c8 = idx & 7;  // row, chunk of 16 codes
+                        uint32_t w[4];
+                        lds<16>(w, src + r * 128 + ((c8 ^ (r & 7)) << 4));
+                        uint32_t h[8];
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            h[2 * i] = cvt8x2_f16x2(w[i] & 0xFFFFu, KVT{});
+                            h[2 * i + 1] = cvt8x2_f16x2(w[i] >> 16, KVT{});
+                        }
+                        // codes 16 c8 .. +15 = f16 chunks 2 (c8 % 4) and +1 of atom c8 / 4
+                        const uint32_t rowb = dst + (c8 >> 2) * C::BN * 128 + r * 128;
+                        const int cf = (c8 & 3) * 2;
+                        asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(rowb + ((cf ^ (r & 7)) << 4)),
+                                     "r"(h[0]), "r"(h[1]), "r"(h[2]), "r"(h[3])
+                                     : "memory");
+                        asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(rowb + (((cf + 1) ^ (r & 7)) << 4)),
+                                     "r"(h[4]), "r"(h[5]), "r"(h[6]), "r"(h[7])
+                                     : "memory");
+                    }
+                }
+                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                __syncwarp();
+                if (lane == 0) {
+                    tc::mbar_arrive(bar_stg_empty(sst));
+                    tc::mbar_arrive(bar_kv_full(st));
+                }
+            }
+        }
     } else {
         // ================= softmax: one thread per query row =======================
         const int t = warp >> 2;                  // query tile (0: A, 1: B)
@@ -460,7 +589,12 @@ __global__ void __launch_bounds__(320, 1)
         const int pos = causal ? ctx + tok0 + rtok : L - 1;
         const uint32_t lane_bits = (uint32_t)((warp & 3) * 32) << 16;
         const uint32_t ocol = tmem + lane_bits + C::COL_O + 128u * t;
-        const float sl2 = p.qk_scale_log2;  // > 0
+        float sl2 = p.qk_scale_log2;  // > 0
+        if constexpr (C::KV8) {  // q was scaled by 2^e on its way to f16
+            if (!__all_sync(tc::kFull, tc::wait_phase(bar_q_ready, 0, abort_flag, p.err))) sl2 = 0.f;
+            const int e = *reinterpret_cast<volatile int *>(smem + C::OFF_QEXP);
+            sl2 *= __uint_as_float((uint32_t)(127 - e) << 23);
+        }
         float m_ref = -CUDART_INF_F, l = 0.f;
         bool ok = true;
         for (int j = 0; j < nt; ++j) {
@@ -501,11 +635,11 @@ __global__ void __launch_bounds__(320, 1)
                     const float p0 = ex2(fmaf(__uint_as_float(sv[c0 + 2 * i]), sl2, nmb));
                     const float p1 = ex2(fmaf(__uint_as_float(sv[c0 + 2 * i + 1]), sl2, nmb));
                     ps[i & 3] += p0 + p1;
-                    hi[i] = tc::pack2(p0, p1, T{});
+                    hi[i] = tc::pack2(p0, p1, OpT{});
                     if constexpr (C::HILO) {
                         float h0, h1;
                         tc::unpack2(hi[i], h0, h1, bf16_t{});
-                        lo[i] = tc::pack2(p0 - h0, p1 - h1, T{});
+                        lo[i] = tc::pack2(p0 - h0, p1 - h1, OpT{});
                     }
                 }
                 tc::st16(scol + c0 / 2, hi);
@@ -542,7 +676,7 @@ __global__ void __launch_bounds__(320, 1)
             // ---- epilogue: out = O / l, rounded once to the q dtype ----------------
             // (shared-prefix mode: the partial o / l and its log-sum-exp, fp32)
             tc::fence_after();
-            const float inv = l > 0.f ? 1.f / l : 0.f;
+            const float inv = l > 0.f ? p.v_scale / l : 0.f;  // v_scale: 1 for 16-bit caches
             const int64_t row = ((int64_t)(q0 + tok0 + rtok) * p.num_q_heads + (int64_t)kvh * g + r % g);
             uint4 *dst = reinterpret_cast<uint4 *>(static_cast<uint16_t *>(p.out) + row * D);
             if (!causal) {
@@ -612,15 +746,16 @@ bool encode_q_map(CUtensorMap *m, const void *q, int d, int hq, int64_t tokens, 
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <typename T, int D>
+template <typename T, int D, typename KVT>
 cudaError_t launch_prefill_t(const PrefillParams &p, cudaStream_t stream) {
-    using C = PfCfg<T, D>;
+    using C = PfCfg<T, D, KVT>;
     const int64_t rows = (int64_t)p.num_blocks * p.num_kv_heads * p.block_size;
+    constexpr int EB = Elem<KVT>::kBytes;
     CUtensorMap mq, mk, mv;
     if (!encode_q_map(&mq, p.q, D, p.num_q_heads, p.num_tokens, p.group, p.tok_per_tile) ||
-        !encode_pool_map(&mk, p.k_cache, 2, D, rows) || !encode_pool_map(&mv, p.v_cache, 2, D, rows))
+        !encode_pool_map(&mk, p.k_cache, EB, D, rows) || !encode_pool_map(&mv, p.v_cache, EB, D, rows))
         return cudaErrorInvalidValue;
-    auto kern = prefill_kernel<T, D>;
+    auto kern = prefill_kernel<T, D, KVT>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
     if (e != cudaSuccess) return e;
     const int per_cta = 2 * p.tok_per_tile;  // two query tiles
@@ -634,11 +769,22 @@ cudaError_t launch_prefill_t(const PrefillParams &p, cudaStream_t stream) {
 
 bool prefill_supported() { return encode_fn() != nullptr; }
 
-cudaError_t launch_prefill(const PrefillParams &p, DType q, int head_dim, cudaStream_t stream) {
+template <typename T>
+static cudaError_t prefill_by_kv(const PrefillParams &p, DType kv, int head_dim, cudaStream_t stream) {
+    switch (kv) {
+        case DType::E4M3: return launch_prefill_t<T, 128, e4m3_t>(p, stream);
+        case DType::E5M2: return launch_prefill_t<T, 128, e5m2_t>(p, stream);
+        case DType::I8: return launch_prefill_t<T, 128, i8_t>(p, stream);
+        default:
+            return head_dim == 64 ? launch_prefill_t<T, 64, T>(p, stream) : launch_prefill_t<T, 128, T>(p, stream);
+    }
+}
+
+cudaError_t launch_prefill(const PrefillParams &p, DType q, DType kv, int head_dim, cudaStream_t stream) {
     if (p.num_seqs <= 0 || p.num_tokens <= 0 || p.max_query_len <= 0) return cudaSuccess;
-    if (q == DType::F16)
-        return head_dim == 64 ? launch_prefill_t<f16_t, 64>(p, stream) : launch_prefill_t<f16_t, 128>(p, stream);
-    return head_dim == 64 ? launch_prefill_t<bf16_t, 64>(p, stream) : launch_prefill_t<bf16_t, 128>(p, stream);
+    if (is_8bit(kv) && head_dim != 128) return cudaErrorInvalidValue;
+    return q == DType::F16 ? prefill_by_kv<f16_t>(p, kv, head_dim, stream)
+                           : prefill_by_kv<bf16_t>(p, kv, head_dim, stream);
 }
 
 }  // namespace pa

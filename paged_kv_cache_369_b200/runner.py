@@ -133,7 +133,8 @@ class PagedDecode:
             pa_decode_shared_prefix(self.out, self.q, self.k_cache, self.v_cache,
                                     self.block_tables, self.seq_lens, w.softmax_scale,
                                     self.prefix_len, self.partition_size, self.max_seq_len,
-                                    self.workspace, self.dev_err, self.stream)
+                                    self.workspace, self.dev_err, self.stream, w.k_scale,
+                                    w.v_scale)
             return
         if self.mode == "single":
             pa_decode(self.out, self.q, self.k_cache, self.v_cache, self.block_tables,
@@ -214,8 +215,8 @@ class PagedPrefill:
         self.seq_lens = torch.from_numpy(np.ascontiguousarray(w.seq_lens)).to(dev)
         self.query_start = torch.from_numpy(np.ascontiguousarray(w.query_start)).to(dev)
         shape = (w.num_blocks, w.num_kv_heads, w.block_size, w.head_dim)
-        self.k_cache = torch.empty(shape, dtype=act, device=dev)
-        self.v_cache = torch.empty(shape, dtype=act, device=dev)
+        self.k_cache = torch.empty(shape, dtype=pool_torch_dtype(w.kv_dtype), device=dev)
+        self.v_cache = torch.empty(shape, dtype=pool_torch_dtype(w.kv_dtype), device=dev)
         self.k_cache.view(torch.uint8).fill_(0xFF)
         self.v_cache.view(torch.uint8).fill_(0xFF)
         self.slots = torch.empty(max(T, 1), dtype=torch.int64, device=dev)
@@ -252,7 +253,8 @@ class PagedPrefill:
     def attend(self) -> None:
         w = self.w
         pa_prefill(self.out, self.q, self.k_cache, self.v_cache, self.block_tables, self.seq_lens,
-                   self.query_start, w.max_query_len, w.softmax_scale, self.dev_err, self.stream)
+                   self.query_start, w.max_query_len, w.softmax_scale, self.dev_err, self.stream,
+                   w.k_scale, w.v_scale)
 
     def step(self) -> None:
         self.write_chunk()

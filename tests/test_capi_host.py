@@ -183,11 +183,13 @@ def test_prefill_checks(pa):
     L = pa.lib()
 
     def call(out=A, q=A, qs=A, S=2, T=8, mq=4, Hq=8, Hk=2, d=128, B=16, NB=10, qd=pa.PA_BF16,
-             kvd=pa.PA_BF16, scale=0.1):
+             kvd=pa.PA_BF16, scale=0.1, ks=1.0, vs=1.0):
         return L.pa_prefill(out, q, A, A, A, 4, A, qs, S, T, mq, Hq, Hk, d, B, NB, scale, qd, kvd,
-                            None, None)
+                            ks, vs, None, None)
 
-    assert call(kvd=pa.PA_FP8_E4M3) == 2     # E4M3 caches: not on the prefill path
+    assert call(kvd=pa.PA_FP8_E4M3, d=64) == 2   # 8-bit caches: head_dim 128
+    assert call(kvd=pa.PA_FP8_E4M3, ks=0.0) == 1  # 8-bit caches need positive scales
+    assert call(kvd=pa.PA_INT8, vs=float("inf")) == 1
     assert call(qd=pa.PA_F16) == 2           # cache dtype must be the q dtype
     assert call(d=96) == 2
     assert call(B=64) == 2
@@ -234,11 +236,14 @@ def test_shared_prefix_checks(pa):
     assert need == 256 + (2 * 8 * 3 * 128 * 4 + 255) // 256 * 256
     assert pa.pa_shared_prefix_workspace_bytes(2, 8, 128, 1000, 512, 0) == 0
 
-    def call(prefix=512, P=256, kv=pa.PA_BF16, ws=A, wsb=need, maxlen=1000, B=16, scale=0.1):
-        return L.pa_decode_shared_prefix(A, A, A, A, A, 80, A, 2, 8, 2, 128, B, 10, scale,
-                                         pa.PA_BF16, kv, prefix, P, maxlen, ws, wsb, None, None)
+    def call(prefix=512, P=256, kv=pa.PA_BF16, ws=A, wsb=need, maxlen=1000, B=16, scale=0.1,
+             ks=1.0, d=128):
+        return L.pa_decode_shared_prefix(A, A, A, A, A, 80, A, 2, 8, 2, d, B, 10, scale,
+                                         pa.PA_BF16, kv, ks, 1.0, prefix, P, maxlen, ws, wsb, None,
+                                         None)
 
-    assert call(kv=pa.PA_FP8_E4M3) == 2     # 16-bit caches only
+    assert call(kv=pa.PA_FP8_E4M3, d=64) == 2   # 8-bit caches: head_dim 128
+    assert call(kv=pa.PA_FP8_E4M3, ks=-1.0) == 1
     assert call(prefix=0) == 1
     assert call(prefix=24) == 1              # not a multiple of the block size
     assert call(prefix=1200) == 1            # longer than max_seq_len

@@ -193,6 +193,8 @@ CASCADE = [
     (4, 4, 128, "bf16", [17, 18, 200], 16, 16),
     (32, 8, 128, "f16", [97, 300, 65], 64, 32),
     (24, 8, 64, "bf16", [130, 129], 128, 16),       # GQA 3
+    (32, 8, 128, "bf16", [100, 65, 66, 700], 64, 16, "e4m3"),
+    (8, 8, 128, "f16", [1040, 1100], 1024, 16, "int8"),
 ]
 
 
@@ -202,8 +204,9 @@ def test_shared_prefix_decode_parity(case, P, kernel_choice):
     """pa_decode_shared_prefix: the prefix attended once for all sequences
     (tensor-core pass), tails split, merged -- against the oracle's decode."""
     pa, PagedDecode = _pa()
-    Hq, Hk, d, act, lens, prefix, B = CASCADE[case]
-    w = workload.build(f"casc{case}", 5000 + case, lens, Hq, Hk, d, act, act,
+    Hq, Hk, d, act, lens, prefix, B = CASCADE[case][:7]
+    kv = CASCADE[case][7] if len(CASCADE[case]) > 7 else act
+    w = workload.build(f"casc{case}", 5000 + case, lens, Hq, Hk, d, act, kv,
                        shared_prefix_tokens=prefix, block_size=B, extra_table_cols=1)
     dec = PagedDecode(w, mode="cascade", partition_size=P)
     dec.step()

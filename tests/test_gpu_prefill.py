@@ -153,3 +153,26 @@ def test_prefill_block_size_32(case):
     assert np.array_equal(pool_bytes(pre.k_cache), kc.view(np.uint8).reshape(pool_bytes(pre.k_cache).shape))
     ref = oracle.prefill_for(w, kc, vc)
     assert_close(_f64(pre.out), ref, f"prefill block 32 case {case}")
+
+
+@pytest.mark.parametrize("case", [
+    # (context lens, chunk lens, Hq, Hk, act, kv)
+    ([0, 100, 300], [128, 33, 200], 32, 8, "bf16", "e4m3"),
+    ([0, 64, 1000], [130, 3, 257], 64, 8, "bf16", "int8"),
+    ([3, 250], [29, 64], 4, 4, "f16", "e5m2"),
+    ([20, 0, 127], [9, 17, 1], 6, 2, "f16", "e4m3"),
+])
+def test_prefill_8bit_caches(case):
+    """8-bit caches (per-tensor scales): the converter warp widens each tile
+    to f16 in shared memory; against the oracle, which dequantises the same
+    codes (pools compared bit for bit first)."""
+    ctx, chunk, Hq, Hk, act, kv = case
+    w = workload.build_chunked(f"pf8_{kv}", 2200 + Hq, ctx, chunk, Hq, Hk, 128, act, kv,
+                               extra_table_cols=2)
+    pre = _run(w)
+    assert pre.error() == 0
+    kc, vc = oracle.chunked_caches_for(w)
+    assert np.array_equal(pool_bytes(pre.k_cache), kc.view(np.uint8).reshape(pool_bytes(pre.k_cache).shape))
+    assert np.array_equal(pool_bytes(pre.v_cache), vc.view(np.uint8).reshape(pool_bytes(pre.v_cache).shape))
+    ref = oracle.prefill_for(w, kc, vc)
+    assert_close(_f64(pre.out), ref, f"prefill {kv} {case}")

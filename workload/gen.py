@@ -554,15 +554,19 @@ PREFILL_NAMES = {
 }
 
 
-def prefill_config(cfg: int) -> ChunkedWorkload:
+def prefill_config(cfg: int, kv_dtype: Optional[str] = None) -> ChunkedWorkload:
     """Named chunked-prefill workloads: 512-token chunks (the chunk size the
-    pages give) on the decode configurations' model shapes."""
+    pages give) on the decode configurations' model shapes; ``kv_dtype``
+    swaps in an 8-bit cache (per-tensor scales)."""
     seed = SEED_BASE + 100 + cfg
     rng = np.random.default_rng([seed, 1])
+    kv = kv_dtype or "bf16"
     if cfg == 1:
         ctx = rng.integers(0, 3584, size=16, endpoint=True)
-        return build_chunked(PREFILL_NAMES[1], seed, ctx, [512] * 16, 32, 8, 128, "bf16", "bf16")
+        name = PREFILL_NAMES[1] if kv == "bf16" else f"{PREFILL_NAMES[1]}, {kv} cache"
+        return build_chunked(name, seed, ctx, [512] * 16, 32, 8, 128, "bf16", kv)
     if cfg == 2:
         ctx = rng.integers(1536, 2048, size=8, endpoint=True)
-        return build_chunked(PREFILL_NAMES[2], seed, ctx, [512] * 8, 64, 8, 128, "bf16", "bf16")
+        name = PREFILL_NAMES[2] if kv == "bf16" else f"{PREFILL_NAMES[2]}, {kv} cache"
+        return build_chunked(name, seed, ctx, [512] * 8, 64, 8, 128, "bf16", kv)
     raise ValueError(f"unknown prefill config {cfg}")
