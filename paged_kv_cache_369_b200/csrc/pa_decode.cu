@@ -410,16 +410,40 @@ __global__ void __launch_bounds__(kDecodeWarps * 32)
 }
 
 // ---------------------------------------------------------------------------
-// split-KV reduce: one CTA per (sequence, query head), one thread per element.
-// The partition weights w_p = exp(lse_p - M) are computed once per chunk of
-// up to D partitions into shared memory; the weighted sum then issues
-// independent loads (no dependent-load chain across partitions).
+// split-KV reduce: one CTA of kReduceWarps warps per (sequence, query head).
+// Each lane owns D / 32 consecutive elements (one vector load per partition);
+// the warps take interleaved partitions, keeping kReduceUnroll partitions'
+// loads in flight per lane, and their sums meet in shared memory.  The
+// partition weights w_p = exp(lse_p - M) come from lse values every lane of
+// the warp reads at the same address (one broadcast load).
 // ---------------------------------------------------------------------------
 
+constexpr int kReduceWarps = 4;
+constexpr int kReduceUnroll = 8;
+
+template <int V> struct VecF;
+template <> struct VecF<4> {
+    using T = float4;
+    __device__ static void add(float *acc, float w, const T &v) {
+        acc[0] = fmaf(w, v.x, acc[0]); acc[1] = fmaf(w, v.y, acc[1]);
+        acc[2] = fmaf(w, v.z, acc[2]); acc[3] = fmaf(w, v.w, acc[3]);
+    }
+};
+template <> struct VecF<2> {
+    using T = float2;
+    __device__ static void add(float *acc, float w, const T &v) {
+        acc[0] = fmaf(w, v.x, acc[0]); acc[1] = fmaf(w, v.y, acc[1]);
+    }
+};
+
 template <typename QT, int D>
-__global__ void __launch_bounds__(D) reduce_kernel(const ReduceParams p) {
-    __shared__ float w_s[D];
-    __shared__ float red[D / 32];
+__global__ void __launch_bounds__(kReduceWarps * 32) reduce_kernel(const ReduceParams p) {
+    constexpr int V = D / 32;  // elements per lane
+    using VF = VecF<V>;
+    using VT = typename VF::T;
+    __shared__ float red[kReduceWarps];
+    __shared__ float part_num[kReduceWarps][D];
+    __shared__ float part_den[kReduceWarps];
     pdl_wait();
     const int64_t row = blockIdx.x;
     const int s = (int)(row / p.num_q_heads);
@@ -430,46 +454,63 @@ __global__ void __launch_bounds__(D) reduce_kernel(const ReduceParams p) {
     L = L < 0 ? 0 : (L > cap ? cap : L);
     const int np = p.extra + (L + p.partition_size - 1) / p.partition_size;
     const float *lse = p.ws_lse + row * NP;
-    const float *o = p.ws_o + row * NP * D;
-    const int d = threadIdx.x, lane = d & 31, wid = d >> 5;
+    const VT *o = reinterpret_cast<const VT *>(p.ws_o + row * NP * D);
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
 
     // M = max_p lse_p
     float m = -CUDART_INF_F;
-    for (int i = d; i < np; i += D) m = fmaxf(m, lse[i]);
+    for (int i = threadIdx.x; i < np; i += kReduceWarps * 32) m = fmaxf(m, lse[i]);
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, off));
     if (lane == 0) red[wid] = m;
     __syncthreads();
     float M = red[0];
 #pragma unroll
-    for (int w = 1; w < D / 32; ++w) M = fmaxf(M, red[w]);
+    for (int w = 1; w < kReduceWarps; ++w) M = fmaxf(M, red[w]);
 
-    float num = 0.f, den = 0.f;
+    float acc[V];
+#pragma unroll
+    for (int j = 0; j < V; ++j) acc[j] = 0.f;
+    float den = 0.f;
     if (M != -CUDART_INF_F) {
-        for (int base = 0; base < np; base += D) {
-            const int n = np - base < D ? np - base : D;
-            __syncthreads();  // previous chunk's weights are consumed
-            if (d < n) w_s[d] = expf(lse[base + d] - M);
-            __syncthreads();
-            const float *ob = o + (int64_t)base * D + d;
-            int i = 0;
-            for (; i + 4 <= n; i += 4) {
-                const float o0 = ob[(int64_t)i * D], o1 = ob[(int64_t)(i + 1) * D];
-                const float o2 = ob[(int64_t)(i + 2) * D], o3 = ob[(int64_t)(i + 3) * D];
-                num = fmaf(w_s[i], o0, num);
-                num = fmaf(w_s[i + 1], o1, num);
-                num = fmaf(w_s[i + 2], o2, num);
-                num = fmaf(w_s[i + 3], o3, num);
-                den += (w_s[i] + w_s[i + 1]) + (w_s[i + 2] + w_s[i + 3]);
+        constexpr int STRIDE = kReduceWarps * kReduceUnroll;
+        int i0 = wid;
+        for (; i0 + (kReduceUnroll - 1) * kReduceWarps < np; i0 += STRIDE) {
+            VT v[kReduceUnroll];
+            float lv[kReduceUnroll];
+#pragma unroll
+            for (int u = 0; u < kReduceUnroll; ++u) {
+                const int i = i0 + u * kReduceWarps;
+                v[u] = o[(int64_t)i * (D / V) + lane];
+                lv[u] = lse[i];
             }
-            for (; i < n; ++i) {
-                num = fmaf(w_s[i], ob[(int64_t)i * D], num);
-                den += w_s[i];
+#pragma unroll
+            for (int u = 0; u < kReduceUnroll; ++u) {
+                const float w = expf(lv[u] - M);
+                den += w;
+                VF::add(acc, w, v[u]);
             }
         }
+        for (int i = i0; i < np; i += kReduceWarps) {
+            const float w = expf(lse[i] - M);
+            den += w;
+            VF::add(acc, w, o[(int64_t)i * (D / V) + lane]);
+        }
     }
-    const float r = den > 0.f ? num / den : 0.f;
-    reinterpret_cast<uint16_t *>(p.out)[row * D + d] = from_float(QT{}, r);
+#pragma unroll
+    for (int j = 0; j < V; ++j) part_num[wid][lane * V + j] = acc[j];
+    if (lane == 0) part_den[wid] = den;
+    __syncthreads();
+    for (int d = threadIdx.x; d < D; d += kReduceWarps * 32) {
+        float num = 0.f, dsum = 0.f;
+#pragma unroll
+        for (int w = 0; w < kReduceWarps; ++w) {
+            num += part_num[w][d];
+            dsum += part_den[w];
+        }
+        const float r = dsum > 0.f ? num / dsum : 0.f;
+        reinterpret_cast<uint16_t *>(p.out)[row * D + d] = from_float(QT{}, r);
+    }
 }
 
 // ---------------------------------------------------------------------------
@@ -543,12 +584,13 @@ cudaError_t launch_decode(const DecodeParams &p, DType q, DType kv, int head_dim
 cudaError_t launch_reduce(const ReduceParams &p, DType q, int head_dim, cudaStream_t stream) {
     if (p.num_seqs <= 0) return cudaSuccess;
     const dim3 grid((unsigned)((int64_t)p.num_seqs * p.num_q_heads));
+    const dim3 block(kReduceWarps * 32);
     if (q == DType::F16) {
-        if (head_dim == 64) return launch_pdl(reduce_kernel<f16_t, 64>, grid, dim3(64), 0, stream, p);
-        return launch_pdl(reduce_kernel<f16_t, 128>, grid, dim3(128), 0, stream, p);
+        if (head_dim == 64) return launch_pdl(reduce_kernel<f16_t, 64>, grid, block, 0, stream, p);
+        return launch_pdl(reduce_kernel<f16_t, 128>, grid, block, 0, stream, p);
     }
-    if (head_dim == 64) return launch_pdl(reduce_kernel<bf16_t, 64>, grid, dim3(64), 0, stream, p);
-    return launch_pdl(reduce_kernel<bf16_t, 128>, grid, dim3(128), 0, stream, p);
+    if (head_dim == 64) return launch_pdl(reduce_kernel<bf16_t, 64>, grid, block, 0, stream, p);
+    return launch_pdl(reduce_kernel<bf16_t, 128>, grid, block, 0, stream, p);
 }
 
 }  // namespace pa
