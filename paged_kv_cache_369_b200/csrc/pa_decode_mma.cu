@@ -166,7 +166,15 @@ template <typename QT, typename KVT, int D, int GT, int NW_ = kDecodeWarps> stru
     static constexpr int BOX_BYTES = kBlockSize * 128;  // 2 KiB
     static constexpr int TILE_BYTES = NBOX * BOX_BYTES;
     static constexpr int STAGE_BYTES = 2 * TILE_BYTES;
-    static constexpr int NST = (16384 / STAGE_BYTES) < 2 ? 2 : (16384 / STAGE_BYTES);
+    // Residency.  8-bit tiles (4 KiB a stage) with 8 MMA rows: 3 stages a warp
+    // and 16 warps an SM at 128 registers a thread -- the 8-bit path is
+    // latency-bound, and 16 warps beat 12 warps with 4 stages (long-context
+    // E4M3: 129.7 -> 120.3 us; 10 two-warp CTAs with 2 stages, 126.4 us).
+    // Otherwise 16 KiB of stages a warp and 12 warps an SM (16-bit tiles:
+    // shared memory bound; 16 MMA rows: their accumulators need the registers).
+    static constexpr bool WIDE = FP8 && GT == 8;
+    static constexpr int NST = WIDE ? 3 : ((16384 / STAGE_BYTES) < 2 ? 2 : (16384 / STAGE_BYTES));
+    static constexpr int MIN_CTAS = (WIDE ? 16 : 12) / NW_;
     static constexpr int KS = D / 16;   // k-steps of q.K
     static constexpr int MT = D / 16;   // m-tiles (16 rows of d) of O^T = V^T P^T
     static constexpr int NH = GT / 8;   // n-tiles (8 heads) of O^T
@@ -188,7 +196,7 @@ __device__ __forceinline__ uint32_t swz(int r, int c) {
 // CHAN: per-channel scales (8-bit caches only), a separate instantiation so
 // that the per-tensor kernels compile exactly as without them
 template <typename QT, typename KVT, int D, int GT, bool CHAN, int NWARPS>
-__global__ void __launch_bounds__(NWARPS * 32, 12 / NWARPS)
+__global__ void __launch_bounds__(NWARPS * 32, MmaCfg<QT, KVT, D, GT, NWARPS>::MIN_CTAS)
     decode_mma_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmap_k,
                       const __grid_constant__ CUtensorMap tmap_v) {
     using C = MmaCfg<QT, KVT, D, GT, NWARPS>;
