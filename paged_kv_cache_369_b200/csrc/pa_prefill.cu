@@ -159,6 +159,24 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap *map
         : "memory");
 }
 
+// Four 8-bit codes of one word -> two f16x2 (codes 0,1 in lo; 2,3 in hi), exact.
+template <typename KT>
+__device__ __forceinline__ void widen4(uint32_t w, uint32_t &lo, uint32_t &hi, KT) {
+    lo = cvt8x2_f16x2(w & 0xFFFFu, KT{});
+    hi = cvt8x2_f16x2(w >> 16, KT{});
+}
+// INT8, a word at a time: one bias flip (b ^ 0x80 = b + 128) for the four
+// bytes, each pair under the f16 exponent byte 0x64 (value 1024 + 128 + b),
+// then 1152 subtracted from both halves.
+__device__ __forceinline__ void widen4(uint32_t w, uint32_t &lo, uint32_t &hi, i8_t) {
+    const uint32_t x = w ^ 0x80808080u;
+    uint32_t a, b;
+    asm("prmt.b32 %0, %1, %2, 0x5140;" : "=r"(a) : "r"(x), "r"(0x6464u));
+    asm("prmt.b32 %0, %1, %2, 0x5342;" : "=r"(b) : "r"(x), "r"(0x6464u));
+    asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(lo) : "r"(a), "r"(0x64806480u));
+    asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(hi) : "r"(b), "r"(0x64806480u));
+}
+
 __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
 }
@@ -240,8 +258,10 @@ template <typename T, int D, typename KVT = T> struct PfCfg {
                                          ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
     static constexpr uint32_t IDESC_PV = (1u << 4) | (FMT << 7) | (FMT << 10) | (1u << 16) |
                                          ((uint32_t)(D >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
-    // 8 softmax warps, a TMA warp, an MMA warp (+ a converter warp for 8-bit caches)
-    static constexpr int THREADS = KV8 ? 352 : 320;
+    // 8 softmax warps, a TMA warp, an MMA warp (+ two converter warps, K and V,
+    // for 8-bit caches)
+    static constexpr int CONVERTERS = KV8 ? 2 : 0;
+    static constexpr int THREADS = 320 + 32 * CONVERTERS;
     static_assert(D == 64 || D == 128, "head_dim 64 or 128");
     static_assert(!KV8 || D == 128, "8-bit caches: head_dim 128");
     static_assert(ST >= 3, "two key tiles of look-ahead plus the one in PV");
@@ -311,7 +331,7 @@ __global__ void __launch_bounds__(PfCfg<T, D, KVT>::THREADS, 1)
         mbar_init(bar_q, 1);
 #pragma unroll
         for (int st = 0; st < C::ST; ++st) {
-            mbar_init(bar_kv_full(st), 1);
+            mbar_init(bar_kv_full(st), C::KV8 ? C::CONVERTERS : 1);  // TMA, or the converters
             mbar_init(bar_kv_empty(st), 1);
         }
 #pragma unroll
@@ -327,7 +347,7 @@ __global__ void __launch_bounds__(PfCfg<T, D, KVT>::THREADS, 1)
 #pragma unroll
         for (int st = 0; st < C::SST; ++st) {
             mbar_init(bar_stg_full(st), 1);
-            mbar_init(bar_stg_empty(st), 1);
+            mbar_init(bar_stg_empty(st), C::CONVERTERS);
         }
         *abort_flag = 0;
         mbar_init_fence();
@@ -489,16 +509,18 @@ __global__ void __launch_bounds__(PfCfg<T, D, KVT>::THREADS, 1)
             (void)mbar_wait_bounded(bar_drain, 0, kWaitLimitNs);
         }
         __syncwarp();
-    } else if (warp == 10) {
-        // ================= converter (8-bit caches only) ============================
-        // widens q (bf16 -> f16, scaled by a power of two so its largest
-        // magnitude sits near 2^14; the inverse folds into the logit scale)
-        // and every landed 8-bit K / V tile to f16 in the swizzled operand
-        // layout the MMAs read; each code's value is exact in f16
+    } else if (warp >= 10) {
+        // ================= converters (8-bit caches only) ===========================
+        // warp 10 widens q (bf16 -> f16, scaled by a power of two so its
+        // largest magnitude sits near 2^14; the inverse folds into the logit
+        // scale) and every landed 8-bit K tile, warp 11 every V tile, to f16
+        // in the swizzled operand layout the MMAs read; each code's value is
+        // exact in f16
         if constexpr (C::KV8) {
-            bool ok = __all_sync(tc::kFull, tc::wait_phase(bar_q, 0, abort_flag, p.err));
+            const int kv = warp - 10;  // 0: K, 1: V
+            bool ok = kv == 1 || __all_sync(tc::kFull, tc::wait_phase(bar_q, 0, abort_flag, p.err));
             int e = 0;
-            if (ok && std::is_same<T, bf16_t>::value) {
+            if (kv == 0 && ok && std::is_same<T, bf16_t>::value) {
                 const int rows = tpt * g;  // rows the copy wrote in each tile
                 float amax = 0.f;
                 for (int t = 0; t < 2; ++t)
@@ -535,9 +557,11 @@ __global__ void __launch_bounds__(PfCfg<T, D, KVT>::THREADS, 1)
                         }
                 asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
             }
-            if (lane == 0) *reinterpret_cast<volatile int *>(smem + C::OFF_QEXP) = e;
-            __syncwarp();
-            if (lane == 0) tc::mbar_arrive(bar_q_ready);
+            if (kv == 0) {
+                if (lane == 0) *reinterpret_cast<volatile int *>(smem + C::OFF_QEXP) = e;
+                __syncwarp();
+                if (lane == 0) tc::mbar_arrive(bar_q_ready);
+            }
             for (int j = 0; ok && j < nt; ++j) {
                 const int sst = j % C::SST, st = j % C::ST;
                 ok = __all_sync(tc::kFull, tc::wait_phase(bar_stg_full(sst), (j / C::SST) & 1, abort_flag, p.err));
@@ -547,8 +571,7 @@ __global__ void __launch_bounds__(PfCfg<T, D, KVT>::THREADS, 1)
                                     tc::wait_phase(bar_kv_empty(st), ((j / C::ST) - 1) & 1, abort_flag, p.err));
                     if (!ok) break;
                 }
-#pragma unroll
-                for (int kv = 0; kv < 2; ++kv) {
+                {
                     const uint32_t src = kv ? stg_v(sst) : stg_k(sst);
                     const uint32_t dst = kv ? v_smem(st) : k_smem(st);
                     for (int idx = lane; idx < C::BN * 8; idx += 32) {
@@ -557,10 +580,7 @@ __global__ void __launch_bounds__(PfCfg<T, D, KVT>::THREADS, 1)
                         lds<16>(w, src + r * 128 + ((c8 ^ (r & 7)) << 4));
                         uint32_t h[8];
 #pragma unroll
-                        for (int i = 0; i < 4; ++i) {
-                            h[2 * i] = cvt8x2_f16x2(w[i] & 0xFFFFu, KVT{});
-                            h[2 * i + 1] = cvt8x2_f16x2(w[i] >> 16, KVT{});
-                        }
+                        for (int i = 0; i < 4; ++i) tc::widen4(w[i], h[2 * i], h[2 * i + 1], KVT{});
                         // codes 16 c8 .. +15 = f16 chunks 2 (c8 % 4) and +1 of atom c8 / 4
                         const uint32_t rowb = dst + (c8 >> 2) * C::BN * 128 + r * 128;
                         const int cf = (c8 & 3) * 2;
