@@ -80,10 +80,10 @@ def measured_hbm_peak():
 DECODE_SOURCES = ("pa_decode.cu", "pa_decode_mma.cu", "pa_device.cuh", "pa_internal.h", "pa_tmap.h")
 
 
-def kernel_source_hash() -> str:
+def kernel_source_hash(sources=DECODE_SOURCES) -> str:
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "paged_kv_cache_369_b200", "csrc")
-    for name in DECODE_SOURCES:
+    for name in sources:
         with open(os.path.join(csrc, name), "rb") as f:
             h.update(name.encode())
             h.update(f.read())
@@ -101,7 +101,7 @@ def recorded_traffic(cfg: int, mode: str):
         return None
     key = f"config{cfg}_{mode}"
     ent = rec.get(key)
-    if not ent or ent.get("kernel_hash") != kernel_source_hash():
+    if not ent or ent.get("kernel_hash") != kernel_source_hash(tuple(ent.get("sources", DECODE_SOURCES))):
         return None
     return ent.get("dram_bytes_per_launch")
 

@@ -360,14 +360,16 @@ pa_status pa_decode_per_channel(void *out, const void *q, const void *k_cache, c
  * softmax_scale > 0, GQA groups up to 128.  Three launches on `stream`:
  *   1. the prefix: for each KV head, the queries of all sequences against the
  *      prefix keys as one dense tensor-core pass (the prefix K/V is read once,
- *      not once per sequence), giving each (sequence, head) a partial
- *      (lse, o) in workspace slot 0;
+ *      not once per sequence).  The prefix's keys are cut into Z contiguous
+ *      ranges (Z = min(8, ceil(prefix_len / 256)), fewer if a range would be
+ *      empty) that run side by side; each gives every (sequence, head) a
+ *      partial (lse, o) in workspace slot z;
  *   2. the tails (positions prefix_len .. L - 1) in partitions of
- *      partition_size tokens (a positive multiple of 16): slots 1 ..;
- *   3. the merge of slot 0 with the tail partitions into out.
+ *      partition_size tokens (a positive multiple of 16): slots Z ..;
+ *   3. the merge of all slots into out.
  * workspace: >= pa_shared_prefix_workspace_bytes(num_seqs, num_q_heads,
  * head_dim, max_seq_len, prefix_len, partition_size) bytes, 256-byte aligned:
- * lse [S, Hq, NP] fp32, then o [S, Hq, NP, d] fp32, NP = 1 +
+ * lse [S, Hq, NP] fp32, then o [S, Hq, NP, d] fp32, NP = Z +
  * ceil((max_seq_len - prefix_len) / partition_size), each section on a
  * 256-byte boundary.  Other arguments and errors as for
  * pa_decode_split_reduce.

@@ -8,6 +8,7 @@
 
 #include "../../include/pa.h"
 #include "pa_internal.h"
+#include "pa_shared_prefix.h"
 
 namespace {
 
@@ -496,7 +497,7 @@ size_t pa_shared_prefix_workspace_bytes(int num_seqs, int num_q_heads, int head_
         partition_size <= 0)
         return 0;
     const int tail = max_seq_len > prefix_len ? max_seq_len - prefix_len : 0;
-    const size_t np = 1 + (size_t)((tail + partition_size - 1) / partition_size);
+    const size_t np = (size_t)pa::prefix_splits(prefix_len) + (size_t)((tail + partition_size - 1) / partition_size);
     const size_t rows = (size_t)num_seqs * (size_t)num_q_heads * np;
     return align256(rows * sizeof(float)) + align256(rows * (size_t)head_dim * sizeof(float));
 }
@@ -534,14 +535,15 @@ pa_status pa_decode_shared_prefix(void *out, const void *q, const void *k_cache,
         return PA_ERR_INVALID_ARG;
     if (!pa::prefill_supported()) return PA_ERR_CUDA;  // no tensor-map encoder in the driver
     const int np_tail = (max_seq_len - prefix_len + partition_size - 1) / partition_size;
-    const int np = 1 + np_tail;
+    const int nz = pa::prefix_splits(prefix_len);  // prefix key ranges: slots 0 .. nz - 1
+    const int np = nz + np_tail;
     if ((int64_t)num_seqs * (np_tail > 0 ? np_tail : 1) > 0x7FFFFFFF) return PA_ERR_UNSUPPORTED;
     const size_t rows = (size_t)num_seqs * num_q_heads * np;
     float *ws_lse = static_cast<float *>(workspace);
     float *ws_o = reinterpret_cast<float *>(static_cast<uint8_t *>(workspace) + align256(rows * sizeof(float)));
     const cudaStream_t s = static_cast<cudaStream_t>(stream);
 
-    // 1. the prefix, once for every sequence: workspace slot 0
+    // 1. the prefix, once for every sequence: workspace slots 0 .. nz - 1
     pa::PrefillParams f = {};
     f.q = q;
     f.k_cache = k_cache;
@@ -570,7 +572,7 @@ pa_status pa_decode_shared_prefix(void *out, const void *q, const void *k_cache,
     if (pa::launch_prefill(f, to_internal(q_dtype), to_internal(kv_dtype), head_dim, s) != cudaSuccess)
         return PA_ERR_CUDA;
 
-    // 2. every sequence's tail, split into partitions: slots 1 .. np - 1
+    // 2. every sequence's tail, split into partitions: slots nz .. np - 1
     if (np_tail > 0) {
         pa::DecodeParams p = make_decode_params(a, dev_err);
         p.ws_lse = ws_lse;
@@ -579,12 +581,12 @@ pa_status pa_decode_shared_prefix(void *out, const void *q, const void *k_cache,
         p.num_partitions = np_tail;
         p.split = 1;
         p.tile_begin = prefix_len / pa::kBlockSize;
-        p.ws_offset = 1;
+        p.ws_offset = nz;
         p.ws_np = np;
         if (launch_any_decode(p, q_dtype, kv_dtype, head_dim, s) != cudaSuccess) return PA_ERR_CUDA;
     }
 
-    // 3. merge the prefix partial with the tail partitions
+    // 3. merge the prefix partials with the tail partitions
     pa::ReduceParams r = {};
     r.out = out;
     r.ws_lse = ws_lse;
@@ -594,7 +596,7 @@ pa_status pa_decode_shared_prefix(void *out, const void *q, const void *k_cache,
     r.num_q_heads = num_q_heads;
     r.num_partitions = np;
     r.partition_size = partition_size;
-    r.extra = 1;
+    r.extra = nz;
     r.token_begin = prefix_len;
     return from_cuda(pa::launch_reduce(r, to_internal(q_dtype), head_dim, s));
 }

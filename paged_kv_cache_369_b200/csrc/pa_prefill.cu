@@ -47,6 +47,7 @@
 #include <type_traits>
 
 #include "pa_device.cuh"
+#include "pa_shared_prefix.h"
 #include "pa_tmap.h"
 
 namespace pa {
@@ -286,7 +287,9 @@ __global__ void __launch_bounds__(PfCfg<T, D, KVT>::THREADS, 1)
     const uint32_t base = (raw + 1023u) & ~1023u;
     uint8_t *smem = smem_raw + (base - raw);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int cta_tile = blockIdx.x, kvh = blockIdx.y, s = blockIdx.z;
+    // z: the sequence (chunked prefill), or the prefix key range (shared mode)
+    const int cta_tile = blockIdx.x, kvh = blockIdx.y;
+    const int s = p.shared_len > 0 ? 0 : (int)blockIdx.z;
     const int g = p.group, tpt = p.tok_per_tile;
 
     // ---- this CTA's rows and keys (uniform over the CTA) ---------------------
@@ -303,8 +306,24 @@ __global__ void __launch_bounds__(PfCfg<T, D, KVT>::THREADS, 1)
     if (tok0 >= n) return;
     const int ntok = min(2 * tpt, n - tok0);
     const int ctx = L - n;
-    // key tiles up to the last row's position (all of the prefix without the mask)
-    const int nt = causal ? (ctx + tok0 + ntok - 1) / C::BN + 1 : (L + C::BN - 1) / C::BN;
+    // key tiles up to the last row's position (all of the prefix without the mask);
+    // shared mode: tiles j0 .. j0 + nt - 1 of the prefix, range blockIdx.z
+    int nt = causal ? (ctx + tok0 + ntok - 1) / C::BN + 1 : (L + C::BN - 1) / C::BN;
+    int j0 = 0;
+    const int split = causal ? 0 : (int)blockIdx.z;
+    if (!causal) {
+        const int per = (nt + (int)gridDim.z - 1) / (int)gridDim.z;
+        j0 = split * per;
+        nt = min(per, nt - j0);
+        if (nt <= 0) {  // an empty range (the host never makes one): an empty partial
+            for (int i = threadIdx.x; i < ntok * g; i += C::THREADS) {
+                const int64_t row = (int64_t)(q0 + tok0 + i / g) * p.num_q_heads + (int64_t)kvh * g + i % g;
+                p.ws_lse[row * p.ws_np + split] = -CUDART_INF_F;
+                for (int d = 0; d < D; ++d) p.ws_o[(row * p.ws_np + split) * D + d] = 0.f;
+            }
+            return;
+        }
+    }
     if (nt <= 0) return;  // an empty prefix
     const int nblk_seq = (L + kBlockSize - 1) / kBlockSize;  // 16-token tiles
     const int tile_mask = (1 << p.tile_shift) - 1;
@@ -400,7 +419,7 @@ __global__ void __launch_bounds__(PfCfg<T, D, KVT>::THREADS, 1)
                 mbar_arrive_expect_tx(full_bar(st), C::KV8 ? 2u * C::KV8_BYTES : 2u * C::KV_BYTES);
 #pragma unroll 1
                 for (int b = 0; b < C::BN / kBlockSize; ++b) {
-                    const int y = row_of(j * (C::BN / kBlockSize) + b);
+                    const int y = row_of((j0 + j) * (C::BN / kBlockSize) + b);
                     if constexpr (C::KV8) {  // 16 rows x 128 codes, 128B swizzle
                         const uint32_t off = b * kBlockSize * 128;
                         tc::tma_load_2d(stg_k(st) + off, &tmap_k, 0, y, full_bar(st));
@@ -467,9 +486,9 @@ __global__ void __launch_bounds__(PfCfg<T, D, KVT>::THREADS, 1)
         auto kv_ready = [&](int j) {
             const int st = j % C::ST;
             if (!wait_all(bar_kv_full(st), (j / C::ST) & 1)) return false;
-            if (j == j_tail) {
+            if (j0 + j == j_tail) {
                 // clear the V rows of the last block's unused slots (positions >= L)
-                const int r0 = L - j * C::BN, r1 = nblk_seq * kBlockSize - j * C::BN;
+                const int r0 = L - (j0 + j) * C::BN, r1 = nblk_seq * kBlockSize - (j0 + j) * C::BN;
                 const int chunks = (r1 - r0) * C::ATOMS * 8;
                 for (int c = lane; c < chunks; c += 32) {
                     const int row = r0 + c / (C::ATOMS * 8), rem = c % (C::ATOMS * 8);
@@ -627,7 +646,7 @@ __global__ void __launch_bounds__(PfCfg<T, D, KVT>::THREADS, 1)
             for (int c = 0; c < C::BN; c += 32) tc::ld32(scol + c, sv + c);
             tc::wait_ld<C::BN>(sv);
             // keys of this tile the row may see: all, a prefix (diagonal tile), none
-            const int lim = row_ok ? pos - j * C::BN + 1 : 0;
+            const int lim = row_ok ? pos - (j0 + j) * C::BN + 1 : 0;
             if (lim < C::BN) {
 #pragma unroll
                 for (int c = 0; c < C::BN; ++c)
@@ -700,9 +719,9 @@ __global__ void __launch_bounds__(PfCfg<T, D, KVT>::THREADS, 1)
             const int64_t row = ((int64_t)(q0 + tok0 + rtok) * p.num_q_heads + (int64_t)kvh * g + r % g);
             uint4 *dst = reinterpret_cast<uint4 *>(static_cast<uint16_t *>(p.out) + row * D);
             if (!causal) {
-                float4 *wo = reinterpret_cast<float4 *>(p.ws_o + row * p.ws_np * D);
+                float4 *wo = reinterpret_cast<float4 *>(p.ws_o + (row * p.ws_np + split) * D);
                 if (row_ok)
-                    p.ws_lse[row * p.ws_np] =
+                    p.ws_lse[row * p.ws_np + split] =
                         l > 0.f ? (m_ref + log2f(l)) * 0.69314718055994530942f : -CUDART_INF_F;
 #pragma unroll
                 for (int c = 0; c < D; c += 32) {
@@ -779,8 +798,10 @@ cudaError_t launch_prefill_t(const PrefillParams &p, cudaStream_t stream) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
     if (e != cudaSuccess) return e;
     const int per_cta = 2 * p.tok_per_tile;  // two query tiles
+    static_assert(C::BN == kPrefixKeyTile, "shared-prefix key ranges are counted in key tiles");
+    const int z = p.shared_len > 0 ? prefix_splits(p.shared_len) : p.num_seqs;
     const dim3 grid((unsigned)((p.max_query_len + per_cta - 1) / per_cta), (unsigned)p.num_kv_heads,
-                    (unsigned)p.num_seqs);
+                    (unsigned)z);
     kern<<<grid, C::THREADS, C::SMEM, stream>>>(p, mq, mk, mv);
     return cudaGetLastError();
 }

@@ -232,8 +232,19 @@ def test_per_channel_checks(pa):
 def test_shared_prefix_checks(pa):
     L = pa.lib()
     need = pa.pa_shared_prefix_workspace_bytes(2, 8, 128, 1000, 512, 256)
-    # 1 prefix slot + ceil(488 / 256) = 2 tail partitions
-    assert need == 256 + (2 * 8 * 3 * 128 * 4 + 255) // 256 * 256
+    # 2 prefix key ranges (ceil(512 / 256)) + ceil(488 / 256) = 2 tail partitions
+    assert need == 256 + (2 * 8 * 4 * 128 * 4 + 255) // 256 * 256
+
+    def slots(prefix, max_len, P=256):  # workspace slots per (sequence, head)
+        b = pa.pa_shared_prefix_workspace_bytes(1, 1, 64, max_len, prefix, P)
+        return (b - 256) // (64 * 4)
+
+    assert slots(16, 16) == 1                 # one key tile: one range, no tail
+    assert slots(256, 256) == 1
+    assert slots(1024, 1024) == 4             # 16 tiles in 4 ranges of 4
+    assert slots(1024, 1024 + 300) == 4 + 2
+    assert slots(4096, 4096) == 8             # at most 8 ranges
+    assert slots(320, 320) == 2               # 5 tiles: ranges of 3 and 2
     assert pa.pa_shared_prefix_workspace_bytes(2, 8, 128, 1000, 512, 0) == 0
 
     def call(prefix=512, P=256, kv=pa.PA_BF16, ws=A, wsb=need, maxlen=1000, B=16, scale=0.1,
