@@ -1,17 +1,20 @@
 """Benchmark of one paged decode step on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--config 2] [--mode fused|fused_single|split|single] [--partition 512]
+                    [--config 2] [--mode fused|fused_single|split|single|cascade]
+                    [--partition P]   (default 1024 tokens; 512 for config 4)
+    python bench.py --config 4 --kv int8 [--channel-scales]   (other 8-bit caches)
+    python bench.py --config 5 --mode cascade   (shared prefix attended once)
     python bench.py --op copy_blocks [--config 2] [--pairs 4096]
-    python bench.py --config 4 --kv int8     (another 8-bit cache format)
-    python bench.py --op prefill [--pconfig 1]
+    python bench.py --op prefill [--pconfig 1|2] [--kv e4m3|e5m2|int8]
 
 A step is one pass of the whole hot path over one batch: slot mapping of the
 new tokens, cache write of their K/V rows, and decode attention.  The default
 mode ("fused") makes it one pa_decode_append call: the split-KV decode kernel
 stores the new tokens itself, then the reduce kernel merges the partitions
 (2 launches).  "split" / "single" run pa_slot_mapping + pa_cache_write and
-then pa_decode_split_reduce / pa_decode (4 / 3 launches).  The default workload is the Qwen3-8B-shaped
+then pa_decode_split_reduce / pa_decode (4 / 3 launches); "cascade" runs them
+and then pa_decode_shared_prefix.  The default workload is the Qwen3-8B-shaped
 decode step: 64 sequences, 32 query / 8 KV heads, head_dim 128, bf16, lengths
 U[512, 4096], 16-token blocks in a shuffled pool.  Its K/V (~585 MB) is larger
 than L2 (126 MB), so no L2 flush is needed between steps.
@@ -21,7 +24,9 @@ Output: one JSON line on rank 0.  ``value`` is KV GB/s of the whole job
 the same with the step's inputs copied from pinned host memory and its output
 read back inside the timed region; ``roofline`` is for the attention launch
 (decode kernel + reduce kernel, event-timed together) against the measured HBM
-copy bandwidth;
+copy bandwidth, with ``traffic`` the DRAM bytes of those launches from the
+committed ncu record (profiles/decode_traffic.json) while its kernel sources
+are unchanged;
 ``cpu_baseline`` times the CPU oracle on a bounded sample.
 
 ``--impl reference`` times the CPU oracle itself as the reference arm (rank 0
