@@ -735,9 +735,10 @@ cudaError_t launch_mma_t(const DecodeParams &p, cudaStream_t stream) {
 // Warps per CTA.  Four warps share a partition's tiles and merge their
 // softmax states; with many partitions per sequence (long contexts) two warps
 // per CTA do better: half the per-CTA q preparation and merge work for the
-// same 12 warps per SM (long-context E4M3 shape, 512-token partitions: 146.6
-// -> 130.1 us), while for shorter, uneven sequences the smaller work units of
-// four warps balance better over the SMs (Qwen3-8B shape: 105.2 vs 111.9 us).
+// same warps per SM (long-context E4M3 shape, 512-token partitions, 12 warps
+// an SM: 146.6 -> 130.1 us), while for shorter, uneven sequences the smaller
+// work units of four warps balance better over the SMs (Qwen3-8B shape: 105.2
+// vs 111.9 us).
 constexpr int kLongSplitPartitions = 16;
 
 template <typename QT, typename KVT, int D, bool CHAN>

@@ -37,6 +37,14 @@
 //     otherwise p is taken against the old max, at most 2^8), P written back
 //     over S (bf16 as hi + lo halves so P keeps ~16 bits; f16 as one half),
 //     O / l at the end.
+//   - 8-bit caches (E4M3 / E5M2 / INT8, per-tensor scales, d = 128): the
+//     copies land in a staging ring; warp 10 widens Q (bf16 to f16 times a
+//     power of two) and each K tile, warp 11 each V tile, to f16 in the
+//     operand layout, so the MMAs run f16 x f16 (each code is exact in f16).
+// Shared-prefix mode (pa_decode_shared_prefix): the rows are the decoding
+// sequences' queries, every one of them sees all prefix keys (no mask), and
+// the prefix's key tiles are cut into gridDim.z ranges, each writing its own
+// partial (lse, o) workspace slot for the reduce to merge.
 // V rows past the sequence's last token (the tail of its last block) are
 // cleared in shared memory before P.V: p = 0 there, but 0 x NaN poison = NaN.
 // Every wait is bounded; a timeout reports PA_ERR_DEVICE_TIMEOUT, makes the
@@ -219,8 +227,8 @@ __device__ __forceinline__ void unpack2(uint32_t w, float &lo, float &hi, bf16_t
 
 }  // namespace tc
 
-// T: q / out dtype; KVT: cache dtype (T, or an 8-bit code for which a
-// converter warp widens each landed K/V tile to f16 in shared memory).
+// T: q / out dtype; KVT: cache dtype (T, or an 8-bit code for which two
+// converter warps widen each landed K and V tile to f16 in shared memory).
 template <typename T, int D, typename KVT = T> struct PfCfg {
     static constexpr bool KV8 = Elem<KVT>::kBytes == 1;
     static constexpr int BM = 128;  // query rows per tile (TMEM lanes); two tiles per CTA
