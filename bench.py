@@ -119,10 +119,10 @@ def same_run_copy_gbs(device, stream, nbytes: int = 512 * 1024 * 1024, reps: int
     return 2.0 * nbytes / (ms * 1e-3) / 1e9
 
 
-def recorded_traffic(cfg: int, mode: str):
+def recorded_traffic(cfg: int, mode: str, path=None):
     """DRAM bytes per attention launch from the committed ncu summary, if it
     was taken on the current kernel sources (else None)."""
-    path = os.path.join(ROOT, "profiles", "decode_traffic.json")
+    path = path or os.path.join(ROOT, "profiles", "decode_traffic.json")
     try:
         with open(path) as f:
             rec = json.load(f)

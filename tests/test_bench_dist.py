@@ -48,3 +48,22 @@ def test_single_process_helpers_are_identity():
 
     assert bench.max_over_ranks(3.5, "cpu") == 3.5
     assert bench.sum_over_ranks(2.0, "cpu") == 2.0
+
+
+
+def test_recorded_traffic_follows_the_kernel_sources(tmp_path):
+    """roofline.traffic is reported only while every source an entry lists
+    hashes as it did when the counters were taken."""
+    import json
+
+    import bench
+
+    rec = {"config2_fused": {"dram_bytes_per_launch": 123, "kernel_hash": bench.kernel_source_hash()},
+           "config5_cascade": {"dram_bytes_per_launch": 456, "sources": ["pa_prefill.cu"],
+                               "kernel_hash": "0" * 16}}
+    path = tmp_path / "decode_traffic.json"
+    path.write_text(json.dumps(rec))
+    assert bench.recorded_traffic(2, "fused", str(path)) == 123
+    assert bench.recorded_traffic(5, "cascade", str(path)) is None  # the listed source changed
+    assert bench.recorded_traffic(3, "fused", str(path)) is None    # no capture
+    assert bench.recorded_traffic(2, "fused", str(tmp_path / "missing.json")) is None
