@@ -67,13 +67,22 @@ def test_prefill_vs_torch_sdpa_causal(orc, ctx, chunk, Hq, Hk, d, act):
     np.testing.assert_allclose(got, ref, rtol=1e-10, atol=1e-12)
 
 
-def test_prefill_fp8_vs_sdpa_on_dequantised(orc):
-    w = workload.build_chunked("pf8", 5, [30, 2], [20, 33], 8, 2, 32, "bf16", "e4m3")
+def _dequantise(codes, kv):
+    """8-bit codes to fp64 by torch's fp8 decoders / numpy's int8 view, not the oracle's."""
+    if kv == "int8":
+        return codes.view(np.int8).astype(np.float64)
+    fmt = torch.float8_e4m3fn if kv == "e4m3" else torch.float8_e5m2
+    return torch.from_numpy(codes).view(fmt).double().numpy()
+
+
+@pytest.mark.parametrize("kv", ["e4m3", "e5m2", "int8"])
+def test_prefill_8bit_vs_sdpa_on_dequantised(orc, kv):
+    w = workload.build_chunked("pf8", 5, [30, 2], [20, 33], 8, 2, 32, "bf16", kv)
     kc, vc = orc.chunked_caches_for(w)
     got = orc.prefill_for(w, kc, vc)
-    # rebuild the generator's rows from the E4M3 codes the oracle stored, via torch's decoder
-    k_deq = torch.from_numpy(kc).view(torch.float8_e4m3fn).double().numpy() * w.k_scale
-    v_deq = torch.from_numpy(vc).view(torch.float8_e4m3fn).double().numpy() * w.v_scale
+    # rebuild the generator's rows from the codes the oracle stored, decoded independently
+    k_deq = _dequantise(kc, kv) * w.k_scale
+    v_deq = _dequantise(vc, kv) * w.v_scale
     q = workload.bits_to_f32(w.q, w.act_dtype).astype(np.float64)
     for s in range(w.num_seqs):
         L, a, b = int(w.seq_lens[s]), int(w.query_start[s]), int(w.query_start[s + 1])
