@@ -195,6 +195,8 @@ CASCADE = [
     (24, 8, 64, "bf16", [130, 129], 128, 16),       # GQA 3
     (32, 8, 128, "bf16", [100, 65, 66, 700], 64, 16, "e4m3"),
     (8, 8, 128, "f16", [1040, 1100], 1024, 16, "int8"),
+    (16, 4, 128, "bf16", [401, 420, 999], 400, 16),   # 2 prefix key ranges, partial last tile
+    (8, 8, 128, "f16", [1041, 1300], 1040, 16),       # 5 ranges, the last one a 16-key tile
 ]
 
 
