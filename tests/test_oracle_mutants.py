@@ -48,6 +48,11 @@ MUTANTS = {
     "prefill_gqa_interleaved": ("int h = kvh * g + hh;", "int h = hh * num_kv_heads + kvh;"),
     "e5m2_bias_off_by_one": ("v = ldexp((double)(4 + m), e - 17);", "v = ldexp((double)(4 + m), e - 16);"),
     "e5m2_saturates_early": ("if (a >= 57344.0) return sign | 0x7B;", "if (a >= 49152.0) return sign | 0x7B;"),
+    "int8_decoded_unsigned": ("double orc_int8_decode(uint8_t c) { return (double)(int8_t)c; }",
+                              "double orc_int8_decode(uint8_t c) { return (double)c; }"),
+    "e5m2_round_half_up": ("double n = orc_rne(ldexp(a, 2 - e)); /* in [4, 8] */",
+                           "double n = floor(ldexp(a, 2 - e) + 0.5);"),
+    "e5m2_subnormal_step": ("double n = orc_rne(a * 65536.0);", "double n = orc_rne(a * 32768.0);"),
     "int8_clamps_at_128": ("if (n > 127.0) n = 127.0;", "if (n > 128.0) n = 128.0;"),
     "int8_round_half_up": ("double n = orc_rne(fabs((double)y));", "double n = floor(fabs((double)y) + 0.5);"),
     "int8_scale_dropped_in_gather": ("rows[(int64_t)t * head_dim + i] = orc_is_8bit(kv_dtype) ? v * sc : v;",
@@ -85,6 +90,8 @@ def _run_pins(golden_dir):
         ("int8", lambda: kvf.test_int8_codec_vs_numpy(oracle)),
         ("sdpa_e5m2", lambda: kvf.test_decode_8bit_vs_torch_sdpa_on_dequantised(oracle, "e5m2")),
         ("sdpa_int8", lambda: kvf.test_decode_8bit_vs_torch_sdpa_on_dequantised(oracle, "int8")),
+        ("prefill_e5m2", lambda: pre.test_prefill_8bit_vs_sdpa_on_dequantised(oracle, "e5m2")),
+        ("prefill_int8", lambda: pre.test_prefill_8bit_vs_sdpa_on_dequantised(oracle, "int8")),
         ("chan_write", lambda: kvf.test_cache_write_per_channel_vs_torch_quantiser(oracle)),
         ("chan_sdpa", lambda: kvf.test_decode_per_channel_vs_torch_sdpa(oracle, "e4m3")),
         ("cow_example", lambda: cow.test_cow_beam_search_example(oracle, golden_dir)),
