@@ -218,8 +218,8 @@ size_t pa_split_workspace_bytes(int num_seqs, int num_q_heads, int head_dim, int
  *        o[s][h][p][:] = sum_t softmax-weight_t V_t over the partition (0 if empty)
  *   2. Reduce: M = max_p lse, w_p = exp(lse_p - M),
  *        out[s][h] = sum_p w_p o_p / sum_p w_p      (0 if every partition is empty)
- * partition_size P is a positive multiple of 16 (a partition may end inside a
- * 32-token block); max_seq_len bounds
+ * partition_size P is a positive multiple of 16, at most 2^30 (a partition
+ * may end inside a 32-token block); max_seq_len, at most 2^30, bounds
  * every seq_lens[s] (a longer one is truncated and flags PA_ERR_DEVICE_BOUNDS).
  * workspace (device, caller-owned, >= pa_split_workspace_bytes(...) bytes,
  * 256-byte aligned) holds the partials in the layout above after the call;

@@ -24,6 +24,12 @@ bool is_8bit(pa_dtype t) { return t == PA_FP8_E4M3 || t == PA_FP8_E5M2 || t == P
 pa::DType to_internal(pa_dtype t) { return static_cast<pa::DType>(static_cast<int>(t)); }
 
 size_t align256(size_t n) { return (n + 255) & ~size_t(255); }
+// ceil(a / b) for a >= 0, b > 0, without int overflow
+int64_t ceil_div64(int64_t a, int64_t b) { return (a + b - 1) / b; }
+// largest partition and max_seq_len the split entry points take: then every
+// token count the kernels form (partitions x partition size) stays in int
+constexpr int kMaxPartitionSize = 1 << 30;
+constexpr int kMaxSeqLen = 1 << 30;
 
 // Template group size (1, 2, 4 or 8) used for a GQA group of g query heads;
 // groups larger than 8 run as ceil(g / 8) CTAs per KV head.
@@ -269,7 +275,8 @@ pa_status pa_decode_append(void *out, const void *q, const void *k_new, const vo
                           softmax_scale, q_dtype, kv_dtype, k_scale, v_scale};
     pa_status st = check_decode(a);
     if (st != PA_OK) return st;
-    if (partition_size < 0 || partition_size % pa::kBlockSize != 0 || max_seq_len < 0)
+    if (partition_size < 0 || partition_size > kMaxPartitionSize || partition_size % pa::kBlockSize != 0 ||
+        max_seq_len < 0 || max_seq_len > kMaxSeqLen)
         return PA_ERR_INVALID_ARG;
     if (num_seqs == 0) return PA_OK;
     if (!k_new || !v_new || !aligned16(k_new) || !aligned16(v_new)) return PA_ERR_INVALID_ARG;
@@ -280,7 +287,7 @@ pa_status pa_decode_append(void *out, const void *q, const void *k_new, const vo
                                                      partition_size);
         if (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u))
             return PA_ERR_INVALID_ARG;
-        np = max_seq_len > 0 ? (max_seq_len + partition_size - 1) / partition_size : 1;
+        np = max_seq_len > 0 ? (int)ceil_div64(max_seq_len, partition_size) : 1;
         if ((int64_t)num_seqs * np > 0x7FFFFFFF) return PA_ERR_UNSUPPORTED;
     }
     pa::DecodeParams p = make_decode_params(a, dev_err);
@@ -450,7 +457,8 @@ pa_status pa_decode_per_channel(void *out, const void *q, const void *k_cache, c
     if (!is_8bit(kv_dtype)) return PA_ERR_UNSUPPORTED;
     const pa_status st = check_decode(a);
     if (st != PA_OK) return st;
-    if (partition_size < 0 || partition_size % pa::kBlockSize != 0 || max_seq_len < 0)
+    if (partition_size < 0 || partition_size > kMaxPartitionSize || partition_size % pa::kBlockSize != 0 ||
+        max_seq_len < 0 || max_seq_len > kMaxSeqLen)
         return PA_ERR_INVALID_ARG;
     if (num_seqs == 0) return PA_OK;
     if (!k_scales || !v_scales || (reinterpret_cast<uintptr_t>(k_scales) & 3u) ||
@@ -470,7 +478,7 @@ pa_status pa_decode_per_channel(void *out, const void *q, const void *k_cache, c
                                                  partition_size);
     if (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u))
         return PA_ERR_INVALID_ARG;
-    const int np = max_seq_len > 0 ? (max_seq_len + partition_size - 1) / partition_size : 1;
+    const int np = max_seq_len > 0 ? (int)ceil_div64(max_seq_len, partition_size) : 1;
     if ((int64_t)num_seqs * np > 0x7FFFFFFF) return PA_ERR_UNSUPPORTED;
     const size_t rows = (size_t)num_seqs * num_q_heads * np;
     p.ws_lse = static_cast<float *>(workspace);
@@ -497,7 +505,7 @@ size_t pa_shared_prefix_workspace_bytes(int num_seqs, int num_q_heads, int head_
         partition_size <= 0)
         return 0;
     const int tail = max_seq_len > prefix_len ? max_seq_len - prefix_len : 0;
-    const size_t np = (size_t)pa::prefix_splits(prefix_len) + (size_t)((tail + partition_size - 1) / partition_size);
+    const size_t np = (size_t)pa::prefix_splits(prefix_len) + (size_t)ceil_div64(tail, partition_size);
     const size_t rows = (size_t)num_seqs * (size_t)num_q_heads * np;
     return align256(rows * sizeof(float)) + align256(rows * (size_t)head_dim * sizeof(float));
 }
@@ -520,7 +528,8 @@ pa_status pa_decode_shared_prefix(void *out, const void *q, const void *k_cache,
     const int g = num_q_heads / num_kv_heads;
     if (g > 128) return PA_ERR_UNSUPPORTED;
     if (!(softmax_scale > 0.f)) return PA_ERR_INVALID_ARG;
-    if (partition_size <= 0 || partition_size % pa::kBlockSize != 0 || max_seq_len < 0)
+    if (partition_size <= 0 || partition_size > kMaxPartitionSize || partition_size % pa::kBlockSize != 0 ||
+        max_seq_len < 0 || max_seq_len > kMaxSeqLen)
         return PA_ERR_INVALID_ARG;
     if (prefix_len <= 0 || prefix_len % block_size != 0 || prefix_len > max_seq_len ||
         prefix_len > max_blocks_per_seq * block_size)
@@ -534,7 +543,7 @@ pa_status pa_decode_shared_prefix(void *out, const void *q, const void *k_cache,
     if (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u))
         return PA_ERR_INVALID_ARG;
     if (!pa::prefill_supported()) return PA_ERR_CUDA;  // no tensor-map encoder in the driver
-    const int np_tail = (max_seq_len - prefix_len + partition_size - 1) / partition_size;
+    const int np_tail = (int)ceil_div64((int64_t)max_seq_len - prefix_len, partition_size);
     const int nz = pa::prefix_splits(prefix_len);  // prefix key ranges: slots 0 .. nz - 1
     const int np = nz + np_tail;
     if ((int64_t)num_seqs * (np_tail > 0 ? np_tail : 1) > 0x7FFFFFFF) return PA_ERR_UNSUPPORTED;
@@ -606,7 +615,7 @@ size_t pa_split_workspace_bytes(int num_seqs, int num_q_heads, int head_dim, int
     if (num_seqs < 0 || num_q_heads <= 0 || head_dim <= 0 || max_seq_len < 0 ||
         partition_size <= 0)
         return 0;
-    const size_t np = max_seq_len > 0 ? (size_t)((max_seq_len + partition_size - 1) / partition_size) : 1;
+    const size_t np = max_seq_len > 0 ? (size_t)ceil_div64(max_seq_len, partition_size) : 1;
     const size_t rows = (size_t)num_seqs * (size_t)num_q_heads * np;
     return align256(rows * sizeof(float)) + align256(rows * (size_t)head_dim * sizeof(float));
 }
@@ -625,14 +634,15 @@ pa_status pa_decode_split_reduce(void *out, const void *q, const void *k_cache,
                           softmax_scale, q_dtype, kv_dtype, k_scale, v_scale};
     pa_status st = check_decode(a);
     if (st != PA_OK) return st;
-    if (partition_size <= 0 || partition_size % pa::kBlockSize != 0 || max_seq_len < 0)
+    if (partition_size <= 0 || partition_size > kMaxPartitionSize || partition_size % pa::kBlockSize != 0 ||
+        max_seq_len < 0 || max_seq_len > kMaxSeqLen)
         return PA_ERR_INVALID_ARG;
     if (num_seqs == 0) return PA_OK;
     const size_t need = pa_split_workspace_bytes(num_seqs, num_q_heads, head_dim, max_seq_len,
                                                  partition_size);
     if (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u))
         return PA_ERR_INVALID_ARG;
-    const int np = max_seq_len > 0 ? (max_seq_len + partition_size - 1) / partition_size : 1;
+    const int np = max_seq_len > 0 ? (int)ceil_div64(max_seq_len, partition_size) : 1;
     if ((int64_t)num_seqs * np > 0x7FFFFFFF) return PA_ERR_UNSUPPORTED;
 
     pa::DecodeParams p = make_decode_params(a, dev_err);

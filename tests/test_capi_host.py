@@ -120,6 +120,12 @@ def test_split_checks(pa):
     assert call(wsb=need - 1) == 1    # workspace too small
     assert call(ws=0) == 1
     assert call(ws=A + 128) == 1      # workspace must be 256-byte aligned
+    assert call(P=(1 << 30) + 16) == 1                     # partitions of at most 2^30 tokens
+    assert call(maxlen=(1 << 30) + 1) == 1                 # max_seq_len at most 2^30
+    # near the int range the partition count is still exact (no overflow):
+    # ceil((2^31 - 1) / 2^30) = 2 partitions
+    big = pa.pa_split_workspace_bytes(1, 1, 64, (1 << 31) - 1, 1 << 30)
+    assert big == 256 + 2 * 64 * 4
 
 
 def test_cache_write_and_slot_checks(pa):
