@@ -6,7 +6,10 @@ lengths, and K/V pools filled with 0xFF (NaN in every cache format) into which
 the earlier tokens are written by the library's own slot-mapping and
 cache-write kernels.  ``step()`` is one pass of the hot path, all through the
 C ABI: slot mapping of the new tokens, cache write, decode (single pass or
-split-KV partition + reduce).
+split-KV partition + reduce); in the fused modes one pa_decode_append call
+whose decode kernel stores the new tokens itself; in cascade mode the write
+then pa_decode_shared_prefix.  ``PagedPrefill`` does the same for one
+chunked-prefill step.
 
 PyTorch only provides device memory and streams here.
 """
@@ -194,10 +197,10 @@ def algorithmic_decode_bytes(w) -> int:
 
 class PagedPrefill:
     """One chunked-prefill step resident on a GPU (any object with the
-    attributes of ``workload.ChunkedWorkload``).  The context tokens are
-    written into 0xFF-poisoned pools at construction; ``step()`` appends the
-    chunk's K/V rows (pa_slot_mapping with token positions + pa_cache_write)
-    and runs pa_prefill."""
+    attributes of ``workload.ChunkedWorkload``; 16-bit or 8-bit caches).  The
+    context tokens are written into 0xFF-poisoned pools at construction;
+    ``step()`` appends the chunk's K/V rows (pa_slot_mapping with token
+    positions + pa_cache_write) and runs pa_prefill."""
 
     def __init__(self, w, device: str = "cuda", stream: Optional[torch.cuda.Stream] = None):
         self.w = w
