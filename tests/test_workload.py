@@ -73,3 +73,34 @@ def test_e4m3_scale_is_amax_over_448():
     k = np.concatenate([workload.bits_to_f32(w.k_prefill, "bf16").ravel(),
                         workload.bits_to_f32(w.k_new, "bf16").ravel()])
     assert w.k_scale == float(np.float32(np.abs(k).max()) / np.float32(448))
+
+
+@pytest.mark.parametrize("kv", ["e4m3", "e5m2", "int8"])
+def test_chunked_8bit_scale_is_amax_over_largest_code(kv):
+    """Chunked workloads with an 8-bit cache: per-tensor scales over every
+    context and chunk row, as for decode."""
+    w = workload.build_chunked("c8", 4, [10, 0], [7, 12], 4, 2, 32, "f16", kv)
+    for rows, scale in (((w.k_ctx, w.k_chunk), w.k_scale), ((w.v_ctx, w.v_chunk), w.v_scale)):
+        x = np.concatenate([workload.bits_to_f32(r, "f16").ravel() for r in rows])
+        largest = {"e4m3": 448.0, "e5m2": 57344.0, "int8": 127.0}[kv]  # each format's largest code
+        assert scale == float(np.float32(np.abs(x).max()) / np.float32(largest))
+
+
+def test_chunked_structure():
+    """A chunk is the last n of a sequence's L tokens; the context is the rest."""
+    w = workload.build_chunked("cs", 9, [5, 0, 33], [4, 9, 1], 8, 2, 64, "bf16", "bf16")
+    assert w.query_start.tolist() == [0, 4, 13, 14]
+    assert w.seq_lens.tolist() == [9, 9, 34]
+    for s in range(w.num_seqs):
+        L, n = int(w.seq_lens[s]), int(w.query_start[s + 1] - w.query_start[s])
+        assert sorted(w.chunk_pos[w.chunk_seq == s].tolist()) == list(range(L - n, L))
+        assert sorted(w.ctx_pos[w.ctx_seq == s].tolist()) == list(range(0, L - n))
+
+
+def test_prefill_config_with_8bit_cache():
+    """--op prefill --kv: the same sequences and shapes with an 8-bit cache."""
+    a, b = workload.prefill_config(1), workload.prefill_config(1, kv_dtype="int8")
+    assert b.kv_dtype == "int8" and a.kv_dtype == "bf16"
+    assert np.array_equal(a.seq_lens, b.seq_lens) and np.array_equal(a.query_start, b.query_start)
+    assert (b.num_q_heads, b.num_kv_heads, b.head_dim) == (a.num_q_heads, a.num_kv_heads, a.head_dim)
+    assert b.k_scale > 0 and b.v_scale > 0 and "int8" in b.name
