@@ -56,6 +56,28 @@ def check_pools(dec, kc, vc):
     assert np.array_equal(pool_bytes(dec.v_cache), vc.view(np.uint8).reshape(pool_bytes(dec.v_cache).shape))
 
 
+GUARD = 4096  # bytes of poison on each side of a guarded buffer (keeps 256-byte alignment)
+GUARD_BYTE = 0xA5
+
+
+def guarded_like(t: torch.Tensor):
+    """A tensor shaped and typed like ``t`` inside a larger buffer whose
+    GUARD bytes before and after it are filled with GUARD_BYTE; returns
+    (buffer, view).  A kernel that writes past either end of the view changes
+    the guard bytes."""
+    n = t.numel() * t.element_size()
+    buf = torch.full((n + 2 * GUARD,), GUARD_BYTE, dtype=torch.uint8, device=t.device)
+    view = buf[GUARD:GUARD + n].view(t.dtype).view(t.shape)
+    view.copy_(t)
+    return buf, view
+
+
+def check_guards(buf: torch.Tensor, what: str):
+    head, tail = buf[:GUARD].cpu().numpy(), buf[-GUARD:].cpu().numpy()
+    assert (head == GUARD_BYTE).all(), f"{what}: write before the buffer"
+    assert (tail == GUARD_BYTE).all(), f"{what}: write past the end of the buffer"
+
+
 def sample_pairs(w, n, seed=0):
     rng = np.random.default_rng(seed)
     S, Hq = w.num_seqs, w.num_q_heads
@@ -112,9 +134,14 @@ def test_small_full_parity(case, mode, P, kernel_choice):
     w = workload.build(f"small{case}", 1000 + case, lens, Hq, Hk, d, act, kv,
                        shared_prefix_tokens=prefix, extra_table_cols=2)
     dec = PagedDecode(w, mode=mode, partition_size=P)
+    # out and the split workspace sit between poisoned guard bands
+    out_buf, dec.out = guarded_like(dec.out)
+    ws_buf, dec.workspace = guarded_like(dec.workspace)
     dec.step()
     torch.cuda.synchronize()
     assert dec.error() == 0
+    check_guards(out_buf, "out")
+    check_guards(ws_buf, "workspace")
     kc, vc = oracle.caches_for(w)
     check_pools(dec, kc, vc)
     ref = oracle.decode_for(w, kc, vc)
@@ -211,9 +238,13 @@ def test_shared_prefix_decode_parity(case, P, kernel_choice):
     w = workload.build(f"casc{case}", 5000 + case, lens, Hq, Hk, d, act, kv,
                        shared_prefix_tokens=prefix, block_size=B, extra_table_cols=1)
     dec = PagedDecode(w, mode="cascade", partition_size=P)
+    out_buf, dec.out = guarded_like(dec.out)
+    ws_buf, dec.workspace = guarded_like(dec.workspace)
     dec.step()
     torch.cuda.synchronize()
     assert dec.error() == 0
+    check_guards(out_buf, "out")
+    check_guards(ws_buf, "workspace")
     kc, vc = oracle.caches_for(w)
     check_pools(dec, kc, vc)
     assert_close(_to_f64(dec.out), oracle.decode_for(w, kc, vc),
@@ -340,10 +371,18 @@ def _full(cfg, kv=None):
 @pytest.mark.parametrize("cfg,kv", [(1, None), (2, None), (3, None), (4, None), (5, None),
                                     (4, "e5m2"), (4, "int8"), (4, "e4m3-channel")])
 def test_named_workload_parity(cfg, kv):
+    """Each named workload at full size, first in exactly the launch
+    configuration bench.py times (fused step, the workload's default
+    split-KV partition), then split, single-pass and CUDA-core launches on the
+    same state, and split-KV at 512-token partitions where the default
+    differs."""
     pa, PagedDecode = _pa()
+    from paged_kv_cache_369_b200.runner import default_partition_size
+
     w, kc, vc = _full(cfg, kv)
     chan = w.k_chan is not None
-    dec = PagedDecode(w, mode="split" if chan else "fused", partition_size=512)
+    P = default_partition_size(w, cfg)
+    dec = PagedDecode(w, mode="split" if chan else "fused", partition_size=P)
     dec.step()  # pa_decode_append: the attention launch stores the new tokens
     torch.cuda.synchronize()
     assert dec.error() == 0
@@ -352,12 +391,20 @@ def test_named_workload_parity(cfg, kv):
     assert np.isfinite(out_split).all()
     pairs = sample_pairs(w, 64 if cfg > 1 else w.num_seqs * w.num_q_heads, seed=cfg)
     ref = oracle.decode_for(w, kc, vc, pairs)
-    assert_close(out_split[pairs[:, 0], pairs[:, 1]], ref, f"config {cfg} fused split")
+    assert_close(out_split[pairs[:, 0], pairs[:, 1]], ref, f"config {cfg} fused split P={P}")
     # unfused split attention on the same state
     dec.mode = "split"
     dec.attend()
     torch.cuda.synchronize()
-    assert_close(_to_f64(dec.out)[pairs[:, 0], pairs[:, 1]], ref, f"config {cfg} split")
+    assert_close(_to_f64(dec.out)[pairs[:, 0], pairs[:, 1]], ref, f"config {cfg} split P={P}")
+    if P != 512:  # the other partition size the kernels are tuned for
+        dec.partition_size = 512
+        need = pa.pa_split_workspace_bytes(w.num_seqs, w.num_q_heads, w.head_dim,
+                                           dec.max_seq_len, 512)
+        dec.workspace = torch.empty(max(need, 256), dtype=torch.uint8, device="cuda")
+        dec.attend()
+        torch.cuda.synchronize()
+        assert_close(_to_f64(dec.out)[pairs[:, 0], pairs[:, 1]], ref, f"config {cfg} split P=512")
     # single-pass launch on the same state
     dec.mode = "single"
     dec.attend()
