@@ -407,12 +407,16 @@ pa_status pa_decode_shared_prefix(void *out, const void *q, const void *k_cache,
  *
  * Arguments and result are those of pa_decode_split_reduce without
  * `workspace` / `workspace_bytes`.
- *   - Returns PA_ERR_INVALID_ARG, before touching the GPU, when the partials
+ *   - Argument errors are those of pa_decode_split_reduce and are returned
+ *     before the GPU is touched; so is PA_ERR_INVALID_ARG when the partials
  *     for these sizes, pa_split_workspace_bytes(num_seqs, num_q_heads,
  *     head_dim, max_seq_len, partition_size), exceed PA_STATIC_SCRATCH_BYTES.
- *   - The first call on a device looks up the array's device address on that
- *     (current) device; make that first call before any stream capture.
- *     PA_ERR_CUDA if the lookup fails.
+ *   - The first call in a CUDA context looks up the array's device address
+ *     on the current device; make that first call before any stream capture.
+ *     The address is remembered per device with the context's id, so a call
+ *     in another context of the device (e.g. after cudaDeviceReset, which
+ *     discards the array and its contents) looks it up again.  PA_ERR_CUDA
+ *     if the lookup fails.
  *   - Every call, on every stream, shares the one array per device, and the
  *     array keeps the last call's partials: nothing in it has to start at zero
  *     (each partial is written before it is read), but calls that overlap on

@@ -162,6 +162,16 @@ pa::DecodeParams make_decode_params(const DecodeArgs &a, int *dev_err) {
     const double log2e = 1.4426950408889634074;
     p.qk_scale_log2 = (float)((double)a.softmax_scale * (fp8 ? (double)a.k_scale : 1.0) * log2e);
     p.v_scale = fp8 ? a.v_scale : 1.0f;
+    // failure-detection test hook: PA369_TEST_DECODE_STALL_NS=<ns> makes every
+    // decode warp's first copy wait run out after <ns> nanoseconds (see
+    // DecodeParams); unset in normal use
+    if (const char *env = getenv("PA369_TEST_DECODE_STALL_NS")) {
+        const long long ns = atoll(env);
+        if (ns > 0) {
+            p.wait_limit_ns = (uint64_t)ns;
+            p.hold_first_tile = 1;
+        }
+    }
     return p;
 }
 
@@ -620,6 +630,39 @@ size_t pa_split_workspace_bytes(int num_seqs, int num_q_heads, int head_dim, int
     return align256(rows * sizeof(float)) + align256(rows * (size_t)head_dim * sizeof(float));
 }
 
+}  // extern "C"
+
+namespace pa {
+
+// The host-side checks of pa_decode_split_reduce, workspace aside (no GPU
+// access): PA_OK or the status the call returns before any launch.
+int check_split_reduce_args(const void *out, const void *q, const void *k_cache,
+                            const void *v_cache, const int32_t *block_tables,
+                            int max_blocks_per_seq, const int32_t *seq_lens, int num_seqs,
+                            int num_q_heads, int num_kv_heads, int head_dim, int block_size,
+                            int num_blocks, float softmax_scale, int q_dtype, int kv_dtype,
+                            float k_scale, float v_scale, int partition_size, int max_seq_len) {
+    // the checks only test out for null and alignment
+    const DecodeArgs a = {const_cast<void *>(out), q, k_cache, v_cache, block_tables,
+                          max_blocks_per_seq, seq_lens,
+                          num_seqs, num_q_heads, num_kv_heads, head_dim, block_size, num_blocks,
+                          softmax_scale, static_cast<pa_dtype>(q_dtype),
+                          static_cast<pa_dtype>(kv_dtype), k_scale, v_scale};
+    const pa_status st = check_decode(a);
+    if (st != PA_OK) return st;
+    if (partition_size <= 0 || partition_size > kMaxPartitionSize || partition_size % kBlockSize != 0 ||
+        max_seq_len < 0 || max_seq_len > kMaxSeqLen)
+        return PA_ERR_INVALID_ARG;
+    if (num_seqs == 0) return PA_OK;
+    const int64_t np = max_seq_len > 0 ? ceil_div64(max_seq_len, partition_size) : 1;
+    if ((int64_t)num_seqs * np > 0x7FFFFFFF) return PA_ERR_UNSUPPORTED;
+    return PA_OK;
+}
+
+}  // namespace pa
+
+extern "C" {
+
 pa_status pa_decode_split_reduce(void *out, const void *q, const void *k_cache,
                                  const void *v_cache, const int32_t *block_tables,
                                  int max_blocks_per_seq, const int32_t *seq_lens, int num_seqs,
@@ -629,21 +672,19 @@ pa_status pa_decode_split_reduce(void *out, const void *q, const void *k_cache,
                                  float v_scale, int partition_size, int max_seq_len,
                                  void *workspace, size_t workspace_bytes, int *dev_err,
                                  void *stream) {
+    const pa_status st = static_cast<pa_status>(pa::check_split_reduce_args(
+        out, q, k_cache, v_cache, block_tables, max_blocks_per_seq, seq_lens, num_seqs,
+        num_q_heads, num_kv_heads, head_dim, block_size, num_blocks, softmax_scale, q_dtype,
+        kv_dtype, k_scale, v_scale, partition_size, max_seq_len));
+    if (st != PA_OK || num_seqs == 0) return st;
     const DecodeArgs a = {out, q, k_cache, v_cache, block_tables, max_blocks_per_seq, seq_lens,
                           num_seqs, num_q_heads, num_kv_heads, head_dim, block_size, num_blocks,
                           softmax_scale, q_dtype, kv_dtype, k_scale, v_scale};
-    pa_status st = check_decode(a);
-    if (st != PA_OK) return st;
-    if (partition_size <= 0 || partition_size > kMaxPartitionSize || partition_size % pa::kBlockSize != 0 ||
-        max_seq_len < 0 || max_seq_len > kMaxSeqLen)
-        return PA_ERR_INVALID_ARG;
-    if (num_seqs == 0) return PA_OK;
     const size_t need = pa_split_workspace_bytes(num_seqs, num_q_heads, head_dim, max_seq_len,
                                                  partition_size);
     if (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u))
         return PA_ERR_INVALID_ARG;
     const int np = max_seq_len > 0 ? (int)ceil_div64(max_seq_len, partition_size) : 1;
-    if ((int64_t)num_seqs * np > 0x7FFFFFFF) return PA_ERR_UNSUPPORTED;
 
     pa::DecodeParams p = make_decode_params(a, dev_err);
     const size_t rows = (size_t)num_seqs * num_q_heads * np;

@@ -222,7 +222,9 @@ __global__ void __launch_bounds__(kDecodeWarps * 32)
     };
 
     const int npre = nk < NST ? nk : NST;
-    for (int k = 0; k < npre; ++k) issue(k);
+    const int first_issued = p.hold_first_tile ? 1 : 0;  // test hook: tile 0 never issued
+    for (int k = first_issued; k < npre; ++k) issue(k);
+    const uint64_t wait_limit = p.wait_limit_ns ? p.wait_limit_ns : kWaitLimitNs;
 
     // ---- main loop over this warp's blocks --------------------------------
     float m_run = -CUDART_INF_F, l_run = 0.f;
@@ -243,7 +245,7 @@ __global__ void __launch_bounds__(kDecodeWarps * 32)
             bt_nxt = nk > (cur_batch + 1) * 32 ? load_batch(cur_batch + 1) : 0;
         }
         const int st = k % NST;
-        const bool ok = __all_sync(kFull, mbar_wait_bounded(bar0 + 8 * st, (k / NST) & 1, kWaitLimitNs));
+        const bool ok = __all_sync(kFull, mbar_wait_bounded(bar0 + 8 * st, (k / NST) & 1, wait_limit));
         if (!ok) {
             if (lane == 0) flag_error(p.err, kErrTimeout);
             timed_out = true;
@@ -353,7 +355,7 @@ __global__ void __launch_bounds__(kDecodeWarps * 32)
     if (timed_out) {
         // let copies still in flight land before the buffers are reused
         if (lane == 0) {
-            for (int kk = k; kk < nk && kk < k + NST; ++kk)
+            for (int kk = k > first_issued ? k : first_issued; kk < nk && kk < k + NST; ++kk)
                 (void)mbar_wait_bounded(bar0 + 8 * (kk % NST), (kk / NST) & 1, kWaitLimitNs / 16);
         }
         __syncwarp();

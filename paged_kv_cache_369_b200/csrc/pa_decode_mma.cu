@@ -291,7 +291,9 @@ __global__ void __launch_bounds__(NWARPS * 32, MmaCfg<QT, KVT, D, GT, NWARPS>::M
         }
     };
     const int npre = nk < NST ? nk : NST;
-    for (int k = 0; k < npre; ++k) issue(k);
+    const int first_issued = p.hold_first_tile ? 1 : 0;  // test hook: tile 0 never issued
+    for (int k = first_issued; k < npre; ++k) issue(k);
+    const uint64_t wait_limit = p.wait_limit_ns ? p.wait_limit_ns : kWaitLimitNs;
 
     // ---- q as MMA A fragments (rows = heads of this group) ----------------
     // a[ks][0]: row g, a[ks][1]: row g+8, a[ks][2]: row g (k+8), a[ks][3]: row g+8 (k+8)
@@ -402,7 +404,7 @@ __global__ void __launch_bounds__(NWARPS * 32, MmaCfg<QT, KVT, D, GT, NWARPS>::M
             bt_nxt = nk > (cur_batch + 1) * 32 ? load_batch(cur_batch + 1) : 0;
         }
         const int st = k % NST;
-        const bool ok = __all_sync(kFull, mbar_wait_bounded(bar0 + 8 * st, (k / NST) & 1, kWaitLimitNs));
+        const bool ok = __all_sync(kFull, mbar_wait_bounded(bar0 + 8 * st, (k / NST) & 1, wait_limit));
         if (!ok) {
             if (lane == 0) flag_error(p.err, kErrTimeout);
             timed_out = true;
@@ -593,7 +595,7 @@ __global__ void __launch_bounds__(NWARPS * 32, MmaCfg<QT, KVT, D, GT, NWARPS>::M
 
     if (timed_out) {
         if (lane == 0) {
-            for (int kk = k; kk < nk && kk < k + NST; ++kk)
+            for (int kk = k > first_issued ? k : first_issued; kk < nk && kk < k + NST; ++kk)
                 (void)mbar_wait_bounded(bar0 + 8 * (kk % NST), (kk / NST) & 1, kWaitLimitNs / 16);
         }
         __syncwarp();
@@ -676,17 +678,17 @@ __global__ void __launch_bounds__(NWARPS * 32, MmaCfg<QT, KVT, D, GT, NWARPS>::M
 // ---------------------------------------------------------------------------
 
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-    static bool tried = false;
-    if (!tried) {
-        tried = true;
+    // looked up once; a function-local static is initialised exactly once
+    // even when several host threads make their first call together
+    static const PFN_cuTensorMapEncodeTiled_v12000 fn = []() -> PFN_cuTensorMapEncodeTiled_v12000 {
         void *f = nullptr;
         cudaDriverEntryPointQueryResult q;
         if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) ==
                 cudaSuccess &&
             q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
-    }
+            return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+        return nullptr;
+    }();
     return fn;
 }
 

@@ -98,6 +98,14 @@ struct DecodeParams {
     uint8_t *v_pool_w;
     float k_scale_w;            // E4M3 quantisation scales (1 for 16-bit caches)
     float v_scale_w;
+    // failure-detection test hook, never set through the public ABI (the C
+    // shim reads it from the environment variable PA369_TEST_DECODE_STALL_NS):
+    // the main loop's copy waits give up after wait_limit_ns (0: kWaitLimitNs),
+    // and with hold_first_tile every warp leaves its first tile's copies
+    // unissued, so that the first wait can only run out.  The drain of the
+    // copies that were issued keeps its own bound.
+    uint64_t wait_limit_ns;
+    int hold_first_tile;
 };
 
 struct AppendParams {  // decode-form slot mapping + cache write in one kernel
@@ -176,6 +184,16 @@ struct ReduceParams {
     int extra;
     int token_begin;
 };
+
+// Host-side argument checks of pa_decode_split_reduce, the workspace aside;
+// touches no GPU.  Returns PA_OK (0) or the pa_status the call would return
+// before any launch.  q_dtype / kv_dtype are pa_dtype values.
+int check_split_reduce_args(const void *out, const void *q, const void *k_cache,
+                            const void *v_cache, const int32_t *block_tables,
+                            int max_blocks_per_seq, const int32_t *seq_lens, int num_seqs,
+                            int num_q_heads, int num_kv_heads, int head_dim, int block_size,
+                            int num_blocks, float softmax_scale, int q_dtype, int kv_dtype,
+                            float k_scale, float v_scale, int partition_size, int max_seq_len);
 
 // Launchers: return cudaSuccess or the launch error.
 cudaError_t launch_slot_mapping(const SlotParams &p, cudaStream_t stream);

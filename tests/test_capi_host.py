@@ -128,6 +128,31 @@ def test_split_checks(pa):
     assert big == 256 + 2 * 64 * 4
 
 
+def test_static_scratch_checks_arguments_before_the_device(pa):
+    """The allocation-free split entry point returns the argument errors of
+    pa_decode_split_reduce without touching the GPU (none here), so they never
+    turn into PA_ERR_CUDA."""
+    L = pa.lib()
+
+    def call(S=2, Hq=8, Hk=2, d=128, P=512, maxlen=1000, scale=0.1, kvd=None, out=A):
+        return L.pa_decode_split_reduce_static_scratch(
+            out, A, A, A, A, 4, A, S, Hq, Hk, d, 16, 10, scale, pa.PA_BF16,
+            pa.PA_BF16 if kvd is None else kvd, 1.0, 1.0, P, maxlen, None, None)
+
+    assert call(Hq=0) == 1
+    assert call(Hq=6, Hk=4) == 1      # not a whole GQA group
+    assert call(P=0) == 1
+    assert call(P=24) == 1
+    assert call(maxlen=-1) == 1
+    assert call(scale=float("nan")) == 1
+    assert call(out=A + 8) == 1       # misaligned
+    assert call(d=96) == 2            # unsupported head_dim
+    assert call(kvd=pa.PA_F16) == 2   # 16-bit cache of another dtype
+    assert call(S=0) == 0             # empty batch: nothing to do, no device needed
+    # too large for the built-in array (checked before the device as well)
+    assert call(S=1024, Hq=64, Hk=8, maxlen=32768) == 1
+
+
 def test_cache_write_and_slot_checks(pa):
     L = pa.lib()
     cw = lambda **k: L.pa_cache_write(k.get("kn", A), A, k.get("kc", A), A, k.get("sm", A),

@@ -3,34 +3,29 @@
 pa_decode_split_reduce_static_scratch serves callers that cannot allocate
 device memory (no allocator handed to them, HBM already reserved for the KV
 pool, or no room for cudaMalloc's synchronisation on their path): its partials
-live in a device array inside the library.  This test calls it through the C
-ABI twice in a row and checks both outputs against pa_decode_split_reduce with
-a caller-provided workspace, within the parity tolerance the other tests use.
-It sits in its own file, collected last, and must pass alone in a fresh
-process as well as after every other test (the first call on a device does the
-one-time address lookup)."""
-
-import ctypes
+live in a device array inside the library.  It runs the same partition and
+reduce kernels as pa_decode_split_reduce on the same partitions, only with
+another scratch address, so its output must equal that entry point's bit for
+bit.  This test calls it through the C ABI twice in a row per workload,
+checks both outputs for bit equality with pa_decode_split_reduce given a
+caller-allocated workspace, and checks the tiny workload against the oracle
+within the parity tolerance (max-abs 1e-2, relative L2 2e-3).  One case runs a
+large workload and then a small one in the same process: the small call must
+not pick up partials the large one left in the shared array.  The file is
+collected last and must pass alone in a fresh process as well as after every
+other test (the first call in a context does the one-time address lookup)."""
 
 import numpy as np
 import pytest
 import torch
 
+import oracle
 import workload
 
 pytestmark = pytest.mark.gpu
 
 MAX_ABS = 1e-2
 REL_L2 = 2e-3
-
-
-def _close(got: torch.Tensor, ref: torch.Tensor):
-    g = got.float().cpu().numpy().astype(np.float64)
-    r = ref.float().cpu().numpy().astype(np.float64)
-    assert np.isfinite(g).all()
-    max_abs = float(np.abs(g - r).max())
-    rel = float(np.linalg.norm(g - r) / max(np.linalg.norm(r), 1e-30))
-    assert max_abs <= MAX_ABS and rel <= REL_L2, (max_abs, rel)
 
 
 def _call_static(pa, dec, out, P):
@@ -44,18 +39,19 @@ def _call_static(pa, dec, out, P):
         torch.cuda.current_stream().cuda_stream)
 
 
-@pytest.mark.parametrize("cfg", [1, 2, 4])
-def test_static_scratch_matches_workspace_entry_point(cfg):
-    import paged_kv_cache_369_b200 as pa
+def _decoder(cfg, P):
+    """A workload resident on the GPU with its new tokens written and its
+    output computed by pa_decode_split_reduce with a torch-allocated workspace."""
     from paged_kv_cache_369_b200.runner import PagedDecode
 
-    w = workload.config(cfg)
-    P = 512
-    dec = PagedDecode(w, mode="split", partition_size=P)
-    dec.step()  # cache write + pa_decode_split_reduce with a torch-allocated workspace
+    dec = PagedDecode(workload.config(cfg), mode="split", partition_size=P)
+    dec.step()
     torch.cuda.synchronize()
     assert dec.error() == 0
-    ref = dec.out.clone()
+    return dec, dec.out.clone()
+
+
+def _static_twice(pa, dec, ref, P):
     out = torch.empty_like(ref)
     for _ in range(2):  # two calls in a row share (and reuse) the library's array
         out.fill_(float("nan"))
@@ -63,7 +59,38 @@ def test_static_scratch_matches_workspace_entry_point(cfg):
         torch.cuda.synchronize()
         assert status == pa.PA_OK, pa.pa_status_string(status)
         assert dec.error() == 0
-        _close(out, ref)
+        assert torch.equal(out.view(torch.int16), ref.view(torch.int16))
+    return out
+
+
+@pytest.mark.parametrize("cfg", [1, 2, 4])
+def test_static_scratch_matches_workspace_entry_point(cfg):
+    import paged_kv_cache_369_b200 as pa
+
+    P = 512
+    dec, ref = _decoder(cfg, P)
+    out = _static_twice(pa, dec, ref, P)
+    if cfg == 1:  # small enough to compare every output with the oracle
+        kc, vc = oracle.caches_for(dec.w)
+        want = oracle.decode_for(dec.w, kc, vc)
+        got = out.float().cpu().numpy().astype(np.float64)
+        max_abs = float(np.abs(got - want).max())
+        rel = float(np.linalg.norm(got - want) / np.linalg.norm(want))
+        assert max_abs <= MAX_ABS and rel <= REL_L2, (max_abs, rel)
+
+
+def test_static_scratch_small_call_after_a_large_one():
+    """Config 4 (long contexts, 64 partitions a row) fills most of the array;
+    config 1 then reuses its start.  Both must equal the workspace entry point
+    bit for bit, the second one included."""
+    import paged_kv_cache_369_b200 as pa
+
+    P = 512
+    big, big_ref = _decoder(4, P)
+    small, small_ref = _decoder(1, P)
+    _static_twice(pa, big, big_ref, P)
+    _static_twice(pa, small, small_ref, P)
+    _static_twice(pa, big, big_ref, P)
 
 
 def test_static_scratch_rejects_sizes_beyond_its_array():
