@@ -505,6 +505,193 @@ def run_prefill(args):
 # the CUDA path
 # ---------------------------------------------------------------------------
 
+def time_device_steps(dec, stream, steps: int, fused: bool, flush=None):
+    """Event-timed decode steps on `stream` with inputs resident in HBM.
+    Returns (step ms without the L2 flushes, attention ms, cache-write ms)
+    averaged over the steps.  The caller has warmed up and synchronised."""
+    import torch
+
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+    flush_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(steps)] \
+        if flush is not None else None
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        t_start.record(stream)
+        for i in range(steps):
+            e0, e1, e2 = ev[i]
+            e0.record(stream)
+            if fused:
+                e1.record(stream)
+                dec.step()  # one call: new tokens stored by the attention launch
+            else:
+                dec.write_new()
+                e1.record(stream)
+                dec.attend()
+            e2.record(stream)
+            if flush is not None:
+                flush_ev[i][0].record(stream)
+                flush.fill_(1)
+                flush_ev[i][1].record(stream)
+        t_end.record(stream)
+    t_end.synchronize()
+    total_ms = t_start.elapsed_time(t_end)
+    flush_ms = sum(a.elapsed_time(b) for a, b in flush_ev) if flush_ev else 0.0
+    step_ms = (total_ms - flush_ms) / steps
+    attn_ms = statistics.mean(e1.elapsed_time(e2) for _, e1, e2 in ev)
+    write_ms = statistics.mean(e0.elapsed_time(e1) for e0, e1, _ in ev)
+    return step_ms, attn_ms, write_ms
+
+
+def time_graph_steps(dec, stream, steps: int, flush=None, barrier=None):
+    """`steps` decode steps captured back to back in one CUDA graph (no
+    events between them, so a step's first launch overlaps the previous
+    step's last through programmatic dependent launch, and no host launch
+    overhead), replayed once untimed and then once between two events on
+    `stream`, with `barrier` (a rank barrier + device synchronise) on both
+    sides of the timed replay.  With an L2 flush after every step, the
+    flushes are timed in a graph of their own and subtracted.  Returns ms per
+    step."""
+    import torch
+
+    def timed(body):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream, capture_error_mode="relaxed"):
+            body()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            g.replay()  # the first replay uploads the graph; not timed
+        if barrier is not None:
+            barrier()
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            g.replay()
+            e1.record(stream)
+        if barrier is not None:
+            barrier()
+        e1.synchronize()
+        ms = e0.elapsed_time(e1)
+        del g
+        return ms
+
+    def steps_body():
+        for _ in range(steps):
+            dec.step()
+            if flush is not None:
+                flush.fill_(1)
+
+    total = timed(steps_body)
+    if flush is not None:
+        def flush_body():
+            for _ in range(steps):
+                flush.fill_(1)
+        total -= timed(flush_body)
+    return total / steps
+
+
+E2E_INPUTS = ("q", "k_new", "v_new", "block_tables", "seq_lens")
+
+
+def time_end_to_end(dec, stream, device, steps: int, flush=None):
+    """Decode steps end to end: every step copies its inputs (q, the new K/V
+    rows, block tables, lengths) from pinned host memory and reads its output
+    back into pinned host memory.  The copies of step i + 1's inputs and of
+    step i - 1's output run on two copy streams while step i attends: inputs
+    and outputs are double-buffered on the device, and events order each
+    buffer's copy-in -> step -> copy-out -> reuse.  Returns (ms per step from
+    the first input copy to the last output copy, H2D bytes per step, D2H
+    bytes per step)."""
+    import torch
+
+    host = {n: getattr(dec, n).cpu().pin_memory() for n in E2E_INPUTS}
+    keep = {n: getattr(dec, n) for n in E2E_INPUTS + ("out",)}
+    bufs = [dict(keep), {n: torch.empty_like(t) for n, t in keep.items()}]
+    host_out = [torch.empty_like(dec.out, device="cpu").pin_memory() for _ in range(2)]
+    h2d_bytes = sum(t.numel() * t.element_size() for t in host.values())
+    d2h_bytes = host_out[0].numel() * host_out[0].element_size()
+    h2d_s, d2h_s = torch.cuda.Stream(device), torch.cuda.Stream(device)
+    ev_in = [torch.cuda.Event() for _ in range(2)]    # inputs of buffer b landed
+    ev_done = [torch.cuda.Event() for _ in range(2)]  # step on buffer b finished
+    ev_out = [torch.cuda.Event() for _ in range(2)]   # output of buffer b read back
+    e_s = torch.cuda.Event(enable_timing=True)
+    e_e = torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize(device)
+    e_s.record(h2d_s)
+    for i in range(steps):
+        b = i & 1
+        buf = bufs[b]
+        if i >= 2:
+            h2d_s.wait_event(ev_done[b])  # step i - 2 no longer reads these inputs
+        with torch.cuda.stream(h2d_s):
+            for n in E2E_INPUTS:
+                buf[n].copy_(host[n], non_blocking=True)
+        ev_in[b].record(h2d_s)
+        stream.wait_event(ev_in[b])
+        if i >= 2:
+            stream.wait_event(ev_out[b])  # step i - 2's output has been read back
+        for n, t in buf.items():
+            setattr(dec, n, t)
+        with torch.cuda.stream(stream):
+            dec.step()
+            ev_done[b].record(stream)
+            if flush is not None:
+                flush.fill_(1)
+        d2h_s.wait_event(ev_done[b])
+        with torch.cuda.stream(d2h_s):
+            host_out[b].copy_(buf["out"], non_blocking=True)
+        ev_out[b].record(d2h_s)
+    e_e.record(d2h_s)
+    torch.cuda.synchronize(device)
+    for n, t in keep.items():
+        setattr(dec, n, t)
+    return e_s.elapsed_time(e_e) / steps, h2d_bytes, d2h_bytes
+
+
+def per_config_measurements(device, stream, steps: int, warmup: int):
+    """Attention time, roofline fraction and clocks of the other named decode
+    workloads, each in its default launch configuration: configs 3 and 4 as a
+    fused step (1024- / 512-token partitions), config 5 with its shared prefix
+    attended once (cascade).  Each is timed like the headline, on its own."""
+    import torch
+
+    import workload
+    from paged_kv_cache_369_b200.runner import (PagedDecode, algorithmic_cascade_bytes,
+                                                default_partition_size)
+
+    peak, _ = measured_hbm_peak()
+    res = {}
+    for cfg, mode in ((3, "fused"), (4, "fused"), (5, "cascade")):
+        w = workload.config(cfg)
+        P = default_partition_size(w, cfg)
+        with torch.cuda.stream(stream):
+            dec = PagedDecode(w, device=str(device), mode=mode, partition_size=P, stream=stream)
+            for _ in range(warmup):
+                dec.step()
+        torch.cuda.synchronize(device)
+        dec.dev_err.zero_()
+        fused = mode.startswith("fused")
+        attn_bytes = w.step_bytes() if fused else algorithmic_cascade_bytes(w)
+        clocks = ClockSampler(device.index if device.index is not None else 0)
+        clocks.start()
+        step_ms = time_graph_steps(dec, stream, steps)
+        clocks.stop()
+        _, ev_attn_ms, write_ms = time_device_steps(dec, stream, steps, fused)
+        attn_ms = step_ms if fused else ev_attn_ms
+        achieved = attn_bytes / (attn_ms * 1e-3) / 1e9
+        res[f"config{cfg}"] = {
+            "workload": w.name, "mode": mode, "partition_size": P, "steps": steps,
+            "us_per_step": step_ms * 1e3, "attention_us": attn_ms * 1e3,
+            "cache_write_us": None if fused else write_ms * 1e3,
+            "algorithmic_bytes_per_launch": attn_bytes, "achieved_gbs": achieved,
+            "frac": achieved / peak, "tokens_per_s": w.num_seqs / (step_ms * 1e-3),
+            "gpu_launches": steps * dec.launches_per_step(), "clocks": clocks.summary(),
+            "traffic": recorded_traffic(cfg, mode), "device_error": dec.error(),
+        }
+        del dec
+        torch.cuda.empty_cache()
+    return res
+
 def run_ours(args):
     import torch
     import torch.distributed as dist
@@ -552,72 +739,30 @@ def run_ours(args):
                 flush.fill_(1)
     barrier()
     dec.dev_err.zero_()
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
-    flush_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)] \
-        if flush is not None else None
     clocks = ClockSampler(device.index if device.index is not None else 0)
     clocks.start()
-    barrier()
-    t_start = torch.cuda.Event(enable_timing=True)
-    t_end = torch.cuda.Event(enable_timing=True)
-    with torch.cuda.stream(stream):
-        t_start.record(stream)
-        for i in range(args.steps):
-            e0, e1, e2 = ev[i]
-            e0.record(stream)
-            if fused:
-                e1.record(stream)
-                dec.step()  # one call: new tokens stored by the attention launch
-            else:
-                dec.write_new()
-                e1.record(stream)
-                dec.attend()
-            e2.record(stream)
-            if flush is not None:
-                flush_ev[i][0].record(stream)
-                flush.fill_(1)
-                flush_ev[i][1].record(stream)
-        t_end.record(stream)
-    barrier()
+    step_ms_local = time_graph_steps(dec, stream, args.steps, flush, barrier)
     clocks.stop()
-    total_ms = t_start.elapsed_time(t_end)
-    flush_ms = sum(a.elapsed_time(b) for a, b in flush_ev) if flush_ev else 0.0
-    step_ms_local = (total_ms - flush_ms) / args.steps
-    attn_ms = statistics.mean(e1.elapsed_time(e2) for _, e1, e2 in ev)
-    write_ms = statistics.mean(e0.elapsed_time(e1) for e0, e1, _ in ev)
+    # the same steps issued one by one, each bracketed by events: the split of a
+    # step into cache write and attention, and the cost of per-step launches
+    barrier()
+    ev_step_ms_local, ev_attn_ms, write_ms = time_device_steps(dec, stream, args.steps, fused, flush)
+    barrier()
     err = dec.error()
     step_ms = max_over_ranks(step_ms_local, device)
+    # attention time per step: the whole graph-timed step where the step is
+    # the attention launches alone (a fused step stores the new tokens inside
+    # them); else the event-timed attention launches
+    attn_ms = step_ms_local if fused else ev_attn_ms
     total_bytes = sum_over_ranks(float(step_bytes), device)
     value = total_bytes / (step_ms * 1e-3) / 1e9
 
     # ---- end to end: pinned host inputs in, output out, every step --------
-    host_q = dec.q.cpu().pin_memory()
-    host_kn = dec.k_new.cpu().pin_memory()
-    host_vn = dec.v_new.cpu().pin_memory()
-    host_bt = dec.block_tables.cpu().pin_memory()
-    host_sl = dec.seq_lens.cpu().pin_memory()
-    host_out = torch.empty_like(dec.out, device="cpu").pin_memory()
-    h2d = sum(t.numel() * t.element_size() for t in (host_q, host_kn, host_vn, host_bt, host_sl))
-    d2h = host_out.numel() * host_out.element_size()
     e2e_steps = max(1, min(args.steps, 200))
     barrier()
-    e_s = torch.cuda.Event(enable_timing=True)
-    e_e = torch.cuda.Event(enable_timing=True)
-    with torch.cuda.stream(stream):
-        e_s.record(stream)
-        for _ in range(e2e_steps):
-            dec.q.copy_(host_q, non_blocking=True)
-            dec.k_new.copy_(host_kn, non_blocking=True)
-            dec.v_new.copy_(host_vn, non_blocking=True)
-            dec.block_tables.copy_(host_bt, non_blocking=True)
-            dec.seq_lens.copy_(host_sl, non_blocking=True)
-            dec.step()
-            host_out.copy_(dec.out, non_blocking=True)
-            if flush is not None:
-                flush.fill_(1)
-        e_e.record(stream)
+    e2e_ms_local, h2d, d2h = time_end_to_end(dec, stream, device, e2e_steps, flush)
     barrier()
-    e2e_ms = max_over_ranks(e_s.elapsed_time(e_e) / e2e_steps, device)
+    e2e_ms = max_over_ranks(e2e_ms_local, device)
     e2e_value = total_bytes / (e2e_ms * 1e-3) / 1e9
     copy_gbs = same_run_copy_gbs(device, stream)
 
@@ -638,6 +783,11 @@ def run_ours(args):
             "tokens_per_s": world * w.num_seqs / (step_ms * 1e-3),
             "attention_us": attn_ms * 1e3,
             "cache_write_us": None if fused else write_ms * 1e3,
+            "timing": "the K timed steps run as one CUDA graph (captured launches, programmatic "
+                      "dependent launch between them) between two events on the launch stream",
+            "event_timed": {"us_per_step": ev_step_ms_local * 1e3, "attention_us": ev_attn_ms * 1e3,
+                            "note": "the same K steps launched one by one from Python with events "
+                                    "around every step's launches"},
             "kv_bytes_per_step": w.kv_bytes_logical(),
             "step_bytes": step_bytes,
             "roofline": {
@@ -657,7 +807,10 @@ def run_ours(args):
                 "frac_of_spec": achieved / SPEC_HBM_GBS,
             },
             "e2e": {"value": e2e_value, "unit": "GB/s", "h2d_bytes_per_step": h2d,
-                    "d2h_bytes_per_step": d2h, "steps": e2e_steps},
+                    "d2h_bytes_per_step": d2h, "steps": e2e_steps, "ms_per_step": e2e_ms,
+                    "copies": "every step: its inputs H2D from pinned memory and its output "
+                              "D2H, on two copy streams overlapping the neighbouring steps' "
+                              "kernels (double-buffered)"},
             "gpu_launches": args.steps * dec.launches_per_step(),
             "clocks": clocks.summary(),
             "device_error": err,
@@ -666,6 +819,12 @@ def run_ours(args):
         dist.barrier()
         dist.destroy_process_group()
     if rank == 0:
+        if world == 1 and not args.no_per_config and args.config == 2 and args.mode == "fused" \
+                and args.kv is None:
+            del dec
+            torch.cuda.empty_cache()
+            result["per_config"] = per_config_measurements(device, stream, args.per_config_steps,
+                                                           min(args.warmup, 10))
         if world == 1 and not args.no_cpu_baseline:
             result["cpu_baseline"] = cpu_baseline(w, budget_s=args.cpu_budget)
         print(json.dumps(result), flush=True)
@@ -687,6 +846,10 @@ def main(argv=None):
                          "prescribes, else 1024)")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-per-config", action="store_true",
+                    help="skip timing the other named workloads (configs 3, 4, 5) after the "
+                         "headline line's own measurement")
+    ap.add_argument("--per-config-steps", type=int, default=300)
     ap.add_argument("--op", choices=("decode", "copy_blocks", "prefill"), default="decode",
                     help="decode: the decode step (default); copy_blocks: pa_copy_blocks alone; "
                          "prefill: a chunked-prefill step")

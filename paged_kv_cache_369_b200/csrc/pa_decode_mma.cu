@@ -78,6 +78,32 @@ __device__ __forceinline__ void mma16816(float *c, const uint32_t *a, uint32_t b
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
+// m16n8k32 with A and B in the 8-bit cache format (fp32 accumulate; INT8:
+// s32 accumulate, exact)
+__device__ __forceinline__ void mma_k32(float *c, const uint32_t *a, uint32_t b0, uint32_t b1,
+                                        e4m3_t) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k32.row.col.f32.e4m3.e4m3.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+        "{%8,%9}, {%0,%1,%2,%3};"
+        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ void mma_k32(float *c, const uint32_t *a, uint32_t b0, uint32_t b1,
+                                        e5m2_t) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k32.row.col.f32.e5m2.e5m2.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+        "{%8,%9}, {%0,%1,%2,%3};"
+        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ void mma_k32(int *c, const uint32_t *a, uint32_t b0, uint32_t b1, i8_t) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+        "{%8,%9}, {%0,%1,%2,%3};"
+        : "+r"(c[0]), "+r"(c[1]), "+r"(c[2]), "+r"(c[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
 __device__ __forceinline__ void ldsm_x4(uint32_t *r, uint32_t addr) {
     asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
                  : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
@@ -136,18 +162,29 @@ __device__ __forceinline__ uint32_t pack2(float lo, float hi, bf16_t) {
     return r;
 }
 
+// 2^x on the MUFU unit (-inf -> +0; results below 2^-126 flush to 0, which
+// only drops weights too small to matter next to the row maximum's 1)
+__device__ __forceinline__ float ex2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
 __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t sel) {
     uint32_t r;
     asm("prmt.b32 %0, %1, 0, %2;" : "=r"(r) : "r"(a), "r"(sel));
     return r;
 }
 
+// a tensor-map tile copy with an L2 eviction-priority policy (createpolicy):
+// the K/V stream is read once, so it goes first when L2 needs room, and the
+// split partials the reduce reads back stay resident
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, int x, int y,
-                                            uint32_t bar) {
+                                            uint32_t bar, uint64_t policy) {
     asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, "
-        "{%2, %3}], [%4];" ::"r"(dst),
-        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint "
+        "[%0], [%1, {%2, %3}], [%4], %5;" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar), "l"(policy)
         : "memory");
 }
 
@@ -175,7 +212,25 @@ template <typename QT, typename KVT, int D, int GT, int NW_ = kDecodeWarps> stru
     static constexpr bool WIDE = FP8 && GT == 8;
     static constexpr int NST = WIDE ? 3 : ((16384 / STAGE_BYTES) < 2 ? 2 : (16384 / STAGE_BYTES));
     static constexpr int MIN_CTAS = (WIDE ? 16 : 12) / NW_;
-    static constexpr int KS = D / 16;   // k-steps of q.K
+    static constexpr int KS = D / 16;   // k-steps of q.K (16-bit: m16n8k16; 8-bit: pairs of them
+                                        // make one m16n8k32 step)
+    // 8-bit caches: q.K runs in the cache's format with q split into QT8
+    // terms (term t scaled by 2^(QSH t)); the largest |q| is put at 2^QB
+    static constexpr bool INT8 = std::is_same<KVT, i8_t>::value;
+    static constexpr bool E5M2 = std::is_same<KVT, e5m2_t>::value;
+    static constexpr int QT8 = INT8 ? 2 : ((E5M2 || std::is_same<QT, f16_t>::value) ? 3 : 2);
+    static constexpr int QSH = INT8 ? 7 : (E5M2 ? 3 : 4);
+    static constexpr int QB = INT8 ? 5 : (E5M2 ? 14 : 7);
+    // with 8 MMA rows for 8 heads, A rows 8-15 carry the next q term (rows
+    // 0-7 term 2m, rows 8-15 term 2m+1 of MMA m), so the rows the GQA group
+    // leaves empty do useful work; 16 heads need one MMA per term
+    static constexpr bool PACK8 = GT == 8;
+    // the 8-bit q.K path where two terms suffice (E4M3 against a bf16 q,
+    // INT8 against either) and pack into one MMA (groups of up to 8 heads);
+    // three-term cases (E5M2, E4M3 against an f16 q) and 16-row groups would
+    // run out of registers and keep widening K to f16
+    static constexpr bool K8MMA = FP8 && QT8 == 2 && PACK8;
+    static constexpr int NA8 = PACK8 ? (QT8 + 1) / 2 : QT8;  // A-operand sets (MMAs per k32 step)
     static constexpr int MT = D / 16;   // m-tiles (16 rows of d) of O^T = V^T P^T
     static constexpr int NH = GT / 8;   // n-tiles (8 heads) of O^T
     static constexpr int SZ_STAGES = NW * NST * STAGE_BYTES;
@@ -262,6 +317,7 @@ __global__ void __launch_bounds__(NWARPS * 32, MmaCfg<QT, KVT, D, GT, NWARPS>::M
         return k < nk ? bt_row[(blk_begin + warp + NW * k) >> p.tile_shift] : 0;
     };
     const int tile_mask = (1 << p.tile_shift) - 1;
+    const uint64_t kv_policy = policy_evict_first();
     int cur_batch = 0;
     int bt_cur = load_batch(0);
     int bt_nxt = nk > 32 ? load_batch(1) : 0;
@@ -270,14 +326,13 @@ __global__ void __launch_bounds__(NWARPS * 32, MmaCfg<QT, KVT, D, GT, NWARPS>::M
         const int b = __shfl_sync(kFull, bt_nxt, k & 31);
         return (k >> 5) == cur_batch ? a : b;
     };
-    auto issue = [&](int k) {  // whole warp calls; lane 0 issues the copies
+    auto issue = [&](int k, int st) {  // whole warp calls; lane 0 issues the copies; st = k % NST
         int phys = bt_of(k);
         if (lane == 0) {
             if ((unsigned)phys >= (unsigned)p.num_blocks) {
                 flag_error(p.err, kErrBounds);
                 phys = 0;  // a valid block whose tokens are all masked
             }
-            const int st = k % NST;
             const uint32_t bar = bar0 + 8 * st;
             const uint32_t dst = stage0 + st * C::STAGE_BYTES;
             const int sub = (blk_begin + warp + NW * k) & tile_mask;  // tile within the block
@@ -285,19 +340,23 @@ __global__ void __launch_bounds__(NWARPS * 32, MmaCfg<QT, KVT, D, GT, NWARPS>::M
             mbar_arrive_expect_tx(bar, C::STAGE_BYTES);
 #pragma unroll
             for (int b = 0; b < C::NBOX; ++b) {
-                tma_load_2d(dst + b * C::BOX_BYTES, &tmap_k, b * C::BOX_ELEMS, y, bar);
-                tma_load_2d(dst + C::TILE_BYTES + b * C::BOX_BYTES, &tmap_v, b * C::BOX_ELEMS, y, bar);
+                tma_load_2d(dst + b * C::BOX_BYTES, &tmap_k, b * C::BOX_ELEMS, y, bar, kv_policy);
+                tma_load_2d(dst + C::TILE_BYTES + b * C::BOX_BYTES, &tmap_v, b * C::BOX_ELEMS, y, bar,
+                            kv_policy);
             }
         }
     };
     const int npre = nk < NST ? nk : NST;
     const int first_issued = p.hold_first_tile ? 1 : 0;  // test hook: tile 0 never issued
-    for (int k = first_issued; k < npre; ++k) issue(k);
+    for (int k = first_issued; k < npre; ++k) issue(k, k);
     const uint64_t wait_limit = p.wait_limit_ns ? p.wait_limit_ns : kWaitLimitNs;
 
     // ---- q as MMA A fragments (rows = heads of this group) ----------------
-    // a[ks][0]: row g, a[ks][1]: row g+8, a[ks][2]: row g (k+8), a[ks][3]: row g+8 (k+8)
-    uint32_t qa[C::KS][4];
+    // 16-bit caches, k-step ks: qa[ks][0]: row g, [1]: row g+8, [2]: row g (k+8),
+    // [3]: row g+8 (k+8).  8-bit caches, k32-step jj, term t: q8[t][jj][0]: row g
+    // codes k 4kq..4kq+3, [1]: row g+8, [2] / [3]: the same at k + 16.
+    uint32_t qa[C::K8MMA ? 1 : C::KS][4];
+    uint32_t q8[C::K8MMA ? C::NA8 : 1][C::K8MMA ? C::KS / 2 : 1][4];
     float qscale = p.qk_scale_log2;
     {
         const int group_base = hg * GT;
@@ -332,11 +391,11 @@ __global__ void __launch_bounds__(NWARPS * 32, MmaCfg<QT, KVT, D, GT, NWARPS>::M
                 qv[hh][ks][0] = v0; qv[hh][ks][1] = v1; qv[hh][ks][2] = v2; qv[hh][ks][3] = v3;
             }
         }
-        if constexpr (!std::is_same<QT, ET>::value || CHAN) {
-            // bf16 q against an f16 tensor-core path (8-bit cache), or q times
-            // per-channel scales: scale q by a power of two so its largest
-            // element sits near 2^14, convert to f16, and fold the inverse
-            // power into the logit scale (exact).
+        if constexpr (C::FP8 || CHAN) {
+            // 8-bit caches (and q times per-channel scales): scale q by a power
+            // of two so its largest element sits at 2^QB (8-bit q.K: then split
+            // into terms of the cache's format) or at 2^14 (converted to f16),
+            // and fold the inverse power into the logit scale (exact).
             float amax = 0.f;
 #pragma unroll
             for (int hh = 0; hh < 2; ++hh)
@@ -349,7 +408,7 @@ __global__ void __launch_bounds__(NWARPS * 32, MmaCfg<QT, KVT, D, GT, NWARPS>::M
             int e = 0;
             if (amax > 0.f) {
                 const int ex = (int)((__float_as_uint(amax) >> 23) & 0xFF) - 127;  // floor(log2)
-                e = 14 - ex;
+                e = (C::K8MMA ? C::QB : 14) - ex;
                 if (e > 100) e = 100;
                 if (e < -100) e = -100;
             }
@@ -362,8 +421,53 @@ __global__ void __launch_bounds__(NWARPS * 32, MmaCfg<QT, KVT, D, GT, NWARPS>::M
 #pragma unroll
                     for (int i = 0; i < 4; ++i) qv[hh][ks][i] *= up;
         }
+        if constexpr (C::K8MMA) {
+            // term t: the codes of the remainder left by the terms before it,
+            // times 2^(QSH t): q 2^e = sum_t code_t 2^(-QSH t).  Two terms hold a
+            // bf16 q exactly against E4M3 (4 + 4 significant bits) or INT8
+            // (integer part + 7 bits); three hold an f16 q, or q against E5M2
+            // (3 bits a term).  Elements below 2^(QB - 20) of the largest may
+            // lose low bits, an error far below the logits' fp32 rounding.
+            constexpr float kUp = (float)(1 << C::QSH);
 #pragma unroll
-        for (int ks = 0; ks < C::KS; ++ks) {
+            for (int a = 0; a < C::NA8; ++a)
+#pragma unroll
+                for (int jj = 0; jj < C::KS / 2; ++jj)
+#pragma unroll
+                    for (int r = 0; r < 4; ++r) q8[a][jj][r] = 0u;
+#pragma unroll
+            for (int t = 0; t < C::QT8; ++t) {
+#pragma unroll
+                for (int jj = 0; jj < C::KS / 2; ++jj) {
+#pragma unroll
+                    for (int r = 0; r < (C::PACK8 ? 4 : 4); ++r) {
+                        // PACK8: rows g only (hh 0), term t in MMA t / 2, rows
+                        // g (t even) or g + 8 (t odd); else row g + 8 * hh
+                        if (C::PACK8 && (r & 1)) continue;
+                        const int hh = r & 1, ks = 2 * jj + (r >> 1);
+                        float *v = qv[hh][ks];
+                        const uint16_t c01 = code8x2(v[0], v[1], KVT{});
+                        const uint16_t c23 = code8x2(v[2], v[3], KVT{});
+                        const uint32_t word = (uint32_t)c01 | ((uint32_t)c23 << 16);
+                        if constexpr (C::PACK8)
+                            q8[t >> 1][jj][r + (t & 1)] = word;
+                        else
+                            q8[t][jj][r] = word;
+                        if (t + 1 < C::QT8) {
+                            float d0, d1, d2, d3;
+                            unpack2_8<KVT>(c01, d0, d1);
+                            unpack2_8<KVT>(c23, d2, d3);
+                            v[0] = (v[0] - d0) * kUp;
+                            v[1] = (v[1] - d1) * kUp;
+                            v[2] = (v[2] - d2) * kUp;
+                            v[3] = (v[3] - d3) * kUp;
+                        }
+                    }
+                }
+            }
+        }
+#pragma unroll
+        for (int ks = 0; ks < (C::K8MMA ? 0 : C::KS); ++ks) {
             qa[ks][0] = pack2(qv[0][ks][0], qv[0][ks][1], ET{});
             qa[ks][1] = pack2(qv[1][ks][0], qv[1][ks][1], ET{});
             qa[ks][2] = pack2(qv[0][ks][2], qv[0][ks][3], ET{});
@@ -396,6 +500,8 @@ __global__ void __launch_bounds__(NWARPS * 32, MmaCfg<QT, KVT, D, GT, NWARPS>::M
     const int lsel_v = lane >> 4;                       // P.V: chunk +0 | +1
     bool timed_out = false;
     int k = 0;
+    int st = 0;          // k % NST
+    uint32_t phase = 0;  // (k / NST) & 1
 
     for (; k < nk; ++k) {
         if (k > 0 && (k & 31) == 0) {
@@ -403,8 +509,7 @@ __global__ void __launch_bounds__(NWARPS * 32, MmaCfg<QT, KVT, D, GT, NWARPS>::M
             ++cur_batch;
             bt_nxt = nk > (cur_batch + 1) * 32 ? load_batch(cur_batch + 1) : 0;
         }
-        const int st = k % NST;
-        const bool ok = __all_sync(kFull, mbar_wait_bounded(bar0 + 8 * st, (k / NST) & 1, wait_limit));
+        const bool ok = __all_sync(kFull, mbar_wait_bounded(bar0 + 8 * st, phase, wait_limit));
         if (!ok) {
             if (lane == 0) flag_error(p.err, kErrTimeout);
             timed_out = true;
@@ -465,7 +570,8 @@ __global__ void __launch_bounds__(NWARPS * 32, MmaCfg<QT, KVT, D, GT, NWARPS>::M
                 mma16816(sc[0], qa[ks], b[0], b[1], ET{});
                 mma16816(sc[1], qa[ks], b[2], b[3], ET{});
             }
-        } else {
+        } else if constexpr (!C::K8MMA) {
+            // 8-bit codes widened to f16 (exact), d permuted consistently in q
 #pragma unroll
             for (int jj = 0; jj < C::KS / 2; ++jj) {
                 uint32_t w[4];  // (nt0, ks=2jj), (nt0, 2jj+1), (nt1, 2jj), (nt1, 2jj+1)
@@ -480,6 +586,43 @@ __global__ void __launch_bounds__(NWARPS * 32, MmaCfg<QT, KVT, D, GT, NWARPS>::M
                     mma16816(sc[1], qa[ks], b2, b3, ET{});
                 }
             }
+        } else {
+            // the K codes feed the 8-bit MMA as they landed: an ldmatrix row is
+            // 16 codes of one token, so each lane's word holds the 4 codes of
+            // k 4kq..4kq+3 that the m16n8k32 B fragment wants
+            using AccT = typename std::conditional<C::INT8, int, float>::type;
+            AccT acc[C::NA8][2][4];
+#pragma unroll
+            for (int a = 0; a < C::NA8; ++a)
+#pragma unroll
+                for (int n = 0; n < 2; ++n)
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) acc[a][n][i] = 0;
+#pragma unroll
+            for (int jj = 0; jj < C::KS / 2; ++jj) {
+                uint32_t w[4];  // (tokens 0-7, k 0-15), (0-7, k 16-31), (8-15, k 0-15), (8-15, k 16-31)
+                ldsm_x4(w, kt + swz(lrow_b, 2 * jj + lsel_b));
+#pragma unroll
+                for (int a = 0; a < C::NA8; ++a) {
+                    mma_k32(acc[a][0], q8[a][jj], w[0], w[1], KVT{});
+                    mma_k32(acc[a][1], q8[a][jj], w[2], w[3], KVT{});
+                }
+            }
+            // S = sum_t 2^(-QSH t) (term t . K); term t of row i sits in
+            // acc[t / 2][n][i + 2 (t & 1)] (PACK8) or acc[t][n][i]
+            constexpr float kDown = 1.f / (float)(1 << C::QSH);
+            auto term = [&](int t, int n, int i) -> float {
+                return C::PACK8 ? (float)acc[t >> 1][n][i + 2 * (t & 1)] : (float)acc[t][n][i];
+            };
+#pragma unroll
+            for (int n = 0; n < 2; ++n)
+#pragma unroll
+                for (int i = 0; i < (C::PACK8 ? 2 : 4); ++i) {
+                    float v = term(C::QT8 - 1, n, i);
+#pragma unroll
+                    for (int t = C::QT8 - 2; t >= 0; --t) v = fmaf(v, kDown, term(t, n, i));
+                    sc[n][i] = v;
+                }
         }
 
         // online softmax; lane holds S[row g (+8)][tokens 2kq, 2kq+1, 8+2kq, 9+2kq]
@@ -501,9 +644,9 @@ __global__ void __launch_bounds__(NWARPS * 32, MmaCfg<QT, KVT, D, GT, NWARPS>::M
 #pragma unroll
             for (int i = 0; i < 4; ++i) pr[r][i] = 0.f;
             if (m_new != -CUDART_INF_F) {
-                alpha[r] = exp2f(m_run[r] - m_new);
+                alpha[r] = ex2(m_run[r] - m_new);
 #pragma unroll
-                for (int i = 0; i < 4; ++i) pr[r][i] = exp2f(sv[i] - m_new);
+                for (int i = 0; i < 4; ++i) pr[r][i] = ex2(sv[i] - m_new);
             }
             l_run[r] = l_run[r] * alpha[r] + ((pr[r][0] + pr[r][1]) + (pr[r][2] + pr[r][3]));
             m_run[r] = m_new;
@@ -590,7 +733,11 @@ __global__ void __launch_bounds__(NWARPS * 32, MmaCfg<QT, KVT, D, GT, NWARPS>::M
             }
         }
         __syncwarp();
-        if (k + NST < nk) issue(k + NST);
+        if (k + NST < nk) issue(k + NST, st);
+        if (++st == NST) {
+            st = 0;
+            phase ^= 1u;
+        }
     }
 
     if (timed_out) {

@@ -54,6 +54,45 @@ def test_prefill_small_full_parity(case):
     assert_close(_f64(pre.out), ref, f"prefill case {case}")
 
 
+def _scale_rows(bits, dtype, factor, rows=slice(None)):
+    """Multiply the given token rows of 16-bit patterns by a power of two (exact)."""
+    f = workload.bits_to_f32(bits, dtype).astype(np.float32)
+    f[rows] *= np.float32(factor)
+    return workload.f32_to_bits(f, dtype)
+
+
+@pytest.mark.parametrize("kind", ["huge", "tiny", "early_block", "late_block"])
+def test_prefill_bf16_value_range(kind):
+    """bf16 caches: P.V runs in f16 on V tiles scaled by 2^-k (k from each
+    tile's largest magnitude), so V values far outside f16's range must come
+    out as the oracle's: all V times 2^20 or 2^-40, or one 16-token block of
+    the context times 2^18 in the first key tile (later tiles get a smaller P
+    scale) or in a later one (the output is rescaled when it arrives).  Each
+    sequence's rows are compared after dividing by a power of two near their
+    largest magnitude (exact), with the usual bars."""
+    w = workload.build_chunked(f"range {kind}", 2900, [0, 230, 90], [150, 40, 64], 32, 8, 128,
+                               "bf16", "bf16")
+    if kind in ("huge", "tiny"):
+        fac = 2.0 ** 20 if kind == "huge" else 2.0 ** -40
+        w.v_ctx = _scale_rows(w.v_ctx, "bf16", fac)
+        w.v_chunk = _scale_rows(w.v_chunk, "bf16", fac)
+    else:
+        lo = 16 if kind == "early_block" else 192  # context positions of the scaled block
+        rows = np.nonzero((w.ctx_pos >= lo) & (w.ctx_pos < lo + 16))[0]
+        w.v_ctx = _scale_rows(w.v_ctx, "bf16", 2.0 ** 18, rows)
+    pre = _run(w)
+    assert pre.error() == 0
+    kc, vc = oracle.chunked_caches_for(w)
+    ref = oracle.prefill_for(w, kc, vc)
+    got = _f64(pre.out)
+    for s in range(w.num_seqs):
+        r = slice(int(w.query_start[s]), int(w.query_start[s + 1]))
+        if r.start == r.stop:
+            continue
+        norm = 2.0 ** -np.round(np.log2(np.abs(ref[r]).max()))
+        assert_close(got[r] * norm, ref[r] * norm, f"{kind} seq {s}")
+
+
 def test_prefill_rows_independent_of_chunking_bitwise():
     """One 300-token prompt prefilled as one chunk, or as chunks of 100, 77
     and 123 over the growing cache: every row is bit-identical (each row's
