@@ -146,8 +146,7 @@ __device__ __forceinline__ void cvt8x4_f16x2(uint32_t w, uint32_t &lo, uint32_t 
         hi = hsub2(prmt2(x, 0x6464u, kHi), 0x64806480u);
     } else {
         const uint32_t a = (SEL_LO == 0x10u) ? w : prmt2(w, 0u, 0x3120u);
-        lo = cvt8x2_f16x2<KVT>(a);
-        hi = cvt8x2_f16x2<KVT>(a >> 16);
+        cvt8x4_halves(a, lo, hi, KVT{});
     }
 }
 
@@ -225,11 +224,13 @@ template <typename QT, typename KVT, int D, int GT, int NW_ = kDecodeWarps> stru
     // 0-7 term 2m, rows 8-15 term 2m+1 of MMA m), so the rows the GQA group
     // leaves empty do useful work; 16 heads need one MMA per term
     static constexpr bool PACK8 = GT == 8;
-    // the 8-bit q.K path where two terms suffice (E4M3 against a bf16 q,
-    // INT8 against either) and pack into one MMA (groups of up to 8 heads);
-    // three-term cases (E5M2, E4M3 against an f16 q) and 16-row groups would
-    // run out of registers and keep widening K to f16
-    static constexpr bool K8MMA = FP8 && QT8 == 2 && PACK8;
+    // the 8-bit q.K path for INT8 caches with groups of up to 8 heads (two
+    // terms, packed into one MMA): its widening costs five instructions per
+    // four codes, and the integer MMA measured faster (long-context INT8:
+    // 117.6 -> 112.4 us).  E4M3 keeps widening K to f16: its two-instruction
+    // widening beat the E4M3 MMA (110.1 vs 114.8 us); E5M2, f16-q and 16-row
+    // cases would need three terms and run out of registers.
+    static constexpr bool K8MMA = INT8 && PACK8;
     static constexpr int NA8 = PACK8 ? (QT8 + 1) / 2 : QT8;  // A-operand sets (MMAs per k32 step)
     static constexpr int MT = D / 16;   // m-tiles (16 rows of d) of O^T = V^T P^T
     static constexpr int NH = GT / 8;   // n-tiles (8 heads) of O^T

@@ -63,6 +63,21 @@ __device__ __forceinline__ uint32_t cvt8x2_f16x2(uint32_t two, e5m2_t) {
     asm("cvt.rn.f16x2.e5m2x2 %0, %1;" : "=r"(h2) : "h"((uint16_t)two));
     return h2;
 }
+// Four codes of one word (low byte first) -> two f16x2: codes 0, 1 in lo and
+// 2, 3 in hi.  The word is split into its two 16-bit halves inside the asm, so
+// no shift is needed to reach the high pair.
+__device__ __forceinline__ void cvt8x4_halves(uint32_t w, uint32_t &lo, uint32_t &hi, e4m3_t) {
+    asm("{\n\t.reg .b16 l, h;\n\tmov.b32 {l, h}, %2;\n\t"
+        "cvt.rn.f16x2.e4m3x2 %0, l;\n\tcvt.rn.f16x2.e4m3x2 %1, h;\n\t}"
+        : "=r"(lo), "=r"(hi)
+        : "r"(w));
+}
+__device__ __forceinline__ void cvt8x4_halves(uint32_t w, uint32_t &lo, uint32_t &hi, e5m2_t) {
+    asm("{\n\t.reg .b16 l, h;\n\tmov.b32 {l, h}, %2;\n\t"
+        "cvt.rn.f16x2.e5m2x2 %0, l;\n\tcvt.rn.f16x2.e5m2x2 %1, h;\n\t}"
+        : "=r"(lo), "=r"(hi)
+        : "r"(w));
+}
 // INT8: the biased byte b ^ 0x80 = b + 128 becomes the low mantissa byte of an
 // f16 with exponent byte 0x64 (the value 1024 + b + 128, exact); subtracting
 // 1152 leaves b.

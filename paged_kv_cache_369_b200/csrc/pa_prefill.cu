@@ -171,8 +171,7 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap *map
 // Four 8-bit codes of one word -> two f16x2 (codes 0,1 in lo; 2,3 in hi), exact.
 template <typename KT>
 __device__ __forceinline__ void widen4(uint32_t w, uint32_t &lo, uint32_t &hi, KT) {
-    lo = cvt8x2_f16x2(w & 0xFFFFu, KT{});
-    hi = cvt8x2_f16x2(w >> 16, KT{});
+    cvt8x4_halves(w, lo, hi, KT{});
 }
 // INT8, a word at a time: one bias flip (b ^ 0x80 = b + 128) for the four
 // bytes, each pair under the f16 exponent byte 0x64 (value 1024 + 128 + b),
@@ -233,8 +232,8 @@ template <typename T, int D, typename KVT = T> struct PfCfg {
     static constexpr bool KV8 = Elem<KVT>::kBytes == 1;
     static constexpr int BM = 128;  // query rows per tile (TMEM lanes); two tiles per CTA
     static constexpr int BN = 64;   // keys per tile = 4 blocks
-    // stages of each operand ring (K, V): Q.K^T reads K tile j + 2 while P.V
-    // reads V tile j; 8-bit caches: 3 each beside the 4-stage staging ring
+    // K/V operand ring stages (16-bit): the MMA issuer reads tile j + 2's
+    // stage while PV(j) still holds tile j's, so at least 3
     static constexpr int ST = KV8 ? 3 : 4;
     static constexpr int SST = KV8 ? 4 : 0;  // 8-bit staging ring stages
     static constexpr int ATOMS = D / 64;  // 128-byte swizzle atoms across d (16-bit)
@@ -242,49 +241,34 @@ template <typename T, int D, typename KVT = T> struct PfCfg {
     static constexpr int KV_BYTES = ATOMS * BN * 128;
     static constexpr int KV8_BYTES = BN * D;          // one 8-bit tile (d = 128: 128-byte rows)
     static constexpr int OFF_Q = 0;                   // tile A, then tile B
-    // K and V operand rings of ST stages each (K stages, then V stages): K
-    // tile j is freed once Q.K^T of both query tiles has read it, V tile j
-    // once P.V has, so each refills on its own schedule and loads run ~3 key
-    // tiles ahead of their use
-    static constexpr int OFF_KV = 2 * Q_BYTES;
+    static constexpr int OFF_KV = 2 * Q_BYTES;        // stage st: K, then V
     static constexpr int OFF_STG = OFF_KV + ST * 2 * KV_BYTES;  // 8-bit stage: K, then V
     static constexpr int OFF_BAR = OFF_STG + SST * 2 * KV8_BYTES;
-    // bf16 caches: the two converter warps turn each landed V tile into f16 in
-    // place, scaled by a power of two 2^-k per tile chosen from the tile's
-    // largest magnitude, so that P.V runs as one f16 x f16 MMA with P in f16
-    // (11 bits): bf16 values with |v| in [2^-6, 65280] are exact in f16 and
-    // keep k = 0; other tiles are brought to [2^14, 2^15) and the softmax
-    // folds 2^k into P and the output
-    static constexpr bool VCONV = !KV8 && std::is_same<KVT, bf16_t>::value;
-    // q_full, k_full[ST], k_empty[ST], then per (tile, score buffer):
-    // s_full, p_full, pv_done; drain; q_ready, stg_full[SST], stg_empty[SST],
-    // v_ready[ST], vmax_full[ST] (bf16 caches), v_full[ST], v_empty[ST]
-    static constexpr int NBAR = 1 + 2 * ST + 4 + 4 + 4 + 1 + 1 + 2 * SST + 4 * ST;
+    // q_full, kv_full[ST], kv_empty[ST], then per (tile, score buffer):
+    // s_full, p_full, pv_done; drain; q_ready, stg_full[SST], stg_empty[SST]
+    static constexpr int NBAR = 1 + 2 * ST + 4 + 4 + 4 + 1 + 1 + 2 * SST;
     static constexpr int OFF_SLOT = OFF_BAR + NBAR * 8;
     static constexpr int OFF_ABORT = OFF_SLOT + 4;
     static constexpr int OFF_QEXP = OFF_ABORT + 4;    // log2 of the q scaling (8-bit caches)
-    static constexpr int OFF_VEXP = OFF_QEXP + 4;     // k of each stage's V tile (bf16 caches)
-    static constexpr int OFF_VAMAX = OFF_VEXP + 4 * ST;  // per stage, per converter warp
-    static constexpr int USED = OFF_VAMAX + 8 * ST;
+    static constexpr int USED = OFF_QEXP + 4;
     // at least 120 KiB so that one CTA holds an SM (and its 512 TMEM columns)
     static constexpr int SMEM = 1024 + (USED < 120 * 1024 ? 120 * 1024 : USED);
-    // operand types: Q.K^T in T (f16 for 8-bit caches, whose codes widen to
-    // f16 exactly); P.V always f16 x f16
-    static constexpr bool QK_BF16 = std::is_same<T, bf16_t>::value && !KV8;
+    // MMA operand type: T, or f16 for 8-bit caches (codes widen to f16 exactly)
+    static constexpr bool OP_BF16 = std::is_same<T, bf16_t>::value && !KV8;
+    static constexpr bool HILO = OP_BF16;
     static constexpr uint32_t TMEM_COLS = 512;
     // score buffer b of tile t at column 64 (2 t + b) (P written over it), O
     // of tile t at 256 + 128 t
     static constexpr uint32_t COL_S = 0, COL_O = 256;
-    static constexpr uint32_t FMT_QK = QK_BF16 ? 1u : 0u;  // kind::f16 operand format: f16 0, bf16 1
-    static constexpr uint32_t FMT_PV = 0u;
+    static constexpr uint32_t FMT = OP_BF16 ? 1u : 0u;  // kind::f16 operand format: f16 0, bf16 1
     // instruction descriptors: fp32 accumulate, A/B format, majors, N >> 3, M >> 4
-    static constexpr uint32_t IDESC_QK = (1u << 4) | (FMT_QK << 7) | (FMT_QK << 10) |
+    static constexpr uint32_t IDESC_QK = (1u << 4) | (FMT << 7) | (FMT << 10) |
                                          ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
-    static constexpr uint32_t IDESC_PV = (1u << 4) | (FMT_PV << 7) | (FMT_PV << 10) | (1u << 16) |
+    static constexpr uint32_t IDESC_PV = (1u << 4) | (FMT << 7) | (FMT << 10) | (1u << 16) |
                                          ((uint32_t)(D >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
-    // 8 softmax warps, a TMA warp, an MMA warp, + two converter warps (K and V
-    // for 8-bit caches; both V for bf16 caches)
-    static constexpr int CONVERTERS = (KV8 || VCONV) ? 2 : 0;
+    // 8 softmax warps, a TMA warp, an MMA warp (+ two converter warps, K and V,
+    // for 8-bit caches)
+    static constexpr int CONVERTERS = KV8 ? 2 : 0;
     static constexpr int THREADS = 320 + 32 * CONVERTERS;
     static_assert(D == 64 || D == 128, "head_dim 64 or 128");
     static_assert(!KV8 || D == 128, "8-bit caches: head_dim 128");
@@ -304,6 +288,7 @@ __global__ void __launch_bounds__(PfCfg<T, D, KVT>::THREADS, 1)
                    const __grid_constant__ CUtensorMap tmap_k,
                    const __grid_constant__ CUtensorMap tmap_v) {
     using C = PfCfg<T, D, KVT>;
+    using OpT = typename std::conditional<C::OP_BF16, bf16_t, f16_t>::type;  // MMA operand type
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_addr(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;
@@ -352,8 +337,8 @@ __global__ void __launch_bounds__(PfCfg<T, D, KVT>::THREADS, 1)
 
     const uint32_t bars = base + C::OFF_BAR;
     const uint32_t bar_q = bars;
-    auto bar_k_full = [&](int st) { return bars + 8u * (1 + st); };
-    auto bar_k_empty = [&](int st) { return bars + 8u * (1 + C::ST + st); };
+    auto bar_kv_full = [&](int st) { return bars + 8u * (1 + st); };
+    auto bar_kv_empty = [&](int st) { return bars + 8u * (1 + C::ST + st); };
     // one barrier per (tile, score buffer): a buffer's next phase needs the
     // other roles to have used the last one, so no wait can see a phase twice
     auto bar_s_full = [&](int t, int b) { return bars + 8u * (1 + 2 * C::ST + 2 * t + b); };
@@ -364,13 +349,6 @@ __global__ void __launch_bounds__(PfCfg<T, D, KVT>::THREADS, 1)
     const uint32_t bar_q_ready = bars + 8u * (14 + 2 * C::ST);
     auto bar_stg_full = [&](int st) { return bars + 8u * (15 + 2 * C::ST + st); };
     auto bar_stg_empty = [&](int st) { return bars + 8u * (15 + 2 * C::ST + C::SST + st); };
-    // bf16 caches: stage st's V tile converted to f16 (and its exponent k stored)
-    auto bar_v_ready = [&](int st) { return bars + 8u * (15 + 2 * C::ST + 2 * C::SST + st); };
-    // bf16 caches: both converter warps' partial largest magnitudes of stage st stored
-    auto bar_vmax = [&](int st) { return bars + 8u * (15 + 3 * C::ST + 2 * C::SST + st); };
-    auto bar_v_full = [&](int st) { return bars + 8u * (15 + 4 * C::ST + 2 * C::SST + st); };
-    auto bar_v_empty = [&](int st) { return bars + 8u * (15 + 5 * C::ST + 2 * C::SST + st); };
-    volatile int *vexp = reinterpret_cast<volatile int *>(smem + C::OFF_VEXP);
     auto s_col = [&](int t, int b) { return C::COL_S + 64u * (2 * t + b); };
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + C::OFF_ABORT);
     uint32_t *slot = reinterpret_cast<uint32_t *>(smem + C::OFF_SLOT);
@@ -379,11 +357,8 @@ __global__ void __launch_bounds__(PfCfg<T, D, KVT>::THREADS, 1)
         mbar_init(bar_q, 1);
 #pragma unroll
         for (int st = 0; st < C::ST; ++st) {
-            // filled by the TMA (16-bit), or by the K / V converter (8-bit)
-            mbar_init(bar_k_full(st), 1);
-            mbar_init(bar_k_empty(st), 1);
-            mbar_init(bar_v_full(st), 1);
-            mbar_init(bar_v_empty(st), 1);
+            mbar_init(bar_kv_full(st), C::KV8 ? C::CONVERTERS : 1);  // TMA, or the converters
+            mbar_init(bar_kv_empty(st), 1);
         }
 #pragma unroll
         for (int t = 0; t < 2; ++t)
@@ -400,13 +375,6 @@ __global__ void __launch_bounds__(PfCfg<T, D, KVT>::THREADS, 1)
             mbar_init(bar_stg_full(st), 1);
             mbar_init(bar_stg_empty(st), C::CONVERTERS);
         }
-        if constexpr (C::VCONV) {
-#pragma unroll
-            for (int st = 0; st < C::ST; ++st) {
-                mbar_init(bar_v_ready(st), C::CONVERTERS);
-                mbar_init(bar_vmax(st), C::CONVERTERS);
-            }
-        }
         *abort_flag = 0;
         mbar_init_fence();
     }
@@ -417,16 +385,13 @@ __global__ void __launch_bounds__(PfCfg<T, D, KVT>::THREADS, 1)
     const uint32_t tmem = *slot;
 
     auto q_smem = [&](int t) { return base + C::OFF_Q + (uint32_t)(t * C::Q_BYTES); };
-    auto k_smem = [&](int st) { return base + C::OFF_KV + (uint32_t)(st * C::KV_BYTES); };
-    auto v_smem = [&](int st) { return base + C::OFF_KV + (uint32_t)((C::ST + st) * C::KV_BYTES); };
+    auto k_smem = [&](int st) { return base + C::OFF_KV + (uint32_t)(st * 2 * C::KV_BYTES); };
+    auto v_smem = [&](int st) { return k_smem(st) + (uint32_t)C::KV_BYTES; };
     auto stg_k = [&](int st) { return base + C::OFF_STG + (uint32_t)(st * 2 * C::KV8_BYTES); };
     auto stg_v = [&](int st) { return stg_k(st) + (uint32_t)C::KV8_BYTES; };
 
     if (warp == 8) {
         // ================= TMA producer ===========================================
-        // The whole warp walks the key tiles; each lane holds the pool row of
-        // one 16-token tile of the current batch of 32 (and the next batch is
-        // read ahead), so no copy waits on a block-table read; lane 0 issues.
         if (lane == 0) {
             asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_q)) : "memory");
             asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_k)) : "memory");
@@ -438,113 +403,48 @@ __global__ void __launch_bounds__(PfCfg<T, D, KVT>::THREADS, 1)
                 for (int a = 0; a < C::ATOMS; ++a)
                     tc::tma_load_3d(q_smem(t) + a * C::BM * 128, &tmap_q, a * 64, kvh * g,
                                     q0 + tok0 + t * tpt, bar_q);
-        }
-        const int32_t *bt = p.block_tables + (int64_t)s * p.max_blocks_per_seq;
-        constexpr int TPK = C::BN / kBlockSize;  // 16-token tiles per key tile
-        const int tile0 = j0 * TPK, ntiles = nt * TPK;
-        auto rows_of_batch = [&](int batch) -> int {  // this lane's tile of the batch
-            const int i = batch * 32 + lane;
-            int y = p.oob_row;  // past the pool: the copy fills zeros
-            const int lb = tile0 + i;
-            if (i < ntiles && lb < nblk_seq) {
-                const int phys = bt[lb >> p.tile_shift];
-                if ((unsigned)phys < (unsigned)p.num_blocks)
-                    y = (phys * p.num_kv_heads + kvh) * p.block_size + (lb & tile_mask) * kBlockSize;
-                else
-                    flag_error(p.err, kErrBounds);
-            }
-            return y;
-        };
-        int rows_cur = rows_of_batch(0), rows_nxt = rows_of_batch(1), cur_batch = 0;
-        // pool row of 16-token tile i (i never more than one batch ahead of
-        // the current one, whose start moves with the V tiles)
-        auto row_at = [&](int i) {
-            const int a = __shfl_sync(tc::kFull, rows_cur, i & 31);
-            const int b = __shfl_sync(tc::kFull, rows_nxt, i & 31);
-            return (i >> 5) == cur_batch ? a : b;
-        };
-        auto advance_to = [&](int i) {  // uniform: make tile i's batch the current one
-            if ((i >> 5) != cur_batch) {
-                rows_cur = rows_nxt;
-                ++cur_batch;
-                rows_nxt = rows_of_batch(cur_batch + 1);
-            }
-        };
-        int j = 0, jk = 0;  // V (or 8-bit pair) tiles issued; 16-bit K tiles issued
-        if constexpr (C::KV8) {
-            // 8-bit caches: K and V codes of key tile j land together in the
-            // staging ring; the converter warps move them to the operand rings
-            for (; j < nt; ++j) {
-                const int st = j % C::SST;
-                if (j >= C::SST &&
-                    !__all_sync(tc::kFull, tc::wait_phase(bar_stg_empty(st), ((j / C::SST) - 1) & 1, abort_flag, p.err)))
-                    break;
-                if (lane == 0) mbar_arrive_expect_tx(bar_stg_full(st), 2u * C::KV8_BYTES);
-#pragma unroll
-                for (int b = 0; b < TPK; ++b) {
-                    const int i = j * TPK + b;
-                    advance_to(i);
-                    const int y = row_at(i);
-                    if (lane == 0) {  // 16 rows x 128 codes, 128B swizzle
-                        const uint32_t off = b * kBlockSize * 128;
-                        tc::tma_load_2d(stg_k(st) + off, &tmap_k, 0, y, bar_stg_full(st));
-                        tc::tma_load_2d(stg_v(st) + off, &tmap_v, 0, y, bar_stg_full(st));
-                    }
+            const int32_t *bt = p.block_tables + (int64_t)s * p.max_blocks_per_seq;
+            auto row_of = [&](int lb) -> int {  // pool row of 16-token tile lb (past the pool: zeros)
+                int y = p.oob_row;
+                if (lb < nblk_seq) {
+                    const int phys = bt[lb >> p.tile_shift];
+                    if ((unsigned)phys < (unsigned)p.num_blocks)
+                        y = (phys * p.num_kv_heads + kvh) * p.block_size + (lb & tile_mask) * kBlockSize;
+                    else
+                        flag_error(p.err, kErrBounds);
                 }
-            }
-        } else {
-            // 16-bit caches: K tile j + 2 goes out with V tile j (Q.K^T runs two
-            // key tiles ahead of P.V); each waits for its own ring's free stage
-            auto issue_tile = [&](int jt, bool is_k) -> bool {
-                const int st = jt % C::ST;
-                const uint32_t full = is_k ? bar_k_full(st) : bar_v_full(st);
-                const uint32_t empty = is_k ? bar_k_empty(st) : bar_v_empty(st);
-                if (jt >= C::ST &&
-                    !__all_sync(tc::kFull, tc::wait_phase(empty, ((jt / C::ST) - 1) & 1, abort_flag, p.err)))
-                    return false;
-                if (lane == 0) mbar_arrive_expect_tx(full, (uint32_t)C::KV_BYTES);
-                const uint32_t dst = is_k ? k_smem(st) : v_smem(st);
-#pragma unroll
-                for (int b = 0; b < TPK; ++b) {
-                    const int y = row_at(jt * TPK + b);
-                    if (lane == 0) {
-#pragma unroll
-                        for (int a = 0; a < C::ATOMS; ++a)
-                            tc::tma_load_2d(dst + a * C::BN * 128 + b * kBlockSize * 128, is_k ? &tmap_k : &tmap_v,
-                                            a * 64, y, full);
-                    }
-                }
-                return true;
+                return y;
             };
-            // j / jk count the tiles actually issued (the drain below waits on them)
-            bool ok = true;
-            while (ok && jk < 2 && jk < nt) {
-                ok = issue_tile(jk, true);
-                if (ok) ++jk;
-            }
-            while (ok && j < nt) {
-                advance_to(j * TPK);
-                ok = issue_tile(j, false);
-                if (!ok) break;
-                ++j;
-                if (jk < nt) {
-                    ok = issue_tile(jk, true);
-                    if (ok) ++jk;
+            constexpr int RING = C::KV8 ? C::SST : C::ST;  // the ring the copies land in
+            auto full_bar = [&](int st) { return C::KV8 ? bar_stg_full(st) : bar_kv_full(st); };
+            auto empty_bar = [&](int st) { return C::KV8 ? bar_stg_empty(st) : bar_kv_empty(st); };
+            int j = 0;
+            for (; j < nt; ++j) {
+                const int st = j % RING;
+                if (j >= RING && !tc::wait_phase(empty_bar(st), ((j / RING) - 1) & 1, abort_flag, p.err))
+                    break;
+                mbar_arrive_expect_tx(full_bar(st), C::KV8 ? 2u * C::KV8_BYTES : 2u * C::KV_BYTES);
+#pragma unroll 1
+                for (int b = 0; b < C::BN / kBlockSize; ++b) {
+                    const int y = row_of((j0 + j) * (C::BN / kBlockSize) + b);
+                    if constexpr (C::KV8) {  // 16 rows x 128 codes, 128B swizzle
+                        const uint32_t off = b * kBlockSize * 128;
+                        tc::tma_load_2d(stg_k(st) + off, &tmap_k, 0, y, full_bar(st));
+                        tc::tma_load_2d(stg_v(st) + off, &tmap_v, 0, y, full_bar(st));
+                    } else {
+#pragma unroll
+                        for (int a = 0; a < C::ATOMS; ++a) {
+                            const uint32_t off = a * C::BN * 128 + b * kBlockSize * 128;
+                            tc::tma_load_2d(k_smem(st) + off, &tmap_k, a * 64, y, full_bar(st));
+                            tc::tma_load_2d(v_smem(st) + off, &tmap_v, a * 64, y, full_bar(st));
+                        }
+                    }
                 }
             }
-        }
-        if (lane == 0) {
             // nothing may still be landing in shared memory when the CTA exits
             (void)mbar_wait_bounded(bar_q, 0, kWaitLimitNs);
-            if constexpr (C::KV8) {
-                for (int jj = j - C::SST < 0 ? 0 : j - C::SST; jj < j; ++jj)
-                    (void)mbar_wait_bounded(bar_stg_full(jj % C::SST), (jj / C::SST) & 1, kWaitLimitNs);
-            } else {
-                for (int jj = j - C::ST < 0 ? 0 : j - C::ST; jj < j; ++jj)
-                    (void)mbar_wait_bounded(bar_v_full(jj % C::ST), (jj / C::ST) & 1, kWaitLimitNs);
-                for (int jj = jk - C::ST < 0 ? 0 : jk - C::ST; jj < jk; ++jj)
-                    (void)mbar_wait_bounded(bar_k_full(jj % C::ST), (jj / C::ST) & 1, kWaitLimitNs);
-            }
+            for (int jj = j - RING < 0 ? 0 : j - RING; jj < j; ++jj)
+                (void)mbar_wait_bounded(full_bar(jj % RING), (jj / RING) & 1, kWaitLimitNs);
         }
         __syncwarp();
     } else if (warp == 9) {
@@ -565,7 +465,6 @@ __global__ void __launch_bounds__(PfCfg<T, D, KVT>::THREADS, 1)
                                C::IDESC_QK, ks > 0);
                 }
                 tc::commit(bar_s_full(t, j & 1));
-                if (t == 1) tc::commit(bar_k_empty(j % C::ST));  // last reader of the K stage
             }
             __syncwarp();
         };
@@ -579,9 +478,11 @@ __global__ void __launch_bounds__(PfCfg<T, D, KVT>::THREADS, 1)
                 for (int ks = 0; ks < C::BN / 16; ++ks) {
                     const uint64_t bdesc = tc::sdesc(vaddr + ks * 2048, C::BN * 128, 1024);
                     tc::mma_ts(ocol, pcol + ks * 8, bdesc, C::IDESC_PV, (j > 0 || ks > 0));
+                    if constexpr (C::HILO)
+                        tc::mma_ts(ocol, pcol + C::BN / 2 + ks * 8, bdesc, C::IDESC_PV, 1);
                 }
                 tc::commit(bar_pv(t, j & 1));
-                if (t == 1) tc::commit(bar_v_empty(j % C::ST));  // last reader of the V stage
+                if (t == 1) tc::commit(bar_kv_empty(j % C::ST));  // last reader of the stage
             }
             __syncwarp();
         };
@@ -589,12 +490,10 @@ __global__ void __launch_bounds__(PfCfg<T, D, KVT>::THREADS, 1)
             return __all_sync(tc::kFull, tc::wait_phase(bar, parity, abort_flag, p.err));
         };
         const int j_tail = (L & (kBlockSize - 1)) ? (nblk_seq - 1) / (C::BN / kBlockSize) : -1;
-        auto k_ready = [&](int j) { return wait_all(bar_k_full(j % C::ST), (j / C::ST) & 1); };
-        auto v_ready = [&](int j) {
+        auto kv_ready = [&](int j) {
             const int st = j % C::ST;
-            // bf16 caches: converted to f16 (the converters also cleared the tail)
-            if (!wait_all(C::VCONV ? bar_v_ready(st) : bar_v_full(st), (j / C::ST) & 1)) return false;
-            if (!C::VCONV && j0 + j == j_tail) {
+            if (!wait_all(bar_kv_full(st), (j / C::ST) & 1)) return false;
+            if (j0 + j == j_tail) {
                 // clear the V rows of the last block's unused slots (positions >= L)
                 const int r0 = L - (j0 + j) * C::BN, r1 = nblk_seq * kBlockSize - (j0 + j) * C::BN;
                 const int chunks = (r1 - r0) * C::ATOMS * 8;
@@ -610,7 +509,7 @@ __global__ void __launch_bounds__(PfCfg<T, D, KVT>::THREADS, 1)
         };
         bool ok = wait_all(C::KV8 ? bar_q_ready : bar_q, 0);  // 8-bit caches: q converted
         for (int j = 0; ok && j < 2 && j < nt; ++j) {
-            ok = k_ready(j);
+            ok = kv_ready(j);
             if (!ok) break;
             issue_qk(0, j);
             issue_qk(1, j);
@@ -618,12 +517,10 @@ __global__ void __launch_bounds__(PfCfg<T, D, KVT>::THREADS, 1)
         for (int j = 0; ok && j < nt; ++j) {
             ok = wait_all(bar_p_full(0, j & 1), (j >> 1) & 1);
             if (!ok) break;
-            ok = v_ready(j);
-            if (!ok) break;
             issue_pv(0, j);
             const bool more = j + 2 < nt;
             if (more) {
-                ok = k_ready(j + 2);
+                ok = kv_ready(j + 2);
                 if (!ok) break;
                 issue_qk(0, j + 2);
             }
@@ -645,95 +542,7 @@ __global__ void __launch_bounds__(PfCfg<T, D, KVT>::THREADS, 1)
         // scale) and every landed 8-bit K tile, warp 11 every V tile, to f16
         // in the swizzled operand layout the MMAs read; each code's value is
         // exact in f16
-        if constexpr (C::VCONV) {
-            // bf16 V tile -> f16 in place: warp 10 takes rows 0 .. BN/2 - 1,
-            // warp 11 the rest.  Pass 1 finds the tile's largest magnitude
-            // (bf16 bit patterns order like magnitudes), the warps exchange it,
-            // pass 2 converts with 2^-k.
-            const int half = warp - 10;
-            const int j_tail = (L & (kBlockSize - 1)) ? (nblk_seq - 1) / (C::BN / kBlockSize) : -1;
-            constexpr int ROWS = C::BN / 2, CH = ROWS * C::ATOMS * 8;  // 16-byte chunks per warp
-            uint32_t *vamax = reinterpret_cast<uint32_t *>(smem + C::OFF_VAMAX);
-            bool ok = true;
-            for (int j = 0; ok && j < nt; ++j) {
-                const int st = j % C::ST;
-                ok = __all_sync(tc::kFull, tc::wait_phase(bar_v_full(st), (j / C::ST) & 1, abort_flag, p.err));
-                if (!ok) break;
-                const uint32_t vb = v_smem(st);
-                auto chunk_addr = [&](int c) {  // chunk c of this warp's rows
-                    const int row = half * ROWS + c / (C::ATOMS * 8), rem = c % (C::ATOMS * 8);
-                    return vb + (rem >> 3) * C::BN * 128 + row * 128 + (rem & 7) * 16;
-                };
-                if (j0 + j == j_tail) {
-                    // positions >= L of the last block: zero (p = 0 there, but
-                    // 0 x NaN poison = NaN), before the largest magnitude is taken
-                    const int r0 = L - (j0 + j) * C::BN;
-                    for (int c = lane; c < CH; c += 32) {
-                        const int row = half * ROWS + c / (C::ATOMS * 8);
-                        if (row >= r0)
-                            asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(chunk_addr(c)), "r"(0u)
-                                         : "memory");
-                    }
-                    __syncwarp();
-                }
-                uint32_t m2 = 0;  // per 16-bit half: largest |bf16| bit pattern
-#pragma unroll 4
-                for (int c = lane; c < CH; c += 32) {
-                    uint32_t w[4];
-                    lds<16>(w, chunk_addr(c));
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        uint32_t r;
-                        asm("max.u16x2 %0, %1, %2;" : "=r"(r) : "r"(m2), "r"(w[i] & 0x7FFF7FFFu));
-                        m2 = r;
-                    }
-                }
-                uint32_t am = max(m2 & 0xFFFFu, m2 >> 16);
-#pragma unroll
-                for (int o = 16; o > 0; o >>= 1) am = max(am, __shfl_xor_sync(tc::kFull, am, o));
-                // exchange with the other converter warp (a bounded wait: a
-                // timeout elsewhere makes both give up)
-                if (lane == 0) {
-                    reinterpret_cast<volatile uint32_t *>(vamax)[2 * st + half] = am;
-                    tc::mbar_arrive(bar_vmax(st));
-                }
-                ok = __all_sync(tc::kFull, tc::wait_phase(bar_vmax(st), (j / C::ST) & 1, abort_flag, p.err));
-                if (!ok) break;
-                am = max(reinterpret_cast<volatile uint32_t *>(vamax)[2 * st],
-                         reinterpret_cast<volatile uint32_t *>(vamax)[2 * st + 1]);
-                const int eb = (int)(am >> 7);  // biased exponent of the largest magnitude
-                int k = 0;
-                if (am == 0) {
-                    k = -100;  // an all-zero tile: any scale
-                } else if (eb < 255 && (eb < 127 - 6 || am > 0x477Fu)) {
-                    k = (eb == 0 ? -127 : eb - 127) - 14;  // largest magnitude to [2^14, 2^15)
-                    k = k < -100 ? -100 : (k > 100 ? 100 : k);
-                }  // (Inf / NaN: k = 0, carried into f16 as Inf / NaN)
-                const float down = __uint_as_float((uint32_t)(127 - k) << 23);  // 2^-k, exact
-#pragma unroll 4
-                for (int c = lane; c < CH; c += 32) {
-                    const uint32_t addr = chunk_addr(c);
-                    uint32_t w[4];
-                    lds<16>(w, addr);
-                    uint32_t h[4];
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        float lo, hi;
-                        tc::unpack2(w[i], lo, hi, bf16_t{});
-                        h[i] = tc::pack2(lo * down, hi * down, f16_t{});
-                    }
-                    asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(h[0]), "r"(h[1]),
-                                 "r"(h[2]), "r"(h[3])
-                                 : "memory");
-                }
-                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-                __syncwarp();
-                if (lane == 0) {
-                    if (half == 0) vexp[st] = k;
-                    tc::mbar_arrive(bar_v_ready(st));
-                }
-            }
-        } else if constexpr (C::KV8) {
+        if constexpr (C::KV8) {
             const int kv = warp - 10;  // 0: K, 1: V
             bool ok = kv == 1 || __all_sync(tc::kFull, tc::wait_phase(bar_q, 0, abort_flag, p.err));
             int e = 0;
@@ -785,36 +594,48 @@ __global__ void __launch_bounds__(PfCfg<T, D, KVT>::THREADS, 1)
                 if (!ok) break;
                 if (j >= C::ST) {  // the MMAs are done with this operand stage
                     ok = __all_sync(tc::kFull,
-                                    tc::wait_phase(kv ? bar_v_empty(st) : bar_k_empty(st), ((j / C::ST) - 1) & 1,
-                                                   abort_flag, p.err));
+                                    tc::wait_phase(bar_kv_empty(st), ((j / C::ST) - 1) & 1, abort_flag, p.err));
                     if (!ok) break;
                 }
                 {
                     const uint32_t src = kv ? stg_v(sst) : stg_k(sst);
                     const uint32_t dst = kv ? v_smem(st) : k_smem(st);
-                    for (int idx = lane; idx < C::BN * 8; idx += 32) {
-                        const int r = idx >> 3, c8 = idx & 7;  // row, chunk of 16 codes
-                        uint32_t w[4];
-                        lds<16>(w, src + r * 128 + ((c8 ^ (r & 7)) << 4));
-                        uint32_t h[8];
+                    // BN * 8 chunks of 16 codes, batches of 4 a lane: the loads of
+                    // a batch go out together, then its conversions and stores
+                    constexpr int NB = 4, PER = C::BN * 8 / 32;
+                    static_assert(PER % NB == 0, "batches");
 #pragma unroll
-                        for (int i = 0; i < 4; ++i) tc::widen4(w[i], h[2 * i], h[2 * i + 1], KVT{});
-                        // codes 16 c8 .. +15 = f16 chunks 2 (c8 % 4) and +1 of atom c8 / 4
-                        const uint32_t rowb = dst + (c8 >> 2) * C::BN * 128 + r * 128;
-                        const int cf = (c8 & 3) * 2;
-                        asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(rowb + ((cf ^ (r & 7)) << 4)),
-                                     "r"(h[0]), "r"(h[1]), "r"(h[2]), "r"(h[3])
-                                     : "memory");
-                        asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(rowb + (((cf + 1) ^ (r & 7)) << 4)),
-                                     "r"(h[4]), "r"(h[5]), "r"(h[6]), "r"(h[7])
-                                     : "memory");
+                    for (int i0 = 0; i0 < PER; i0 += NB) {
+                        uint32_t w[NB][4];
+#pragma unroll
+                        for (int b = 0; b < NB; ++b) {
+                            const int idx = lane + 32 * (i0 + b), r = idx >> 3, c8 = idx & 7;
+                            lds<16>(w[b], src + r * 128 + ((c8 ^ (r & 7)) << 4));
+                        }
+#pragma unroll
+                        for (int b = 0; b < NB; ++b) {
+                            const int idx = lane + 32 * (i0 + b);
+                            const int r = idx >> 3, c8 = idx & 7;  // row, chunk of 16 codes
+                            uint32_t h[8];
+#pragma unroll
+                            for (int i = 0; i < 4; ++i) tc::widen4(w[b][i], h[2 * i], h[2 * i + 1], KVT{});
+                            // codes 16 c8 .. +15 = f16 chunks 2 (c8 % 4) and +1 of atom c8 / 4
+                            const uint32_t rowb = dst + (c8 >> 2) * C::BN * 128 + r * 128;
+                            const int cf = (c8 & 3) * 2;
+                            asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(rowb + ((cf ^ (r & 7)) << 4)),
+                                         "r"(h[0]), "r"(h[1]), "r"(h[2]), "r"(h[3])
+                                         : "memory");
+                            asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(rowb + (((cf + 1) ^ (r & 7)) << 4)),
+                                         "r"(h[4]), "r"(h[5]), "r"(h[6]), "r"(h[7])
+                                         : "memory");
+                        }
                     }
                 }
                 asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
                 __syncwarp();
                 if (lane == 0) {
                     tc::mbar_arrive(bar_stg_empty(sst));
-                    tc::mbar_arrive(kv ? bar_v_full(st) : bar_k_full(st));
+                    tc::mbar_arrive(bar_kv_full(st));
                 }
             }
         }
@@ -834,7 +655,6 @@ __global__ void __launch_bounds__(PfCfg<T, D, KVT>::THREADS, 1)
             sl2 *= __uint_as_float((uint32_t)(127 - e) << 23);
         }
         float m_ref = -CUDART_INF_F, l = 0.f;
-        int vE = -1000;     // bf16 caches: largest V exponent k so far (O holds sum p V 2^-vE)
         bool ok = true;
         for (int j = 0; j < nt; ++j) {
             ok = __all_sync(tc::kFull, tc::wait_phase(bar_s_full(t, j & 1), (j >> 1) & 1, abort_flag, p.err));
@@ -865,40 +685,27 @@ __global__ void __launch_bounds__(PfCfg<T, D, KVT>::THREADS, 1)
             }
             const float nmb = m_ref == -CUDART_INF_F ? 0.f : -m_ref;
             l *= alpha;
-            // bf16 caches: this tile's V is V 2^-k in f16; P gets 2^(k - vE) so
-            // that O keeps sum p V 2^-vE; a larger k rescales O by 2^(vE - k)
-            float oalpha = alpha, pscale = 1.f;
-            bool vgrow = false;
-            if constexpr (C::VCONV) {
-                const int st = j % C::ST;
-                ok = __all_sync(tc::kFull, tc::wait_phase(bar_v_ready(st), (j / C::ST) & 1, abort_flag, p.err));
-                if (!ok) break;
-                const int k = vexp[st];
-                if (k > vE) {
-                    if (j > 0) oalpha *= ldexpf(1.f, vE - k < -126 ? -126 : vE - k);
-                    vgrow = j > 0;
-                    vE = k;
-                }
-                pscale = ldexpf(1.f, k - vE < -126 ? -126 : k - vE);  // <= 1, exact
-            }
             float ps[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
             for (int c0 = 0; c0 < C::BN; c0 += 32) {
-                uint32_t ph[16];
+                uint32_t hi[16], lo[16];
 #pragma unroll
                 for (int i = 0; i < 16; ++i) {
                     const float p0 = ex2(fmaf(__uint_as_float(sv[c0 + 2 * i]), sl2, nmb));
                     const float p1 = ex2(fmaf(__uint_as_float(sv[c0 + 2 * i + 1]), sl2, nmb));
                     ps[i & 3] += p0 + p1;
-                    if (C::VCONV && pscale != 1.f)
-                        ph[i] = tc::pack2(p0 * pscale, p1 * pscale, f16_t{});
-                    else
-                        ph[i] = tc::pack2(p0, p1, f16_t{});
+                    hi[i] = tc::pack2(p0, p1, OpT{});
+                    if constexpr (C::HILO) {
+                        float h0, h1;
+                        tc::unpack2(hi[i], h0, h1, bf16_t{});
+                        lo[i] = tc::pack2(p0 - h0, p1 - h1, OpT{});
+                    }
                 }
-                tc::st16(scol + c0 / 2, ph);
+                tc::st16(scol + c0 / 2, hi);
+                if constexpr (C::HILO) tc::st16(scol + C::BN / 2 + c0 / 2, lo);
             }
             l += (ps[0] + ps[1]) + (ps[2] + ps[3]);
-            if (j > 0 && (vgrow || __any_sync(tc::kFull, grow))) {
+            if (j > 0 && __any_sync(tc::kFull, grow)) {
                 // O may be rescaled only once the previous P.V of this tile is
                 // complete (the earlier ones completed before it)
                 ok = __all_sync(tc::kFull, tc::wait_phase(bar_pv(t, (j - 1) & 1), ((j - 1) >> 1) & 1,
@@ -912,7 +719,7 @@ __global__ void __launch_bounds__(PfCfg<T, D, KVT>::THREADS, 1)
                         tc::ld32(ocol + c, o);
                         tc::wait_ld<32>(o);
 #pragma unroll
-                        for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * oalpha);
+                        for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
                         tc::st32(ocol + c, o);
                     }
                 }
@@ -928,9 +735,7 @@ __global__ void __launch_bounds__(PfCfg<T, D, KVT>::THREADS, 1)
             // ---- epilogue: out = O / l, rounded once to the q dtype ----------------
             // (shared-prefix mode: the partial o / l and its log-sum-exp, fp32)
             tc::fence_after();
-            // v_scale: 1 for 16-bit caches; bf16 caches: O holds sum p V 2^-vE
-            float inv = l > 0.f ? p.v_scale / l : 0.f;
-            if (C::VCONV && nt > 0) inv *= ldexpf(1.f, vE);
+            const float inv = l > 0.f ? p.v_scale / l : 0.f;  // v_scale: 1 for 16-bit caches
             const int64_t row = ((int64_t)(q0 + tok0 + rtok) * p.num_q_heads + (int64_t)kvh * g + r % g);
             uint4 *dst = reinterpret_cast<uint4 *>(static_cast<uint16_t *>(p.out) + row * D);
             if (!causal) {
