@@ -392,6 +392,10 @@ __global__ void __launch_bounds__(PfCfg<T, D, KVT>::THREADS, 1)
 
     if (warp == 8) {
         // ================= TMA producer ===========================================
+        // Lane 0 issues the copies.  The whole warp holds the pool rows of the
+        // 16-token tiles: lane i the row of tile 32 b + i of the current batch b
+        // and of the next one, read a batch ahead, so no copy waits on a
+        // block-table load.
         if (lane == 0) {
             asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_q)) : "memory");
             asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_k)) : "memory");
@@ -403,45 +407,64 @@ __global__ void __launch_bounds__(PfCfg<T, D, KVT>::THREADS, 1)
                 for (int a = 0; a < C::ATOMS; ++a)
                     tc::tma_load_3d(q_smem(t) + a * C::BM * 128, &tmap_q, a * 64, kvh * g,
                                     q0 + tok0 + t * tpt, bar_q);
-            const int32_t *bt = p.block_tables + (int64_t)s * p.max_blocks_per_seq;
-            auto row_of = [&](int lb) -> int {  // pool row of 16-token tile lb (past the pool: zeros)
-                int y = p.oob_row;
-                if (lb < nblk_seq) {
-                    const int phys = bt[lb >> p.tile_shift];
-                    if ((unsigned)phys < (unsigned)p.num_blocks)
-                        y = (phys * p.num_kv_heads + kvh) * p.block_size + (lb & tile_mask) * kBlockSize;
-                    else
-                        flag_error(p.err, kErrBounds);
-                }
-                return y;
-            };
-            constexpr int RING = C::KV8 ? C::SST : C::ST;  // the ring the copies land in
-            auto full_bar = [&](int st) { return C::KV8 ? bar_stg_full(st) : bar_kv_full(st); };
-            auto empty_bar = [&](int st) { return C::KV8 ? bar_stg_empty(st) : bar_kv_empty(st); };
-            int j = 0;
-            for (; j < nt; ++j) {
-                const int st = j % RING;
-                if (j >= RING && !tc::wait_phase(empty_bar(st), ((j / RING) - 1) & 1, abort_flag, p.err))
-                    break;
+        }
+        const int32_t *bt = p.block_tables + (int64_t)s * p.max_blocks_per_seq;
+        constexpr int TPK = C::BN / kBlockSize;  // 16-token tiles per key tile
+        static_assert(32 % TPK == 0, "a batch of 32 tiles holds whole key tiles");
+        const int tile0 = j0 * TPK, ntiles = nt * TPK;
+        auto rows_of_batch = [&](int batch) -> int {  // pool row of this lane's tile (past the pool: zeros)
+            const int i = batch * 32 + lane, lb = tile0 + i;
+            int y = p.oob_row;
+            if (i < ntiles && lb < nblk_seq) {
+                const int phys = bt[lb >> p.tile_shift];
+                if ((unsigned)phys < (unsigned)p.num_blocks)
+                    y = (phys * p.num_kv_heads + kvh) * p.block_size + (lb & tile_mask) * kBlockSize;
+                else
+                    flag_error(p.err, kErrBounds);
+            }
+            return y;
+        };
+        int rows_cur = rows_of_batch(0), rows_nxt = ntiles > 32 ? rows_of_batch(1) : p.oob_row;
+        int cur_batch = 0;
+        constexpr int RING = C::KV8 ? C::SST : C::ST;  // the ring the copies land in
+        auto full_bar = [&](int st) { return C::KV8 ? bar_stg_full(st) : bar_kv_full(st); };
+        auto empty_bar = [&](int st) { return C::KV8 ? bar_stg_empty(st) : bar_kv_empty(st); };
+        int j = 0;
+        for (; j < nt; ++j) {
+            const int st = j % RING;
+            if (j >= RING) {
+                int ok = lane == 0 ? (int)tc::wait_phase(empty_bar(st), ((j / RING) - 1) & 1, abort_flag, p.err) : 0;
+                if (!__shfl_sync(tc::kFull, ok, 0)) break;
+            }
+            if ((j * TPK) >> 5 != cur_batch) {  // uniform: the next batch becomes current
+                rows_cur = rows_nxt;
+                ++cur_batch;
+                rows_nxt = (cur_batch + 1) * 32 < ntiles ? rows_of_batch(cur_batch + 1) : p.oob_row;
+            }
+            int y[TPK];
+#pragma unroll
+            for (int b = 0; b < TPK; ++b) y[b] = __shfl_sync(tc::kFull, rows_cur, (j * TPK + b) & 31);
+            if (lane == 0) {
                 mbar_arrive_expect_tx(full_bar(st), C::KV8 ? 2u * C::KV8_BYTES : 2u * C::KV_BYTES);
-#pragma unroll 1
-                for (int b = 0; b < C::BN / kBlockSize; ++b) {
-                    const int y = row_of((j0 + j) * (C::BN / kBlockSize) + b);
+#pragma unroll
+                for (int b = 0; b < TPK; ++b) {
                     if constexpr (C::KV8) {  // 16 rows x 128 codes, 128B swizzle
                         const uint32_t off = b * kBlockSize * 128;
-                        tc::tma_load_2d(stg_k(st) + off, &tmap_k, 0, y, full_bar(st));
-                        tc::tma_load_2d(stg_v(st) + off, &tmap_v, 0, y, full_bar(st));
+                        tc::tma_load_2d(stg_k(st) + off, &tmap_k, 0, y[b], full_bar(st));
+                        tc::tma_load_2d(stg_v(st) + off, &tmap_v, 0, y[b], full_bar(st));
                     } else {
 #pragma unroll
                         for (int a = 0; a < C::ATOMS; ++a) {
                             const uint32_t off = a * C::BN * 128 + b * kBlockSize * 128;
-                            tc::tma_load_2d(k_smem(st) + off, &tmap_k, a * 64, y, full_bar(st));
-                            tc::tma_load_2d(v_smem(st) + off, &tmap_v, a * 64, y, full_bar(st));
+                            tc::tma_load_2d(k_smem(st) + off, &tmap_k, a * 64, y[b], full_bar(st));
+                            tc::tma_load_2d(v_smem(st) + off, &tmap_v, a * 64, y[b], full_bar(st));
                         }
                     }
                 }
             }
-            // nothing may still be landing in shared memory when the CTA exits
+        }
+        // nothing may still be landing in shared memory when the CTA exits
+        if (lane == 0) {
             (void)mbar_wait_bounded(bar_q, 0, kWaitLimitNs);
             for (int jj = j - RING < 0 ? 0 : j - RING; jj < j; ++jj)
                 (void)mbar_wait_bounded(full_bar(jj % RING), (jj / RING) & 1, kWaitLimitNs);
@@ -449,88 +472,86 @@ __global__ void __launch_bounds__(PfCfg<T, D, KVT>::THREADS, 1)
         __syncwarp();
     } else if (warp == 9) {
         // ================= MMA issuer ==============================================
-        // order per key tile j: PV_A(j), QK_A(j+2), PV_B(j), QK_B(j+2) -- each
+        // One lane does all of it (waits included), so nothing between two MMA
+        // groups waits on the rest of the warp; the shared-memory descriptors
+        // are formed once and stepped by constant offsets.
+        // Order per key tile j: PV_A(j), QK_A(j+2), PV_B(j), QK_B(j+2) -- each
         // tile's scores are computed two key tiles ahead into its other S
-        // buffer, and the two query tiles ping-pong on the tensor cores
-        auto issue_qk = [&](int t, int j) {
-            const uint32_t kaddr = k_smem(j % C::ST), qaddr = q_smem(t);
-            const uint32_t d = tmem + s_col(t, j & 1);
-            if (lane == 0) {
+        // buffer, and the two query tiles ping-pong on the tensor cores.
+        if (lane == 0) {
+            const uint64_t qdesc = tc::sdesc(q_smem(0), 16, 1024);
+            const uint64_t kdesc = tc::sdesc(k_smem(0), 16, 1024);
+            const uint64_t vdesc = tc::sdesc(v_smem(0), C::BN * 128, 1024);
+            auto issue_qk = [&](int t, int j) {
+                const uint64_t qd = qdesc + (uint64_t)((t * C::Q_BYTES) >> 4);
+                const uint64_t kd = kdesc + (uint64_t)(((j % C::ST) * 2 * C::KV_BYTES) >> 4);
+                const uint32_t d = tmem + s_col(t, j & 1);
                 tc::fence_after();
 #pragma unroll
                 for (int ks = 0; ks < D / 16; ++ks) {
                     const uint32_t in_atom = (ks & 3) * 32;
-                    tc::mma_ss(d, tc::sdesc(qaddr + (ks >> 2) * (C::BM * 128) + in_atom, 16, 1024),
-                               tc::sdesc(kaddr + (ks >> 2) * (C::BN * 128) + in_atom, 16, 1024),
-                               C::IDESC_QK, ks > 0);
+                    tc::mma_ss(d, qd + (uint64_t)(((ks >> 2) * (C::BM * 128) + in_atom) >> 4),
+                               kd + (uint64_t)(((ks >> 2) * (C::BN * 128) + in_atom) >> 4), C::IDESC_QK, ks > 0);
                 }
                 tc::commit(bar_s_full(t, j & 1));
-            }
-            __syncwarp();
-        };
-        auto issue_pv = [&](int t, int j) {
-            const uint32_t vaddr = v_smem(j % C::ST);
-            const uint32_t pcol = tmem + s_col(t, j & 1);
-            const uint32_t ocol = tmem + C::COL_O + 128u * t;
-            if (lane == 0) {
+            };
+            auto issue_pv = [&](int t, int j) {
+                const uint64_t vd = vdesc + (uint64_t)(((j % C::ST) * 2 * C::KV_BYTES) >> 4);
+                const uint32_t pcol = tmem + s_col(t, j & 1);
+                const uint32_t ocol = tmem + C::COL_O + 128u * t;
                 tc::fence_after();
 #pragma unroll
                 for (int ks = 0; ks < C::BN / 16; ++ks) {
-                    const uint64_t bdesc = tc::sdesc(vaddr + ks * 2048, C::BN * 128, 1024);
-                    tc::mma_ts(ocol, pcol + ks * 8, bdesc, C::IDESC_PV, (j > 0 || ks > 0));
-                    if constexpr (C::HILO)
-                        tc::mma_ts(ocol, pcol + C::BN / 2 + ks * 8, bdesc, C::IDESC_PV, 1);
+                    const uint64_t bd = vd + (uint64_t)((ks * 2048) >> 4);
+                    tc::mma_ts(ocol, pcol + ks * 8, bd, C::IDESC_PV, (j > 0 || ks > 0));
+                    if constexpr (C::HILO) tc::mma_ts(ocol, pcol + C::BN / 2 + ks * 8, bd, C::IDESC_PV, 1);
                 }
                 tc::commit(bar_pv(t, j & 1));
                 if (t == 1) tc::commit(bar_kv_empty(j % C::ST));  // last reader of the stage
-            }
-            __syncwarp();
-        };
-        auto wait_all = [&](uint32_t bar, uint32_t parity) {
-            return __all_sync(tc::kFull, tc::wait_phase(bar, parity, abort_flag, p.err));
-        };
-        const int j_tail = (L & (kBlockSize - 1)) ? (nblk_seq - 1) / (C::BN / kBlockSize) : -1;
-        auto kv_ready = [&](int j) {
-            const int st = j % C::ST;
-            if (!wait_all(bar_kv_full(st), (j / C::ST) & 1)) return false;
-            if (j0 + j == j_tail) {
-                // clear the V rows of the last block's unused slots (positions >= L)
-                const int r0 = L - (j0 + j) * C::BN, r1 = nblk_seq * kBlockSize - (j0 + j) * C::BN;
-                const int chunks = (r1 - r0) * C::ATOMS * 8;
-                for (int c = lane; c < chunks; c += 32) {
-                    const int row = r0 + c / (C::ATOMS * 8), rem = c % (C::ATOMS * 8);
-                    const uint32_t addr = v_smem(st) + (rem >> 3) * C::BN * 128 + row * 128 + (rem & 7) * 16;
-                    asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(addr), "r"(0u) : "memory");
+            };
+            auto wait1 = [&](uint32_t bar, uint32_t parity) {
+                return tc::wait_phase(bar, parity, abort_flag, p.err);
+            };
+            const int j_tail = (L & (kBlockSize - 1)) ? (nblk_seq - 1) / (C::BN / kBlockSize) : -1;
+            auto kv_ready = [&](int j) {
+                const int st = j % C::ST;
+                if (!wait1(bar_kv_full(st), (j / C::ST) & 1)) return false;
+                if (j0 + j == j_tail) {
+                    // clear the V rows of the last block's unused slots (positions >= L)
+                    const int r0 = L - (j0 + j) * C::BN, r1 = nblk_seq * kBlockSize - (j0 + j) * C::BN;
+                    const int chunks = (r1 - r0) * C::ATOMS * 8;
+                    for (int c = 0; c < chunks; ++c) {
+                        const int row = r0 + c / (C::ATOMS * 8), rem = c % (C::ATOMS * 8);
+                        const uint32_t addr = v_smem(st) + (rem >> 3) * C::BN * 128 + row * 128 + (rem & 7) * 16;
+                        asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(addr), "r"(0u) : "memory");
+                    }
+                    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
                 }
-                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-                __syncwarp();
-            }
-            return true;
-        };
-        bool ok = wait_all(C::KV8 ? bar_q_ready : bar_q, 0);  // 8-bit caches: q converted
-        for (int j = 0; ok && j < 2 && j < nt; ++j) {
-            ok = kv_ready(j);
-            if (!ok) break;
-            issue_qk(0, j);
-            issue_qk(1, j);
-        }
-        for (int j = 0; ok && j < nt; ++j) {
-            ok = wait_all(bar_p_full(0, j & 1), (j >> 1) & 1);
-            if (!ok) break;
-            issue_pv(0, j);
-            const bool more = j + 2 < nt;
-            if (more) {
-                ok = kv_ready(j + 2);
+                return true;
+            };
+            bool ok = wait1(C::KV8 ? bar_q_ready : bar_q, 0);  // 8-bit caches: q converted
+            for (int j = 0; ok && j < 2 && j < nt; ++j) {
+                ok = kv_ready(j);
                 if (!ok) break;
-                issue_qk(0, j + 2);
+                issue_qk(0, j);
+                issue_qk(1, j);
             }
-            ok = wait_all(bar_p_full(1, j & 1), (j >> 1) & 1);
-            if (!ok) break;
-            issue_pv(1, j);
-            if (more) issue_qk(1, j + 2);
-        }
-        // every MMA of this thread must be complete before TMEM is freed
-        if (lane == 0) {
+            for (int j = 0; ok && j < nt; ++j) {
+                ok = wait1(bar_p_full(0, j & 1), (j >> 1) & 1);
+                if (!ok) break;
+                issue_pv(0, j);
+                const bool more = j + 2 < nt;
+                if (more) {
+                    ok = kv_ready(j + 2);
+                    if (!ok) break;
+                    issue_qk(0, j + 2);
+                }
+                ok = wait1(bar_p_full(1, j & 1), (j >> 1) & 1);
+                if (!ok) break;
+                issue_pv(1, j);
+                if (more) issue_qk(1, j + 2);
+            }
+            // every MMA of this thread must be complete before TMEM is freed
             tc::commit(bar_drain);
             (void)mbar_wait_bounded(bar_drain, 0, kWaitLimitNs);
         }
