@@ -441,25 +441,23 @@ __global__ void __launch_bounds__(PfCfg<T, D, KVT>::THREADS, 1)
                 ++cur_batch;
                 rows_nxt = (cur_batch + 1) * 32 < ntiles ? rows_of_batch(cur_batch + 1) : p.oob_row;
             }
-            int y[TPK];
-#pragma unroll
-            for (int b = 0; b < TPK; ++b) y[b] = __shfl_sync(tc::kFull, rows_cur, (j * TPK + b) & 31);
-            if (lane == 0) {
+            // one copy per lane: lane l takes block l % TPK of the key tile, then
+            // (16-bit caches) atom l / TPK % ATOMS, K for l < NCOPY / 2 and V after
+            const int y = __shfl_sync(tc::kFull, rows_cur, (j * TPK + lane % TPK) & 31);
+            if (lane == 0)
                 mbar_arrive_expect_tx(full_bar(st), C::KV8 ? 2u * C::KV8_BYTES : 2u * C::KV_BYTES);
-#pragma unroll
-                for (int b = 0; b < TPK; ++b) {
-                    if constexpr (C::KV8) {  // 16 rows x 128 codes, 128B swizzle
-                        const uint32_t off = b * kBlockSize * 128;
-                        tc::tma_load_2d(stg_k(st) + off, &tmap_k, 0, y[b], full_bar(st));
-                        tc::tma_load_2d(stg_v(st) + off, &tmap_v, 0, y[b], full_bar(st));
-                    } else {
-#pragma unroll
-                        for (int a = 0; a < C::ATOMS; ++a) {
-                            const uint32_t off = a * C::BN * 128 + b * kBlockSize * 128;
-                            tc::tma_load_2d(k_smem(st) + off, &tmap_k, a * 64, y[b], full_bar(st));
-                            tc::tma_load_2d(v_smem(st) + off, &tmap_v, a * 64, y[b], full_bar(st));
-                        }
-                    }
+            __syncwarp();
+            constexpr int NCOPY = 2 * TPK * (C::KV8 ? 1 : C::ATOMS);
+            static_assert(NCOPY <= 32, "one copy per lane");
+            if (lane < NCOPY) {
+                const int b = lane % TPK, is_v = lane >= NCOPY / 2;
+                if constexpr (C::KV8) {  // 16 rows x 128 codes, 128B swizzle
+                    const uint32_t dst = (is_v ? stg_v(st) : stg_k(st)) + b * kBlockSize * 128;
+                    tc::tma_load_2d(dst, is_v ? &tmap_v : &tmap_k, 0, y, full_bar(st));
+                } else {
+                    const int a = (lane / TPK) % C::ATOMS;
+                    const uint32_t dst = (is_v ? v_smem(st) : k_smem(st)) + a * C::BN * 128 + b * kBlockSize * 128;
+                    tc::tma_load_2d(dst, is_v ? &tmap_v : &tmap_k, a * 64, y, full_bar(st));
                 }
             }
         }
