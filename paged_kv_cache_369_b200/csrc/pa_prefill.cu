@@ -245,12 +245,14 @@ template <typename T, int D, typename KVT = T> struct PfCfg {
     static constexpr int OFF_STG = OFF_KV + ST * 2 * KV_BYTES;  // 8-bit stage: K, then V
     static constexpr int OFF_BAR = OFF_STG + SST * 2 * KV8_BYTES;
     // q_full, kv_full[ST], kv_empty[ST], then per (tile, score buffer):
-    // s_full, p_full, pv_done; drain; q_ready, stg_full[SST], stg_empty[SST]
-    static constexpr int NBAR = 1 + 2 * ST + 4 + 4 + 4 + 1 + 1 + 2 * SST;
+    // s_full, p_full, pv_done; drain; q_ready, stg_full[SST], stg_empty[SST];
+    // drain of the second MMA issuer; tail cleared
+    static constexpr int NBAR = 1 + 2 * ST + 4 + 4 + 4 + 1 + 1 + 2 * SST + 2;
     static constexpr int OFF_SLOT = OFF_BAR + NBAR * 8;
     static constexpr int OFF_ABORT = OFF_SLOT + 4;
     static constexpr int OFF_QEXP = OFF_ABORT + 4;    // log2 of the q scaling (8-bit caches)
-    static constexpr int USED = OFF_QEXP + 4;
+    static constexpr int OFF_TAIL = OFF_QEXP + 4;     // the tail of V has been claimed for clearing
+    static constexpr int USED = OFF_TAIL + 4;
     // at least 120 KiB so that one CTA holds an SM (and its 512 TMEM columns)
     static constexpr int SMEM = 1024 + (USED < 120 * 1024 ? 120 * 1024 : USED);
     // MMA operand type: T, or f16 for 8-bit caches (codes widen to f16 exactly)
@@ -266,10 +268,11 @@ template <typename T, int D, typename KVT = T> struct PfCfg {
                                          ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
     static constexpr uint32_t IDESC_PV = (1u << 4) | (FMT << 7) | (FMT << 10) | (1u << 16) |
                                          ((uint32_t)(D >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
-    // 8 softmax warps, a TMA warp, an MMA warp (+ two converter warps, K and V,
-    // for 8-bit caches)
+    // 8 softmax warps, a TMA warp, an MMA warp per query tile (9 for A and
+    // MMA_B for B), + two converter warps (K and V) for 8-bit caches
     static constexpr int CONVERTERS = KV8 ? 2 : 0;
-    static constexpr int THREADS = 320 + 32 * CONVERTERS;
+    static constexpr int MMA_B = 10 + CONVERTERS;
+    static constexpr int THREADS = 352 + 32 * CONVERTERS;
     static_assert(D == 64 || D == 128, "head_dim 64 or 128");
     static_assert(!KV8 || D == 128, "8-bit caches: head_dim 128");
     static_assert(ST >= 3, "two key tiles of look-ahead plus the one in PV");
@@ -349,6 +352,8 @@ __global__ void __launch_bounds__(PfCfg<T, D, KVT>::THREADS, 1)
     const uint32_t bar_q_ready = bars + 8u * (14 + 2 * C::ST);
     auto bar_stg_full = [&](int st) { return bars + 8u * (15 + 2 * C::ST + st); };
     auto bar_stg_empty = [&](int st) { return bars + 8u * (15 + 2 * C::ST + C::SST + st); };
+    const uint32_t bar_drain_b = bars + 8u * (15 + 2 * C::ST + 2 * C::SST);
+    const uint32_t bar_tail = bars + 8u * (16 + 2 * C::ST + 2 * C::SST);
     auto s_col = [&](int t, int b) { return C::COL_S + 64u * (2 * t + b); };
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + C::OFF_ABORT);
     uint32_t *slot = reinterpret_cast<uint32_t *>(smem + C::OFF_SLOT);
@@ -358,7 +363,7 @@ __global__ void __launch_bounds__(PfCfg<T, D, KVT>::THREADS, 1)
 #pragma unroll
         for (int st = 0; st < C::ST; ++st) {
             mbar_init(bar_kv_full(st), C::KV8 ? C::CONVERTERS : 1);  // TMA, or the converters
-            mbar_init(bar_kv_empty(st), 1);
+            mbar_init(bar_kv_empty(st), 2);  // both MMA issuers
         }
 #pragma unroll
         for (int t = 0; t < 2; ++t)
@@ -369,6 +374,9 @@ __global__ void __launch_bounds__(PfCfg<T, D, KVT>::THREADS, 1)
                 mbar_init(bar_pv(t, b), 1);
             }
         mbar_init(bar_drain, 1);
+        mbar_init(bar_drain_b, 1);
+        mbar_init(bar_tail, 1);
+        *reinterpret_cast<volatile int *>(smem + C::OFF_TAIL) = 0;
         mbar_init(bar_q_ready, 1);
 #pragma unroll
         for (int st = 0; st < C::SST; ++st) {
@@ -468,20 +476,24 @@ __global__ void __launch_bounds__(PfCfg<T, D, KVT>::THREADS, 1)
                 (void)mbar_wait_bounded(full_bar(jj % RING), (jj / RING) & 1, kWaitLimitNs);
         }
         __syncwarp();
-    } else if (warp == 9) {
-        // ================= MMA issuer ==============================================
-        // One lane does all of it (waits included), so nothing between two MMA
-        // groups waits on the rest of the warp; the shared-memory descriptors
-        // are formed once and stepped by constant offsets.
-        // Order per key tile j: PV_A(j), QK_A(j+2), PV_B(j), QK_B(j+2) -- each
-        // tile's scores are computed two key tiles ahead into its other S
-        // buffer, and the two query tiles ping-pong on the tensor cores.
+    } else if (warp == 9 || warp == C::MMA_B) {
+        // ================= MMA issuers ============================================
+        // One per query tile (warp 9: A, warp MMA_B: B), so that while one waits
+        // for its softmax the other keeps the tensor core fed; one lane of each
+        // does all of it, and the shared-memory descriptors are formed once
+        // and stepped by constant offsets.  Order per key tile j: PV_t(j),
+        // QK_t(j+2) -- the tile's scores are computed two key tiles ahead into
+        // its other S buffer; tcgen05 operations of one thread run in issue
+        // order, which makes reusing a score buffer's columns for P and then
+        // for the scores two tiles later safe.  A K/V stage is free once both
+        // issuers' P.V of it is done (kv_empty counts two commits).
+        const int t = warp == 9 ? 0 : 1;
         if (lane == 0) {
-            const uint64_t qdesc = tc::sdesc(q_smem(0), 16, 1024);
+            const uint64_t qd = tc::sdesc(q_smem(t), 16, 1024);
             const uint64_t kdesc = tc::sdesc(k_smem(0), 16, 1024);
             const uint64_t vdesc = tc::sdesc(v_smem(0), C::BN * 128, 1024);
-            auto issue_qk = [&](int t, int j) {
-                const uint64_t qd = qdesc + (uint64_t)((t * C::Q_BYTES) >> 4);
+            const uint32_t ocol = tmem + C::COL_O + 128u * t;
+            auto issue_qk = [&](int j) {
                 const uint64_t kd = kdesc + (uint64_t)(((j % C::ST) * 2 * C::KV_BYTES) >> 4);
                 const uint32_t d = tmem + s_col(t, j & 1);
                 tc::fence_after();
@@ -493,10 +505,9 @@ __global__ void __launch_bounds__(PfCfg<T, D, KVT>::THREADS, 1)
                 }
                 tc::commit(bar_s_full(t, j & 1));
             };
-            auto issue_pv = [&](int t, int j) {
+            auto issue_pv = [&](int j) {
                 const uint64_t vd = vdesc + (uint64_t)(((j % C::ST) * 2 * C::KV_BYTES) >> 4);
                 const uint32_t pcol = tmem + s_col(t, j & 1);
-                const uint32_t ocol = tmem + C::COL_O + 128u * t;
                 tc::fence_after();
 #pragma unroll
                 for (int ks = 0; ks < C::BN / 16; ++ks) {
@@ -505,17 +516,22 @@ __global__ void __launch_bounds__(PfCfg<T, D, KVT>::THREADS, 1)
                     if constexpr (C::HILO) tc::mma_ts(ocol, pcol + C::BN / 2 + ks * 8, bd, C::IDESC_PV, 1);
                 }
                 tc::commit(bar_pv(t, j & 1));
-                if (t == 1) tc::commit(bar_kv_empty(j % C::ST));  // last reader of the stage
+                tc::commit(bar_kv_empty(j % C::ST));  // this issuer's last read of the stage
             };
             auto wait1 = [&](uint32_t bar, uint32_t parity) {
                 return tc::wait_phase(bar, parity, abort_flag, p.err);
             };
-            const int j_tail = (L & (kBlockSize - 1)) ? (nblk_seq - 1) / (C::BN / kBlockSize) : -1;
-            auto kv_ready = [&](int j) {
-                const int st = j % C::ST;
-                if (!wait1(bar_kv_full(st), (j / C::ST) & 1)) return false;
-                if (j0 + j == j_tail) {
-                    // clear the V rows of the last block's unused slots (positions >= L)
+            auto kv_ready = [&](int j) { return wait1(bar_kv_full(j % C::ST), (j / C::ST) & 1); };
+            const int j_tail = (L & (kBlockSize - 1)) ? (nblk_seq - 1) / (C::BN / kBlockSize) - j0 : -1;
+            // Before P.V of the key tile holding the sequence's last block: the
+            // V rows of its unused slots (positions >= L) are cleared (p = 0
+            // there, but 0 x NaN poison = NaN).  The first issuer to get there
+            // clears them (its Q.K^T of the tile came after the copies landed),
+            // the other waits until it is done.
+            auto tail_ready = [&](int j) {
+                if (j != j_tail) return true;
+                if (atomicCAS(reinterpret_cast<int *>(smem + C::OFF_TAIL), 0, 1) == 0) {
+                    const int st = j % C::ST;
                     const int r0 = L - (j0 + j) * C::BN, r1 = nblk_seq * kBlockSize - (j0 + j) * C::BN;
                     const int chunks = (r1 - r0) * C::ATOMS * 8;
                     for (int c = 0; c < chunks; ++c) {
@@ -524,37 +540,33 @@ __global__ void __launch_bounds__(PfCfg<T, D, KVT>::THREADS, 1)
                         asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(addr), "r"(0u) : "memory");
                     }
                     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                    tc::mbar_arrive(bar_tail);
                 }
-                return true;
+                return wait1(bar_tail, 0);
             };
             bool ok = wait1(C::KV8 ? bar_q_ready : bar_q, 0);  // 8-bit caches: q converted
             for (int j = 0; ok && j < 2 && j < nt; ++j) {
                 ok = kv_ready(j);
                 if (!ok) break;
-                issue_qk(0, j);
-                issue_qk(1, j);
+                issue_qk(j);
             }
             for (int j = 0; ok && j < nt; ++j) {
-                ok = wait1(bar_p_full(0, j & 1), (j >> 1) & 1);
+                ok = wait1(bar_p_full(t, j & 1), (j >> 1) & 1) && tail_ready(j);
                 if (!ok) break;
-                issue_pv(0, j);
-                const bool more = j + 2 < nt;
-                if (more) {
+                issue_pv(j);
+                if (j + 2 < nt) {
                     ok = kv_ready(j + 2);
                     if (!ok) break;
-                    issue_qk(0, j + 2);
+                    issue_qk(j + 2);
                 }
-                ok = wait1(bar_p_full(1, j & 1), (j >> 1) & 1);
-                if (!ok) break;
-                issue_pv(1, j);
-                if (more) issue_qk(1, j + 2);
             }
             // every MMA of this thread must be complete before TMEM is freed
-            tc::commit(bar_drain);
-            (void)mbar_wait_bounded(bar_drain, 0, kWaitLimitNs);
+            const uint32_t drain = t == 0 ? bar_drain : bar_drain_b;
+            tc::commit(drain);
+            (void)mbar_wait_bounded(drain, 0, kWaitLimitNs);
         }
         __syncwarp();
-    } else if (warp >= 10) {
+    } else if (warp >= 10 && warp < 10 + C::CONVERTERS) {
         // ================= converters (8-bit caches only) ===========================
         // warp 10 widens q (bf16 -> f16, scaled by a power of two so its
         // largest magnitude sits near 2^14; the inverse folds into the logit
