@@ -270,6 +270,12 @@ pa_status pa_decode_split_reduce(void *out, const void *q, const void *k_cache,
  * than its sequence or than max_query_len, a length past the table, or a
  * table entry outside the pool flags PA_ERR_DEVICE_BOUNDS (that sequence's
  * rows are then not written, or the bad block reads as zeros).
+ *
+ * The launch is persistent (one CTA per SM taking work items from a device
+ * counter inside the library).  The library keeps 64 such counters and gives
+ * each launch the next one in turn, so at most 64 pa_prefill or
+ * pa_decode_shared_prefix launches may be in flight at the same time (on
+ * different streams); a launch resets its counter when it finishes.
  */
 pa_status pa_prefill(void *out, const void *q, const void *k_cache, const void *v_cache,
                      const int32_t *block_tables, int max_blocks_per_seq, const int32_t *seq_lens,

@@ -168,6 +168,12 @@ struct PrefillParams {  // chunked prefill (pa_prefill)
     float *ws_o;
     float *ws_lse;
     int ws_np;
+    // set by the launch: the work items are items_x (query tile pairs) x
+    // num_kv_heads x items_z (sequences, or prefix key ranges), and
+    // work_slot names the launch's work counter
+    int items_x;
+    int items_z;
+    int work_slot;
 };
 
 struct ReduceParams {

@@ -52,6 +52,8 @@
 #include <cuda.h>
 #include <math_constants.h>
 
+#include <atomic>
+#include <cstdint>
 #include <type_traits>
 
 #include "pa_device.cuh"
@@ -246,13 +248,15 @@ template <typename T, int D, typename KVT = T> struct PfCfg {
     static constexpr int OFF_BAR = OFF_STG + SST * 2 * KV8_BYTES;
     // q_full, kv_full[ST], kv_empty[ST], then per (tile, score buffer):
     // s_full, p_full, pv_done; drain; q_ready, stg_full[SST], stg_empty[SST];
-    // drain of the second MMA issuer; tail cleared
-    static constexpr int NBAR = 1 + 2 * ST + 4 + 4 + 4 + 1 + 1 + 2 * SST + 2;
+    // drain of the second MMA issuer; tail cleared; q_empty; o_free[2];
+    // item_full[2], item_empty[2]
+    static constexpr int NBAR = 1 + 2 * ST + 4 + 4 + 4 + 1 + 1 + 2 * SST + 2 + 7;
     static constexpr int OFF_SLOT = OFF_BAR + NBAR * 8;
     static constexpr int OFF_ABORT = OFF_SLOT + 4;
-    static constexpr int OFF_QEXP = OFF_ABORT + 4;    // log2 of the q scaling (8-bit caches)
-    static constexpr int OFF_TAIL = OFF_QEXP + 4;     // the tail of V has been claimed for clearing
-    static constexpr int USED = OFF_TAIL + 4;
+    static constexpr int OFF_QEXP = OFF_ABORT + 4;    // log2 of the q scaling, per item parity (8-bit caches)
+    static constexpr int OFF_TAIL = OFF_QEXP + 8;     // tails of V claimed for clearing so far
+    static constexpr int OFF_ITEM = OFF_TAIL + 4;     // the item ring's two slots
+    static constexpr int USED = OFF_ITEM + 8;
     // at least 120 KiB so that one CTA holds an SM (and its 512 TMEM columns)
     static constexpr int SMEM = 1024 + (USED < 120 * 1024 ? 120 * 1024 : USED);
     // MMA operand type: T, or f16 for 8-bit caches (codes widen to f16 exactly)
@@ -285,6 +289,63 @@ __device__ __forceinline__ float ex2(float x) {  // 2^x; -inf -> +0
     return y;
 }
 
+// Work-item counters of the persistent launch: [next item, CTAs finished] per
+// slot.  The host gives each launch the next of kWorkSlots slots in turn; the
+// last CTA of a launch to finish resets its slot to zero.
+constexpr int kWorkSlots = 64;
+__device__ unsigned int g_prefill_work[kWorkSlots][2];
+
+// One work item: a (pair of query tiles, KV head, sequence or prefix key range).
+struct PfItem {
+    int kvh, s, split, L, q0, tok0, ntok, ctx, nt, j0, nblk;
+    int state;  // 0: attend; 1: nothing to do; 2: an empty key range (write an empty partial)
+};
+
+template <int BN>
+__device__ __forceinline__ PfItem decode_item(const PrefillParams &p, int item, bool flag_errors) {
+    PfItem w{};
+    const int x = item % p.items_x, rest = item / p.items_x;
+    w.kvh = rest % p.num_kv_heads;
+    const int z = rest / p.num_kv_heads;
+    const bool causal = p.shared_len == 0;
+    w.s = causal ? z : 0;
+    w.split = causal ? 0 : z;
+    w.L = causal ? p.seq_lens[w.s] : p.shared_len;
+    w.q0 = causal ? p.query_start[w.s] : 0;
+    const int n = causal ? p.query_start[w.s + 1] - w.q0 : p.num_tokens;
+    w.state = 1;
+    if (w.L < 0 || w.L > p.max_blocks_per_seq * p.block_size || n < 0 || (causal && n > w.L) || w.q0 < 0 ||
+        w.q0 + n > p.num_tokens || n > p.max_query_len) {
+        if (flag_errors && x == 0 && w.kvh == 0) flag_error(p.err, kErrBounds);
+        return w;
+    }
+    w.tok0 = x * 2 * p.tok_per_tile;  // query tile A: tok0 .., tile B: tok0 + tpt ..
+    if (w.tok0 >= n) return w;
+    w.ntok = min(2 * p.tok_per_tile, n - w.tok0);
+    w.ctx = w.L - n;
+    // key tiles up to the last row's position (all of the prefix without the
+    // mask); shared mode: tiles j0 .. j0 + nt - 1 of the prefix, range z
+    w.nt = causal ? (w.ctx + w.tok0 + w.ntok - 1) / BN + 1 : (w.L + BN - 1) / BN;
+    if (!causal) {
+        const int per = (w.nt + p.items_z - 1) / p.items_z;
+        w.j0 = w.split * per;
+        w.nt = min(per, w.nt - w.j0);
+        if (w.nt <= 0) {  // an empty range (the host never makes one)
+            w.state = 2;
+            return w;
+        }
+    }
+    if (w.nt <= 0) return w;  // an empty prefix
+    w.nblk = (w.L + kBlockSize - 1) / kBlockSize;  // 16-token tiles
+    w.state = 0;
+    return w;
+}
+
+// Persistent: gridDim.x CTAs (one an SM) take work items from the launch's
+// counter until they run out.  The TMA warp takes each item and passes it to
+// the other roles through a two-slot ring in shared memory; every role then
+// runs the item with its barrier phases continuing from the previous one, so
+// one item's loads and first MMAs overlap the previous item's last tiles.
 template <typename T, int D, typename KVT>
 __global__ void __launch_bounds__(PfCfg<T, D, KVT>::THREADS, 1)
     prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tmap_q,
@@ -297,45 +358,9 @@ __global__ void __launch_bounds__(PfCfg<T, D, KVT>::THREADS, 1)
     const uint32_t base = (raw + 1023u) & ~1023u;
     uint8_t *smem = smem_raw + (base - raw);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    // z: the sequence (chunked prefill), or the prefix key range (shared mode)
-    const int cta_tile = blockIdx.x, kvh = blockIdx.y;
-    const int s = p.shared_len > 0 ? 0 : (int)blockIdx.z;
     const int g = p.group, tpt = p.tok_per_tile;
-
-    // ---- this CTA's rows and keys (uniform over the CTA) ---------------------
     const bool causal = p.shared_len == 0;
-    const int L = causal ? p.seq_lens[s] : p.shared_len;
-    const int q0 = causal ? p.query_start[s] : 0;
-    const int n = causal ? p.query_start[s + 1] - q0 : p.num_tokens;
-    if (L < 0 || L > p.max_blocks_per_seq * p.block_size || n < 0 || (causal && n > L) || q0 < 0 ||
-        q0 + n > p.num_tokens || n > p.max_query_len) {
-        if (threadIdx.x == 0 && cta_tile == 0 && kvh == 0) flag_error(p.err, kErrBounds);
-        return;
-    }
-    const int tok0 = cta_tile * 2 * tpt;  // query tile A: tok0 .., tile B: tok0 + tpt ..
-    if (tok0 >= n) return;
-    const int ntok = min(2 * tpt, n - tok0);
-    const int ctx = L - n;
-    // key tiles up to the last row's position (all of the prefix without the mask);
-    // shared mode: tiles j0 .. j0 + nt - 1 of the prefix, range blockIdx.z
-    int nt = causal ? (ctx + tok0 + ntok - 1) / C::BN + 1 : (L + C::BN - 1) / C::BN;
-    int j0 = 0;
-    const int split = causal ? 0 : (int)blockIdx.z;
-    if (!causal) {
-        const int per = (nt + (int)gridDim.z - 1) / (int)gridDim.z;
-        j0 = split * per;
-        nt = min(per, nt - j0);
-        if (nt <= 0) {  // an empty range (the host never makes one): an empty partial
-            for (int i = threadIdx.x; i < ntok * g; i += C::THREADS) {
-                const int64_t row = (int64_t)(q0 + tok0 + i / g) * p.num_q_heads + (int64_t)kvh * g + i % g;
-                p.ws_lse[row * p.ws_np + split] = -CUDART_INF_F;
-                for (int d = 0; d < D; ++d) p.ws_o[(row * p.ws_np + split) * D + d] = 0.f;
-            }
-            return;
-        }
-    }
-    if (nt <= 0) return;  // an empty prefix
-    const int nblk_seq = (L + kBlockSize - 1) / kBlockSize;  // 16-token tiles
+    const int n_items = p.items_x * p.num_kv_heads * p.items_z;
     const int tile_mask = (1 << p.tile_shift) - 1;
 
     const uint32_t bars = base + C::OFF_BAR;
@@ -354,9 +379,19 @@ __global__ void __launch_bounds__(PfCfg<T, D, KVT>::THREADS, 1)
     auto bar_stg_empty = [&](int st) { return bars + 8u * (15 + 2 * C::ST + C::SST + st); };
     const uint32_t bar_drain_b = bars + 8u * (15 + 2 * C::ST + 2 * C::SST);
     const uint32_t bar_tail = bars + 8u * (16 + 2 * C::ST + 2 * C::SST);
+    // both issuers' last Q.K^T of an item done (Q may be reloaded); tile t's
+    // O read out by its softmax warps (the next item's P.V may overwrite it);
+    // the item ring: slot written / read by every consumer warp
+    const uint32_t bar_q_empty = bars + 8u * (17 + 2 * C::ST + 2 * C::SST);
+    auto bar_o_free = [&](int t) { return bars + 8u * (18 + 2 * C::ST + 2 * C::SST + t); };
+    auto bar_item_full = [&](int b) { return bars + 8u * (20 + 2 * C::ST + 2 * C::SST + b); };
+    auto bar_item_empty = [&](int b) { return bars + 8u * (22 + 2 * C::ST + 2 * C::SST + b); };
+    volatile int *item_slot = reinterpret_cast<volatile int *>(smem + C::OFF_ITEM);
+    volatile int *qexp = reinterpret_cast<volatile int *>(smem + C::OFF_QEXP);  // per item parity
     auto s_col = [&](int t, int b) { return C::COL_S + 64u * (2 * t + b); };
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + C::OFF_ABORT);
     uint32_t *slot = reinterpret_cast<uint32_t *>(smem + C::OFF_SLOT);
+    constexpr int CONSUMERS = 8 + 2 + C::CONVERTERS;  // warps that read the item ring
 
     if (threadIdx.x == 0) {
         mbar_init(bar_q, 1);
@@ -383,6 +418,13 @@ __global__ void __launch_bounds__(PfCfg<T, D, KVT>::THREADS, 1)
             mbar_init(bar_stg_full(st), 1);
             mbar_init(bar_stg_empty(st), C::CONVERTERS);
         }
+        mbar_init(bar_q_empty, 2);
+        mbar_init(bar_o_free(0), 128);
+        mbar_init(bar_o_free(1), 128);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(bar_item_full(b), 1);
+            mbar_init(bar_item_empty(b), CONSUMERS);
+        }
         *abort_flag = 0;
         mbar_init_fence();
     }
@@ -397,83 +439,120 @@ __global__ void __launch_bounds__(PfCfg<T, D, KVT>::THREADS, 1)
     auto v_smem = [&](int st) { return k_smem(st) + (uint32_t)C::KV_BYTES; };
     auto stg_k = [&](int st) { return base + C::OFF_STG + (uint32_t)(st * 2 * C::KV8_BYTES); };
     auto stg_v = [&](int st) { return stg_k(st) + (uint32_t)C::KV8_BYTES; };
+    // a consumer warp's next item (-1: none left); k counts the items taken
+    auto next_item = [&](int k) -> int {
+        const bool ok = __all_sync(tc::kFull, tc::wait_phase(bar_item_full(k & 1), (k >> 1) & 1, abort_flag, p.err));
+        const int item = ok ? item_slot[k & 1] : -1;
+        __syncwarp();
+        if (lane == 0) tc::mbar_arrive(bar_item_empty(k & 1));
+        return item;
+    };
 
     if (warp == 8) {
         // ================= TMA producer ===========================================
-        // Lane 0 issues the copies.  The whole warp holds the pool rows of the
-        // 16-token tiles: lane i the row of tile 32 b + i of the current batch b
-        // and of the next one, read a batch ahead, so no copy waits on a
-        // block-table load.
+        // Takes the items.  Lane 0 issues the copies.  The whole warp holds the
+        // pool rows of an item's 16-token tiles: lane i the row of tile 32 b + i
+        // of the current batch b and of the next one, read a batch ahead, so no
+        // copy waits on a block-table load.
         if (lane == 0) {
             asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_q)) : "memory");
             asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_k)) : "memory");
             asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_v)) : "memory");
-            mbar_arrive_expect_tx(bar_q, (uint32_t)(2 * C::ATOMS * tpt * g * 128));
-#pragma unroll
-            for (int t = 0; t < 2; ++t)
-#pragma unroll
-                for (int a = 0; a < C::ATOMS; ++a)
-                    tc::tma_load_3d(q_smem(t) + a * C::BM * 128, &tmap_q, a * 64, kvh * g,
-                                    q0 + tok0 + t * tpt, bar_q);
         }
-        const int32_t *bt = p.block_tables + (int64_t)s * p.max_blocks_per_seq;
         constexpr int TPK = C::BN / kBlockSize;  // 16-token tiles per key tile
         static_assert(32 % TPK == 0, "a batch of 32 tiles holds whole key tiles");
-        const int tile0 = j0 * TPK, ntiles = nt * TPK;
-        auto rows_of_batch = [&](int batch) -> int {  // pool row of this lane's tile (past the pool: zeros)
-            const int i = batch * 32 + lane, lb = tile0 + i;
-            int y = p.oob_row;
-            if (i < ntiles && lb < nblk_seq) {
-                const int phys = bt[lb >> p.tile_shift];
-                if ((unsigned)phys < (unsigned)p.num_blocks)
-                    y = (phys * p.num_kv_heads + kvh) * p.block_size + (lb & tile_mask) * kBlockSize;
-                else
-                    flag_error(p.err, kErrBounds);
-            }
-            return y;
-        };
-        int rows_cur = rows_of_batch(0), rows_nxt = ntiles > 32 ? rows_of_batch(1) : p.oob_row;
-        int cur_batch = 0;
         constexpr int RING = C::KV8 ? C::SST : C::ST;  // the ring the copies land in
         auto full_bar = [&](int st) { return C::KV8 ? bar_stg_full(st) : bar_kv_full(st); };
         auto empty_bar = [&](int st) { return C::KV8 ? bar_stg_empty(st) : bar_kv_empty(st); };
-        int j = 0;
-        for (; j < nt; ++j) {
-            const int st = j % RING;
-            if (j >= RING) {
-                int ok = lane == 0 ? (int)tc::wait_phase(empty_bar(st), ((j / RING) - 1) & 1, abort_flag, p.err) : 0;
-                if (!__shfl_sync(tc::kFull, ok, 0)) break;
+        int U = 0, kq = 0;  // key tiles issued, items with work (Q loads)
+        bool ok = true;
+        for (int k = 0; ok; ++k) {
+            // take an item and publish it to the ring (slot k & 1)
+            int item = -1;
+            if (lane == 0) {
+                item = (int)atomicAdd(&g_prefill_work[p.work_slot][0], 1u);
+                if (item >= n_items) item = -1;
+                if (k >= 2) ok = tc::wait_phase(bar_item_empty(k & 1), ((k >> 1) - 1) & 1, abort_flag, p.err);
+                item_slot[k & 1] = ok ? item : -1;
+                tc::mbar_arrive(bar_item_full(k & 1));
             }
-            if ((j * TPK) >> 5 != cur_batch) {  // uniform: the next batch becomes current
-                rows_cur = rows_nxt;
-                ++cur_batch;
-                rows_nxt = (cur_batch + 1) * 32 < ntiles ? rows_of_batch(cur_batch + 1) : p.oob_row;
+            ok = __shfl_sync(tc::kFull, (int)ok, 0) != 0;
+            item = __shfl_sync(tc::kFull, item, 0);
+            if (!ok || item < 0) break;
+            const PfItem w = decode_item<C::BN>(p, item, true);
+            if (w.state != 0) continue;
+            // Q of both tiles, once both issuers are done with the previous item's
+            if (lane == 0) {
+                if (kq > 0) ok = tc::wait_phase(bar_q_empty, (kq - 1) & 1, abort_flag, p.err);
+                if (ok) {
+                    mbar_arrive_expect_tx(bar_q, (uint32_t)(2 * C::ATOMS * tpt * g * 128));
+#pragma unroll
+                    for (int t = 0; t < 2; ++t)
+#pragma unroll
+                        for (int a = 0; a < C::ATOMS; ++a)
+                            tc::tma_load_3d(q_smem(t) + a * C::BM * 128, &tmap_q, a * 64, w.kvh * g,
+                                            w.q0 + w.tok0 + t * tpt, bar_q);
+                }
             }
-            // one copy per lane: lane l takes block l % TPK of the key tile, then
-            // (16-bit caches) atom l / TPK % ATOMS, K for l < NCOPY / 2 and V after
-            const int y = __shfl_sync(tc::kFull, rows_cur, (j * TPK + lane % TPK) & 31);
-            if (lane == 0)
-                mbar_arrive_expect_tx(full_bar(st), C::KV8 ? 2u * C::KV8_BYTES : 2u * C::KV_BYTES);
-            __syncwarp();
-            constexpr int NCOPY = 2 * TPK * (C::KV8 ? 1 : C::ATOMS);
-            static_assert(NCOPY <= 32, "one copy per lane");
-            if (lane < NCOPY) {
-                const int b = lane % TPK, is_v = lane >= NCOPY / 2;
-                if constexpr (C::KV8) {  // 16 rows x 128 codes, 128B swizzle
-                    const uint32_t dst = (is_v ? stg_v(st) : stg_k(st)) + b * kBlockSize * 128;
-                    tc::tma_load_2d(dst, is_v ? &tmap_v : &tmap_k, 0, y, full_bar(st));
-                } else {
-                    const int a = (lane / TPK) % C::ATOMS;
-                    const uint32_t dst = (is_v ? v_smem(st) : k_smem(st)) + a * C::BN * 128 + b * kBlockSize * 128;
-                    tc::tma_load_2d(dst, is_v ? &tmap_v : &tmap_k, a * 64, y, full_bar(st));
+            ok = __shfl_sync(tc::kFull, (int)ok, 0) != 0;
+            if (!ok) break;
+            ++kq;
+            const int32_t *bt = p.block_tables + (int64_t)w.s * p.max_blocks_per_seq;
+            const int tile0 = w.j0 * TPK, ntiles = w.nt * TPK;
+            auto rows_of_batch = [&](int batch) -> int {  // pool row of this lane's tile (past the pool: zeros)
+                const int i = batch * 32 + lane, lb = tile0 + i;
+                int y = p.oob_row;
+                if (i < ntiles && lb < w.nblk) {
+                    const int phys = bt[lb >> p.tile_shift];
+                    if ((unsigned)phys < (unsigned)p.num_blocks)
+                        y = (phys * p.num_kv_heads + w.kvh) * p.block_size + (lb & tile_mask) * kBlockSize;
+                    else
+                        flag_error(p.err, kErrBounds);
+                }
+                return y;
+            };
+            int rows_cur = rows_of_batch(0), rows_nxt = ntiles > 32 ? rows_of_batch(1) : p.oob_row;
+            int cur_batch = 0;
+            for (int j = 0; j < w.nt; ++j, ++U) {
+                const int st = U % RING;
+                if (U >= RING) {
+                    int r = lane == 0 ? (int)tc::wait_phase(empty_bar(st), ((U / RING) - 1) & 1, abort_flag, p.err) : 0;
+                    if (!__shfl_sync(tc::kFull, r, 0)) {
+                        ok = false;
+                        break;
+                    }
+                }
+                if ((j * TPK) >> 5 != cur_batch) {  // uniform: the next batch becomes current
+                    rows_cur = rows_nxt;
+                    ++cur_batch;
+                    rows_nxt = (cur_batch + 1) * 32 < ntiles ? rows_of_batch(cur_batch + 1) : p.oob_row;
+                }
+                // one copy per lane: lane l takes block l % TPK of the key tile, then
+                // (16-bit caches) atom l / TPK % ATOMS, K for l < NCOPY / 2 and V after
+                const int y = __shfl_sync(tc::kFull, rows_cur, (j * TPK + lane % TPK) & 31);
+                if (lane == 0)
+                    mbar_arrive_expect_tx(full_bar(st), C::KV8 ? 2u * C::KV8_BYTES : 2u * C::KV_BYTES);
+                __syncwarp();
+                constexpr int NCOPY = 2 * TPK * (C::KV8 ? 1 : C::ATOMS);
+                static_assert(NCOPY <= 32, "one copy per lane");
+                if (lane < NCOPY) {
+                    const int b = lane % TPK, is_v = lane >= NCOPY / 2;
+                    if constexpr (C::KV8) {  // 16 rows x 128 codes, 128B swizzle
+                        const uint32_t dst = (is_v ? stg_v(st) : stg_k(st)) + b * kBlockSize * 128;
+                        tc::tma_load_2d(dst, is_v ? &tmap_v : &tmap_k, 0, y, full_bar(st));
+                    } else {
+                        const int a = (lane / TPK) % C::ATOMS;
+                        const uint32_t dst = (is_v ? v_smem(st) : k_smem(st)) + a * C::BN * 128 + b * kBlockSize * 128;
+                        tc::tma_load_2d(dst, is_v ? &tmap_v : &tmap_k, a * 64, y, full_bar(st));
+                    }
                 }
             }
         }
         // nothing may still be landing in shared memory when the CTA exits
         if (lane == 0) {
-            (void)mbar_wait_bounded(bar_q, 0, kWaitLimitNs);
-            for (int jj = j - RING < 0 ? 0 : j - RING; jj < j; ++jj)
-                (void)mbar_wait_bounded(full_bar(jj % RING), (jj / RING) & 1, kWaitLimitNs);
+            if (kq > 0) (void)mbar_wait_bounded(bar_q, (kq - 1) & 1, kWaitLimitNs);
+            for (int u = U - RING < 0 ? 0 : U - RING; u < U; ++u)
+                (void)mbar_wait_bounded(full_bar(u % RING), (u / RING) & 1, kWaitLimitNs);
         }
         __syncwarp();
     } else if (warp == 9 || warp == C::MMA_B) {
@@ -488,79 +567,107 @@ __global__ void __launch_bounds__(PfCfg<T, D, KVT>::THREADS, 1)
         // for the scores two tiles later safe.  A K/V stage is free once both
         // issuers' P.V of it is done (kv_empty counts two commits).
         const int t = warp == 9 ? 0 : 1;
-        if (lane == 0) {
-            const uint64_t qd = tc::sdesc(q_smem(t), 16, 1024);
-            const uint64_t kdesc = tc::sdesc(k_smem(0), 16, 1024);
-            const uint64_t vdesc = tc::sdesc(v_smem(0), C::BN * 128, 1024);
-            const uint32_t ocol = tmem + C::COL_O + 128u * t;
-            auto issue_qk = [&](int j) {
-                const uint64_t kd = kdesc + (uint64_t)(((j % C::ST) * 2 * C::KV_BYTES) >> 4);
-                const uint32_t d = tmem + s_col(t, j & 1);
-                tc::fence_after();
+        const uint64_t qd = tc::sdesc(q_smem(t), 16, 1024);
+        const uint64_t kdesc = tc::sdesc(k_smem(0), 16, 1024);
+        const uint64_t vdesc = tc::sdesc(v_smem(0), C::BN * 128, 1024);
+        const uint32_t ocol = tmem + C::COL_O + 128u * t;
+        int J = 0, kq = 0, ntail = 0;  // key tiles done (all items), items with work, tails cleared
+        bool ok = true;
+        for (int k = 0; ok; ++k) {
+            const int item = next_item(k);
+            if (item < 0) break;
+            const PfItem w = decode_item<C::BN>(p, item, false);
+            if (w.state != 0) continue;
+            if (lane == 0) {
+                const int nt = w.nt;
+                // key tile j of this item: stage (J + j) % ST, score buffer (J + j) & 1
+                auto issue_qk = [&](int j) {
+                    const int jj = J + j;
+                    const uint64_t kd = kdesc + (uint64_t)(((jj % C::ST) * 2 * C::KV_BYTES) >> 4);
+                    const uint32_t d = tmem + s_col(t, jj & 1);
+                    tc::fence_after();
 #pragma unroll
-                for (int ks = 0; ks < D / 16; ++ks) {
-                    const uint32_t in_atom = (ks & 3) * 32;
-                    tc::mma_ss(d, qd + (uint64_t)(((ks >> 2) * (C::BM * 128) + in_atom) >> 4),
-                               kd + (uint64_t)(((ks >> 2) * (C::BN * 128) + in_atom) >> 4), C::IDESC_QK, ks > 0);
-                }
-                tc::commit(bar_s_full(t, j & 1));
-            };
-            auto issue_pv = [&](int j) {
-                const uint64_t vd = vdesc + (uint64_t)(((j % C::ST) * 2 * C::KV_BYTES) >> 4);
-                const uint32_t pcol = tmem + s_col(t, j & 1);
-                tc::fence_after();
-#pragma unroll
-                for (int ks = 0; ks < C::BN / 16; ++ks) {
-                    const uint64_t bd = vd + (uint64_t)((ks * 2048) >> 4);
-                    tc::mma_ts(ocol, pcol + ks * 8, bd, C::IDESC_PV, (j > 0 || ks > 0));
-                    if constexpr (C::HILO) tc::mma_ts(ocol, pcol + C::BN / 2 + ks * 8, bd, C::IDESC_PV, 1);
-                }
-                tc::commit(bar_pv(t, j & 1));
-                tc::commit(bar_kv_empty(j % C::ST));  // this issuer's last read of the stage
-            };
-            auto wait1 = [&](uint32_t bar, uint32_t parity) {
-                return tc::wait_phase(bar, parity, abort_flag, p.err);
-            };
-            auto kv_ready = [&](int j) { return wait1(bar_kv_full(j % C::ST), (j / C::ST) & 1); };
-            const int j_tail = (L & (kBlockSize - 1)) ? (nblk_seq - 1) / (C::BN / kBlockSize) - j0 : -1;
-            // Before P.V of the key tile holding the sequence's last block: the
-            // V rows of its unused slots (positions >= L) are cleared (p = 0
-            // there, but 0 x NaN poison = NaN).  The first issuer to get there
-            // clears them (its Q.K^T of the tile came after the copies landed),
-            // the other waits until it is done.
-            auto tail_ready = [&](int j) {
-                if (j != j_tail) return true;
-                if (atomicCAS(reinterpret_cast<int *>(smem + C::OFF_TAIL), 0, 1) == 0) {
-                    const int st = j % C::ST;
-                    const int r0 = L - (j0 + j) * C::BN, r1 = nblk_seq * kBlockSize - (j0 + j) * C::BN;
-                    const int chunks = (r1 - r0) * C::ATOMS * 8;
-                    for (int c = 0; c < chunks; ++c) {
-                        const int row = r0 + c / (C::ATOMS * 8), rem = c % (C::ATOMS * 8);
-                        const uint32_t addr = v_smem(st) + (rem >> 3) * C::BN * 128 + row * 128 + (rem & 7) * 16;
-                        asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(addr), "r"(0u) : "memory");
+                    for (int ks = 0; ks < D / 16; ++ks) {
+                        const uint32_t in_atom = (ks & 3) * 32;
+                        tc::mma_ss(d, qd + (uint64_t)(((ks >> 2) * (C::BM * 128) + in_atom) >> 4),
+                                   kd + (uint64_t)(((ks >> 2) * (C::BN * 128) + in_atom) >> 4), C::IDESC_QK, ks > 0);
                     }
-                    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-                    tc::mbar_arrive(bar_tail);
-                }
-                return wait1(bar_tail, 0);
-            };
-            bool ok = wait1(C::KV8 ? bar_q_ready : bar_q, 0);  // 8-bit caches: q converted
-            for (int j = 0; ok && j < 2 && j < nt; ++j) {
-                ok = kv_ready(j);
-                if (!ok) break;
-                issue_qk(j);
-            }
-            for (int j = 0; ok && j < nt; ++j) {
-                ok = wait1(bar_p_full(t, j & 1), (j >> 1) & 1) && tail_ready(j);
-                if (!ok) break;
-                issue_pv(j);
-                if (j + 2 < nt) {
-                    ok = kv_ready(j + 2);
+                    tc::commit(bar_s_full(t, jj & 1));
+                    if (j == nt - 1) tc::commit(bar_q_empty);  // this issuer's last read of Q
+                };
+                auto issue_pv = [&](int j) {
+                    const int jj = J + j;
+                    const uint64_t vd = vdesc + (uint64_t)(((jj % C::ST) * 2 * C::KV_BYTES) >> 4);
+                    const uint32_t pcol = tmem + s_col(t, jj & 1);
+                    tc::fence_after();
+#pragma unroll
+                    for (int ks = 0; ks < C::BN / 16; ++ks) {
+                        const uint64_t bd = vd + (uint64_t)((ks * 2048) >> 4);
+                        tc::mma_ts(ocol, pcol + ks * 8, bd, C::IDESC_PV, (j > 0 || ks > 0));
+                        if constexpr (C::HILO) tc::mma_ts(ocol, pcol + C::BN / 2 + ks * 8, bd, C::IDESC_PV, 1);
+                    }
+                    tc::commit(bar_pv(t, jj & 1));
+                    tc::commit(bar_kv_empty(jj % C::ST));  // this issuer's last read of the stage
+                };
+                auto wait1 = [&](uint32_t bar, uint32_t parity) {
+                    return tc::wait_phase(bar, parity, abort_flag, p.err);
+                };
+                auto kv_ready = [&](int j) {
+                    const int jj = J + j;
+                    return wait1(bar_kv_full(jj % C::ST), (jj / C::ST) & 1);
+                };
+                const int j_tail = (w.L & (kBlockSize - 1)) ? (w.nblk - 1) / (C::BN / kBlockSize) - w.j0 : -1;
+                // the tail tile's unused rows: [r0, r1) of its key tile
+                const int tail_r0 = w.L - (w.j0 + j_tail) * C::BN, tail_r1 = w.nblk * kBlockSize - (w.j0 + j_tail) * C::BN;
+                // Before P.V of the key tile holding the sequence's last block: the
+                // V rows of its unused slots (positions >= L) are cleared (p = 0
+                // there, but 0 x NaN poison = NaN).  The first issuer to get there
+                // clears them (its Q.K^T of the tile came after the copies landed),
+                // the other waits until it is done.
+                auto tail_ready = [&](int j) {
+                    if (j != j_tail) return true;
+                    if (atomicCAS(reinterpret_cast<int *>(smem + C::OFF_TAIL), ntail, ntail + 1) == ntail) {
+                        const int st = (J + j) % C::ST;
+                        const int chunks = (tail_r1 - tail_r0) * C::ATOMS * 8;
+                        for (int c = 0; c < chunks; ++c) {
+                            const int row = tail_r0 + c / (C::ATOMS * 8), rem = c % (C::ATOMS * 8);
+                            const uint32_t addr = v_smem(st) + (rem >> 3) * C::BN * 128 + row * 128 + (rem & 7) * 16;
+                            asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(addr), "r"(0u) : "memory");
+                        }
+                        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                        tc::mbar_arrive(bar_tail);
+                    }
+                    return wait1(bar_tail, (ntail++) & 1);
+                };
+                ok = wait1(C::KV8 ? bar_q_ready : bar_q, kq & 1);  // 8-bit caches: q converted
+                for (int j = 0; ok && j < 2 && j < nt; ++j) {
+                    ok = kv_ready(j);
                     if (!ok) break;
-                    issue_qk(j + 2);
+                    issue_qk(j);
+                }
+                // the previous item's O has been read out of tile t's accumulator
+                if (ok && kq > 0) {
+                    ok = wait1(bar_o_free(t), (kq - 1) & 1);
+                    tc::fence_after();
+                }
+                for (int j = 0; ok && j < nt; ++j) {
+                    const int jj = J + j;
+                    ok = wait1(bar_p_full(t, jj & 1), (jj >> 1) & 1) && tail_ready(j);
+                    if (!ok) break;
+                    issue_pv(j);
+                    if (j + 2 < nt) {
+                        ok = kv_ready(j + 2);
+                        if (!ok) break;
+                        issue_qk(j + 2);
+                    }
                 }
             }
-            // every MMA of this thread must be complete before TMEM is freed
+            ok = __shfl_sync(tc::kFull, (int)ok, 0) != 0;
+            J += w.nt;
+            ++kq;
+        }
+        // every MMA of this thread must be complete before TMEM is freed
+        if (lane == 0) {
             const uint32_t drain = t == 0 ? bar_drain : bar_drain_b;
             tc::commit(drain);
             (void)mbar_wait_bounded(drain, 0, kWaitLimitNs);
@@ -575,174 +682,209 @@ __global__ void __launch_bounds__(PfCfg<T, D, KVT>::THREADS, 1)
         // exact in f16
         if constexpr (C::KV8) {
             const int kv = warp - 10;  // 0: K, 1: V
-            bool ok = kv == 1 || __all_sync(tc::kFull, tc::wait_phase(bar_q, 0, abort_flag, p.err));
-            int e = 0;
-            if (kv == 0 && ok && std::is_same<T, bf16_t>::value) {
-                const int rows = tpt * g;  // rows the copy wrote in each tile
-                float amax = 0.f;
-                for (int t = 0; t < 2; ++t)
-                    for (int a = 0; a < C::ATOMS; ++a)
-                        for (int idx = lane; idx < rows * 8; idx += 32) {
-                            uint32_t w[4];
-                            lds<16>(w, q_smem(t) + a * C::BM * 128 + (idx >> 3) * 128 + (idx & 7) * 16);
-                            float f[8];
-                            Unpack<bf16_t, 8>::run(w, f);
+            int U = 0, kq = 0;          // key tiles converted (all items), items with work
+            bool ok = true;
+            for (int k = 0; ok; ++k) {
+                const int item = next_item(k);
+                if (item < 0) break;
+                const PfItem w = decode_item<C::BN>(p, item, false);
+                if (w.state != 0) continue;
+                if (kv == 0) {
+                    ok = __all_sync(tc::kFull, tc::wait_phase(bar_q, kq & 1, abort_flag, p.err));
+                    int e = 0;
+                    if (ok && std::is_same<T, bf16_t>::value) {
+                        const int rows = tpt * g;  // rows the copy wrote in each tile
+                        float amax = 0.f;
+                        for (int t = 0; t < 2; ++t)
+                            for (int a = 0; a < C::ATOMS; ++a)
+                                for (int idx = lane; idx < rows * 8; idx += 32) {
+                                    uint32_t wv[4];
+                                    lds<16>(wv, q_smem(t) + a * C::BM * 128 + (idx >> 3) * 128 + (idx & 7) * 16);
+                                    float f[8];
+                                    Unpack<bf16_t, 8>::run(wv, f);
 #pragma unroll
-                            for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(f[i]));
+                                    for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(f[i]));
+                                }
+#pragma unroll
+                        for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(tc::kFull, amax, o));
+                        if (amax > 0.f && amax <= 3.0e38f) {
+                            e = 14 - ((int)((__float_as_uint(amax) >> 23) & 0xFF) - 127);
+                            e = e > 100 ? 100 : (e < -100 ? -100 : e);
                         }
+                        const float up = __uint_as_float((uint32_t)(127 + e) << 23);  // 2^e, exact
+                        for (int t = 0; t < 2; ++t)
+                            for (int a = 0; a < C::ATOMS; ++a)
+                                for (int idx = lane; idx < rows * 8; idx += 32) {
+                                    const uint32_t addr = q_smem(t) + a * C::BM * 128 + (idx >> 3) * 128 + (idx & 7) * 16;
+                                    uint32_t wv[4];
+                                    lds<16>(wv, addr);
+                                    float f[8];
+                                    Unpack<bf16_t, 8>::run(wv, f);
+                                    uint32_t h[4];
 #pragma unroll
-                for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(tc::kFull, amax, o));
-                if (amax > 0.f && amax <= 3.0e38f) {
-                    e = 14 - ((int)((__float_as_uint(amax) >> 23) & 0xFF) - 127);
-                    e = e > 100 ? 100 : (e < -100 ? -100 : e);
+                                    for (int i = 0; i < 4; ++i) h[i] = tc::pack2(f[2 * i] * up, f[2 * i + 1] * up, f16_t{});
+                                    asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(h[0]),
+                                                 "r"(h[1]), "r"(h[2]), "r"(h[3])
+                                                 : "memory");
+                                }
+                        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                    }
+                    if (lane == 0) qexp[kq & 1] = e;
+                    __syncwarp();
+                    if (lane == 0) tc::mbar_arrive(bar_q_ready);
                 }
-                const float up = __uint_as_float((uint32_t)(127 + e) << 23);  // 2^e, exact
-                for (int t = 0; t < 2; ++t)
-                    for (int a = 0; a < C::ATOMS; ++a)
-                        for (int idx = lane; idx < rows * 8; idx += 32) {
-                            const uint32_t addr = q_smem(t) + a * C::BM * 128 + (idx >> 3) * 128 + (idx & 7) * 16;
-                            uint32_t w[4];
-                            lds<16>(w, addr);
-                            float f[8];
-                            Unpack<bf16_t, 8>::run(w, f);
-                            uint32_t h[4];
-#pragma unroll
-                            for (int i = 0; i < 4; ++i) h[i] = tc::pack2(f[2 * i] * up, f[2 * i + 1] * up, f16_t{});
-                            asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(h[0]),
-                                         "r"(h[1]), "r"(h[2]), "r"(h[3])
-                                         : "memory");
-                        }
-                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-            }
-            if (kv == 0) {
-                if (lane == 0) *reinterpret_cast<volatile int *>(smem + C::OFF_QEXP) = e;
-                __syncwarp();
-                if (lane == 0) tc::mbar_arrive(bar_q_ready);
-            }
-            for (int j = 0; ok && j < nt; ++j) {
-                const int sst = j % C::SST, st = j % C::ST;
-                ok = __all_sync(tc::kFull, tc::wait_phase(bar_stg_full(sst), (j / C::SST) & 1, abort_flag, p.err));
-                if (!ok) break;
-                if (j >= C::ST) {  // the MMAs are done with this operand stage
-                    ok = __all_sync(tc::kFull,
-                                    tc::wait_phase(bar_kv_empty(st), ((j / C::ST) - 1) & 1, abort_flag, p.err));
+                for (int j = 0; ok && j < w.nt; ++j) {
+                    const int uu = U + j;
+                    const int sst = uu % C::SST, st = uu % C::ST;
+                    ok = __all_sync(tc::kFull, tc::wait_phase(bar_stg_full(sst), (uu / C::SST) & 1, abort_flag, p.err));
                     if (!ok) break;
-                }
-                {
-                    const uint32_t src = kv ? stg_v(sst) : stg_k(sst);
-                    const uint32_t dst = kv ? v_smem(st) : k_smem(st);
-                    // BN * 8 chunks of 16 codes, batches of 4 a lane: the loads of
-                    // a batch go out together, then its conversions and stores
-                    constexpr int NB = 4, PER = C::BN * 8 / 32;
-                    static_assert(PER % NB == 0, "batches");
+                    if (uu >= C::ST) {  // the MMAs are done with this operand stage
+                        ok = __all_sync(tc::kFull,
+                                        tc::wait_phase(bar_kv_empty(st), ((uu / C::ST) - 1) & 1, abort_flag, p.err));
+                        if (!ok) break;
+                    }
+                    {
+                        const uint32_t src = kv ? stg_v(sst) : stg_k(sst);
+                        const uint32_t dst = kv ? v_smem(st) : k_smem(st);
+                        // BN * 8 chunks of 16 codes, batches of 4 a lane: the loads of
+                        // a batch go out together, then its conversions and stores
+                        constexpr int NB = 4, PER = C::BN * 8 / 32;
+                        static_assert(PER % NB == 0, "batches");
 #pragma unroll
-                    for (int i0 = 0; i0 < PER; i0 += NB) {
-                        uint32_t w[NB][4];
+                        for (int i0 = 0; i0 < PER; i0 += NB) {
+                            uint32_t wv[NB][4];
 #pragma unroll
-                        for (int b = 0; b < NB; ++b) {
-                            const int idx = lane + 32 * (i0 + b), r = idx >> 3, c8 = idx & 7;
-                            lds<16>(w[b], src + r * 128 + ((c8 ^ (r & 7)) << 4));
-                        }
+                            for (int b = 0; b < NB; ++b) {
+                                const int idx = lane + 32 * (i0 + b), r = idx >> 3, c8 = idx & 7;
+                                lds<16>(wv[b], src + r * 128 + ((c8 ^ (r & 7)) << 4));
+                            }
 #pragma unroll
-                        for (int b = 0; b < NB; ++b) {
-                            const int idx = lane + 32 * (i0 + b);
-                            const int r = idx >> 3, c8 = idx & 7;  // row, chunk of 16 codes
-                            uint32_t h[8];
+                            for (int b = 0; b < NB; ++b) {
+                                const int idx = lane + 32 * (i0 + b);
+                                const int r = idx >> 3, c8 = idx & 7;  // row, chunk of 16 codes
+                                uint32_t h[8];
 #pragma unroll
-                            for (int i = 0; i < 4; ++i) tc::widen4(w[b][i], h[2 * i], h[2 * i + 1], KVT{});
-                            // codes 16 c8 .. +15 = f16 chunks 2 (c8 % 4) and +1 of atom c8 / 4
-                            const uint32_t rowb = dst + (c8 >> 2) * C::BN * 128 + r * 128;
-                            const int cf = (c8 & 3) * 2;
-                            asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(rowb + ((cf ^ (r & 7)) << 4)),
-                                         "r"(h[0]), "r"(h[1]), "r"(h[2]), "r"(h[3])
-                                         : "memory");
-                            asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(rowb + (((cf + 1) ^ (r & 7)) << 4)),
-                                         "r"(h[4]), "r"(h[5]), "r"(h[6]), "r"(h[7])
-                                         : "memory");
+                                for (int i = 0; i < 4; ++i) tc::widen4(wv[b][i], h[2 * i], h[2 * i + 1], KVT{});
+                                // codes 16 c8 .. +15 = f16 chunks 2 (c8 % 4) and +1 of atom c8 / 4
+                                const uint32_t rowb = dst + (c8 >> 2) * C::BN * 128 + r * 128;
+                                const int cf = (c8 & 3) * 2;
+                                asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(rowb + ((cf ^ (r & 7)) << 4)),
+                                             "r"(h[0]), "r"(h[1]), "r"(h[2]), "r"(h[3])
+                                             : "memory");
+                                asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(rowb + (((cf + 1) ^ (r & 7)) << 4)),
+                                             "r"(h[4]), "r"(h[5]), "r"(h[6]), "r"(h[7])
+                                             : "memory");
+                            }
                         }
                     }
+                    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                    __syncwarp();
+                    if (lane == 0) {
+                        tc::mbar_arrive(bar_stg_empty(sst));
+                        tc::mbar_arrive(bar_kv_full(st));
+                    }
                 }
-                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-                __syncwarp();
-                if (lane == 0) {
-                    tc::mbar_arrive(bar_stg_empty(sst));
-                    tc::mbar_arrive(bar_kv_full(st));
-                }
+                U += w.nt;
+                ++kq;
             }
         }
     } else {
         // ================= softmax: one thread per query row =======================
         const int t = warp >> 2;                  // query tile (0: A, 1: B)
         const int r = (warp & 3) * 32 + lane;     // row = TMEM lane
-        const int rtok = t * tpt + r / g;         // token within the CTA's range
-        const bool row_ok = r < tpt * g && rtok < ntok;
-        const int pos = causal ? ctx + tok0 + rtok : L - 1;
         const uint32_t lane_bits = (uint32_t)((warp & 3) * 32) << 16;
         const uint32_t ocol = tmem + lane_bits + C::COL_O + 128u * t;
-        float sl2 = p.qk_scale_log2;  // > 0
-        if constexpr (C::KV8) {  // q was scaled by 2^e on its way to f16
-            if (!__all_sync(tc::kFull, tc::wait_phase(bar_q_ready, 0, abort_flag, p.err))) sl2 = 0.f;
-            const int e = *reinterpret_cast<volatile int *>(smem + C::OFF_QEXP);
-            sl2 *= __uint_as_float((uint32_t)(127 - e) << 23);
-        }
-        float m_ref = -CUDART_INF_F, l = 0.f;
+        int J = 0, kq = 0;  // key tiles done (all items), items with work
         bool ok = true;
-        for (int j = 0; j < nt; ++j) {
-            ok = __all_sync(tc::kFull, tc::wait_phase(bar_s_full(t, j & 1), (j >> 1) & 1, abort_flag, p.err));
-            if (!ok) break;
-            tc::fence_after();
-            const uint32_t scol = tmem + lane_bits + s_col(t, j & 1);
-            uint32_t sv[C::BN];
-#pragma unroll
-            for (int c = 0; c < C::BN; c += 32) tc::ld32(scol + c, sv + c);
-            tc::wait_ld<C::BN>(sv);
-            // keys of this tile the row may see: all, a prefix (diagonal tile), none
-            const int lim = row_ok ? pos - (j0 + j) * C::BN + 1 : 0;
-            if (lim < C::BN) {
-#pragma unroll
-                for (int c = 0; c < C::BN; ++c)
-                    if (c >= lim) sv[c] = __float_as_uint(-CUDART_INF_F);
-            }
-            float m4[4] = {-CUDART_INF_F, -CUDART_INF_F, -CUDART_INF_F, -CUDART_INF_F};
-#pragma unroll
-            for (int c = 0; c < C::BN; ++c) m4[c & 3] = fmaxf(m4[c & 3], __uint_as_float(sv[c]));
-            const float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * sl2;
-            // lazy rescale: move the reference max only when it grows by > 8
-            float alpha = 1.f;
-            const bool grow = mx > m_ref + 8.f;
-            if (grow) {
-                alpha = m_ref == -CUDART_INF_F ? 0.f : ex2(m_ref - mx);
-                m_ref = mx;
-            }
-            const float nmb = m_ref == -CUDART_INF_F ? 0.f : -m_ref;
-            l *= alpha;
-            float ps[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-            for (int c0 = 0; c0 < C::BN; c0 += 32) {
-                uint32_t hi[16], lo[16];
-#pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    const float p0 = ex2(fmaf(__uint_as_float(sv[c0 + 2 * i]), sl2, nmb));
-                    const float p1 = ex2(fmaf(__uint_as_float(sv[c0 + 2 * i + 1]), sl2, nmb));
-                    ps[i & 3] += p0 + p1;
-                    hi[i] = tc::pack2(p0, p1, OpT{});
-                    if constexpr (C::HILO) {
-                        float h0, h1;
-                        tc::unpack2(hi[i], h0, h1, bf16_t{});
-                        lo[i] = tc::pack2(p0 - h0, p1 - h1, OpT{});
-                    }
+        for (int k = 0; ok; ++k) {
+            const int item = next_item(k);
+            if (item < 0) break;
+            const PfItem w = decode_item<C::BN>(p, item, false);
+            if (w.state == 2) {
+                // an empty key range: an empty partial (lse = -inf, o = 0) for this
+                // warp's rows
+                const int rtok = t * tpt + r / g;
+                if (r < tpt * g && rtok < w.ntok) {
+                    const int64_t row = (int64_t)(w.q0 + w.tok0 + rtok) * p.num_q_heads + (int64_t)w.kvh * g + r % g;
+                    p.ws_lse[row * p.ws_np + w.split] = -CUDART_INF_F;
+                    for (int d = 0; d < D; ++d) p.ws_o[(row * p.ws_np + w.split) * D + d] = 0.f;
                 }
-                tc::st16(scol + c0 / 2, hi);
-                if constexpr (C::HILO) tc::st16(scol + C::BN / 2 + c0 / 2, lo);
+                continue;
             }
-            l += (ps[0] + ps[1]) + (ps[2] + ps[3]);
-            if (j > 0 && __any_sync(tc::kFull, grow)) {
-                // O may be rescaled only once the previous P.V of this tile is
-                // complete (the earlier ones completed before it)
-                ok = __all_sync(tc::kFull, tc::wait_phase(bar_pv(t, (j - 1) & 1), ((j - 1) >> 1) & 1,
-                                                         abort_flag, p.err));
+            if (w.state != 0) continue;
+            const int nt = w.nt;
+            const int rtok = t * tpt + r / g;  // token within the item's range
+            const bool row_ok = r < tpt * g && rtok < w.ntok;
+            // the row's last visible key, counted from the item's first key tile
+            const int pos0 = (causal ? w.ctx + w.tok0 + rtok : w.L - 1) - w.j0 * C::BN;
+            const int64_t row = ((int64_t)(w.q0 + w.tok0 + rtok) * p.num_q_heads + (int64_t)w.kvh * g + r % g);
+            const int split = w.split;
+            float sl2 = p.qk_scale_log2;  // > 0
+            if constexpr (C::KV8) {  // q was scaled by 2^e on its way to f16
+                if (!__all_sync(tc::kFull, tc::wait_phase(bar_q_ready, kq & 1, abort_flag, p.err))) {
+                    ok = false;
+                    break;
+                }
+                const int e = qexp[kq & 1];
+                sl2 *= __uint_as_float((uint32_t)(127 - e) << 23);
+            }
+            float m_ref = -CUDART_INF_F, l = 0.f;
+            for (int j = 0; j < nt; ++j) {
+                const int jj = J + j;
+                ok = __all_sync(tc::kFull, tc::wait_phase(bar_s_full(t, jj & 1), (jj >> 1) & 1, abort_flag, p.err));
                 if (!ok) break;
-                {
+                tc::fence_after();
+                const uint32_t scol = tmem + lane_bits + s_col(t, jj & 1);
+                uint32_t sv[C::BN];
+#pragma unroll
+                for (int c = 0; c < C::BN; c += 32) tc::ld32(scol + c, sv + c);
+                tc::wait_ld<C::BN>(sv);
+                // keys of this tile the row may see: all, a prefix (diagonal tile), none
+                const int lim = row_ok ? pos0 - j * C::BN + 1 : 0;
+                if (lim < C::BN) {
+#pragma unroll
+                    for (int c = 0; c < C::BN; ++c)
+                        if (c >= lim) sv[c] = __float_as_uint(-CUDART_INF_F);
+                }
+                float m4[4] = {-CUDART_INF_F, -CUDART_INF_F, -CUDART_INF_F, -CUDART_INF_F};
+#pragma unroll
+                for (int c = 0; c < C::BN; ++c) m4[c & 3] = fmaxf(m4[c & 3], __uint_as_float(sv[c]));
+                const float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * sl2;
+                // lazy rescale: move the reference max only when it grows by > 8
+                float alpha = 1.f;
+                const bool grow = mx > m_ref + 8.f;
+                if (grow) {
+                    alpha = m_ref == -CUDART_INF_F ? 0.f : ex2(m_ref - mx);
+                    m_ref = mx;
+                }
+                const float nmb = m_ref == -CUDART_INF_F ? 0.f : -m_ref;
+                l *= alpha;
+                float ps[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                for (int c0 = 0; c0 < C::BN; c0 += 32) {
+                    uint32_t hi[16], lo[16];
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        const float p0 = ex2(fmaf(__uint_as_float(sv[c0 + 2 * i]), sl2, nmb));
+                        const float p1 = ex2(fmaf(__uint_as_float(sv[c0 + 2 * i + 1]), sl2, nmb));
+                        ps[i & 3] += p0 + p1;
+                        hi[i] = tc::pack2(p0, p1, OpT{});
+                        if constexpr (C::HILO) {
+                            float h0, h1;
+                            tc::unpack2(hi[i], h0, h1, bf16_t{});
+                            lo[i] = tc::pack2(p0 - h0, p1 - h1, OpT{});
+                        }
+                    }
+                    tc::st16(scol + c0 / 2, hi);
+                    if constexpr (C::HILO) tc::st16(scol + C::BN / 2 + c0 / 2, lo);
+                }
+                l += (ps[0] + ps[1]) + (ps[2] + ps[3]);
+                if (j > 0 && __any_sync(tc::kFull, grow)) {
+                    // O may be rescaled only once the previous P.V of this tile is
+                    // complete (the earlier ones completed before it)
+                    ok = __all_sync(tc::kFull, tc::wait_phase(bar_pv(t, (jj - 1) & 1), ((jj - 1) >> 1) & 1,
+                                                             abort_flag, p.err));
+                    if (!ok) break;
                     tc::fence_after();
 #pragma unroll
                     for (int c = 0; c < D; c += 32) {
@@ -754,22 +896,40 @@ __global__ void __launch_bounds__(PfCfg<T, D, KVT>::THREADS, 1)
                         tc::st32(ocol + c, o);
                     }
                 }
+                tc::wait_st();
+                tc::fence_before();
+                tc::mbar_arrive(bar_p_full(t, jj & 1));
             }
-            tc::wait_st();
-            tc::fence_before();
-            tc::mbar_arrive(bar_p_full(t, j & 1));
-        }
-        if (ok)
-            ok = __all_sync(tc::kFull, tc::wait_phase(bar_pv(t, (nt - 1) & 1), ((nt - 1) >> 1) & 1,
-                                                     abort_flag, p.err));
-        if (ok) {
+            if (ok) {
+                const int jl = J + nt - 1;
+                ok = __all_sync(tc::kFull, tc::wait_phase(bar_pv(t, jl & 1), (jl >> 1) & 1, abort_flag, p.err));
+            }
+            if (!ok) break;
             // ---- epilogue: out = O / l, rounded once to the q dtype ----------------
-            // (shared-prefix mode: the partial o / l and its log-sum-exp, fp32)
+            // (shared-prefix mode: the partial o / l and its log-sum-exp, fp32).
+            // Once O is out of TMEM, tile t's accumulator is handed to the next
+            // item's P.V (o_free).
             tc::fence_after();
             const float inv = l > 0.f ? p.v_scale / l : 0.f;  // v_scale: 1 for 16-bit caches
-            const int64_t row = ((int64_t)(q0 + tok0 + rtok) * p.num_q_heads + (int64_t)kvh * g + r % g);
-            uint4 *dst = reinterpret_cast<uint4 *>(static_cast<uint16_t *>(p.out) + row * D);
-            if (!causal) {
+            if (causal) {
+                uint4 *dst = reinterpret_cast<uint4 *>(static_cast<uint16_t *>(p.out) + row * D);
+#pragma unroll
+                for (int c = 0; c < D; c += 32) {
+                    uint32_t o[32];
+                    tc::ld32(ocol + c, o);
+                    tc::wait_ld<32>(o);
+                    uint32_t wv[16];
+#pragma unroll
+                    for (int i = 0; i < 16; ++i)
+                        wv[i] = tc::pack2(__uint_as_float(o[2 * i]) * inv, __uint_as_float(o[2 * i + 1]) * inv, T{});
+                    if (row_ok) {
+#pragma unroll
+                        for (int v = 0; v < 4; ++v) dst[c / 8 + v] = make_uint4(wv[4 * v], wv[4 * v + 1], wv[4 * v + 2], wv[4 * v + 3]);
+                    }
+                }
+                tc::fence_before();
+                tc::mbar_arrive(bar_o_free(t));
+            } else {
                 float4 *wo = reinterpret_cast<float4 *>(p.ws_o + (row * p.ws_np + split) * D);
                 if (row_ok)
                     p.ws_lse[row * p.ws_np + split] =
@@ -786,23 +946,11 @@ __global__ void __launch_bounds__(PfCfg<T, D, KVT>::THREADS, 1)
                                                         __uint_as_float(o[4 * v + 2]) * inv, __uint_as_float(o[4 * v + 3]) * inv);
                     }
                 }
-            } else {
-#pragma unroll
-                for (int c = 0; c < D; c += 32) {
-                    uint32_t o[32];
-                    tc::ld32(ocol + c, o);
-                    tc::wait_ld<32>(o);
-                    uint32_t w[16];
-#pragma unroll
-                    for (int i = 0; i < 16; ++i)
-                        w[i] = tc::pack2(__uint_as_float(o[2 * i]) * inv, __uint_as_float(o[2 * i + 1]) * inv, T{});
-                    if (row_ok) {
-#pragma unroll
-                        for (int v = 0; v < 4; ++v)
-                            dst[c / 8 + v] = make_uint4(w[4 * v], w[4 * v + 1], w[4 * v + 2], w[4 * v + 3]);
-                    }
-                }
+                tc::fence_before();
+                tc::mbar_arrive(bar_o_free(t));
             }
+            J += nt;
+            ++kq;
         }
     }
 
@@ -812,6 +960,14 @@ __global__ void __launch_bounds__(PfCfg<T, D, KVT>::THREADS, 1)
     if (warp == 0) {
         tc::fence_after();
         tc::dealloc(tmem, C::TMEM_COLS);
+    }
+    // the launch's last CTA to finish resets its work counter for the next launch
+    if (threadIdx.x == 0) {
+        __threadfence();
+        if (atomicAdd(&g_prefill_work[p.work_slot][1], 1u) == gridDim.x - 1) {
+            atomicExch(&g_prefill_work[p.work_slot][0], 0u);
+            atomicExch(&g_prefill_work[p.work_slot][1], 0u);
+        }
     }
 }
 
@@ -850,10 +1006,20 @@ cudaError_t launch_prefill_t(const PrefillParams &p, cudaStream_t stream) {
     if (e != cudaSuccess) return e;
     const int per_cta = 2 * p.tok_per_tile;  // two query tiles
     static_assert(C::BN == kPrefixKeyTile, "shared-prefix key ranges are counted in key tiles");
-    const int z = p.shared_len > 0 ? prefix_splits(p.shared_len) : p.num_seqs;
-    const dim3 grid((unsigned)((p.max_query_len + per_cta - 1) / per_cta), (unsigned)p.num_kv_heads,
-                    (unsigned)z);
-    kern<<<grid, C::THREADS, C::SMEM, stream>>>(p, mq, mk, mv);
+    PrefillParams q = p;
+    q.items_x = (p.max_query_len + per_cta - 1) / per_cta;
+    q.items_z = p.shared_len > 0 ? prefix_splits(p.shared_len) : p.num_seqs;
+    const int64_t items = (int64_t)q.items_x * p.num_kv_heads * q.items_z;
+    if (items <= 0) return cudaSuccess;
+    if (items > INT32_MAX) return cudaErrorInvalidValue;
+    int dev = 0, sms = 0;
+    e = cudaGetDevice(&dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return e;
+    static std::atomic<unsigned> next_slot{0};
+    q.work_slot = (int)(next_slot.fetch_add(1u) % (unsigned)kWorkSlots);
+    const unsigned grid = (unsigned)(items < sms ? items : sms);  // one CTA an SM, persistent
+    kern<<<grid, C::THREADS, C::SMEM, stream>>>(q, mq, mk, mv);
     return cudaGetLastError();
 }
 
