@@ -603,8 +603,13 @@ __global__ void __launch_bounds__(PfCfg<T, D, KVT>::THREADS, 1)
 #pragma unroll
                     for (int ks = 0; ks < C::BN / 16; ++ks) {
                         const uint64_t bd = vd + (uint64_t)((ks * 2048) >> 4);
-                        tc::mma_ts(ocol, pcol + ks * 8, bd, C::IDESC_PV, (j > 0 || ks > 0));
-                        if constexpr (C::HILO) tc::mma_ts(ocol, pcol + C::BN / 2 + ks * 8, bd, C::IDESC_PV, 1);
+                        if constexpr (C::HILO) {  // hi of keys 16 ks .. in column 32 (ks / 2) + 8 (ks % 2), lo 16 after
+                            const uint32_t pc = pcol + (ks >> 1) * 32 + (ks & 1) * 8;
+                            tc::mma_ts(ocol, pc, bd, C::IDESC_PV, (j > 0 || ks > 0));
+                            tc::mma_ts(ocol, pc + 16, bd, C::IDESC_PV, 1);
+                        } else {
+                            tc::mma_ts(ocol, pcol + ks * 8, bd, C::IDESC_PV, (j > 0 || ks > 0));
+                        }
                     }
                     tc::commit(bar_pv(t, jj & 1));
                     tc::commit(bar_kv_empty(jj % C::ST));  // this issuer's last read of the stage
@@ -862,7 +867,8 @@ __global__ void __launch_bounds__(PfCfg<T, D, KVT>::THREADS, 1)
                 float ps[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
                 for (int c0 = 0; c0 < C::BN; c0 += 32) {
-                    uint32_t hi[16], lo[16];
+                    uint32_t hl[32];  // hi pairs, then lo pairs (bf16 caches)
+                    uint32_t *hi = hl, *lo = hl + 16;
 #pragma unroll
                     for (int i = 0; i < 16; ++i) {
                         const float p0 = ex2(fmaf(__uint_as_float(sv[c0 + 2 * i]), sl2, nmb));
@@ -875,8 +881,10 @@ __global__ void __launch_bounds__(PfCfg<T, D, KVT>::THREADS, 1)
                             lo[i] = tc::pack2(p0 - h0, p1 - h1, OpT{});
                         }
                     }
-                    tc::st16(scol + c0 / 2, hi);
-                    if constexpr (C::HILO) tc::st16(scol + C::BN / 2 + c0 / 2, lo);
+                    // bf16 caches: one store of the chunk's 16 hi and 16 lo columns
+                    // (columns c0 .. c0 + 31); f16: its 16 columns at c0 / 2
+                    if constexpr (C::HILO) tc::st32(scol + c0, hl);
+                    else tc::st16(scol + c0 / 2, hi);
                 }
                 l += (ps[0] + ps[1]) + (ps[2] + ps[3]);
                 if (j > 0 && __any_sync(tc::kFull, grow)) {
