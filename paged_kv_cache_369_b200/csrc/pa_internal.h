@@ -174,6 +174,13 @@ struct PrefillParams {  // chunked prefill (pa_prefill)
     int items_x;
     int items_z;
     int work_slot;
+    // failure-detection test hook, never set through the public ABI (the
+    // launch reads it from the environment variable PA369_TEST_PREFILL_STALL_NS):
+    // every device wait gives up after wait_limit_ns (0: kWaitLimitNs), and
+    // with hold_first_tile each CTA leaves its first K/V stage's copies
+    // unissued, so that the first wait on it can only run out
+    uint64_t wait_limit_ns;
+    int hold_first_tile;
 };
 
 struct ReduceParams {

@@ -53,6 +53,7 @@
 #include <math_constants.h>
 
 #include <atomic>
+#include <cstdlib>
 #include <cstdint>
 #include <type_traits>
 
@@ -195,7 +196,7 @@ __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
 // the CTA has already given up (abort flag); the thread that runs out of
 // time raises the flag and reports the timeout.
 __device__ __forceinline__ bool wait_phase(uint32_t bar, uint32_t parity, volatile int *abort_flag,
-                                           int *err) {
+                                           int *err, uint64_t limit_ns = kWaitLimitNs) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = global_ns();
     for (;;) {
@@ -203,7 +204,7 @@ __device__ __forceinline__ bool wait_phase(uint32_t bar, uint32_t parity, volati
         for (int i = 0; i < 64; ++i)
             if (mbar_try_wait(bar, parity)) return true;
         if (*abort_flag) return false;
-        if (global_ns() - t0 > kWaitLimitNs) {
+        if (global_ns() - t0 > limit_ns) {
             *abort_flag = 1;
             flag_error(err, kErrTimeout);
             return false;
@@ -361,6 +362,7 @@ __global__ void __launch_bounds__(PfCfg<T, D, KVT>::THREADS, 1)
     const int g = p.group, tpt = p.tok_per_tile;
     const bool causal = p.shared_len == 0;
     const int n_items = p.items_x * p.num_kv_heads * p.items_z;
+    const uint64_t wl = p.wait_limit_ns ? p.wait_limit_ns : kWaitLimitNs;  // bound on every wait
     const int tile_mask = (1 << p.tile_shift) - 1;
 
     const uint32_t bars = base + C::OFF_BAR;
@@ -441,7 +443,7 @@ __global__ void __launch_bounds__(PfCfg<T, D, KVT>::THREADS, 1)
     auto stg_v = [&](int st) { return stg_k(st) + (uint32_t)C::KV8_BYTES; };
     // a consumer warp's next item (-1: none left); k counts the items taken
     auto next_item = [&](int k) -> int {
-        const bool ok = __all_sync(tc::kFull, tc::wait_phase(bar_item_full(k & 1), (k >> 1) & 1, abort_flag, p.err));
+        const bool ok = __all_sync(tc::kFull, tc::wait_phase(bar_item_full(k & 1), (k >> 1) & 1, abort_flag, p.err, wl));
         const int item = ok ? item_slot[k & 1] : -1;
         __syncwarp();
         if (lane == 0) tc::mbar_arrive(bar_item_empty(k & 1));
@@ -472,7 +474,7 @@ __global__ void __launch_bounds__(PfCfg<T, D, KVT>::THREADS, 1)
             if (lane == 0) {
                 item = (int)atomicAdd(&g_prefill_work[p.work_slot][0], 1u);
                 if (item >= n_items) item = -1;
-                if (k >= 2) ok = tc::wait_phase(bar_item_empty(k & 1), ((k >> 1) - 1) & 1, abort_flag, p.err);
+                if (k >= 2) ok = tc::wait_phase(bar_item_empty(k & 1), ((k >> 1) - 1) & 1, abort_flag, p.err, wl);
                 item_slot[k & 1] = ok ? item : -1;
                 tc::mbar_arrive(bar_item_full(k & 1));
             }
@@ -483,7 +485,7 @@ __global__ void __launch_bounds__(PfCfg<T, D, KVT>::THREADS, 1)
             if (w.state != 0) continue;
             // Q of both tiles, once both issuers are done with the previous item's
             if (lane == 0) {
-                if (kq > 0) ok = tc::wait_phase(bar_q_empty, (kq - 1) & 1, abort_flag, p.err);
+                if (kq > 0) ok = tc::wait_phase(bar_q_empty, (kq - 1) & 1, abort_flag, p.err, wl);
                 if (ok) {
                     mbar_arrive_expect_tx(bar_q, (uint32_t)(2 * C::ATOMS * tpt * g * 128));
 #pragma unroll
@@ -516,7 +518,7 @@ __global__ void __launch_bounds__(PfCfg<T, D, KVT>::THREADS, 1)
             for (int j = 0; j < w.nt; ++j, ++U) {
                 const int st = U % RING;
                 if (U >= RING) {
-                    int r = lane == 0 ? (int)tc::wait_phase(empty_bar(st), ((U / RING) - 1) & 1, abort_flag, p.err) : 0;
+                    int r = lane == 0 ? (int)tc::wait_phase(empty_bar(st), ((U / RING) - 1) & 1, abort_flag, p.err, wl) : 0;
                     if (!__shfl_sync(tc::kFull, r, 0)) {
                         ok = false;
                         break;
@@ -535,7 +537,7 @@ __global__ void __launch_bounds__(PfCfg<T, D, KVT>::THREADS, 1)
                 __syncwarp();
                 constexpr int NCOPY = 2 * TPK * (C::KV8 ? 1 : C::ATOMS);
                 static_assert(NCOPY <= 32, "one copy per lane");
-                if (lane < NCOPY) {
+                if (lane < NCOPY && !(p.hold_first_tile && U == 0)) {
                     const int b = lane % TPK, is_v = lane >= NCOPY / 2;
                     if constexpr (C::KV8) {  // 16 rows x 128 codes, 128B swizzle
                         const uint32_t dst = (is_v ? stg_v(st) : stg_k(st)) + b * kBlockSize * 128;
@@ -550,9 +552,9 @@ __global__ void __launch_bounds__(PfCfg<T, D, KVT>::THREADS, 1)
         }
         // nothing may still be landing in shared memory when the CTA exits
         if (lane == 0) {
-            if (kq > 0) (void)mbar_wait_bounded(bar_q, (kq - 1) & 1, kWaitLimitNs);
+            if (kq > 0) (void)mbar_wait_bounded(bar_q, (kq - 1) & 1, wl);
             for (int u = U - RING < 0 ? 0 : U - RING; u < U; ++u)
-                (void)mbar_wait_bounded(full_bar(u % RING), (u / RING) & 1, kWaitLimitNs);
+                (void)mbar_wait_bounded(full_bar(u % RING), (u / RING) & 1, wl);
         }
         __syncwarp();
     } else if (warp == 9 || warp == C::MMA_B) {
@@ -615,7 +617,7 @@ __global__ void __launch_bounds__(PfCfg<T, D, KVT>::THREADS, 1)
                     tc::commit(bar_kv_empty(jj % C::ST));  // this issuer's last read of the stage
                 };
                 auto wait1 = [&](uint32_t bar, uint32_t parity) {
-                    return tc::wait_phase(bar, parity, abort_flag, p.err);
+                    return tc::wait_phase(bar, parity, abort_flag, p.err, wl);
                 };
                 auto kv_ready = [&](int j) {
                     const int jj = J + j;
@@ -675,7 +677,7 @@ __global__ void __launch_bounds__(PfCfg<T, D, KVT>::THREADS, 1)
         if (lane == 0) {
             const uint32_t drain = t == 0 ? bar_drain : bar_drain_b;
             tc::commit(drain);
-            (void)mbar_wait_bounded(drain, 0, kWaitLimitNs);
+            (void)mbar_wait_bounded(drain, 0, wl);
         }
         __syncwarp();
     } else if (warp >= 10 && warp < 10 + C::CONVERTERS) {
@@ -695,7 +697,7 @@ __global__ void __launch_bounds__(PfCfg<T, D, KVT>::THREADS, 1)
                 const PfItem w = decode_item<C::BN>(p, item, false);
                 if (w.state != 0) continue;
                 if (kv == 0) {
-                    ok = __all_sync(tc::kFull, tc::wait_phase(bar_q, kq & 1, abort_flag, p.err));
+                    ok = __all_sync(tc::kFull, tc::wait_phase(bar_q, kq & 1, abort_flag, p.err, wl));
                     int e = 0;
                     if (ok && std::is_same<T, bf16_t>::value) {
                         const int rows = tpt * g;  // rows the copy wrote in each tile
@@ -741,11 +743,11 @@ __global__ void __launch_bounds__(PfCfg<T, D, KVT>::THREADS, 1)
                 for (int j = 0; ok && j < w.nt; ++j) {
                     const int uu = U + j;
                     const int sst = uu % C::SST, st = uu % C::ST;
-                    ok = __all_sync(tc::kFull, tc::wait_phase(bar_stg_full(sst), (uu / C::SST) & 1, abort_flag, p.err));
+                    ok = __all_sync(tc::kFull, tc::wait_phase(bar_stg_full(sst), (uu / C::SST) & 1, abort_flag, p.err, wl));
                     if (!ok) break;
                     if (uu >= C::ST) {  // the MMAs are done with this operand stage
                         ok = __all_sync(tc::kFull,
-                                        tc::wait_phase(bar_kv_empty(st), ((uu / C::ST) - 1) & 1, abort_flag, p.err));
+                                        tc::wait_phase(bar_kv_empty(st), ((uu / C::ST) - 1) & 1, abort_flag, p.err, wl));
                         if (!ok) break;
                     }
                     {
@@ -826,7 +828,7 @@ __global__ void __launch_bounds__(PfCfg<T, D, KVT>::THREADS, 1)
             const int split = w.split;
             float sl2 = p.qk_scale_log2;  // > 0
             if constexpr (C::KV8) {  // q was scaled by 2^e on its way to f16
-                if (!__all_sync(tc::kFull, tc::wait_phase(bar_q_ready, kq & 1, abort_flag, p.err))) {
+                if (!__all_sync(tc::kFull, tc::wait_phase(bar_q_ready, kq & 1, abort_flag, p.err, wl))) {
                     ok = false;
                     break;
                 }
@@ -836,7 +838,7 @@ __global__ void __launch_bounds__(PfCfg<T, D, KVT>::THREADS, 1)
             float m_ref = -CUDART_INF_F, l = 0.f;
             for (int j = 0; j < nt; ++j) {
                 const int jj = J + j;
-                ok = __all_sync(tc::kFull, tc::wait_phase(bar_s_full(t, jj & 1), (jj >> 1) & 1, abort_flag, p.err));
+                ok = __all_sync(tc::kFull, tc::wait_phase(bar_s_full(t, jj & 1), (jj >> 1) & 1, abort_flag, p.err, wl));
                 if (!ok) break;
                 tc::fence_after();
                 const uint32_t scol = tmem + lane_bits + s_col(t, jj & 1);
@@ -891,7 +893,7 @@ __global__ void __launch_bounds__(PfCfg<T, D, KVT>::THREADS, 1)
                     // O may be rescaled only once the previous P.V of this tile is
                     // complete (the earlier ones completed before it)
                     ok = __all_sync(tc::kFull, tc::wait_phase(bar_pv(t, (jj - 1) & 1), ((jj - 1) >> 1) & 1,
-                                                             abort_flag, p.err));
+                                                             abort_flag, p.err, wl));
                     if (!ok) break;
                     tc::fence_after();
 #pragma unroll
@@ -910,7 +912,7 @@ __global__ void __launch_bounds__(PfCfg<T, D, KVT>::THREADS, 1)
             }
             if (ok) {
                 const int jl = J + nt - 1;
-                ok = __all_sync(tc::kFull, tc::wait_phase(bar_pv(t, jl & 1), (jl >> 1) & 1, abort_flag, p.err));
+                ok = __all_sync(tc::kFull, tc::wait_phase(bar_pv(t, jl & 1), (jl >> 1) & 1, abort_flag, p.err, wl));
             }
             if (!ok) break;
             // ---- epilogue: out = O / l, rounded once to the q dtype ----------------
@@ -1024,6 +1026,14 @@ cudaError_t launch_prefill_t(const PrefillParams &p, cudaStream_t stream) {
     e = cudaGetDevice(&dev);
     if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     if (e != cudaSuccess) return e;
+    // failure-detection test hook (see PrefillParams); unset in normal use
+    if (const char *env = getenv("PA369_TEST_PREFILL_STALL_NS")) {
+        const long long ns = atoll(env);
+        if (ns > 0) {
+            q.wait_limit_ns = (uint64_t)ns;
+            q.hold_first_tile = 1;
+        }
+    }
     static std::atomic<unsigned> next_slot{0};
     q.work_slot = (int)(next_slot.fetch_add(1u) % (unsigned)kWorkSlots);
     const unsigned grid = (unsigned)(items < sms ? items : sms);  // one CTA an SM, persistent

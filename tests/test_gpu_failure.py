@@ -91,3 +91,39 @@ def test_timeout_then_other_kernels_still_run(monkeypatch):
     pkc, pvc = oracle.chunked_caches_for(pw)
     assert_close(pre.out.float().cpu().numpy().astype(np.float64),
                  oracle.prefill_for(pw, pkc, pvc), "prefill after a timeout")
+
+
+@pytest.mark.parametrize("kv", ["bf16", "e4m3"])
+def test_prefill_wait_timeout_is_reported(kv, monkeypatch):
+    """The chunked prefill's abort path: with PA369_TEST_PREFILL_STALL_NS set
+    (read by the launch), every CTA leaves its first K/V stage's copies
+    unissued, so the wait on that stage runs out; the role that gives up raises
+    the CTA's abort flag, every other role leaves its own bounded wait, the
+    copies that were issued are drained and TMEM is freed.  The launch reports
+    PA_ERR_DEVICE_TIMEOUT, and a normal prefill on the same context right after
+    matches the oracle."""
+    pa, _ = _pa()
+    from paged_kv_cache_369_b200.runner import PagedPrefill
+
+    w = workload.build_chunked("prefill timeout", 6103, [5, 300], [40, 200], 16, 4, 128, "bf16", kv)
+    pkc, pvc = oracle.chunked_caches_for(w)
+    ref = oracle.prefill_for(w, pkc, pvc)
+    pre = PagedPrefill(w)
+    pre.step()
+    torch.cuda.synchronize()
+    assert pre.error() == 0
+    assert_close(pre.out.float().cpu().numpy().astype(np.float64), ref, "prefill before the timeout")
+
+    monkeypatch.setenv("PA369_TEST_PREFILL_STALL_NS", STALL_NS)
+    pre.dev_err.zero_()
+    pre.attend()
+    torch.cuda.synchronize()
+    assert pre.error() == pa.PA_ERR_DEVICE_TIMEOUT
+
+    monkeypatch.delenv("PA369_TEST_PREFILL_STALL_NS")
+    pre.dev_err.zero_()
+    pre.out.fill_(float("nan"))
+    pre.attend()
+    torch.cuda.synchronize()
+    assert pre.error() == 0
+    assert_close(pre.out.float().cpu().numpy().astype(np.float64), ref, "prefill after the timeout")
