@@ -162,7 +162,7 @@ struct PrefillParams {  // chunked prefill (pa_prefill)
     // shared-prefix mode (shared_len > 0): one "sequence" = the first
     // shared_len tokens of block table row 0; the T query rows (one per
     // decoding sequence) all see every one of them (no causal mask).  The
-    // keys are cut into gridDim.z ranges; range z writes each row's partial
+    // keys are cut into items_z ranges; range z writes each row's partial
     // (lse, o / l) to workspace slot z of ws_np per row
     int shared_len;
     float *ws_o;

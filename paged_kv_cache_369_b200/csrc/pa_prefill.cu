@@ -12,24 +12,30 @@
 // KV Cache、PagedAttention 与 vLLM", §3.3).  A decode step is the one-token
 // chunk.
 //
-// Work decomposition: one CTA per (sequence, KV head, pair of query tiles).
-// A query tile is 128 rows = floor(128 / g) chunk tokens x the g query heads
-// of the KV head (row r: token r / g, head r % g), so the whole GQA group
-// shares each K/V tile it reads; the CTA's two tiles (A, B: consecutive token
-// ranges) share them too.  Keys come in tiles of 64 = 4 blocks of 16 tokens.
-//   - warp 8 (one lane), TMA producer: both Q tiles once through a 3-D
-//     tensor map over q [T, Hq, d]; per key tile, the 4 K and 4 V blocks named
-//     by the block table through the pool's 2-D map (16-row x 128-byte boxes,
-//     128B swizzle) into a 4-stage ring.  Blocks past the sequence's end are
-//     fetched from past the end of the map, which the copy fills with zeros.
-//   - warp 9 (one lane), MMA issuer: S_t = Q_t K_j^T (M 128, N 64, K d) into
-//     one of tile t's two TMEM score buffers; O_t += P_t V_j with A = P read
-//     from TMEM and B = V from shared memory (MN-major).  Issue order per key
-//     tile j: PV_A(j), QK_A(j+2), PV_B(j), QK_B(j+2) -- every tile's next
-//     scores are ready before its softmax finishes, and the two tiles
-//     ping-pong on the tensor cores; tcgen05 operations of one thread run in
-//     issue order, which makes reusing a score buffer's columns for P and
-//     then for the scores two tiles later safe.
+// Work decomposition: a work item is (pair of query tiles, KV head,
+// sequence).  A query tile is 128 rows = floor(128 / g) chunk tokens x the g
+// query heads of the KV head (row r: token r / g, head r % g), so the whole
+// GQA group shares each K/V tile it reads; the item's two tiles (A, B:
+// consecutive token ranges) share them too.  Keys come in tiles of 64 = 4
+// blocks of 16 tokens.  The launch is persistent: one CTA an SM takes items
+// from a device counter until none are left, and every role below runs the
+// items in the same order with its barrier phases continuing from item to
+// item, so one item's first loads and MMAs overlap the previous one's last.
+//   - warp 8, TMA producer: takes the items and passes them on; per item both
+//     Q tiles through a 3-D tensor map over q [T, Hq, d], and per key tile the
+//     4 K and 4 V blocks named by the block table through the pool's 2-D map
+//     (16-row x 128-byte boxes, 128B swizzle; one copy per lane) into a
+//     4-stage ring.  Blocks past the sequence's end are fetched from past the
+//     end of the map, which the copy fills with zeros.
+//   - warps 9 (tile A) and 10 (tile B; 12 for 8-bit caches), MMA issuers, one
+//     lane each: S_t = Q_t K_j^T (M 128, N 64, K d) into one of tile t's two
+//     TMEM score buffers; O_t += P_t V_j with A = P read from TMEM and B = V
+//     from shared memory (MN-major).  Issue order per key tile j: PV_t(j),
+//     QK_t(j+2) -- the tile's next scores are ready before its softmax
+//     finishes, and while one issuer waits for its softmax the other keeps the
+//     tensor core busy; tcgen05 operations of one thread run in issue order,
+//     which makes reusing a score buffer's columns for P and then for the
+//     scores two tiles later safe.
 //   - warps 0-3 (tile A) and 4-7 (tile B), one thread per row: S from TMEM,
 //     causal mask by select on the diagonal tile only, the scale folded into
 //     one FFMA before ex2, online softmax with a lazy rescale (O and l are
@@ -43,7 +49,7 @@
 //     operand layout, so the MMAs run f16 x f16 (each code is exact in f16).
 // Shared-prefix mode (pa_decode_shared_prefix): the rows are the decoding
 // sequences' queries, every one of them sees all prefix keys (no mask), and
-// the prefix's key tiles are cut into gridDim.z ranges, each writing its own
+// the prefix's key tiles are cut into items_z ranges, each writing its own
 // partial (lse, o) workspace slot for the reduce to merge.
 // V rows past the sequence's last token (the tail of its last block) are
 // cleared in shared memory before P.V: p = 0 there, but 0 x NaN poison = NaN.
