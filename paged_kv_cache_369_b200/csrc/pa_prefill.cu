@@ -263,7 +263,13 @@ template <typename T, int D, typename KVT = T> struct PfCfg {
     static constexpr int OFF_QEXP = OFF_ABORT + 4;    // log2 of the q scaling, per item parity (8-bit caches)
     static constexpr int OFF_TAIL = OFF_QEXP + 8;     // tails of V claimed for clearing so far
     static constexpr int OFF_ITEM = OFF_TAIL + 4;     // the item ring's two slots
-    static constexpr int USED = OFF_ITEM + 8;
+    // 16-bit caches: each softmax warp's output rows pass through 4 KiB of
+    // shared memory (32 rows x 128 bytes, one 64-column half at a time), so the
+    // epilogue's global stores cover whole 128-byte row segments (8-bit caches
+    // have no room left for it)
+    static constexpr bool OSTAGE = !KV8;
+    static constexpr int OFF_OSTG = (OFF_ITEM + 8 + 127) / 128 * 128;
+    static constexpr int USED = OSTAGE ? OFF_OSTG + 8 * 4096 : OFF_ITEM + 8;
     // at least 120 KiB so that one CTA holds an SM (and its 512 TMEM columns)
     static constexpr int SMEM = 1024 + (USED < 120 * 1024 ? 120 * 1024 : USED);
     // MMA operand type: T, or f16 for 8-bit caches (codes widen to f16 exactly)
@@ -927,7 +933,50 @@ __global__ void __launch_bounds__(PfCfg<T, D, KVT>::THREADS, 1)
             // item's P.V (o_free).
             tc::fence_after();
             const float inv = l > 0.f ? p.v_scale / l : 0.f;  // v_scale: 1 for 16-bit caches
-            if (causal) {
+            if (causal && C::OSTAGE) {
+                // per 64-column half: the warp's 32 rows x 128 bytes into its
+                // shared-memory slab (16-byte chunk c of row r at chunk
+                // c ^ (r & 7): conflict-free), then read back four rows at a
+                // time, each lane one 16-byte chunk, and stored as 128-byte
+                // row segments
+                const uint32_t slab = base + C::OFF_OSTG + (uint32_t)warp * 4096u;
+                uint4 *out16 = reinterpret_cast<uint4 *>(p.out);
+                const int64_t row16 = row * (D / 8);  // 16-byte units
+#pragma unroll
+                for (int a = 0; a < C::ATOMS; ++a) {
+                    uint32_t wv[32];
+#pragma unroll
+                    for (int c = 0; c < 64; c += 32) {
+                        uint32_t o[32];
+                        tc::ld32(ocol + a * 64 + c, o);
+                        tc::wait_ld<32>(o);
+#pragma unroll
+                        for (int i = 0; i < 16; ++i)
+                            wv[c / 2 + i] =
+                                tc::pack2(__uint_as_float(o[2 * i]) * inv, __uint_as_float(o[2 * i + 1]) * inv, T{});
+                    }
+                    if (a == C::ATOMS - 1) {  // O is out of TMEM
+                        tc::fence_before();
+                        tc::mbar_arrive(bar_o_free(t));
+                    }
+#pragma unroll
+                    for (int c = 0; c < 8; ++c)
+                        asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(slab + lane * 128 + ((c ^ (lane & 7)) << 4)),
+                                     "r"(wv[4 * c]), "r"(wv[4 * c + 1]), "r"(wv[4 * c + 2]), "r"(wv[4 * c + 3])
+                                     : "memory");
+                    __syncwarp();
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        const int rr = 4 * i + (lane >> 3), c = lane & 7;  // the warp's row, its chunk
+                        const int ok_r = __shfl_sync(tc::kFull, (int)row_ok, rr);
+                        const int64_t dst = (int64_t)__shfl_sync(tc::kFull, (long long)row16, rr) + a * 8 + c;
+                        uint32_t v[4];
+                        lds<16>(v, slab + rr * 128 + ((c ^ (rr & 7)) << 4));
+                        if (ok_r) out16[dst] = make_uint4(v[0], v[1], v[2], v[3]);
+                    }
+                    __syncwarp();
+                }
+            } else if (causal) {
                 uint4 *dst = reinterpret_cast<uint4 *>(static_cast<uint16_t *>(p.out) + row * D);
 #pragma unroll
                 for (int c = 0; c < D; c += 32) {
