@@ -416,8 +416,9 @@ __global__ void __launch_bounds__(kDecodeWarps * 32)
 // Each lane owns D / 32 consecutive elements (one vector load per partition);
 // the warps take interleaved partitions, keeping kReduceUnroll partitions'
 // loads in flight per lane, and their sums meet in shared memory.  The
-// partition weights w_p = exp(lse_p - M) come from lse values every lane of
-// the warp reads at the same address (one broadcast load).
+// partition weights exp(lse_p - m) come from lse values every lane of the
+// warp reads at the same address (one broadcast load), against a running
+// maximum m per warp.
 // ---------------------------------------------------------------------------
 
 constexpr int kReduceWarps = 4;
@@ -459,22 +460,26 @@ __global__ void __launch_bounds__(kReduceWarps * 32) reduce_kernel(const ReduceP
     const VT *o = reinterpret_cast<const VT *>(p.ws_o + row * NP * D);
     const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
 
-    // M = max_p lse_p
-    float m = -CUDART_INF_F;
-    for (int i = threadIdx.x; i < np; i += kReduceWarps * 32) m = fmaxf(m, lse[i]);
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, off));
-    if (lane == 0) red[wid] = m;
-    __syncthreads();
-    float M = red[0];
-#pragma unroll
-    for (int w = 1; w < kReduceWarps; ++w) M = fmaxf(M, red[w]);
-
+    // One pass: each warp keeps a running (m, den, acc) over its partitions,
+    // rescaled when a batch brings a larger lse (no separate pass for the
+    // maximum); the warps' states meet in shared memory.
+    float m = -CUDART_INF_F, den = 0.f;
     float acc[V];
 #pragma unroll
     for (int j = 0; j < V; ++j) acc[j] = 0.f;
-    float den = 0.f;
-    if (M != -CUDART_INF_F) {
+    auto absorb = [&](float lv, const VT &v) {  // one partition, m already >= lv
+        const float w = lv == -CUDART_INF_F ? 0.f : expf(lv - m);
+        den += w;
+        VF::add(acc, w, v);
+    };
+    auto rescale_to = [&](float mb) {  // raise m to mb (> m)
+        const float sc = m == -CUDART_INF_F ? 0.f : expf(m - mb);
+        den *= sc;
+#pragma unroll
+        for (int j = 0; j < V; ++j) acc[j] *= sc;
+        m = mb;
+    };
+    {
         constexpr int STRIDE = kReduceWarps * kReduceUnroll;
         int i0 = wid;
         for (; i0 + (kReduceUnroll - 1) * kReduceWarps < np; i0 += STRIDE) {
@@ -486,22 +491,29 @@ __global__ void __launch_bounds__(kReduceWarps * 32) reduce_kernel(const ReduceP
                 v[u] = o[(int64_t)i * (D / V) + lane];
                 lv[u] = lse[i];
             }
+            float mb = lv[0];
 #pragma unroll
-            for (int u = 0; u < kReduceUnroll; ++u) {
-                const float w = expf(lv[u] - M);
-                den += w;
-                VF::add(acc, w, v[u]);
-            }
+            for (int u = 1; u < kReduceUnroll; ++u) mb = fmaxf(mb, lv[u]);
+            if (mb > m) rescale_to(mb);
+#pragma unroll
+            for (int u = 0; u < kReduceUnroll; ++u) absorb(lv[u], v[u]);
         }
         for (int i = i0; i < np; i += kReduceWarps) {
-            const float w = expf(lse[i] - M);
-            den += w;
-            VF::add(acc, w, o[(int64_t)i * (D / V) + lane]);
+            const float lv = lse[i];
+            const VT v = o[(int64_t)i * (D / V) + lane];
+            if (lv > m) rescale_to(lv);
+            absorb(lv, v);
         }
     }
+    if (lane == 0) red[wid] = m;
+    __syncthreads();
+    float M = red[0];
 #pragma unroll
-    for (int j = 0; j < V; ++j) part_num[wid][lane * V + j] = acc[j];
-    if (lane == 0) part_den[wid] = den;
+    for (int w = 1; w < kReduceWarps; ++w) M = fmaxf(M, red[w]);
+    const float sc = m == -CUDART_INF_F ? 0.f : expf(m - M);  // this warp's share at M
+#pragma unroll
+    for (int j = 0; j < V; ++j) part_num[wid][lane * V + j] = acc[j] * sc;
+    if (lane == 0) part_den[wid] = den * sc;
     __syncthreads();
     for (int d = threadIdx.x; d < D; d += kReduceWarps * 32) {
         float num = 0.f, dsum = 0.f;
