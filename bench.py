@@ -119,16 +119,17 @@ def same_run_copy_gbs(device, stream, nbytes: int = 512 * 1024 * 1024, reps: int
     return 2.0 * nbytes / (ms * 1e-3) / 1e9
 
 
-def recorded_traffic(cfg: int, mode: str, path=None):
+def recorded_traffic(cfg: int, mode: str, path=None, key=None):
     """DRAM bytes per attention launch from the committed ncu summary, if it
-    was taken on the current kernel sources (else None)."""
+    was taken on the current kernel sources (else None).  `key` names an
+    entry directly (e.g. a prefill workload)."""
     path = path or os.path.join(ROOT, "profiles", "decode_traffic.json")
     try:
         with open(path) as f:
             rec = json.load(f)
     except Exception:  # noqa: BLE001
         return None
-    key = f"config{cfg}_{mode}"
+    key = key or f"config{cfg}_{mode}"
     ent = rec.get(key)
     if not ent or ent.get("kernel_hash") != kernel_source_hash(tuple(ent.get("sources", DECODE_SOURCES))):
         return None
@@ -492,7 +493,9 @@ def run_prefill(args):
         "attention_us": attn_ms * 1e3, "cache_write_us": (step_ms - attn_ms) * 1e3,
         "tokens_per_s": w.num_tokens / (step_ms * 1e-3),
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                     "frac": achieved / peak, "traffic": None, "kernel": "prefill_kernel (tcgen05)",
+                     "frac": achieved / peak,
+                     "traffic": recorded_traffic(0, "", key=f"prefill_pconfig{args.pconfig}_{w.kv_dtype}"),
+                     "kernel": "prefill_kernel (tcgen05)",
                      "algorithmic_flops_per_launch": flops,
                      "peak_source": f"{kind} dense bf16 (cuBLAS burst, MEASURED_PEAKS.json bf16_tflops)"},
         "gpu_launches": 3 * args.steps, "clocks": clocks.summary(), "device_error": pre.error(),
