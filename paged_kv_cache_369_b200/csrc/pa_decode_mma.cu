@@ -284,6 +284,17 @@ __global__ void __launch_bounds__(NWARPS * 32, MmaCfg<QT, KVT, D, GT, NWARPS>::M
 
     pdl_wait();
 
+    // ---- the block-table entries of this warp's first 32 tiles, one per lane,
+    // read before the sequence length is known (any index inside the table
+    // row is readable), so the two loads are in flight together
+    const int32_t *bt_row = p.block_tables + (int64_t)s * p.max_blocks_per_seq;
+    const int blk_begin = p.tile_begin + part * p.partition_blocks;
+    auto table_at = [&](int k) -> int {  // the block holding the warp's tile k
+        const int idx = (blk_begin + warp + NW * k) >> p.tile_shift;
+        return (unsigned)idx < (unsigned)p.max_blocks_per_seq ? bt_row[idx] : 0;
+    };
+    const int bt_first = table_at(lane);
+
     // ---- sequence length and this CTA's block range -----------------------
     const int max_tokens = p.max_blocks_per_seq * p.block_size;
     int L = p.seq_lens[s];
@@ -304,7 +315,6 @@ __global__ void __launch_bounds__(NWARPS * 32, MmaCfg<QT, KVT, D, GT, NWARPS>::M
         if (threadIdx.x == 0 && part == 0) flag_error(p.err, kErrBounds);
         L = p.tile_begin * kBlockSize;
     }
-    const int blk_begin = p.tile_begin + part * p.partition_blocks;
     int blk_end = blk_begin + p.partition_blocks;
     if (blk_end > nblk_seq) blk_end = nblk_seq;
     if (p.split && blk_begin >= blk_end) return;
@@ -312,15 +322,14 @@ __global__ void __launch_bounds__(NWARPS * 32, MmaCfg<QT, KVT, D, GT, NWARPS>::M
     const int nk = nblk > warp ? (nblk - warp + NW - 1) / NW : 0;
 
     // ---- block table entries of this warp, one per lane --------------------
-    const int32_t *bt_row = p.block_tables + (int64_t)s * p.max_blocks_per_seq;
     auto load_batch = [&](int batch) -> int {  // the block holding each of the warp's tiles
         const int k = batch * 32 + lane;
-        return k < nk ? bt_row[(blk_begin + warp + NW * k) >> p.tile_shift] : 0;
+        return k < nk ? table_at(k) : 0;
     };
     const int tile_mask = (1 << p.tile_shift) - 1;
     const uint64_t kv_policy = policy_evict_first();
     int cur_batch = 0;
-    int bt_cur = load_batch(0);
+    int bt_cur = lane < nk ? bt_first : 0;
     int bt_nxt = nk > 32 ? load_batch(1) : 0;
     auto bt_of = [&](int k) -> int {
         const int a = __shfl_sync(kFull, bt_cur, k & 31);
