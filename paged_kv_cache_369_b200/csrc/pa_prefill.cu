@@ -235,6 +235,13 @@ __device__ __forceinline__ void unpack2(uint32_t w, float &lo, float &hi, bf16_t
 
 }  // namespace tc
 
+// Work items are taken longest first where that is cheap to know: with up to
+// kOrderSeqs sequences the TMA warp ranks them by cached context (the chunks
+// of one launch are alike) and hands out, per sequence in that order, its
+// query tile pairs last first (they see the most keys); the item index it
+// publishes is the natural one below.
+constexpr int kOrderSeqs = 128;
+
 // T: q / out dtype; KVT: cache dtype (T, or an 8-bit code for which two
 // converter warps widen each landed K and V tile to f16 in shared memory).
 template <typename T, int D, typename KVT = T> struct PfCfg {
@@ -263,13 +270,14 @@ template <typename T, int D, typename KVT = T> struct PfCfg {
     static constexpr int OFF_QEXP = OFF_ABORT + 4;    // log2 of the q scaling, per item parity (8-bit caches)
     static constexpr int OFF_TAIL = OFF_QEXP + 8;     // tails of V claimed for clearing so far
     static constexpr int OFF_ITEM = OFF_TAIL + 4;     // the item ring's two slots
+    static constexpr int OFF_ORDER = OFF_ITEM + 8;    // sequences by context length, then their contexts
     // 16-bit caches: each softmax warp's output rows pass through 4 KiB of
     // shared memory (32 rows x 128 bytes, one 64-column half at a time), so the
     // epilogue's global stores cover whole 128-byte row segments (8-bit caches
     // have no room left for it)
     static constexpr bool OSTAGE = !KV8;
-    static constexpr int OFF_OSTG = (OFF_ITEM + 8 + 127) / 128 * 128;
-    static constexpr int USED = OSTAGE ? OFF_OSTG + 8 * 4096 : OFF_ITEM + 8;
+    static constexpr int OFF_OSTG = (OFF_ORDER + 8 * kOrderSeqs + 127) / 128 * 128;
+    static constexpr int USED = OSTAGE ? OFF_OSTG + 8 * 4096 : OFF_ORDER + 8 * kOrderSeqs;
     // at least 120 KiB so that one CTA holds an SM (and its 512 TMEM columns)
     static constexpr int SMEM = 1024 + (USED < 120 * 1024 ? 120 * 1024 : USED);
     // MMA operand type: T, or f16 for 8-bit caches (codes widen to f16 exactly)
@@ -480,12 +488,38 @@ __global__ void __launch_bounds__(PfCfg<T, D, KVT>::THREADS, 1)
         auto empty_bar = [&](int st) { return C::KV8 ? bar_stg_empty(st) : bar_kv_empty(st); };
         int U = 0, kq = 0;  // key tiles issued, items with work (Q loads)
         bool ok = true;
+        // the order items are handed out in (see kOrderSeqs)
+        int *order = reinterpret_cast<int *>(smem + C::OFF_ORDER);
+        const bool ordered = causal && p.num_seqs <= kOrderSeqs;
+        if (ordered) {
+            volatile int *ctxs = order + kOrderSeqs;
+            for (int q = lane; q < p.num_seqs; q += 32)
+                ctxs[q] = p.seq_lens[q] - (p.query_start[q + 1] - p.query_start[q]);
+            __syncwarp();
+            for (int q = lane; q < p.num_seqs; q += 32) {
+                const int cq = ctxs[q];
+                int rank = 0;
+                for (int o = 0; o < p.num_seqs; ++o) {
+                    const int co = ctxs[o];
+                    rank += (co > cq) || (co == cq && o < q);
+                }
+                order[rank] = q;
+            }
+            __syncwarp();
+        }
+        auto natural_item = [&](int c) -> int {  // c-th item handed out -> its natural index
+            if (!ordered) return c;
+            const int per_seq = p.items_x * p.num_kv_heads;
+            const int r = c / per_seq, rem = c - r * per_seq;
+            const int x = p.items_x - 1 - rem / p.num_kv_heads, kvh = rem % p.num_kv_heads;
+            return (order[r] * p.num_kv_heads + kvh) * p.items_x + x;
+        };
         for (int k = 0; ok; ++k) {
             // take an item and publish it to the ring (slot k & 1)
             int item = -1;
             if (lane == 0) {
                 item = (int)atomicAdd(&g_prefill_work[p.work_slot][0], 1u);
-                if (item >= n_items) item = -1;
+                item = item < n_items ? natural_item(item) : -1;
                 if (k >= 2) ok = tc::wait_phase(bar_item_empty(k & 1), ((k >> 1) - 1) & 1, abort_flag, p.err, wl);
                 item_slot[k & 1] = ok ? item : -1;
                 tc::mbar_arrive(bar_item_full(k & 1));
