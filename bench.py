@@ -653,18 +653,19 @@ def time_end_to_end(dec, stream, device, steps: int, flush=None):
 
 def per_config_measurements(device, stream, steps: int, warmup: int):
     """Attention time, roofline fraction and clocks of the other named decode
-    workloads, each in its default launch configuration: configs 3 and 4 as a
-    fused step (1024- / 512-token partitions), config 5 with its shared prefix
-    attended once (cascade).  Each is timed like the headline, on its own."""
+    workloads, each in its default launch configuration: config 3 as a fused
+    single-pass step, config 4 as a fused step with the 512-token partitions
+    it prescribes, config 5 with its shared prefix attended once (cascade,
+    768-token partitions).  Each is timed like the headline, on its own."""
     import torch
 
     import workload
     from paged_kv_cache_369_b200.runner import (PagedDecode, algorithmic_cascade_bytes,
-                                                default_partition_size)
+                                                default_mode, default_partition_size)
 
     peak, _ = measured_hbm_peak()
     res = {}
-    for cfg, mode in ((3, "fused"), (4, "fused"), (5, "cascade")):
+    for cfg, mode in ((3, default_mode(3)), (4, default_mode(4)), (5, "cascade")):
         w = workload.config(cfg)
         P = default_partition_size(w, cfg)
         with torch.cuda.stream(stream):
@@ -842,11 +843,12 @@ def main(argv=None):
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--config", type=int, default=2, choices=(1, 2, 3, 4, 5))
     ap.add_argument("--mode", choices=("fused", "fused_single", "split", "single", "cascade"),
-                    default="fused",
-                    help="cascade: the shared-prefix decode (config 5's common prefix attended once)")
+                    default=None,
+                    help="default: fused_single for config 3, else fused; cascade: the "
+                         "shared-prefix decode (config 5's common prefix attended once)")
     ap.add_argument("--partition", type=int, default=None,
                     help="split-KV partition in tokens (default: 512 for config 4, as it "
-                         "prescribes, else 1024)")
+                         "prescribes, 768 for config 5, else 1024)")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-per-config", action="store_true",
@@ -867,8 +869,12 @@ def main(argv=None):
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
-    if args.partition is None:  # as runner.default_partition_size: 512 where prescribed
-        args.partition = 512 if args.config == 4 else 1024
+    if args.mode is None or args.partition is None:
+        from paged_kv_cache_369_b200.runner import default_mode, default_partition_size
+        if args.mode is None:
+            args.mode = default_mode(args.config)
+        if args.partition is None:
+            args.partition = default_partition_size(None, args.config)
     if args.channel_scales:
         if args.kv is None and args.config != 4:
             ap.error("--channel-scales needs an 8-bit cache (--kv or config 4)")

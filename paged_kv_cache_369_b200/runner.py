@@ -178,13 +178,25 @@ class PagedDecode:
 
 def default_partition_size(w, config_id=None) -> int:
     """Split-KV partition for a named decode workload: 512 tokens where the
-    workload prescribes it (the long-context configuration, config 4), else
-    1024 -- measured on B200 with 256 / 512 / 768 / 1024: Qwen3-8B shape
-    113.5 / 105.8 / 103.7 / 102.6 us, Llama-3-70B shape 76.2 / 67.4 / 66.6 /
-    67.1 us, shared-prefix batch 285.7 / 239.5 / 229.8 / 233.1 us."""
+    workload prescribes it (the long-context configuration, config 4); 768
+    for the shared-prefix batch (config 5); else 1024.  Measured on B200
+    (graph-timed steps) with 512 / 768 / 1024 / 2048: Qwen3-8B shape 96.7 /
+    96.1 / 95.1 / 100.0 us; shared-prefix batch, cascade, 214.0 / 211.0 /
+    212.6 / 217.0 us."""
     if config_id == 4:
         return 512
+    if config_id == 5:
+        return 768
     return 1024
+
+
+def default_mode(config_id=None) -> str:
+    """Step for a named decode workload: the fused step (the decode kernel
+    stores the new tokens) with split-KV partitions, except for the
+    Llama-3-70B shape (config 3), whose even lengths (2048-2560) run best in
+    one pass per (sequence, KV head): 52.1 us, against 58.4 / 56.2 / 52.7 us
+    with 1024- / 2048- / 2560-token partitions."""
+    return "fused_single" if config_id == 3 else "fused"
 
 
 def algorithmic_decode_bytes(w) -> int:

@@ -372,17 +372,18 @@ def _full(cfg, kv=None):
                                     (4, "e5m2"), (4, "int8"), (4, "e4m3-channel")])
 def test_named_workload_parity(cfg, kv):
     """Each named workload at full size, first in exactly the launch
-    configuration bench.py times (fused step, the workload's default
+    configuration bench.py times (the workload's default fused step and
     split-KV partition), then split, single-pass and CUDA-core launches on the
     same state, and split-KV at 512-token partitions where the default
     differs."""
     pa, PagedDecode = _pa()
-    from paged_kv_cache_369_b200.runner import default_partition_size
+    from paged_kv_cache_369_b200.runner import default_mode, default_partition_size
 
     w, kc, vc = _full(cfg, kv)
     chan = w.k_chan is not None
     P = default_partition_size(w, cfg)
-    dec = PagedDecode(w, mode="split" if chan else "fused", partition_size=P)
+    mode = "split" if chan else default_mode(cfg)
+    dec = PagedDecode(w, mode=mode, partition_size=P)
     dec.step()  # pa_decode_append: the attention launch stores the new tokens
     torch.cuda.synchronize()
     assert dec.error() == 0
@@ -391,7 +392,7 @@ def test_named_workload_parity(cfg, kv):
     assert np.isfinite(out_split).all()
     pairs = sample_pairs(w, 64 if cfg > 1 else w.num_seqs * w.num_q_heads, seed=cfg)
     ref = oracle.decode_for(w, kc, vc, pairs)
-    assert_close(out_split[pairs[:, 0], pairs[:, 1]], ref, f"config {cfg} fused split P={P}")
+    assert_close(out_split[pairs[:, 0], pairs[:, 1]], ref, f"config {cfg} {mode} P={P}")
     # unfused split attention on the same state
     dec.mode = "split"
     dec.attend()
