@@ -63,13 +63,13 @@ def _scale_rows(bits, dtype, factor, rows=slice(None)):
 
 @pytest.mark.parametrize("kind", ["huge", "tiny", "early_block", "late_block"])
 def test_prefill_bf16_value_range(kind):
-    """bf16 caches: P.V runs in f16 on V tiles scaled by 2^-k (k from each
-    tile's largest magnitude), so V values far outside f16's range must come
-    out as the oracle's: all V times 2^20 or 2^-40, or one 16-token block of
-    the context times 2^18 in the first key tile (later tiles get a smaller P
-    scale) or in a later one (the output is rescaled when it arrives).  Each
-    sequence's rows are compared after dividing by a power of two near their
-    largest magnitude (exact), with the usual bars."""
+    """bf16 caches hold values far outside f16's range, which a P.V in f16
+    (V converted per tile with a power-of-two scale) would have to carry and
+    the bf16 hi + lo P.V carries as they are: all V times 2^20 or 2^-40, or
+    one 16-token block of the context times 2^18, in the first key tile or in
+    a later one.  The output must come out as the oracle's.  Each sequence's
+    rows are compared after dividing by a power of two near their largest
+    magnitude (exact), with the usual bars."""
     w = workload.build_chunked(f"range {kind}", 2900, [0, 230, 90], [150, 40, 64], 32, 8, 128,
                                "bf16", "bf16")
     if kind in ("huge", "tiny"):
