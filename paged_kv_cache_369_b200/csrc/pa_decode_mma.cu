@@ -33,6 +33,7 @@
 #include <cudaTypedefs.h>
 #include <math_constants.h>
 
+#include <cstdlib>
 #include <type_traits>
 
 #include "pa_device.cuh"
@@ -250,8 +251,9 @@ __device__ __forceinline__ uint32_t swz(int r, int c) {
 }
 
 // CHAN: per-channel scales (8-bit caches only), a separate instantiation so
-// that the per-tensor kernels compile exactly as without them
-template <typename QT, typename KVT, int D, int GT, bool CHAN, int NWARPS>
+// that the per-tensor kernels compile exactly as without them.  CHAINED: each
+// warp attends p.chain consecutive partitions alone (long split contexts).
+template <typename QT, typename KVT, int D, int GT, bool CHAN, int NWARPS, bool CHAINED>
 __global__ void __launch_bounds__(NWARPS * 32, MmaCfg<QT, KVT, D, GT, NWARPS>::MIN_CTAS)
     decode_mma_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmap_k,
                       const __grid_constant__ CUtensorMap tmap_v) {
@@ -267,7 +269,12 @@ __global__ void __launch_bounds__(NWARPS * 32, MmaCfg<QT, KVT, D, GT, NWARPS>::M
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int g = lane >> 2, kq = lane & 3;  // MMA fragment coordinates
     const int NP = p.num_partitions;
-    const int s = blockIdx.x / NP, part = blockIdx.x - s * NP;
+    // chained (long split contexts): each warp attends p.chain consecutive
+    // partitions alone; otherwise the CTA's warps share one partition
+    constexpr bool chain = CHAINED;
+    const int cps = chain ? (NP + NW * p.chain - 1) / (NW * p.chain) : NP;  // CTAs per sequence
+    const int s = blockIdx.x / cps, cta = blockIdx.x - s * cps;
+    const int part = chain ? (cta * NW + warp) * p.chain : cta;  // the (first) partition
     const int kvh = blockIdx.y / p.head_groups, hg = blockIdx.y - kvh * p.head_groups;
 
     const uint32_t bar0 = base_addr + C::OFF_BAR + warp * NST * 8;
@@ -289,8 +296,11 @@ __global__ void __launch_bounds__(NWARPS * 32, MmaCfg<QT, KVT, D, GT, NWARPS>::M
     // row is readable), so the two loads are in flight together
     const int32_t *bt_row = p.block_tables + (int64_t)s * p.max_blocks_per_seq;
     const int blk_begin = p.tile_begin + part * p.partition_blocks;
+    auto tile_of = [&](int k) -> int {  // the warp's k-th 16-token tile
+        return chain ? blk_begin + k : blk_begin + warp + NW * k;
+    };
     auto table_at = [&](int k) -> int {  // the block holding the warp's tile k
-        const int idx = (blk_begin + warp + NW * k) >> p.tile_shift;
+        const int idx = tile_of(k) >> p.tile_shift;
         return (unsigned)idx < (unsigned)p.max_blocks_per_seq ? bt_row[idx] : 0;
     };
     const int bt_first = table_at(lane);
@@ -315,11 +325,13 @@ __global__ void __launch_bounds__(NWARPS * 32, MmaCfg<QT, KVT, D, GT, NWARPS>::M
         if (threadIdx.x == 0 && part == 0) flag_error(p.err, kErrBounds);
         L = p.tile_begin * kBlockSize;
     }
-    int blk_end = blk_begin + p.partition_blocks;
+    int span = p.partition_blocks;
+    if (chain) span *= NP - part < p.chain ? (NP - part > 0 ? NP - part : 0) : p.chain;
+    int blk_end = blk_begin + span;
     if (blk_end > nblk_seq) blk_end = nblk_seq;
-    if (p.split && blk_begin >= blk_end) return;
+    if (p.split && blk_begin >= blk_end) return;  // (chained: no CTA barrier follows)
     const int nblk = blk_end > blk_begin ? blk_end - blk_begin : 0;
-    const int nk = nblk > warp ? (nblk - warp + NW - 1) / NW : 0;
+    const int nk = chain ? nblk : (nblk > warp ? (nblk - warp + NW - 1) / NW : 0);
 
     // ---- block table entries of this warp, one per lane --------------------
     auto load_batch = [&](int batch) -> int {  // the block holding each of the warp's tiles
@@ -345,7 +357,7 @@ __global__ void __launch_bounds__(NWARPS * 32, MmaCfg<QT, KVT, D, GT, NWARPS>::M
             }
             const uint32_t bar = bar0 + 8 * st;
             const uint32_t dst = stage0 + st * C::STAGE_BYTES;
-            const int sub = (blk_begin + warp + NW * k) & tile_mask;  // tile within the block
+            const int sub = tile_of(k) & tile_mask;  // tile within the block
             const int y = (phys * p.num_kv_heads + kvh) * p.block_size + sub * kBlockSize;
             mbar_arrive_expect_tx(bar, C::STAGE_BYTES);
 #pragma unroll
@@ -508,6 +520,75 @@ __global__ void __launch_bounds__(NWARPS * 32, MmaCfg<QT, KVT, D, GT, NWARPS>::M
     const int lsel_b = (lane >> 3) & 1;                 // q.K: chunk +0 | +1
     const int lrow_v = (lane & 7) + 8 * ((lane >> 3) & 1);  // P.V: tokens 0-7 | 8-15
     const int lsel_v = lane >> 4;                       // P.V: chunk +0 | +1
+    // chained: partition pp's partial (lse, o / l) straight from the
+    // registers, then a fresh softmax state for the next partition
+    auto flush = [&](int pp) {
+        const int ws_np = p.ws_np > 0 ? p.ws_np : NP, slot = p.ws_offset + pp;
+        const int group_base = hg * GT;
+        const int64_t row0 = (int64_t)s * p.num_q_heads + (int64_t)kvh * p.group + group_base;
+        float lq[NR];
+#pragma unroll
+        for (int r = 0; r < NR; ++r) {
+            lq[r] = l_run[r] + __shfl_xor_sync(kFull, l_run[r], 1);
+            lq[r] += __shfl_xor_sync(kFull, lq[r], 2);
+        }
+        if (kq == 0) {
+#pragma unroll
+            for (int r = 0; r < NR; ++r) {
+                const int head = g + 8 * r;
+                if (group_base + head < p.group)
+                    p.ws_lse[(row0 + head) * ws_np + slot] =
+                        lq[r] > 0.f ? (m_run[r] + log2f(lq[r])) * 0.69314718055994530942f : -CUDART_INF_F;
+            }
+        }
+#pragma unroll
+        for (int nh = 0; nh < C::NH; ++nh) {
+            // the O^T columns of this lane: heads ha = 8 nh + 2 kq and ha + 1,
+            // whose sums sit in the lanes with that softmax row
+            const int ha = 8 * nh + 2 * kq;
+            const float la = __shfl_sync(kFull, lq[nh], (2 * kq) * 4);
+            const float lb = __shfl_sync(kFull, lq[nh], (2 * kq + 1) * 4);
+            const float ia = la > 0.f ? 1.f / la : 0.f, ib = lb > 0.f ? 1.f / lb : 0.f;
+            const bool va = group_base + ha < p.group, vb = group_base + ha + 1 < p.group;
+            float *oa = p.ws_o + ((row0 + ha) * ws_np + slot) * D;
+            float *ob = oa + (int64_t)ws_np * D;
+#pragma unroll
+            for (int mt = 0; mt < C::MT; ++mt) {
+                if constexpr (C::FP8) {  // d-rows 2g, 2g + 1 of m-tile mt
+                    const int d0 = 16 * mt + 2 * g;
+                    float s0 = p.v_scale, s1 = p.v_scale;
+                    if constexpr (CHAN) {
+                        s0 = p.v_chan[(int64_t)kvh * D + d0];
+                        s1 = p.v_chan[(int64_t)kvh * D + d0 + 1];
+                    }
+                    if (va) *reinterpret_cast<float2 *>(oa + d0) = make_float2(o[mt][nh][0] * ia * s0, o[mt][nh][2] * ia * s1);
+                    if (vb) *reinterpret_cast<float2 *>(ob + d0) = make_float2(o[mt][nh][1] * ib * s0, o[mt][nh][3] * ib * s1);
+                } else {  // d-rows g, g + 8
+                    const int d0 = 16 * mt + g;
+                    if (va) {
+                        oa[d0] = o[mt][nh][0] * ia * p.v_scale;
+                        oa[d0 + 8] = o[mt][nh][2] * ia * p.v_scale;
+                    }
+                    if (vb) {
+                        ob[d0] = o[mt][nh][1] * ib * p.v_scale;
+                        ob[d0 + 8] = o[mt][nh][3] * ib * p.v_scale;
+                    }
+                }
+            }
+        }
+#pragma unroll
+        for (int r = 0; r < NR; ++r) {
+            m_run[r] = -CUDART_INF_F;
+            l_run[r] = 0.f;
+        }
+#pragma unroll
+        for (int mt = 0; mt < C::MT; ++mt)
+#pragma unroll
+            for (int nh = 0; nh < C::NH; ++nh)
+#pragma unroll
+                for (int i = 0; i < 4; ++i) o[mt][nh][i] = 0.f;
+    };
+
     bool timed_out = false;
     int k = 0;
     int st = 0;          // k % NST
@@ -525,7 +606,7 @@ __global__ void __launch_bounds__(NWARPS * 32, MmaCfg<QT, KVT, D, GT, NWARPS>::M
             timed_out = true;
             break;
         }
-        const int j = blk_begin + warp + NW * k;
+        const int j = tile_of(k);
         const bool valid = (unsigned)bt_of(k) < (unsigned)p.num_blocks;
         int nvalid = L - j * kBlockSize;
         nvalid = valid ? (nvalid < kBlockSize ? nvalid : kBlockSize) : 0;
@@ -748,6 +829,9 @@ __global__ void __launch_bounds__(NWARPS * 32, MmaCfg<QT, KVT, D, GT, NWARPS>::M
             st = 0;
             phase ^= 1u;
         }
+        if constexpr (CHAINED) {
+            if ((k + 1) % p.partition_blocks == 0 || k + 1 == nk) flush(part + k / p.partition_blocks);
+        }
     }
 
     if (timed_out) {
@@ -759,6 +843,7 @@ __global__ void __launch_bounds__(NWARPS * 32, MmaCfg<QT, KVT, D, GT, NWARPS>::M
     }
 
     pdl_launch_dependents();
+    if constexpr (CHAINED) return;  // every partition's partial is written
 
     // ---- merge the warps' partial states ---------------------------------------
 #pragma unroll
@@ -867,7 +952,7 @@ bool encode_pool_map(CUtensorMap *m, const void *base, int elem_bytes, int d, in
 
 namespace {
 
-template <typename QT, typename KVT, int D, int GT, bool CHAN, int NWARPS>
+template <typename QT, typename KVT, int D, int GT, bool CHAN, int NWARPS, bool CHAINED>
 cudaError_t launch_mma_t(const DecodeParams &p, cudaStream_t stream) {
     using C = MmaCfg<QT, KVT, D, GT, NWARPS>;
     const int64_t rows = (int64_t)p.num_blocks * p.num_kv_heads * p.block_size;
@@ -875,11 +960,13 @@ cudaError_t launch_mma_t(const DecodeParams &p, cudaStream_t stream) {
     if (!encode_pool_map(&mk, p.k_cache, C::EB, D, rows) ||
         !encode_pool_map(&mv, p.v_cache, C::EB, D, rows))
         return cudaErrorInvalidValue;
-    auto kern = decode_mma_kernel<QT, KVT, D, GT, CHAN, NWARPS>;
+    auto kern = decode_mma_kernel<QT, KVT, D, GT, CHAN, NWARPS, CHAINED>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)(p.num_seqs * p.num_partitions), (unsigned)(p.num_kv_heads * p.head_groups));
+    if (CHAINED != (p.chain > 0)) return cudaErrorInvalidValue;
+    const int cps = CHAINED ? (p.num_partitions + C::NW * p.chain - 1) / (C::NW * p.chain) : p.num_partitions;
+    cfg.gridDim = dim3((unsigned)(p.num_seqs * cps), (unsigned)(p.num_kv_heads * p.head_groups));
     cfg.blockDim = dim3(C::NW * 32);
     cfg.dynamicSmemBytes = C::SMEM;
     cfg.stream = stream;
@@ -900,13 +987,49 @@ cudaError_t launch_mma_t(const DecodeParams &p, cudaStream_t stream) {
 // vs 111.9 us).
 constexpr int kLongSplitPartitions = 16;
 
+// Long split contexts: with at least as many partitions as the device holds
+// resident warps, each warp attends floor(partitions / resident warps) (at
+// most 4) consecutive partitions alone (DecodeParams::chain): no merge of
+// warps' states within a CTA, and the partials written straight from
+// registers (long-context E4M3 shape, 4096 partitions of 512 tokens over
+// 2368 resident warps: 109.8 us with two warps sharing each partition, 100.4
+// with one warp a partition, 108.4 with two partitions a warp).  With fewer
+// partitions (0 here) a CTA's two warps share each one, so that every
+// resident warp has work.  The environment variable PA369_DECODE_CHAIN (a
+// count, 1 .. 64) overrides the choice; it is kept for A/B measurement and
+// tests.
+template <typename C> int chain_length(const DecodeParams &p) {
+    if (const char *env = getenv("PA369_DECODE_CHAIN")) {
+        const int r = atoi(env);
+        if (r > 0) return r < 64 ? r : 64;
+    }
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0)
+        sms = 148;
+    const int64_t slots = (int64_t)sms * C::MIN_CTAS * C::NW;  // resident warps
+    const int64_t parts = (int64_t)p.num_seqs * p.num_partitions * p.num_kv_heads * p.head_groups;
+    const int64_t r = parts / slots;
+    return (int)(r > 4 ? 4 : r);
+}
+
 template <typename QT, typename KVT, int D, bool CHAN>
 cudaError_t mma_by_warps(const DecodeParams &p, int gt, cudaStream_t stream) {
-    if (p.split && p.num_partitions >= kLongSplitPartitions)
-        return gt == 16 ? launch_mma_t<QT, KVT, D, 16, CHAN, 2>(p, stream)
-                        : launch_mma_t<QT, KVT, D, 8, CHAN, 2>(p, stream);
-    return gt == 16 ? launch_mma_t<QT, KVT, D, 16, CHAN, kDecodeWarps>(p, stream)
-                    : launch_mma_t<QT, KVT, D, 8, CHAN, kDecodeWarps>(p, stream);
+    if (p.split && p.num_partitions >= kLongSplitPartitions) {
+        DecodeParams q = p;
+        if (gt == 16) {
+            q.chain = chain_length<MmaCfg<QT, KVT, D, 16, 2>>(p);
+            return q.chain > 0 ? launch_mma_t<QT, KVT, D, 16, CHAN, 2, true>(q, stream)
+                               : launch_mma_t<QT, KVT, D, 16, CHAN, 2, false>(q, stream);
+        }
+        q.chain = chain_length<MmaCfg<QT, KVT, D, 8, 2>>(p);
+        return q.chain > 0 ? launch_mma_t<QT, KVT, D, 8, CHAN, 2, true>(q, stream)
+                           : launch_mma_t<QT, KVT, D, 8, CHAN, 2, false>(q, stream);
+    }
+    DecodeParams q = p;
+    q.chain = 0;
+    return gt == 16 ? launch_mma_t<QT, KVT, D, 16, CHAN, kDecodeWarps, false>(q, stream)
+                    : launch_mma_t<QT, KVT, D, 8, CHAN, kDecodeWarps, false>(q, stream);
 }
 
 template <typename QT, typename KVT, int D>

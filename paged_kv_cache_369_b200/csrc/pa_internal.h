@@ -83,6 +83,11 @@ struct DecodeParams {
     int tile_begin;
     int ws_offset;
     int ws_np;
+    // split mode, tensor-core kernel: 0, or each warp attends `chain`
+    // consecutive partitions on its own, one after another (its copies run
+    // ahead across their boundaries), writing each one's partial from its
+    // registers; set by the launcher for long contexts
+    int chain;
     float qk_scale_log2;        // softmax_scale * k_scale * log2(e)
     float v_scale;              // applied to the output (1 for 16-bit caches)
     // per-channel scales of an 8-bit cache, [Hk, D] fp32, or null: K's are

@@ -32,8 +32,14 @@ def _pa():
 
 
 @pytest.mark.parametrize("kernel", ["auto", "simt"])
-@pytest.mark.parametrize("mode,P", [("single", 512), ("split", 64), ("fused", 64)])
-def test_decode_wait_timeout_is_reported(mode, P, kernel, monkeypatch):
+@pytest.mark.parametrize("mode,P,chain", [("single", 512, None), ("split", 64, None), ("fused", 64, None),
+                                          ("split", 32, "2"), ("fused", 32, "1")])
+def test_decode_wait_timeout_is_reported(mode, P, chain, kernel, monkeypatch):
+    """With 32-token partitions (22 for the longest sequence) the
+    tensor-core kernel's warps take 2 (or 1) partitions in a row
+    (PA369_DECODE_CHAIN)."""
+    if chain:
+        monkeypatch.setenv("PA369_DECODE_CHAIN", chain)
     if kernel == "simt":
         monkeypatch.setenv("PA369_DECODE_KERNEL", "simt")
     else:

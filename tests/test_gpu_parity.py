@@ -153,6 +153,34 @@ def test_small_full_parity(case, mode, P, kernel_choice):
             assert not got[s].any()
 
 
+@pytest.mark.parametrize("chain", ["2", "3"])
+@pytest.mark.parametrize("mode", ["split", "fused"])
+@pytest.mark.parametrize("case", [c for c in range(len(SMALL)) if max(SMALL[c][5]) > 16 * 16])
+def test_chained_partitions_parity(case, mode, chain, monkeypatch):
+    """Long split contexts (16 or more partitions) run with each warp taking
+    several consecutive partitions in a row and writing each one's partial as
+    it crosses into the next; PA369_DECODE_CHAIN forces 2 or 3 a warp, so
+    that the boundaries fall inside a warp's run, at sequence ends and in a
+    CTA's second warp.  16-token partitions."""
+    monkeypatch.setenv("PA369_DECODE_CHAIN", chain)
+    pa, PagedDecode = _pa()
+    Hq, Hk, d, act, kv, lens, prefix = SMALL[case]
+    w = workload.build(f"small{case}", 1000 + case, lens, Hq, Hk, d, act, kv,
+                       shared_prefix_tokens=prefix, extra_table_cols=2)
+    dec = PagedDecode(w, mode=mode, partition_size=16)
+    out_buf, dec.out = guarded_like(dec.out)
+    ws_buf, dec.workspace = guarded_like(dec.workspace)
+    dec.step()
+    torch.cuda.synchronize()
+    assert dec.error() == 0
+    check_guards(out_buf, "out")
+    check_guards(ws_buf, "workspace")
+    kc, vc = oracle.caches_for(w)
+    check_pools(dec, kc, vc)
+    ref = oracle.decode_for(w, kc, vc)
+    assert_close(_to_f64(dec.out), ref, f"case {case} {mode} chain={chain}")
+
+
 PER_CHANNEL = [
     # (Hq, Hk, d, act, kv, lens)
     (64, 8, 128, "bf16", "e4m3", [600, 1, 17, 1024]),
@@ -283,10 +311,15 @@ def test_shared_prefix_shorter_sequence_is_reported():
     assert torch.isfinite(dec.out.float()).all()
 
 
-def test_split_partials_match_oracle(kernel_choice):
+@pytest.mark.parametrize("P,chain", [(128, None), (32, "1"), (32, "3")])
+def test_split_partials_match_oracle(kernel_choice, P, chain, monkeypatch):
+    """Every partition's (lse, o) against the oracle's; with 32-token
+    partitions (35 of them) the tensor-core kernel's warps take 1 or 3
+    partitions in a row."""
+    if chain:
+        monkeypatch.setenv("PA369_DECODE_CHAIN", chain)
     pa, PagedDecode = _pa()
     w = workload.build("partials", 77, [1, 16, 17, 100, 513, 1100], 16, 4, 128, "bf16", "bf16")
-    P = 128
     dec = PagedDecode(w, mode="split", partition_size=P)
     dec.step()
     torch.cuda.synchronize()
