@@ -14,7 +14,10 @@
 //   - one CTA per (sequence, partition, KV head, head group of <= 16); 4 warps
 //     (2 for long split contexts), each owning every 4th (2nd) 16-token tile of
 //     the partition with a private ring of shared-memory stages filled by TMA
-//     (cp.async.bulk.tensor.2d, no multicast);
+//     (cp.async.bulk.tensor.2d, no multicast); for long split contexts with
+//     at least as many partitions as resident warps, each warp instead takes
+//     whole partitions alone, one after another (CHAINED), and writes each
+//     one's partial from its registers;
 //   - a tile row is 128 bytes per TMA box (d = 64 16-bit, or half of d = 128
 //     16-bit, or d = 128 E4M3) and the box lands 128B-swizzled, so ldmatrix of
 //     8 token rows at one 16-byte column touches 8 distinct bank groups;
